@@ -1,0 +1,255 @@
+"""fp64 CPU oracle for draft-tree verification -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may import
+this package.  The product path (the CUDA library and its Python binding) never does: it shares no
+code with this module, and this module imports nothing from it.
+
+Every function is a thin ctypes marshaller around the plain C definitions in ``oracle.c``; the
+per-request composition below only slices rows and calls those definitions in order.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import numpy as np
+
+from . import _build
+
+_lib = None
+
+I32P = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+I64P = np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS")
+U64P = np.ctypeslib.ndpointer(np.uint64, flags="C_CONTIGUOUS")
+U16P = np.ctypeslib.ndpointer(np.uint16, flags="C_CONTIGUOUS")
+F64P = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
+F32P = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+
+OK, EINVAL, EUNSUPPORTED, ENOSPACE = 0, -1, -2, -6
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        L.oracle_max_threads.restype = C.c_int
+        L.oracle_ancestry.argtypes = [C.c_int, I32P, U64P, I32P]
+        L.oracle_ancestry.restype = C.c_int
+        L.oracle_attention.argtypes = [C.c_int, I32P, I32P, I32P, I64P, U16P, U16P, U16P, U16P,
+                                       U16P, C.c_int, C.c_int, C.c_int, C.c_double, C.c_int,
+                                       C.c_void_p, F64P, F64P, C.c_int]
+        L.oracle_attention.restype = C.c_int
+        L.oracle_logits.argtypes = [C.c_int, I32P, C.c_int, C.c_int, U16P, U16P, F64P, C.c_int]
+        L.oracle_logits.restype = None
+        L.oracle_row_top2.argtypes = [C.c_int, C.c_int, F64P, I32P, F64P, F64P]
+        L.oracle_row_top2.restype = None
+        L.oracle_walk_greedy.argtypes = [C.c_int, I32P, I32P, I32P, I32P, I32P]
+        L.oracle_walk_greedy.restype = C.c_int
+        L.oracle_philox4x64.argtypes = [U64P, U64P, U64P]
+        L.oracle_philox4x64.restype = None
+        L.oracle_uniform.argtypes = [C.c_uint64, C.c_uint64, C.c_uint32, C.c_uint32, C.c_uint32,
+                                     C.c_uint32]
+        L.oracle_uniform.restype = C.c_double
+        L.oracle_race.argtypes = [C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int, C.c_int,
+                                  C.POINTER(C.c_double)]
+        L.oracle_race.restype = C.c_int
+        L.oracle_accept_chain.argtypes = [C.c_int, I32P, I32P, F64P, F32P, C.c_int, C.c_double,
+                                          C.c_uint64, C.c_uint64, C.c_int, I32P, I32P, I32P]
+        L.oracle_accept_chain.restype = C.c_int
+        L.oracle_kv_compact.argtypes = [C.c_int, I32P, I32P, I64P, I32P, I32P, I32P, U16P, U16P,
+                                        U16P, U16P, C.c_int, C.c_int64, C.c_int64, C.c_int,
+                                        C.c_int, I32P]
+        L.oracle_kv_compact.restype = C.c_int
+        L.oracle_accept_chain_batch.argtypes = [C.c_int, I32P, I32P, I32P, F64P, F32P, C.c_int,
+                                                C.c_double, C.c_uint64, C.c_uint64, I32P, I32P,
+                                                I32P, I32P, C.c_int]
+        L.oracle_accept_chain_batch.restype = None
+        L.oracle_race_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
+                                       C.c_int, I32P, C.c_int]
+        L.oracle_race_many.restype = None
+        _lib = L
+    return _lib
+
+
+def max_threads() -> int:
+    return int(lib().oracle_max_threads())
+
+
+def _u16(x) -> np.ndarray:
+    """uint16 bits of a bf16 torch tensor or a uint16 numpy array (no copy when contiguous)."""
+    if isinstance(x, np.ndarray):
+        return np.ascontiguousarray(x, dtype=np.uint16)
+    import torch
+    t = x.detach().cpu().contiguous()
+    assert t.dtype == torch.bfloat16
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _i32(x) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(x), dtype=np.int32)
+
+
+# ------------------------------------------------------------------------------------ primitives
+def ancestry(parent):
+    parent = _i32(parent)
+    n = len(parent)
+    anc = np.zeros(max(n, 1), dtype=np.uint64)
+    dep = np.zeros(max(n, 1), dtype=np.int32)
+    st = lib().oracle_ancestry(n, parent, anc, dep)
+    return st, anc[:n], dep[:n]
+
+
+def attention(cu_nodes, parent, kv_len, slot_base, q, k_tree, v_tree, k_cache, v_cache, hq, hkv,
+              scale, rows=None, nthreads=0):
+    """(out [k, d] fp64, lse [k] fp64, status) for the listed (node, head) rows, or all rows."""
+    cu = _i32(cu_nodes)
+    B = len(cu) - 1
+    qn = _u16(q)
+    d = qn.shape[-1] if qn.ndim > 1 else 128
+    if rows is None:
+        nrows, rp, count = 0, None, int(cu[-1]) * hq
+    else:
+        rr = _i32(rows).reshape(-1, 2)
+        nrows, rp, count = len(rr), rr.ctypes.data_as(C.c_void_p), len(rr)
+    out = np.zeros((max(count, 1), d), dtype=np.float64)
+    lse = np.zeros(max(count, 1), dtype=np.float64)
+    st = lib().oracle_attention(B, cu, _i32(parent), _i32(kv_len),
+                                np.ascontiguousarray(slot_base, dtype=np.int64), qn.reshape(-1),
+                                _u16(k_tree).reshape(-1), _u16(v_tree).reshape(-1),
+                                _u16(k_cache).reshape(-1), _u16(v_cache).reshape(-1), hq, hkv, d,
+                                float(scale), nrows, rp, out, lse, int(nthreads))
+    return out[:count], lse[:count], st
+
+
+def logits(hidden, w, rows, nthreads=0):
+    hn = _u16(hidden)
+    wn = _u16(w)
+    H = wn.shape[1]
+    V = wn.shape[0]
+    rows = _i32(rows)
+    z = np.empty((len(rows), V), dtype=np.float64)
+    if len(rows):
+        lib().oracle_logits(len(rows), rows, H, V, hn.reshape(-1), wn.reshape(-1), z,
+                            int(nthreads))
+    return z
+
+
+def row_top2(z):
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    n, V = z.shape
+    arg = np.empty(n, dtype=np.int32)
+    t1 = np.empty(n, dtype=np.float64)
+    t2 = np.empty(n, dtype=np.float64)
+    if n:
+        lib().oracle_row_top2(n, V, z, arg, t1, t2)
+    return arg, t1, t2
+
+
+def walk_greedy(parent, tokens, arg):
+    path = np.empty(64, dtype=np.int32)
+    out = np.empty(65, dtype=np.int32)
+    a = lib().oracle_walk_greedy(len(parent), _i32(parent), _i32(tokens), _i32(arg), path, out)
+    return a, path, out
+
+
+def philox4x64(ctr, key):
+    out = np.empty(4, dtype=np.uint64)
+    lib().oracle_philox4x64(np.ascontiguousarray(ctr, dtype=np.uint64),
+                            np.ascontiguousarray(key, dtype=np.uint64), out)
+    return out
+
+
+def uniform(seed, step, r, node, v, stream):
+    return float(lib().oracle_uniform(seed, step, r, node, v, stream))
+
+
+def race(w, seed, step, r, node):
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    bk = C.c_double()
+    tok = lib().oracle_race(len(w), w, seed, step, r, node, C.byref(bk))
+    return tok, bk.value
+
+
+def accept_chain(parent, tokens, z, q, T, seed, step, r):
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    n, V = z.shape
+    path = np.empty(64, dtype=np.int32)
+    out = np.empty(65, dtype=np.int32)
+    info = np.zeros(3, dtype=np.int32)
+    a = lib().oracle_accept_chain(n, _i32(parent), _i32(tokens), z, q, V, float(T), seed, step,
+                                  r, path, out, info)
+    return a, path, out, info
+
+
+def accept_chain_batch(cu_nodes, parent, tokens, z, q, T, seed, step, nthreads=0):
+    """Batched oracle_accept_chain; returns (accept_len [B], path [B,64], out [B,65], info [B,3])."""
+    cu = _i32(cu_nodes)
+    B = len(cu) - 1
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    V = z.shape[1]
+    a = np.empty(B, dtype=np.int32)
+    path = np.empty((B, 64), dtype=np.int32)
+    out = np.empty((B, 65), dtype=np.int32)
+    info = np.zeros((B, 3), dtype=np.int32)
+    lib().oracle_accept_chain_batch(B, cu, _i32(parent), _i32(tokens), z.reshape(-1),
+                                    q.reshape(-1), V, float(T), seed, step, a, path.reshape(-1),
+                                    out.reshape(-1), info.reshape(-1), int(nthreads))
+    return a, path, out, info
+
+
+def race_many(w, n, seed, step, r0, node, nthreads=0):
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    out = np.empty(n, dtype=np.int32)
+    lib().oracle_race_many(n, len(w), w, seed, step, r0, node, out, int(nthreads))
+    return out
+
+
+def kv_compact(cu_nodes, kv_len, slot_base, slot_cap, accept_len, path, k_tree, v_tree, k_cache,
+               v_cache, n_layers, tree_layer_stride, cache_layer_stride, hkv, d):
+    """Compacts in place into the given uint16 caches; returns (status, kv_len_out)."""
+    cu = _i32(cu_nodes)
+    B = len(cu) - 1
+    out = np.empty(B, dtype=np.int32)
+    kc = k_cache if isinstance(k_cache, np.ndarray) else _u16(k_cache)
+    vc = v_cache if isinstance(v_cache, np.ndarray) else _u16(v_cache)
+    st = lib().oracle_kv_compact(B, cu, _i32(kv_len), np.ascontiguousarray(slot_base, np.int64),
+                                 _i32(slot_cap), _i32(accept_len),
+                                 _i32(path).reshape(-1), _u16(k_tree).reshape(-1),
+                                 _u16(v_tree).reshape(-1), kc.reshape(-1), vc.reshape(-1),
+                                 n_layers, tree_layer_stride, cache_layer_stride, hkv, d, out)
+    return st, out
+
+
+# --------------------------------------------------------------------------- per-request passes
+def lmhead_accept(wl, requests=None, nthreads=0, keep_logits=False):
+    """The oracle's LM head + acceptance for the listed requests of a Workload.
+
+    Returns a dict of per-request results: accept_len, path [64], out_tokens [65], and for T=0
+    per-node argmax, top1, top2; for T>0 the stop node / rejection / fallback info.
+    """
+    reqs = range(wl.B) if requests is None else requests
+    res = {}
+    for r in reqs:
+        a0, a1 = int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])
+        rows = np.arange(a0, a1, dtype=np.int32)
+        z = logits(wl.hidden, wl.w_lm, rows, nthreads)
+        par = wl.parent[a0:a1]
+        tok = wl.tokens[a0:a1]
+        if wl.temperature == 0.0:
+            arg, t1, t2 = row_top2(z)
+            a, path, out = walk_greedy(par, tok, arg)
+            res[r] = dict(accept_len=a, path=path, out_tokens=out, argmax=arg, top1=t1, top2=t2)
+        else:
+            qd = wl.q_draft[a0:a1].numpy()
+            a, path, out, info = accept_chain(par, tok, z, qd, wl.temperature, wl.seed, wl.step,
+                                              r)
+            res[r] = dict(accept_len=a, path=path, out_tokens=out, info=info,
+                          z=z if keep_logits else None)
+    return res
+
+
+def scale_of(head_dim: int) -> float:
+    return 1.0 / float(np.sqrt(head_dim))
+

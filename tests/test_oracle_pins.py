@@ -1,0 +1,459 @@
+"""Pins for the fp64 oracle: checks against facts fixed outside the oracle itself.
+
+Each check is chosen so that a plausible slip in the oracle (a dropped ancestor, the wrong parent
+row, an inverted p/q ratio, a wrong Philox constant, an off-by-one in the compaction slots) fails
+it.  Sources of truth: torch's fp64 scaled-dot-product attention with a mask built a different
+way (positions, transitive closure), numpy's matmul, numpy's Philox4x64-10 bit generator, closed
+forms of speculative sampling, chi-square tests and direct enumeration.  The pages (EAGLE-4
+write-ups) print no worked example, so no stored values are used.
+"""
+import hashlib
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+from scipy import stats
+
+import oracle
+from draft_tree_verification_masked_b200 import workload as wlm
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+
+# --------------------------------------------------------------------------------------- Philox
+def _minus_one(ctr):
+    c = [int(x) for x in ctr]
+    for i in range(4):
+        if c[i] > 0:
+            c[i] -= 1
+            break
+        c[i] = (1 << 64) - 1
+    return np.array(c, dtype=np.uint64)
+
+
+@pytest.mark.parametrize("ctr,key", [
+    ([1, 0, 0, 0], [0, 0]),
+    ([0, 0, 0, 0], [1, 2]),
+    ([5, 7, 11, 1], [0xE7EE0004, 3]),
+    ([2**64 - 1, 2**63, 12345, 2**40], [2**64 - 1, 2**64 - 1]),
+])
+def test_philox_matches_numpy_bit_generator(ctr, key):
+    """numpy's Philox is Philox4x64-10; it advances the counter by one before each block."""
+    ours = oracle.philox4x64(ctr, key)
+    bg = np.random.Philox(counter=_minus_one(ctr), key=np.array(key, dtype=np.uint64))
+    assert (bg.random_raw(4).astype(np.uint64) == ours).all()
+
+
+def test_philox_random_counters_match_numpy():
+    g = np.random.default_rng(7)
+    for _ in range(200):
+        ctr = g.integers(0, 2**63, size=4, dtype=np.uint64) + np.uint64(1)
+        key = g.integers(0, 2**63, size=2, dtype=np.uint64)
+        bg = np.random.Philox(counter=_minus_one(ctr), key=key)
+        assert (bg.random_raw(4).astype(np.uint64) == oracle.philox4x64(ctr, key)).all()
+
+
+def test_uniform_is_24bit_centred_and_uniform():
+    us = np.array([oracle.uniform(0xE7EE0004, 9, r, r % 5, v, 0)
+                   for r in range(400) for v in range(50)])
+    assert (us > 0).all() and (us < 1).all()
+    k = us * 2**24 - 0.5
+    assert np.allclose(k, np.round(k), atol=0, rtol=0)
+    counts, _ = np.histogram(us, bins=20, range=(0, 1))
+    assert stats.chisquare(counts).pvalue > 1e-4
+    # stream 1 and stream 0 are different draws
+    assert oracle.uniform(1, 0, 0, 1, 0, 1) != oracle.uniform(1, 0, 0, 1, 0, 0)
+
+
+# ------------------------------------------------------------------------------------- ancestry
+def _closure(parent):
+    n = len(parent)
+    A = np.zeros((n, n), dtype=bool)
+    for i in range(1, n):
+        A[i, parent[i]] = True
+    R = np.eye(n, dtype=bool)
+    for _ in range(n):
+        R = R | ((R.astype(np.int64) @ A.astype(np.int64)) > 0)
+    return R
+
+
+def test_ancestry_equals_transitive_closure():
+    g = np.random.default_rng(3)
+    for n, depth, branch, width in [(1, 0, None, None), (16, 6, 4, None), (64, 8, None, 16),
+                                    (4, 3, 1, None), (64, 63, 1, None), (33, 5, 8, None)]:
+        par = wlm.make_tree(n, depth, branch, width, g)
+        st, anc, dep = oracle.ancestry(par)
+        assert st == 0
+        R = _closure(par)
+        for i in range(n):
+            bits = [(int(anc[i]) >> j) & 1 for j in range(n)]
+            assert bits == list(R[i].astype(int)), (n, i)
+            assert dep[i] == R[i].sum() - 1
+
+
+@pytest.mark.parametrize("par", [[0, 0], [-1, 1], [-1, 0, 3, 1], [-1, -1], [-1, 0, 2]])
+def test_ancestry_rejects_malformed(par):
+    st, _, _ = oracle.ancestry(np.array(par, dtype=np.int32))
+    assert st == oracle.EINVAL
+
+
+# ------------------------------------------------------------------------------------ attention
+def _small(n_nodes, depth, branch, B=2, hq=4, hkv=2, kv=(37, 37), seed=11, width=None):
+    return wlm.generate("tiny", seed=seed, B=B, hq=hq, hkv=hkv, n_nodes=n_nodes, depth=depth,
+                        depth_min=depth, branch=branch, width=width, kv_len=kv, hidden=64,
+                        vocab=32)
+
+
+def _f64(t):
+    return t.to(torch.float64)
+
+
+def _sdpa_rows(wl, r, mask_fn):
+    """torch fp64 SDPA for every node/head of request r with the boolean mask from mask_fn."""
+    a0, a1 = int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])
+    n, L = a1 - a0, int(wl.kv_len[r])
+    sb = int(wl.slot_base[r])
+    G = wl.hq // wl.hkv
+    outs = torch.zeros(n, wl.hq, wl.head_dim, dtype=torch.float64)
+    lses = torch.zeros(n, wl.hq, dtype=torch.float64)
+    mask = torch.as_tensor(mask_fn(n, L))
+    for h in range(wl.hq):
+        kvh = h // G
+        K = torch.cat([_f64(wl.k_cache[sb:sb + L, kvh]), _f64(wl.k_tree[a0:a1, kvh])])
+        Vv = torch.cat([_f64(wl.v_cache[sb:sb + L, kvh]), _f64(wl.v_tree[a0:a1, kvh])])
+        Q = _f64(wl.q[a0:a1, h])
+        scale = 1.0 / np.sqrt(wl.head_dim)
+        o = F.scaled_dot_product_attention(Q[None, None], K[None, None], Vv[None, None],
+                                           attn_mask=mask[None, None], scale=scale)
+        outs[:, h] = o[0, 0]
+        s = (Q @ K.T) * scale
+        lses[:, h] = torch.logsumexp(s.masked_fill(~mask, float("-inf")), dim=1)
+    return outs.numpy(), lses.numpy()
+
+
+def _oracle_all(wl):
+    out, lse, st = oracle.attention(wl.cu_nodes, wl.parent, wl.kv_len, wl.slot_base, wl.q,
+                                    wl.k_tree, wl.v_tree, wl.k_cache, wl.v_cache, wl.hq, wl.hkv,
+                                    oracle.scale_of(wl.head_dim))
+    assert st == 0
+    return out.reshape(-1, wl.hq, wl.head_dim), lse.reshape(-1, wl.hq)
+
+
+def test_chain_tree_equals_causal_attention():
+    """A chain is ordinary causal attention over [cache; chain] with positions compared."""
+    wl = _small(n_nodes=6, depth=5, branch=1, kv=(37, 37))
+    out, lse = _oracle_all(wl)
+
+    def causal(n, L):
+        qpos = L + np.arange(n)
+        kpos = np.arange(L + n)
+        return kpos[None, :] <= qpos[:, None]
+
+    for r in range(wl.B):
+        a0, a1 = int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])
+        ref, ref_lse = _sdpa_rows(wl, r, causal)
+        assert np.abs(out[a0:a1] - ref).max() < 1e-12
+        assert np.abs(lse[a0:a1] - ref_lse).max() < 1e-12
+
+
+def test_single_node_tree_equals_one_token_decode():
+    wl = _small(n_nodes=1, depth=0, branch=None, kv=(50, 50), B=3)
+    out, lse = _oracle_all(wl)
+    for r in range(wl.B):
+        ref, ref_lse = _sdpa_rows(wl, r, lambda n, L: np.ones((n, L + n), dtype=bool))
+        assert np.abs(out[r:r + 1] - ref).max() < 1e-12
+        assert np.abs(lse[r:r + 1] - ref_lse).max() < 1e-12
+
+
+@pytest.mark.parametrize("n,depth,branch,width", [(16, 6, 4, None), (64, 8, None, 16),
+                                                  (33, 4, 16, None)])
+def test_tree_attention_equals_dense_closure_mask(n, depth, branch, width):
+    wl = _small(n_nodes=n, depth=depth, branch=branch, width=width, kv=(20, 70), B=3, hq=6,
+                hkv=2)
+    out, lse = _oracle_all(wl)
+    for r in range(wl.B):
+        a0, a1 = int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])
+        R = _closure(wl.parent[a0:a1])
+
+        def closure_mask(n_, L):
+            return np.concatenate([np.ones((n_, L), dtype=bool), R], axis=1)
+
+        ref, ref_lse = _sdpa_rows(wl, r, closure_mask)
+        assert np.abs(out[a0:a1] - ref).max() < 1e-12
+        assert np.abs(lse[a0:a1] - ref_lse).max() < 1e-12
+
+
+def test_attention_ignores_non_ancestors_and_sees_ancestors():
+    wl = _small(n_nodes=16, depth=6, branch=4, B=1)
+    out, _ = _oracle_all(wl)
+    R = _closure(wl.parent)
+    i = 15
+    non = [j for j in range(16) if not R[i, j]]
+    anc = [j for j in range(16) if R[i, j]]
+    assert non and anc
+    k2, v2 = wl.k_tree.clone(), wl.v_tree.clone()
+    k2[non] = torch.randn(len(non), wl.hkv, wl.head_dim).to(torch.bfloat16)
+    v2[non] = torch.randn(len(non), wl.hkv, wl.head_dim).to(torch.bfloat16)
+    o2, _, _ = oracle.attention(wl.cu_nodes, wl.parent, wl.kv_len, wl.slot_base, wl.q, k2, v2,
+                                wl.k_cache, wl.v_cache, wl.hq, wl.hkv, oracle.scale_of(128))
+    o2 = o2.reshape(-1, wl.hq, 128)
+    assert np.array_equal(o2[i], out[i])
+    v3 = wl.v_tree.clone()
+    v3[anc[-1]] += 1.0
+    o3, _, _ = oracle.attention(wl.cu_nodes, wl.parent, wl.kv_len, wl.slot_base, wl.q, wl.k_tree,
+                                v3, wl.k_cache, wl.v_cache, wl.hq, wl.hkv, oracle.scale_of(128))
+    assert not np.array_equal(o3.reshape(-1, wl.hq, 128)[i], out[i])
+
+
+def test_attention_row_subset_matches_full():
+    wl = _small(n_nodes=16, depth=6, branch=4, B=2)
+    out, lse = _oracle_all(wl)
+    rows = np.array([[0, 0], [17, 3], [31, 1], [5, 2]], dtype=np.int32)
+    o, l_, st = oracle.attention(wl.cu_nodes, wl.parent, wl.kv_len, wl.slot_base, wl.q,
+                                 wl.k_tree, wl.v_tree, wl.k_cache, wl.v_cache, wl.hq, wl.hkv,
+                                 oracle.scale_of(128), rows=rows)
+    assert st == 0
+    for k, (g, h) in enumerate(rows):
+        assert np.array_equal(o[k], out[g, h]) and l_[k] == lse[g, h]
+
+
+# -------------------------------------------------------------------------------------- LM head
+def test_logits_equal_numpy_matmul():
+    g = torch.Generator().manual_seed(5)
+    hid = torch.randn(7, 300, generator=g).to(torch.bfloat16)
+    w = (0.02 * torch.randn(1000, 300, generator=g)).to(torch.bfloat16)
+    rows = np.array([6, 0, 3], dtype=np.int32)
+    z = oracle.logits(hid, w, rows)
+    ref = hid.double().numpy()[rows] @ w.double().numpy().T
+    assert np.abs(z - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_row_top2_ties_and_order():
+    z = np.array([[0.0, 1.0, 3.0, 3.0, -1.0], [5.0, 4.0, 4.0, 2.0, 5.0 - 1e-9]])
+    arg, t1, t2 = oracle.row_top2(z)
+    assert list(arg) == [2, 0]
+    assert t1[0] == 3.0 and t2[0] == 3.0
+    assert t1[1] == 5.0 and t2[1] == 5.0 - 1e-9
+
+
+def _f_prefix(prefix, V):
+    h = hashlib.sha256(np.array(prefix, dtype=np.int64).tobytes()).digest()
+    return np.random.default_rng(int.from_bytes(h[:8], "little")).standard_normal(V)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_greedy_walk_equals_sequential_greedy_decoding(seed):
+    """Accepted tokens + bonus = what step-by-step greedy decoding emits (same logits)."""
+    V = 16
+    g = np.random.default_rng(100 + seed)
+    n = int(g.integers(1, 40))
+    while True:
+        try:
+            par = wlm.make_tree(n, int(g.integers(1, 10)), int(g.integers(1, 5)), None, g)
+            break
+        except ValueError:  # caps too tight for n nodes: draw again
+            continue
+    n = len(par)
+    tok = np.zeros(n, dtype=np.int32)
+    tok[0] = g.integers(V)
+    prefix = {0: (int(tok[0]),)}
+    for u in range(n):
+        kids = [c for c in range(1, n) if par[c] == u]
+        best = int(np.argmax(_f_prefix(prefix[u], V)))
+        used = set()
+        for c in kids:
+            t = best if (best not in used and g.random() < 0.7) else None
+            while t is None or t in used:
+                t = int(g.integers(V))
+            used.add(t)
+            tok[c] = t
+            prefix[c] = prefix[u] + (t,)
+    z = np.stack([_f_prefix(prefix[i], V) for i in range(n)])
+    arg, _, _ = oracle.row_top2(z)
+    a, path, out = oracle.walk_greedy(par, tok, arg)
+    # sequential greedy decoding from the root, no tree involved
+    y, pre = [], (int(tok[0]),)
+    for _ in range(n + 1):
+        t = int(np.argmax(_f_prefix(pre, V)))
+        y.append(t)
+        pre = pre + (t,)
+    # deepest tree node whose root path spells a prefix of y
+    depth = {i: len(prefix[i]) - 1 for i in range(n)}
+    consistent = [i for i in range(n) if list(prefix[i][1:]) == y[:depth[i]]]
+    deepest = max(consistent, key=lambda i: depth[i])
+    assert a == depth[deepest]
+    assert list(out[:a + 1]) == y[:a + 1]
+    assert path[a] == deepest and path[0] == 0
+    assert (out[a + 1:] == -1).all() and (path[a + 1:] == -1).all()
+
+
+# ------------------------------------------------------------------------ stochastic acceptance
+def _softmax(x):
+    e = np.exp(x - x.max())
+    return e / e.sum()
+
+
+def _chain_trials(z_rows, q_rows, T, ntrial, seed, chunk=250_000):
+    """Run ntrial requests of one chain (len = rows) with tokens drafted from q of the parent."""
+    n, V = z_rows.shape
+    g = np.random.default_rng(seed)
+    firsts, seconds, alen = [], [], []
+    done = 0
+    step = 0
+    while done < ntrial:
+        m = min(chunk, ntrial - done)
+        cu = (np.arange(m + 1) * n).astype(np.int32)
+        par = np.tile(np.arange(-1, n - 1, dtype=np.int32), m)
+        tok = np.zeros((m, n), dtype=np.int32)
+        for k in range(1, n):
+            c = np.cumsum(q_rows[k - 1].astype(np.float64))
+            tok[:, k] = np.minimum(V - 1, np.searchsorted(c, g.random(m) * c[-1], side="right"))
+        z = np.broadcast_to(z_rows, (m, n, V)).reshape(m * n, V)
+        q = np.broadcast_to(q_rows, (m, n, V)).reshape(m * n, V)
+        a, path, out, info = oracle.accept_chain_batch(cu, par, tok.reshape(-1), z, q, T,
+                                                       seed, step)
+        assert (a >= 0).all()
+        firsts.append(out[:, 0])
+        seconds.append(np.where(a >= 1, out[:, 1], -1))
+        alen.append(a)
+        done += m
+        step += 1
+    return np.concatenate(firsts), np.concatenate(seconds), np.concatenate(alen)
+
+
+def _chisq_p(samples, probs):
+    counts = np.bincount(samples, minlength=len(probs))
+    exp = probs * len(samples)
+    keep = exp > 0
+    assert counts[~keep].sum() == 0
+    return stats.chisquare(counts[keep], exp[keep]).pvalue
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("T", [1.0, 0.7])
+def test_first_emitted_token_follows_target(T):
+    """1e6 trials, V=16: the first emitted token ~ p_root, whatever the draft; the acceptance
+    probability of the first draft equals sum_v min(p, q) (closed form)."""
+    V = 16
+    g = np.random.default_rng(21)
+    z = g.normal(0, 1.5, size=(2, V))
+    q = np.stack([_softmax(g.normal(0, 1.5, size=V)) for _ in range(2)]).astype(np.float32)
+    first, _, a = _chain_trials(z, q, T, 1_000_000, seed=0xE7EE0100)
+    p0 = _softmax(z[0] / T)
+    assert _chisq_p(first, p0) > 1e-4
+    acc = (a >= 1).mean()
+    want = np.minimum(p0, q[0].astype(np.float64)).sum()
+    assert abs(acc - want) < 5 * np.sqrt(want * (1 - want) / len(a))
+
+
+@pytest.mark.slow
+def test_second_emitted_token_follows_target_given_accepted_prefix():
+    V = 16
+    g = np.random.default_rng(22)
+    T = 0.8
+    z = g.normal(0, 1.5, size=(3, V))
+    q = np.stack([_softmax(g.normal(0, 1.0, size=V)) for _ in range(3)]).astype(np.float32)
+    first, second, a = _chain_trials(z, q, T, 1_000_000, seed=0xE7EE0200)
+    assert _chisq_p(first, _softmax(z[0] / T)) > 1e-4
+    sel = a >= 1
+    assert _chisq_p(second[sel], _softmax(z[1] / T)) > 1e-4
+
+
+@pytest.mark.slow
+def test_identical_draft_is_always_accepted_and_bonus_follows_target():
+    V = 16
+    g = np.random.default_rng(23)
+    z = g.normal(0, 1.0, size=(2, V))
+    q = np.stack([_softmax(z[0]), _softmax(g.normal(size=V))]).astype(np.float32)
+    # p uses fp64 softmax while q was rounded to fp32: both are the same distribution, so the
+    # draft is accepted unless U*q >= p, which only rounding can cause.
+    first, second, a = _chain_trials(z, q, 1.0, 400_000, seed=0xE7EE0300)
+    assert (a >= 1).mean() > 0.9999
+    sel = a == 1
+    assert _chisq_p(second[sel], _softmax(z[1])) > 1e-4
+
+
+@pytest.mark.slow
+def test_exponential_race_is_an_exact_sampler():
+    w = np.array([0.0, 1.0, 2.0, 0.0, 3.0, 0.5, 0.0, 4.0, 1e-3, 2.5, 0.0, 1.0, 0.25, 0.0, 6.0,
+                  0.75])
+    out = oracle.race_many(w, 1_000_000, 0xE7EE0400, 0, 0, 3)
+    assert _chisq_p(out, w / w.sum()) > 1e-4
+    assert oracle.race(np.zeros(16), 1, 0, 0, 0)[0] == -1
+
+
+def test_accept_chain_rejects_branching_trees_and_bad_parents():
+    z = np.zeros((3, 8))
+    q = np.full((3, 8), 1 / 8, dtype=np.float32)
+    tok = np.array([1, 2, 3], dtype=np.int32)
+    a, *_ = oracle.accept_chain(np.array([-1, 0, 0], np.int32), tok, z, q, 1.0, 1, 0, 0)
+    assert a == oracle.EUNSUPPORTED
+    a, *_ = oracle.accept_chain(np.array([-1, 2, 1], np.int32), tok, z, q, 1.0, 1, 0, 0)
+    assert a == oracle.EINVAL
+
+
+def test_rejected_draft_residual_excludes_the_rejected_token_mass():
+    """p = q except token 0 where the draft overshoots: a rejection can only bonus tokens with
+    p > q, i.e. never token 0."""
+    V = 8
+    p = np.full(V, 1 / V)
+    q = p.copy()
+    q[0] += 0.3
+    q[1:] -= 0.3 / (V - 1)
+    z = np.log(np.stack([p, p]))
+    tok = np.array([5, 0], dtype=np.int32)
+    seen = set()
+    for r in range(3000):
+        a, path, out, info = oracle.accept_chain(np.array([-1, 0], np.int32), tok, z,
+                                                 np.stack([q, q]).astype(np.float32), 1.0, 99, 0,
+                                                 r)
+        if a == 0:
+            assert info[1] == 1 and out[0] != 0
+            seen.add(int(out[0]))
+    assert len(seen) == V - 1
+
+
+# ----------------------------------------------------------------------------------- compaction
+def test_kv_compact_equals_numpy_gather():
+    g = np.random.default_rng(9)
+    B, hkv, d, layers = 5, 2, 8, 3
+    n = np.array([1, 4, 16, 7, 64])
+    cu = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    kv_len = g.integers(0, 40, size=B).astype(np.int32)
+    cap = (kv_len + 64).astype(np.int32)
+    base = np.concatenate([[0], np.cumsum(cap)[:-1]]).astype(np.int64)
+    slots = int(base[-1] + cap[-1])
+    a = np.array([0, 3, 5, 2, 63], dtype=np.int32)
+    path = np.full((B, 64), -1, dtype=np.int32)
+    for r in range(B):
+        path[r, 0] = 0
+        path[r, 1:a[r] + 1] = np.sort(g.choice(np.arange(1, n[r]), a[r], replace=False))
+    tree_k = g.integers(0, 65535, size=(layers, cu[-1], hkv, d), dtype=np.uint16)
+    tree_v = g.integers(0, 65535, size=(layers, cu[-1], hkv, d), dtype=np.uint16)
+    ck = g.integers(0, 65535, size=(layers, slots, hkv, d), dtype=np.uint16)
+    cv = g.integers(0, 65535, size=(layers, slots, hkv, d), dtype=np.uint16)
+    ek, ev = ck.copy(), cv.copy()
+    for r in range(B):
+        dst = base[r] + kv_len[r] + np.arange(a[r] + 1)
+        src = cu[r] + path[r, :a[r] + 1]
+        ek[:, dst] = tree_k[:, src]
+        ev[:, dst] = tree_v[:, src]
+    st, newlen = oracle.kv_compact(cu, kv_len, base, cap, a, path, tree_k, tree_v, ck, cv, layers,
+                                   cu[-1] * hkv * d, slots * hkv * d, hkv, d)
+    assert st == 0
+    assert np.array_equal(ck, ek) and np.array_equal(cv, ev)
+    assert np.array_equal(newlen, kv_len + a + 1)
+
+
+def test_kv_compact_capacity_overflow_leaves_request_untouched():
+    cu = np.array([0, 4], dtype=np.int32)
+    kv_len = np.array([10], dtype=np.int32)
+    cap = np.array([12], dtype=np.int32)
+    path = np.full((1, 64), -1, dtype=np.int32)
+    path[0, :4] = [0, 1, 2, 3]
+    tk = np.ones((4, 1, 8), dtype=np.uint16)
+    ck = np.zeros((12, 1, 8), dtype=np.uint16)
+    st, newlen = oracle.kv_compact(cu, kv_len, np.zeros(1, np.int64), cap, np.array([3], np.int32),
+                                   path, tk, tk, ck, ck.copy(), 1, 32, 96, 1, 8)
+    assert st == oracle.ENOSPACE and newlen[0] == 10 and not ck.any()
