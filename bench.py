@@ -1,0 +1,486 @@
+#!/usr/bin/env python
+"""Benchmark of one draft-tree verification step on B200.
+
+A step is the whole hot path over one batch of synthetic input already resident in HBM:
+tree-masked attention (one layer) -> LM head + acceptance walk -> KV compaction (one layer).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl etree|reference]
+
+Prints ONE JSON line (rank 0).  `value` is accepted tokens/s over all ranks (sum of a_r + 1 per
+request per step), device-timed with CUDA events, max over ranks.  L2 is flushed (a 512 MiB
+write) before every timed step, outside the per-call events.  `e2e` repeats the measurement
+through the same C-ABI calls with the step's inputs copied from pinned host memory and the
+accept results copied back inside the timed region.  `--impl reference` times the fp64 CPU
+oracle on the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("tree-verify µs/step & accepted tokens/s at B=1/64/512; "
+          "HBM GB/s & TC util vs peak")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- algorithmic work
+def attn_work(wl):
+    """Algorithmic bytes (KV cache read once, tree K/V, Q in, O out) and FLOPs of one layer."""
+    D = wl.head_dim
+    kv = 2 * int(wl.kv_len.sum()) * wl.hkv * D * 2
+    tree = 2 * wl.n_total * wl.hkv * D * 2
+    qo = 2 * wl.n_total * wl.hq * D * 2
+    anc = 0
+    for r in range(wl.B):
+        a0, a1 = int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])
+        depth = np.zeros(a1 - a0, dtype=np.int64)
+        for i in range(1, a1 - a0):
+            depth[i] = depth[wl.parent[a0 + i]] + 1
+        anc += int((depth + 1).sum())
+    keys = sum(int(wl.kv_len[r]) * wl.nodes(r) for r in range(wl.B)) + anc
+    flops = 4 * wl.hq * D * keys
+    return kv + tree + qo, flops
+
+
+def lmhead_work(wl):
+    return wl.vocab * wl.hidden_dim * 2 + wl.n_total * wl.hidden_dim * 2, \
+        2 * wl.n_total * wl.vocab * wl.hidden_dim
+
+
+def compact_work(wl, accept_len, n_layers=1):
+    return 2 * 2 * int((accept_len + 1).sum()) * wl.hkv * wl.head_dim * 2 * n_layers
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "draft_tree_verification_masked_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str, src_hash: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[f"{kernel}@{workload}"]
+        return e["bytes_per_launch"] if e.get("source_hash") == src_hash else None
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------------------------ timing
+def time_steps(dev, steps, warmup, flush):
+    for _ in range(warmup):
+        dev.step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        e = ev[i]
+        e[0].record()
+        dev.attn()
+        e[1].record()
+        dev.lmhead()
+        e[2].record()
+        dev.compact()
+        e[3].record()
+    torch.cuda.synchronize()
+    attn = [e[0].elapsed_time(e[1]) for e in ev]
+    lm = [e[1].elapsed_time(e[2]) for e in ev]
+    cp = [e[2].elapsed_time(e[3]) for e in ev]
+    step = [e[0].elapsed_time(e[3]) for e in ev]
+    return dict(attn_ms=attn, lmhead_ms=lm, compact_ms=cp, step_ms=step)
+
+
+def time_e2e(dev, wl, steps, warmup, flush):
+    """Same step through the C ABI with inputs in pinned host memory: H2D of the step's inputs
+    and D2H of the accept results inside the timed region."""
+    ins = [(dev.cu_nodes, wl.cu_nodes), (dev.parent, wl.parent), (dev.tokens, wl.tokens),
+           (dev.kv_len, wl.kv_len), (dev.slot_base, wl.slot_base), (dev.slot_cap, wl.slot_cap),
+           (dev.q, wl.q), (dev.k_tree, wl.k_tree), (dev.v_tree, wl.v_tree),
+           (dev.hidden, wl.hidden)]
+    if dev.q_draft is not None:
+        ins.append((dev.q_draft, wl.q_draft))
+    host_in = []
+    for d, h in ins:
+        t = torch.as_tensor(h) if not isinstance(h, torch.Tensor) else h
+        host_in.append((d, t.to(d.dtype).contiguous().pin_memory()))
+    outs = [dev.accept_len, dev.path, dev.out_tokens]
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
+    d2h = sum(h.numel() * h.element_size() for h in host_out)
+
+    def one():
+        for d, h in host_in:
+            d.copy_(h, non_blocking=True)
+        dev.step()
+        for o, h in zip(outs, host_out):
+            h.copy_(o, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        one()
+        b.record()
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    return ms, h2d, d2h
+
+
+# -------------------------------------------------------------------------------- CPU oracle
+def oracle_step(wl, requests, nthreads=0):
+    """One oracle verification step over the listed requests: attention of all their rows,
+    LM head + acceptance, compaction.  Returns accepted tokens (sum of a + 1)."""
+    import oracle
+    rows = []
+    for r in requests:
+        for g in range(int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])):
+            for h in range(wl.hq):
+                rows.append((g, h))
+    rows = np.asarray(rows, dtype=np.int32)
+    oracle.attention(wl.cu_nodes, wl.parent, wl.kv_len, wl.slot_base, wl.q, wl.k_tree,
+                     wl.v_tree, wl.k_cache, wl.v_cache, wl.hq, wl.hkv,
+                     oracle.scale_of(wl.head_dim), rows=rows, nthreads=nthreads)
+    res = oracle.lmhead_accept(wl, requests, nthreads=nthreads)
+    toks = 0
+    for r in requests:
+        o = res[r]
+        a = int(o["accept_len"])
+        toks += a + 1
+        base, cap = int(wl.slot_base[r]), int(wl.slot_cap[r])
+        a0, a1 = int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])
+        sub_k = oracle._u16(wl.k_cache[base:base + cap]).copy()
+        sub_v = oracle._u16(wl.v_cache[base:base + cap]).copy()
+        oracle.kv_compact(np.array([0, a1 - a0], np.int32), wl.kv_len[r:r + 1],
+                          np.zeros(1, np.int64), wl.slot_cap[r:r + 1], np.array([a], np.int32),
+                          o["path"].reshape(1, 64), wl.k_tree[a0:a1], wl.v_tree[a0:a1], sub_k,
+                          sub_v, 1, (a1 - a0) * wl.hkv * wl.head_dim,
+                          cap * wl.hkv * wl.head_dim, wl.hkv, wl.head_dim)
+    return toks
+
+
+def sample_requests(wl, budget_rows=64):
+    """A bounded sample: whole requests, in order, up to ~budget_rows tree nodes."""
+    reqs, rows = [], 0
+    for r in range(wl.B):
+        if reqs and rows + wl.nodes(r) > budget_rows:
+            break
+        reqs.append(r)
+        rows += wl.nodes(r)
+    return reqs
+
+
+def cpu_baseline(wl, min_seconds=10.0, max_reps=5):
+    import oracle
+    reqs = sample_requests(wl)
+    t0 = time.perf_counter()
+    toks, reps = 0, 0
+    while reps < max_reps and (reps == 0 or time.perf_counter() - t0 < min_seconds):
+        toks += oracle_step(wl, reqs)
+        reps += 1
+    dt = time.perf_counter() - t0
+    return {"value": toks / dt, "unit": "tok/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{len(reqs)} of {wl.B} requests ({sum(wl.nodes(r) for r in reqs)} tree "
+                      f"nodes) of workload {wl.name}, {reps} full oracle steps (attention all "
+                      f"rows, LM head + acceptance, compaction), {dt:.1f} s"}
+
+
+# -------------------------------------------------------------------------------------- main
+def run_config(name, steps, warmup, peaks, rank, flush, with_e2e=True):
+    from draft_tree_verification_masked_b200 import etree_attn_plan
+    from draft_tree_verification_masked_b200 import workload as W
+    from draft_tree_verification_masked_b200.runner import DeviceStep
+
+    wl = W.generate(name, seed=W.config_seed(name) + 7919 * rank)
+    dev = DeviceStep(wl)
+    dev.step()
+    st, det = dev.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} detail {det}")
+    acc = dev.accept_len.cpu().numpy()
+    toks = int((acc + 1).sum())
+    t = time_steps(dev, steps, warmup, flush)
+    plan = etree_attn_plan(dev.batch, wl.hq, wl.hkv)
+    launches = plan["launches"] + (2 if wl.temperature == 0.0 else 5) + 1
+    res = dict(wl=wl, dev=dev, toks=toks, t=t, plan=plan, launches=launches)
+    if with_e2e:
+        res["e2e"] = time_e2e(dev, wl, steps, max(3, warmup), flush)
+    return res
+
+
+def kernel_report(wl, t, acc, peaks):
+    hbm = float(peaks["hbm_gbs"])
+    tc = float(peaks["bf16_tflops"])
+    ab, af = attn_work(wl)
+    lb, lf = lmhead_work(wl)
+    cb = compact_work(wl, acc)
+    am = statistics.mean(t["attn_ms"]) * 1e-3
+    lm = statistics.mean(t["lmhead_ms"]) * 1e-3
+    cm = statistics.mean(t["compact_ms"]) * 1e-3
+    rep = {
+        "attn": {"us": am * 1e6, "GB/s": ab / am / 1e9, "TFLOP/s": af / am / 1e12,
+                 "hbm_frac": ab / am / 1e9 / hbm, "tc_frac": af / am / 1e12 / tc,
+                 "bytes": ab, "flops": af},
+        "lmhead": {"us": lm * 1e6, "GB/s": lb / lm / 1e9, "TFLOP/s": lf / lm / 1e12,
+                   "hbm_frac": lb / lm / 1e9 / hbm, "tc_frac": lf / lm / 1e12 / tc,
+                   "bytes": lb, "flops": lf},
+        "compact": {"us": cm * 1e6, "GB/s": cb / cm / 1e9, "hbm_frac": cb / cm / 1e9 / hbm,
+                    "bytes": cb},
+    }
+    return rep
+
+
+def roofline(wl, rep, peaks, peak_kind, workload):
+    dom = max(("attn", "lmhead", "compact"), key=lambda k: rep[k]["us"])
+    k = rep[dom]
+    hbm, tc = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
+    src = {"attn": "attn_tree.cu", "lmhead": "lmhead.cu", "compact": "compact.cu"}[dom]
+    traffic = ncu_traffic(dom, workload, source_hash(src))
+    if dom == "compact" or k["bytes"] / (hbm * 1e9) >= k.get("flops", 0) / (tc * 1e12):
+        return {"kernel": dom, "bound": "hbm", "achieved": k["GB/s"], "peak": hbm,
+                "unit": "GB/s", "frac": k["GB/s"] / hbm, "traffic": traffic,
+                "algorithmic_bytes": k["bytes"], "peak_source": peak_kind}
+    return {"kernel": dom, "bound": "tensor", "achieved": k["TFLOP/s"], "peak": tc,
+            "unit": "TFLOP/s", "frac": k["TFLOP/s"] / tc, "traffic": traffic,
+            "algorithmic_flops": k["flops"], "peak_source": peak_kind}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="etree", choices=["etree", "reference"])
+    ap.add_argument("--config", default="dense27b_b1")
+    ap.add_argument("--by-batch", default="batch64,conc512",
+                    help="extra workloads measured in the same run (comma list, '' for none)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return main_reference(args, rank, world)
+
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    peaks, peak_kind = load_peaks()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    main_res = run_config(args.config, args.steps, args.warmup, peaks, rank, flush)
+    clk = clocks.stop()
+    barrier()
+    wl, t = main_res["wl"], main_res["t"]
+    step_s = sum(t["step_ms"]) * 1e-3
+    tokens = main_res["toks"] * args.steps
+    e2e_ms, h2d, d2h = main_res["e2e"]
+    e2e_s = sum(e2e_ms) * 1e-3
+    if world > 1:
+        v = torch.tensor([step_s, e2e_s, float(tokens)], device="cuda", dtype=torch.float64)
+        mx = v.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        dist.all_reduce(v, op=dist.ReduceOp.SUM)
+        step_s, e2e_s, tokens_all = float(mx[0]), float(mx[1]), float(v[2])
+    else:
+        tokens_all = float(tokens)
+    acc = main_res["dev"].accept_len.cpu().numpy()
+    rep = kernel_report(wl, t, acc, peaks)
+    rl = roofline(wl, rep, peaks, peak_kind, args.config)
+    head_plan, head_launches = main_res["plan"], main_res["launches"]
+
+    by_batch = {}
+    for name in [x for x in args.by_batch.split(",") if x]:
+        del main_res["dev"]
+        torch.cuda.empty_cache()
+        r = run_config(name, max(5, args.steps // 2), args.warmup, peaks, rank, flush,
+                       with_e2e=False)
+        racc = r["dev"].accept_len.cpu().numpy()
+        rrep = kernel_report(r["wl"], r["t"], racc, peaks)
+        sms = statistics.mean(r["t"]["step_ms"])
+        by_batch[name] = {
+            "B": r["wl"].B, "us_per_step": sms * 1e3,
+            "accepted_tok_per_s": r["toks"] / (sms * 1e-3),
+            "kernels": {k: {kk: round(vv, 4) if isinstance(vv, float) else vv
+                            for kk, vv in v.items()} for k, v in rrep.items()},
+            "roofline": roofline(r["wl"], rrep, peaks, peak_kind, name),
+            "attn_plan": r["plan"], "gpu_launches_per_step": r["launches"],
+        }
+        main_res = r
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC,
+        "value": tokens_all / step_s,
+        "unit": "accepted tok/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_s / args.steps * 1e3,
+        "us_per_step": step_s / args.steps * 1e6,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; random-init LM head, N(0,1) activations and KV)",
+        "config": {"workload": args.config, "B": wl.B, "tree_nodes": int(wl.n_max),
+                   "kv_len": int(wl.kv_len_max), "hidden": wl.hidden_dim, "vocab": wl.vocab,
+                   "heads": f"{wl.hq}/{wl.hkv}", "head_dim": wl.head_dim,
+                   "temperature": wl.temperature, "layers": 1,
+                   "l2": "flushed: 512 MiB write before every timed step",
+                   "attn_plan": head_plan,
+                   "parallelism": f"dp{world} (independent requests per rank)"},
+        "clocks": clk,
+        "e2e": {"value": tokens_all / e2e_s, "unit": "accepted tok/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "us_per_step": e2e_s / args.steps * 1e6},
+        "gpu_launches": head_launches * args.steps,
+        "roofline": rl,
+        "kernels": {k: {kk: round(vv, 4) if isinstance(vv, float) else vv for kk, vv in v.items()}
+                    for k, v in rep.items()},
+        "cpu_baseline": cpu,
+        "by_batch": by_batch,
+    }
+    print(json.dumps(line))
+
+
+def main_reference(args, rank, world):
+    """The oracle arm: the fp64 CPU oracle on the same workload (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    from draft_tree_verification_masked_b200 import workload as W
+    wl = W.generate(args.config)
+    reqs = sample_requests(wl)
+    for _ in range(min(args.warmup, 1)):
+        oracle_step(wl, reqs)
+    times, toks = [], 0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        toks += oracle_step(wl, reqs)
+        times.append(time.perf_counter() - t0)
+    dt = sum(times)
+    value = toks / dt
+    line = {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": "accepted tok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.config, "B": wl.B, "sampled_requests": len(reqs)},
+        "cpu_baseline": {"value": value, "unit": "accepted tok/s", "cores": oracle.max_threads(),
+                         "kind": "oracle",
+                         "sample": f"{len(reqs)} of {wl.B} requests per step, full oracle "
+                                   f"step (attention, LM head + acceptance, compaction)"},
+        "e2e": {"value": value, "unit": "accepted tok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,303 @@
+// accept.cu -- per-row reductions of the LM-head partials and the acceptance walk (sm_100a).
+//
+// The target accepts the drafted prefix that is consistent with its own distribution and adds
+// one token of its own after the first rejection ("Eagle-4 Released: Outpaces DFlash2 and DSpark
+// ...", section "Technical Background").  With a tree, the accepted prefix is a root-to-node
+// path (same section: a draft tree lets one verification cover several paths).  T = 0 is the
+// deterministic greedy setting ("EAGLE-4 ... 961.6 tokens/s是怎么测出来的", whatsnewx.com);
+// at T > 0 verification keeps the target's output distribution ("EAGLE-4 官方推理代码发布 ...",
+// arex-research.com, paragraph on the repository's positioning), which the min(1, p/q) test
+// with a residual resample achieves.
+//
+// One CTA per request: its warps reduce the request's rows across vocab tiles, then one warp
+// walks the tree with ballots over the (<= 64) nodes.
+#include "kernels.cuh"
+#include "philox.cuh"
+
+namespace etree {
+
+
+// Merge (top1, id, top2) summaries: the larger top1 wins (lower id on equal values); the
+// merged top2 is the larger of the winner's top2 and the loser's top1.
+__device__ __forceinline__ void merge_top2(float& t1, int& id, float& t2, float o1, int oid,
+                                           float o2) {
+  const bool other_wins = (o1 > t1) || (o1 == t1 && oid >= 0 && (id < 0 || oid < id));
+  if (other_wins) {
+    t2 = fmaxf(o2, t1);
+    t1 = o1;
+    id = oid;
+  } else {
+    t2 = fmaxf(t2, o1);
+  }
+}
+
+__device__ __forceinline__ void merge_key(float& k, int& id, float ok, int oid) {
+  if (oid < 0) return;
+  if (id < 0 || ok > k || (ok == k && oid < id)) {
+    k = ok;
+    id = oid;
+  }
+}
+
+// Merge two (max, sum 2^(x - max)) summaries in log2 units; an empty side has max = -inf.
+__device__ __forceinline__ void merge_lse(float& m, float& s, float om, float os) {
+  if (om == -INFINITY) return;
+  if (m == -INFINITY) {
+    m = om;
+    s = os;
+    return;
+  }
+  const float nm = fmaxf(m, om);
+  s = s * exp2f(m - nm) + os * exp2f(om - nm);
+  m = nm;
+}
+
+// Validates request r's parent array (parent[0] = -1, 0 <= parent[i] < i); all threads call.
+__device__ bool tree_ok(const AcceptParams& p, int base, int n, int* flag_s) {
+  if (threadIdx.x == 0) *flag_s = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int pi = p.parent[base + i];
+    if ((i == 0 && pi != -1) || (i > 0 && (pi < 0 || pi >= i))) atomicOr(flag_s, 1);
+  }
+  __syncthreads();
+  return *flag_s == 0;
+}
+
+// ------------------------------------------------------------------------------------ T == 0
+__global__ void __launch_bounds__(256) accept_greedy_kernel(AcceptParams p) {
+  __shared__ int am_s[64], par_s[64], tok_s[64], pth_s[64];
+  __shared__ int flag_s;
+  const int r = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int base = p.cu_nodes[r];
+  const int n = p.cu_nodes[r + 1] - base;
+  int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
+  int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
+  if (n < 1 || n > p.n_max) {
+    if (threadIdx.x == 0) report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
+    if (threadIdx.x < 64) path[threadIdx.x] = -1;
+    if (threadIdx.x < 65) outt[threadIdx.x] = -1;
+    if (threadIdx.x == 0) p.accept_len[r] = 0;
+    return;
+  }
+  const bool ok = tree_ok(p, base, n, &flag_s);
+  for (int i = warp; i < n; i += blockDim.x / 32) {
+    float t1 = -INFINITY, t2 = -INFINITY;
+    int id = -1;
+    const float4* row = p.part + (size_t)(base + i) * p.n_tiles;
+    for (int t = lane; t < p.n_tiles; t += 32) {
+      const float4 v = row[t];
+      merge_top2(t1, id, t2, v.x, __float_as_int(v.y), v.z);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float o1 = __shfl_xor_sync(0xffffffffu, t1, off);
+      const int oid = __shfl_xor_sync(0xffffffffu, id, off);
+      const float o2 = __shfl_xor_sync(0xffffffffu, t2, off);
+      merge_top2(t1, id, t2, o1, oid, o2);
+    }
+    if (lane == 0) {
+      am_s[i] = id;
+      par_s[i] = p.parent[base + i];
+      tok_s[i] = p.tokens[base + i];
+      if (p.node_argmax) p.node_argmax[base + i] = id;
+      if (p.node_gap) p.node_gap[base + i] = t1 - t2;
+    }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  if (!ok) report(p.ws, ETREE_EDEVICE, DET_BAD_PARENT);
+  // walk: from the root, follow the lowest-index child that carries argmax(current)
+  int u = 0, a = 0;
+  if (lane == 0) pth_s[0] = 0;
+  if (ok) {
+    for (int step = 0; step < 64; ++step) {
+      const int want = am_s[u];
+      const int j0 = lane, j1 = lane + 32;
+      const bool m0 = j0 >= 1 && j0 < n && par_s[j0] == u && tok_s[j0] == want;
+      const bool m1 = j1 < n && par_s[j1] == u && tok_s[j1] == want;
+      const unsigned b0 = __ballot_sync(0xffffffffu, m0);
+      const unsigned b1 = __ballot_sync(0xffffffffu, m1);
+      if (b0 == 0 && b1 == 0) break;
+      const int c = b0 ? (__ffs(b0) - 1) : (32 + __ffs(b1) - 1);
+      ++a;
+      if (lane == 0) pth_s[a] = c;
+      u = c;
+    }
+  }
+  __syncwarp();
+  const int bonus = am_s[u];
+  // outputs: path[0..a], then -1; out_tokens[0..a-1] accepted tokens, [a] bonus, then -1
+  for (int k = lane; k < 64; k += 32) path[k] = (k <= a) ? pth_s[k] : -1;
+  for (int k = lane; k < 65; k += 32)
+    outt[k] = (k < a) ? tok_s[pth_s[k + 1]] : (k == a ? bonus : -1);
+  if (lane == 0) p.accept_len[r] = a;
+}
+
+// ------------------------------------------------------------------------------------- T > 0
+// Chain check and the child token of every row (read by the LM-head epilogue).
+__global__ void chain_prep_kernel(AcceptParams p, int32_t* child_tok) {
+  __shared__ int flag_s;
+  const int r = blockIdx.x;
+  const int base = p.cu_nodes[r];
+  const int n = p.cu_nodes[r + 1] - base;
+  if (n < 1 || n > p.n_max) return;
+  if (threadIdx.x == 0) flag_s = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int pi = p.parent[base + i];
+    if (i == 0 ? pi != -1 : pi != i - 1) atomicOr(&flag_s, 1);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    int ct = -1;
+    if (flag_s == 0 && i + 1 < n) {
+      ct = p.tokens[base + i + 1];
+      if (ct < 0 || ct >= p.V) ct = -1;
+    }
+    child_tok[base + i] = ct;
+  }
+}
+
+__global__ void __launch_bounds__(128) accept_chain_kernel(AcceptParams p) {
+  __shared__ float lse_s[64];
+  __shared__ int info_s[2];
+  const int r = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int base = p.cu_nodes[r];
+  const int n = p.cu_nodes[r + 1] - base;
+  int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
+  int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
+  const bool n_ok = n >= 1 && n <= p.n_max;
+  // per-row log2-sum-exp of z * log2(e) / T
+  if (n_ok) {
+    for (int i = warp; i < n; i += blockDim.x / 32) {
+      const float4* row = p.part + (size_t)(base + i) * p.n_tiles;
+      float m = -INFINITY, s = 0.f;
+      for (int t = lane; t < p.n_tiles; t += 32) {
+        const float4 v = row[t];
+        merge_lse(m, s, v.x, v.y);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float om = __shfl_xor_sync(0xffffffffu, m, off);
+        const float os = __shfl_xor_sync(0xffffffffu, s, off);
+        merge_lse(m, s, om, os);
+      }
+      if (lane == 0) {
+        const float l2 = m + log2f(s);
+        lse_s[i] = l2;
+        p.lse2[base + i] = l2;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int a = 0, rejected = 0;
+    bool chain = n_ok;
+    if (n_ok) {
+      for (int i = lane; i < n; i += 32) {
+        const int pi = p.parent[base + i];
+        if (i == 0 ? pi != -1 : pi != i - 1) chain = false;
+      }
+      chain = __all_sync(0xffffffffu, chain);
+    }
+    if (!n_ok) {
+      if (lane == 0) report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
+    } else if (!chain) {
+      if (lane == 0) report(p.ws, ETREE_EUNSUPPORTED, DET_NOT_CHAIN);
+    } else if (lane == 0) {
+      for (int k = 1; k < n; ++k) {
+        const int u = k - 1;
+        const int x = p.tokens[base + k];
+        if (x < 0 || x >= p.V) {
+          report(p.ws, ETREE_EDEVICE, DET_BAD_TOKEN);
+          rejected = 1;
+          break;
+        }
+        const float px = exp2f(p.zchild[base + u] * p.k_log2 - lse_s[u]);
+        const float qx = __ldg(p.q_draft + (size_t)(base + u) * p.V + x);
+        float U[4];
+        uniforms4(p.seed, p.step, 0u, (uint32_t)k, (uint32_t)r, 1u, U);
+        if (U[0] * qx < px) {
+          ++a;
+        } else {
+          rejected = 1;
+          break;
+        }
+      }
+    }
+    a = __shfl_sync(0xffffffffu, a, 0);
+    rejected = __shfl_sync(0xffffffffu, rejected, 0);
+    const bool good = n_ok && chain;
+    for (int k = lane; k < 64; k += 32) path[k] = (good && k <= a) ? k : (k == 0 ? 0 : -1);
+    for (int k = lane; k < 65; k += 32) outt[k] = (good && k < a) ? p.tokens[base + k + 1] : -1;
+    if (lane == 0) {
+      p.accept_len[r] = good ? a : 0;
+      p.stop_row[r] = good ? base + a : (n_ok ? base : 0);
+      p.stop_node[r] = good ? a : 0;
+      p.mode[r] = good ? rejected : 0;
+      info_s[0] = good ? base + a : (n_ok ? base : 0);
+    }
+  }
+  __syncthreads();
+  // gather the stop row's hidden state for the second (race) pass
+  const int src = info_s[0];
+  const uint4* hs = reinterpret_cast<const uint4*>(p.hidden + (size_t)src * p.H);
+  uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
+  for (int i = threadIdx.x; i < p.H / 8; i += blockDim.x) hd[i] = hs[i];
+}
+
+// Reduce the race partials of each request and write its bonus token.
+__global__ void bonus_kernel(AcceptParams p) {
+  const int r = blockIdx.x;
+  const int lane = threadIdx.x;
+  const float4* row = p.part2 + (size_t)r * p.n_tiles;
+  float kr = -INFINITY, kp = -INFINITY;
+  int ir = -1, ip = -1;
+  for (int t = lane; t < p.n_tiles; t += 32) {
+    const float4 v = row[t];
+    merge_key(kr, ir, v.x, __float_as_int(v.y));
+    merge_key(kp, ip, v.z, __float_as_int(v.w));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float okr = __shfl_xor_sync(0xffffffffu, kr, off);
+    const int oir = __shfl_xor_sync(0xffffffffu, ir, off);
+    const float okp = __shfl_xor_sync(0xffffffffu, kp, off);
+    const int oip = __shfl_xor_sync(0xffffffffu, ip, off);
+    merge_key(kr, ir, okr, oir);
+    merge_key(kp, ip, okp, oip);
+  }
+  if (lane == 0) {
+    const int base = p.cu_nodes[r];
+    const int n = p.cu_nodes[r + 1] - base;
+    if (n < 1 || n > p.n_max) return;
+    const int a = p.accept_len[r];
+    const int bonus = (p.mode[r] && ir >= 0) ? ir : ip;
+    p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = bonus;
+  }
+}
+
+cudaError_t launch_accept_greedy(const AcceptParams& p, cudaStream_t s) {
+  accept_greedy_kernel<<<p.B, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStream_t s) {
+  chain_prep_kernel<<<p.B, 64, 0, s>>>(p, child_tok);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_accept_chain(const AcceptParams& p, cudaStream_t s) {
+  accept_chain_kernel<<<p.B, 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bonus(const AcceptParams& p, cudaStream_t s) {
+  bonus_kernel<<<p.B, 32, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace etree

@@ -1,0 +1,506 @@
+// api.cu -- the C ABI of libetree: argument validation, workspace layout, TMA descriptors and
+// launch planning for the three verification calls.  Every step of the computation runs in the
+// kernels of attn_tree.cu, lmhead.cu, accept.cu and compact.cu; this file only plans and
+// enqueues them.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+
+#include <cstdarg>
+
+#include "kernels.cuh"
+
+namespace etree {
+
+// ------------------------------------------------------------------------------- error text
+static thread_local char g_err[512] = "";
+
+static etree_status fail(etree_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+static etree_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(ETREE_ECUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------------------------- device info
+static int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+static int env_int(const char* name, int dflt) {
+  const char* v = getenv(name);
+  if (!v || !*v) return dflt;
+  return atoi(v);
+}
+
+// ------------------------------------------------------------------------------ attention plan
+struct AttnPlan {
+  int G, nw, mchunks, nsplit, tps, stages;
+};
+
+static AttnPlan plan_attn(const etree_batch* b, int hq, int hkv) {
+  AttnPlan pl{};
+  pl.G = hq / hkv;
+  const int m16 = (b->n_max * pl.G + 15) / 16;
+  if (m16 <= 8) {
+    pl.nw = std::max(1, m16);
+    pl.mchunks = 1;
+  } else {
+    pl.mchunks = (m16 + 7) / 8;
+    pl.nw = (m16 + pl.mchunks - 1) / pl.mchunks;
+  }
+  const int pairs = b->B * hkv * pl.mchunks;
+  const int tiles_max = (b->kv_len_max + 63) / 64 + 1;
+  const int target = 4 * sm_count();
+  int nsplit = (target + pairs - 1) / pairs;
+  nsplit = std::min(nsplit, std::max(1, tiles_max / 4));
+  nsplit = std::max(1, std::min(nsplit, tiles_max));
+  const int forced = env_int("ETREE_NSPLIT", 0);
+  if (forced > 0) nsplit = std::min(forced, tiles_max);
+  pl.tps = (tiles_max + nsplit - 1) / nsplit;
+  pl.nsplit = (tiles_max + pl.tps - 1) / pl.tps;
+  pl.stages = env_int("ETREE_STAGES", 3) == 4 ? 4 : 3;
+  return pl;
+}
+
+// ------------------------------------------------------------------------------ workspace map
+struct WsLayout {
+  size_t o_part, ml_part, part, child_tok, zchild, lse2, stop_row, stop_node, mode, hid2, part2;
+  size_t total;
+  int n_tiles;
+};
+
+static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static WsLayout layout(const etree_batch* b, int hq, int hkv, int hidden_dim, int vocab) {
+  WsLayout w{};
+  size_t off = sizeof(WsHeader);
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = up256(off + bytes);
+    return at;
+  };
+  const size_t nt = (size_t)std::max(0, b->n_total);
+  const size_t B = (size_t)std::max(0, b->B);
+  size_t nsplit = 1;
+  if (hq > 0 && hkv > 0 && hq % hkv == 0) nsplit = (size_t)plan_attn(b, hq, hkv).nsplit;
+  const size_t rows = nt * (size_t)std::max(0, hq);
+  w.o_part = take(nsplit > 1 ? rows * nsplit * 128 * sizeof(float) : 0);
+  w.ml_part = take(nsplit > 1 ? rows * nsplit * sizeof(float2) : 0);
+  w.n_tiles = vocab > 0 ? (vocab + 255) / 256 : 0;
+  w.part = take(nt * (size_t)w.n_tiles * sizeof(float4));
+  w.child_tok = take(nt * sizeof(int32_t));
+  w.zchild = take(nt * sizeof(float));
+  w.lse2 = take(nt * sizeof(float));
+  w.stop_row = take(B * sizeof(int32_t));
+  w.stop_node = take(B * sizeof(int32_t));
+  w.mode = take(B * sizeof(int32_t));
+  w.hid2 = take(B * (size_t)std::max(0, hidden_dim) * 2);
+  w.part2 = take(B * (size_t)w.n_tiles * sizeof(float4));
+  w.total = off;
+  return w;
+}
+
+// ----------------------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct MapKey {
+  uintptr_t ptr;
+  uint64_t d0, d1, d2;
+  uint32_t b0, b1, b2, rank;
+  int dev;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && b0 == o.b0 && b1 == o.b1 &&
+           b2 == o.b2 && rank == o.rank && dev == o.dev;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    size_t h = std::hash<uintptr_t>()(k.ptr);
+    h ^= std::hash<uint64_t>()(k.d0 * 1315423911u + k.d1 * 2654435761u + k.d2) + 0x9e3779b9 +
+         (h << 6) + (h >> 2);
+    h ^= (size_t)k.b0 * 31 + k.b1 * 17 + k.b2 * 7 + k.rank + (size_t)k.dev * 101;
+    return h;
+  }
+};
+
+static std::mutex g_map_mu;
+static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
+
+// bf16 tensor map with 128-byte swizzle.  rank 2: dims {d0, d1}, row stride d0*2 bytes;
+// rank 3: dims {d0, d1, d2}, strides {d0*2, d0*d1*2}.  Cached per (pointer, shape, box, device).
+static etree_status get_map(const void* ptr, int rank, uint64_t d0, uint64_t d1, uint64_t d2,
+                            uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMap* out) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  MapKey key{reinterpret_cast<uintptr_t>(ptr), d0, d1, d2, b0, b1, b2, (uint32_t)rank, dev};
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *out = it->second;
+      return ETREE_OK;
+    }
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(ETREE_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMap m;
+  CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ETREE_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    if (g_maps.size() > 4096) g_maps.clear();
+    g_maps.emplace(key, m);
+  }
+  *out = m;
+  return ETREE_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static etree_status check_batch(const etree_batch* b) {
+  if (!b) return fail(ETREE_EINVAL, "batch is NULL");
+  if (b->B < 1 || b->B > ETREE_MAX_REQUESTS)
+    return fail(ETREE_EINVAL, "B=%d outside [1, %d]", b->B, ETREE_MAX_REQUESTS);
+  if (b->n_max < 1 || b->n_max > ETREE_MAX_NODES)
+    return fail(ETREE_EINVAL, "n_max=%d outside [1, %d]", b->n_max, ETREE_MAX_NODES);
+  if (b->n_total < b->B || (int64_t)b->n_total > (int64_t)b->B * b->n_max)
+    return fail(ETREE_EINVAL, "n_total=%d inconsistent with B=%d, n_max=%d", b->n_total, b->B,
+                b->n_max);
+  if (b->kv_len_max < 0) return fail(ETREE_EINVAL, "kv_len_max < 0");
+  if (!b->cu_nodes || !b->parent || !b->tokens || !b->kv_len || !b->slot_base || !b->slot_cap)
+    return fail(ETREE_EINVAL, "a batch array is NULL");
+  return ETREE_OK;
+}
+
+static etree_status check_ws(const etree_batch* b, int hq, int hkv, int hidden_dim, int vocab,
+                             void* ws, size_t bytes) {
+  if (!ws) return fail(ETREE_EINVAL, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0)
+    return fail(ETREE_EINVAL, "workspace is not 256-byte aligned");
+  const size_t need = layout(b, hq, hkv, hidden_dim, vocab).total;
+  if (bytes < need) return fail(ETREE_EINVAL, "workspace has %zu bytes, needs %zu", bytes, need);
+  return ETREE_OK;
+}
+
+template <class T>
+static T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace etree
+
+using namespace etree;
+
+// =================================================================================== C ABI
+extern "C" {
+
+int etree_version(void) { return 100; }
+
+const char* etree_strerror(etree_status s) {
+  switch (s) {
+    case ETREE_OK: return "ok";
+    case ETREE_EINVAL: return "invalid argument";
+    case ETREE_EUNSUPPORTED: return "unsupported configuration";
+    case ETREE_ECUDA: return "CUDA error";
+    case ETREE_EDEVICE: return "device-detected input error";
+    case ETREE_ETIMEOUT: return "on-device wait timed out";
+    case ETREE_ENOSPACE: return "request cache slots exhausted";
+  }
+  return "unknown status";
+}
+
+const char* etree_last_error(void) { return g_err; }
+
+etree_status etree_attn_plan(const etree_batch* batch, int hq, int hkv, int32_t* warps,
+                             int32_t* row_chunks, int32_t* splits, int32_t* tiles_per_split,
+                             int32_t* launches) {
+  etree_status st = check_batch(batch);
+  if (st) return st;
+  if (hq < 1 || hkv < 1 || hq % hkv != 0 || hq / hkv > 64)
+    return fail(ETREE_EINVAL, "hq=%d, hkv=%d", hq, hkv);
+  const AttnPlan pl = plan_attn(batch, hq, hkv);
+  if (warps) *warps = pl.nw;
+  if (row_chunks) *row_chunks = pl.mchunks;
+  if (splits) *splits = pl.nsplit;
+  if (tiles_per_split) *tiles_per_split = pl.tps;
+  if (launches) *launches = pl.nsplit > 1 ? 2 : 1;
+  return ETREE_OK;
+}
+
+size_t etree_workspace_size(const etree_batch* batch, int hq, int hkv, int head_dim,
+                            int hidden_dim, int vocab) {
+  (void)head_dim;
+  if (check_batch(batch) != ETREE_OK) return 0;
+  return layout(batch, hq, hkv, hidden_dim, vocab).total;
+}
+
+etree_status etree_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || workspace_bytes < sizeof(WsHeader))
+    return fail(ETREE_EINVAL, "workspace too small");
+  cudaError_t e =
+      cudaMemsetAsync(workspace, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_workspace_init");
+}
+
+etree_status etree_device_status(void* workspace, void* stream, int32_t* detail) {
+  if (!workspace) return fail(ETREE_EINVAL, "workspace is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "etree_device_status sync");
+  int32_t h[2] = {0, 0};
+  e = cudaMemcpy(h, workspace, sizeof h, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "etree_device_status read");
+  e = cudaMemsetAsync(workspace, 0, sizeof h, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "etree_device_status clear");
+  if (detail) *detail = h[1];
+  return static_cast<etree_status>(h[0]);
+}
+
+etree_status etree_verify_attn(const etree_batch* b, const uint16_t* q, const uint16_t* k_tree,
+                               const uint16_t* v_tree, const uint16_t* k_cache,
+                               const uint16_t* v_cache, int64_t cache_slots, int hq, int hkv,
+                               int head_dim, float scale, uint16_t* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  etree_status st = check_batch(b);
+  if (st) return st;
+  if (head_dim != ETREE_HEAD_DIM)
+    return fail(ETREE_EUNSUPPORTED, "head_dim=%d (only 128 is built)", head_dim);
+  if (hq < 1 || hkv < 1 || hq % hkv != 0 || hq / hkv > 64)
+    return fail(ETREE_EINVAL, "hq=%d, hkv=%d: need hq %% hkv == 0 and hq/hkv <= 64", hq, hkv);
+  if (!q || !k_tree || !v_tree || !k_cache || !v_cache || !out)
+    return fail(ETREE_EINVAL, "a tensor pointer is NULL");
+  if (!aligned16(q) || !aligned16(k_tree) || !aligned16(v_tree) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(out) || (lse && ((uintptr_t)lse & 3)))
+    return fail(ETREE_EINVAL, "tensors must be 16-byte aligned");
+  if (cache_slots < 1 || cache_slots > INT32_MAX)
+    return fail(ETREE_EINVAL, "cache_slots=%lld outside [1, 2^31)", (long long)cache_slots);
+  if (!std::isfinite(scale)) return fail(ETREE_EINVAL, "scale is not finite");
+  if ((st = check_ws(b, hq, hkv, 0, 0, workspace, workspace_bytes))) return st;
+
+  const AttnPlan pl = plan_attn(b, hq, hkv);
+  CUtensorMap kc, vc, kt, vt;
+  if ((st = get_map(k_cache, 3, 128, hkv, cache_slots, 64, 1, 64, &kc))) return st;
+  if ((st = get_map(v_cache, 3, 128, hkv, cache_slots, 64, 1, 64, &vc))) return st;
+  if ((st = get_map(k_tree, 3, 128, hkv, b->n_total, 64, 1, 64, &kt))) return st;
+  if ((st = get_map(v_tree, 3, 128, hkv, b->n_total, 64, 1, 64, &vt))) return st;
+
+  const WsLayout w = layout(b, hq, hkv, 0, 0);
+  AttnParams p{};
+  p.cu_nodes = b->cu_nodes;
+  p.parent = b->parent;
+  p.kv_len = b->kv_len;
+  p.slot_base = b->slot_base;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.o_part = at<float>(workspace, w.o_part);
+  p.ml_part = at<float2>(workspace, w.ml_part);
+  p.ws = at<WsHeader>(workspace, 0);
+  p.B = b->B;
+  p.hq = hq;
+  p.hkv = hkv;
+  p.G = pl.G;
+  p.n_max = b->n_max;
+  p.kv_len_max = b->kv_len_max;
+  p.cache_slots = cache_slots;
+  p.mchunks = pl.mchunks;
+  p.nsplit = pl.nsplit;
+  p.tps = pl.tps;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaError_t e = launch_attn(kc, vc, kt, vt, p, pl.nw, pl.stages, b->n_total,
+                              static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_verify_attn launch");
+}
+
+etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
+                                 const uint16_t* w_lm, int hidden_dim, int vocab,
+                                 float temperature, const float* q_draft, uint64_t seed,
+                                 uint64_t step, int32_t* accept_len, int32_t* path,
+                                 int32_t* out_tokens, int32_t* node_argmax, float* node_gap,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  etree_status st = check_batch(b);
+  if (st) return st;
+  if (hidden_dim < 64 || hidden_dim % 64 != 0)
+    return fail(ETREE_EUNSUPPORTED, "hidden_dim=%d must be a positive multiple of 64",
+                hidden_dim);
+  if (vocab < 1) return fail(ETREE_EINVAL, "vocab=%d", vocab);
+  if (!(temperature >= 0.f) || !std::isfinite(temperature))
+    return fail(ETREE_EINVAL, "temperature must be finite and >= 0");
+  if (temperature > 0.f && !q_draft) return fail(ETREE_EINVAL, "T > 0 needs q_draft");
+  if (!hidden || !w_lm || !accept_len || !path || !out_tokens)
+    return fail(ETREE_EINVAL, "a tensor pointer is NULL");
+  if (!aligned16(hidden) || !aligned16(w_lm))
+    return fail(ETREE_EINVAL, "hidden and w_lm must be 16-byte aligned");
+  if ((st = check_ws(b, 0, 0, hidden_dim, vocab, workspace, workspace_bytes))) return st;
+  // the workspace regions used here do not depend on the attention shape
+  const WsLayout w = layout(b, 0, 0, hidden_dim, vocab);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  CUtensorMap ta, tb;
+  if ((st = get_map(hidden, 2, hidden_dim, b->n_total, 1, 64, 128, 1, &ta))) return st;
+  if ((st = get_map(w_lm, 2, hidden_dim, vocab, 1, 64, 256, 1, &tb))) return st;
+
+  GemmParams g{};
+  g.M = b->n_total;
+  g.V = vocab;
+  g.K = hidden_dim;
+  g.m_tiles = (b->n_total + 127) / 128;
+  g.n_tiles = w.n_tiles;
+  g.num_tiles = g.m_tiles * g.n_tiles;
+  g.k_blocks = hidden_dim / 64;
+  g.ws = at<WsHeader>(workspace, 0);
+  g.part = at<float4>(workspace, w.part);
+  g.child_tok = at<int32_t>(workspace, w.child_tok);
+  g.zchild = at<float>(workspace, w.zchild);
+  g.k_log2 = temperature > 0.f ? 1.4426950408889634f / temperature : 0.f;
+  g.stop_row = at<int32_t>(workspace, w.stop_row);
+  g.stop_node = at<int32_t>(workspace, w.stop_node);
+  g.mode = at<int32_t>(workspace, w.mode);
+  g.lse2 = at<float>(workspace, w.lse2);
+  g.q_draft = q_draft;
+  g.seed = seed;
+  g.step = step;
+
+  AcceptParams a{};
+  a.B = b->B;
+  a.n_max = b->n_max;
+  a.V = vocab;
+  a.n_tiles = w.n_tiles;
+  a.cu_nodes = b->cu_nodes;
+  a.parent = b->parent;
+  a.tokens = b->tokens;
+  a.part = g.part;
+  a.accept_len = accept_len;
+  a.path = path;
+  a.out_tokens = out_tokens;
+  a.node_argmax = node_argmax;
+  a.node_gap = node_gap;
+  a.ws = g.ws;
+  a.k_log2 = g.k_log2;
+  a.zchild = g.zchild;
+  a.lse2 = at<float>(workspace, w.lse2);
+  a.q_draft = q_draft;
+  a.seed = seed;
+  a.step = step;
+  a.stop_row = at<int32_t>(workspace, w.stop_row);
+  a.stop_node = at<int32_t>(workspace, w.stop_node);
+  a.mode = at<int32_t>(workspace, w.mode);
+  a.hidden = reinterpret_cast<const __nv_bfloat16*>(hidden);
+  a.hid2 = at<__nv_bfloat16>(workspace, w.hid2);
+  a.H = hidden_dim;
+  a.part2 = at<float4>(workspace, w.part2);
+
+  const int sms = sm_count();
+  cudaError_t e;
+  if (temperature == 0.f) {
+    e = launch_lmhead(0, ta, tb, g, std::min(g.num_tiles, sms), s);
+    if (e == cudaSuccess) e = launch_accept_greedy(a, s);
+    return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T=0)");
+  }
+  e = launch_chain_prep(a, at<int32_t>(workspace, w.child_tok), s);
+  if (e == cudaSuccess) e = launch_lmhead(1, ta, tb, g, std::min(g.num_tiles, sms), s);
+  if (e == cudaSuccess) e = launch_accept_chain(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "etree_lmhead_accept (T>0, pass 1)");
+  CUtensorMap th;
+  if ((st = get_map(a.hid2, 2, hidden_dim, b->B, 1, 64, 128, 1, &th))) return st;
+  GemmParams g2 = g;
+  g2.M = b->B;
+  g2.m_tiles = (b->B + 127) / 128;
+  g2.num_tiles = g2.m_tiles * g2.n_tiles;
+  g2.part = at<float4>(workspace, w.part2);
+  e = launch_lmhead(2, th, tb, g2, std::min(g2.num_tiles, sms), s);
+  if (e == cudaSuccess) e = launch_bonus(a, s);
+  return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T>0, pass 2)");
+}
+
+etree_status etree_kv_compact(const etree_batch* b, const int32_t* accept_len,
+                              const int32_t* path, const uint16_t* k_tree,
+                              const uint16_t* v_tree, uint16_t* k_cache, uint16_t* v_cache,
+                              int n_layers, int64_t tree_layer_stride,
+                              int64_t cache_layer_stride, int hkv, int head_dim,
+                              int32_t* kv_len_out, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  etree_status st = check_batch(b);
+  if (st) return st;
+  if (head_dim != ETREE_HEAD_DIM)
+    return fail(ETREE_EUNSUPPORTED, "head_dim=%d (only 128 is built)", head_dim);
+  if (hkv < 1 || n_layers < 1 || n_layers > 65535)
+    return fail(ETREE_EINVAL, "hkv=%d, n_layers=%d", hkv, n_layers);
+  if (!accept_len || !path || !k_tree || !v_tree || !k_cache || !v_cache || !kv_len_out)
+    return fail(ETREE_EINVAL, "a pointer is NULL");
+  if (kv_len_out == b->kv_len) return fail(ETREE_EINVAL, "kv_len_out aliases batch->kv_len");
+  if (!aligned16(k_tree) || !aligned16(v_tree) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(ETREE_EINVAL, "K/V tensors must be 16-byte aligned");
+  const int64_t row = (int64_t)hkv * head_dim;
+  if (n_layers > 1 && (tree_layer_stride < row * b->n_total || cache_layer_stride < row ||
+                       tree_layer_stride % 8 || cache_layer_stride % 8))
+    return fail(ETREE_EINVAL, "layer strides must cover a layer and be multiples of 8");
+  if ((st = check_ws(b, 0, 0, 0, 0, workspace, workspace_bytes))) return st;
+  CompactParams p{};
+  p.cu_nodes = b->cu_nodes;
+  p.kv_len = b->kv_len;
+  p.slot_base = b->slot_base;
+  p.slot_cap = b->slot_cap;
+  p.accept_len = accept_len;
+  p.path = path;
+  p.k_tree = reinterpret_cast<const uint4*>(k_tree);
+  p.v_tree = reinterpret_cast<const uint4*>(v_tree);
+  p.k_cache = reinterpret_cast<uint4*>(k_cache);
+  p.v_cache = reinterpret_cast<uint4*>(v_cache);
+  p.kv_len_out = kv_len_out;
+  p.ws = at<WsHeader>(workspace, 0);
+  p.B = b->B;
+  p.n_max = b->n_max;
+  p.n_layers = n_layers;
+  p.tree_layer_stride16 = tree_layer_stride / 8;
+  p.cache_layer_stride16 = cache_layer_stride / 8;
+  p.row16 = (int)(row / 8);
+  cudaError_t e = launch_compact(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_kv_compact launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,94 @@
+// kernels.cuh -- parameter blocks and launchers of the etree kernels, shared by the kernel
+// translation units and the C-ABI layer.
+#pragma once
+#include "common.cuh"
+
+namespace etree {
+
+struct AttnParams {
+  const int32_t* cu_nodes;
+  const int32_t* parent;
+  const int32_t* kv_len;
+  const int64_t* slot_base;
+  const __nv_bfloat16* q;
+  __nv_bfloat16* out;
+  float* lse;
+  float* o_part;
+  float2* ml_part;
+  WsHeader* ws;
+  int B, hq, hkv, G, n_max, kv_len_max;
+  int64_t cache_slots;
+  int mchunks, nsplit, tps;
+  float scale_log2;
+};
+cudaError_t launch_attn(const CUtensorMap& kc, const CUtensorMap& vc, const CUtensorMap& kt,
+                        const CUtensorMap& vt, const AttnParams& p, int nw, int stages,
+                        int n_total, cudaStream_t stream);
+
+struct GemmParams {
+  int M, V, K, m_tiles, n_tiles, num_tiles, k_blocks;
+  WsHeader* ws;
+  float4* part;
+  const int32_t* child_tok;
+  float* zchild;
+  float k_log2;
+  const int32_t* stop_row;
+  const int32_t* stop_node;
+  const int32_t* mode;
+  const float* lse2;
+  const float* q_draft;
+  uint64_t seed, step;
+};
+cudaError_t launch_lmhead(int epi, const CUtensorMap& ta, const CUtensorMap& tb,
+                          const GemmParams& p, int grid, cudaStream_t stream);
+
+struct AcceptParams {
+  int B, n_max, V, n_tiles;
+  const int32_t* cu_nodes;
+  const int32_t* parent;
+  const int32_t* tokens;
+  const float4* part;
+  int32_t* accept_len;
+  int32_t* path;
+  int32_t* out_tokens;
+  int32_t* node_argmax;
+  float* node_gap;
+  WsHeader* ws;
+  float k_log2;
+  const float* zchild;
+  float* lse2;
+  const float* q_draft;
+  uint64_t seed, step;
+  int32_t* stop_row;
+  int32_t* stop_node;
+  int32_t* mode;
+  const __nv_bfloat16* hidden;
+  __nv_bfloat16* hid2;
+  int H;
+  const float4* part2;
+};
+cudaError_t launch_accept_greedy(const AcceptParams& p, cudaStream_t s);
+cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStream_t s);
+cudaError_t launch_accept_chain(const AcceptParams& p, cudaStream_t s);
+cudaError_t launch_bonus(const AcceptParams& p, cudaStream_t s);
+
+struct CompactParams {
+  const int32_t* cu_nodes;
+  const int32_t* kv_len;
+  const int64_t* slot_base;
+  const int32_t* slot_cap;
+  const int32_t* accept_len;
+  const int32_t* path;
+  const uint4* k_tree;
+  const uint4* v_tree;
+  uint4* k_cache;
+  uint4* v_cache;
+  int32_t* kv_len_out;
+  WsHeader* ws;
+  int B, n_max, n_layers;
+  int64_t tree_layer_stride16, cache_layer_stride16;
+  int row16;
+};
+cudaError_t launch_compact(const CompactParams& p, cudaStream_t s);
+
+}  // namespace etree

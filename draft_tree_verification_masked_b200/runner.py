@@ -1,0 +1,101 @@
+"""Device-side driver of one verification step over a workload (marshalling only).
+
+Uploads a :class:`~draft_tree_verification_masked_b200.workload.Workload` to the GPU, allocates
+the outputs and the workspace with PyTorch, and calls the three C-ABI entry points in order:
+tree attention (one layer), LM head + acceptance, KV compaction.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (etree_device_status, etree_kv_compact, etree_lmhead_accept, etree_verify_attn,
+               etree_workspace_init, etree_workspace_size, make_batch)
+
+
+class DeviceStep:
+    def __init__(self, wl, device: str = "cuda", n_layers: int = 1, pin: bool = False):
+        self.wl = wl
+        self.device = device
+        dev = torch.device(device)
+        i32 = torch.int32
+
+        def up(x, dtype=None):
+            t = torch.as_tensor(x) if not isinstance(x, torch.Tensor) else x
+            if dtype is not None:
+                t = t.to(dtype)
+            return t.contiguous().to(dev)
+
+        self.cu_nodes = up(wl.cu_nodes, i32)
+        self.parent = up(wl.parent, i32)
+        self.tokens = up(wl.tokens, i32)
+        self.kv_len = up(wl.kv_len, i32)
+        self.slot_base = up(wl.slot_base, torch.int64)
+        self.slot_cap = up(wl.slot_cap, i32)
+        self.batch = make_batch(self.cu_nodes, self.parent, self.tokens, self.kv_len,
+                                self.slot_base, self.slot_cap, wl.n_max, wl.kv_len_max)
+        self.q = up(wl.q)
+        self.k_tree = up(wl.k_tree)
+        self.v_tree = up(wl.v_tree)
+        self.k_cache = up(wl.k_cache)
+        self.v_cache = up(wl.v_cache)
+        self.hidden = up(wl.hidden)
+        self.w_lm = up(wl.w_lm)
+        self.q_draft = up(wl.q_draft) if wl.q_draft is not None else None
+        ntot, B = wl.n_total, wl.B
+        self.out = torch.empty(ntot, wl.hq, wl.head_dim, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(ntot, wl.hq, dtype=torch.float32, device=dev)
+        self.accept_len = torch.empty(B, dtype=i32, device=dev)
+        self.path = torch.empty(B, 64, dtype=i32, device=dev)
+        self.out_tokens = torch.empty(B, 65, dtype=i32, device=dev)
+        self.node_argmax = torch.empty(ntot, dtype=i32, device=dev)
+        self.node_gap = torch.empty(ntot, dtype=torch.float32, device=dev)
+        self.kv_len_out = torch.empty(B, dtype=i32, device=dev)
+        self.n_layers = n_layers
+        if n_layers == 1:
+            self.kt_layers, self.vt_layers = self.k_tree, self.v_tree
+            self.kc_layers, self.vc_layers = self.k_cache, self.v_cache
+        else:
+            # stacked per-layer copies; layer 0 holds the workload's tensors
+            self.kt_layers = self.k_tree.unsqueeze(0).repeat(n_layers, 1, 1, 1)
+            self.vt_layers = self.v_tree.unsqueeze(0).repeat(n_layers, 1, 1, 1)
+            self.kc_layers = torch.zeros((n_layers,) + tuple(self.k_cache.shape),
+                                         dtype=torch.bfloat16, device=dev)
+            self.vc_layers = torch.zeros_like(self.kc_layers)
+        self.tree_layer_stride = self.k_tree.numel()
+        self.cache_layer_stride = self.k_cache.numel()
+        size = etree_workspace_size(self.batch, wl.hq, wl.hkv, wl.head_dim, wl.hidden_dim,
+                                    wl.vocab)
+        self.ws = torch.zeros(max(size, 256), dtype=torch.uint8, device=dev)
+        etree_workspace_init(self.ws)
+        self.scale = 1.0 / float(wl.head_dim) ** 0.5
+
+    # --- the three calls
+    def attn(self, stream=None):
+        etree_verify_attn(self.batch, self.q, self.k_tree, self.v_tree, self.k_cache,
+                          self.v_cache, self.scale, self.out, self.lse, self.ws, stream)
+
+    def lmhead(self, stream=None):
+        etree_lmhead_accept(self.batch, self.hidden, self.w_lm, self.wl.temperature,
+                            self.q_draft, self.wl.seed, self.wl.step, self.accept_len, self.path,
+                            self.out_tokens, self.node_argmax, self.node_gap, self.ws, stream)
+
+    def compact(self, stream=None):
+        etree_kv_compact(self.batch, self.accept_len, self.path, self.kt_layers, self.vt_layers,
+                         self.kc_layers, self.vc_layers, self.n_layers, self.tree_layer_stride,
+                         self.cache_layer_stride, self.kv_len_out, self.ws, stream)
+
+    def step(self, stream=None):
+        self.attn(stream)
+        self.lmhead(stream)
+        self.compact(stream)
+
+    def status(self):
+        return etree_device_status(self.ws)
+
+    def results(self):
+        torch.cuda.synchronize()
+        return dict(out=self.out.float().cpu(), lse=self.lse.cpu(),
+                    accept_len=self.accept_len.cpu().numpy(), path=self.path.cpu().numpy(),
+                    out_tokens=self.out_tokens.cpu().numpy(),
+                    node_argmax=self.node_argmax.cpu().numpy(),
+                    node_gap=self.node_gap.cpu().numpy(), kv_len_out=self.kv_len_out.cpu().numpy())

@@ -250,15 +250,22 @@ def generate(name: str, *, seed: int | None = None, step: int = 0, **overrides) 
     T = float(cfg["temperature"])
 
     # --- per-request trees, lengths and tokens
-    lo, hi = cfg["kv_len"]
-    kv_len = _rng(seed, "kv_len").integers(lo, hi + 1, size=B).astype(np.int32) if hi > lo \
-        else np.full(B, lo, dtype=np.int32)
+    if isinstance(cfg["kv_len"], list):            # explicit per-request lengths
+        kv_len = np.asarray(cfg["kv_len"], dtype=np.int32)
+        assert len(kv_len) == B
+    else:
+        lo, hi = cfg["kv_len"]
+        kv_len = _rng(seed, "kv_len").integers(lo, hi + 1, size=B).astype(np.int32) \
+            if hi > lo else np.full(B, lo, dtype=np.int32)
+    n_nodes = cfg["n_nodes"]
+    n_nodes = list(n_nodes) if isinstance(n_nodes, (list, tuple)) else [n_nodes] * B
+    assert len(n_nodes) == B
     parents, sizes = [], []
     for r in range(B):
         g = _rng(seed, "tree", r)
         dmin = cfg.get("depth_min", cfg["depth"])
         d = int(g.integers(dmin, cfg["depth"] + 1)) if dmin < cfg["depth"] else cfg["depth"]
-        p = make_tree(cfg["n_nodes"], d, cfg["branch"], cfg["width"], g)
+        p = make_tree(int(n_nodes[r]), d, cfg["branch"], cfg["width"], g)
         parents.append(p)
         sizes.append(len(p))
     cu = np.zeros(B + 1, dtype=np.int32)

@@ -1,0 +1,183 @@
+/*
+ * etree.h -- C ABI of libetree: the target model's one-pass verification of a draft token tree
+ * (EAGLE-style speculative decoding) on NVIDIA B200 (sm_100a).
+ *
+ * What the three calls compute.  Speculative decoding lets a small draft model propose tokens
+ * that the target model then checks all at once, in one parallel forward pass: the target keeps
+ * the longest drafted prefix consistent with its own distribution and adds one token of its own
+ * after the first rejected position ("Eagle-4 Released: Outpaces DFlash2 and DSpark ...",
+ * kongchang.com/en, section "Technical Background", speculative-decoding paragraph).  EAGLE-2's
+ * dynamic draft tree lets one verification cover several candidate paths (same section).  Tree
+ * verification needs an unquantized KV cache, and engines admit trees and chains for up to 512
+ * running requests ("EAGLE-4 官方推理代码发布：eagle-harness v0.1.0 ...", arex-research.com,
+ * paragraph on hardware coverage and limits).  Per-sequence acceptance lengths under continuous
+ * batching are the main engineering difficulty ("Eagle-4 Released ...", section "Current
+ * Limitation").
+ *
+ *   etree_verify_attn    tree-masked GQA attention of every tree node against its request's
+ *                        bf16 KV cache plus the tree nodes that are its ancestors (or itself);
+ *   etree_lmhead_accept  LM-head projection of every node's hidden state fused with a per-row
+ *                        argmax (T = 0) or max / log-sum-exp (T > 0) reduction -- logits are
+ *                        never written to memory -- followed by the acceptance walk that returns
+ *                        the longest accepted path and the bonus token;
+ *   etree_kv_compact     copies the root's and the accepted nodes' K/V into the request's next
+ *                        cache slots.
+ *
+ * Conventions shared by every call:
+ *  - Pointers are DEVICE pointers unless stated; the caller owns all memory.  bf16 tensors are
+ *    passed as uint16_t bit patterns.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *  - Calls are asynchronous: they validate host-visible arguments, enqueue kernels and return.
+ *  - Problems visible on the host return at once (ETREE_EINVAL / ETREE_EUNSUPPORTED) and enqueue
+ *    nothing.  Problems visible only on the device (a malformed parent array, a KV length past
+ *    its bound, a full cache) are recorded in the workspace status word; the affected request is
+ *    skipped with safe outputs and etree_device_status() returns the code.  No kernel traps.
+ *  - The library allocates no device memory.  The caller passes a workspace of at least
+ *    etree_workspace_size() bytes (256-byte aligned), zeroed once by etree_workspace_init().
+ *    One workspace serves one stream at a time.
+ *  - The only global state is a per-process cache of TMA descriptors keyed by pointer and shape.
+ */
+#ifndef ETREE_H
+#define ETREE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ETREE_OK = 0,
+  ETREE_EINVAL = -1,        /* bad argument: null pointer, size out of range, misalignment   */
+  ETREE_EUNSUPPORTED = -2,  /* valid but not supported: head_dim != 128, T > 0 on a tree ...  */
+  ETREE_ECUDA = -3,         /* a CUDA runtime/driver call failed                              */
+  ETREE_EDEVICE = -4,       /* device-detected input error (malformed tree, bad length, ...)  */
+  ETREE_ETIMEOUT = -5,      /* a bounded on-device wait gave up                               */
+  ETREE_ENOSPACE = -6       /* a request's cache slots cannot hold the accepted tokens        */
+} etree_status;
+
+/* Limits of this build. */
+#define ETREE_MAX_NODES 64      /* nodes per tree, root included (ancestor masks are uint64)  */
+#define ETREE_MAX_REQUESTS 4096
+#define ETREE_HEAD_DIM 128
+#define ETREE_PATH_STRIDE 64    /* path is [B][64]                                            */
+#define ETREE_OUT_STRIDE 65     /* out_tokens is [B][65]: up to 63 accepted + 1 bonus, padded */
+
+/*
+ * One verification step's batch of requests.  Request r owns nodes cu_nodes[r] ..
+ * cu_nodes[r+1]-1 (its "local" node j is global node cu_nodes[r] + j).  Local node 0 is the
+ * root, the last committed token: its K/V are produced by this step and are NOT yet in the
+ * cache.  Every other node is a draft token whose parent has a smaller local index.
+ */
+typedef struct etree_batch {
+  int32_t B;                  /* requests, 1 .. ETREE_MAX_REQUESTS                          */
+  int32_t n_total;            /* total nodes = cu_nodes[B]                                   */
+  int32_t n_max;              /* max nodes of one request, 1 .. ETREE_MAX_NODES              */
+  int32_t kv_len_max;         /* host-side upper bound on every kv_len[r] (sizes the grid)  */
+  const int32_t *cu_nodes;    /* device [B+1], cu_nodes[0] = 0, non-decreasing               */
+  const int32_t *parent;      /* device [n_total], LOCAL parent; -1 for the root            */
+  const int32_t *tokens;      /* device [n_total], token id of each node                     */
+  const int32_t *kv_len;      /* device [B], tokens already in request r's cache             */
+  const int64_t *slot_base;   /* device [B], first pooled-cache slot of request r            */
+  const int32_t *slot_cap;    /* device [B], slots reserved for request r                    */
+} etree_batch;
+
+/* Bytes of workspace that the three calls need for this batch and these shapes. */
+size_t etree_workspace_size(const etree_batch *batch, int hq, int hkv, int head_dim,
+                            int hidden_dim, int vocab);
+
+/* Zeroes the status words of a fresh workspace (asynchronous, on `stream`). */
+etree_status etree_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Tree-masked GQA attention.  For node i of request r and query head h (KV head h / (hq/hkv)):
+ * keys = the kv_len[r] cached positions (pooled rows slot_base[r] + t) followed by the tree nodes
+ * j with j == i or j an ancestor of i;  out = softmax(scale * q k^T) v;  lse = log sum exp.
+ *   q        [n_total][hq][head_dim]  bf16
+ *   k_tree   [n_total][hkv][head_dim] bf16, v_tree likewise (this step's K/V of every node)
+ *   k_cache  [cache_slots][hkv][head_dim] bf16 pooled cache, v_cache likewise
+ *   out      [n_total][hq][head_dim]  bf16
+ *   lse      [n_total][hq] fp32 natural-log log-sum-exp of the scaled scores; may be NULL
+ * head_dim must be 128; hq % hkv == 0; hq/hkv <= 64; all tensors 16-byte aligned.
+ * The library reads `cache_slots` rows at most; cached rows at positions >= kv_len[r] are ignored.
+ */
+etree_status etree_verify_attn(const etree_batch *batch, const uint16_t *q,
+                               const uint16_t *k_tree, const uint16_t *v_tree,
+                               const uint16_t *k_cache, const uint16_t *v_cache,
+                               int64_t cache_slots, int hq, int hkv, int head_dim, float scale,
+                               uint16_t *out, float *lse, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/*
+ * LM head + acceptance.  z = hidden W^T (fp32 accumulate over bf16 inputs) for every node row.
+ *  T == 0 (greedy): t*(u) = argmax z_u (lowest id on ties).  From the root, repeatedly move to
+ *    the lowest-index child whose token equals t*(current); the node where no child matches
+ *    stops the walk and t* there is the bonus token.
+ *  T > 0 (chains only, every node has <= 1 child): p_u = softmax(z_u / T); node k's token x was
+ *    drafted from q_draft row k-1; it is accepted iff U * q(x) < p(x), U a seeded uniform.  At
+ *    the first rejection (node u) the bonus is drawn from norm(max(0, p_u - q_u)); when all are
+ *    accepted it is drawn from p of the last node.  Draws use an exponential race with
+ *    Philox4x64-10 uniforms keyed by (seed, step) and countered by (vocab id/4, node, request,
+ *    stream), so results are reproducible bit for bit.  A branching tree records
+ *    ETREE_EUNSUPPORTED (detail 5, "not a chain") and that request accepts nothing.
+ *   hidden      [n_total][hidden_dim] bf16;   w_lm [vocab][hidden_dim] bf16 (K contiguous)
+ *   q_draft     [n_total][vocab] fp32 draft probabilities (T > 0 only, else may be NULL)
+ *   accept_len  [B] accepted draft nodes a_r (0 .. n_r - 1)
+ *   path        [B][64] local node ids: path[r][0] = 0 (root), path[r][1..a_r]; rest -1
+ *   out_tokens  [B][65] tokens of the accepted nodes, then the bonus token; rest -1
+ *   node_argmax [n_total] per-node argmax (T == 0 only; may be NULL)
+ *   node_gap    [n_total] per-node top1 - top2 logit gap, fp32 (T == 0 only; may be NULL)
+ * hidden_dim must be a multiple of 64; vocab >= 256.
+ */
+etree_status etree_lmhead_accept(const etree_batch *batch, const uint16_t *hidden,
+                                 const uint16_t *w_lm, int hidden_dim, int vocab,
+                                 float temperature, const float *q_draft, uint64_t seed,
+                                 uint64_t step, int32_t *accept_len, int32_t *path,
+                                 int32_t *out_tokens, int32_t *node_argmax, float *node_gap,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * KV compaction.  For each of n_layers layers and each request r with a = accept_len[r]:
+ *   cache[slot_base[r] + kv_len[r] + k] <- tree[cu_nodes[r] + path[r][k]],  k = 0 .. a,
+ * for K and V, then kv_len_out[r] = kv_len[r] + a + 1 (the bonus token's K/V come next step).
+ * Rows are [hkv][head_dim] bf16.  Layer l of the tree K/V starts tree_layer_stride ELEMENTS after
+ * layer l-1, likewise for the caches.  kv_len_out must not alias batch->kv_len.  A request whose
+ * new rows would pass slot_cap[r] is left untouched (kv_len_out = kv_len) with ETREE_ENOSPACE.
+ */
+etree_status etree_kv_compact(const etree_batch *batch, const int32_t *accept_len,
+                              const int32_t *path, const uint16_t *k_tree,
+                              const uint16_t *v_tree, uint16_t *k_cache, uint16_t *v_cache,
+                              int n_layers, int64_t tree_layer_stride,
+                              int64_t cache_layer_stride, int hkv, int head_dim,
+                              int32_t *kv_len_out, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/*
+ * Synchronizes `stream`, reads the workspace status word (the first device-detected error since
+ * the last read, ETREE_OK if none), stores its detail code in *detail (if not NULL) and clears
+ * both words.
+ */
+etree_status etree_device_status(void *workspace, void *stream, int32_t *detail);
+
+/* Static description of a status code. */
+const char *etree_strerror(etree_status status);
+
+/* Message describing the last host-side failure of a call on this thread ("" if none). */
+const char *etree_last_error(void);
+
+/*
+ * The launch plan etree_verify_attn uses for this batch and head shape (host-only, no device
+ * work): consumer warps per CTA, row chunks per (request, KV head), KV splits, 64-key tiles per
+ * split, and the number of kernels the call launches (1, or 2 with the split combine).
+ */
+etree_status etree_attn_plan(const etree_batch *batch, int hq, int hkv, int32_t *warps,
+                             int32_t *row_chunks, int32_t *splits, int32_t *tiles_per_split,
+                             int32_t *launches);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int etree_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ETREE_H */

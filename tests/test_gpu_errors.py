@@ -1,0 +1,100 @@
+"""Error behaviour through the C ABI on the GPU: host-visible problems return at once,
+device-visible problems set the workspace status word and never trap; the context stays usable.
+"""
+import pytest
+import torch
+
+import draft_tree_verification_masked_b200 as et
+from draft_tree_verification_masked_b200 import workload as W
+from draft_tree_verification_masked_b200.runner import DeviceStep
+
+pytestmark = pytest.mark.gpu
+
+EINVAL, EUNSUP, EDEVICE, ENOSPACE = -1, -2, -4, -6
+
+
+def _dev(**kw):
+    wl = W.generate("tiny", B=2, kv_len=[100, 300], hidden=256, vocab=512, **kw)
+    return wl, DeviceStep(wl)
+
+
+def _still_works():
+    wl, dev = _dev()
+    dev.step()
+    assert dev.status() == (0, 0)
+
+
+def test_malformed_parent_sets_device_status():
+    wl, dev = _dev()
+    dev.parent[int(wl.cu_nodes[1]) + 3] = 7          # parent not below its child
+    dev.step()
+    assert dev.status() == (EDEVICE, 1)
+    assert dev.status() == (0, 0)                     # read clears
+    _still_works()
+
+
+def test_kv_len_above_declared_bound():
+    wl, dev = _dev()
+    dev.kv_len[0] = wl.kv_len_max + 1
+    dev.attn()
+    assert dev.status() == (EDEVICE, 3)
+    _still_works()
+
+
+def test_cache_capacity_overflow_leaves_request_untouched():
+    wl, dev = _dev()
+    dev.slot_cap[1] = int(wl.kv_len[1])               # no room for even the root
+    before = dev.k_cache.clone()
+    dev.step()
+    assert dev.status() == (ENOSPACE, 4)
+    assert int(dev.kv_len_out[1]) == int(wl.kv_len[1])
+    b1 = int(wl.slot_base[1])
+    assert torch.equal(dev.k_cache[b1:], before[b1:])
+    _still_works()
+
+
+def test_stochastic_acceptance_on_a_branching_tree_is_unsupported():
+    wl = W.generate("tiny", B=2, kv_len=[100, 300], hidden=256, vocab=512)
+    wl.temperature = 1.0
+    wl.q_draft = torch.full((wl.n_total, wl.vocab), 1.0 / wl.vocab)
+    dev = DeviceStep(wl)
+    dev.lmhead()
+    assert dev.status() == (EUNSUP, 5)
+    _still_works()
+
+
+def test_host_argument_errors():
+    wl, dev = _dev()
+    b = dev.batch
+    call = dict(check=False)
+    # n_max above 64
+    old = b.n_max
+    b.n_max = 65
+    assert et.etree_verify_attn(b, dev.q, dev.k_tree, dev.v_tree, dev.k_cache, dev.v_cache,
+                                dev.scale, dev.out, dev.lse, dev.ws, **call) == EINVAL
+    b.n_max = old
+    # head_dim 64 is not built
+    q64 = torch.zeros(wl.n_total, wl.hq, 64, dtype=torch.bfloat16, device="cuda")
+    k64 = torch.zeros(wl.n_total, wl.hkv, 64, dtype=torch.bfloat16, device="cuda")
+    assert et.etree_verify_attn(b, q64, k64, k64, dev.k_cache, dev.v_cache, dev.scale,
+                                dev.out, dev.lse, dev.ws, **call) == EUNSUP
+    # misaligned tensor
+    buf = torch.zeros(dev.q.numel() + 8, dtype=torch.bfloat16, device="cuda")
+    qm = buf[1:1 + dev.q.numel()].view(dev.q.shape)
+    assert qm.data_ptr() % 16 == 2
+    assert et.etree_verify_attn(b, qm, dev.k_tree, dev.v_tree, dev.k_cache, dev.v_cache,
+                                dev.scale, dev.out, dev.lse, dev.ws, **call) == EINVAL
+    # workspace too small
+    small = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    assert et.etree_lmhead_accept(b, dev.hidden, dev.w_lm, 0.0, None, 0, 0, dev.accept_len,
+                                  dev.path, dev.out_tokens, None, None, small, **call) == EINVAL
+    # negative temperature; T > 0 without draft probabilities
+    assert et.etree_lmhead_accept(b, dev.hidden, dev.w_lm, -1.0, None, 0, 0, dev.accept_len,
+                                  dev.path, dev.out_tokens, None, None, dev.ws, **call) == EINVAL
+    assert et.etree_lmhead_accept(b, dev.hidden, dev.w_lm, 1.0, None, 0, 0, dev.accept_len,
+                                  dev.path, dev.out_tokens, None, None, dev.ws, **call) == EINVAL
+    # kv_len_out aliasing the batch's kv_len
+    assert et.etree_kv_compact(b, dev.accept_len, dev.path, dev.k_tree, dev.v_tree, dev.k_cache,
+                               dev.v_cache, 1, 0, 0, dev.kv_len, dev.ws, **call) == EINVAL
+    assert dev.status() == (0, 0)
+    _still_works()

@@ -1,0 +1,166 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same seeded inputs.
+
+Small cases compare every output; full-size workloads (the launch configuration the benchmark
+times) compare every output the oracle can afford and sampled attention rows otherwise.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from draft_tree_verification_masked_b200 import workload as W
+from draft_tree_verification_masked_b200.runner import DeviceStep
+
+from . import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(wl, n_layers=1):
+    dev = DeviceStep(wl, n_layers=n_layers)
+    dev.step()
+    st, det = dev.status()
+    assert st == 0, (st, det)
+    return dev, dev.results()
+
+
+def _full_check(wl, attn_rows=None, requests=None):
+    dev, res = _run(wl)
+    P.attn_compare(wl, dev, rows=attn_rows)
+    reqs = list(range(wl.B)) if requests is None else requests
+    if wl.temperature == 0.0:
+        excused, near, ores = P.greedy_compare(wl, res, reqs)
+    else:
+        excused, near, ores = P.chain_compare(wl, res, reqs)
+    P.compact_compare(wl, dev, ores, reqs, excused)
+    assert near <= max(1, len(reqs) // 10), near
+    return dev, res
+
+
+def test_tiny_config():
+    _full_check(W.generate("tiny"))
+
+
+def test_dense27b_single_request_full_size():
+    _full_check(W.generate("dense27b_b1"))
+
+
+@pytest.mark.parametrize("name", ["long32k", "long128k"])
+def test_long_context(name):
+    wl = W.generate(name)
+    _full_check(wl, attn_rows=P.sample_rows(wl, 40))
+
+
+def test_batch64():
+    wl = W.generate("batch64")
+    g = np.random.default_rng(1)
+    reqs = sorted(g.choice(wl.B, 8, replace=False).tolist())
+    _full_check(wl, attn_rows=P.sample_rows(wl, 4), requests=reqs)
+
+
+def test_conc512_stochastic_chains():
+    wl = W.generate("conc512")
+    g = np.random.default_rng(2)
+    reqs = sorted(g.choice(wl.B, 24, replace=False).tolist())
+    _full_check(wl, attn_rows=P.sample_rows(wl, 1), requests=reqs)
+
+
+def test_ragged_trees_and_lengths():
+    wl = W.generate("tiny", B=6, n_nodes=[1, 4, 16, 33, 64, 2], kv_len=[0, 1, 63, 64, 65, 200],
+                    depth=8, depth_min=1, branch=None, width=16, vocab=4096 + 128 + 5,
+                    hidden=1024)
+    _full_check(wl)
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 2), (32, 1), (12, 4)])
+def test_gqa_group_sizes(hq, hkv):
+    wl = W.generate("tiny", B=3, hq=hq, hkv=hkv, kv_len=(100, 700), hidden=512, vocab=2048)
+    _full_check(wl)
+
+
+def test_chain_of_64_and_single_node():
+    wl = W.generate("tiny", B=2, n_nodes=[64, 1], depth=63, depth_min=63, branch=1,
+                    kv_len=[300, 5], hidden=256, vocab=1000)
+    _full_check(wl)
+
+
+@pytest.mark.parametrize("nsplit", ["1", "2", "3", "7"])
+def test_split_count_does_not_change_results(nsplit, monkeypatch):
+    monkeypatch.setenv("ETREE_NSPLIT", nsplit)
+    wl = W.generate("tiny", B=2, kv_len=[1000, 333], hidden=256, vocab=512)
+    _full_check(wl)
+
+
+def test_many_row_tiles_and_ragged_vocab():
+    wl = W.generate("tiny", B=9, kv_len=(10, 300), hidden=1024, vocab=4096 + 200)
+    assert wl.n_total > 128
+    _full_check(wl)
+
+
+@pytest.mark.parametrize("T", [1.0, 0.6])
+def test_stochastic_chains_small(T):
+    wl = W.generate("conc512", B=37, n_nodes=[4, 5, 6, 1, 2] * 7 + [4, 4], depth=5,
+                    depth_min=5, kv_len=(20, 400), hidden=512, vocab=4096 + 3, temperature=T)
+    _full_check(wl)
+
+
+def test_four_stage_kv_ring(monkeypatch):
+    monkeypatch.setenv("ETREE_STAGES", "4")
+    wl = W.generate("tiny", B=2, kv_len=[700, 64], hidden=256, vocab=512)
+    _full_check(wl)
+
+
+def test_repeat_is_bitwise_deterministic():
+    wl = W.generate("tiny", B=3, kv_len=(100, 900), hidden=512, vocab=2048)
+    dev = DeviceStep(wl)
+    dev.step()
+    first = dev.results()
+    dev.step()
+    second = dev.results()
+    for k in first:
+        a, b = first[k], second[k]
+        if isinstance(a, torch.Tensor):
+            assert torch.equal(a, b), k
+        else:
+            assert np.array_equal(a, b), k
+
+
+def test_multi_layer_compaction_against_oracle():
+    """Host-built accept lengths and paths, 5 layers with distinct contents, ragged requests."""
+    import oracle
+    wl = W.generate("tiny", B=5, n_nodes=[1, 4, 16, 33, 64], kv_len=[0, 7, 63, 64, 65],
+                    depth=8, depth_min=1, branch=None, width=16, hidden=256, vocab=512)
+    L = 5
+    g = np.random.default_rng(3)
+    a = np.array([0, 3, 5, 1, 63], dtype=np.int32)
+    path = np.full((wl.B, 64), -1, dtype=np.int32)
+    for r in range(wl.B):
+        n = wl.nodes(r)
+        path[r, 0] = 0
+        path[r, 1:a[r] + 1] = g.choice(np.arange(1, n), a[r], replace=False)
+    dev = DeviceStep(wl, n_layers=L)
+    kt = (torch.randn(L, wl.n_total, wl.hkv, 128) * 3).to(torch.bfloat16)
+    vt = (torch.randn(L, wl.n_total, wl.hkv, 128) * 3).to(torch.bfloat16)
+    kc = torch.randn(L, wl.slots, wl.hkv, 128).to(torch.bfloat16)
+    vc = torch.randn(L, wl.slots, wl.hkv, 128).to(torch.bfloat16)
+    dev.kt_layers.copy_(kt)
+    dev.vt_layers.copy_(vt)
+    dev.kc_layers.copy_(kc)
+    dev.vc_layers.copy_(vc)
+    dev.accept_len.copy_(torch.from_numpy(a))
+    dev.path.copy_(torch.from_numpy(path))
+    dev.compact()
+    assert dev.status()[0] == 0
+    ek, ev = oracle._u16(kc).copy(), oracle._u16(vc).copy()
+    st, newlen = oracle.kv_compact(wl.cu_nodes, wl.kv_len, wl.slot_base, wl.slot_cap, a, path,
+                                   kt, vt, ek, ev, L, wl.n_total * wl.hkv * 128,
+                                   wl.slots * wl.hkv * 128, wl.hkv, 128)
+    assert st == 0
+    assert np.array_equal(oracle._u16(dev.kc_layers.cpu()), ek)
+    assert np.array_equal(oracle._u16(dev.vc_layers.cpu()), ev)
+    assert np.array_equal(dev.kv_len_out.cpu().numpy(), newlen)
+
+
+def test_env_is_clean():
+    assert "ETREE_NSPLIT" not in os.environ
