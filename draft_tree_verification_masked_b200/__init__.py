@@ -25,7 +25,8 @@ import torch
 
 __all__ = [
     "EtreeError", "Batch", "make_batch", "lib", "library_path", "etree_workspace_size",
-    "etree_workspace_init", "etree_verify_attn", "etree_lmhead_accept", "etree_kv_compact",
+    "etree_workspace_init", "etree_verify_attn", "etree_verify_attn_noalloc",
+    "etree_lmhead_accept", "etree_kv_compact",
     "etree_device_status", "etree_strerror", "etree_version", "etree_attn_plan", "STATUS",
 ]
 
@@ -39,7 +40,7 @@ DETAIL = {0: "none", 1: "bad parent", 2: "bad node count", 3: "bad kv_len", 4: "
 
 EXPORTS = ["etree_workspace_size", "etree_workspace_init", "etree_verify_attn",
            "etree_lmhead_accept", "etree_kv_compact", "etree_device_status", "etree_strerror",
-           "etree_version", "etree_last_error", "etree_attn_plan"]
+           "etree_version", "etree_last_error", "etree_attn_plan", "etree_verify_attn_noalloc"]
 
 
 class EtreeError(RuntimeError):
@@ -94,6 +95,9 @@ def lib():
     L.etree_last_error.restype = C.c_char_p
     L.etree_version.argtypes = []
     L.etree_version.restype = C.c_int
+    L.etree_verify_attn_noalloc.argtypes = [bp, vp, vp, vp, vp, vp, i64, C.c_int, C.c_int,
+                                            C.c_int, f32, vp, vp, vp, vp]
+    L.etree_verify_attn_noalloc.restype = C.c_int
     ip = C.POINTER(C.c_int32)
     L.etree_attn_plan.argtypes = [bp, C.c_int, C.c_int, ip, ip, ip, ip, ip]
     L.etree_attn_plan.restype = C.c_int
@@ -175,6 +179,21 @@ def etree_verify_attn(batch: Batch, q, k_tree, v_tree, k_cache, v_cache, scale: 
         _ptr(k_cache, bf, "k_cache"), _ptr(v_cache, bf, "v_cache"), k_cache.shape[0], hq, hkv,
         d, float(scale), _ptr(out, bf, "out"), _ptr(lse, torch.float32, "lse"),
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
+    return _check(st) if check else st
+
+
+def etree_verify_attn_noalloc(batch: Batch, q, k_tree, v_tree, k_cache, v_cache, scale: float,
+                              out, lse, status_out=None, stream=None, check: bool = True) -> int:
+    """Tree attention backed by the library's static scratch array: for callers that cannot
+    allocate device memory (no workspace argument; see etree.h for the contract)."""
+    bf = torch.bfloat16
+    hq, d = q.shape[1], q.shape[2]
+    hkv = k_tree.shape[1]
+    st = lib().etree_verify_attn_noalloc(
+        C.byref(batch), _ptr(q, bf, "q"), _ptr(k_tree, bf, "k_tree"), _ptr(v_tree, bf, "v_tree"),
+        _ptr(k_cache, bf, "k_cache"), _ptr(v_cache, bf, "v_cache"), k_cache.shape[0], hq, hkv,
+        d, float(scale), _ptr(out, bf, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(status_out, torch.int32, "status_out"), _stream(stream))
     return _check(st) if check else st
 
 

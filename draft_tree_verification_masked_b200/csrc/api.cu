@@ -230,6 +230,35 @@ static T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+
+// ------------------------------------------------------------------ statically backed scratch
+// Scratch for etree_verify_attn_noalloc: a fixed array in device global memory, created when the
+// library's module is loaded on a device and held until the process exits.  Host code must not
+// use the symbol as a pointer; it asks the runtime for the device address once per device.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) uint8_t g_attn_scratch[kStaticScratchBytes];
+
+static std::mutex g_scratch_mu;
+static void* g_scratch_ptr[64] = {nullptr};
+
+// Device address of g_attn_scratch on the current device, resolved on the first call per device.
+static etree_status static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "etree_verify_attn_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(ETREE_EUNSUPPORTED, "device ordinal %d >= 64", dev);
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_attn_scratch);
+    if (e != cudaSuccess || !p)
+      return cuda_fail(e, "etree_verify_attn_noalloc: cudaGetSymbolAddress");
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return ETREE_OK;
+}
+
 }  // namespace etree
 
 using namespace etree;
@@ -501,6 +530,40 @@ etree_status etree_kv_compact(const etree_batch* b, const int32_t* accept_len,
   p.row16 = (int)(row / 8);
   cudaError_t e = launch_compact(p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_kv_compact launch");
+}
+
+// Tree attention without a caller workspace: the split partials and the status words live in
+// the library's static scratch array (see etree.h for the contract).
+etree_status etree_verify_attn_noalloc(const etree_batch* b, const uint16_t* q,
+                                       const uint16_t* k_tree, const uint16_t* v_tree,
+                                       const uint16_t* k_cache, const uint16_t* v_cache,
+                                       int64_t cache_slots, int hq, int hkv, int head_dim,
+                                       float scale, uint16_t* out, float* lse,
+                                       int32_t* status_out, void* stream) {
+  etree_status st = check_batch(b);
+  if (st) return st;
+  if (hq < 1 || hkv < 1 || hq % hkv != 0 || hq / hkv > 64)
+    return fail(ETREE_EINVAL, "hq=%d, hkv=%d: need hq %% hkv == 0 and hq/hkv <= 64", hq, hkv);
+  const size_t need = layout(b, hq, hkv, 0, 0).total;
+  if (need > kStaticScratchBytes)
+    return fail(ETREE_EINVAL,
+                "etree_verify_attn_noalloc: this batch needs %zu bytes of scratch, more than the "
+                "%zu-byte static array; use etree_verify_attn with a workspace",
+                need, kStaticScratchBytes);
+  void* ws = nullptr;
+  if ((st = static_scratch(&ws))) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the status words must start at zero for every call; the partials are written before read
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), s);
+  if (e != cudaSuccess) return cuda_fail(e, "etree_verify_attn_noalloc: clear status");
+  st = etree_verify_attn(b, q, k_tree, v_tree, k_cache, v_cache, cache_slots, hq, hkv, head_dim,
+                         scale, out, lse, ws, kStaticScratchBytes, stream);
+  if (st) return st;
+  if (status_out) {
+    e = cudaMemcpyAsync(status_out, ws, 2 * sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "etree_verify_attn_noalloc: copy status");
+  }
+  return ETREE_OK;
 }
 
 }  // extern "C"

@@ -109,6 +109,33 @@ etree_status etree_verify_attn(const etree_batch *batch, const uint16_t *q,
                                size_t workspace_bytes, void *stream);
 
 /*
+ * Tree attention for callers that cannot allocate device memory.  Serving engines commonly
+ * reserve nearly all of HBM for their own KV-cache pool at start-up, so a later cudaMalloc can
+ * fail; cudaMalloc can also synchronise the device and stall a latency-critical decode loop; and
+ * some plugin hosts hand their plugins no allocator at all.  Such callers cannot size and pass a
+ * workspace.  The paper has no counterpart: this is a deployment convenience.
+ * Same arguments, computation and output as etree_verify_attn, without a workspace: the split
+ * partials and the status words live in one static 32 MiB device array inside the library, which
+ * every device that loads the library holds until the process exits.  The call allocates nothing
+ * (no cudaMalloc / cudaFree, no allocating library routine).
+ *  - A batch that needs more than 32 MiB of scratch (etree_workspace_size with hidden_dim = 0 and
+ *    vocab = 0) is rejected with ETREE_EINVAL before any device work; use etree_verify_attn.
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress) and
+ *    caches it; make that first call before any stream capture.
+ *  - Every call clears the status words, then reuses the array, which keeps the last call's
+ *    contents.  Calls whose kernels overlap on the GPU (other streams, other threads) race on
+ *    the array: serialise them.
+ *  - status_out (device, 2 int32, may be NULL) receives the call's device status and detail code
+ *    (the values etree_device_status would return), written asynchronously on `stream`.
+ */
+etree_status etree_verify_attn_noalloc(const etree_batch *batch, const uint16_t *q,
+                                       const uint16_t *k_tree, const uint16_t *v_tree,
+                                       const uint16_t *k_cache, const uint16_t *v_cache,
+                                       int64_t cache_slots, int hq, int hkv, int head_dim,
+                                       float scale, uint16_t *out, float *lse,
+                                       int32_t *status_out, void *stream);
+
+/*
  * LM head + acceptance.  z = hidden W^T (fp32 accumulate over bf16 inputs) for every node row.
  *  T == 0 (greedy): t*(u) = argmax z_u (lowest id on ties).  From the root, repeatedly move to
  *    the lowest-index child whose token equals t*(current); the node where no child matches
