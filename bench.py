@@ -146,6 +146,19 @@ def ncu_traffic(kernel: str, workload: str, src_hash: str):
         return None
 
 
+# ----------------------------------------------------------------------------- multi-rank
+def reduce_over_ranks(step_s: float, e2e_s: float, tokens: int, world: int, device: str):
+    """Whole-job figures: the slowest rank's device times and the sum of accepted tokens."""
+    if world <= 1:
+        return step_s, e2e_s, float(tokens)
+    import torch.distributed as dist
+    v = torch.tensor([step_s, e2e_s, float(tokens)], device=device, dtype=torch.float64)
+    mx = v.clone()
+    dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    dist.all_reduce(v, op=dist.ReduceOp.SUM)
+    return float(mx[0]), float(mx[1]), float(v[2])
+
+
 # ------------------------------------------------------------------------------------ timing
 def time_steps(dev, steps, warmup, flush):
     for _ in range(warmup):
@@ -373,14 +386,7 @@ def main():
     tokens = main_res["toks"] * args.steps
     e2e_ms, h2d, d2h = main_res["e2e"]
     e2e_s = sum(e2e_ms) * 1e-3
-    if world > 1:
-        v = torch.tensor([step_s, e2e_s, float(tokens)], device="cuda", dtype=torch.float64)
-        mx = v.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        dist.all_reduce(v, op=dist.ReduceOp.SUM)
-        step_s, e2e_s, tokens_all = float(mx[0]), float(mx[1]), float(v[2])
-    else:
-        tokens_all = float(tokens)
+    step_s, e2e_s, tokens_all = reduce_over_ranks(step_s, e2e_s, tokens, world, "cuda")
     acc = main_res["dev"].accept_len.cpu().numpy()
     rep = kernel_report(wl, t, acc, peaks)
     rl = roofline(wl, rep, peaks, peak_kind, args.config)

@@ -99,7 +99,7 @@ def lib():
                                             C.c_int, f32, vp, vp, vp, vp]
     L.etree_verify_attn_noalloc.restype = C.c_int
     ip = C.POINTER(C.c_int32)
-    L.etree_attn_plan.argtypes = [bp, C.c_int, C.c_int, ip, ip, ip, ip, ip]
+    L.etree_attn_plan.argtypes = [bp, C.c_int, C.c_int, ip, ip, ip, ip, ip, ip]
     L.etree_attn_plan.restype = C.c_int
     _lib = L
     return L
@@ -228,10 +228,10 @@ def etree_kv_compact(batch: Batch, accept_len, path, k_tree, v_tree, k_cache, v_
 
 
 def etree_attn_plan(batch: Batch, hq: int, hkv: int) -> dict:
-    v = [C.c_int32(0) for _ in range(5)]
+    v = [C.c_int32(0) for _ in range(6)]
     _check(lib().etree_attn_plan(C.byref(batch), hq, hkv, *[C.byref(x) for x in v]))
-    return dict(zip(["warps", "row_chunks", "splits", "tiles_per_split", "launches"],
-                    [int(x.value) for x in v]))
+    return dict(zip(["kernel", "rows_per_cta", "row_blocks", "splits", "tiles_per_split",
+                     "launches"], [int(x.value) for x in v]))
 
 
 def etree_device_status(workspace: torch.Tensor, stream=None) -> tuple[int, int]:

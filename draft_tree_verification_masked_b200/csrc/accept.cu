@@ -52,86 +52,106 @@ __device__ __forceinline__ void merge_lse(float& m, float& s, float om, float os
   m = nm;
 }
 
-// Validates request r's parent array (parent[0] = -1, 0 <= parent[i] < i); all threads call.
-__device__ bool tree_ok(const AcceptParams& p, int base, int n, int* flag_s) {
-  if (threadIdx.x == 0) *flag_s = 0;
-  __syncthreads();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int pi = p.parent[base + i];
-    if ((i == 0 && pi != -1) || (i > 0 && (pi < 0 || pi >= i))) atomicOr(flag_s, 1);
+// ------------------------------------------------------------------------------------ T == 0
+// One warp per node row: merge the row's vocab-tile summaries into its argmax and top1 - top2 gap.
+__global__ void __launch_bounds__(256) row_top2_kernel(AcceptParams p, int32_t* arg_ws) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= p.n_total) return;
+  const float4* part = p.part + (size_t)row * p.n_tiles;
+  float t1 = -INFINITY, t2 = -INFINITY;
+  int id = -1;
+  int t = lane;
+  for (; t + 96 < p.n_tiles; t += 128) {             // four loads in flight per lane
+    const float4 a = part[t], b = part[t + 32], c = part[t + 64], d = part[t + 96];
+    merge_top2(t1, id, t2, a.x, __float_as_int(a.y), a.z);
+    merge_top2(t1, id, t2, b.x, __float_as_int(b.y), b.z);
+    merge_top2(t1, id, t2, c.x, __float_as_int(c.y), c.z);
+    merge_top2(t1, id, t2, d.x, __float_as_int(d.y), d.z);
   }
-  __syncthreads();
-  return *flag_s == 0;
+  for (; t < p.n_tiles; t += 32) {
+    const float4 a = part[t];
+    merge_top2(t1, id, t2, a.x, __float_as_int(a.y), a.z);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o1 = __shfl_xor_sync(0xffffffffu, t1, off);
+    const int oid = __shfl_xor_sync(0xffffffffu, id, off);
+    const float o2 = __shfl_xor_sync(0xffffffffu, t2, off);
+    merge_top2(t1, id, t2, o1, oid, o2);
+  }
+  if (lane == 0) {
+    arg_ws[row] = id;
+    if (p.node_argmax) p.node_argmax[row] = id;
+    if (p.node_gap) p.node_gap[row] = t1 - t2;
+  }
 }
 
-// ------------------------------------------------------------------------------------ T == 0
-__global__ void __launch_bounds__(256) accept_greedy_kernel(AcceptParams p) {
-  __shared__ int am_s[64], par_s[64], tok_s[64], pth_s[64];
-  __shared__ int flag_s;
-  const int r = blockIdx.x;
+// One warp per request: validate the tree, then walk from the root along the lowest-index child
+// that carries argmax(current node); the node where no child matches gives the bonus token.
+__global__ void __launch_bounds__(128) walk_greedy_kernel(AcceptParams p, const int32_t* arg_ws) {
+  __shared__ int am_s[4][64], par_s[4][64], tok_s[4][64], pth_s[4][64];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 4 + warp;
+  if (r >= p.B) return;
   const int base = p.cu_nodes[r];
   const int n = p.cu_nodes[r + 1] - base;
   int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
   int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
   if (n < 1 || n > p.n_max) {
-    if (threadIdx.x == 0) report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
-    if (threadIdx.x < 64) path[threadIdx.x] = -1;
-    if (threadIdx.x < 65) outt[threadIdx.x] = -1;
-    if (threadIdx.x == 0) p.accept_len[r] = 0;
+    if (lane == 0) {
+      report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
+      p.accept_len[r] = 0;
+    }
+    path[lane] = -1;
+    path[lane + 32] = -1;
+    outt[lane] = -1;
+    outt[lane + 32] = -1;
+    if (lane == 0) outt[64] = -1;
     return;
   }
-  const bool ok = tree_ok(p, base, n, &flag_s);
-  for (int i = warp; i < n; i += blockDim.x / 32) {
-    float t1 = -INFINITY, t2 = -INFINITY;
-    int id = -1;
-    const float4* row = p.part + (size_t)(base + i) * p.n_tiles;
-    for (int t = lane; t < p.n_tiles; t += 32) {
-      const float4 v = row[t];
-      merge_top2(t1, id, t2, v.x, __float_as_int(v.y), v.z);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float o1 = __shfl_xor_sync(0xffffffffu, t1, off);
-      const int oid = __shfl_xor_sync(0xffffffffu, id, off);
-      const float o2 = __shfl_xor_sync(0xffffffffu, t2, off);
-      merge_top2(t1, id, t2, o1, oid, o2);
-    }
-    if (lane == 0) {
-      am_s[i] = id;
-      par_s[i] = p.parent[base + i];
-      tok_s[i] = p.tokens[base + i];
-      if (p.node_argmax) p.node_argmax[base + i] = id;
-      if (p.node_gap) p.node_gap[base + i] = t1 - t2;
+  int* am = am_s[warp];
+  int* par = par_s[warp];
+  int* tok = tok_s[warp];
+  int* pth = pth_s[warp];
+  bool ok = true;
+  for (int j = lane; j < 64; j += 32) {
+    if (j < n) {
+      const int pj = p.parent[base + j];
+      ok = ok && ((j == 0) ? pj == -1 : (pj >= 0 && pj < j));
+      par[j] = pj;
+      tok[j] = p.tokens[base + j];
+      am[j] = arg_ws[base + j];
+    } else {
+      par[j] = -2;
+      tok[j] = -1;
+      am[j] = -1;
     }
   }
-  __syncthreads();
-  if (warp != 0) return;
-  if (!ok) report(p.ws, ETREE_EDEVICE, DET_BAD_PARENT);
-  // walk: from the root, follow the lowest-index child that carries argmax(current)
+  ok = __all_sync(0xffffffffu, ok);
+  __syncwarp();
+  if (!ok && lane == 0) report(p.ws, ETREE_EDEVICE, DET_BAD_PARENT);
   int u = 0, a = 0;
-  if (lane == 0) pth_s[0] = 0;
+  if (lane == 0) pth[0] = 0;
   if (ok) {
     for (int step = 0; step < 64; ++step) {
-      const int want = am_s[u];
-      const int j0 = lane, j1 = lane + 32;
-      const bool m0 = j0 >= 1 && j0 < n && par_s[j0] == u && tok_s[j0] == want;
-      const bool m1 = j1 < n && par_s[j1] == u && tok_s[j1] == want;
+      const int want = am[u];
+      const bool m0 = lane >= 1 && par[lane] == u && tok[lane] == want;
+      const bool m1 = par[lane + 32] == u && tok[lane + 32] == want;
       const unsigned b0 = __ballot_sync(0xffffffffu, m0);
       const unsigned b1 = __ballot_sync(0xffffffffu, m1);
       if (b0 == 0 && b1 == 0) break;
       const int c = b0 ? (__ffs(b0) - 1) : (32 + __ffs(b1) - 1);
       ++a;
-      if (lane == 0) pth_s[a] = c;
+      if (lane == 0) pth[a] = c;
       u = c;
     }
   }
   __syncwarp();
-  const int bonus = am_s[u];
-  // outputs: path[0..a], then -1; out_tokens[0..a-1] accepted tokens, [a] bonus, then -1
-  for (int k = lane; k < 64; k += 32) path[k] = (k <= a) ? pth_s[k] : -1;
+  const int bonus = am[u];
+  for (int k = lane; k < 64; k += 32) path[k] = (k <= a) ? pth[k] : -1;
   for (int k = lane; k < 65; k += 32)
-    outt[k] = (k < a) ? tok_s[pth_s[k + 1]] : (k == a ? bonus : -1);
+    outt[k] = (k < a) ? tok[pth[k + 1]] : (k == a ? bonus : -1);
   if (lane == 0) p.accept_len[r] = a;
 }
 
@@ -160,8 +180,35 @@ __global__ void chain_prep_kernel(AcceptParams p, int32_t* child_tok) {
   }
 }
 
+// One warp per node row: merge the (max, sum) summaries into log2 sum 2^(z log2(e) / T).
+__global__ void __launch_bounds__(256) row_lse_kernel(AcceptParams p) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= p.n_total) return;
+  const float4* part = p.part + (size_t)row * p.n_tiles;
+  float m = -INFINITY, s = 0.f;
+  int t = lane;
+  for (; t + 96 < p.n_tiles; t += 128) {
+    const float4 a = part[t], b = part[t + 32], c = part[t + 64], d = part[t + 96];
+    merge_lse(m, s, a.x, a.y);
+    merge_lse(m, s, b.x, b.y);
+    merge_lse(m, s, c.x, c.y);
+    merge_lse(m, s, d.x, d.y);
+  }
+  for (; t < p.n_tiles; t += 32) {
+    const float4 a = part[t];
+    merge_lse(m, s, a.x, a.y);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, m, off);
+    const float os = __shfl_xor_sync(0xffffffffu, s, off);
+    merge_lse(m, s, om, os);
+  }
+  if (lane == 0) p.lse2[row] = m + log2f(s);
+}
+
 __global__ void __launch_bounds__(128) accept_chain_kernel(AcceptParams p) {
-  __shared__ float lse_s[64];
   __shared__ int info_s[2];
   const int r = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -170,28 +217,7 @@ __global__ void __launch_bounds__(128) accept_chain_kernel(AcceptParams p) {
   int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
   int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
   const bool n_ok = n >= 1 && n <= p.n_max;
-  // per-row log2-sum-exp of z * log2(e) / T
-  if (n_ok) {
-    for (int i = warp; i < n; i += blockDim.x / 32) {
-      const float4* row = p.part + (size_t)(base + i) * p.n_tiles;
-      float m = -INFINITY, s = 0.f;
-      for (int t = lane; t < p.n_tiles; t += 32) {
-        const float4 v = row[t];
-        merge_lse(m, s, v.x, v.y);
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float om = __shfl_xor_sync(0xffffffffu, m, off);
-        const float os = __shfl_xor_sync(0xffffffffu, s, off);
-        merge_lse(m, s, om, os);
-      }
-      if (lane == 0) {
-        const float l2 = m + log2f(s);
-        lse_s[i] = l2;
-        p.lse2[base + i] = l2;
-      }
-    }
-  }
+  const float* lse_s = p.lse2 + base;
   __syncthreads();
   if (warp == 0) {
     int a = 0, rejected = 0;
@@ -218,8 +244,8 @@ __global__ void __launch_bounds__(128) accept_chain_kernel(AcceptParams p) {
         }
         const float px = exp2f(p.zchild[base + u] * p.k_log2 - lse_s[u]);
         const float qx = __ldg(p.q_draft + (size_t)(base + u) * p.V + x);
-        float U[4];
-        uniforms4(p.seed, p.step, 0u, (uint32_t)k, (uint32_t)r, 1u, U);
+        float U[8];
+        uniforms8(p.seed, p.step, 0u, (uint32_t)k, (uint32_t)r, 1u, U);
         if (U[0] * qx < px) {
           ++a;
         } else {
@@ -253,10 +279,10 @@ __global__ void __launch_bounds__(128) accept_chain_kernel(AcceptParams p) {
 __global__ void bonus_kernel(AcceptParams p) {
   const int r = blockIdx.x;
   const int lane = threadIdx.x;
-  const float4* row = p.part2 + (size_t)r * p.n_tiles;
+  const float4* row = p.part2 + (size_t)r * p.n_tiles2;
   float kr = -INFINITY, kp = -INFINITY;
   int ir = -1, ip = -1;
-  for (int t = lane; t < p.n_tiles; t += 32) {
+  for (int t = lane; t < p.n_tiles2; t += 32) {
     const float4 v = row[t];
     merge_key(kr, ir, v.x, __float_as_int(v.y));
     merge_key(kp, ip, v.z, __float_as_int(v.w));
@@ -280,8 +306,9 @@ __global__ void bonus_kernel(AcceptParams p) {
   }
 }
 
-cudaError_t launch_accept_greedy(const AcceptParams& p, cudaStream_t s) {
-  accept_greedy_kernel<<<p.B, 256, 0, s>>>(p);
+cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, cudaStream_t s) {
+  row_top2_kernel<<<(p.n_total + 7) / 8, 256, 0, s>>>(p, arg_ws);
+  walk_greedy_kernel<<<(p.B + 3) / 4, 128, 0, s>>>(p, arg_ws);
   return cudaGetLastError();
 }
 
@@ -291,6 +318,7 @@ cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStr
 }
 
 cudaError_t launch_accept_chain(const AcceptParams& p, cudaStream_t s) {
+  row_lse_kernel<<<(p.n_total + 7) / 8, 256, 0, s>>>(p);
   accept_chain_kernel<<<p.B, 128, 0, s>>>(p);
   return cudaGetLastError();
 }

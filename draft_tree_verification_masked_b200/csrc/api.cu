@@ -53,19 +53,31 @@ static int env_int(const char* name, int dflt) {
 
 // ------------------------------------------------------------------------------ attention plan
 struct AttnPlan {
-  int G, nw, mchunks, nsplit, tps, stages;
+  int G, tc, nw, nb, mchunks, nsplit, tps, stages;
 };
 
+// Launch plan of the attention call.  The tcgen05 kernel (default) takes 128-row blocks of
+// nb = floor(128 / G) whole nodes; the warp-MMA kernel (ETREE_ATTN=mma) takes 16-row warps.
+// Splits of the KV range are added until about four CTAs per SM exist, keeping >= 4 key tiles
+// per split.
 static AttnPlan plan_attn(const etree_batch* b, int hq, int hkv) {
   AttnPlan pl{};
   pl.G = hq / hkv;
-  const int m16 = (b->n_max * pl.G + 15) / 16;
-  if (m16 <= 8) {
-    pl.nw = std::max(1, m16);
-    pl.mchunks = 1;
+  const char* kind = getenv("ETREE_ATTN");
+  pl.tc = !(kind && strcmp(kind, "mma") == 0) && pl.G <= 128;
+  if (pl.tc) {
+    pl.nb = 128 / pl.G;
+    pl.mchunks = (b->n_max + pl.nb - 1) / pl.nb;
+    pl.nw = 4;
   } else {
-    pl.mchunks = (m16 + 7) / 8;
-    pl.nw = (m16 + pl.mchunks - 1) / pl.mchunks;
+    const int m16 = (b->n_max * pl.G + 15) / 16;
+    if (m16 <= 8) {
+      pl.nw = std::max(1, m16);
+      pl.mchunks = 1;
+    } else {
+      pl.mchunks = (m16 + 7) / 8;
+      pl.nw = (m16 + pl.mchunks - 1) / pl.mchunks;
+    }
   }
   const int pairs = b->B * hkv * pl.mchunks;
   const int tiles_max = (b->kv_len_max + 63) / 64 + 1;
@@ -77,7 +89,7 @@ static AttnPlan plan_attn(const etree_batch* b, int hq, int hkv) {
   if (forced > 0) nsplit = std::min(forced, tiles_max);
   pl.tps = (tiles_max + nsplit - 1) / nsplit;
   pl.nsplit = (tiles_max + pl.tps - 1) / pl.tps;
-  pl.stages = env_int("ETREE_STAGES", 3) == 4 ? 4 : 3;
+  pl.stages = env_int("ETREE_STAGES", pl.tc ? 4 : 3) == 4 ? 4 : 3;
   return pl;
 }
 
@@ -105,7 +117,8 @@ static WsLayout layout(const etree_batch* b, int hq, int hkv, int hidden_dim, in
   const size_t rows = nt * (size_t)std::max(0, hq);
   w.o_part = take(nsplit > 1 ? rows * nsplit * 128 * sizeof(float) : 0);
   w.ml_part = take(nsplit > 1 ? rows * nsplit * sizeof(float2) : 0);
-  w.n_tiles = vocab > 0 ? (vocab + 255) / 256 : 0;
+  // two summaries per vocab tile, at the narrowest tile width the LM head may pick (128)
+  w.n_tiles = vocab > 0 ? 2 * ((vocab + 127) / 128) : 0;
   w.part = take(nt * (size_t)w.n_tiles * sizeof(float4));
   w.child_tok = take(nt * sizeof(int32_t));
   w.zchild = take(nt * sizeof(float));
@@ -283,16 +296,17 @@ const char* etree_strerror(etree_status s) {
 
 const char* etree_last_error(void) { return g_err; }
 
-etree_status etree_attn_plan(const etree_batch* batch, int hq, int hkv, int32_t* warps,
-                             int32_t* row_chunks, int32_t* splits, int32_t* tiles_per_split,
-                             int32_t* launches) {
+etree_status etree_attn_plan(const etree_batch* batch, int hq, int hkv, int32_t* kernel,
+                             int32_t* rows_per_cta, int32_t* row_blocks, int32_t* splits,
+                             int32_t* tiles_per_split, int32_t* launches) {
   etree_status st = check_batch(batch);
   if (st) return st;
   if (hq < 1 || hkv < 1 || hq % hkv != 0 || hq / hkv > 64)
     return fail(ETREE_EINVAL, "hq=%d, hkv=%d", hq, hkv);
   const AttnPlan pl = plan_attn(batch, hq, hkv);
-  if (warps) *warps = pl.nw;
-  if (row_chunks) *row_chunks = pl.mchunks;
+  if (kernel) *kernel = pl.tc;
+  if (rows_per_cta) *rows_per_cta = pl.tc ? pl.nb * pl.G : pl.nw * 16;
+  if (row_blocks) *row_blocks = pl.mchunks;
   if (splits) *splits = pl.nsplit;
   if (tiles_per_split) *tiles_per_split = pl.tps;
   if (launches) *launches = pl.nsplit > 1 ? 2 : 1;
@@ -380,8 +394,16 @@ etree_status etree_verify_attn(const etree_batch* b, const uint16_t* q, const ui
   p.nsplit = pl.nsplit;
   p.tps = pl.tps;
   p.scale_log2 = scale * 1.4426950408889634f;
-  cudaError_t e = launch_attn(kc, vc, kt, vt, p, pl.nw, pl.stages, b->n_total,
-                              static_cast<cudaStream_t>(stream));
+  cudaError_t e;
+  if (pl.tc) {
+    CUtensorMap tq;
+    if ((st = get_map(q, 3, 128, hq, b->n_total, 64, pl.G, pl.nb, &tq))) return st;
+    e = launch_attn_tc(tq, kc, vc, kt, vt, p, pl.nb, pl.stages, b->n_total,
+                       static_cast<cudaStream_t>(stream));
+  } else {
+    e = launch_attn(kc, vc, kt, vt, p, pl.nw, pl.stages, b->n_total,
+                    static_cast<cudaStream_t>(stream));
+  }
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_verify_attn launch");
 }
 
@@ -409,16 +431,18 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
   const WsLayout w = layout(b, 0, 0, hidden_dim, vocab);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
+  const int sms = sm_count();
+  const int bn = lmhead_pick_bn(b->n_total, vocab, sms);
   CUtensorMap ta, tb;
   if ((st = get_map(hidden, 2, hidden_dim, b->n_total, 1, 64, 128, 1, &ta))) return st;
-  if ((st = get_map(w_lm, 2, hidden_dim, vocab, 1, 64, 256, 1, &tb))) return st;
+  if ((st = get_map(w_lm, 2, hidden_dim, vocab, 1, 64, bn, 1, &tb))) return st;
 
   GemmParams g{};
   g.M = b->n_total;
   g.V = vocab;
   g.K = hidden_dim;
   g.m_tiles = (b->n_total + 127) / 128;
-  g.n_tiles = w.n_tiles;
+  g.n_tiles = (vocab + bn - 1) / bn;
   g.num_tiles = g.m_tiles * g.n_tiles;
   g.k_blocks = hidden_dim / 64;
   g.ws = at<WsHeader>(workspace, 0);
@@ -436,9 +460,10 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
 
   AcceptParams a{};
   a.B = b->B;
+  a.n_total = b->n_total;
   a.n_max = b->n_max;
   a.V = vocab;
-  a.n_tiles = w.n_tiles;
+  a.n_tiles = 2 * g.n_tiles;
   a.cu_nodes = b->cu_nodes;
   a.parent = b->parent;
   a.tokens = b->tokens;
@@ -463,25 +488,28 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
   a.H = hidden_dim;
   a.part2 = at<float4>(workspace, w.part2);
 
-  const int sms = sm_count();
   cudaError_t e;
   if (temperature == 0.f) {
-    e = launch_lmhead(0, ta, tb, g, std::min(g.num_tiles, sms), s);
-    if (e == cudaSuccess) e = launch_accept_greedy(a, s);
+    e = launch_lmhead(0, bn, ta, tb, g, std::min(g.num_tiles, sms), s);
+    if (e == cudaSuccess) e = launch_accept_greedy(a, at<int32_t>(workspace, w.child_tok), s);
     return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T=0)");
   }
   e = launch_chain_prep(a, at<int32_t>(workspace, w.child_tok), s);
-  if (e == cudaSuccess) e = launch_lmhead(1, ta, tb, g, std::min(g.num_tiles, sms), s);
+  if (e == cudaSuccess) e = launch_lmhead(1, bn, ta, tb, g, std::min(g.num_tiles, sms), s);
   if (e == cudaSuccess) e = launch_accept_chain(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "etree_lmhead_accept (T>0, pass 1)");
-  CUtensorMap th;
+  const int bn2 = lmhead_pick_bn(b->B, vocab, sms);
+  CUtensorMap th, tb2;
   if ((st = get_map(a.hid2, 2, hidden_dim, b->B, 1, 64, 128, 1, &th))) return st;
+  if ((st = get_map(w_lm, 2, hidden_dim, vocab, 1, 64, bn2, 1, &tb2))) return st;
   GemmParams g2 = g;
   g2.M = b->B;
   g2.m_tiles = (b->B + 127) / 128;
+  g2.n_tiles = (vocab + bn2 - 1) / bn2;
   g2.num_tiles = g2.m_tiles * g2.n_tiles;
   g2.part = at<float4>(workspace, w.part2);
-  e = launch_lmhead(2, th, tb, g2, std::min(g2.num_tiles, sms), s);
+  a.n_tiles2 = 2 * g2.n_tiles;
+  e = launch_lmhead(2, bn2, th, tb2, g2, std::min(g2.num_tiles, sms), s);
   if (e == cudaSuccess) e = launch_bonus(a, s);
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T>0, pass 2)");
 }

@@ -376,6 +376,10 @@ cudaError_t launch_attn(const CUtensorMap& kc, const CUtensorMap& vc, const CUte
     default: e = launch_attn_nw<8>(kc, vc, kt, vt, p, stages, stream); break;
   }
   if (e != cudaSuccess || p.nsplit == 1) return e;
+  return launch_attn_combine(p, n_total, stream);
+}
+
+cudaError_t launch_attn_combine(const AttnParams& p, int n_total, cudaStream_t stream) {
   const int rows = n_total * p.hq;
   const int threads = 256;
   const int blocks = (rows * 32 + threads - 1) / threads;

@@ -24,6 +24,10 @@ struct AttnParams {
 cudaError_t launch_attn(const CUtensorMap& kc, const CUtensorMap& vc, const CUtensorMap& kt,
                         const CUtensorMap& vt, const AttnParams& p, int nw, int stages,
                         int n_total, cudaStream_t stream);
+cudaError_t launch_attn_combine(const AttnParams& p, int n_total, cudaStream_t stream);
+cudaError_t launch_attn_tc(const CUtensorMap& q, const CUtensorMap& kc, const CUtensorMap& vc,
+                           const CUtensorMap& kt, const CUtensorMap& vt, const AttnParams& p,
+                           int nb, int stages, int n_total, cudaStream_t stream);
 
 struct GemmParams {
   int M, V, K, m_tiles, n_tiles, num_tiles, k_blocks;
@@ -39,11 +43,12 @@ struct GemmParams {
   const float* q_draft;
   uint64_t seed, step;
 };
-cudaError_t launch_lmhead(int epi, const CUtensorMap& ta, const CUtensorMap& tb,
+int lmhead_pick_bn(int M, int V, int grid);
+cudaError_t launch_lmhead(int epi, int bn, const CUtensorMap& ta, const CUtensorMap& tb,
                           const GemmParams& p, int grid, cudaStream_t stream);
 
 struct AcceptParams {
-  int B, n_max, V, n_tiles;
+  int B, n_total, n_max, V, n_tiles, n_tiles2;
   const int32_t* cu_nodes;
   const int32_t* parent;
   const int32_t* tokens;
@@ -67,7 +72,7 @@ struct AcceptParams {
   int H;
   const float4* part2;
 };
-cudaError_t launch_accept_greedy(const AcceptParams& p, cudaStream_t s);
+cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, cudaStream_t s);
 cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStream_t s);
 cudaError_t launch_accept_chain(const AcceptParams& p, cudaStream_t s);
 cudaError_t launch_bonus(const AcceptParams& p, cudaStream_t s);

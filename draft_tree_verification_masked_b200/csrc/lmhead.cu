@@ -25,15 +25,120 @@
 
 namespace etree {
 
-constexpr int kBM = 128, kBN = 256, kBK = 64, kGStages = 4;
-constexpr int kABytes = kBM * kBK * 2, kBBytes = kBN * kBK * 2;
+constexpr int kBM = 128, kBK = 64, kGStages = 4;
+constexpr int kABytes = kBM * kBK * 2;
 enum Epi { EPI_ARGMAX = 0, EPI_LSE = 1, EPI_RACE = 2 };
 
+// Per-row running state of the epilogue over one vocab tile.
+struct EpiRow {
+  float r0 = -INFINITY, r2 = -INFINITY, r1f = 0.f;   // ARGMAX: top1, top2 | LSE: max, sum
+  int r1 = -1, r3 = -1;                              // ARGMAX: id | RACE: ids (residual, p)
+  int ct = -1;                                       // LSE: child token of the row
+  float zc = 0.f;                                    // LSE: its logit
+  bool found = false;
+  int unode = 0, md = 0, req = 0;                    // RACE: stop node, mode, request
+  float L2 = 0.f;                                    // RACE: log2 sum 2^(z k)
+  const float* qrow = nullptr;                       // RACE: q_draft row
+};
 
-template <int EPI>
-__global__ void __launch_bounds__(192, 1)
+// Folds W consecutive logits v (columns col0 .. col0+W-1) into the row state.
+template <int EPI, int W>
+__device__ __forceinline__ void epi_chunk(const GemmParams& p, EpiRow& st, const float (&v)[W],
+                                          int col0) {
+  if constexpr (EPI == EPI_ARGMAX) {
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+      const float x = v[j];
+      if (col0 + j < p.V) {
+        if (x > st.r0) {
+          st.r2 = st.r0;
+          st.r0 = x;
+          st.r1 = col0 + j;
+        } else if (x > st.r2) {
+          st.r2 = x;
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_LSE) {
+    float cm = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < W; ++j)
+      if (col0 + j < p.V) cm = fmaxf(cm, v[j] * p.k_log2);
+    if (cm > st.r0) {
+      st.r1f *= exp2f(st.r0 - cm);
+      st.r0 = cm;
+    }
+#pragma unroll
+    for (int j = 0; j < W; ++j)
+      if (col0 + j < p.V) st.r1f += exp2f(v[j] * p.k_log2 - st.r0);
+    if (st.ct >= col0 && st.ct < col0 + W) {
+#pragma unroll
+      for (int j = 0; j < W; ++j)
+        if (col0 + j == st.ct) st.zc = v[j];
+      st.found = true;
+    }
+  } else {
+    // draft probabilities of this chunk, loaded ahead of the Philox work
+    float q[W];
+    if (st.md) {
+      if ((p.V & 3) == 0) {
+#pragma unroll
+        for (int j = 0; j < W; j += 4) {
+          float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (col0 + j < p.V) t = __ldg(reinterpret_cast<const float4*>(st.qrow + col0 + j));
+          q[j] = t.x;
+          q[j + 1] = t.y;
+          q[j + 2] = t.z;
+          q[j + 3] = t.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < W; ++j) q[j] = (col0 + j < p.V) ? __ldg(st.qrow + col0 + j) : 0.f;
+      }
+    }
+    // Exponential race in ratio form: the winner maximises w_v / E_v with E_v = -log U_v, the
+    // same token as argmax (log w_v - log E_v).
+#pragma unroll
+    for (int jj = 0; jj < W / 8; ++jj) {
+      const int cb = col0 + 8 * jj;
+      if (cb >= p.V) break;
+      float u[8];
+      uniforms8(p.seed, p.step, (uint32_t)(cb >> 3), (uint32_t)st.unode, (uint32_t)st.req, 0u, u);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int cc = cb + e;
+        if (cc < p.V) {
+          const float pv = exp2f(v[8 * jj + e] * p.k_log2 - st.L2);
+          const float E = -logf(u[e]);
+          const float kp = __fdividef(pv, E);
+          if (kp > st.r2) {
+            st.r2 = kp;
+            st.r3 = cc;
+          }
+          if (st.md) {
+            const float w = pv - q[8 * jj + e];
+            if (w > 0.f) {
+              const float kr = __fdividef(w, E);
+              if (kr > st.r0) {
+                st.r0 = kr;
+                st.r1 = cc;
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
+constexpr int kEpiWarps = 8;                 // two warps per TMEM lane quarter
+constexpr int kGemmThreads = 32 * (2 + kEpiWarps);
+
+template <int EPI, int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
 lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    GemmParams p) {
+  constexpr int kBBytes = BN * kBK * 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -53,7 +158,7 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accf[b], 1);
-      mbar_init(&acce[b], 4);
+      mbar_init(&acce[b], kEpiWarps);
     }
     fence_barrier_init();
   }
@@ -85,14 +190,14 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           }
           mbar_arrive_expect_tx(&full[st], kABytes + kBBytes);
           tma_load_2d(sA + st * kABytes, &tm_a, &full[st], kb * kBK, mt * kBM);
-          tma_load_2d(sB + st * kBBytes, &tm_b, &full[st], kb * kBK, nt * kBN);
+          tma_load_2d(sB + st * kBBytes, &tm_b, &full[st], kb * kBK, nt * BN);
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, kBN);
+      const uint32_t idesc = idesc_bf16_f32(kBM, BN);
       int it = 0, ai = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++ai) {
@@ -103,7 +208,7 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + buf * kBN;
+        const uint32_t d = tmem + buf * BN;
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int st = it % kGStages;
           const uint32_t ph = (it / kGStages) & 1;
@@ -125,7 +230,13 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     }
   } else {
     // ------------------------------------------------------------------------ epilogue warps
-    const int wq = warp & 3;                 // this warp may read TMEM lanes 32*wq .. 32*wq+31
+    // Warp w reads TMEM lanes 32*(w%4) .. +31 (one output row per thread); the two warps of a
+    // lane quarter take alternate 32-column chunks of the tile and write separate summaries.
+    const int wq = warp & 3;
+    const int half = (warp - 2) >> 2;
+    constexpr int kChunks = BN / 32;
+    constexpr int kTailHalf = (kChunks & 1) ? 1 : 0;   // the 16-column tail goes to the half
+                                                        // with fewer full chunks
     int ai = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++ai) {
       const int buf = ai & 1;
@@ -139,97 +250,29 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       const int row = wq * 32 + lane;
       const int grow = mt * kBM + row;
       const bool active = grow < p.M;
-      const uint32_t tbase = tmem + ((uint32_t)(wq * 32) << 16) + buf * kBN;
+      const uint32_t tbase = tmem + ((uint32_t)(wq * 32) << 16) + buf * BN;
 
-      float r0 = -INFINITY, r2 = -INFINITY, r1f = 0.f;
-      int r1 = -1, r3 = -1;
-      // EPI_LSE extras
-      int ct = -1;
-      float zc = 0.f;
-      bool found = false;
-      // EPI_RACE extras
-      int g = 0, unode = 0, md = 0;
-      float L2 = 0.f;
-      const float* qrow = nullptr;
-      if (EPI == EPI_LSE && active) ct = p.child_tok[grow];
+      EpiRow st;
+      if (EPI == EPI_LSE && active) st.ct = p.child_tok[grow];
       if (EPI == EPI_RACE && active) {
-        g = p.stop_row[grow];
-        unode = p.stop_node[grow];
-        md = p.mode[grow];
-        L2 = p.lse2[g];
-        qrow = p.q_draft + (size_t)g * p.V;
+        const int g = p.stop_row[grow];
+        st.unode = p.stop_node[grow];
+        st.md = p.mode[grow];
+        st.req = grow;
+        st.L2 = p.lse2[g];
+        st.qrow = p.q_draft + (size_t)g * p.V;
       }
-
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = half; c < kChunks; c += 2) {
         float v[32];
         tmem_ld32(tbase + c * 32, v);
-        const int col0 = nt * kBN + c * 32;
-        if (!active) continue;
-        if (EPI == EPI_ARGMAX) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float x = v[j];
-            if (col0 + j < p.V) {
-              if (x > r0) {
-                r2 = r0;
-                r0 = x;
-                r1 = col0 + j;
-              } else if (x > r2) {
-                r2 = x;
-              }
-            }
-          }
-        } else if (EPI == EPI_LSE) {
-          float cm = -INFINITY;
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (col0 + j < p.V) cm = fmaxf(cm, v[j] * p.k_log2);
-          if (cm > r0) {
-            r1f *= exp2f(r0 - cm);
-            r0 = cm;
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (col0 + j < p.V) r1f += exp2f(v[j] * p.k_log2 - r0);
-          if (ct >= col0 && ct < col0 + 32) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j == ct) zc = v[j];
-            found = true;
-          }
-        } else {  // EPI_RACE
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int cb = col0 + 4 * jj;
-            if (cb >= p.V) break;
-            float u[4];
-            uniforms4(p.seed, p.step, (uint32_t)(cb >> 2), (uint32_t)unode, (uint32_t)grow, 0u,
-                      u);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int cc = cb + e;
-              if (cc < p.V) {
-                const float lp2 = v[4 * jj + e] * p.k_log2 - L2;
-                const float gum = -logf(-logf(u[e]));
-                const float kp = lp2 * 0.69314718055994531f + gum;
-                if (kp > r2) {
-                  r2 = kp;
-                  r3 = cc;
-                }
-                if (md) {
-                  const float w = exp2f(lp2) - __ldg(qrow + cc);
-                  if (w > 0.f) {
-                    const float kr = logf(w) + gum;
-                    if (kr > r0) {
-                      r0 = kr;
-                      r1 = cc;
-                    }
-                  }
-                }
-              }
-            }
-          }
+        if (active) epi_chunk<EPI, 32>(p, st, v, nt * BN + c * 32);
+      }
+      if constexpr (BN % 32 == 16) {
+        if (half == kTailHalf) {
+          float v[16];
+          tmem_ld16(tbase + kChunks * 32, v);
+          if (active) epi_chunk<EPI, 16>(p, st, v, nt * BN + kChunks * 32);
         }
       }
       tc_fence_before();
@@ -238,13 +281,13 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       if (active) {
         float4 out;
         if (EPI == EPI_ARGMAX)
-          out = make_float4(r0, __int_as_float(r1), r2, 0.f);
+          out = make_float4(st.r0, __int_as_float(st.r1), st.r2, 0.f);
         else if (EPI == EPI_LSE)
-          out = make_float4(r0, r1f, 0.f, 0.f);
+          out = make_float4(st.r0, st.r1f, 0.f, 0.f);
         else
-          out = make_float4(r0, __int_as_float(r1), r2, __int_as_float(r3));
-        p.part[(size_t)grow * p.n_tiles + nt] = out;
-        if (EPI == EPI_LSE && found) p.zchild[grow] = zc;
+          out = make_float4(st.r0, __int_as_float(st.r1), st.r2, __int_as_float(st.r3));
+        p.part[(size_t)grow * p.n_tiles * 2 + nt * 2 + half] = out;
+        if (EPI == EPI_LSE && st.found) p.zchild[grow] = st.zc;
       }
     }
   }
@@ -256,31 +299,66 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   }
 }
 
-size_t lmhead_smem_bytes() {
-  return (size_t)kGStages * (kABytes + kBBytes) + 1024 + (2 * kGStages + 4) * 8 + 16;
+// Vocab-tile widths with a kernel instantiation.  Each is a multiple of 16 (the M=128 MMA's N
+// granularity) and fits two accumulators in the 512 TMEM columns.
+static const int kWidths[] = {256, 224, 208, 192, 176, 160, 144, 128};
+
+int lmhead_pick_bn(int M, int V, int grid) {
+  const int forced = getenv("ETREE_BN") ? atoi(getenv("ETREE_BN")) : 0;
+  for (int bn : kWidths)
+    if (bn == forced) return bn;
+  // time ~ (rounds of tiles per CTA) x (tile width + a fixed per-tile cost of ~48 columns)
+  const long m_tiles = (M + kBM - 1) / kBM;
+  int best = 256;
+  long best_cost = -1;
+  for (int bn : kWidths) {
+    const long tiles = m_tiles * ((V + bn - 1) / bn);
+    const long rounds = (tiles + grid - 1) / grid;
+    const long cost = rounds * (bn + 48);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
 }
 
-cudaError_t launch_lmhead(int epi, const CUtensorMap& ta, const CUtensorMap& tb,
-                          const GemmParams& p, int grid, cudaStream_t stream) {
-  const size_t smem = lmhead_smem_bytes();
-  cudaError_t e;
-  if (epi == EPI_ARGMAX) {
-    auto k = lmhead_gemm_kernel<EPI_ARGMAX>;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 192, smem, stream>>>(ta, tb, p);
-  } else if (epi == EPI_LSE) {
-    auto k = lmhead_gemm_kernel<EPI_LSE>;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 192, smem, stream>>>(ta, tb, p);
-  } else {
-    auto k = lmhead_gemm_kernel<EPI_RACE>;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 192, smem, stream>>>(ta, tb, p);
-  }
+size_t lmhead_smem_bytes(int bn) {
+  return (size_t)kGStages * (kABytes + bn * kBK * 2) + 1024 + (2 * kGStages + 4) * 8 + 16;
+}
+
+template <int EPI, int BN>
+static cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+                             int grid, cudaStream_t stream) {
+  const size_t smem = lmhead_smem_bytes(BN);
+  auto k = lmhead_gemm_kernel<EPI, BN>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, kGemmThreads, smem, stream>>>(ta, tb, p);
   return cudaGetLastError();
+}
+
+template <int EPI>
+static cudaError_t launch_epi(int bn, const CUtensorMap& ta, const CUtensorMap& tb,
+                              const GemmParams& p, int grid, cudaStream_t s) {
+  switch (bn) {
+    case 256: return launch_bn<EPI, 256>(ta, tb, p, grid, s);
+    case 224: return launch_bn<EPI, 224>(ta, tb, p, grid, s);
+    case 208: return launch_bn<EPI, 208>(ta, tb, p, grid, s);
+    case 192: return launch_bn<EPI, 192>(ta, tb, p, grid, s);
+    case 176: return launch_bn<EPI, 176>(ta, tb, p, grid, s);
+    case 160: return launch_bn<EPI, 160>(ta, tb, p, grid, s);
+    case 144: return launch_bn<EPI, 144>(ta, tb, p, grid, s);
+    case 128: return launch_bn<EPI, 128>(ta, tb, p, grid, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_lmhead(int epi, int bn, const CUtensorMap& ta, const CUtensorMap& tb,
+                          const GemmParams& p, int grid, cudaStream_t stream) {
+  if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX>(bn, ta, tb, p, grid, stream);
+  if (epi == EPI_LSE) return launch_epi<EPI_LSE>(bn, ta, tb, p, grid, stream);
+  return launch_epi<EPI_RACE>(bn, ta, tb, p, grid, stream);
 }
 
 }  // namespace etree

@@ -27,20 +27,20 @@ __device__ __forceinline__ void philox4x64_10(uint64_t c0, uint64_t c1, uint64_t
   out[3] = c3;
 }
 
-// Uniform in (0,1) from the top 24 bits of a 64-bit word, centred: exact in fp32.
-__device__ __forceinline__ float u24(uint64_t x) {
-  return (static_cast<float>(static_cast<uint32_t>(x >> 40)) + 0.5f) * (1.0f / 16777216.0f);
-}
-
-// The four uniforms for vocab ids 4*vb .. 4*vb+3 at (node, request, stream) under (seed, step).
-__device__ __forceinline__ void uniforms4(uint64_t seed, uint64_t step, uint32_t vb, uint32_t node,
-                                          uint32_t req, uint32_t stream, float (&u)[4]) {
+// The eight uniforms of vocab ids 8*vb .. 8*vb+7 at (node, request, stream) under (seed, step):
+// each 64-bit output word holds two 23-bit fields, bits 63..41 (even id) and bits 31..9 (odd
+// id), centred: U = (field + 0.5) * 2^-23.  Single precision holds every such value exactly,
+// and all lie in [2^-24, 1 - 2^-24], so -log U is finite and positive.
+__device__ __forceinline__ void uniforms8(uint64_t seed, uint64_t step, uint32_t vb, uint32_t node,
+                                          uint32_t req, uint32_t stream, float (&u)[8]) {
   uint64_t w[4];
   philox4x64_10(vb, node, req, stream, seed, step, w);
-  u[0] = u24(w[0]);
-  u[1] = u24(w[1]);
-  u[2] = u24(w[2]);
-  u[3] = u24(w[3]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    u[2 * i] = (static_cast<float>(static_cast<uint32_t>(w[i] >> 41)) + 0.5f) * (1.0f / 8388608.0f);
+    u[2 * i + 1] =
+        (static_cast<float>(static_cast<uint32_t>(w[i]) >> 9) + 0.5f) * (1.0f / 8388608.0f);
+  }
 }
 
 }  // namespace etree

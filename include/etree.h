@@ -194,12 +194,14 @@ const char *etree_last_error(void);
 
 /*
  * The launch plan etree_verify_attn uses for this batch and head shape (host-only, no device
- * work): consumer warps per CTA, row chunks per (request, KV head), KV splits, 64-key tiles per
- * split, and the number of kernels the call launches (1, or 2 with the split combine).
+ * work): which kernel (1 = tcgen05/TMEM kernel, the default; 0 = warp-level mma.sync kernel,
+ * selected by the environment variable ETREE_ATTN=mma), query rows per CTA, row blocks per
+ * (request, KV head), KV splits, 64-key tiles per split, and the number of kernels the call
+ * launches (1, or 2 with the split combine).  Any output pointer may be NULL.
  */
-etree_status etree_attn_plan(const etree_batch *batch, int hq, int hkv, int32_t *warps,
-                             int32_t *row_chunks, int32_t *splits, int32_t *tiles_per_split,
-                             int32_t *launches);
+etree_status etree_attn_plan(const etree_batch *batch, int hq, int hkv, int32_t *kernel,
+                             int32_t *rows_per_cta, int32_t *row_blocks, int32_t *splits,
+                             int32_t *tiles_per_split, int32_t *launches);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int etree_version(void);

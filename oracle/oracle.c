@@ -21,7 +21,7 @@
  *    lowest node index is taken;
  *  - T>0 is defined for chains only: node k's token was drafted from q of node k-1; accept iff
  *    U*q < p (strict); the bonus/residual token is drawn by an exponential race
- *    argmax_v [log w_v - log(-log U_v)] with Philox4x64-10 uniforms.
+ *    argmax_v [log w_v - log(-log U_v)] with Philox4x64-10 uniforms (8 per block).
  */
 #include <math.h>
 #include <stdint.h>
@@ -284,17 +284,21 @@ void oracle_philox4x64(const uint64_t ctr[4], const uint64_t key[2], uint64_t ou
     out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
 }
 
-/* The method's seeded uniform in (0,1): counter (v/4, node, request, stream) under key
- * (seed, step), word v%4, top 24 bits, centred: U = (x>>40 + 0.5) * 2^-24.  stream 0 feeds the
- * bonus/residual race (v = vocab id), stream 1 the accept tests (v = 0, node = the child). */
+/* The method's seeded uniform in (0,1).  One Philox block (counter (v/8, node, request, stream)
+ * under key (seed, step)) gives 4 words of 64 bits; each word holds two 23-bit fields, bits
+ * 63..41 and bits 31..9.  Vocab id v takes word (v/2) % 4, the high field for even v and the
+ * low field for odd v, centred: U = (field + 0.5) * 2^-23, a value that single precision holds
+ * exactly and that lies in [2^-24, 1 - 2^-24].  stream 0 feeds the bonus/residual race
+ * (v = vocab id), stream 1 the accept tests (v = 0, node = the child). */
 double oracle_uniform(uint64_t seed, uint64_t step, uint32_t r, uint32_t node, uint32_t v,
                       uint32_t stream) {
-    uint64_t ctr[4] = {v >> 2, node, r, stream};
+    uint64_t ctr[4] = {v >> 3, node, r, stream};
     uint64_t key[2] = {seed, step};
     uint64_t out[4];
     oracle_philox4x64(ctr, key, out);
-    uint64_t x = out[v & 3u];
-    return ((double)(x >> 40) + 0.5) * (1.0 / 16777216.0);
+    uint64_t x = out[(v >> 1) & 3u];
+    uint64_t field = (v & 1u) ? ((x & 0xFFFFFFFFull) >> 9) : (x >> 41);
+    return ((double)field + 0.5) * (1.0 / 8388608.0);
 }
 
 /* Exponential race over weights w (>= 0): the winner is argmax over w_v > 0 of

@@ -164,3 +164,16 @@ def test_multi_layer_compaction_against_oracle():
 
 def test_env_is_clean():
     assert "ETREE_NSPLIT" not in os.environ
+
+
+@pytest.mark.parametrize("case", ["tiny", "ragged"])
+def test_warp_mma_attention_kernel(case, monkeypatch):
+    """The warp-level mma.sync attention kernel, kept for comparison, against the oracle."""
+    monkeypatch.setenv("ETREE_ATTN", "mma")
+    if case == "tiny":
+        wl = W.generate("tiny")
+    else:
+        wl = W.generate("tiny", B=6, n_nodes=[1, 4, 16, 33, 64, 2],
+                        kv_len=[0, 1, 63, 64, 65, 200], depth=8, depth_min=1, branch=None,
+                        width=16, vocab=1000, hidden=256)
+    _full_check(wl)

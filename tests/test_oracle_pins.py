@@ -54,12 +54,17 @@ def test_philox_random_counters_match_numpy():
         assert (bg.random_raw(4).astype(np.uint64) == oracle.philox4x64(ctr, key)).all()
 
 
-def test_uniform_is_24bit_centred_and_uniform():
+def test_uniform_is_23bit_centred_exact_in_float32_and_uniform():
     us = np.array([oracle.uniform(0xE7EE0004, 9, r, r % 5, v, 0)
                    for r in range(400) for v in range(50)])
     assert (us > 0).all() and (us < 1).all()
-    k = us * 2**24 - 0.5
+    k = us * 2**23 - 0.5
     assert np.allclose(k, np.round(k), atol=0, rtol=0)
+    # every value of the form (f + 1/2) 2^-23 survives a round trip through float32, and the
+    # extreme fields stay strictly inside (0, 1)
+    assert np.array_equal(us.astype(np.float32).astype(np.float64), us)
+    top = np.float32((2**23 - 1 + 0.5) * 2.0**-23)
+    assert float(top) == (2**23 - 0.5) * 2.0**-23 and top < 1.0
     counts, _ = np.histogram(us, bins=20, range=(0, 1))
     assert stats.chisquare(counts).pvalue > 1e-4
     # stream 1 and stream 0 are different draws
