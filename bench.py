@@ -223,6 +223,48 @@ def time_e2e(dev, wl, steps, warmup, flush):
     return ms, h2d, d2h
 
 
+def time_compact_layers(dev, wl, flush, layers=64, reps=10):
+    """KV compaction over `layers` stacked layers with the step's real accept lengths and paths,
+    into a compaction-only pool (every request given 64 free slots), timed alone."""
+    from draft_tree_verification_masked_b200 import etree_kv_compact, make_batch
+    B, hkv, D = wl.B, wl.hkv, wl.head_dim
+    i32 = dict(dtype=torch.int32, device="cuda")
+    kv0 = torch.zeros(B, **i32)
+    cap = torch.full((B,), 64, **i32)
+    sbase = torch.arange(B, dtype=torch.int64, device="cuda") * 64
+    batch = make_batch(dev.cu_nodes, dev.parent, dev.tokens, kv0, sbase, cap, wl.n_max, 0)
+    kt = torch.empty(layers, wl.n_total, hkv, D, dtype=torch.bfloat16, device="cuda")
+    vt = torch.empty_like(kt)
+    kt.normal_()
+    vt.normal_()
+    kc = torch.zeros(layers, B * 64, hkv, D, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    out = torch.empty(B, **i32)
+
+    def one():
+        etree_kv_compact(batch, dev.accept_len, dev.path, kt, vt, kc, vc, layers,
+                         kt[0].numel(), kc[0].numel(), out, dev.ws)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        one()
+        b.record()
+        b.synchronize()
+        tot += a.elapsed_time(b)
+    us = tot / reps * 1e3
+    acc = dev.accept_len.cpu().numpy()
+    nbytes = compact_work(wl, acc, layers)
+    del kt, vt, kc, vc
+    torch.cuda.empty_cache()
+    return us, nbytes
+
+
 # -------------------------------------------------------------------------------- CPU oracle
 def oracle_step(wl, requests, nthreads=0):
     """One oracle verification step over the listed requests: attention of all their rows,
@@ -304,6 +346,13 @@ def run_config(name, steps, warmup, peaks, rank, flush, with_e2e=True):
     return res
 
 
+def compact_layers_report(dev, wl, flush, peaks, layers=64):
+    us, nbytes = time_compact_layers(dev, wl, flush, layers)
+    hbm = float(peaks["hbm_gbs"])
+    return {"layers": layers, "us": us, "GB/s": nbytes / us / 1e3, "hbm_frac": nbytes / us / 1e3 / hbm,
+            "bytes": nbytes}
+
+
 def kernel_report(wl, t, acc, peaks):
     hbm = float(peaks["hbm_gbs"])
     tc = float(peaks["bf16_tflops"])
@@ -330,7 +379,7 @@ def roofline(wl, rep, peaks, peak_kind, workload):
     dom = max(("attn", "lmhead", "compact"), key=lambda k: rep[k]["us"])
     k = rep[dom]
     hbm, tc = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
-    src = {"attn": "attn_tree.cu", "lmhead": "lmhead.cu", "compact": "compact.cu"}[dom]
+    src = {"attn": "attn_tc.cu", "lmhead": "lmhead.cu", "compact": "compact.cu"}[dom]
     traffic = ncu_traffic(dom, workload, source_hash(src))
     if dom == "compact" or k["bytes"] / (hbm * 1e9) >= k.get("flops", 0) / (tc * 1e12):
         return {"kernel": dom, "bound": "hbm", "achieved": k["GB/s"], "peak": hbm,
@@ -389,6 +438,7 @@ def main():
     step_s, e2e_s, tokens_all = reduce_over_ranks(step_s, e2e_s, tokens, world, "cuda")
     acc = main_res["dev"].accept_len.cpu().numpy()
     rep = kernel_report(wl, t, acc, peaks)
+    rep["compact_64layers"] = compact_layers_report(main_res["dev"], wl, flush, peaks)
     rl = roofline(wl, rep, peaks, peak_kind, args.config)
     head_plan, head_launches = main_res["plan"], main_res["launches"]
 
@@ -400,6 +450,7 @@ def main():
                        with_e2e=False)
         racc = r["dev"].accept_len.cpu().numpy()
         rrep = kernel_report(r["wl"], r["t"], racc, peaks)
+        rrep["compact_64layers"] = compact_layers_report(r["dev"], r["wl"], flush, peaks)
         sms = statistics.mean(r["t"]["step_ms"])
         by_batch[name] = {
             "B": r["wl"].B, "us_per_step": sms * 1e3,

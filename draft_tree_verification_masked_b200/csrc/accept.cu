@@ -275,17 +275,24 @@ __global__ void __launch_bounds__(128) accept_chain_kernel(AcceptParams p) {
   for (int i = threadIdx.x; i < p.H / 8; i += blockDim.x) hd[i] = hs[i];
 }
 
-// Reduce the race partials of each request and write its bonus token.
+// The first level of the two-level draw, per request: the exponential race among the 128-id
+// block totals (key W_b / E_b with E_b = -log U_b, stream 2), ties to the lowest block; the
+// bonus is the inverse-CDF pick the GEMM epilogue made inside the winning block.  Residual
+// weights are used after a rejection unless none is positive, then p.
 __global__ void bonus_kernel(AcceptParams p) {
   const int r = blockIdx.x;
   const int lane = threadIdx.x;
+  const int node = p.stop_node[r];
   const float4* row = p.part2 + (size_t)r * p.n_tiles2;
   float kr = -INFINITY, kp = -INFINITY;
   int ir = -1, ip = -1;
-  for (int t = lane; t < p.n_tiles2; t += 32) {
-    const float4 v = row[t];
-    merge_key(kr, ir, v.x, __float_as_int(v.y));
-    merge_key(kp, ip, v.z, __float_as_int(v.w));
+  for (int b = lane; b < p.n_tiles2; b += 32) {
+    const float4 v = row[b];
+    float u[8];
+    uniforms8(p.seed, p.step, (uint32_t)(b >> 3), (uint32_t)node, (uint32_t)r, 2u, u);
+    const float E = -logf(u[b & 7]);
+    if (v.x > 0.f) merge_key(kr, ir, __fdividef(v.x, E), __float_as_int(v.y));
+    if (v.z > 0.f) merge_key(kp, ip, __fdividef(v.z, E), __float_as_int(v.w));
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {

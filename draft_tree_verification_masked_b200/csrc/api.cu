@@ -81,8 +81,11 @@ static AttnPlan plan_attn(const etree_batch* b, int hq, int hkv) {
   }
   const int pairs = b->B * hkv * pl.mchunks;
   const int tiles_max = (b->kv_len_max + 63) / 64 + 1;
-  const int target = 4 * sm_count();
-  int nsplit = (target + pairs - 1) / pairs;
+  // The tcgen05 kernel runs one CTA per SM: split the KV range only to fill a single wave
+  // (a second, partial wave costs more than longer splits); keep >= 4 key tiles per split.
+  // The warp-MMA kernel aims at about four CTAs per SM.
+  const int sms = sm_count();
+  int nsplit = pl.tc ? std::max(1, sms / pairs) : (4 * sms + pairs - 1) / pairs;
   nsplit = std::min(nsplit, std::max(1, tiles_max / 4));
   nsplit = std::max(1, std::min(nsplit, tiles_max));
   const int forced = env_int("ETREE_NSPLIT", 0);
@@ -498,7 +501,7 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
   if (e == cudaSuccess) e = launch_lmhead(1, bn, ta, tb, g, std::min(g.num_tiles, sms), s);
   if (e == cudaSuccess) e = launch_accept_chain(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "etree_lmhead_accept (T>0, pass 1)");
-  const int bn2 = lmhead_pick_bn(b->B, vocab, sms);
+  const int bn2 = 256;                       // the draw's 128-id blocks pair up in a tile
   CUtensorMap th, tb2;
   if ((st = get_map(a.hid2, 2, hidden_dim, b->B, 1, 64, 128, 1, &th))) return st;
   if ((st = get_map(w_lm, 2, hidden_dim, vocab, 1, 64, bn2, 1, &tb2))) return st;
@@ -525,7 +528,7 @@ etree_status etree_kv_compact(const etree_batch* b, const int32_t* accept_len,
   if (st) return st;
   if (head_dim != ETREE_HEAD_DIM)
     return fail(ETREE_EUNSUPPORTED, "head_dim=%d (only 128 is built)", head_dim);
-  if (hkv < 1 || n_layers < 1 || n_layers > 65535)
+  if (hkv < 1 || n_layers < 1 || n_layers > 65535 || (int64_t)hkv * head_dim * 2 % 16)
     return fail(ETREE_EINVAL, "hkv=%d, n_layers=%d", hkv, n_layers);
   if (!accept_len || !path || !k_tree || !v_tree || !k_cache || !v_cache || !kv_len_out)
     return fail(ETREE_EINVAL, "a pointer is NULL");
@@ -556,7 +559,7 @@ etree_status etree_kv_compact(const etree_batch* b, const int32_t* accept_len,
   p.tree_layer_stride16 = tree_layer_stride / 8;
   p.cache_layer_stride16 = cache_layer_stride / 8;
   p.row16 = (int)(row / 8);
-  cudaError_t e = launch_compact(p, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_compact(p, sm_count(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_kv_compact launch");
 }
 

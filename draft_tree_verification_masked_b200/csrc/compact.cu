@@ -6,75 +6,101 @@
 // "Current Limitation").  After the walk, the root's and the accepted nodes' K/V rows (this
 // step's tree K/V, in path order) are copied to the request's next cache slots, layer by layer.
 //
-// One CTA per (request, layer): it validates the request's accept length and path, then streams
-// the 2 x (a + 1) rows of hkv * 128 bf16 with 16-byte vector loads and stores.  The copy is a
-// bit copy and is HBM-bound.
+// The copy is a bit copy and is HBM-bound: every byte moved is read once and written once.
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace etree {
 
 
-__global__ void __launch_bounds__(256) kv_compact_kernel(CompactParams p) {
+// One CTA per (request, chunk of layers).  Its first two warps read the request's accept length
+// and path entries in parallel and validate them once; then all 256 threads stream the
+// 2 x (a + 1) rows of every layer in the chunk, one 16-byte word per thread per row and
+// tensor (K, V), four rows in flight per thread.
+__global__ void __launch_bounds__(256) kv_compact_kernel(CompactParams p, int layers_per_cta) {
   __shared__ int src_s[64];
-  __shared__ int info_s[2];
+  __shared__ int rows_s, code_s, detail_s, bad_s;
+  __shared__ long long dst_s;
   const int r = blockIdx.x;
-  const int layer = blockIdx.y;
-  if (threadIdx.x == 0) {
+  const int l0 = blockIdx.y * layers_per_cta;
+  const int l1 = min(p.n_layers, l0 + layers_per_cta);
+  const int tid = threadIdx.x;
+  if (tid == 0) {
     const int base = p.cu_nodes[r];
     const int n = p.cu_nodes[r + 1] - base;
     const int a = p.accept_len[r];
     const int L = p.kv_len[r];
-    int ok = 1, detail = DET_NONE, code = ETREE_OK;
+    int code = ETREE_OK, detail = DET_NONE;
     if (n < 1 || n > p.n_max || a < 0 || a >= n || L < 0) {
-      ok = 0;
       code = ETREE_EDEVICE;
       detail = DET_BAD_PATH;
     } else if ((int64_t)L + a + 1 > (int64_t)p.slot_cap[r]) {
-      ok = 0;
       code = ETREE_ENOSPACE;
       detail = DET_CAPACITY;
-    } else {
-      for (int k = 0; k <= a; ++k) {
-        const int j = p.path[(size_t)r * ETREE_PATH_STRIDE + k];
-        if (j < 0 || j >= n) {
-          ok = 0;
-          code = ETREE_EDEVICE;
-          detail = DET_BAD_PATH;
-          break;
-        }
-        src_s[k] = base + j;
-      }
     }
-    if (!ok && layer == 0) report(p.ws, code, detail);
-    if (layer == 0) p.kv_len_out[r] = ok ? L + a + 1 : L;
-    info_s[0] = ok ? a + 1 : 0;
+    code_s = code;
+    detail_s = detail;
+    rows_s = code == ETREE_OK ? a + 1 : 0;
+    bad_s = 0;
+    dst_s = p.slot_base[r] + L;
   }
   __syncthreads();
-  const int rows = info_s[0];
+  const int rows0 = rows_s;
+  if (tid < rows0) {                                   // path entries, read in parallel
+    const int base = p.cu_nodes[r];
+    const int n = p.cu_nodes[r + 1] - base;
+    const int j = p.path[(size_t)r * ETREE_PATH_STRIDE + tid];
+    if (j < 0 || j >= n) atomicOr(&bad_s, 1);
+    src_s[tid] = base + j;
+  }
+  __syncthreads();
+  if (tid == 0 && blockIdx.y == 0) {
+    int code = code_s, detail = detail_s;
+    if (code == ETREE_OK && bad_s) {
+      code = ETREE_EDEVICE;
+      detail = DET_BAD_PATH;
+    }
+    if (code != ETREE_OK) report(p.ws, code, detail);
+    p.kv_len_out[r] = code == ETREE_OK ? p.kv_len[r] + rows0 : p.kv_len[r];
+  }
+  const int rows = bad_s ? 0 : rows0;
   if (rows == 0) return;
-  const int64_t dst0 = p.slot_base[r] + p.kv_len[r];
-  const uint4* kt = p.k_tree + (size_t)layer * p.tree_layer_stride16;
-  const uint4* vt = p.v_tree + (size_t)layer * p.tree_layer_stride16;
-  uint4* kc = p.k_cache + (size_t)layer * p.cache_layer_stride16;
-  uint4* vc = p.v_cache + (size_t)layer * p.cache_layer_stride16;
-  const int per = rows * p.row16;
-  // K and V interleaved in one index space so both streams are in flight together
-  for (int i = threadIdx.x; i < 2 * per; i += blockDim.x) {
-    const int which = i >= per;
-    const int e = which ? i - per : i;
-    const int k = e / p.row16, c = e - k * p.row16;
-    const size_t src = (size_t)src_s[k] * p.row16 + c;
-    const size_t dst = (size_t)(dst0 + k) * p.row16 + c;
-    if (which)
-      vc[dst] = __ldg(vt + src);
-    else
-      kc[dst] = __ldg(kt + src);
+  const long long dst0 = dst_s;
+  const int w16 = p.row16;                            // 16-byte words per row
+  for (int layer = l0; layer < l1; ++layer) {
+    const uint4* kt = p.k_tree + (size_t)layer * p.tree_layer_stride16;
+    const uint4* vt = p.v_tree + (size_t)layer * p.tree_layer_stride16;
+    uint4* kc = p.k_cache + (size_t)layer * p.cache_layer_stride16;
+    uint4* vc = p.v_cache + (size_t)layer * p.cache_layer_stride16;
+    for (int c = tid; c < 2 * w16; c += blockDim.x) {
+      const bool isv = c >= w16;
+      const int cc = isv ? c - w16 : c;
+      const uint4* src = isv ? vt : kt;
+      uint4* dst = isv ? vc : kc;
+      int k = 0;
+      for (; k + 4 <= rows; k += 4) {
+        uint4 v0 = __ldg(src + (size_t)src_s[k] * w16 + cc);
+        uint4 v1 = __ldg(src + (size_t)src_s[k + 1] * w16 + cc);
+        uint4 v2 = __ldg(src + (size_t)src_s[k + 2] * w16 + cc);
+        uint4 v3 = __ldg(src + (size_t)src_s[k + 3] * w16 + cc);
+        dst[(size_t)(dst0 + k) * w16 + cc] = v0;
+        dst[(size_t)(dst0 + k + 1) * w16 + cc] = v1;
+        dst[(size_t)(dst0 + k + 2) * w16 + cc] = v2;
+        dst[(size_t)(dst0 + k + 3) * w16 + cc] = v3;
+      }
+      for (; k < rows; ++k) dst[(size_t)(dst0 + k) * w16 + cc] = __ldg(src + (size_t)src_s[k] * w16 + cc);
+    }
   }
 }
 
-cudaError_t launch_compact(const CompactParams& p, cudaStream_t s) {
-  dim3 grid(p.B, p.n_layers);
-  kv_compact_kernel<<<grid, 256, 0, s>>>(p);
+cudaError_t launch_compact(const CompactParams& p, int sms, cudaStream_t s) {
+  // spread the layers over enough CTAs to give every SM a few, at least one layer per CTA
+  const int want = std::max(1, (4 * sms + p.B - 1) / p.B);
+  const int chunks = std::min(p.n_layers, want);
+  const int per = (p.n_layers + chunks - 1) / chunks;
+  dim3 grid(p.B, (p.n_layers + per - 1) / per);
+  kv_compact_kernel<<<grid, 256, 0, s>>>(p, per);
   return cudaGetLastError();
 }
 

@@ -94,6 +94,6 @@ struct CompactParams {
   int64_t tree_layer_stride16, cache_layer_stride16;
   int row16;
 };
-cudaError_t launch_compact(const CompactParams& p, cudaStream_t s);
+cudaError_t launch_compact(const CompactParams& p, int sms, cudaStream_t s);
 
 }  // namespace etree

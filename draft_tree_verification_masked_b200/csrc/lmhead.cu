@@ -18,8 +18,9 @@
 //   EPI_ARGMAX  per row and tile: top-1 value, its vocab id (lowest on ties) and top-2 value;
 //   EPI_LSE     per row and tile: m = max z*log2(e)/T and sum 2^(z*log2(e)/T - m), plus the
 //               logit of the row's child token when it falls in the tile;
-//   EPI_RACE    per row and tile: the exponential-race winners log w_v - log(-log U_v) for
-//               w = max(0, p - q) and for w = p, with Philox4x64-10 uniforms.
+//   EPI_RACE    per row and 128-id block: the block totals of w = max(0, p - q) and w = p and,
+//               for each, the id where the block's running sum passes u_b times its total
+//               (two passes over the block in TMEM); the block race happens in bonus_kernel.
 #include "kernels.cuh"
 #include "philox.cuh"
 
@@ -77,55 +78,65 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, EpiRow& st, const
         if (col0 + j == st.ct) st.zc = v[j];
       st.found = true;
     }
-  } else {
-    // draft probabilities of this chunk, loaded ahead of the Philox work
-    float q[W];
-    if (st.md) {
+  }
+}
+
+// Two-level draw, first pass over one 128-id block: block totals of the residual weights
+// max(0, p - q) and of p, summed in increasing id order.  Returns nothing; updates Wr, Wp.
+__device__ __forceinline__ void race_sum(const GemmParams& p, const EpiRow& st, const float (&v)[32],
+                                         int col0, float& Wr, float& Wp) {
+  float q[32];
+  if (st.md) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
       if ((p.V & 3) == 0) {
-#pragma unroll
-        for (int j = 0; j < W; j += 4) {
-          float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (col0 + j < p.V) t = __ldg(reinterpret_cast<const float4*>(st.qrow + col0 + j));
-          q[j] = t.x;
-          q[j + 1] = t.y;
-          q[j + 2] = t.z;
-          q[j + 3] = t.w;
-        }
+        if (col0 + j < p.V) t = __ldg(reinterpret_cast<const float4*>(st.qrow + col0 + j));
       } else {
-#pragma unroll
-        for (int j = 0; j < W; ++j) q[j] = (col0 + j < p.V) ? __ldg(st.qrow + col0 + j) : 0.f;
+        t.x = col0 + j < p.V ? __ldg(st.qrow + col0 + j) : 0.f;
+        t.y = col0 + j + 1 < p.V ? __ldg(st.qrow + col0 + j + 1) : 0.f;
+        t.z = col0 + j + 2 < p.V ? __ldg(st.qrow + col0 + j + 2) : 0.f;
+        t.w = col0 + j + 3 < p.V ? __ldg(st.qrow + col0 + j + 3) : 0.f;
       }
+      q[j] = t.x;
+      q[j + 1] = t.y;
+      q[j + 2] = t.z;
+      q[j + 3] = t.w;
     }
-    // Exponential race in ratio form: the winner maximises w_v / E_v with E_v = -log U_v, the
-    // same token as argmax (log w_v - log E_v).
+  }
 #pragma unroll
-    for (int jj = 0; jj < W / 8; ++jj) {
-      const int cb = col0 + 8 * jj;
-      if (cb >= p.V) break;
-      float u[8];
-      uniforms8(p.seed, p.step, (uint32_t)(cb >> 3), (uint32_t)st.unode, (uint32_t)st.req, 0u, u);
+  for (int j = 0; j < 32; ++j) {
+    if (col0 + j < p.V) {
+      const float pv = exp2f(v[j] * p.k_log2 - st.L2);
+      Wp += pv;
+      if (st.md) Wr += fmaxf(pv - q[j], 0.f);
+    }
+  }
+}
+
+// Second pass: the first id whose running sum exceeds its threshold (inverse CDF inside the
+// block); the arithmetic repeats the first pass exactly, so the running sums end at the totals.
+__device__ __forceinline__ void race_scan(const GemmParams& p, const EpiRow& st,
+                                          const float (&v)[32], int col0, float thr_r, float thr_p,
+                                          float& run_r, float& run_p, int& pick_r, int& pick_p,
+                                          int& last_r, int& last_p) {
+  float q[32];
+  if (st.md) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int cc = cb + e;
-        if (cc < p.V) {
-          const float pv = exp2f(v[8 * jj + e] * p.k_log2 - st.L2);
-          const float E = -logf(u[e]);
-          const float kp = __fdividef(pv, E);
-          if (kp > st.r2) {
-            st.r2 = kp;
-            st.r3 = cc;
-          }
-          if (st.md) {
-            const float w = pv - q[8 * jj + e];
-            if (w > 0.f) {
-              const float kr = __fdividef(w, E);
-              if (kr > st.r0) {
-                st.r0 = kr;
-                st.r1 = cc;
-              }
-            }
-          }
-        }
+    for (int j = 0; j < 32; ++j) q[j] = col0 + j < p.V ? __ldg(st.qrow + col0 + j) : 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (col0 + j < p.V) {
+      const float pv = exp2f(v[j] * p.k_log2 - st.L2);
+      run_p += pv;
+      if (pv > 0.f) last_p = col0 + j;
+      if (pick_p < 0 && run_p > thr_p) pick_p = col0 + j;
+      if (st.md) {
+        const float w = fmaxf(pv - q[j], 0.f);
+        run_r += w;
+        if (w > 0.f) last_r = col0 + j;
+        if (pick_r < 0 && run_r > thr_r) pick_r = col0 + j;
       }
     }
   }
@@ -262,17 +273,49 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         st.L2 = p.lse2[g];
         st.qrow = p.q_draft + (size_t)g * p.V;
       }
+      if constexpr (EPI == EPI_RACE) {
+        // this half owns one whole 128-id block: columns half*128 .. half*128+127 of the tile
+        static_assert(BN == 256, "the two-level draw works on 128-id blocks");
+        const int blk = nt * 2 + half;
+        const int colb = blk * 128;
+        float Wr = 0.f, Wp = 0.f;
 #pragma unroll 1
-      for (int c = half; c < kChunks; c += 2) {
-        float v[32];
-        tmem_ld32(tbase + c * 32, v);
-        if (active) epi_chunk<EPI, 32>(p, st, v, nt * BN + c * 32);
-      }
-      if constexpr (BN % 32 == 16) {
-        if (half == kTailHalf) {
-          float v[16];
-          tmem_ld16(tbase + kChunks * 32, v);
-          if (active) epi_chunk<EPI, 16>(p, st, v, nt * BN + kChunks * 32);
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(tbase + (half * 4 + c) * 32, v);
+          if (active) race_sum(p, st, v, colb + c * 32, Wr, Wp);
+        }
+        float u[8];
+        uniforms8(p.seed, p.step, (uint32_t)(blk >> 3), (uint32_t)st.unode, (uint32_t)st.req, 3u,
+                  u);
+        const float ub = u[blk & 7];
+        float run_r = 0.f, run_p = 0.f;
+        int pick_r = -1, pick_p = -1, last_r = -1, last_p = -1;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(tbase + (half * 4 + c) * 32, v);
+          if (active)
+            race_scan(p, st, v, colb + c * 32, ub * Wr, ub * Wp, run_r, run_p, pick_r, pick_p,
+                      last_r, last_p);
+        }
+        st.r0 = Wr;
+        st.r1 = pick_r >= 0 ? pick_r : last_r;
+        st.r2 = Wp;
+        st.r3 = pick_p >= 0 ? pick_p : last_p;
+      } else {
+#pragma unroll 1
+        for (int c = half; c < kChunks; c += 2) {
+          float v[32];
+          tmem_ld32(tbase + c * 32, v);
+          if (active) epi_chunk<EPI, 32>(p, st, v, nt * BN + c * 32);
+        }
+        if constexpr (BN % 32 == 16) {
+          if (half == kTailHalf) {
+            float v[16];
+            tmem_ld16(tbase + kChunks * 32, v);
+            if (active) epi_chunk<EPI, 16>(p, st, v, nt * BN + kChunks * 32);
+          }
         }
       }
       tc_fence_before();
@@ -307,8 +350,11 @@ int lmhead_pick_bn(int M, int V, int grid) {
   const int forced = getenv("ETREE_BN") ? atoi(getenv("ETREE_BN")) : 0;
   for (int bn : kWidths)
     if (bn == forced) return bn;
-  // time ~ (rounds of tiles per CTA) x (tile width + a fixed per-tile cost of ~48 columns)
+  // With several row tiles the GEMM is tensor-bound and the widest tile is the most efficient.
+  // With one row tile it streams W once: time ~ (rounds of tiles per CTA) x (tile width + a
+  // fixed per-tile cost of ~48 columns), so pick the width that balances the last round.
   const long m_tiles = (M + kBM - 1) / kBM;
+  if (m_tiles >= 2) return 256;
   int best = 256;
   long best_cost = -1;
   for (int bn : kWidths) {
@@ -358,7 +404,8 @@ cudaError_t launch_lmhead(int epi, int bn, const CUtensorMap& ta, const CUtensor
                           const GemmParams& p, int grid, cudaStream_t stream) {
   if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX>(bn, ta, tb, p, grid, stream);
   if (epi == EPI_LSE) return launch_epi<EPI_LSE>(bn, ta, tb, p, grid, stream);
-  return launch_epi<EPI_RACE>(bn, ta, tb, p, grid, stream);
+  if (bn != 256) return cudaErrorInvalidValue;
+  return launch_bn<EPI_RACE, 256>(ta, tb, p, grid, stream);
 }
 
 }  // namespace etree

@@ -67,6 +67,11 @@ def lib():
         L.oracle_race_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
                                        C.c_int, I32P, C.c_int]
         L.oracle_race_many.restype = None
+        L.oracle_draw.argtypes = [C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int, C.c_int, I32P]
+        L.oracle_draw.restype = C.c_int
+        L.oracle_draw_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
+                                       C.c_int, I32P, C.c_int]
+        L.oracle_draw_many.restype = None
         _lib = L
     return _lib
 
@@ -197,6 +202,21 @@ def accept_chain_batch(cu_nodes, parent, tokens, z, q, T, seed, step, nthreads=0
                                     q.reshape(-1), V, float(T), seed, step, a, path.reshape(-1),
                                     out.reshape(-1), info.reshape(-1), int(nthreads))
     return a, path, out, info
+
+
+def draw(w, seed, step, r, node):
+    """The acceptance rule's two-level draw; returns (token, block, fell_to_last)."""
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    info = np.zeros(2, dtype=np.int32)
+    tok = lib().oracle_draw(len(w), w, seed, step, r, node, info)
+    return tok, int(info[0]), int(info[1])
+
+
+def draw_many(w, n, seed, step, r0, node, nthreads=0):
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    out = np.empty(n, dtype=np.int32)
+    lib().oracle_draw_many(n, len(w), w, seed, step, r0, node, out, int(nthreads))
+    return out
 
 
 def race_many(w, n, seed, step, r0, node, nthreads=0):

@@ -20,8 +20,9 @@
  *  - greedy: argmax ties go to the lowest vocab id; among children carrying the argmax token the
  *    lowest node index is taken;
  *  - T>0 is defined for chains only: node k's token was drafted from q of node k-1; accept iff
- *    U*q < p (strict); the bonus/residual token is drawn by an exponential race
- *    argmax_v [log w_v - log(-log U_v)] with Philox4x64-10 uniforms (8 per block).
+ *    U*q < p (strict); the bonus/residual token is drawn in two levels with Philox4x64-10
+ *    uniforms: an exponential race among 128-id block totals, then an inverse CDF inside the
+ *    winning block (oracle_draw).
  */
 #include <math.h>
 #include <stdint.h>
@@ -303,7 +304,8 @@ double oracle_uniform(uint64_t seed, uint64_t step, uint32_t r, uint32_t node, u
 
 /* Exponential race over weights w (>= 0): the winner is argmax over w_v > 0 of
  * log w_v - log(-log U_v), ties to the lowest v.  P(winner = v) = w_v / sum w exactly.
- * Returns the token, or -1 when no weight is positive.  *best_key receives the winning key. */
+ * Returns the token, or -1 when no weight is positive.  *best_key receives the winning key.
+ * (Kept as a reference sampler for the tests; the acceptance rule uses oracle_draw below.) */
 int oracle_race(int V, const double *w, uint64_t seed, uint64_t step, int r, int node,
                 double *best_key) {
     int best = -1;
@@ -316,6 +318,44 @@ int oracle_race(int V, const double *w, uint64_t seed, uint64_t step, int r, int
     }
     if (best_key) *best_key = bk;
     return best;
+}
+
+/* The method's draw from weights w (>= 0) in two levels, an exact sampler of w / sum w:
+ *  1. vocab ids form blocks of 128 consecutive ids (b = v / 128); block totals
+ *     W_b = sum_{v in b} w_v (summed in increasing v) race: b* = argmax_{W_b > 0} of
+ *     log W_b - log(-log U_b) with U_b = oracle_uniform(seed, step, r, node, b, 2), ties to the
+ *     lowest b;
+ *  2. inside b*, an inverse CDF with u = oracle_uniform(seed, step, r, node, b*, 3): the first
+ *     v (in increasing order) whose running sum exceeds u * W_b*; if rounding leaves none, the
+ *     last v of b* with w_v > 0.
+ * Returns the token, or -1 when no weight is positive; info (nullable) gets {b*, 0}. */
+int oracle_draw(int V, const double *w, uint64_t seed, uint64_t step, int r, int node,
+                int32_t *info) {
+    const int nb = (V + 127) / 128;
+    int bstar = -1;
+    double bk = -INFINITY, Wstar = 0.0;
+    for (int b = 0; b < nb; ++b) {
+        double W = 0.0;
+        for (int v = b * 128; v < V && v < b * 128 + 128; ++v) W += w[v];
+        if (!(W > 0.0)) continue;
+        double U = oracle_uniform(seed, step, (uint32_t)r, (uint32_t)node, (uint32_t)b, 2);
+        double key = log(W) - log(-log(U));
+        if (bstar < 0 || key > bk) { bk = key; bstar = b; Wstar = W; }
+    }
+    if (bstar < 0) return -1;
+    double u = oracle_uniform(seed, step, (uint32_t)r, (uint32_t)node, (uint32_t)bstar, 3);
+    double thr = u * Wstar, run = 0.0;
+    int last = -1;
+    for (int v = bstar * 128; v < V && v < bstar * 128 + 128; ++v) {
+        run += w[v];
+        if (w[v] > 0.0) last = v;
+        if (run > thr) {
+            if (info) { info[0] = bstar; info[1] = 0; }
+            return v;
+        }
+    }
+    if (info) { info[0] = bstar; info[1] = 1; }
+    return last;
 }
 
 /* p = softmax(z / T) of one row, in fp64. */
@@ -334,7 +374,7 @@ static void softmax_t(int V, const double *z, double T, double *p) {
  * p_u = softmax(z_u / T).  Walk k = 1, 2, ...: accept x_k iff U_k * q_{k-1}(x_k) < p_{k-1}(x_k)
  * (U_k = oracle_uniform(seed, step, r, k, 0, 1)).  At the first rejection (stop node u = k-1) the
  * bonus is drawn from norm(max(0, p_u - q_u)); when every node is accepted (u = n-1) it is drawn
- * from p_u.  Both draws use oracle_race at node u.  If the residual has no positive weight the
+ * from p_u.  Both draws use oracle_draw at node u.  If the residual has no positive weight the
  * draw falls back to p_u.
  * z and q are the request's rows [n][V] (q fp32 as given).  info (nullable) receives
  * {stop node, 1 if a rejection happened else 0, 1 if the residual fell back to p}.
@@ -376,10 +416,10 @@ int oracle_accept_chain(int n, const int32_t *parent, const int32_t *tokens, con
             double d = p[v] - (double)q[(size_t)u * V + v];
             w[v] = d > 0.0 ? d : 0.0;
         }
-        bonus = oracle_race(V, w, seed, step, r, u, NULL);
-        if (bonus < 0) { fell_back = 1; bonus = oracle_race(V, p, seed, step, r, u, NULL); }
+        bonus = oracle_draw(V, w, seed, step, r, u, NULL);
+        if (bonus < 0) { fell_back = 1; bonus = oracle_draw(V, p, seed, step, r, u, NULL); }
     } else {
-        bonus = oracle_race(V, p, seed, step, r, u, NULL);
+        bonus = oracle_draw(V, p, seed, step, r, u, NULL);
     }
     out_tokens[a] = bonus;
     if (info) { info[0] = u; info[1] = rejected; info[2] = fell_back; }
@@ -457,4 +497,12 @@ void oracle_race_many(int n, int V, const double *w, uint64_t seed, uint64_t ste
     set_threads(nthreads);
 #pragma omp parallel for schedule(static)
     for (int k = 0; k < n; ++k) out[k] = oracle_race(V, w, seed, step, r0 + k, node, NULL);
+}
+
+/* n two-level draws over the same weights, draw k using request index r0 + k. */
+void oracle_draw_many(int n, int V, const double *w, uint64_t seed, uint64_t step, int r0,
+                      int node, int32_t *out, int nthreads) {
+    set_threads(nthreads);
+#pragma omp parallel for schedule(static)
+    for (int k = 0; k < n; ++k) out[k] = oracle_draw(V, w, seed, step, r0 + k, node, NULL);
 }

@@ -6,8 +6,9 @@ Tolerances:
 * argmax, paths, accept lengths, bonus tokens, compacted KV: bit-exact, except at logit near-ties
   (fp64 top1 - top2 < 1e-3), which are logged and counted and excuse the rest of that request;
 * per-node top1-top2 gap: |err| <= 1e-3 + 1e-3 |gap| (fp32 accumulation over hidden_dim);
-* T > 0: accept decisions and race winners bit-exact, except sampling near-ties where the fp64
-  quantities compared differ by less than 1e-5 relative (fp32 vs fp64 rounding).
+* T > 0: accept decisions and drawn tokens bit-exact, except sampling near-ties where the fp64
+  quantities compared differ by less than 1e-5 relative (fp32 vs fp64 rounding): U*q vs p for
+  an accept test, the two blocks' race keys, or the inverse-CDF threshold inside a block.
 """
 from __future__ import annotations
 
@@ -111,15 +112,30 @@ def chain_compare(wl, res, requests, nthreads=0):
             u = oa
             tg, to = int(res["out_tokens"][r][oa]), int(o["out_tokens"][oa])
             rejected = o["info"][1] == 1
+            w = np.maximum(p[u] - qd[u], 0.0) if rejected else p[u].copy()
+            if rejected and not (w > 0).any():
+                w = p[u].copy()
+            V = len(w)
+            bg, bo = tg // 128, to // 128
 
-            def key(v):
-                w = max(0.0, p[u, v] - qd[u, v]) if rejected else p[u, v]
-                Uv = oracle.uniform(wl.seed, wl.step, r, u, v, 0)
-                return np.log(w) - np.log(-np.log(Uv)) if w > 0 else -np.inf
+            def bkey(b):
+                Wb = w[b * 128:(b + 1) * 128].sum()
+                Ub = oracle.uniform(wl.seed, wl.step, r, u, b, 2)
+                return np.log(Wb) - np.log(-np.log(Ub)) if Wb > 0 else -np.inf
 
-            kg, ko = key(tg), key(to)
-            assert np.isfinite(kg) and abs(kg - ko) <= SAMPLE_REL * max(1.0, abs(ko)), \
-                (r, tg, to, kg, ko)
+            if bg != bo:
+                kg, ko = bkey(bg), bkey(bo)
+                assert np.isfinite(kg) and abs(kg - ko) <= SAMPLE_REL * max(1.0, abs(ko)), \
+                    (r, tg, to, kg, ko)
+            else:
+                blk = w[bo * 128:min(V, (bo + 1) * 128)]
+                c = np.cumsum(blk)
+                W = c[-1]
+                thr = oracle.uniform(wl.seed, wl.step, r, u, bo, 3) * W
+                i = tg - bo * 128
+                before = c[i - 1] if i > 0 else 0.0
+                assert blk[i] > 0 and c[i] > thr - SAMPLE_REL * W and \
+                    before <= thr + SAMPLE_REL * W, (r, tg, to, c[i], before, thr, W)
         excused.add(r)
         near += 1
     return excused, near, ores

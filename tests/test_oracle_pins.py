@@ -388,6 +388,45 @@ def test_exponential_race_is_an_exact_sampler():
     assert oracle.race(np.zeros(16), 1, 0, 0, 0)[0] == -1
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("V", [16, 300, 1000])
+def test_two_level_draw_is_an_exact_sampler(V):
+    """10^6 draws: frequencies match w / sum w (blocks of 128 ids, ragged last block, zero
+    weights and a zero block included)."""
+    g = np.random.default_rng(V)
+    w = g.exponential(size=V) * (g.random(V) < 0.8)
+    if V >= 300:
+        w[128:256] = 0.0                       # a whole block without weight
+    n = 1_000_000
+    out = oracle.draw_many(w, n, 0xE7EE0500, 0, 0, 2)
+    probs = w / w.sum()
+    if V <= 300:
+        assert _chisq_p(out, probs) > 1e-4
+    else:                                      # pool the rare ids by block for the test
+        blocks = (np.arange(V) // 16)
+        pb = np.bincount(blocks, weights=probs)
+        assert _chisq_p(blocks[out], pb) > 1e-4
+    assert (w[out] > 0).all()
+    assert oracle.draw(np.zeros(V), 1, 0, 0, 0)[0] == -1
+
+
+def test_two_level_draw_blocks_and_inverse_cdf_by_hand():
+    """The draw's two levels written out for one case: the block race over 128-id totals, then
+    the first id whose running sum passes u * W."""
+    g = np.random.default_rng(4)
+    V, seed, step, r, node = 700, 12345, 3, 7, 2
+    w = g.exponential(size=V)
+    W = np.array([w[b * 128:(b + 1) * 128].sum() for b in range(6)])
+    keys = [np.log(W[b]) - np.log(-np.log(oracle.uniform(seed, step, r, node, b, 2)))
+            for b in range(6)]
+    b = int(np.argmax(keys))
+    u = oracle.uniform(seed, step, r, node, b, 3)
+    run = np.cumsum(w[b * 128:(b + 1) * 128])
+    want = b * 128 + int(np.argmax(run > u * W[b]))
+    tok, blk, _ = oracle.draw(w, seed, step, r, node)
+    assert (tok, blk) == (want, b)
+
+
 def test_accept_chain_rejects_branching_trees_and_bad_parents():
     z = np.zeros((3, 8))
     q = np.full((3, 8), 1 / 8, dtype=np.float32)

@@ -50,7 +50,8 @@ def test_noalloc_matches_workspace_entry_point_twice(name):
         assert torch.equal(out, ref_out)            # same kernel, same plan: bit-identical
 
 
-def test_noalloc_rejects_batches_beyond_the_static_scratch():
+def test_noalloc_rejects_batches_beyond_the_static_scratch(monkeypatch):
+    monkeypatch.setenv("ETREE_NSPLIT", "64")        # many KV splits: large partial buffers
     B, n, hq, hkv, L = 2, 64, 40, 8, 32768
     i32 = dict(dtype=torch.int32, device="cuda")
     cu = torch.tensor([0, n, 2 * n], **i32)
