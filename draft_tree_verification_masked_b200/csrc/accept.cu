@@ -277,39 +277,44 @@ __global__ void __launch_bounds__(128) accept_chain_kernel(AcceptParams p) {
 
 // The first level of the two-level draw, per request: the exponential race among the 128-id
 // block totals (key W_b / E_b with E_b = -log U_b, stream 2), ties to the lowest block; the
-// bonus is the inverse-CDF pick the GEMM epilogue made inside the winning block.  Residual
-// weights are used after a rejection unless none is positive, then p.
+// bonus is the inverse-CDF pick the GEMM epilogue made inside the winning block.  A residual
+// with no positive weight anywhere (p <= q everywhere: p = q up to rounding) gives the argmax
+// of p instead, taken from the per-block logit maxima.
 __global__ void bonus_kernel(AcceptParams p) {
   const int r = blockIdx.x;
   const int lane = threadIdx.x;
   const int node = p.stop_node[r];
   const float4* row = p.part2 + (size_t)r * p.n_tiles2;
-  float kr = -INFINITY, kp = -INFINITY;
-  int ir = -1, ip = -1;
-  for (int b = lane; b < p.n_tiles2; b += 32) {
-    const float4 v = row[b];
+  float kb = -INFINITY, zm = -INFINITY;
+  int ib = -1, iz = -1;
+  for (int g = lane; g * 8 < p.n_tiles2; g += 32) {
     float u[8];
-    uniforms8(p.seed, p.step, (uint32_t)(b >> 3), (uint32_t)node, (uint32_t)r, 2u, u);
-    const float E = -logf(u[b & 7]);
-    if (v.x > 0.f) merge_key(kr, ir, __fdividef(v.x, E), __float_as_int(v.y));
-    if (v.z > 0.f) merge_key(kp, ip, __fdividef(v.z, E), __float_as_int(v.w));
+    uniforms8(p.seed, p.step, (uint32_t)g, (uint32_t)node, (uint32_t)r, 2u, u);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int b = g * 8 + e;
+      if (b < p.n_tiles2) {
+        const float4 v = row[b];
+        if (v.x > 0.f) merge_key(kb, ib, __fdividef(v.x, -logf(u[e])), __float_as_int(v.y));
+        merge_key(zm, iz, v.z, __float_as_int(v.w));
+      }
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-    const float okr = __shfl_xor_sync(0xffffffffu, kr, off);
-    const int oir = __shfl_xor_sync(0xffffffffu, ir, off);
-    const float okp = __shfl_xor_sync(0xffffffffu, kp, off);
-    const int oip = __shfl_xor_sync(0xffffffffu, ip, off);
-    merge_key(kr, ir, okr, oir);
-    merge_key(kp, ip, okp, oip);
+    const float okb = __shfl_xor_sync(0xffffffffu, kb, off);
+    const int oib = __shfl_xor_sync(0xffffffffu, ib, off);
+    const float ozm = __shfl_xor_sync(0xffffffffu, zm, off);
+    const int oiz = __shfl_xor_sync(0xffffffffu, iz, off);
+    merge_key(kb, ib, okb, oib);
+    merge_key(zm, iz, ozm, oiz);
   }
   if (lane == 0) {
     const int base = p.cu_nodes[r];
     const int n = p.cu_nodes[r + 1] - base;
     if (n < 1 || n > p.n_max) return;
     const int a = p.accept_len[r];
-    const int bonus = (p.mode[r] && ir >= 0) ? ir : ip;
-    p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = bonus;
+    p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = ib >= 0 ? ib : iz;
   }
 }
 

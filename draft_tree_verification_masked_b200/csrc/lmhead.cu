@@ -18,9 +18,10 @@
 //   EPI_ARGMAX  per row and tile: top-1 value, its vocab id (lowest on ties) and top-2 value;
 //   EPI_LSE     per row and tile: m = max z*log2(e)/T and sum 2^(z*log2(e)/T - m), plus the
 //               logit of the row's child token when it falls in the tile;
-//   EPI_RACE    per row and 128-id block: the block totals of w = max(0, p - q) and w = p and,
-//               for each, the id where the block's running sum passes u_b times its total
-//               (two passes over the block in TMEM); the block race happens in bonus_kernel.
+//   EPI_RACE    per row and 128-id block: the block total of the draw's weights (max(0, p - q)
+//               after a rejection, else p), the id where the block's running sum passes u_b
+//               times that total, and the block's largest logit; the block race happens in
+//               bonus_kernel.
 #include "kernels.cuh"
 #include "philox.cuh"
 
@@ -81,64 +82,22 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, EpiRow& st, const
   }
 }
 
-// Two-level draw, first pass over one 128-id block: block totals of the residual weights
-// max(0, p - q) and of p, summed in increasing id order.  Returns nothing; updates Wr, Wp.
-__device__ __forceinline__ void race_sum(const GemmParams& p, const EpiRow& st, const float (&v)[32],
-                                         int col0, float& Wr, float& Wp) {
-  float q[32];
-  if (st.md) {
+// Draft probabilities of 32 consecutive ids (zero past the vocabulary).
+__device__ __forceinline__ void load_q32(const GemmParams& p, const float* qrow, int col0,
+                                         float (&q)[32]) {
+  if ((p.V & 3) == 0) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4) {
       float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-      if ((p.V & 3) == 0) {
-        if (col0 + j < p.V) t = __ldg(reinterpret_cast<const float4*>(st.qrow + col0 + j));
-      } else {
-        t.x = col0 + j < p.V ? __ldg(st.qrow + col0 + j) : 0.f;
-        t.y = col0 + j + 1 < p.V ? __ldg(st.qrow + col0 + j + 1) : 0.f;
-        t.z = col0 + j + 2 < p.V ? __ldg(st.qrow + col0 + j + 2) : 0.f;
-        t.w = col0 + j + 3 < p.V ? __ldg(st.qrow + col0 + j + 3) : 0.f;
-      }
+      if (col0 + j < p.V) t = __ldg(reinterpret_cast<const float4*>(qrow + col0 + j));
       q[j] = t.x;
       q[j + 1] = t.y;
       q[j + 2] = t.z;
       q[j + 3] = t.w;
     }
-  }
+  } else {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    if (col0 + j < p.V) {
-      const float pv = exp2f(v[j] * p.k_log2 - st.L2);
-      Wp += pv;
-      if (st.md) Wr += fmaxf(pv - q[j], 0.f);
-    }
-  }
-}
-
-// Second pass: the first id whose running sum exceeds its threshold (inverse CDF inside the
-// block); the arithmetic repeats the first pass exactly, so the running sums end at the totals.
-__device__ __forceinline__ void race_scan(const GemmParams& p, const EpiRow& st,
-                                          const float (&v)[32], int col0, float thr_r, float thr_p,
-                                          float& run_r, float& run_p, int& pick_r, int& pick_p,
-                                          int& last_r, int& last_p) {
-  float q[32];
-  if (st.md) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) q[j] = col0 + j < p.V ? __ldg(st.qrow + col0 + j) : 0.f;
-  }
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    if (col0 + j < p.V) {
-      const float pv = exp2f(v[j] * p.k_log2 - st.L2);
-      run_p += pv;
-      if (pv > 0.f) last_p = col0 + j;
-      if (pick_p < 0 && run_p > thr_p) pick_p = col0 + j;
-      if (st.md) {
-        const float w = fmaxf(pv - q[j], 0.f);
-        run_r += w;
-        if (w > 0.f) last_r = col0 + j;
-        if (pick_r < 0 && run_r > thr_r) pick_r = col0 + j;
-      }
-    }
+    for (int j = 0; j < 32; ++j) q[j] = col0 + j < p.V ? __ldg(qrow + col0 + j) : 0.f;
   }
 }
 
@@ -274,35 +233,72 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         st.qrow = p.q_draft + (size_t)g * p.V;
       }
       if constexpr (EPI == EPI_RACE) {
-        // this half owns one whole 128-id block: columns half*128 .. half*128+127 of the tile
+        // This half owns one whole 128-id block (columns half*128 .. +127 of the tile).
+        // Pass 1 turns the logits into the draw's weights -- max(0, p - q) after a rejection,
+        // p otherwise -- sums them in increasing id order, tracks the block's largest logit,
+        // and writes the weights back over the logits in TMEM.  Pass 2 rescans those weights
+        // for the first id whose running sum passes u_b times the block total.
         static_assert(BN == 256, "the two-level draw works on 128-id blocks");
         const int blk = nt * 2 + half;
         const int colb = blk * 128;
-        float Wr = 0.f, Wp = 0.f;
+        const uint32_t tcol = tbase + half * 128;
+        float W = 0.f, zmax = -INFINITY;
+        int zarg = -1;
+        float qa[32], qb[32];
+        if (active && st.md) load_q32(p, st.qrow, colb, qa);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
+          float (&q)[32] = (c & 1) ? qb : qa;
+          float (&qn)[32] = (c & 1) ? qa : qb;
+          if (active && st.md && c < 3) load_q32(p, st.qrow, colb + (c + 1) * 32, qn);
           float v[32];
-          tmem_ld32(tbase + (half * 4 + c) * 32, v);
-          if (active) race_sum(p, st, v, colb + c * 32, Wr, Wp);
+          tmem_ld32(tcol + c * 32, v);
+          if (active) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int col = colb + c * 32 + j;
+              float w = 0.f;
+              if (col < p.V) {
+                if (v[j] > zmax) {
+                  zmax = v[j];
+                  zarg = col;
+                }
+                const float pv = exp2f(v[j] * p.k_log2 - st.L2);
+                w = st.md ? fmaxf(pv - q[j], 0.f) : pv;
+                W += w;
+              }
+              v[j] = w;
+            }
+          }
+          tmem_st32(tcol + c * 32, v);
         }
         float u[8];
         uniforms8(p.seed, p.step, (uint32_t)(blk >> 3), (uint32_t)st.unode, (uint32_t)st.req, 3u,
                   u);
-        const float ub = u[blk & 7];
-        float run_r = 0.f, run_p = 0.f;
-        int pick_r = -1, pick_p = -1, last_r = -1, last_p = -1;
+        float ub = u[0];
+#pragma unroll
+        for (int e = 1; e < 8; ++e)
+          if ((blk & 7) == e) ub = u[e];
+        const float thr = ub * W;
+        float run = 0.f;
+        int pick = -1, last = -1;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float v[32];
-          tmem_ld32(tbase + (half * 4 + c) * 32, v);
-          if (active)
-            race_scan(p, st, v, colb + c * 32, ub * Wr, ub * Wp, run_r, run_p, pick_r, pick_p,
-                      last_r, last_p);
+          tmem_ld32(tcol + c * 32, v);
+          if (active) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              run += v[j];
+              if (v[j] > 0.f) last = colb + c * 32 + j;
+              if (pick < 0 && run > thr) pick = colb + c * 32 + j;
+            }
+          }
         }
-        st.r0 = Wr;
-        st.r1 = pick_r >= 0 ? pick_r : last_r;
-        st.r2 = Wp;
-        st.r3 = pick_p >= 0 ? pick_p : last_p;
+        st.r0 = W;
+        st.r1 = pick >= 0 ? pick : last;
+        st.r2 = zmax;
+        st.r3 = zarg;
       } else {
 #pragma unroll 1
         for (int c = half; c < kChunks; c += 2) {

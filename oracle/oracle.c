@@ -374,8 +374,8 @@ static void softmax_t(int V, const double *z, double T, double *p) {
  * p_u = softmax(z_u / T).  Walk k = 1, 2, ...: accept x_k iff U_k * q_{k-1}(x_k) < p_{k-1}(x_k)
  * (U_k = oracle_uniform(seed, step, r, k, 0, 1)).  At the first rejection (stop node u = k-1) the
  * bonus is drawn from norm(max(0, p_u - q_u)); when every node is accepted (u = n-1) it is drawn
- * from p_u.  Both draws use oracle_draw at node u.  If the residual has no positive weight the
- * draw falls back to p_u.
+ * from p_u.  Both draws use oracle_draw at node u.  If the residual has no positive weight
+ * (p <= q everywhere, which only rounding can produce) the bonus is the argmax of p_u.
  * z and q are the request's rows [n][V] (q fp32 as given).  info (nullable) receives
  * {stop node, 1 if a rejection happened else 0, 1 if the residual fell back to p}.
  * Returns a, OR_EINVAL for a malformed tree or OR_EUNSUPPORTED for a tree that is not a chain.
@@ -417,7 +417,14 @@ int oracle_accept_chain(int n, const int32_t *parent, const int32_t *tokens, con
             w[v] = d > 0.0 ? d : 0.0;
         }
         bonus = oracle_draw(V, w, seed, step, r, u, NULL);
-        if (bonus < 0) { fell_back = 1; bonus = oracle_draw(V, p, seed, step, r, u, NULL); }
+        if (bonus < 0) {
+            /* no positive residual weight: p <= q everywhere, i.e. p = q up to rounding; the
+             * bonus is then the mode of p (lowest id on ties) */
+            fell_back = 1;
+            bonus = 0;
+            for (int v = 1; v < V; ++v)
+                if (p[v] > p[bonus]) bonus = v;
+        }
     } else {
         bonus = oracle_draw(V, p, seed, step, r, u, NULL);
     }
