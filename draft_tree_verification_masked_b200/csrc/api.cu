@@ -53,23 +53,33 @@ static int env_int(const char* name, int dflt) {
 
 // ------------------------------------------------------------------------------ attention plan
 struct AttnPlan {
-  int G, tc, nw, nb, mchunks, nsplit, tps, stages;
+  int G, tc, keys, nw, nb, mchunks, nsplit, tps, stages;
 };
 
 // Launch plan of the attention call.  The tcgen05 kernel (default) takes 128-row blocks of
-// nb = floor(128 / G) whole nodes; the warp-MMA kernel (ETREE_ATTN=mma) takes 16-row warps.
-// Splits of the KV range are added until about four CTAs per SM exist, keeping >= 4 key tiles
-// per split.
+// nb = min(floor(128 / G), n_max) whole nodes; with at least one (request, KV head, row block) per
+// SM it uses 32-key tiles and two CTAs per SM, otherwise 64-key tiles and one CTA per SM.  The KV range
+// is split only to fill one wave of CTAs (a second, partial wave costs more than longer splits),
+// keeping >= 4 key tiles per split.  The warp-MMA kernel (ETREE_ATTN=mma) takes 16-row warps,
+// 64-key tiles, and aims at about four CTAs per SM.
 static AttnPlan plan_attn(const etree_batch* b, int hq, int hkv) {
   AttnPlan pl{};
   pl.G = hq / hkv;
   const char* kind = getenv("ETREE_ATTN");
   pl.tc = !(kind && strcmp(kind, "mma") == 0) && pl.G <= 128;
+  const int sms = sm_count();
   if (pl.tc) {
-    pl.nb = 128 / pl.G;
+    pl.nb = std::min(128 / pl.G, b->n_max);           // nodes per Q box (row block)
     pl.mchunks = (b->n_max + pl.nb - 1) / pl.nb;
     pl.nw = 4;
+    const int pairs0 = b->B * hkv * pl.mchunks;
+    // 32-key tiles (two CTAs per SM) pay off once there is at least one row block per SM;
+    // few, long work items (one request, long context) prefer 64-key tiles split over the SMs
+    pl.keys = pairs0 >= sms ? 32 : 64;
+    const int forced = env_int("ETREE_ATTN_KEYS", 0);
+    if (forced == 32 || forced == 64) pl.keys = forced;
   } else {
+    pl.keys = 64;
     const int m16 = (b->n_max * pl.G + 15) / 16;
     if (m16 <= 8) {
       pl.nw = std::max(1, m16);
@@ -80,25 +90,24 @@ static AttnPlan plan_attn(const etree_batch* b, int hq, int hkv) {
     }
   }
   const int pairs = b->B * hkv * pl.mchunks;
-  const int tiles_max = (b->kv_len_max + 63) / 64 + 1;
-  // The tcgen05 kernel runs one CTA per SM: split the KV range only to fill a single wave
-  // (a second, partial wave costs more than longer splits); keep >= 4 key tiles per split.
-  // The warp-MMA kernel aims at about four CTAs per SM.
-  const int sms = sm_count();
-  int nsplit = pl.tc ? std::max(1, sms / pairs) : (4 * sms + pairs - 1) / pairs;
+  const int tiles_max =
+      (b->kv_len_max + pl.keys - 1) / pl.keys + (b->n_max + pl.keys - 1) / pl.keys;
+  const int per_sm = pl.tc ? (pl.keys == 32 ? 2 : 1) : 4;
+  int nsplit = pl.tc ? std::max(1, per_sm * sms / pairs) : (per_sm * sms + pairs - 1) / pairs;
   nsplit = std::min(nsplit, std::max(1, tiles_max / 4));
   nsplit = std::max(1, std::min(nsplit, tiles_max));
   const int forced = env_int("ETREE_NSPLIT", 0);
   if (forced > 0) nsplit = std::min(forced, tiles_max);
   pl.tps = (tiles_max + nsplit - 1) / nsplit;
   pl.nsplit = (tiles_max + pl.tps - 1) / pl.tps;
-  pl.stages = env_int("ETREE_STAGES", pl.tc ? 4 : 3) == 4 ? 4 : 3;
+  pl.stages = env_int("ETREE_STAGES", 3) == 4 ? 4 : 3;
   return pl;
 }
 
 // ------------------------------------------------------------------------------ workspace map
 struct WsLayout {
-  size_t o_part, ml_part, part, child_tok, zchild, lse2, stop_row, stop_node, mode, hid2, part2;
+  size_t order, o_part, ml_part, part, child_tok, zchild, lse2, stop_row, stop_node, mode, hid2,
+      part2;
   size_t total;
   int n_tiles;
 };
@@ -118,6 +127,7 @@ static WsLayout layout(const etree_batch* b, int hq, int hkv, int hidden_dim, in
   size_t nsplit = 1;
   if (hq > 0 && hkv > 0 && hq % hkv == 0) nsplit = (size_t)plan_attn(b, hq, hkv).nsplit;
   const size_t rows = nt * (size_t)std::max(0, hq);
+  w.order = take(hq > 0 ? B * sizeof(int32_t) : 0);
   w.o_part = take(nsplit > 1 ? rows * nsplit * 128 * sizeof(float) : 0);
   w.ml_part = take(nsplit > 1 ? rows * nsplit * sizeof(float2) : 0);
   // two summaries per vocab tile, at the narrowest tile width the LM head may pick (128)
@@ -312,7 +322,7 @@ etree_status etree_attn_plan(const etree_batch* batch, int hq, int hkv, int32_t*
   if (row_blocks) *row_blocks = pl.mchunks;
   if (splits) *splits = pl.nsplit;
   if (tiles_per_split) *tiles_per_split = pl.tps;
-  if (launches) *launches = pl.nsplit > 1 ? 2 : 1;
+  if (launches) *launches = (pl.nsplit > 1 ? 2 : 1) + (batch->B >= 8 ? 1 : 0);
   return ETREE_OK;
 }
 
@@ -369,13 +379,15 @@ etree_status etree_verify_attn(const etree_batch* b, const uint16_t* q, const ui
 
   const AttnPlan pl = plan_attn(b, hq, hkv);
   CUtensorMap kc, vc, kt, vt;
-  if ((st = get_map(k_cache, 3, 128, hkv, cache_slots, 64, 1, 64, &kc))) return st;
-  if ((st = get_map(v_cache, 3, 128, hkv, cache_slots, 64, 1, 64, &vc))) return st;
-  if ((st = get_map(k_tree, 3, 128, hkv, b->n_total, 64, 1, 64, &kt))) return st;
-  if ((st = get_map(v_tree, 3, 128, hkv, b->n_total, 64, 1, 64, &vt))) return st;
+  const uint32_t kb = (uint32_t)pl.keys;
+  if ((st = get_map(k_cache, 3, 128, hkv, cache_slots, 64, 1, kb, &kc))) return st;
+  if ((st = get_map(v_cache, 3, 128, hkv, cache_slots, 64, 1, kb, &vc))) return st;
+  if ((st = get_map(k_tree, 3, 128, hkv, b->n_total, 64, 1, kb, &kt))) return st;
+  if ((st = get_map(v_tree, 3, 128, hkv, b->n_total, 64, 1, kb, &vt))) return st;
 
   const WsLayout w = layout(b, hq, hkv, 0, 0);
   AttnParams p{};
+  p.order = nullptr;
   p.cu_nodes = b->cu_nodes;
   p.parent = b->parent;
   p.kv_len = b->kv_len;
@@ -396,12 +408,21 @@ etree_status etree_verify_attn(const etree_batch* b, const uint16_t* q, const ui
   p.mchunks = pl.mchunks;
   p.nsplit = pl.nsplit;
   p.tps = pl.tps;
+  p.keys = pl.keys;
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaError_t e;
+  // with many requests of mixed lengths, dispatch the longest first
+  p.order = nullptr;
+  if (b->B >= 8 && env_int("ETREE_ATTN_LPT", 1)) {
+    p.order = at<int32_t>(workspace, w.order);
+    e = launch_attn_order(b->kv_len, b->B, at<int32_t>(workspace, w.order),
+                          static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "etree_verify_attn order");
+  }
   if (pl.tc) {
     CUtensorMap tq;
     if ((st = get_map(q, 3, 128, hq, b->n_total, 64, pl.G, pl.nb, &tq))) return st;
-    e = launch_attn_tc(tq, kc, vc, kt, vt, p, pl.nb, pl.stages, b->n_total,
+    e = launch_attn_tc(tq, kc, vc, kt, vt, p, pl.nb, b->n_total,
                        static_cast<cudaStream_t>(stream));
   } else {
     e = launch_attn(kc, vc, kt, vt, p, pl.nw, pl.stages, b->n_total,

@@ -5,28 +5,31 @@
 // DFlash2 and DSpark ...", section "Technical Background"), with both matrix products on the
 // 5th-generation tensor cores:
 //
-//   S  = Q K^T   tcgen05.mma M=128 (query rows) x N=64 (keys) x K=128, fp32 into TMEM;
-//   O += P V     tcgen05.mma M=128 x N=128 (head dims) x K=64 (keys), fp32 accumulated in TMEM.
+//   S  = Q K^T   tcgen05.mma M=128 (query rows) x N=KEYS x K=128, fp32 into TMEM;
+//   O += P V     tcgen05.mma M=128 x N=128 (head dims) x K=KEYS, fp32 accumulated in TMEM.
 //
 // One CTA = (request, KV head, 128-row block, KV split).  The query rows are the (node, group
 // head) pairs of one KV head, row = node * G + g; one TMA box {64 dims, G heads, NB nodes} of the
 // [n_total][hq][128] query tensor lands them in exactly that order (NB = floor(128 / G)).
-// Warp 0 streams Q once and the 64-key K/V tiles through a STAGES-deep ring; warp 1 issues the
-// MMAs; warps 2-5 own one query row per thread (= one TMEM lane): they read S from TMEM, apply
-// the key mask (cache length, or the row's ancestor bitmask on the tree tile), run the online
-// softmax in log2 units, and write P (bf16, 128-byte swizzle) to shared memory for the PV
-// product.  S is double-buffered in TMEM so QK^T of tile j+1 overlaps the softmax of tile j.
-// O is rescaled lazily: only when a row's running maximum grows by more than 2^8 does the
-// softmax read-modify-write O in TMEM, so P stays below 256 and the usual case has no O traffic.
+// Warp 0 streams Q once and the KEYS-key K/V tiles through a STAGES-deep ring; warp 1 issues the
+// MMAs; the softmax warps own one query row per thread (= one TMEM lane; with 64-key tiles two
+// warps share a row, 32 keys each, and exchange row maxima): they read S from TMEM, apply
+// the key mask (cache length, or the row's ancestor bitmask on the tree tiles), run the online
+// softmax in log2 units, and write P (bf16, swizzled) to shared memory for the PV product.
+// S and P are double-buffered so QK^T of tile j+1 and PV of tile j overlap the softmax.  O is
+// rescaled lazily: only when a row's running maximum grows by more than 2^8 does the softmax
+// read-modify-write O in TMEM, so P stays below 256 and the usual case has no O traffic.
+//
+// Two shapes are built.  KEYS = 64 with a 4-deep ring runs one CTA per SM (for few, long
+// work items).  KEYS = 32 with a 3-deep ring fits two CTAs per SM, which overlaps one CTA's
+// start-up and tail with the other's streaming; its Q rows are rotated into a different TMEM
+// lane quarter per CTA so that co-resident CTAs run their softmax on different SM partitions.
 #include "kernels.cuh"
 
 namespace etree {
 
 namespace {
-constexpr int kKeys = 64;
-constexpr int kKV = 4 * 8192;               // K lo/hi + V lo/hi boxes of [64 keys][64 dims]
 constexpr int kQBytes = 2 * 16384;          // Q lo/hi boxes of [128 rows][64 dims]
-constexpr int kPBytes = 16384;              // one P buffer: [128 rows][64 keys] bf16
 constexpr float kLazy = 8.0f;               // rescale O only when the max grows by > 2^8
 
 struct TcSmem {
@@ -34,26 +37,38 @@ struct TcSmem {
   uint64_t kv_full[4], kv_empty[4], q_full, s_full[2], s_free[2], p_full[2], p_free[2];
   uint64_t anc[64];
   int32_t par[64];
+  float xmax[2][2][128];                    // row-max exchange: [tile parity][key half][row]
+  float xl[2][128];                         // final row sums of the two key halves
+  uint64_t xbar[4][2], xlbar[4];            // exchange barriers of the warp pairs (bounded waits)
   uint32_t tmem;
+};
+
+template <int KEYS>
+struct TcShape {
+  static constexpr int kBox = KEYS * 128;   // one [KEYS keys][64 dims] bf16 box
+  static constexpr int kKV = 4 * kBox;      // K lo/hi + V lo/hi
+  static constexpr int kPRow = KEYS * 2;    // bytes per P row
+  static constexpr int kPBytes = 128 * kPRow;
 };
 }  // namespace
 
-template <int STAGES>
-__global__ void __launch_bounds__(192, 1)
+template <int KEYS, int STAGES, int SW>
+__global__ void __launch_bounds__(32 * (2 + SW), KEYS == 32 ? 2 : 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kt,
                const __grid_constant__ CUtensorMap tm_vt, AttnParams p, int NB) {
+  using Sh = TcShape<KEYS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;                                   // 32 KB
-  uint8_t* sKV = smem + kQBytes;                        // STAGES x 32 KB
-  uint8_t* sP = sKV + STAGES * kKV;                     // 2 x 16 KB (double buffer)
-  TcSmem* sh = reinterpret_cast<TcSmem*>(sP + 2 * kPBytes);
+  uint8_t* sKV = smem + kQBytes;                        // STAGES x kKV
+  uint8_t* sP = sKV + STAGES * Sh::kKV;                 // 2 x kPBytes (double buffer)
+  TcSmem* sh = reinterpret_cast<TcSmem*>(sP + 2 * Sh::kPBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_req = p.hkv * p.mchunks;
-  const int r = blockIdx.x / per_req;
+  const int r = p.order ? p.order[blockIdx.x / per_req] : blockIdx.x / per_req;
   const int kvh = (blockIdx.x % per_req) / p.mchunks;
   const int mb = blockIdx.x % p.mchunks;
   const int s = blockIdx.y;
@@ -71,14 +86,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
   const int node0 = mb * NB;
   if (node0 >= n) return;
-  const int nt_cache = (L + kKeys - 1) / kKeys;
-  const int total = nt_cache + 1;                       // the tree tile comes last
+  const int nt_cache = (L + KEYS - 1) / KEYS;
+  const int total = nt_cache + (n + KEYS - 1) / KEYS;   // the tree tiles come last
   const int t0 = s * p.tps;
   const int t1 = min(total, t0 + p.tps);
   if (t0 >= t1) return;
   const int T = t1 - t0;
-  const bool has_tree = (t1 == total);
+  const bool has_tree = (t1 > nt_cache);
   const int qrows = NB * G;                             // rows the Q box fills
+  // lane quarter rotation of the Q rows (see the header)
+  int rot = 0;
+  if (KEYS == 32) {
+    if (qrows <= 32) rot = 32 * (blockIdx.x & 3);
+    else if (qrows <= 64) rot = 64 * (blockIdx.x & 1);
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -88,9 +109,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     mbar_init(&sh->q_full, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->s_full[b], 1);
-      mbar_init(&sh->s_free[b], 4);
-      mbar_init(&sh->p_full[b], 4);
+      mbar_init(&sh->s_free[b], SW);
+      mbar_init(&sh->p_full[b], SW);
       mbar_init(&sh->p_free[b], 1);
+    }
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&sh->xbar[q][0], 2);
+      mbar_init(&sh->xbar[q][1], 2);
+      mbar_init(&sh->xlbar[q], 2);
     }
     fence_barrier_init();
   }
@@ -119,9 +145,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       sh->anc[i] = m;
     }
   }
-  // rows past the Q box are zero so that their (unused) products stay finite
-  for (int i = threadIdx.x; i < (128 - qrows) * 16; i += blockDim.x) {
-    const int row = qrows + i / 16, c = i % 16;
+  // rows outside the Q box are zero so that their (unused) products stay finite
+  for (int i = threadIdx.x; i < 128 * 16; i += blockDim.x) {
+    const int row = i / 16, c = i % 16;
+    if (row >= rot && row < rot + qrows) continue;
     uint4* dst = reinterpret_cast<uint4*>(sQ + (c >> 3) * 16384 + row * 128 + (c & 7) * 16);
     *dst = make_uint4(0u, 0u, 0u, 0u);
   }
@@ -137,8 +164,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       prefetch_tmap(&tm_kc);
       prefetch_tmap(&tm_vc);
       mbar_arrive_expect_tx(&sh->q_full, 2 * qrows * 128);
-      tma_load_3d(sQ, &tm_q, &sh->q_full, 0, kvh * G, base + node0);
-      tma_load_3d(sQ + 16384, &tm_q, &sh->q_full, 64, kvh * G, base + node0);
+      tma_load_3d(sQ + rot * 128, &tm_q, &sh->q_full, 0, kvh * G, base + node0);
+      tma_load_3d(sQ + 16384 + rot * 128, &tm_q, &sh->q_full, 64, kvh * G, base + node0);
       for (int j = 0; j < T; ++j) {
         const int t = t0 + j;
         const int st = j % STAGES;
@@ -147,26 +174,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           report(p.ws, ETREE_ETIMEOUT, DET_WAIT_ATTN);
           break;
         }
-        uint8_t* dst = sKV + st * kKV;
-        mbar_arrive_expect_tx(&sh->kv_full[st], kKV);
+        uint8_t* dst = sKV + st * Sh::kKV;
+        mbar_arrive_expect_tx(&sh->kv_full[st], Sh::kKV);
         if (t < nt_cache) {
-          const int32_t slot = static_cast<int32_t>(sbase + (int64_t)t * kKeys);
+          const int32_t slot = static_cast<int32_t>(sbase + (int64_t)t * KEYS);
           tma_load_3d(dst, &tm_kc, &sh->kv_full[st], 0, kvh, slot);
-          tma_load_3d(dst + 8192, &tm_kc, &sh->kv_full[st], 64, kvh, slot);
-          tma_load_3d(dst + 16384, &tm_vc, &sh->kv_full[st], 0, kvh, slot);
-          tma_load_3d(dst + 24576, &tm_vc, &sh->kv_full[st], 64, kvh, slot);
+          tma_load_3d(dst + Sh::kBox, &tm_kc, &sh->kv_full[st], 64, kvh, slot);
+          tma_load_3d(dst + 2 * Sh::kBox, &tm_vc, &sh->kv_full[st], 0, kvh, slot);
+          tma_load_3d(dst + 3 * Sh::kBox, &tm_vc, &sh->kv_full[st], 64, kvh, slot);
         } else {
-          tma_load_3d(dst, &tm_kt, &sh->kv_full[st], 0, kvh, base);
-          tma_load_3d(dst + 8192, &tm_kt, &sh->kv_full[st], 64, kvh, base);
-          tma_load_3d(dst + 16384, &tm_vt, &sh->kv_full[st], 0, kvh, base);
-          tma_load_3d(dst + 24576, &tm_vt, &sh->kv_full[st], 64, kvh, base);
+          const int node = base + (t - nt_cache) * KEYS;
+          tma_load_3d(dst, &tm_kt, &sh->kv_full[st], 0, kvh, node);
+          tma_load_3d(dst + Sh::kBox, &tm_kt, &sh->kv_full[st], 64, kvh, node);
+          tma_load_3d(dst + 2 * Sh::kBox, &tm_vt, &sh->kv_full[st], 0, kvh, node);
+          tma_load_3d(dst + 3 * Sh::kBox, &tm_vt, &sh->kv_full[st], 64, kvh, node);
         }
       }
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idS = idesc_bf16_f32(128, kKeys);
+      const uint32_t idS = idesc_bf16_f32(128, KEYS);
       const uint32_t idO = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) is MN-major
       bool ok = mbar_wait(&sh->q_full, 0);
       tc_fence_after();
@@ -175,11 +203,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int pb = jj & 1;
         if (!mbar_wait(&sh->p_full[pb], (jj >> 1) & 1)) return false;
         tc_fence_after();
-        const uint64_t dp = smem_desc_sw128(sP + pb * kPBytes);
-        const uint8_t* v0 = sKV + (jj % STAGES) * kKV + 16384;
+        const uint8_t* pbuf = sP + pb * Sh::kPBytes;
+        const uint64_t dp = KEYS == 64 ? smem_desc_sw128(pbuf) : smem_desc_sw64(pbuf);
+        const uint8_t* v0 = sKV + (jj % STAGES) * Sh::kKV + 2 * Sh::kBox;
 #pragma unroll
-        for (int k = 0; k < kKeys / 16; ++k)
-          tc_mma_bf16(tmem + 128, dp + 2 * k, smem_desc_sw128_mn(v0 + k * 2048, 8192), idO,
+        for (int k = 0; k < KEYS / 16; ++k)
+          tc_mma_bf16(tmem + 128, dp + 2 * k, smem_desc_sw128_mn(v0 + k * 2048, Sh::kBox), idO,
                       (jj > 0 || k > 0) ? 1u : 0u);
         tc_commit(&sh->p_free[pb]);
         tc_commit(&sh->kv_empty[jj % STAGES]);
@@ -191,11 +220,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!mbar_wait(&sh->kv_full[st], (j / STAGES) & 1)) { ok = false; break; }
         if (j >= 2 && !mbar_wait(&sh->s_free[sb], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint8_t* k0 = sKV + st * kKV;
-        const uint64_t dk0 = smem_desc_sw128(k0), dk1 = smem_desc_sw128(k0 + 8192);
+        const uint8_t* k0 = sKV + st * Sh::kKV;
+        const uint64_t dk0 = smem_desc_sw128(k0), dk1 = smem_desc_sw128(k0 + Sh::kBox);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          tc_mma_bf16(tmem + sb * kKeys, (k < 4 ? dq0 : dq1) + 2 * (k & 3),
+          tc_mma_bf16(tmem + sb * KEYS, (k < 4 ? dq0 : dq1) + 2 * (k & 3),
                       (k < 4 ? dk0 : dk1) + 2 * (k & 3), idS, k > 0 ? 1u : 0u);
         tc_commit(&sh->s_full[sb]);
         if (j >= 1 && !pv(j - 1)) { ok = false; break; }
@@ -204,12 +233,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (!ok) report(p.ws, ETREE_ETIMEOUT, DET_WAIT_ATTN);
     }
   } else {
-    // ------------------------------------------------------------------- softmax warpgroup
+    // ------------------------------------------------------------------- softmax warps
+    // SW/4 warps per TMEM lane quarter; warp half `kh` of a quarter owns keys
+    // [kh*CW, kh*CW + CW) of every tile (CW = KEYS / (SW/4)) and O columns [kh*OW, kh*OW + OW).
+    constexpr int NH = SW / 4;
+    constexpr int CW = KEYS / NH;
+    constexpr int OW = 128 / NH;
     const int wq = warp & 3;
+    const int kh = (warp - 2) >> 2;
     const int row = wq * 32 + lane;
-    const int node_l = row / G, g = row - node_l * G;
+    const int lrow = row - rot;
+    const bool inbox = lrow >= 0 && lrow < qrows;
+    const int node_l = inbox ? lrow / G : 0, g = inbox ? lrow - node_l * G : 0;
     const int node = node0 + node_l;
-    const bool valid = row < qrows && node < n;
+    const bool valid = inbox && node < n;
     const uint64_t anc = (has_tree && valid) ? sh->anc[node] : 0ull;
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     float m_ref = -INFINITY, l = 0.f;
@@ -219,39 +256,46 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int sb = j & 1;
       if (!mbar_wait(&sh->s_full[sb], (j >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      float sc[64];
+      float sc[CW];
       {
-        float a[32], b[32];
-        tmem_ld32(lane_base + sb * kKeys, a);
-        tmem_ld32(lane_base + sb * kKeys + 32, b);
+        float a[32];
+        tmem_ld32(lane_base + sb * KEYS + kh * CW, a);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          sc[c] = a[c];
-          sc[32 + c] = b[c];
+        for (int c = 0; c < 32; ++c) sc[c] = a[c];
+        if constexpr (CW == 64) {
+          tmem_ld32(lane_base + sb * KEYS + 32, a);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sc[32 + c] = a[c];
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->s_free[sb]);
 
-      // keep-mask of this row's 64 keys: the cache positions below kv_len, or on the tree
-      // tile the row's ancestor bits
-      uint32_t klo, khi;
+      // keep-mask of this thread's keys: the cache positions below kv_len, or on a tree tile
+      // the row's ancestor bits for the tile's nodes
+      uint32_t kw[CW / 32];
+      const int k0 = kh * CW;                           // first key of this thread in the tile
       if (!valid) {
-        klo = khi = 0u;
-      } else if (t == nt_cache) {
-        klo = static_cast<uint32_t>(anc);
-        khi = static_cast<uint32_t>(anc >> 32);
+#pragma unroll
+        for (int w = 0; w < CW / 32; ++w) kw[w] = 0u;
+      } else if (t >= nt_cache) {
+        const int sh0 = (t - nt_cache) * KEYS + k0;
+#pragma unroll
+        for (int w = 0; w < CW / 32; ++w) kw[w] = static_cast<uint32_t>(anc >> (sh0 + 32 * w));
       } else {
-        const int lim = L - t * kKeys;                  // >= 1 on a cache tile
-        klo = lim >= 32 ? 0xffffffffu : ((1u << lim) - 1u);
-        khi = lim >= 64 ? 0xffffffffu : (lim > 32 ? ((1u << (lim - 32)) - 1u) : 0u);
+        const int lim = L - t * KEYS - k0;
+#pragma unroll
+        for (int w = 0; w < CW / 32; ++w) {
+          const int lw = lim - 32 * w;
+          kw[w] = lw >= 32 ? 0xffffffffu : (lw > 0 ? ((1u << lw) - 1u) : 0u);
+        }
       }
       const float sl = p.scale_log2;
       float t0m = -INFINITY, t1m = -INFINITY, t2m = -INFINITY, t3m = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 64; c += 4) {
-        const uint32_t w = c < 32 ? klo : khi;
+      for (int c = 0; c < CW; c += 4) {
+        const uint32_t w = kw[c >> 5];
         const int b0 = c & 31;
         const float v0 = ((w >> b0) & 1u) ? sc[c] * sl : -INFINITY;
         const float v1 = ((w >> (b0 + 1)) & 1u) ? sc[c + 1] * sl : -INFINITY;
@@ -266,16 +310,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         t2m = fmaxf(t2m, v2);
         t3m = fmaxf(t3m, v3);
       }
-      const float tmax = fmaxf(fmaxf(t0m, t1m), fmaxf(t2m, t3m));
+      float tmax = fmaxf(fmaxf(t0m, t1m), fmaxf(t2m, t3m));
+      if constexpr (NH == 2) {                          // combine the two key halves of the row
+        sh->xmax[j & 1][kh][row] = tmax;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->xbar[wq][j & 1]);
+        if (!mbar_wait(&sh->xbar[wq][j & 1], (j >> 1) & 1)) { ok = false; break; }
+        tmax = fmaxf(tmax, sh->xmax[j & 1][kh ^ 1][row]);
+      }
       const bool need = tmax > m_ref + kLazy;           // also true for the first finite max
       const bool any = __any_sync(0xffffffffu, need);
       const float m_new = need ? tmax : m_ref;
       const float off = (m_new == -INFINITY) ? 0.f : m_new;
       const float corr = need ? exp2f(m_ref - m_new) : 1.f;
       float ls0 = 0.f, ls1 = 0.f;
-      uint32_t pk[32];
+      uint32_t pk[CW / 2];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < CW / 2; ++c) {
         const float e0 = ex2_approx(sc[2 * c] - off), e1 = ex2_approx(sc[2 * c + 1] - off);
         ls0 += e0;
         ls1 += e1;
@@ -288,12 +339,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!mbar_wait(&sh->p_free[(j - 1) & 1], ((j - 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < OW / 32; ++c) {
           float o[32];
-          tmem_ld32(lane_base + 128 + c * 32, o);
+          const uint32_t ta = lane_base + 128 + kh * OW + c * 32;
+          tmem_ld32(ta, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= corr;
-          tmem_st32(lane_base + 128 + c * 32, o);
+          tmem_st32(ta, o);
         }
       }
       // P buffer j % 2 is free once PV(j - 2) has completed
@@ -301,11 +353,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (j >= 2) {
         if (!mbar_wait(&sh->p_free[pb], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
       }
-      uint8_t* prow = sP + pb * kPBytes + row * 128;
+      uint8_t* prow = sP + pb * Sh::kPBytes + row * Sh::kPRow;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v;
+      for (int c = 0; c < CW / 8; ++c) {
+        const uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        const int lc = kh * (CW / 8) + c;               // 16-byte chunk within the P row
+        const int phys = KEYS == 64 ? (lc ^ (row & 7)) : (lc ^ ((row >> 1) & 3));
+        *reinterpret_cast<uint4*>(prow + (phys << 4)) = v;
       }
       fence_proxy_async();
       tc_fence_before();
@@ -314,16 +368,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     if (ok && !mbar_wait(&sh->p_free[(T - 1) & 1], ((T - 1) >> 1) & 1)) ok = false;
     if (!ok) report(p.ws, ETREE_ETIMEOUT, DET_WAIT_ATTN);
+    if constexpr (NH == 2) {                            // the row sum covers both key halves
+      sh->xl[kh][row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->xlbar[wq]);
+      if (!mbar_wait(&sh->xlbar[wq], 0)) report(p.ws, ETREE_ETIMEOUT, DET_WAIT_ATTN);
+      l += sh->xl[kh ^ 1][row];
+    }
     tc_fence_after();
     const size_t gidx = (size_t)(base + (valid ? node : 0)) * p.hq + kvh * G + g;
     if (p.nsplit == 1) {
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < OW / 32; ++c) {
+        const int col = kh * OW + c * 32;
         float o[32];
-        tmem_ld32(lane_base + 128 + c * 32, o);
+        tmem_ld32(lane_base + 128 + col, o);
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + gidx * 128 + c * 32);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + gidx * 128 + col);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             dst[q] = make_uint4(pack_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
@@ -332,21 +394,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
         }
       }
-      if (valid && p.lse) p.lse[gidx] = (m_ref + log2f(l)) * 0.69314718055994531f;
+      if (valid && kh == 0 && p.lse) p.lse[gidx] = (m_ref + log2f(l)) * 0.69314718055994531f;
     } else {
       float* op = p.o_part + (gidx * p.nsplit + s) * 128;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < OW / 32; ++c) {
+        const int col = kh * OW + c * 32;
         float o[32];
-        tmem_ld32(lane_base + 128 + c * 32, o);
+        tmem_ld32(lane_base + 128 + col, o);
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(op + c * 32);
+          float4* dst = reinterpret_cast<float4*>(op + col);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
         }
       }
-      if (valid) p.ml_part[gidx * p.nsplit + s] = make_float2(m_ref, l);
+      if (valid && kh == 0) p.ml_part[gidx * p.nsplit + s] = make_float2(m_ref, l);
     }
   }
   tc_fence_before();
@@ -357,29 +420,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
 }
 
-size_t attn_tc_smem_bytes(int stages) {
-  return 1024 + kQBytes + (size_t)stages * kKV + 2 * kPBytes + sizeof(TcSmem);
+template <int KEYS, int STAGES, int SW>
+static cudaError_t launch_shape(const CUtensorMap& q, const CUtensorMap& kc, const CUtensorMap& vc,
+                                const CUtensorMap& kt, const CUtensorMap& vt, const AttnParams& p,
+                                int nb, cudaStream_t stream) {
+  using Sh = TcShape<KEYS>;
+  const size_t smem = 1024 + kQBytes + (size_t)STAGES * Sh::kKV + 2 * Sh::kPBytes + sizeof(TcSmem);
+  auto k = attn_tc_kernel<KEYS, STAGES, SW>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.B * p.hkv * p.mchunks, p.nsplit);
+  k<<<grid, 32 * (2 + SW), smem, stream>>>(q, kc, vc, kt, vt, p, nb);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_attn_tc(const CUtensorMap& q, const CUtensorMap& kc, const CUtensorMap& vc,
                            const CUtensorMap& kt, const CUtensorMap& vt, const AttnParams& p,
-                           int nb, int stages, int n_total, cudaStream_t stream) {
-  dim3 grid(p.B * p.hkv * p.mchunks, p.nsplit);
-  cudaError_t e;
-  if (stages >= 4) {
-    auto k = attn_tc_kernel<4>;
-    const size_t smem = attn_tc_smem_bytes(4);
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 192, smem, stream>>>(q, kc, vc, kt, vt, p, nb);
-  } else {
-    auto k = attn_tc_kernel<3>;
-    const size_t smem = attn_tc_smem_bytes(3);
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 192, smem, stream>>>(q, kc, vc, kt, vt, p, nb);
-  }
-  e = cudaGetLastError();
+                           int nb, int n_total, cudaStream_t stream) {
+  cudaError_t e = p.keys == 32 ? launch_shape<32, 3, 4>(q, kc, vc, kt, vt, p, nb, stream)
+                               : launch_shape<64, 4, 8>(q, kc, vc, kt, vt, p, nb, stream);
   if (e != cudaSuccess || p.nsplit == 1) return e;
   return launch_attn_combine(p, n_total, stream);
 }

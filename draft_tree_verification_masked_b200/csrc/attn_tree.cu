@@ -44,7 +44,7 @@ attn_tree_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_req = p.hkv * p.mchunks;
-  const int r = blockIdx.x / per_req;
+  const int r = p.order ? p.order[blockIdx.x / per_req] : blockIdx.x / per_req;
   const int kvh = (blockIdx.x % per_req) / p.mchunks;
   const int mc = blockIdx.x % p.mchunks;
   const int s = blockIdx.y;
@@ -312,7 +312,7 @@ __global__ void attn_combine_kernel(AttnParams p, int n_total) {
   const int L = p.kv_len[lo];
   const int n = p.cu_nodes[lo + 1] - p.cu_nodes[lo];
   if (n < 1 || n > p.n_max || L < 0 || L > p.kv_len_max) return;   // reported by the main kernel
-  const int total = (L + kTileKeys - 1) / kTileKeys + 1;
+  const int total = (L + p.keys - 1) / p.keys + (n + p.keys - 1) / p.keys;
   const int used = min(p.nsplit, (total + p.tps - 1) / p.tps);
   float M = -INFINITY;
   for (int s = 0; s < used; ++s) M = fmaxf(M, p.ml_part[(size_t)gw * p.nsplit + s].x);
@@ -377,6 +377,30 @@ cudaError_t launch_attn(const CUtensorMap& kc, const CUtensorMap& vc, const CUte
   }
   if (e != cudaSuccess || p.nsplit == 1) return e;
   return launch_attn_combine(p, n_total, stream);
+}
+
+// Longest-first dispatch order: request r's rank is the number of requests with a longer KV
+// cache (ties by index), so order[rank] lists requests by decreasing length.  CTAs are
+// dispatched roughly in block order, and starting the long work first shortens the tail of a
+// batch with mixed lengths.
+__global__ void attn_order_kernel(const int32_t* kv_len, int B, int32_t* order) {
+  extern __shared__ int32_t len_s[];
+  for (int i = threadIdx.x; i < B; i += blockDim.x) len_s[i] = kv_len[i];
+  __syncthreads();
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= B) return;
+  const int L = len_s[r];
+  int rank = 0;
+  for (int i = 0; i < B; ++i) {
+    const int Li = len_s[i];
+    rank += (Li > L) || (Li == L && i < r);
+  }
+  order[rank] = r;
+}
+
+cudaError_t launch_attn_order(const int32_t* kv_len, int B, int32_t* order, cudaStream_t stream) {
+  attn_order_kernel<<<(B + 255) / 256, 256, B * sizeof(int32_t), stream>>>(kv_len, B, order);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_attn_combine(const AttnParams& p, int n_total, cudaStream_t stream) {

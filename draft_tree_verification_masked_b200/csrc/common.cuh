@@ -221,6 +221,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void* tile) {
   return d;
 }
 
+// Descriptor for a K-major bf16 tile with 64-byte swizzle: rows of 32 elements (64 B), 8-row
+// swizzle atoms 512 B apart.  A thread writing such a tile puts 16-byte chunk c of row r at
+// chunk c ^ ((r >> 1) & 3).
+__device__ __forceinline__ uint64_t smem_desc_sw64(const void* tile) {
+  uint64_t addr = smem_u32(tile);
+  uint64_t d = 0;
+  d |= (addr >> 4) & 0x3FFFull;
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;                  // layout: 64-byte swizzle
+  return d;
+}
+
 // Descriptor for an MN-major bf16 operand written by TMA with 128-byte swizzle: along MN, 64
 // contiguous elements per 128-byte row and further 64-element blocks `mn_block_bytes` apart
 // (leading byte offset); along K, one row per element, 8-row groups 1024 B apart (stride offset).

@@ -19,15 +19,18 @@ struct AttnParams {
   int B, hq, hkv, G, n_max, kv_len_max;
   int64_t cache_slots;
   int mchunks, nsplit, tps;
+  int keys;                 // keys per KV tile (the tree takes ceil(n / keys) tiles at the end)
+  const int32_t* order;     // [B] requests by decreasing KV length (dispatch order), or null
   float scale_log2;
 };
 cudaError_t launch_attn(const CUtensorMap& kc, const CUtensorMap& vc, const CUtensorMap& kt,
                         const CUtensorMap& vt, const AttnParams& p, int nw, int stages,
                         int n_total, cudaStream_t stream);
 cudaError_t launch_attn_combine(const AttnParams& p, int n_total, cudaStream_t stream);
+cudaError_t launch_attn_order(const int32_t* kv_len, int B, int32_t* order, cudaStream_t stream);
 cudaError_t launch_attn_tc(const CUtensorMap& q, const CUtensorMap& kc, const CUtensorMap& vc,
                            const CUtensorMap& kt, const CUtensorMap& vt, const AttnParams& p,
-                           int nb, int stages, int n_total, cudaStream_t stream);
+                           int nb, int n_total, cudaStream_t stream);
 
 struct GemmParams {
   int M, V, K, m_tiles, n_tiles, num_tiles, k_blocks;

@@ -177,3 +177,25 @@ def test_warp_mma_attention_kernel(case, monkeypatch):
                         kv_len=[0, 1, 63, 64, 65, 200], depth=8, depth_min=1, branch=None,
                         width=16, vocab=1000, hidden=256)
     _full_check(wl)
+
+
+@pytest.mark.parametrize("case", ["ragged", "g1", "g8_chain", "conc_like", "two_blocks"])
+def test_attention_32key_tiles(case, monkeypatch):
+    """The 32-key, two-CTAs-per-SM attention shape: two tree tiles for trees over 32 nodes,
+    lane-quarter rotation of small row blocks, ragged lengths."""
+    monkeypatch.setenv("ETREE_ATTN_KEYS", "32")
+    if case == "ragged":
+        wl = W.generate("tiny", B=6, n_nodes=[1, 4, 16, 33, 64, 2],
+                        kv_len=[0, 1, 31, 32, 33, 200], depth=8, depth_min=1, branch=None,
+                        width=16, vocab=1000, hidden=256)
+    elif case == "g1":
+        wl = W.generate("tiny", B=3, hq=8, hkv=8, kv_len=(100, 700), hidden=256, vocab=512)
+    elif case == "g8_chain":
+        wl = W.generate("tiny", B=2, hq=16, hkv=2, n_nodes=[40, 7], depth=39, depth_min=39,
+                        branch=1, kv_len=[95, 1], hidden=256, vocab=512)
+    elif case == "conc_like":
+        wl = W.generate("conc512", B=9, hq=10, hkv=2, kv_len=(30, 300), hidden=256, vocab=512)
+    else:
+        wl = W.generate("tiny", B=2, hq=40, hkv=8, n_nodes=[64, 30], depth=8, depth_min=8,
+                        branch=None, width=16, kv_len=[500, 77], hidden=256, vocab=512)
+    _full_check(wl)
