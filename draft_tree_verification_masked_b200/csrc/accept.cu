@@ -9,8 +9,9 @@
 // arex-research.com, paragraph on the repository's positioning), which the min(1, p/q) test
 // with a residual resample achieves.
 //
-// One CTA per request: its warps reduce the request's rows across vocab tiles, then one warp
-// walks the tree with ballots over the (<= 64) nodes.
+// One warp per node row reduces the row across the LM head's partial summaries; the warp that
+// completes a request's last row then takes the request's acceptance step (a ballot walk over
+// the <= 64 nodes at T = 0, the sequential accept test along the chain at T > 0).
 #include "kernels.cuh"
 #include "philox.cuh"
 
@@ -52,68 +53,50 @@ __device__ __forceinline__ void merge_lse(float& m, float& s, float om, float os
   m = nm;
 }
 
-// ------------------------------------------------------------------------------------ T == 0
-// One warp per node row: merge the row's vocab-tile summaries into its argmax and top1 - top2 gap.
-__global__ void __launch_bounds__(256) row_top2_kernel(AcceptParams p, int32_t* arg_ws) {
-  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (row >= p.n_total) return;
-  const float4* part = p.part + (size_t)row * p.n_tiles;
-  float t1 = -INFINITY, t2 = -INFINITY;
-  int id = -1;
-  int t = lane;
-  for (; t + 96 < p.n_tiles; t += 128) {             // four loads in flight per lane
-    const float4 a = part[t], b = part[t + 32], c = part[t + 64], d = part[t + 96];
-    merge_top2(t1, id, t2, a.x, __float_as_int(a.y), a.z);
-    merge_top2(t1, id, t2, b.x, __float_as_int(b.y), b.z);
-    merge_top2(t1, id, t2, c.x, __float_as_int(c.y), c.z);
-    merge_top2(t1, id, t2, d.x, __float_as_int(d.y), d.z);
-  }
-  for (; t < p.n_tiles; t += 32) {
-    const float4 a = part[t];
-    merge_top2(t1, id, t2, a.x, __float_as_int(a.y), a.z);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float o1 = __shfl_xor_sync(0xffffffffu, t1, off);
-    const int oid = __shfl_xor_sync(0xffffffffu, id, off);
-    const float o2 = __shfl_xor_sync(0xffffffffu, t2, off);
-    merge_top2(t1, id, t2, o1, oid, o2);
-  }
-  if (lane == 0) {
-    arg_ws[row] = id;
-    if (p.node_argmax) p.node_argmax[row] = id;
-    if (p.node_gap) p.node_gap[row] = t1 - t2;
-  }
+// ---------------------------------------------------------------------------- row ownership
+// Node rows are reduced one warp per row across many CTAs; the warp that finishes the last row
+// of a request (a per-request arrival counter, zeroed by the LM-head GEMM that runs first) then
+// takes that request's acceptance step.  Warps past the last row check one request each and
+// answer malformed ones, which no row ever completes.
+
+__device__ __forceinline__ bool request_ok(const AcceptParams& p, int r, int& base, int& n) {
+  base = __ldg(p.cu_nodes + r);
+  const int end = __ldg(p.cu_nodes + r + 1);
+  n = end - base;
+  return base >= 0 && end <= p.n_total && n >= 1 && n <= p.n_max;
 }
 
-// One warp per request: validate the tree, then walk from the root along the lowest-index child
-// that carries argmax(current node); the node where no child matches gives the bonus token.
-__global__ void __launch_bounds__(128) walk_greedy_kernel(AcceptParams p, const int32_t* arg_ws) {
-  __shared__ int am_s[4][64], par_s[4][64], tok_s[4][64], pth_s[4][64];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * 4 + warp;
-  if (r >= p.B) return;
-  const int base = p.cu_nodes[r];
-  const int n = p.cu_nodes[r + 1] - base;
+// The well-formed request that holds node row `row`, or -1.
+__device__ __forceinline__ int row_owner(const AcceptParams& p, int row, int& base, int& n) {
+  int lo = 0, hi = p.B - 1;                      // largest r with cu_nodes[r] <= row
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.cu_nodes + mid) <= row) lo = mid; else hi = mid - 1;
+  }
+  if (!request_ok(p, lo, base, n) || row < base || row >= base + n) return -1;
+  return lo;
+}
+
+// True in every lane of the warp that brings request r's arrivals to n; that warp then sees
+// every other row's results (fence, atomic, fence).
+__device__ __forceinline__ bool last_arrival(int32_t* cnt, int r, int n, int lane) {
+  int last = 0;
+  if (lane == 0) {
+    __threadfence();
+    last = atomicAdd(cnt + r, 1) == n - 1;
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (last) __threadfence();
+  return last != 0;
+}
+
+// ------------------------------------------------------------------------------------ T == 0
+// Greedy walk of one request: from the root, follow the lowest-index child that carries
+// argmax(current node); the node where no child matches gives the bonus token.
+__device__ void walk_greedy(const AcceptParams& p, const int32_t* arg_ws, int r, int base, int n,
+                            int lane, int* am, int* par, int* tok, int* pth) {
   int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
   int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
-  if (n < 1 || n > p.n_max) {
-    if (lane == 0) {
-      report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
-      p.accept_len[r] = 0;
-    }
-    path[lane] = -1;
-    path[lane + 32] = -1;
-    outt[lane] = -1;
-    outt[lane + 32] = -1;
-    if (lane == 0) outt[64] = -1;
-    return;
-  }
-  int* am = am_s[warp];
-  int* par = par_s[warp];
-  int* tok = tok_s[warp];
-  int* pth = pth_s[warp];
   bool ok = true;
   for (int j = lane; j < 64; j += 32) {
     if (j < n) {
@@ -121,7 +104,7 @@ __global__ void __launch_bounds__(128) walk_greedy_kernel(AcceptParams p, const 
       ok = ok && ((j == 0) ? pj == -1 : (pj >= 0 && pj < j));
       par[j] = pj;
       tok[j] = p.tokens[base + j];
-      am[j] = arg_ws[base + j];
+      am[j] = __ldcg(arg_ws + base + j);
     } else {
       par[j] = -2;
       tok[j] = -1;
@@ -155,6 +138,68 @@ __global__ void __launch_bounds__(128) walk_greedy_kernel(AcceptParams p, const 
   if (lane == 0) p.accept_len[r] = a;
 }
 
+// Outputs of a request with no valid tree: nothing accepted, no bonus.
+__device__ void answer_malformed(const AcceptParams& p, int r, int lane) {
+  int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
+  int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
+  if (lane == 0) {
+    report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
+    p.accept_len[r] = 0;
+  }
+  path[lane] = -1;
+  path[lane + 32] = -1;
+  outt[lane] = -1;
+  outt[lane + 32] = -1;
+  if (lane == 0) outt[64] = -1;
+}
+
+// One warp per node row merges the row's (top1, id, top2) summaries into its argmax and
+// top1 - top2 gap; the last row of a request walks it.
+__global__ void __launch_bounds__(256) greedy_accept_kernel(AcceptParams p, int32_t* arg_ws,
+                                                            int32_t* cnt) {
+  __shared__ int am_s[8][64], par_s[8][64], tok_s[8][64], pth_s[8][64];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int item = blockIdx.x * 8 + warp;
+  if (item >= p.n_total + p.B) return;
+  int base, n;
+  if (item >= p.n_total) {
+    const int r = item - p.n_total;
+    if (!request_ok(p, r, base, n)) answer_malformed(p, r, lane);
+    return;
+  }
+  const int row = item;
+  const float4* part = p.part + (size_t)row * p.n_tiles;
+  float t1 = -INFINITY, t2 = -INFINITY;
+  int id = -1;
+  int t = lane;
+  for (; t + 96 < p.n_tiles; t += 128) {             // four loads in flight per lane
+    const float4 a = part[t], b = part[t + 32], c = part[t + 64], d = part[t + 96];
+    merge_top2(t1, id, t2, a.x, __float_as_int(a.y), a.z);
+    merge_top2(t1, id, t2, b.x, __float_as_int(b.y), b.z);
+    merge_top2(t1, id, t2, c.x, __float_as_int(c.y), c.z);
+    merge_top2(t1, id, t2, d.x, __float_as_int(d.y), d.z);
+  }
+  for (; t < p.n_tiles; t += 32) {
+    const float4 a = part[t];
+    merge_top2(t1, id, t2, a.x, __float_as_int(a.y), a.z);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o1 = __shfl_xor_sync(0xffffffffu, t1, off);
+    const int oid = __shfl_xor_sync(0xffffffffu, id, off);
+    const float o2 = __shfl_xor_sync(0xffffffffu, t2, off);
+    merge_top2(t1, id, t2, o1, oid, o2);
+  }
+  if (lane == 0) {
+    arg_ws[row] = id;
+    if (p.node_argmax) p.node_argmax[row] = id;
+    if (p.node_gap) p.node_gap[row] = t1 - t2;
+  }
+  const int r = row_owner(p, row, base, n);
+  if (r < 0 || !last_arrival(cnt, r, n, lane)) return;
+  walk_greedy(p, arg_ws, r, base, n, lane, am_s[warp], par_s[warp], tok_s[warp], pth_s[warp]);
+}
+
 // ------------------------------------------------------------------------------------- T > 0
 // Chain check and the child token of every row (read by the LM-head epilogue).
 __global__ void chain_prep_kernel(AcceptParams p, int32_t* child_tok) {
@@ -180,11 +225,81 @@ __global__ void chain_prep_kernel(AcceptParams p, int32_t* child_tok) {
   }
 }
 
-// One warp per node row: merge the (max, sum) summaries into log2 sum 2^(z log2(e) / T).
-__global__ void __launch_bounds__(256) row_lse_kernel(AcceptParams p) {
-  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (row >= p.n_total) return;
+// The acceptance chain of one request (one warp): node k is kept while U_k q(x_k) < p(x_k),
+// with p from the row's logit of x_k and its log-sum-exp; then the stop row's hidden state is
+// copied out for the second (draw) pass.
+__device__ void accept_chain(const AcceptParams& p, int r, int base, int n, int lane) {
+  int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
+  int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
+  bool chain = true;
+  for (int i = lane; i < n; i += 32) {
+    const int pi = p.parent[base + i];
+    if (i == 0 ? pi != -1 : pi != i - 1) chain = false;
+  }
+  chain = __all_sync(0xffffffffu, chain);
+  int a = 0, rejected = 0;
+  if (!chain) {
+    if (lane == 0) report(p.ws, ETREE_EUNSUPPORTED, DET_NOT_CHAIN);
+  } else if (lane == 0) {
+    for (int k = 1; k < n; ++k) {
+      const int u = k - 1;
+      const int x = p.tokens[base + k];
+      if (x < 0 || x >= p.V) {
+        report(p.ws, ETREE_EDEVICE, DET_BAD_TOKEN);
+        rejected = 1;
+        break;
+      }
+      const float px = exp2f(p.zchild[base + u] * p.k_log2 - __ldcg(p.lse2 + base + u));
+      const float qx = __ldg(p.q_draft + (size_t)(base + u) * p.V + x);
+      float U[8];
+      uniforms8(p.seed, p.step, 0u, (uint32_t)k, (uint32_t)r, 1u, U);
+      if (U[0] * qx < px) {
+        ++a;
+      } else {
+        rejected = 1;
+        break;
+      }
+    }
+  }
+  a = __shfl_sync(0xffffffffu, a, 0);
+  rejected = __shfl_sync(0xffffffffu, rejected, 0);
+  for (int k = lane; k < 64; k += 32) path[k] = (chain && k <= a) ? k : (k == 0 ? 0 : -1);
+  for (int k = lane; k < 65; k += 32) outt[k] = (chain && k < a) ? p.tokens[base + k + 1] : -1;
+  const int src = chain ? base + a : base;
+  if (lane == 0) {
+    p.accept_len[r] = chain ? a : 0;
+    p.stop_row[r] = src;
+    p.stop_node[r] = chain ? a : 0;
+    p.mode[r] = chain ? rejected : 0;
+  }
+  const uint4* hs = reinterpret_cast<const uint4*>(p.hidden + (size_t)src * p.H);
+  uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
+  for (int i = lane; i < p.H / 8; i += 32) hd[i] = hs[i];
+}
+
+// One warp per node row merges the row's (max, sum) summaries into log2 sum 2^(z log2(e) / T);
+// the last row of a request runs its acceptance chain.  Malformed requests accept nothing and
+// draw from row 0 so that the second pass reads defined data.
+__global__ void __launch_bounds__(256) chain_accept_kernel(AcceptParams p, int32_t* cnt) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int item = blockIdx.x * 8 + warp;
+  if (item >= p.n_total + p.B) return;
+  int base, n;
+  if (item >= p.n_total) {
+    const int r = item - p.n_total;
+    if (request_ok(p, r, base, n)) return;
+    answer_malformed(p, r, lane);
+    if (lane == 0) {
+      p.stop_row[r] = 0;
+      p.stop_node[r] = 0;
+      p.mode[r] = 0;
+    }
+    const uint4* hs = reinterpret_cast<const uint4*>(p.hidden);
+    uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
+    for (int i = lane; i < p.H / 8; i += 32) hd[i] = hs[i];
+    return;
+  }
+  const int row = item;
   const float4* part = p.part + (size_t)row * p.n_tiles;
   float m = -INFINITY, s = 0.f;
   int t = lane;
@@ -206,73 +321,9 @@ __global__ void __launch_bounds__(256) row_lse_kernel(AcceptParams p) {
     merge_lse(m, s, om, os);
   }
   if (lane == 0) p.lse2[row] = m + log2f(s);
-}
-
-__global__ void __launch_bounds__(128) accept_chain_kernel(AcceptParams p) {
-  __shared__ int info_s[2];
-  const int r = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int base = p.cu_nodes[r];
-  const int n = p.cu_nodes[r + 1] - base;
-  int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
-  int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
-  const bool n_ok = n >= 1 && n <= p.n_max;
-  const float* lse_s = p.lse2 + base;
-  __syncthreads();
-  if (warp == 0) {
-    int a = 0, rejected = 0;
-    bool chain = n_ok;
-    if (n_ok) {
-      for (int i = lane; i < n; i += 32) {
-        const int pi = p.parent[base + i];
-        if (i == 0 ? pi != -1 : pi != i - 1) chain = false;
-      }
-      chain = __all_sync(0xffffffffu, chain);
-    }
-    if (!n_ok) {
-      if (lane == 0) report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
-    } else if (!chain) {
-      if (lane == 0) report(p.ws, ETREE_EUNSUPPORTED, DET_NOT_CHAIN);
-    } else if (lane == 0) {
-      for (int k = 1; k < n; ++k) {
-        const int u = k - 1;
-        const int x = p.tokens[base + k];
-        if (x < 0 || x >= p.V) {
-          report(p.ws, ETREE_EDEVICE, DET_BAD_TOKEN);
-          rejected = 1;
-          break;
-        }
-        const float px = exp2f(p.zchild[base + u] * p.k_log2 - lse_s[u]);
-        const float qx = __ldg(p.q_draft + (size_t)(base + u) * p.V + x);
-        float U[8];
-        uniforms8(p.seed, p.step, 0u, (uint32_t)k, (uint32_t)r, 1u, U);
-        if (U[0] * qx < px) {
-          ++a;
-        } else {
-          rejected = 1;
-          break;
-        }
-      }
-    }
-    a = __shfl_sync(0xffffffffu, a, 0);
-    rejected = __shfl_sync(0xffffffffu, rejected, 0);
-    const bool good = n_ok && chain;
-    for (int k = lane; k < 64; k += 32) path[k] = (good && k <= a) ? k : (k == 0 ? 0 : -1);
-    for (int k = lane; k < 65; k += 32) outt[k] = (good && k < a) ? p.tokens[base + k + 1] : -1;
-    if (lane == 0) {
-      p.accept_len[r] = good ? a : 0;
-      p.stop_row[r] = good ? base + a : (n_ok ? base : 0);
-      p.stop_node[r] = good ? a : 0;
-      p.mode[r] = good ? rejected : 0;
-      info_s[0] = good ? base + a : (n_ok ? base : 0);
-    }
-  }
-  __syncthreads();
-  // gather the stop row's hidden state for the second (race) pass
-  const int src = info_s[0];
-  const uint4* hs = reinterpret_cast<const uint4*>(p.hidden + (size_t)src * p.H);
-  uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
-  for (int i = threadIdx.x; i < p.H / 8; i += blockDim.x) hd[i] = hs[i];
+  const int r = row_owner(p, row, base, n);
+  if (r < 0 || !last_arrival(cnt, r, n, lane)) return;
+  accept_chain(p, r, base, n, lane);
 }
 
 // The first level of the two-level draw, per request: the exponential race among the 128-id
@@ -318,9 +369,9 @@ __global__ void bonus_kernel(AcceptParams p) {
   }
 }
 
-cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, cudaStream_t s) {
-  row_top2_kernel<<<(p.n_total + 7) / 8, 256, 0, s>>>(p, arg_ws);
-  walk_greedy_kernel<<<(p.B + 3) / 4, 128, 0, s>>>(p, arg_ws);
+cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, int32_t* cnt,
+                                 cudaStream_t s) {
+  greedy_accept_kernel<<<(p.n_total + p.B + 7) / 8, 256, 0, s>>>(p, arg_ws, cnt);
   return cudaGetLastError();
 }
 
@@ -329,9 +380,8 @@ cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStr
   return cudaGetLastError();
 }
 
-cudaError_t launch_accept_chain(const AcceptParams& p, cudaStream_t s) {
-  row_lse_kernel<<<(p.n_total + 7) / 8, 256, 0, s>>>(p);
-  accept_chain_kernel<<<p.B, 128, 0, s>>>(p);
+cudaError_t launch_accept_chain(const AcceptParams& p, int32_t* cnt, cudaStream_t s) {
+  chain_accept_kernel<<<(p.n_total + p.B + 7) / 8, 256, 0, s>>>(p, cnt);
   return cudaGetLastError();
 }
 

@@ -107,7 +107,7 @@ static AttnPlan plan_attn(const etree_batch* b, int hq, int hkv) {
 // ------------------------------------------------------------------------------ workspace map
 struct WsLayout {
   size_t order, o_part, ml_part, part, child_tok, zchild, lse2, stop_row, stop_node, mode, hid2,
-      part2;
+      part2, cnt;
   size_t total;
   int n_tiles;
 };
@@ -141,6 +141,7 @@ static WsLayout layout(const etree_batch* b, int hq, int hkv, int hidden_dim, in
   w.mode = take(B * sizeof(int32_t));
   w.hid2 = take(B * (size_t)std::max(0, hidden_dim) * 2);
   w.part2 = take(B * (size_t)w.n_tiles * sizeof(float4));
+  w.cnt = take(B * sizeof(int32_t));
   w.total = off;
   return w;
 }
@@ -457,15 +458,17 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
 
   const int sms = sm_count();
   const int bn = lmhead_pick_bn(b->n_total, vocab, sms);
+  // up to 64 rows: M=64 MMAs with half-height hidden tiles (the W stream is the cost)
+  const int bm = (b->n_total <= 64 && env_int("ETREE_BM", 0) != 128) ? 64 : 128;
   CUtensorMap ta, tb;
-  if ((st = get_map(hidden, 2, hidden_dim, b->n_total, 1, 64, 128, 1, &ta))) return st;
+  if ((st = get_map(hidden, 2, hidden_dim, b->n_total, 1, 64, bm, 1, &ta))) return st;
   if ((st = get_map(w_lm, 2, hidden_dim, vocab, 1, 64, bn, 1, &tb))) return st;
 
   GemmParams g{};
   g.M = b->n_total;
   g.V = vocab;
   g.K = hidden_dim;
-  g.m_tiles = (b->n_total + 127) / 128;
+  g.m_tiles = (b->n_total + bm - 1) / bm;
   g.n_tiles = (vocab + bn - 1) / bn;
   g.num_tiles = g.m_tiles * g.n_tiles;
   g.k_blocks = hidden_dim / 64;
@@ -481,13 +484,19 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
   g.q_draft = q_draft;
   g.seed = seed;
   g.step = step;
+  const int grid = std::min(g.num_tiles, sms);
+  g.per_cta = g.m_tiles == 1 && env_int("ETREE_PER_TILE", 0) == 0;
+  g.n_parts = g.per_cta ? grid : g.n_tiles;
+  int32_t* cnt = at<int32_t>(workspace, w.cnt);
+  g.cnt = cnt;
+  g.cnt_n = b->B;
 
   AcceptParams a{};
   a.B = b->B;
   a.n_total = b->n_total;
   a.n_max = b->n_max;
   a.V = vocab;
-  a.n_tiles = 2 * g.n_tiles;
+  a.n_tiles = 2 * g.n_parts;
   a.cu_nodes = b->cu_nodes;
   a.parent = b->parent;
   a.tokens = b->tokens;
@@ -514,26 +523,30 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
 
   cudaError_t e;
   if (temperature == 0.f) {
-    e = launch_lmhead(0, bn, ta, tb, g, std::min(g.num_tiles, sms), s);
-    if (e == cudaSuccess) e = launch_accept_greedy(a, at<int32_t>(workspace, w.child_tok), s);
+    e = launch_lmhead(0, bn, bm, ta, tb, g, grid, s);
+    if (e == cudaSuccess) e = launch_accept_greedy(a, at<int32_t>(workspace, w.child_tok), cnt, s);
     return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T=0)");
   }
   e = launch_chain_prep(a, at<int32_t>(workspace, w.child_tok), s);
-  if (e == cudaSuccess) e = launch_lmhead(1, bn, ta, tb, g, std::min(g.num_tiles, sms), s);
-  if (e == cudaSuccess) e = launch_accept_chain(a, s);
+  if (e == cudaSuccess) e = launch_lmhead(1, bn, bm, ta, tb, g, grid, s);
+  if (e == cudaSuccess) e = launch_accept_chain(a, cnt, s);
   if (e != cudaSuccess) return cuda_fail(e, "etree_lmhead_accept (T>0, pass 1)");
   const int bn2 = 256;                       // the draw's 128-id blocks pair up in a tile
+  const int bm2 = (b->B <= 64 && env_int("ETREE_BM", 0) != 128) ? 64 : 128;
   CUtensorMap th, tb2;
-  if ((st = get_map(a.hid2, 2, hidden_dim, b->B, 1, 64, 128, 1, &th))) return st;
+  if ((st = get_map(a.hid2, 2, hidden_dim, b->B, 1, 64, bm2, 1, &th))) return st;
   if ((st = get_map(w_lm, 2, hidden_dim, vocab, 1, 64, bn2, 1, &tb2))) return st;
   GemmParams g2 = g;
   g2.M = b->B;
-  g2.m_tiles = (b->B + 127) / 128;
+  g2.m_tiles = (b->B + bm2 - 1) / bm2;
   g2.n_tiles = (vocab + bn2 - 1) / bn2;
   g2.num_tiles = g2.m_tiles * g2.n_tiles;
   g2.part = at<float4>(workspace, w.part2);
+  g2.per_cta = 0;                            // the draw needs every 128-id block's summary
+  g2.n_parts = g2.n_tiles;
+  g2.cnt = nullptr;
   a.n_tiles2 = 2 * g2.n_tiles;
-  e = launch_lmhead(2, bn2, th, tb2, g2, std::min(g2.num_tiles, sms), s);
+  e = launch_lmhead(2, bn2, bm2, th, tb2, g2, std::min(g2.num_tiles, sms), s);
   if (e == cudaSuccess) e = launch_bonus(a, s);
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T>0, pass 2)");
 }

@@ -34,6 +34,12 @@ cudaError_t launch_attn_tc(const CUtensorMap& q, const CUtensorMap& kc, const CU
 
 struct GemmParams {
   int M, V, K, m_tiles, n_tiles, num_tiles, k_blocks;
+  // per_cta = 1 (one row tile only): each CTA folds all its vocab tiles into one summary per
+  // row and half, at slot blockIdx.x; else one summary per vocab tile, at slot nt.  n_parts is
+  // the number of slots per row.
+  int per_cta, n_parts;
+  int32_t* cnt;                     // if set, CTA 0 zeroes cnt[0 .. cnt_n) (acceptance counters)
+  int cnt_n;
   WsHeader* ws;
   float4* part;
   const int32_t* child_tok;
@@ -47,7 +53,7 @@ struct GemmParams {
   uint64_t seed, step;
 };
 int lmhead_pick_bn(int M, int V, int grid);
-cudaError_t launch_lmhead(int epi, int bn, const CUtensorMap& ta, const CUtensorMap& tb,
+cudaError_t launch_lmhead(int epi, int bn, int bm, const CUtensorMap& ta, const CUtensorMap& tb,
                           const GemmParams& p, int grid, cudaStream_t stream);
 
 struct AcceptParams {
@@ -75,9 +81,10 @@ struct AcceptParams {
   int H;
   const float4* part2;
 };
-cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, cudaStream_t s);
+cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, int32_t* cnt,
+                                 cudaStream_t s);
 cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStream_t s);
-cudaError_t launch_accept_chain(const AcceptParams& p, cudaStream_t s);
+cudaError_t launch_accept_chain(const AcceptParams& p, int32_t* cnt, cudaStream_t s);
 cudaError_t launch_bonus(const AcceptParams& p, cudaStream_t s);
 
 struct CompactParams {

@@ -27,8 +27,12 @@
 
 namespace etree {
 
-constexpr int kBM = 128, kBK = 64, kGStages = 4;
-constexpr int kABytes = kBM * kBK * 2;
+constexpr int kBK = 64;
+
+// Stage count of the smem ring for a (BM, BN) tile: as many as fit in ~210 KB, at most 6.
+__host__ __device__ constexpr int gemm_stages(int bm, int bn) {
+  return (210 * 1024) / ((bm + bn) * kBK * 2) < 6 ? (210 * 1024) / ((bm + bn) * kBK * 2) : 6;
+}
 enum Epi { EPI_ARGMAX = 0, EPI_LSE = 1, EPI_RACE = 2 };
 
 // Per-row running state of the epilogue over one vocab tile.
@@ -104,11 +108,14 @@ __device__ __forceinline__ void load_q32(const GemmParams& p, const float* qrow,
 constexpr int kEpiWarps = 8;                 // two warps per TMEM lane quarter
 constexpr int kGemmThreads = 32 * (2 + kEpiWarps);
 
-template <int EPI, int BN>
+template <int EPI, int BN, int BM>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    GemmParams p) {
+  constexpr int kABytes = BM * kBK * 2;
   constexpr int kBBytes = BN * kBK * 2;
+  constexpr int kGStages = gemm_stages(BM, BN);
+  constexpr int kBM = BM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -121,6 +128,8 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (p.cnt && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < p.cnt_n; i += blockDim.x) p.cnt[i] = 0;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kGStages; ++i) {
       mbar_init(&full[i], 1);
@@ -167,7 +176,7 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   } else if (warp == 1) {
     // ------------------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, BN);
+      const uint32_t idesc = idesc_bf16_f32(BM, BN);
       int it = 0, ai = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++ai) {
@@ -208,6 +217,7 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     constexpr int kTailHalf = (kChunks & 1) ? 1 : 0;   // the 16-column tail goes to the half
                                                         // with fewer full chunks
     int ai = 0;
+    EpiRow st;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++ai) {
       const int buf = ai & 1;
       const uint32_t aph = (ai >> 1) & 1;
@@ -217,12 +227,14 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       }
       tc_fence_after();
       const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
-      const int row = wq * 32 + lane;
+      // M=128: row r sits in TMEM lane r.  M=64: rows 16q .. 16q+15 sit in the first 16 lanes of
+      // lane quarter q, the other 16 lanes of the quarter hold no output.
+      const int row = BM == 128 ? wq * 32 + lane : wq * 16 + (lane & 15);
       const int grow = mt * kBM + row;
-      const bool active = grow < p.M;
+      const bool active = (BM == 128 || lane < 16) && grow < p.M;
       const uint32_t tbase = tmem + ((uint32_t)(wq * 32) << 16) + buf * BN;
 
-      EpiRow st;
+      if (!p.per_cta) st = EpiRow();
       if (EPI == EPI_LSE && active) st.ct = p.child_tok[grow];
       if (EPI == EPI_RACE && active) {
         const int g = p.stop_row[grow];
@@ -317,7 +329,9 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[buf]);
-      if (active) {
+      // per_cta: the row state runs on over this CTA's tiles (increasing ids, so first-seen
+      // still means lowest id) and is written once, after the CTA's last tile.
+      if (active && (!p.per_cta || tile + (int)gridDim.x >= p.num_tiles)) {
         float4 out;
         if (EPI == EPI_ARGMAX)
           out = make_float4(st.r0, __int_as_float(st.r1), st.r2, 0.f);
@@ -325,7 +339,7 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           out = make_float4(st.r0, st.r1f, 0.f, 0.f);
         else
           out = make_float4(st.r0, __int_as_float(st.r1), st.r2, __int_as_float(st.r3));
-        p.part[(size_t)grow * p.n_tiles * 2 + nt * 2 + half] = out;
+        p.part[(size_t)grow * p.n_parts * 2 + (p.per_cta ? (int)blockIdx.x : nt) * 2 + half] = out;
         if (EPI == EPI_LSE && st.found) p.zchild[grow] = st.zc;
       }
     }
@@ -349,7 +363,7 @@ int lmhead_pick_bn(int M, int V, int grid) {
   // With several row tiles the GEMM is tensor-bound and the widest tile is the most efficient.
   // With one row tile it streams W once: time ~ (rounds of tiles per CTA) x (tile width + a
   // fixed per-tile cost of ~48 columns), so pick the width that balances the last round.
-  const long m_tiles = (M + kBM - 1) / kBM;
+  const long m_tiles = (M + 127) / 128;
   if (m_tiles >= 2) return 256;
   int best = 256;
   long best_cost = -1;
@@ -365,43 +379,50 @@ int lmhead_pick_bn(int M, int V, int grid) {
   return best;
 }
 
-size_t lmhead_smem_bytes(int bn) {
-  return (size_t)kGStages * (kABytes + bn * kBK * 2) + 1024 + (2 * kGStages + 4) * 8 + 16;
+template <int BM>
+static size_t lmhead_smem_bytes(int bn) {
+  return (size_t)gemm_stages(BM, bn) * (BM + bn) * kBK * 2 + 1024 + (2 * 6 + 4) * 8 + 16;
 }
 
-template <int EPI, int BN>
+template <int EPI, int BN, int BM>
 static cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                              int grid, cudaStream_t stream) {
-  const size_t smem = lmhead_smem_bytes(BN);
-  auto k = lmhead_gemm_kernel<EPI, BN>;
+  const size_t smem = lmhead_smem_bytes<BM>(BN);
+  auto k = lmhead_gemm_kernel<EPI, BN, BM>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<grid, kGemmThreads, smem, stream>>>(ta, tb, p);
   return cudaGetLastError();
 }
 
-template <int EPI>
+template <int EPI, int BM>
 static cudaError_t launch_epi(int bn, const CUtensorMap& ta, const CUtensorMap& tb,
                               const GemmParams& p, int grid, cudaStream_t s) {
   switch (bn) {
-    case 256: return launch_bn<EPI, 256>(ta, tb, p, grid, s);
-    case 224: return launch_bn<EPI, 224>(ta, tb, p, grid, s);
-    case 208: return launch_bn<EPI, 208>(ta, tb, p, grid, s);
-    case 192: return launch_bn<EPI, 192>(ta, tb, p, grid, s);
-    case 176: return launch_bn<EPI, 176>(ta, tb, p, grid, s);
-    case 160: return launch_bn<EPI, 160>(ta, tb, p, grid, s);
-    case 144: return launch_bn<EPI, 144>(ta, tb, p, grid, s);
-    case 128: return launch_bn<EPI, 128>(ta, tb, p, grid, s);
+    case 256: return launch_bn<EPI, 256, BM>(ta, tb, p, grid, s);
+    case 224: return launch_bn<EPI, 224, BM>(ta, tb, p, grid, s);
+    case 208: return launch_bn<EPI, 208, BM>(ta, tb, p, grid, s);
+    case 192: return launch_bn<EPI, 192, BM>(ta, tb, p, grid, s);
+    case 176: return launch_bn<EPI, 176, BM>(ta, tb, p, grid, s);
+    case 160: return launch_bn<EPI, 160, BM>(ta, tb, p, grid, s);
+    case 144: return launch_bn<EPI, 144, BM>(ta, tb, p, grid, s);
+    case 128: return launch_bn<EPI, 128, BM>(ta, tb, p, grid, s);
   }
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_lmhead(int epi, int bn, const CUtensorMap& ta, const CUtensorMap& tb,
+cudaError_t launch_lmhead(int epi, int bn, int bm, const CUtensorMap& ta, const CUtensorMap& tb,
                           const GemmParams& p, int grid, cudaStream_t stream) {
-  if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX>(bn, ta, tb, p, grid, stream);
-  if (epi == EPI_LSE) return launch_epi<EPI_LSE>(bn, ta, tb, p, grid, stream);
+  if (bm == 64) {
+    if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX, 64>(bn, ta, tb, p, grid, stream);
+    if (epi == EPI_LSE) return launch_epi<EPI_LSE, 64>(bn, ta, tb, p, grid, stream);
+    if (bn != 256) return cudaErrorInvalidValue;
+    return launch_bn<EPI_RACE, 256, 64>(ta, tb, p, grid, stream);
+  }
+  if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX, 128>(bn, ta, tb, p, grid, stream);
+  if (epi == EPI_LSE) return launch_epi<EPI_LSE, 128>(bn, ta, tb, p, grid, stream);
   if (bn != 256) return cudaErrorInvalidValue;
-  return launch_bn<EPI_RACE, 256>(ta, tb, p, grid, stream);
+  return launch_bn<EPI_RACE, 256, 128>(ta, tb, p, grid, stream);
 }
 
 }  // namespace etree

@@ -33,6 +33,27 @@ def test_malformed_parent_sets_device_status():
     _still_works()
 
 
+@pytest.mark.parametrize("T", [0.0, 1.0])
+def test_malformed_node_counts_answer_every_request(T):
+    """A request with no nodes and one with more than n_max: both report bad node counts and
+    accept nothing, with no bonus token, whichever acceptance rule runs."""
+    wl = W.generate("tiny", B=3, n_nodes=[5, 9, 6], depth=63, depth_min=63, branch=1,
+                    kv_len=[100, 300, 50], hidden=256, vocab=512)
+    if T > 0:
+        wl.temperature = T
+        wl.q_draft = torch.full((wl.n_total, wl.vocab), 1.0 / wl.vocab)
+    dev = DeviceStep(wl)
+    dev.accept_len.fill_(7)
+    dev.cu_nodes[1] = 0                               # request 0: no nodes; request 1: 14 > n_max
+    dev.lmhead()
+    assert dev.status() == (EDEVICE, 2)
+    res = dev.results()
+    assert list(res["accept_len"][:2]) == [0, 0]
+    assert (res["out_tokens"][:2] == -1).all()
+    assert int(res["accept_len"][2]) != 7             # the well-formed request still ran
+    _still_works()
+
+
 def test_kv_len_above_declared_bound():
     wl, dev = _dev()
     dev.kv_len[0] = wl.kv_len_max + 1

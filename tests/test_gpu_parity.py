@@ -199,3 +199,21 @@ def test_attention_32key_tiles(case, monkeypatch):
         wl = W.generate("tiny", B=2, hq=40, hkv=8, n_nodes=[64, 30], depth=8, depth_min=8,
                         branch=None, width=16, kv_len=[500, 77], hidden=256, vocab=512)
     _full_check(wl)
+
+
+@pytest.mark.parametrize("bm", ["auto", "128", "per_tile"])
+@pytest.mark.parametrize("T", [0.0, 1.0])
+def test_lmhead_row_tile_heights(bm, T, monkeypatch):
+    """Up to 64 rows the LM head runs M=64 MMAs (rows 16q..16q+15 in the first half of TMEM
+    lane quarter q) and folds each CTA's vocab tiles into one summary per row; the 128-row tile
+    and per-tile summaries must give the same results."""
+    if bm == "128":
+        monkeypatch.setenv("ETREE_BM", bm)
+    elif bm == "per_tile":
+        monkeypatch.setenv("ETREE_PER_TILE", "1")
+    shape = dict(depth=6, depth_min=4, branch=None, width=16) if T == 0.0 else \
+        dict(depth=63, depth_min=63, branch=1)            # sampling verifies chains
+    wl = W.generate("tiny", B=4, n_nodes=[20, 1, 31, 12], kv_len=(50, 400), hidden=512,
+                    vocab=8192 + 77, temperature=T, **shape)
+    assert wl.n_total == 64
+    _full_check(wl)
