@@ -35,6 +35,7 @@ constexpr float kLazy = 8.0f;               // rescale O only when the max grows
 struct TcSmem {
   // barriers and small arrays, placed after the 1024-aligned tile area
   uint64_t kv_full[4], kv_empty[4], q_full, s_full[2], s_free[2], p_full[2], p_free[2];
+  uint64_t drain;                           // the MMA issuer's last commit, waited on at exit
   uint64_t anc[64];
   int32_t par[64];
   float xmax[2][2][128];                    // row-max exchange: [tile parity][key half][row]
@@ -107,6 +108,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(&sh->kv_empty[i], 1);
     }
     mbar_init(&sh->q_full, 1);
+    mbar_init(&sh->drain, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->s_full[b], 1);
       mbar_init(&sh->s_free[b], SW);
@@ -166,6 +168,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_arrive_expect_tx(&sh->q_full, 2 * qrows * 128);
       tma_load_3d(sQ + rot * 128, &tm_q, &sh->q_full, 0, kvh * G, base + node0);
       tma_load_3d(sQ + 16384 + rot * 128, &tm_q, &sh->q_full, 64, kvh * G, base + node0);
+      int issued = 0;
       for (int j = 0; j < T; ++j) {
         const int t = t0 + j;
         const int st = j % STAGES;
@@ -189,7 +192,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tma_load_3d(dst + 2 * Sh::kBox, &tm_vt, &sh->kv_full[st], 0, kvh, node);
           tma_load_3d(dst + 3 * Sh::kBox, &tm_vt, &sh->kv_full[st], 64, kvh, node);
         }
+        issued = j + 1;
       }
+      // Before the CTA may exit, every copy into shared memory has landed: the last STAGES
+      // loads (earlier ones were consumed, which implies landed) and Q.  Bounded, like all waits.
+      bool drained = mbar_wait(&sh->q_full, 0);
+      for (int j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j)
+        drained = mbar_wait(&sh->kv_full[j % STAGES], (j / STAGES) & 1) && drained;
+      if (!drained) report(p.ws, ETREE_ETIMEOUT, DET_WAIT_ATTN);
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------------------- MMA issuer
@@ -230,6 +240,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (j >= 1 && !pv(j - 1)) { ok = false; break; }
       }
       if (ok && !pv(T - 1)) ok = false;
+      // every MMA issued above completes before TMEM is released
+      tc_commit(&sh->drain);
+      if (!mbar_wait(&sh->drain, 0)) ok = false;
       if (!ok) report(p.ws, ETREE_ETIMEOUT, DET_WAIT_ATTN);
     }
   } else {

@@ -125,7 +125,8 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   uint64_t* empty = full + kGStages;
   uint64_t* accf = empty + kGStages;
   uint64_t* acce = accf + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  uint64_t* drain = acce + 2;                // the MMA issuer's last commit, waited on at exit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (p.cnt && blockIdx.x == 0)
@@ -139,6 +140,7 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       mbar_init(&accf[b], 1);
       mbar_init(&acce[b], kEpiWarps);
     }
+    mbar_init(drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -172,6 +174,12 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           tma_load_2d(sB + st * kBBytes, &tm_b, &full[st], kb * kBK, nt * BN);
         }
       }
+      // Before the CTA may exit, the last kGStages loads have landed (earlier ones were
+      // consumed, which implies landed).  Bounded, like every wait here.
+      bool drained = true;
+      for (int j = it > kGStages ? it - kGStages : 0; j < it; ++j)
+        drained = mbar_wait(&full[j % kGStages], (j / kGStages) & 1) && drained;
+      if (!drained) report(p.ws, ETREE_ETIMEOUT, DET_WAIT_GEMM);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------------- MMA issuer
@@ -206,6 +214,9 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         }
         tc_commit(&accf[buf]);
       }
+      // every MMA issued above completes before TMEM is released
+      tc_commit(drain);
+      if (!mbar_wait(drain, 0)) report(p.ws, ETREE_ETIMEOUT, DET_WAIT_GEMM);
     }
   } else {
     // ------------------------------------------------------------------------ epilogue warps
@@ -381,7 +392,7 @@ int lmhead_pick_bn(int M, int V, int grid) {
 
 template <int BM>
 static size_t lmhead_smem_bytes(int bn) {
-  return (size_t)gemm_stages(BM, bn) * (BM + bn) * kBK * 2 + 1024 + (2 * 6 + 4) * 8 + 16;
+  return (size_t)gemm_stages(BM, bn) * (BM + bn) * kBK * 2 + 1024 + (2 * 6 + 5) * 8 + 16;
 }
 
 template <int EPI, int BN, int BM>
