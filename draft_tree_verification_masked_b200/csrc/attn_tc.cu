@@ -15,13 +15,14 @@
 // MMAs; the softmax warps own one query row per thread (= one TMEM lane; with 64-key tiles two
 // warps share a row, 32 keys each, and exchange row maxima): they read S from TMEM, apply
 // the key mask (cache length, or the row's ancestor bitmask on the tree tiles), run the online
-// softmax in log2 units, and write P (bf16, swizzled) to shared memory for the PV product.
-// S and P are double-buffered so QK^T of tile j+1 and PV of tile j overlap the softmax.  O is
-// rescaled lazily: only when a row's running maximum grows by more than 2^8 does the softmax
+// softmax in log2 units, and write P (bf16) back into their own TMEM lane, where the PV product
+// takes it as its A operand; shared memory holds only Q and the K/V ring.  S and P are
+// double-buffered so QK^T of tile j+1 and PV of tile j overlap the softmax.  O is rescaled
+// lazily: only when a row's running maximum grows by more than 2^8 does the softmax
 // read-modify-write O in TMEM, so P stays below 256 and the usual case has no O traffic.
 //
-// Two shapes are built.  KEYS = 64 with a 4-deep ring runs one CTA per SM (for few, long
-// work items).  KEYS = 32 with a 3-deep ring fits two CTAs per SM, which overlaps one CTA's
+// Two shapes are built.  KEYS = 64 with a 5-deep ring runs one CTA per SM (for few, long
+// work items).  KEYS = 32 with a 4-deep ring fits two CTAs per SM, which overlaps one CTA's
 // start-up and tail with the other's streaming; its Q rows are rotated into a different TMEM
 // lane quarter per CTA so that co-resident CTAs run their softmax on different SM partitions.
 #include "kernels.cuh"
@@ -34,7 +35,7 @@ constexpr float kLazy = 8.0f;               // rescale O only when the max grows
 
 struct TcSmem {
   // barriers and small arrays, placed after the 1024-aligned tile area
-  uint64_t kv_full[4], kv_empty[4], q_full, s_full[2], s_free[2], p_full[2], p_free[2];
+  uint64_t kv_full[6], kv_empty[6], q_full, s_full[2], s_free[2], p_full[2], p_free[2];
   uint64_t drain;                           // the MMA issuer's last commit, waited on at exit
   uint64_t anc[64];
   int32_t par[64];
@@ -48,8 +49,10 @@ template <int KEYS>
 struct TcShape {
   static constexpr int kBox = KEYS * 128;   // one [KEYS keys][64 dims] bf16 box
   static constexpr int kKV = 4 * kBox;      // K lo/hi + V lo/hi
-  static constexpr int kPRow = KEYS * 2;    // bytes per P row
-  static constexpr int kPBytes = 128 * kPRow;
+  // TMEM columns: S double buffer at [0, 2 KEYS), O at [128, 256), then the P double buffer
+  // (bf16, KEYS / 2 columns each) at kPCol; the 64-key shape allocates 512 columns.
+  static constexpr int kPCol = KEYS == 64 ? 256 : 64;
+  static constexpr int kTmemCols = KEYS == 64 ? 512 : 256;
 };
 }  // namespace
 
@@ -64,8 +67,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;                                   // 32 KB
   uint8_t* sKV = smem + kQBytes;                        // STAGES x kKV
-  uint8_t* sP = sKV + STAGES * Sh::kKV;                 // 2 x kPBytes (double buffer)
-  TcSmem* sh = reinterpret_cast<TcSmem*>(sP + 2 * Sh::kPBytes);
+  TcSmem* sh = reinterpret_cast<TcSmem*>(sKV + STAGES * Sh::kKV);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_req = p.hkv * p.mchunks;
@@ -123,7 +125,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sh->tmem, 256);
+    tmem_alloc(&sh->tmem, Sh::kTmemCols);
     tmem_relinquish();
   }
   if (has_tree) {
@@ -213,13 +215,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int pb = jj & 1;
         if (!mbar_wait(&sh->p_full[pb], (jj >> 1) & 1)) return false;
         tc_fence_after();
-        const uint8_t* pbuf = sP + pb * Sh::kPBytes;
-        const uint64_t dp = KEYS == 64 ? smem_desc_sw128(pbuf) : smem_desc_sw64(pbuf);
+        // A = P from TMEM (16 keys = 8 columns per MMA), B = V from shared memory
+        const uint32_t pa = tmem + Sh::kPCol + pb * (KEYS / 2);
         const uint8_t* v0 = sKV + (jj % STAGES) * Sh::kKV + 2 * Sh::kBox;
 #pragma unroll
         for (int k = 0; k < KEYS / 16; ++k)
-          tc_mma_bf16(tmem + 128, dp + 2 * k, smem_desc_sw128_mn(v0 + k * 2048, Sh::kBox), idO,
-                      (jj > 0 || k > 0) ? 1u : 0u);
+          tc_mma_bf16_ts(tmem + 128, pa + 8 * k, smem_desc_sw128_mn(v0 + k * 2048, Sh::kBox), idO,
+                         (jj > 0 || k > 0) ? 1u : 0u);
         tc_commit(&sh->p_free[pb]);
         tc_commit(&sh->kv_empty[jj % STAGES]);
         return true;
@@ -285,66 +287,80 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->s_free[sb]);
 
-      // keep-mask of this thread's keys: the cache positions below kv_len, or on a tree tile
-      // the row's ancestor bits for the tile's nodes
-      uint32_t kw[CW / 32];
+      // Key mask.  Whole cache tiles below kv_len keep every key (the common case, tested once
+      // per tile for the CTA); the last cache tile masks by kv_len and tree tiles by the row's
+      // ancestor bits.  Scores stay raw here: the scale (> 0) is folded into the exponent.
       const int k0 = kh * CW;                           // first key of this thread in the tile
-      if (!valid) {
+      const bool full_tile = t < nt_cache && L - t * KEYS >= KEYS;
+      if (!full_tile) {
+        uint32_t kw[CW / 32];
+        if (!valid) {
 #pragma unroll
-        for (int w = 0; w < CW / 32; ++w) kw[w] = 0u;
-      } else if (t >= nt_cache) {
-        const int sh0 = (t - nt_cache) * KEYS + k0;
+          for (int w = 0; w < CW / 32; ++w) kw[w] = 0u;
+        } else if (t >= nt_cache) {
+          const int sh0 = (t - nt_cache) * KEYS + k0;
 #pragma unroll
-        for (int w = 0; w < CW / 32; ++w) kw[w] = static_cast<uint32_t>(anc >> (sh0 + 32 * w));
-      } else {
-        const int lim = L - t * KEYS - k0;
+          for (int w = 0; w < CW / 32; ++w) kw[w] = static_cast<uint32_t>(anc >> (sh0 + 32 * w));
+        } else {
+          const int lim = L - t * KEYS - k0;
 #pragma unroll
-        for (int w = 0; w < CW / 32; ++w) {
-          const int lw = lim - 32 * w;
-          kw[w] = lw >= 32 ? 0xffffffffu : (lw > 0 ? ((1u << lw) - 1u) : 0u);
+          for (int w = 0; w < CW / 32; ++w) {
+            const int lw = lim - 32 * w;
+            kw[w] = lw >= 32 ? 0xffffffffu : (lw > 0 ? ((1u << lw) - 1u) : 0u);
+          }
         }
+#pragma unroll
+        for (int c = 0; c < CW; ++c)
+          if (!((kw[c >> 5] >> (c & 31)) & 1u)) sc[c] = -INFINITY;
       }
-      const float sl = p.scale_log2;
-      float t0m = -INFINITY, t1m = -INFINITY, t2m = -INFINITY, t3m = -INFINITY;
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
       for (int c = 0; c < CW; c += 4) {
-        const uint32_t w = kw[c >> 5];
-        const int b0 = c & 31;
-        const float v0 = ((w >> b0) & 1u) ? sc[c] * sl : -INFINITY;
-        const float v1 = ((w >> (b0 + 1)) & 1u) ? sc[c + 1] * sl : -INFINITY;
-        const float v2 = ((w >> (b0 + 2)) & 1u) ? sc[c + 2] * sl : -INFINITY;
-        const float v3 = ((w >> (b0 + 3)) & 1u) ? sc[c + 3] * sl : -INFINITY;
-        sc[c] = v0;
-        sc[c + 1] = v1;
-        sc[c + 2] = v2;
-        sc[c + 3] = v3;
-        t0m = fmaxf(t0m, v0);
-        t1m = fmaxf(t1m, v1);
-        t2m = fmaxf(t2m, v2);
-        t3m = fmaxf(t3m, v3);
+        mx0 = fmax3(mx0, sc[c], sc[c + 1]);
+        mx1 = fmax3(mx1, sc[c + 2], sc[c + 3]);
       }
-      float tmax = fmaxf(fmaxf(t0m, t1m), fmaxf(t2m, t3m));
-      if constexpr (NH == 2) {                          // combine the two key halves of the row
+      float tmax = fmaxf(mx0, mx1);
+      const float sl = p.scale_log2;
+      // P = 2^(s * scale_log2 - off) for this thread's keys, packed to bf16, with its row sum.
+      float ls0, ls1;
+      uint32_t pk[CW / 2];
+      auto exps = [&](float off) {
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < CW / 2; c += 2) {
+          float x0, x1, x2, x3;
+          ffma2(x0, x1, sc[2 * c], sc[2 * c + 1], sl, -off);
+          ffma2(x2, x3, sc[2 * c + 2], sc[2 * c + 3], sl, -off);
+          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+          const float e2 = ex2_approx(x2), e3 = ex2_approx(x3);
+          fadd2(a0, a1, e0, e1);
+          fadd2(a0, a1, e2, e3);
+          pk[c] = pack_bf16x2(e0, e1);
+          pk[c + 1] = pack_bf16x2(e2, e3);
+        }
+        ls0 = a0;
+        ls1 = a1;
+      };
+      // With two warps per row the row maximum needs the partner's half.  A row that already
+      // has a reference computes P against it while the partner's maximum is in flight, and
+      // recomputes only when the combined maximum moves the reference (rare: see kLazy).
+      if constexpr (NH == 2) {
         sh->xmax[j & 1][kh][row] = tmax;
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->xbar[wq][j & 1]);
+      }
+      const bool early = NH == 2 && __all_sync(0xffffffffu, m_ref != -INFINITY);
+      if (early) exps(m_ref);
+      if constexpr (NH == 2) {
         if (!mbar_wait(&sh->xbar[wq][j & 1], (j >> 1) & 1)) { ok = false; break; }
         tmax = fmaxf(tmax, sh->xmax[j & 1][kh ^ 1][row]);
       }
-      const bool need = tmax > m_ref + kLazy;           // also true for the first finite max
+      const float tms = tmax * sl;                      // row maximum in log2 units
+      const bool need = tms > m_ref + kLazy;            // also true for the first finite max
       const bool any = __any_sync(0xffffffffu, need);
-      const float m_new = need ? tmax : m_ref;
-      const float off = (m_new == -INFINITY) ? 0.f : m_new;
-      const float corr = need ? exp2f(m_ref - m_new) : 1.f;
-      float ls0 = 0.f, ls1 = 0.f;
-      uint32_t pk[CW / 2];
-#pragma unroll
-      for (int c = 0; c < CW / 2; ++c) {
-        const float e0 = ex2_approx(sc[2 * c] - off), e1 = ex2_approx(sc[2 * c + 1] - off);
-        ls0 += e0;
-        ls1 += e1;
-        pk[c] = pack_bf16x2(e0, e1);
-      }
+      const float m_new = need ? tms : m_ref;
+      if (!early || need) exps(m_new == -INFINITY ? 0.f : m_new);
+      const float corr = need ? ex2_approx(m_ref - m_new) : 1.f;
       l = l * corr + (ls0 + ls1);
       m_ref = m_new;
       // A rescale of O needs every earlier PV product finished (the last one wrote O).
@@ -365,16 +381,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int pb = j & 1;
       if (j >= 2) {
         if (!mbar_wait(&sh->p_free[pb], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
       }
-      uint8_t* prow = sP + pb * Sh::kPBytes + row * Sh::kPRow;
-#pragma unroll
-      for (int c = 0; c < CW / 8; ++c) {
-        const uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        const int lc = kh * (CW / 8) + c;               // 16-byte chunk within the P row
-        const int phys = KEYS == 64 ? (lc ^ (row & 7)) : (lc ^ ((row >> 1) & 3));
-        *reinterpret_cast<uint4*>(prow + (phys << 4)) = v;
-      }
-      fence_proxy_async();
+      // this thread's CW keys of P into its own TMEM lane (the PV product's A operand)
+      static_assert(CW == 32, "one 16-column P store per thread");
+      tmem_st16(lane_base + Sh::kPCol + pb * (KEYS / 2) + kh * (CW / 2), pk);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->p_full[pb]);
@@ -429,7 +440,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, Sh::kTmemCols);
   }
 }
 
@@ -438,7 +449,7 @@ static cudaError_t launch_shape(const CUtensorMap& q, const CUtensorMap& kc, con
                                 const CUtensorMap& kt, const CUtensorMap& vt, const AttnParams& p,
                                 int nb, cudaStream_t stream) {
   using Sh = TcShape<KEYS>;
-  const size_t smem = 1024 + kQBytes + (size_t)STAGES * Sh::kKV + 2 * Sh::kPBytes + sizeof(TcSmem);
+  const size_t smem = 1024 + kQBytes + (size_t)STAGES * Sh::kKV + sizeof(TcSmem);
   auto k = attn_tc_kernel<KEYS, STAGES, SW>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -450,8 +461,8 @@ static cudaError_t launch_shape(const CUtensorMap& q, const CUtensorMap& kc, con
 cudaError_t launch_attn_tc(const CUtensorMap& q, const CUtensorMap& kc, const CUtensorMap& vc,
                            const CUtensorMap& kt, const CUtensorMap& vt, const AttnParams& p,
                            int nb, int n_total, cudaStream_t stream) {
-  cudaError_t e = p.keys == 32 ? launch_shape<32, 3, 4>(q, kc, vc, kt, vt, p, nb, stream)
-                               : launch_shape<64, 4, 8>(q, kc, vc, kt, vt, p, nb, stream);
+  cudaError_t e = p.keys == 32 ? launch_shape<32, 4, 4>(q, kc, vc, kt, vt, p, nb, stream)
+                               : launch_shape<64, 5, 8>(q, kc, vc, kt, vt, p, nb, stream);
   if (e != cudaSuccess || p.nsplit == 1) return e;
   return launch_attn_combine(p, n_total, stream);
 }
