@@ -396,7 +396,7 @@ def roofline(wl, rep, peaks, peak_kind, workload):
     k = rep[dom]
     hbm, tc = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
     src = {"attn": "attn_tc.cu", "lmhead": "lmhead.cu", "compact": "compact.cu"}[dom]
-    traffic = ncu_traffic(dom, workload, source_hash(src))
+    traffic = ncu_traffic(dom, workload, source_hash(src, "common.cuh", "kernels.cuh"))
     if dom == "compact" or k["bytes"] / (hbm * 1e9) >= k.get("flops", 0) / (tc * 1e12):
         return {"kernel": dom, "bound": "hbm", "achieved": k["GB/s"], "peak": hbm,
                 "unit": "GB/s", "frac": k["GB/s"] / hbm, "traffic": traffic,
