@@ -64,6 +64,14 @@ def lib():
                                                 C.c_double, C.c_uint64, C.c_uint64, I32P, I32P,
                                                 I32P, I32P, C.c_int]
         L.oracle_accept_chain_batch.restype = None
+        L.oracle_accept_tree.argtypes = [C.c_int, I32P, I32P, F64P, F32P, C.c_int, C.c_double,
+                                         C.c_uint64, C.c_uint64, C.c_int, I32P, I32P, I32P,
+                                         C.POINTER(C.c_double)]
+        L.oracle_accept_tree.restype = C.c_int
+        L.oracle_accept_tree_batch.argtypes = [C.c_int, I32P, I32P, I32P, F64P, F32P, C.c_int,
+                                               C.c_double, C.c_uint64, C.c_uint64, I32P, I32P,
+                                               I32P, I32P, F64P, C.c_int]
+        L.oracle_accept_tree_batch.restype = None
         L.oracle_race_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
                                        C.c_int, I32P, C.c_int]
         L.oracle_race_many.restype = None
@@ -204,6 +212,39 @@ def accept_chain_batch(cu_nodes, parent, tokens, z, q, T, seed, step, nthreads=0
     return a, path, out, info
 
 
+def accept_tree(parent, tokens, z, q, T, seed, step, r):
+    """Multi-candidate acceptance over one request's tree; returns (a, path, out, info, c)."""
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    n, V = z.shape
+    path = np.empty(64, dtype=np.int32)
+    out = np.empty(65, dtype=np.int32)
+    info = np.zeros(3, dtype=np.int32)
+    c = C.c_double()
+    a = lib().oracle_accept_tree(n, _i32(parent), _i32(tokens), z, q, V, float(T), seed, step, r,
+                                 path, out, info, C.byref(c))
+    return a, path, out, info, c.value
+
+
+def accept_tree_batch(cu_nodes, parent, tokens, z, q, T, seed, step, nthreads=0):
+    """Batched oracle_accept_tree; returns (accept_len [B], path [B,64], out [B,65], info [B,3],
+    c [B])."""
+    cu = _i32(cu_nodes)
+    B = len(cu) - 1
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    V = z.shape[1]
+    a = np.empty(B, dtype=np.int32)
+    path = np.empty((B, 64), dtype=np.int32)
+    out = np.empty((B, 65), dtype=np.int32)
+    info = np.zeros((B, 3), dtype=np.int32)
+    c = np.zeros(B, dtype=np.float64)
+    lib().oracle_accept_tree_batch(B, cu, _i32(parent), _i32(tokens), z.reshape(-1),
+                                   q.reshape(-1), V, float(T), seed, step, a, path.reshape(-1),
+                                   out.reshape(-1), info.reshape(-1), c, int(nthreads))
+    return a, path, out, info, c
+
+
 def draw(w, seed, step, r, node):
     """The acceptance rule's two-level draw; returns (token, block, fell_to_last)."""
     w = np.ascontiguousarray(w, dtype=np.float64)
@@ -263,9 +304,14 @@ def lmhead_accept(wl, requests=None, nthreads=0, keep_logits=False):
             res[r] = dict(accept_len=a, path=path, out_tokens=out, argmax=arg, top1=t1, top2=t2)
         else:
             qd = wl.q_draft[a0:a1].numpy()
-            a, path, out, info = accept_chain(par, tok, z, qd, wl.temperature, wl.seed, wl.step,
-                                              r)
-            res[r] = dict(accept_len=a, path=path, out_tokens=out, info=info,
+            if np.array_equal(par, np.arange(-1, a1 - a0 - 1)):
+                a, path, out, info = accept_chain(par, tok, z, qd, wl.temperature, wl.seed,
+                                                  wl.step, r)
+                c = 1.0 if info[1] else 0.0
+            else:
+                a, path, out, info, c = accept_tree(par, tok, z, qd, wl.temperature, wl.seed,
+                                                    wl.step, r)
+            res[r] = dict(accept_len=a, path=path, out_tokens=out, info=info, c=c,
                           z=z if keep_logits else None)
     return res
 

@@ -19,10 +19,13 @@
  *  - attention has no positional term, soft-cap or window: q and k arrive ready to dot;
  *  - greedy: argmax ties go to the lowest vocab id; among children carrying the argmax token the
  *    lowest node index is taken;
- *  - T>0 is defined for chains only: node k's token was drafted from q of node k-1; accept iff
- *    U*q < p (strict); the bonus/residual token is drawn in two levels with Philox4x64-10
- *    uniforms: an exponential race among 128-id block totals, then an inverse CDF inside the
- *    winning block (oracle_draw).
+ *  - T>0 on chains: node k's token was drafted from q of node k-1; accept iff U*q < p (strict);
+ *    the bonus/residual token is drawn in two levels with Philox4x64-10 uniforms: an exponential
+ *    race among 128-id block totals, then an inverse CDF inside the winning block (oracle_draw);
+ *  - T>0 on branching trees (the pages give no rule): siblings are candidates drafted
+ *    independently from their parent's q and are tested in index order by multi-candidate
+ *    speculative sampling, each rejection replacing the target by its normalised residual
+ *    (oracle_accept_tree).
  */
 #include <math.h>
 #include <stdint.h>
@@ -436,6 +439,104 @@ int oracle_accept_chain(int n, const int32_t *parent, const int32_t *tokens, con
 }
 
 /* ---------------------------------------------------------------------------------------------
+ * Stochastic (T>0) acceptance over a general tree: multi-candidate speculative sampling (the
+ * multi-step rule of SpecInfer, Miao et al., "SpecInfer: Accelerating Large Language Model Serving
+ * with Tree-based Speculative Inference and Verification", 2023, restated here).
+ *
+ * The children c_1 < c_2 < ... of node u carry tokens x_i drafted independently from q_u.  The
+ * running target starts at r = p_u = softmax(z_u / T).  Child c_i is accepted iff
+ * U_i * q_u(x_i) < r(x_i), with U_i = oracle_uniform(seed, step, r, c_i, 0, 1) (the chain rule's
+ * stream, keyed by the child); acceptance moves the walk to c_i, whose own target restarts at its
+ * p.  A rejection replaces r by norm(max(0, r - q_u)).  Every such residual has the closed form
+ *     r_i = max(0, p_u - c_i q_u) / N(c_i),   N(c) = sum_v max(0, p_u(v) - c q_u(v)),
+ *     c_0 = 0, N(c_0) = 1,  c_{i+1} = c_i + N(c_i),
+ * since max(0, r_i - q_u) = max(0, p_u - (c_i + N(c_i)) q_u) / N(c_i) wherever it is positive.
+ * With candidates drawn independently from q_u, each step is an exact speculative-sampling step
+ * from the current residual, so the emitted token follows p_u.
+ *
+ * The walk stops at a node with no children or whose children are all rejected; the bonus is
+ * then drawn with oracle_draw at that node from the weights max(0, p_u - c q_u) (c = 0 when no
+ * child was rejected: the weights are p_u).  If a rejection leaves N(c) = 0 (r = q up to
+ * rounding; probability zero in exact arithmetic) the walk stops there and the bonus is the
+ * argmax of p_u, lowest id on ties -- the chain rule's fallback.  On a chain this is exactly
+ * oracle_accept_chain (c = 1 after the single rejection).
+ *
+ * z and q are the request's rows [n][V].  info (nullable): {stop node, rejections at the stop
+ * node, 1 if the fallback was taken}; c_out (nullable): the c of the bonus draw.
+ * Returns a, or OR_EINVAL for a malformed tree or a token outside [0, V).
+ * ------------------------------------------------------------------------------------------- */
+int oracle_accept_tree(int n, const int32_t *parent, const int32_t *tokens, const double *z,
+                       const float *q, int V, double T, uint64_t seed, uint64_t step, int r,
+                       int32_t *path, int32_t *out_tokens, int32_t *info, double *c_out) {
+    uint64_t anc[64];
+    int32_t dep[64];
+    for (int k = 0; k < 64; ++k) path[k] = -1;
+    for (int k = 0; k < 65; ++k) out_tokens[k] = -1;
+    if (oracle_ancestry(n, parent, anc, dep) != OR_OK) return OR_EINVAL;
+    for (int k = 1; k < n; ++k)
+        if (tokens[k] < 0 || tokens[k] >= V) return OR_EINVAL;
+    double *p = (double *)malloc(sizeof(double) * (size_t)V);
+    double *w = (double *)malloc(sizeof(double) * (size_t)V);
+    int u = 0, a = 0, nrej = 0, fell_back = 0;
+    double c = 0.0;
+    path[0] = 0;
+    for (;;) {
+        softmax_t(V, z + (size_t)u * V, T, p);
+        const float *qu = q + (size_t)u * V;
+        double Nc = 1.0;
+        int next = -1;
+        c = 0.0;
+        nrej = 0;
+        for (int j = u + 1; j < n && !fell_back; ++j) {
+            if (parent[j] != u) continue;
+            const int x = tokens[j];
+            const double qx = (double)qu[x];
+            double rx = p[x] - c * qx;
+            rx = rx > 0.0 ? rx / Nc : 0.0;
+            const double U = oracle_uniform(seed, step, (uint32_t)r, (uint32_t)j, 0, 1);
+            if (U * qx < rx) {
+                next = j;
+                break;
+            }
+            ++nrej;
+            c += Nc;
+            Nc = 0.0;
+            for (int v = 0; v < V; ++v) {
+                const double d = p[v] - c * (double)qu[v];
+                if (d > 0.0) Nc += d;
+            }
+            if (!(Nc > 0.0)) fell_back = 1;
+        }
+        if (next < 0) break;
+        out_tokens[a] = tokens[next];
+        ++a;
+        path[a] = next;
+        u = next;
+    }
+    int bonus = -1;
+    if (!fell_back) {
+        const float *qu = q + (size_t)u * V;
+        for (int v = 0; v < V; ++v) {
+            const double d = p[v] - c * (double)qu[v];
+            w[v] = d > 0.0 ? d : 0.0;
+        }
+        bonus = oracle_draw(V, w, seed, step, r, u, NULL);
+        if (bonus < 0) fell_back = 1;
+    }
+    if (fell_back) {
+        bonus = 0;
+        for (int v = 1; v < V; ++v)
+            if (p[v] > p[bonus]) bonus = v;
+    }
+    out_tokens[a] = bonus;
+    if (info) { info[0] = u; info[1] = nrej; info[2] = fell_back; }
+    if (c_out) *c_out = c;
+    free(p);
+    free(w);
+    return a;
+}
+
+/* ---------------------------------------------------------------------------------------------
  * KV compaction.  For every layer l and request r with a = accept_len[r]:
  *   cache[l][slot_base[r] + kv_len[r] + k] <- tree[l][cu_nodes[r] + path[r][k]],  k = 0..a,
  * for K and V (path[r][0] is the root), and kv_len_out[r] = kv_len[r] + a + 1.  A request whose
@@ -495,6 +596,23 @@ void oracle_accept_chain_batch(int B, const int32_t *cu_nodes, const int32_t *pa
                                             q + (size_t)a0 * V, V, T, seed, step, r,
                                             path + (size_t)r * 64, out_tokens + (size_t)r * 65,
                                             info + (size_t)r * 3);
+    }
+}
+
+/* Batched oracle_accept_tree, laid out like oracle_accept_chain_batch; c_out [B]. */
+void oracle_accept_tree_batch(int B, const int32_t *cu_nodes, const int32_t *parent,
+                              const int32_t *tokens, const double *z, const float *q, int V,
+                              double T, uint64_t seed, uint64_t step, int32_t *accept_len,
+                              int32_t *path, int32_t *out_tokens, int32_t *info, double *c_out,
+                              int nthreads) {
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int r = 0; r < B; ++r) {
+        int a0 = cu_nodes[r], n = cu_nodes[r + 1] - cu_nodes[r];
+        accept_len[r] = oracle_accept_tree(n, parent + a0, tokens + a0, z + (size_t)a0 * V,
+                                           q + (size_t)a0 * V, V, T, seed, step, r,
+                                           path + (size_t)r * 64, out_tokens + (size_t)r * 65,
+                                           info + (size_t)r * 3, c_out + r);
     }
 }
 

@@ -458,6 +458,135 @@ def test_rejected_draft_residual_excludes_the_rejected_token_mass():
     assert len(seen) == V - 1
 
 
+# ------------------------------------------------------- stochastic acceptance on branching trees
+def test_tree_rule_equals_chain_rule_on_chains():
+    """On a chain the multi-candidate rule is the chain rule: same accepts, path, tokens, stop
+    node, rejection flag and fallback, with c = 1 after the rejection (residual max(0, p - q))."""
+    g = np.random.default_rng(31)
+    for trial in range(300):
+        n = int(g.integers(1, 9))
+        V = int(g.integers(20, 300))
+        T = float(g.choice([1.0, 0.7, 1.6]))
+        z = g.normal(0, 2.0, size=(n, V))
+        q = np.stack([_softmax(g.normal(0, 2.0, size=V)) for _ in range(n)]).astype(np.float32)
+        par = np.arange(-1, n - 1, dtype=np.int32)
+        tok = g.integers(0, V, size=n).astype(np.int32)
+        for k in range(1, n):                     # draft most tokens from q so some are accepted
+            if g.random() < 0.7:
+                tok[k] = int(np.argmax(q[k - 1]))
+        ac, pc, oc, ic = oracle.accept_chain(par, tok, z, q, T, 77, trial, 5)
+        at, pt, ot, it, c = oracle.accept_tree(par, tok, z, q, T, 77, trial, 5)
+        assert (ac, list(pc), list(oc)) == (at, list(pt), list(ot))
+        assert list(ic) == list(it)
+        assert c == (1.0 if ic[1] else 0.0)
+
+
+def test_tree_rule_rejects_malformed_trees_and_tokens():
+    z = np.zeros((3, 8))
+    q = np.full((3, 8), 1 / 8, dtype=np.float32)
+    a, *_ = oracle.accept_tree(np.array([-1, 2, 1], np.int32), np.array([1, 2, 3], np.int32), z,
+                               q, 1.0, 1, 0, 0)
+    assert a == oracle.EINVAL
+    a, *_ = oracle.accept_tree(np.array([-1, 0, 0], np.int32), np.array([1, 2, 8], np.int32), z,
+                               q, 1.0, 1, 0, 0)
+    assert a == oracle.EINVAL
+
+
+def _tree_trials(k, pz, qz, T, ntrial, seed, chunk=100_000):
+    """ntrial requests of a two-level tree: the root has k children whose tokens are drafted
+    independently from q_root; child with token x has 2 children drafted from q_x.  Target and
+    draft logits depend on the token prefix only: root rows pz[0] / qz[0], rows after first token
+    x pz[1 + x] / qz[1 + x].  Returns the first two emitted tokens and accept lengths."""
+    V = pz.shape[1]
+    g = np.random.default_rng(seed)
+    q_of = np.stack([_softmax(r) for r in qz]).astype(np.float32)
+    n = 1 + k + 2 * k
+    par = np.array([-1] + [0] * k + [1 + i // 2 for i in range(2 * k)], dtype=np.int32)
+    firsts, seconds, alen = [], [], []
+    done, step = 0, 0
+    while done < ntrial:
+        m = min(chunk, ntrial - done)
+        tok = np.zeros((m, n), dtype=np.int32)
+        cq = np.cumsum(q_of.astype(np.float64), axis=1)
+        tok[:, 1:1 + k] = np.minimum(V - 1, np.searchsorted(cq[0], g.random((m, k)) * cq[0, -1]))
+        rowsel = np.zeros((m, n), dtype=np.int64)       # which prefix row each node uses
+        for i in range(k):
+            rowsel[:, 1 + i] = 1 + tok[:, 1 + i]
+        for j in range(2 * k):
+            parent_tok = tok[:, 1 + j // 2]
+            u = g.random(m)
+            tok[:, 1 + k + j] = np.minimum(
+                V - 1, np.array([np.searchsorted(cq[1 + x], uu * cq[1 + x, -1])
+                                 for x, uu in zip(parent_tok, u)]))
+            rowsel[:, 1 + k + j] = 0                    # grandchildren are leaves: rows unused
+        z = pz[rowsel.reshape(-1)]
+        q = q_of[rowsel.reshape(-1)]
+        cu = (np.arange(m + 1) * n).astype(np.int32)
+        a, path, out, info, c = oracle.accept_tree_batch(cu, np.tile(par, m), tok.reshape(-1), z,
+                                                          q, T, seed, step)
+        assert (a >= 0).all()
+        firsts.append(out[:, 0])
+        seconds.append(np.where(a >= 1, out[:, 1], -1))
+        alen.append(a)
+        done += m
+        step += 1
+    return np.concatenate(firsts), np.concatenate(seconds), np.concatenate(alen)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("k,T", [(2, 1.0), (3, 0.7), (4, 1.0)])
+def test_multi_candidate_first_token_follows_target(k, T):
+    """10^6 trials, V=16: with k candidates drafted independently from q_root (duplicates
+    allowed), the first emitted token ~ p_root, through any number of sibling rejections and
+    residual updates; given an accepted first token x, the second ~ p_x."""
+    V = 16
+    g = np.random.default_rng(40 + k)
+    pz = g.normal(0, 1.5, size=(1 + V, V))
+    qz = g.normal(0, 1.5, size=(1 + V, V))          # far from the target: many rejections
+    first, second, a = _tree_trials(k, pz, qz, T, 1_000_000, seed=0xE7EE0600 + k)
+    assert _chisq_p(first, _softmax(pz[0] / T)) > 1e-4
+    acc = a >= 1
+    assert 0.2 < acc.mean() < 0.99
+    x = np.bincount(first[acc], minlength=V).argmax()
+    sel = acc & (first == x)
+    assert _chisq_p(second[sel], _softmax(pz[1 + x] / T)) > 1e-4
+
+
+def test_multi_candidate_identical_draft_accepts_the_first_child():
+    """q = p at every node: the first child is always accepted (U q < p = q for U < 1)."""
+    V = 32
+    g = np.random.default_rng(50)
+    z = g.normal(0, 1.0, size=(7, V))
+    q = np.stack([_softmax(r) for r in z]).astype(np.float32)
+    par = np.array([-1, 0, 0, 0, 1, 1, 2], dtype=np.int32)
+    for r in range(500):
+        tok = g.integers(0, V, size=7).astype(np.int32)
+        a, path, out, info, c = oracle.accept_tree(par, tok, z, q, 1.0, 9, 0, r)
+        assert path[1] == 1 and path[2] == 4 and a == 2 and info[1] == 0 and c == 0.0
+
+
+def test_multi_candidate_residual_excludes_rejected_mass():
+    """After the root's only candidate token is rejected by both siblings, the bonus comes from
+    max(0, p - c q) with c = 1 + N(1) > 1: never token 0, where q exceeds p."""
+    V = 8
+    p = np.full(V, 1 / V)
+    q = p.copy()
+    q[0] += 0.3
+    q[1:] -= 0.3 / (V - 1)
+    z = np.log(np.stack([p, p, p]))
+    qq = np.stack([q, q, q]).astype(np.float32)
+    par = np.array([-1, 0, 0], dtype=np.int32)
+    tok = np.array([5, 0, 0], dtype=np.int32)
+    seen, two = set(), 0
+    for r in range(4000):
+        a, path, out, info, c = oracle.accept_tree(par, tok, z, qq, 1.0, 99, 0, r)
+        if a == 0:
+            assert out[0] != 0 and info[1] == 2 and c > 1.0
+            seen.add(int(out[0]))
+            two += 1
+    assert two > 0 and len(seen) == V - 1
+
+
 # ----------------------------------------------------------------------------------- compaction
 def test_kv_compact_equals_numpy_gather():
     g = np.random.default_rng(9)
