@@ -12,6 +12,8 @@ Entry points (same names as the C ABI in ``include/etree.h``)::
     etree_verify_attn(batch, q, k_tree, v_tree, k_cache, v_cache, scale, out, lse, workspace)
     etree_lmhead_accept(batch, hidden, w_lm, temperature, q_draft, seed, step, accept_len, path,
                         out_tokens, node_argmax, node_gap, workspace)
+    etree_lmhead_accept_tree(batch, hidden, w_lm, temperature, q_draft, seed, step, accept_len,
+                             path, out_tokens, zbuf, workspace)
     etree_kv_compact(batch, accept_len, path, k_tree, v_tree, k_cache, v_cache, n_layers,
                      tree_layer_stride, cache_layer_stride, kv_len_out, workspace)
     etree_device_status(workspace, stream=None) -> (status, detail)
@@ -26,7 +28,7 @@ import torch
 __all__ = [
     "EtreeError", "Batch", "make_batch", "lib", "library_path", "etree_workspace_size",
     "etree_workspace_init", "etree_verify_attn", "etree_verify_attn_noalloc",
-    "etree_lmhead_accept", "etree_kv_compact",
+    "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact",
     "etree_device_status", "etree_strerror", "etree_version", "etree_attn_plan", "STATUS",
 ]
 
@@ -39,7 +41,7 @@ DETAIL = {0: "none", 1: "bad parent", 2: "bad node count", 3: "bad kv_len", 4: "
           5: "not a chain", 6: "bad path", 7: "attention wait", 8: "gemm wait", 9: "bad token"}
 
 EXPORTS = ["etree_workspace_size", "etree_workspace_init", "etree_verify_attn",
-           "etree_lmhead_accept", "etree_kv_compact", "etree_device_status", "etree_strerror",
+           "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact", "etree_device_status", "etree_strerror",
            "etree_version", "etree_last_error", "etree_attn_plan", "etree_verify_attn_noalloc"]
 
 
@@ -84,6 +86,9 @@ def lib():
     L.etree_lmhead_accept.argtypes = [bp, vp, vp, C.c_int, C.c_int, f32, vp, u64, u64, vp, vp,
                                       vp, vp, vp, vp, C.c_size_t, vp]
     L.etree_lmhead_accept.restype = C.c_int
+    L.etree_lmhead_accept_tree.argtypes = [bp, vp, vp, C.c_int, C.c_int, f32, vp, u64, u64, vp,
+                                           vp, vp, vp, C.c_int32, vp, C.c_size_t, vp]
+    L.etree_lmhead_accept_tree.restype = C.c_int
     L.etree_kv_compact.argtypes = [bp, vp, vp, vp, vp, vp, vp, C.c_int, i64, i64, C.c_int,
                                    C.c_int, vp, vp, C.c_size_t, vp]
     L.etree_kv_compact.restype = C.c_int
@@ -208,6 +213,22 @@ def etree_lmhead_accept(batch: Batch, hidden, w_lm, temperature: float, q_draft,
         _ptr(accept_len, torch.int32, "accept_len"), _ptr(path, torch.int32, "path"),
         _ptr(out_tokens, torch.int32, "out_tokens"),
         _ptr(node_argmax, torch.int32, "node_argmax"), _ptr(node_gap, torch.float32, "node_gap"),
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
+    return _check(st) if check else st
+
+
+def etree_lmhead_accept_tree(batch: Batch, hidden, w_lm, temperature: float, q_draft, seed: int,
+                             step: int, accept_len, path, out_tokens, zbuf, workspace,
+                             stream=None, check: bool = True) -> int:
+    """zbuf: fp32 [rows][vocab] device tensor (or None for no rows)."""
+    bf = torch.bfloat16
+    rows = 0 if zbuf is None else int(zbuf.shape[0])
+    st = lib().etree_lmhead_accept_tree(
+        C.byref(batch), _ptr(hidden, bf, "hidden"), _ptr(w_lm, bf, "w_lm"), hidden.shape[1],
+        w_lm.shape[0], float(temperature), _ptr(q_draft, torch.float32, "q_draft"),
+        int(seed) & (2**64 - 1), int(step) & (2**64 - 1),
+        _ptr(accept_len, torch.int32, "accept_len"), _ptr(path, torch.int32, "path"),
+        _ptr(out_tokens, torch.int32, "out_tokens"), _ptr(zbuf, torch.float32, "zbuf"), rows,
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
     return _check(st) if check else st
 

@@ -270,7 +270,7 @@ __device__ void accept_chain(const AcceptParams& p, int r, int base, int n, int 
     p.accept_len[r] = chain ? a : 0;
     p.stop_row[r] = src;
     p.stop_node[r] = chain ? a : 0;
-    p.mode[r] = chain ? rejected : 0;
+    p.cval[r] = (chain && rejected) ? 1.f : 0.f;
   }
   const uint4* hs = reinterpret_cast<const uint4*>(p.hidden + (size_t)src * p.H);
   uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(256) chain_accept_kernel(AcceptParams p, int32
     if (lane == 0) {
       p.stop_row[r] = 0;
       p.stop_node[r] = 0;
-      p.mode[r] = 0;
+      p.cval[r] = 0.f;
     }
     const uint4* hs = reinterpret_cast<const uint4*>(p.hidden);
     uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
@@ -324,6 +324,272 @@ __global__ void __launch_bounds__(256) chain_accept_kernel(AcceptParams p, int32
   const int r = row_owner(p, row, base, n);
   if (r < 0 || !last_arrival(cnt, r, n, lane)) return;
   accept_chain(p, r, base, n, lane);
+}
+
+// ---------------------------------------------------------------- T > 0 on branching trees
+// Multi-candidate speculative sampling (the multi-step rule of SpecInfer, Miao et al. 2023): the
+// children of node u are candidates drafted independently from q_u and are tested in index
+// order against a running target r that starts at p_u; a rejection replaces r by
+// norm(max(0, r - q_u)).  Each residual is r_i = max(0, p_u - c_i q_u) / N(c_i) with
+// N(c) = sum_v max(0, p_u(v) - c q_u(v)), c_0 = 0, N(c_0) = 1, c_{i+1} = c_i + N(c_i), so the
+// walk needs, per rejection that is followed by another sibling, one pass over row u's logits
+// (materialised by the LM-head pass for rows with two or more children) and its q row.
+
+// One CTA: per-node child counts, then a row of the caller's logit buffer for every node with
+// two or more children (in node order).  Nodes past zbuf_rows get none: their requests are
+// answered as malformed by the walk and the status reports ETREE_ENOSPACE.
+__global__ void __launch_bounds__(1024) tree_prep_kernel(AcceptParams p, int32_t* ccount,
+                                                         int32_t* zrow, int zbuf_rows) {
+  __shared__ int32_t part_s[1024];
+  const int tid = threadIdx.x, nt = blockDim.x;
+  for (int g = tid; g < p.n_total; g += nt) ccount[g] = 0;
+  __syncthreads();
+  for (int g = tid; g < p.n_total; g += nt) {
+    int base, n;
+    if (row_owner(p, g, base, n) < 0) continue;
+    const int local = g - base, pl = p.parent[g];
+    if (local >= 1 && pl >= 0 && pl < local) atomicAdd(ccount + base + pl, 1);
+  }
+  __syncthreads();
+  // exclusive scan of the branching flags: each thread owns a contiguous segment
+  const int seg = (p.n_total + nt - 1) / nt;
+  const int g0 = min(p.n_total, tid * seg), g1 = min(p.n_total, g0 + seg);
+  int cnt = 0;
+  for (int g = g0; g < g1; ++g) cnt += ccount[g] >= 2;
+  part_s[tid] = cnt;
+  __syncthreads();
+  for (int off = 1; off < nt; off <<= 1) {            // Hillis-Steele inclusive scan
+    const int v = tid >= off ? part_s[tid - off] : 0;
+    __syncthreads();
+    part_s[tid] += v;
+    __syncthreads();
+  }
+  int next = part_s[tid] - cnt;
+  bool over = false;
+  for (int g = g0; g < g1; ++g) {
+    int zr = -1;
+    if (ccount[g] >= 2) {
+      if (next < zbuf_rows) zr = next; else over = true;
+      ++next;
+    }
+    zrow[g] = zr;
+  }
+  if (over) report(p.ws, ETREE_ENOSPACE, DET_ZBUF);
+}
+
+// One warp per non-root node: the parent row's logit of the node's token,
+// z = hidden[parent] . W[token], in fp32 (the acceptance test's p(x) needs it for every child,
+// and siblings may share a row).  Invalid tokens get -inf and report ETREE_EDEVICE.
+__global__ void __launch_bounds__(256) child_logit_kernel(AcceptParams p,
+                                                          const __nv_bfloat16* w_lm, float* zc) {
+  const int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (g >= p.n_total) return;
+  int base, n;
+  float z = -INFINITY;
+  if (row_owner(p, g, base, n) >= 0 && g > base) {
+    const int pl = p.parent[g], x = p.tokens[g];
+    if (pl >= 0 && pl < g - base && x >= 0 && x < p.V) {
+      const uint4* h = reinterpret_cast<const uint4*>(p.hidden + (size_t)(base + pl) * p.H);
+      const uint4* w = reinterpret_cast<const uint4*>(w_lm + (size_t)x * p.H);
+      float acc = 0.f;
+      for (int i = lane; i < p.H / 8; i += 32) {
+        const uint4 a = h[i], b = __ldg(w + i);
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 fa = __bfloat1622float2(a2[k]), fb = __bfloat1622float2(b2[k]);
+          acc = fmaf(fa.x, fb.x, acc);
+          acc = fmaf(fa.y, fb.y, acc);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      z = acc;
+    } else if (lane == 0 && (x < 0 || x >= p.V)) {
+      report(p.ws, ETREE_EDEVICE, DET_BAD_TOKEN);
+    }
+  }
+  if (lane == 0) zc[g] = z;
+}
+
+// One warp per node row: log2 sum 2^(z log2(e) / T) from the LM head's (max, sum) summaries.
+__global__ void __launch_bounds__(256) row_lse_kernel(AcceptParams p) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= p.n_total) return;
+  const float4* part = p.part + (size_t)row * p.n_tiles;
+  float m = -INFINITY, s = 0.f;
+  int t = lane;
+  for (; t + 96 < p.n_tiles; t += 128) {
+    const float4 a = part[t], b = part[t + 32], c = part[t + 64], d = part[t + 96];
+    merge_lse(m, s, a.x, a.y);
+    merge_lse(m, s, b.x, b.y);
+    merge_lse(m, s, c.x, c.y);
+    merge_lse(m, s, d.x, d.y);
+  }
+  for (; t < p.n_tiles; t += 32) {
+    const float4 a = part[t];
+    merge_lse(m, s, a.x, a.y);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, m, off);
+    const float os = __shfl_xor_sync(0xffffffffu, s, off);
+    merge_lse(m, s, om, os);
+  }
+  if (lane == 0) p.lse2[row] = m + log2f(s);
+}
+
+// N(c) = sum_v max(0, p_u(v) - c q_u(v)) over one materialised logit row, by the whole CTA, in
+// fp64 (p_u(v) = 2^(z_v log2(e) / T - lse2_u) in fp32).
+__device__ double residual_mass(const AcceptParams& p, const float* zr, const float* qr, float L2,
+                                double c, double* red) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  double acc = 0.0;
+  if ((p.V & 3) == 0) {
+    const float4* z4 = reinterpret_cast<const float4*>(zr);
+    const float4* q4 = reinterpret_cast<const float4*>(qr);
+    for (int i = tid; i < p.V / 4; i += nt) {
+      const float4 z = z4[i], q = __ldg(q4 + i);
+      const float zz[4] = {z.x, z.y, z.z, z.w}, qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const double d = (double)exp2f(zz[k] * p.k_log2 - L2) - c * (double)qq[k];
+        acc += d > 0.0 ? d : 0.0;
+      }
+    }
+  } else {
+    for (int v = tid; v < p.V; v += nt) {
+      const double d = (double)exp2f(zr[v] * p.k_log2 - L2) - c * (double)__ldg(qr + v);
+      acc += d > 0.0 ? d : 0.0;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((tid & 31) == 0) red[tid >> 5] = acc;
+  __syncthreads();
+  double tot = 0.0;
+  for (int w = 0; w < (nt >> 5); ++w) tot += red[w];
+  __syncthreads();
+  return tot;
+}
+
+// One CTA per request: the multi-candidate walk.  Thread 0 takes the decisions; the whole CTA
+// evaluates N(c) when a rejected child has a younger sibling still to test.  Writes accept_len,
+// path, the accepted tokens, the stop row / node, the draw offset cval (negative: fall back to
+// argmax p) and the stop row's hidden state for the draw pass.
+__global__ void __launch_bounds__(256) tree_walk_kernel(AcceptParams p, const float* zc,
+                                                        const int32_t* zrow, const float* zbuf) {
+  __shared__ int par_s[64], tok_s[64];
+  __shared__ double red_s[8];
+  __shared__ int act_s, u_s, ok_s, fell_s;
+  __shared__ double c_s;
+  const int r = blockIdx.x, tid = threadIdx.x;
+  int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
+  int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
+  int base, n;
+  const bool n_ok = request_ok(p, r, base, n);
+  if (tid == 0) ok_s = n_ok ? 1 : 0;
+  if (n_ok && tid < n) {
+    par_s[tid] = p.parent[base + tid];
+    tok_s[tid] = p.tokens[base + tid];
+  }
+  __syncthreads();
+  if (n_ok && tid < n) {
+    const int pj = par_s[tid];
+    const bool good = tid == 0 ? pj == -1 : (pj >= 0 && pj < tid);
+    bool fits = true;                                   // a branching node without a logit row
+    int kids = 0;
+    for (int j = tid + 1; j < n; ++j) kids += par_s[j] == tid;
+    if (kids >= 2 && zrow[base + tid] < 0) fits = false;
+    if (!good) { report(p.ws, ETREE_EDEVICE, DET_BAD_PARENT); atomicAnd(&ok_s, 0); }
+    if (tid >= 1 && (tok_s[tid] < 0 || tok_s[tid] >= p.V)) atomicAnd(&ok_s, 0);  // reported by
+                                                                               // child_logit
+    if (!fits) atomicAnd(&ok_s, 0);                      // reported by tree_prep_kernel
+  }
+  __syncthreads();
+  if (!ok_s) {                                          // accept nothing, draw from the root's p
+    if (!n_ok && tid == 0) report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
+    for (int k = tid; k < 64; k += blockDim.x) path[k] = (n_ok && k == 0) ? 0 : -1;
+    for (int k = tid; k < 65; k += blockDim.x) outt[k] = -1;
+    if (tid == 0) {
+      p.accept_len[r] = 0;
+      p.stop_row[r] = n_ok ? base : 0;
+      p.stop_node[r] = 0;
+      p.cval[r] = 0.f;
+      u_s = n_ok ? base : 0;
+    }
+  } else {
+    // thread 0's walk state: node u, last child tested, c and N(c) of the current residual
+    int u = 0, j = 0, a = 0;
+    double c = 0.0, N = 1.0;
+    if (tid == 0) {
+      path[0] = 0;
+      fell_s = 0;
+    }
+    for (int it = 0; it < 2 * 64 + 2; ++it) {          // each node is tested once: bounded
+      __syncthreads();                                  // the previous round's values are read
+      if (tid == 0) {
+        int act = 2;                                    // 0: moved on, 1: need N(c), 2: stop
+        for (j = j + 1; j < n && par_s[j] != u; ++j) {}
+        if (j < n) {
+          const int x = tok_s[j];
+          const float L2 = p.lse2[base + u];
+          const double qx = (double)__ldg(p.q_draft + (size_t)(base + u) * p.V + x);
+          const double pz = (double)exp2f(zc[base + j] * p.k_log2 - L2);
+          const double rx = pz - c * qx > 0.0 ? (pz - c * qx) / N : 0.0;
+          float U[8];
+          uniforms8(p.seed, p.step, 0u, (uint32_t)j, (uint32_t)r, 1u, U);
+          if ((double)U[0] * qx < rx) {                 // accepted: the walk moves to child j
+            ++a;
+            path[a] = j;
+            outt[a - 1] = x;
+            u = j;
+            c = 0.0;
+            N = 1.0;
+            act = 0;
+          } else {                                      // rejected: r <- norm(max(0, r - q))
+            c += N;
+            int k = j + 1;
+            while (k < n && par_s[k] != u) ++k;
+            act = k < n ? 1 : 2;                        // N(c) only if a sibling remains
+          }
+        }
+        act_s = act;
+        u_s = u;
+        c_s = c;
+      }
+      __syncthreads();
+      const int act = act_s;
+      if (act == 2) break;
+      if (act == 1) {
+        const int ur = base + u_s;
+        const double Nn = residual_mass(p, zbuf + (size_t)zrow[ur] * p.V,
+                                        p.q_draft + (size_t)ur * p.V, p.lse2[ur], c_s, red_s);
+        if (tid == 0) {
+          N = Nn;
+          if (!(N > 0.0)) fell_s = 1;                   // no positive residual: argmax p
+        }
+        __syncthreads();
+        if (fell_s) break;
+      }
+    }
+    if (tid == 0) {
+      for (int k = a + 1; k < 64; ++k) path[k] = -1;
+      for (int k = a; k < 65; ++k) outt[k] = -1;
+      p.accept_len[r] = a;
+      p.stop_row[r] = base + u;
+      p.stop_node[r] = u;
+      p.cval[r] = fell_s ? -1.f : (float)c;
+      u_s = base + u;
+    }
+  }
+  __syncthreads();
+  const uint4* hs = reinterpret_cast<const uint4*>(p.hidden + (size_t)u_s * p.H);
+  uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
+  for (int i = tid; i < p.H / 8; i += blockDim.x) hd[i] = hs[i];
 }
 
 // The first level of the two-level draw, per request: the exponential race among the 128-id
@@ -382,6 +648,20 @@ cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStr
 
 cudaError_t launch_accept_chain(const AcceptParams& p, int32_t* cnt, cudaStream_t s) {
   chain_accept_kernel<<<(p.n_total + p.B + 7) / 8, 256, 0, s>>>(p, cnt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tree_prep(const AcceptParams& p, const __nv_bfloat16* w_lm, int32_t* ccount,
+                             int32_t* zrow, int zbuf_rows, float* zc, cudaStream_t s) {
+  tree_prep_kernel<<<1, 1024, 0, s>>>(p, ccount, zrow, zbuf_rows);
+  child_logit_kernel<<<(p.n_total + 7) / 8, 256, 0, s>>>(p, w_lm, zc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32_t* zrow,
+                             const float* zbuf, cudaStream_t s) {
+  row_lse_kernel<<<(p.n_total + 7) / 8, 256, 0, s>>>(p);
+  tree_walk_kernel<<<p.B, 256, 0, s>>>(p, zc, zrow, zbuf);
   return cudaGetLastError();
 }
 

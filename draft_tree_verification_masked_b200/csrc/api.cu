@@ -106,8 +106,8 @@ static AttnPlan plan_attn(const etree_batch* b, int hq, int hkv) {
 
 // ------------------------------------------------------------------------------ workspace map
 struct WsLayout {
-  size_t order, o_part, ml_part, part, child_tok, zchild, lse2, stop_row, stop_node, mode, hid2,
-      part2, cnt;
+  size_t order, o_part, ml_part, part, child_tok, zchild, lse2, stop_row, stop_node, cval, hid2,
+      part2, cnt, ccount, zrow, zc;
   size_t total;
   int n_tiles;
 };
@@ -138,10 +138,13 @@ static WsLayout layout(const etree_batch* b, int hq, int hkv, int hidden_dim, in
   w.lse2 = take(nt * sizeof(float));
   w.stop_row = take(B * sizeof(int32_t));
   w.stop_node = take(B * sizeof(int32_t));
-  w.mode = take(B * sizeof(int32_t));
+  w.cval = take(B * sizeof(float));
   w.hid2 = take(B * (size_t)std::max(0, hidden_dim) * 2);
   w.part2 = take(B * (size_t)w.n_tiles * sizeof(float4));
   w.cnt = take(B * sizeof(int32_t));
+  w.ccount = take(nt * sizeof(int32_t));
+  w.zrow = take(nt * sizeof(int32_t));
+  w.zc = take(nt * sizeof(float));
   w.total = off;
   return w;
 }
@@ -432,12 +435,19 @@ etree_status etree_verify_attn(const etree_batch* b, const uint16_t* q, const ui
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_verify_attn launch");
 }
 
-etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
-                                 const uint16_t* w_lm, int hidden_dim, int vocab,
-                                 float temperature, const float* q_draft, uint64_t seed,
-                                 uint64_t step, int32_t* accept_len, int32_t* path,
-                                 int32_t* out_tokens, int32_t* node_argmax, float* node_gap,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+// The caller's logit buffer of the branching-tree sampler (etree_lmhead_accept_tree).
+struct TreeRows {
+  float* zbuf;
+  int32_t rows;
+};
+
+static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hidden,
+                                       const uint16_t* w_lm, int hidden_dim, int vocab,
+                                       float temperature, const float* q_draft, uint64_t seed,
+                                       uint64_t step, int32_t* accept_len, int32_t* path,
+                                       int32_t* out_tokens, int32_t* node_argmax,
+                                       float* node_gap, const TreeRows* tree, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
   etree_status st = check_batch(b);
   if (st) return st;
   if (hidden_dim < 64 || hidden_dim % 64 != 0)
@@ -479,7 +489,7 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
   g.k_log2 = temperature > 0.f ? 1.4426950408889634f / temperature : 0.f;
   g.stop_row = at<int32_t>(workspace, w.stop_row);
   g.stop_node = at<int32_t>(workspace, w.stop_node);
-  g.mode = at<int32_t>(workspace, w.mode);
+  g.cval = at<float>(workspace, w.cval);
   g.lse2 = at<float>(workspace, w.lse2);
   g.q_draft = q_draft;
   g.seed = seed;
@@ -515,7 +525,7 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
   a.step = step;
   a.stop_row = at<int32_t>(workspace, w.stop_row);
   a.stop_node = at<int32_t>(workspace, w.stop_node);
-  a.mode = at<int32_t>(workspace, w.mode);
+  a.cval = at<float>(workspace, w.cval);
   a.hidden = reinterpret_cast<const __nv_bfloat16*>(hidden);
   a.hid2 = at<__nv_bfloat16>(workspace, w.hid2);
   a.H = hidden_dim;
@@ -527,9 +537,23 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
     if (e == cudaSuccess) e = launch_accept_greedy(a, at<int32_t>(workspace, w.child_tok), cnt, s);
     return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T=0)");
   }
-  e = launch_chain_prep(a, at<int32_t>(workspace, w.child_tok), s);
-  if (e == cudaSuccess) e = launch_lmhead(1, bn, bm, ta, tb, g, grid, s);
-  if (e == cudaSuccess) e = launch_accept_chain(a, cnt, s);
+  if (!tree) {                               // chains: accept tests fused with the row merge
+    e = launch_chain_prep(a, at<int32_t>(workspace, w.child_tok), s);
+    if (e == cudaSuccess) e = launch_lmhead(1, bn, bm, ta, tb, g, grid, s);
+    if (e == cudaSuccess) e = launch_accept_chain(a, cnt, s);
+  } else {                                   // trees: materialised rows of branching nodes
+    int32_t* zrow = at<int32_t>(workspace, w.zrow);
+    float* zc = at<float>(workspace, w.zc);
+    e = launch_tree_prep(a, reinterpret_cast<const __nv_bfloat16*>(w_lm),
+                         at<int32_t>(workspace, w.ccount), zrow, tree->rows, zc, s);
+    g.child_tok = nullptr;
+    g.zrow = zrow;
+    g.zbuf = tree->zbuf;
+    if (e == cudaSuccess) e = launch_lmhead(1, bn, bm, ta, tb, g, grid, s);
+    g.zrow = nullptr;
+    g.zbuf = nullptr;
+    if (e == cudaSuccess) e = launch_tree_walk(a, zc, zrow, tree->zbuf, s);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "etree_lmhead_accept (T>0, pass 1)");
   const int bn2 = 256;                       // the draw's 128-id blocks pair up in a tile
   const int bm2 = (b->B <= 64 && env_int("ETREE_BM", 0) != 128) ? 64 : 128;
@@ -549,6 +573,33 @@ etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
   e = launch_lmhead(2, bn2, bm2, th, tb2, g2, std::min(g2.num_tiles, sms), s);
   if (e == cudaSuccess) e = launch_bonus(a, s);
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T>0, pass 2)");
+}
+
+etree_status etree_lmhead_accept(const etree_batch* b, const uint16_t* hidden,
+                                 const uint16_t* w_lm, int hidden_dim, int vocab,
+                                 float temperature, const float* q_draft, uint64_t seed,
+                                 uint64_t step, int32_t* accept_len, int32_t* path,
+                                 int32_t* out_tokens, int32_t* node_argmax, float* node_gap,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  return lmhead_accept_impl(b, hidden, w_lm, hidden_dim, vocab, temperature, q_draft, seed, step,
+                            accept_len, path, out_tokens, node_argmax, node_gap, nullptr,
+                            workspace, workspace_bytes, stream);
+}
+
+etree_status etree_lmhead_accept_tree(const etree_batch* b, const uint16_t* hidden,
+                                      const uint16_t* w_lm, int hidden_dim, int vocab,
+                                      float temperature, const float* q_draft, uint64_t seed,
+                                      uint64_t step, int32_t* accept_len, int32_t* path,
+                                      int32_t* out_tokens, float* zbuf, int32_t zbuf_rows,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (zbuf_rows < 0 || (zbuf_rows > 0 && !zbuf))
+    return fail(ETREE_EINVAL, "zbuf_rows=%d with zbuf=%p", zbuf_rows, (void*)zbuf);
+  if (zbuf && !aligned16(zbuf)) return fail(ETREE_EINVAL, "zbuf must be 16-byte aligned");
+  const TreeRows tr{zbuf, zbuf_rows};
+  return lmhead_accept_impl(b, hidden, w_lm, hidden_dim, vocab, temperature, q_draft, seed, step,
+                            accept_len, path, out_tokens, nullptr, nullptr,
+                            temperature > 0.f ? &tr : nullptr, workspace, workspace_bytes,
+                            stream);
 }
 
 etree_status etree_kv_compact(const etree_batch* b, const int32_t* accept_len,

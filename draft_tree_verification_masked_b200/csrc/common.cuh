@@ -31,6 +31,7 @@ enum Detail : int32_t {
   DET_WAIT_ATTN = 7,        // a bounded wait gave up in attention
   DET_WAIT_GEMM = 8,        // a bounded wait gave up in the LM-head GEMM
   DET_BAD_TOKEN = 9,        // a token id outside [0, vocab)
+  DET_ZBUF = 10,            // more branching tree nodes than rows in the caller's logit buffer
 };
 
 __device__ __forceinline__ void report(WsHeader* ws, int32_t code, int32_t detail) {

@@ -40,6 +40,8 @@ struct GemmParams {
   int per_cta, n_parts;
   int32_t* cnt;                     // if set, CTA 0 zeroes cnt[0 .. cnt_n) (acceptance counters)
   int cnt_n;
+  const int32_t* zrow;              // EPI_LSE, if set: row g's logits go to zbuf[zrow[g]][V]
+  float* zbuf;                      // when zrow[g] >= 0 (rows of branching tree nodes)
   WsHeader* ws;
   float4* part;
   const int32_t* child_tok;
@@ -47,7 +49,9 @@ struct GemmParams {
   float k_log2;
   const int32_t* stop_row;
   const int32_t* stop_node;
-  const int32_t* mode;
+  // Draw weights of the race pass per request: w = max(0, p - cval q); cval = 0 draws from p,
+  // cval < 0 marks a residual without positive weight (the bonus falls back to argmax p).
+  const float* cval;
   const float* lse2;
   const float* q_draft;
   uint64_t seed, step;
@@ -75,7 +79,7 @@ struct AcceptParams {
   uint64_t seed, step;
   int32_t* stop_row;
   int32_t* stop_node;
-  int32_t* mode;
+  float* cval;
   const __nv_bfloat16* hidden;
   __nv_bfloat16* hid2;
   int H;
@@ -86,6 +90,10 @@ cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, int32_t
 cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStream_t s);
 cudaError_t launch_accept_chain(const AcceptParams& p, int32_t* cnt, cudaStream_t s);
 cudaError_t launch_bonus(const AcceptParams& p, cudaStream_t s);
+cudaError_t launch_tree_prep(const AcceptParams& p, const __nv_bfloat16* w_lm, int32_t* ccount,
+                             int32_t* zrow, int zbuf_rows, float* zc, cudaStream_t s);
+cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32_t* zrow,
+                             const float* zbuf, cudaStream_t s);
 
 struct CompactParams {
   const int32_t* cu_nodes;

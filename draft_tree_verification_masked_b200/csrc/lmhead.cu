@@ -17,10 +17,12 @@
 // output row) per thread, and apply the epilogue:
 //   EPI_ARGMAX  per row and tile: top-1 value, its vocab id (lowest on ties) and top-2 value;
 //   EPI_LSE     per row and tile: m = max z*log2(e)/T and sum 2^(z*log2(e)/T - m), plus the
-//               logit of the row's child token when it falls in the tile;
-//   EPI_RACE    per row and 128-id block: the block total of the draw's weights (max(0, p - q)
-//               after a rejection, else p), the id where the block's running sum passes u_b
-//               times that total, and the block's largest logit; the block race happens in
+//               logit of the row's child token when it falls in the tile; rows of branching tree
+//               nodes also write their logits out (the sibling residuals need whole rows);
+//   EPI_RACE    per row and 128-id block: the block total of the draw's weights
+//               max(0, p - c q) (c = 0: p; c = 1: the residual after one rejection; larger c
+//               after sibling rejections), the id where the block's running sum passes u_b times
+//               that total, and the block's largest logit; the block race happens in
 //               bonus_kernel.
 #include "kernels.cuh"
 #include "philox.cuh"
@@ -42,7 +44,8 @@ struct EpiRow {
   int ct = -1;                                       // LSE: child token of the row
   float zc = 0.f;                                    // LSE: its logit
   bool found = false;
-  int unode = 0, md = 0, req = 0;                    // RACE: stop node, mode, request
+  int unode = 0, req = 0;                            // RACE: stop node, request
+  float c = 0.f;                                     // RACE: residual offset (cval)
   float L2 = 0.f;                                    // RACE: log2 sum 2^(z k)
   const float* qrow = nullptr;                       // RACE: q_draft row
 };
@@ -83,6 +86,22 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, EpiRow& st, const
         if (col0 + j == st.ct) st.zc = v[j];
       st.found = true;
     }
+  }
+}
+
+// W consecutive logits of one row to its materialised copy (columns past the vocab dropped).
+template <int W>
+__device__ __forceinline__ void store_logits(const GemmParams& p, float* zdst, const float (&v)[W],
+                                             int col0) {
+  if ((p.V & 3) == 0) {
+#pragma unroll
+    for (int j = 0; j < W; j += 4)
+      if (col0 + j < p.V)
+        *reinterpret_cast<float4*>(zdst + col0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < W; ++j)
+      if (col0 + j < p.V) zdst[col0 + j] = v[j];
   }
 }
 
@@ -246,11 +265,13 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       const uint32_t tbase = tmem + ((uint32_t)(wq * 32) << 16) + buf * BN;
 
       if (!p.per_cta) st = EpiRow();
-      if (EPI == EPI_LSE && active) st.ct = p.child_tok[grow];
+      if (EPI == EPI_LSE && active && p.child_tok) st.ct = p.child_tok[grow];
+      const int zr = (EPI == EPI_LSE && active && p.zrow) ? p.zrow[grow] : -1;
+      float* zdst = zr >= 0 ? p.zbuf + (size_t)zr * p.V : nullptr;
       if (EPI == EPI_RACE && active) {
         const int g = p.stop_row[grow];
         st.unode = p.stop_node[grow];
-        st.md = p.mode[grow];
+        st.c = p.cval[grow];
         st.req = grow;
         st.L2 = p.lse2[g];
         st.qrow = p.q_draft + (size_t)g * p.V;
@@ -268,12 +289,13 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         float W = 0.f, zmax = -INFINITY;
         int zarg = -1;
         float qa[32], qb[32];
-        if (active && st.md) load_q32(p, st.qrow, colb, qa);
+        const bool md = st.c > 0.f;                     // q enters the weights
+        if (active && md) load_q32(p, st.qrow, colb, qa);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float (&q)[32] = (c & 1) ? qb : qa;
           float (&qn)[32] = (c & 1) ? qa : qb;
-          if (active && st.md && c < 3) load_q32(p, st.qrow, colb + (c + 1) * 32, qn);
+          if (active && md && c < 3) load_q32(p, st.qrow, colb + (c + 1) * 32, qn);
           float v[32];
           tmem_ld32(tcol + c * 32, v);
           if (active) {
@@ -287,7 +309,7 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
                   zarg = col;
                 }
                 const float pv = exp2f(v[j] * p.k_log2 - st.L2);
-                w = st.md ? fmaxf(pv - q[j], 0.f) : pv;
+                w = md ? fmaxf(pv - st.c * q[j], 0.f) : (st.c < 0.f ? 0.f : pv);
                 W += w;
               }
               v[j] = w;
@@ -328,12 +350,14 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           float v[32];
           tmem_ld32(tbase + c * 32, v);
           if (active) epi_chunk<EPI, 32>(p, st, v, nt * BN + c * 32);
+          if (EPI == EPI_LSE && zdst) store_logits<32>(p, zdst, v, nt * BN + c * 32);
         }
         if constexpr (BN % 32 == 16) {
           if (half == kTailHalf) {
             float v[16];
             tmem_ld16(tbase + kChunks * 32, v);
             if (active) epi_chunk<EPI, 16>(p, st, v, nt * BN + kChunks * 32);
+            if (EPI == EPI_LSE && zdst) store_logits<16>(p, zdst, v, nt * BN + kChunks * 32);
           }
         }
       }

@@ -8,12 +8,29 @@ from __future__ import annotations
 
 import torch
 
-from . import (etree_device_status, etree_kv_compact, etree_lmhead_accept, etree_verify_attn,
-               etree_workspace_init, etree_workspace_size, make_batch)
+import numpy as np
+
+from . import (etree_device_status, etree_kv_compact, etree_lmhead_accept,
+               etree_lmhead_accept_tree, etree_verify_attn, etree_workspace_init,
+               etree_workspace_size, make_batch)
+
+
+def branching_nodes(wl) -> int:
+    """Number of tree nodes with two or more children."""
+    cnt = np.zeros(wl.n_total, dtype=np.int64)
+    for r in range(wl.B):
+        a0, a1 = int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])
+        par = np.asarray(wl.parent[a0 + 1:a1], dtype=np.int64)
+        np.add.at(cnt, a0 + par, 1)
+    return int((cnt >= 2).sum())
 
 
 class DeviceStep:
-    def __init__(self, wl, device: str = "cuda", n_layers: int = 1, pin: bool = False):
+    """tree: None picks the branching-tree sampler (etree_lmhead_accept_tree) when T > 0 and a
+    node has two or more children; zbuf_rows overrides the size of its logit buffer."""
+
+    def __init__(self, wl, device: str = "cuda", n_layers: int = 1, pin: bool = False,
+                 tree=None, zbuf_rows=None):
         self.wl = wl
         self.device = device
         dev = torch.device(device)
@@ -68,6 +85,11 @@ class DeviceStep:
         self.ws = torch.zeros(max(size, 256), dtype=torch.uint8, device=dev)
         etree_workspace_init(self.ws)
         self.scale = 1.0 / float(wl.head_dim) ** 0.5
+        nbr = branching_nodes(wl)
+        self.tree = (wl.temperature > 0 and nbr > 0) if tree is None else bool(tree)
+        rows = nbr if zbuf_rows is None else int(zbuf_rows)
+        self.zbuf = (torch.empty(rows, wl.vocab, dtype=torch.float32, device=dev)
+                     if self.tree and rows > 0 else None)
 
     # --- the three calls
     def attn(self, stream=None):
@@ -75,6 +97,11 @@ class DeviceStep:
                           self.v_cache, self.scale, self.out, self.lse, self.ws, stream)
 
     def lmhead(self, stream=None):
+        if self.tree:
+            etree_lmhead_accept_tree(self.batch, self.hidden, self.w_lm, self.wl.temperature,
+                                     self.q_draft, self.wl.seed, self.wl.step, self.accept_len,
+                                     self.path, self.out_tokens, self.zbuf, self.ws, stream)
+            return
         etree_lmhead_accept(self.batch, self.hidden, self.w_lm, self.wl.temperature,
                             self.q_draft, self.wl.seed, self.wl.step, self.accept_len, self.path,
                             self.out_tokens, self.node_argmax, self.node_gap, self.ws, stream)

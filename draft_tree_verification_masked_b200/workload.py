@@ -18,9 +18,9 @@ vocab 151936).  The synthetic recipe and every reading it takes are listed in th
   argmax with overwhelming probability.  A child carries its parent's planted token with the
   configured match probability (at most one sibling does), else a uniform random token distinct
   from its siblings and from t*_u.
-* T>0 (chains): target logits come out N(0,2) by drawing W ~ N(0, 2/sqrt(hidden)); draft
-  distributions are softmax of N(0,2) logits and each draft token is sampled from its parent's
-  draft distribution.
+* T>0: target logits come out N(0,2) by drawing W ~ N(0, 2/sqrt(hidden)); draft distributions
+  are softmax of N(0,2) logits and each draft token is sampled from its parent's draft
+  distribution, independently for siblings (chains and branching trees alike).
 """
 from __future__ import annotations
 
@@ -65,9 +65,14 @@ CONFIGS: dict[str, dict] = {
     "conc512": dict(B=512, hq=40, hkv=8, head_dim=128, hidden=5120, vocab=151936,
                     kv_len=(512, 4096), n_nodes=4, depth=3, depth_min=3, branch=1, width=None,
                     match=None, temperature=1.0, w_sigma=None, draft_sigma=2.0),
+    # 64 requests, KV ~ U[1024, 8192], branching 16-node trees (<= 4 children per node),
+    # stochastic acceptance at T=1 with siblings drafted independently.
+    "tree64_t1": dict(B=64, hq=40, hkv=8, head_dim=128, hidden=5120, vocab=151936,
+                      kv_len=(1024, 8192), n_nodes=16, depth=6, depth_min=2, branch=4,
+                      width=None, match=None, temperature=1.0, w_sigma=None, draft_sigma=2.0),
 }
 CONFIG_INDEX = {"tiny": 0, "dense27b_b1": 1, "long32k": 2, "long128k": 2, "batch64": 3,
-                "conc512": 4}
+                "conc512": 4, "tree64_t1": 5}
 
 
 def config_seed(name: str) -> int:

@@ -144,9 +144,10 @@ etree_status etree_verify_attn_noalloc(const etree_batch *batch, const uint16_t 
  *    drafted from q_draft row k-1; it is accepted iff U * q(x) < p(x), U a seeded uniform.  At
  *    the first rejection (node u) the bonus is drawn from norm(max(0, p_u - q_u)); when all are
  *    accepted it is drawn from p of the last node.  Draws use an exponential race with
- *    Philox4x64-10 uniforms keyed by (seed, step) and countered by (vocab id/4, node, request,
+ *    Philox4x64-10 uniforms keyed by (seed, step) and countered by (vocab id / 8, node, request,
  *    stream), so results are reproducible bit for bit.  A branching tree records
- *    ETREE_EUNSUPPORTED (detail 5, "not a chain") and that request accepts nothing.
+ *    ETREE_EUNSUPPORTED (detail 5, "not a chain") and that request accepts nothing; sample
+ *    branching trees with etree_lmhead_accept_tree.
  *   hidden      [n_total][hidden_dim] bf16;   w_lm [vocab][hidden_dim] bf16 (K contiguous)
  *   q_draft     [n_total][vocab] fp32 draft probabilities (T > 0 only, else may be NULL)
  *   accept_len  [B] accepted draft nodes a_r (0 .. n_r - 1)
@@ -162,6 +163,37 @@ etree_status etree_lmhead_accept(const etree_batch *batch, const uint16_t *hidde
                                  uint64_t step, int32_t *accept_len, int32_t *path,
                                  int32_t *out_tokens, int32_t *node_argmax, float *node_gap,
                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * LM head + stochastic acceptance over general draft trees (T > 0; T == 0 behaves exactly like
+ * etree_lmhead_accept).  The pages verify whole trees in one pass ("Eagle-4 Released: Outpaces
+ * DFlash2 and DSpark ...", section "Technical Background") but give no sampling rule for
+ * siblings; this call takes multi-candidate speculative sampling (SpecInfer, Miao et al. 2023):
+ * the children of node u, whose tokens were drafted independently from q_draft row u, are tested
+ * in node-index order against a running target r that starts at p_u = softmax(z_u / T): child c
+ * with token x is accepted iff U_c * q_u(x) < r(x), and each rejection replaces r by
+ * norm(max(0, r - q_u)), which equals max(0, p_u - c q_u) / N(c) for an offset c that grows by
+ * N(c) = sum_v max(0, p_u(v) - c q_u(v)) per rejection.  An accepted child becomes the node
+ * whose children are tested next.  The walk stops at a leaf or when all children of a node are
+ * rejected; the bonus is drawn there from max(0, p_u - c q_u) (from p_u when nothing was
+ * rejected there) with the two-level draw of etree_lmhead_accept; a residual without positive
+ * weight falls back to argmax p_u.  On chains the results equal etree_lmhead_accept's.
+ *   zbuf       caller-owned device buffer [zbuf_rows][vocab] fp32, 16-byte aligned: the logits
+ *              of every node with two or more children are written there (in node order),
+ *              because each sibling rejection needs a pass over the whole row.  At most
+ *              floor((n_total - B) / 2) rows are ever needed.  A batch with more branching nodes
+ *              than zbuf_rows records ETREE_ENOSPACE (detail 10) and the requests left without a
+ *              row accept nothing: their bonus is drawn from the root's p (a one-token decode).  zbuf may be NULL when zbuf_rows == 0 (chains need no rows).
+ *   Other arguments as in etree_lmhead_accept (no node_argmax / node_gap outputs).
+ * Errors: host-side as etree_lmhead_accept, plus ETREE_EINVAL for zbuf_rows < 0, a NULL zbuf
+ * with zbuf_rows > 0, or a misaligned zbuf.
+ */
+etree_status etree_lmhead_accept_tree(const etree_batch *batch, const uint16_t *hidden,
+                                      const uint16_t *w_lm, int hidden_dim, int vocab,
+                                      float temperature, const float *q_draft, uint64_t seed,
+                                      uint64_t step, int32_t *accept_len, int32_t *path,
+                                      int32_t *out_tokens, float *zbuf, int32_t zbuf_rows,
+                                      void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * KV compaction.  For each of n_layers layers and each request r with a = accept_len[r]:

@@ -141,6 +141,85 @@ def chain_compare(wl, res, requests, nthreads=0):
     return excused, near, ores
 
 
+def _draw_near_tie(wl, r, u, w, tg, to):
+    """The GPU's bonus tg and the oracle's to differ at stop node u with weights w: the two
+    blocks' race keys, or the inverse-CDF threshold inside the common block, must be within
+    rounding."""
+    bg, bo = tg // 128, to // 128
+
+    def bkey(b):
+        Wb = w[b * 128:(b + 1) * 128].sum()
+        Ub = oracle.uniform(wl.seed, wl.step, r, u, b, 2)
+        return np.log(Wb) - np.log(-np.log(Ub)) if Wb > 0 else -np.inf
+
+    if bg != bo:
+        kg, ko = bkey(bg), bkey(bo)
+        assert np.isfinite(kg) and abs(kg - ko) <= SAMPLE_REL * max(1.0, abs(ko)), \
+            (r, tg, to, kg, ko)
+    else:
+        blk = w[bo * 128:min(len(w), (bo + 1) * 128)]
+        c = np.cumsum(blk)
+        W = c[-1]
+        thr = oracle.uniform(wl.seed, wl.step, r, u, bo, 3) * W
+        i = tg - bo * 128
+        before = c[i - 1] if i > 0 else 0.0
+        assert blk[i] > 0 and c[i] > thr - SAMPLE_REL * W and before <= thr + SAMPLE_REL * W, \
+            (r, tg, to, c[i], before, thr, W)
+
+
+def tree_compare(wl, res, requests, nthreads=0):
+    """T > 0 on branching trees: the GPU's walk against the oracle's.  Where they differ, the
+    first differing decision is replayed in fp64 and must be a sampling near-tie: an accept test
+    U q(x) vs r(x) = max(0, p(x) - c q(x)) / N(c), or the bonus draw.  Returns (excused, near)."""
+    ores = oracle.lmhead_accept(wl, requests, nthreads=nthreads, keep_logits=True)
+    excused, near = set(), 0
+    T = wl.temperature
+    for r in requests:
+        o = ores[r]
+        a0, a1 = int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])
+        n = a1 - a0
+        ga, oa = int(res["accept_len"][r]), int(o["accept_len"])
+        if (ga == oa and np.array_equal(res["path"][r], o["path"])
+                and np.array_equal(res["out_tokens"][r], o["out_tokens"])):
+            continue
+        z = o["z"] / T
+        p = np.exp(z - z.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        qd = wl.q_draft[a0:a1].numpy().astype(np.float64)
+        par = wl.parent[a0:a1]
+        tok = wl.tokens[a0:a1]
+        gp, op = list(res["path"][r][:ga + 1]), list(o["path"][:oa + 1])
+        u, depth, settled = 0, 0, False
+        while not settled:
+            gnext = gp[depth + 1] if depth + 1 <= ga else None
+            onext = op[depth + 1] if depth + 1 <= oa else None
+            c, N = 0.0, 1.0
+            for j in [j for j in range(1, n) if par[j] == u]:
+                x = int(tok[j])
+                U = oracle.uniform(wl.seed, wl.step, r, j, 0, 1)
+                uq, rx = U * qd[u, x], max(0.0, p[u, x] - c * qd[u, x]) / N
+                if (onext == j) != (gnext == j):
+                    assert abs(uq - rx) <= SAMPLE_REL * max(uq, rx), (r, u, j, uq, rx)
+                    settled = True
+                    break
+                if onext == j:
+                    break
+                c += N
+                N = np.maximum(p[u] - c * qd[u], 0.0).sum()
+            if settled:
+                break
+            if onext is None and gnext is None:        # same path, different bonus
+                w = np.maximum(p[u] - c * qd[u], 0.0)
+                _draw_near_tie(wl, r, u, w, int(res["out_tokens"][r][ga]),
+                               int(o["out_tokens"][oa]))
+                break
+            assert onext == gnext, (r, gp, op)
+            u, depth = onext, depth + 1
+        excused.add(r)
+        near += 1
+    return excused, near, ores
+
+
 def compact_compare(wl, dev, ores, requests, excused):
     """Bit-exact check of the compacted rows of each request against the oracle's compaction
     of that request's slot range (single layer)."""

@@ -78,7 +78,7 @@ def test_stochastic_acceptance_on_a_branching_tree_is_unsupported():
     wl = W.generate("tiny", B=2, kv_len=[100, 300], hidden=256, vocab=512)
     wl.temperature = 1.0
     wl.q_draft = torch.full((wl.n_total, wl.vocab), 1.0 / wl.vocab)
-    dev = DeviceStep(wl)
+    dev = DeviceStep(wl, tree=False)                  # the chain entry point
     dev.lmhead()
     assert dev.status() == (EUNSUP, 5)
     _still_works()

@@ -17,20 +17,22 @@ from . import _parity as P
 pytestmark = pytest.mark.gpu
 
 
-def _run(wl, n_layers=1):
-    dev = DeviceStep(wl, n_layers=n_layers)
+def _run(wl, n_layers=1, **kw):
+    dev = DeviceStep(wl, n_layers=n_layers, **kw)
     dev.step()
     st, det = dev.status()
     assert st == 0, (st, det)
     return dev, dev.results()
 
 
-def _full_check(wl, attn_rows=None, requests=None):
-    dev, res = _run(wl)
+def _full_check(wl, attn_rows=None, requests=None, **kw):
+    dev, res = _run(wl, **kw)
     P.attn_compare(wl, dev, rows=attn_rows)
     reqs = list(range(wl.B)) if requests is None else requests
     if wl.temperature == 0.0:
         excused, near, ores = P.greedy_compare(wl, res, reqs)
+    elif dev.tree:
+        excused, near, ores = P.tree_compare(wl, res, reqs)
     else:
         excused, near, ores = P.chain_compare(wl, res, reqs)
     P.compact_compare(wl, dev, ores, reqs, excused)
@@ -217,3 +219,60 @@ def test_lmhead_row_tile_heights(bm, T, monkeypatch):
                     vocab=8192 + 77, temperature=T, **shape)
     assert wl.n_total == 64
     _full_check(wl)
+
+
+# ------------------------------------------------------------ T > 0 on branching trees
+def _branching(T, vocab, B=9, seed_nodes=(16, 5, 1, 12, 9, 3, 16, 7, 2)):
+    return W.generate("tree64_t1", B=B, n_nodes=list(seed_nodes[:B]), depth=4, depth_min=2,
+                      branch=4, kv_len=(20, 400), hidden=512, vocab=vocab, temperature=T)
+
+
+@pytest.mark.parametrize("T,vocab", [(1.0, 4096 + 3), (0.6, 8192), (1.6, 2048 + 128)])
+def test_stochastic_branching_trees(T, vocab):
+    """Multi-candidate acceptance: sibling rejections with residual passes over materialised
+    logit rows, ragged and aligned vocab sizes (scalar and float4 paths)."""
+    wl = _branching(T, vocab)
+    dev, res = _full_check(wl)
+    assert dev.tree and dev.zbuf is not None
+
+
+def test_tree_sampler_on_chains_matches_chain_rule():
+    """The branching-tree entry point on chains (no logit rows needed) gives the chain rule."""
+    wl = W.generate("conc512", B=37, n_nodes=[4, 5, 6, 1, 2] * 7 + [4, 4], depth=5,
+                    depth_min=5, kv_len=(20, 400), hidden=512, vocab=4096 + 3, temperature=1.0)
+    dev, res = _run(wl, tree=True)
+    assert dev.zbuf is None
+    excused, near, ores = P.chain_compare(wl, res, list(range(wl.B)))
+    assert near <= 3
+
+
+def test_tree64_t1_full_size():
+    wl = W.generate("tree64_t1")
+    g = np.random.default_rng(3)
+    reqs = sorted(g.choice(wl.B, 8, replace=False).tolist())
+    _full_check(wl, attn_rows=P.sample_rows(wl, 2), requests=reqs)
+
+
+def test_logit_buffer_overflow_reports_and_answers_the_rest():
+    """Fewer logit rows than branching nodes: ETREE_ENOSPACE (detail 10); the requests whose
+    branching nodes all got a row still match the oracle, the others accept nothing."""
+    from draft_tree_verification_masked_b200.runner import branching_nodes
+    wl = _branching(1.0, 4096 + 3)
+    need = branching_nodes(wl)
+    dev = DeviceStep(wl, zbuf_rows=need // 2)
+    dev.lmhead()
+    assert dev.status() == (-6, 10)
+    res = dev.results()
+    # rows are assigned in node order: request r keeps its rows iff all of its branching nodes
+    # come before the cut
+    cnt, got = 0, []
+    for r in range(wl.B):
+        a0, a1 = int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])
+        kids = np.bincount(wl.parent[a0 + 1:a1], minlength=a1 - a0)
+        cnt += int((kids >= 2).sum())
+        if cnt <= need // 2:
+            got.append(r)
+        else:
+            assert res["accept_len"][r] == 0 and res["out_tokens"][r][0] >= 0   # root draw only
+    excused, near, ores = P.tree_compare(wl, res, got)
+    assert near <= 1
