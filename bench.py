@@ -355,7 +355,9 @@ def run_config(name, steps, warmup, peaks, rank, flush, with_e2e=True):
     toks = int((acc + 1).sum())
     t = time_steps(dev, steps, warmup, flush)
     plan = etree_attn_plan(dev.batch, wl.hq, wl.hkv)
-    launches = plan["launches"] + (2 if wl.temperature == 0.0 else 5) + 1
+    # attention + LM head (T=0: GEMM, fused accept; chains: prep, GEMM, accept, draw GEMM, race;
+    # branching trees: prep, child logits, GEMM, row merge, walk, draw GEMM, race) + compaction
+    launches = plan["launches"] + (2 if wl.temperature == 0.0 else (7 if dev.tree else 5)) + 1
     res = dict(wl=wl, dev=dev, toks=toks, t=t, plan=plan, launches=launches)
     if with_e2e:
         res["e2e"] = time_e2e(dev, wl, steps, max(3, warmup), flush)
@@ -413,7 +415,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="etree", choices=["etree", "reference"])
     ap.add_argument("--config", default="dense27b_b1")
-    ap.add_argument("--by-batch", default="batch64,conc512",
+    ap.add_argument("--by-batch", default="batch64,conc512,tree64_t1",
                     help="extra workloads measured in the same run (comma list, '' for none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

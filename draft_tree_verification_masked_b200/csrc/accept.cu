@@ -442,29 +442,47 @@ __global__ void __launch_bounds__(256) row_lse_kernel(AcceptParams p) {
   if (lane == 0) p.lse2[row] = m + log2f(s);
 }
 
-// N(c) = sum_v max(0, p_u(v) - c q_u(v)) over one materialised logit row, by the whole CTA, in
-// fp64 (p_u(v) = 2^(z_v log2(e) / T - lse2_u) in fp32).
+// N(c) = sum_v max(0, p_u(v) - c q_u(v)) over one materialised logit row, by the whole CTA:
+// p_u(v) = 2^(z_v log2(e) / T - lse2_u) and the difference in fp32, summed in fp32 over 16
+// terms, then in fp64 (each thread's partials, then the CTA's).
 __device__ double residual_mass(const AcceptParams& p, const float* zr, const float* qr, float L2,
                                 double c, double* red) {
   const int tid = threadIdx.x, nt = blockDim.x;
+  const float cf = (float)c, kl = p.k_log2;
   double acc = 0.0;
   if ((p.V & 3) == 0) {
     const float4* z4 = reinterpret_cast<const float4*>(zr);
     const float4* q4 = reinterpret_cast<const float4*>(qr);
-    for (int i = tid; i < p.V / 4; i += nt) {
-      const float4 z = z4[i], q = __ldg(q4 + i);
-      const float zz[4] = {z.x, z.y, z.z, z.w}, qq[4] = {q.x, q.y, q.z, q.w};
+    const int n4 = p.V / 4;
+    int i = tid;
+    for (; i + 3 * nt < n4; i += 4 * nt) {            // four float4 pairs in flight per thread
+      float4 z[4], q[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const double d = (double)exp2f(zz[k] * p.k_log2 - L2) - c * (double)qq[k];
-        acc += d > 0.0 ? d : 0.0;
+        z[k] = z4[i + k * nt];
+        q[k] = __ldg(q4 + i + k * nt);
       }
+      float part = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        part += fmaxf(exp2f(z[k].x * kl - L2) - cf * q[k].x, 0.f);
+        part += fmaxf(exp2f(z[k].y * kl - L2) - cf * q[k].y, 0.f);
+        part += fmaxf(exp2f(z[k].z * kl - L2) - cf * q[k].z, 0.f);
+        part += fmaxf(exp2f(z[k].w * kl - L2) - cf * q[k].w, 0.f);
+      }
+      acc += (double)part;
+    }
+    for (; i < n4; i += nt) {
+      const float4 z = z4[i], q = __ldg(q4 + i);
+      const float zz[4] = {z.x, z.y, z.z, z.w}, qq[4] = {q.x, q.y, q.z, q.w};
+      float part = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) part += fmaxf(exp2f(zz[k] * kl - L2) - cf * qq[k], 0.f);
+      acc += (double)part;
     }
   } else {
-    for (int v = tid; v < p.V; v += nt) {
-      const double d = (double)exp2f(zr[v] * p.k_log2 - L2) - c * (double)__ldg(qr + v);
-      acc += d > 0.0 ? d : 0.0;
-    }
+    for (int v = tid; v < p.V; v += nt)
+      acc += (double)fmaxf(exp2f(zr[v] * kl - L2) - cf * __ldg(qr + v), 0.f);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -480,10 +498,10 @@ __device__ double residual_mass(const AcceptParams& p, const float* zr, const fl
 // evaluates N(c) when a rejected child has a younger sibling still to test.  Writes accept_len,
 // path, the accepted tokens, the stop row / node, the draw offset cval (negative: fall back to
 // argmax p) and the stop row's hidden state for the draw pass.
-__global__ void __launch_bounds__(256) tree_walk_kernel(AcceptParams p, const float* zc,
+__global__ void __launch_bounds__(512) tree_walk_kernel(AcceptParams p, const float* zc,
                                                         const int32_t* zrow, const float* zbuf) {
   __shared__ int par_s[64], tok_s[64];
-  __shared__ double red_s[8];
+  __shared__ double red_s[16];
   __shared__ int act_s, u_s, ok_s, fell_s;
   __shared__ double c_s;
   const int r = blockIdx.x, tid = threadIdx.x;
@@ -661,7 +679,7 @@ cudaError_t launch_tree_prep(const AcceptParams& p, const __nv_bfloat16* w_lm, i
 cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32_t* zrow,
                              const float* zbuf, cudaStream_t s) {
   row_lse_kernel<<<(p.n_total + 7) / 8, 256, 0, s>>>(p);
-  tree_walk_kernel<<<p.B, 256, 0, s>>>(p, zc, zrow, zbuf);
+  tree_walk_kernel<<<p.B, 512, 0, s>>>(p, zc, zrow, zbuf);
   return cudaGetLastError();
 }
 
