@@ -38,6 +38,7 @@ GAMMA = 10.0
 _TAGS = {
     "tree": 1, "tokens": 2, "plant": 3, "q": 4, "k_tree": 5, "v_tree": 6, "k_cache": 7,
     "v_cache": 8, "hidden": 9, "w_lm": 10, "kv_len": 11, "draft_logits": 12, "draft_pick": 13,
+    "pages": 14,
 }
 
 CONFIGS: dict[str, dict] = {
@@ -338,3 +339,44 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """Zero-copy uint16 view of a contiguous CPU bf16 tensor."""
     assert t.dtype == torch.bfloat16 and t.is_contiguous()
     return t.view(torch.int16).numpy().view(np.uint16)
+
+
+# ------------------------------------------------------------------------------- paged layout
+@dataclass
+class PagedCache:
+    """A workload's cache laid out in pages of a shared pool (the input of the paged calls)."""
+    page_size: int
+    max_pages: int
+    num_pages: int
+    block_table: np.ndarray          # int32 [B, max_pages], -1 where no page is mapped
+    k_pool: torch.Tensor             # bf16 [num_pages * page_size, hkv, d]
+    v_pool: torch.Tensor
+    slot_cap: np.ndarray             # int32 [B]: mapped pages x page_size
+
+
+def paged(wl: "Workload", page_size: int, spare_pages: int = 3, seed: int = 0) -> PagedCache:
+    """Lays the workload's per-request caches out in page_size-token pages at random distinct
+    pool pages (plus unmapped spare pages): logical position t of request r goes to pool slot
+    block_table[r, t // page_size] * page_size + t % page_size.  Each request maps
+    ceil(slot_cap[r] / page_size) pages, so its capacity is that many pages."""
+    g = _rng(wl.seed, "pages", seed)
+    P = int(page_size)
+    npg = [(int(c) + P - 1) // P for c in wl.slot_cap]
+    total = sum(npg) + spare_pages
+    perm = g.permutation(total).astype(np.int32)
+    maxp = max(npg) if npg else 1
+    bt = np.full((wl.B, maxp), -1, dtype=np.int32)
+    kp = torch.zeros((total * P,) + tuple(wl.k_cache.shape[1:]), dtype=torch.bfloat16)
+    vp = torch.zeros_like(kp)
+    nxt = 0
+    for r in range(wl.B):
+        base, cap = int(wl.slot_base[r]), int(wl.slot_cap[r])
+        for j in range(npg[r]):
+            page = int(perm[nxt])
+            nxt += 1
+            bt[r, j] = page
+            lo, hi = j * P, min(cap, (j + 1) * P)
+            kp[page * P:page * P + hi - lo] = wl.k_cache[base + lo:base + hi]
+            vp[page * P:page * P + hi - lo] = wl.v_cache[base + lo:base + hi]
+    return PagedCache(page_size=P, max_pages=maxp, num_pages=total, block_table=bt, k_pool=kp,
+                      v_pool=vp, slot_cap=np.array([n * P for n in npg], dtype=np.int32))

@@ -5,7 +5,8 @@ this package.  The product path (the CUDA library and its Python binding) never 
 code with this module, and this module imports nothing from it.
 
 Every function is a thin ctypes marshaller around the plain C definitions in ``oracle.c``; the
-per-request composition below only slices rows and calls those definitions in order.
+per-request composition below only slices rows and calls those definitions in order, and the
+paged-cache forms first gather (or scatter) rows through the block tables with numpy indexing.
 """
 from __future__ import annotations
 
@@ -281,6 +282,68 @@ def kv_compact(cu_nodes, kv_len, slot_base, slot_cap, accept_len, path, k_tree, 
                                  _u16(v_tree).reshape(-1), kc.reshape(-1), vc.reshape(-1),
                                  n_layers, tree_layer_stride, cache_layer_stride, hkv, d, out)
     return st, out
+
+
+# ------------------------------------------------------------------------------- paged caches
+# A paged cache holds each request's positions in fixed-size pages of a shared pool: logical
+# position t of request r lives at pool slot block_table[r, t // P] * P + t % P (pool arrays
+# [num_pages * P][hkv][d]).  The oracle's paged calls are the contiguous definitions applied to
+# the logical caches gathered through the block tables (a plain index gather).
+
+def page_slots(block_table, page_size, r, t):
+    """Pool slots of logical positions t (array) of request r."""
+    t = np.asarray(t, dtype=np.int64)
+    return np.asarray(block_table)[r, t // page_size].astype(np.int64) * page_size + t % page_size
+
+
+def attention_paged(cu_nodes, parent, kv_len, block_table, page_size, q, k_tree, v_tree, k_pool,
+                    v_pool, hq, hkv, scale, rows=None, nthreads=0):
+    """Tree attention over a paged cache: each request's first kv_len[r] positions are gathered
+    through its block table into a contiguous cache, then `attention` runs on it."""
+    kp, vp = _u16(k_pool), _u16(v_pool)
+    B = len(kv_len)
+    base = np.zeros(B, dtype=np.int64)
+    ks, vs = [], []
+    off = 0
+    for r in range(B):
+        sl = page_slots(block_table, page_size, r, np.arange(int(kv_len[r])))
+        ks.append(kp[sl])
+        vs.append(vp[sl])
+        base[r] = off
+        off += int(kv_len[r])
+    kc = np.concatenate(ks) if off else np.zeros((1,) + kp.shape[1:], np.uint16)
+    vc = np.concatenate(vs) if off else np.zeros((1,) + vp.shape[1:], np.uint16)
+    return attention(cu_nodes, parent, kv_len, base, q, k_tree, v_tree, kc, vc, hq, hkv, scale,
+                     rows=rows, nthreads=nthreads)
+
+
+def kv_compact_paged(cu_nodes, kv_len, block_table, page_size, slot_cap, accept_len, path,
+                     k_tree, v_tree, k_pool, v_pool, n_layers):
+    """Compaction into a paged cache, in place on the uint16 pools [n_layers][slots][hkv][d]:
+    pool[slot(kv_len[r] + k)] <- tree[cu_nodes[r] + path[r][k]], k = 0..a.  A request whose
+    rows would pass slot_cap[r] is left untouched.  Returns (status, kv_len_out)."""
+    cu = _i32(cu_nodes)
+    B = len(cu) - 1
+    kt, vt = _u16(k_tree), _u16(v_tree)
+    out = np.asarray(kv_len, dtype=np.int32).copy()
+    status = 0
+    for r in range(B):
+        n = int(cu[r + 1] - cu[r])
+        a, L = int(accept_len[r]), int(kv_len[r])
+        pr = np.asarray(path)[r, :a + 1]
+        if n < 1 or a < 0 or a >= n or (pr < 0).any() or (pr >= n).any():
+            status = status or EINVAL
+            continue
+        if L + a + 1 > int(slot_cap[r]):
+            status = status or ENOSPACE
+            continue
+        dst = page_slots(block_table, page_size, r, np.arange(L, L + a + 1))
+        src = int(cu[r]) + pr
+        for layer in range(n_layers):
+            k_pool[layer, dst] = kt[layer, src]
+            v_pool[layer, dst] = vt[layer, src]
+        out[r] = L + a + 1
+    return status, out
 
 
 # --------------------------------------------------------------------------- per-request passes

@@ -619,6 +619,63 @@ def test_kv_compact_equals_numpy_gather():
     assert np.array_equal(newlen, kv_len + a + 1)
 
 
+# ------------------------------------------------------------------------------ paged caches
+def test_paged_attention_is_independent_of_page_placement():
+    """The same logical caches scattered over shuffled pages of sizes 16 and 64 give bit-for-bit
+    the contiguous attention (same keys, same order)."""
+    wl = wlm.generate("tiny", B=4, n_nodes=[1, 6, 16, 9], depth=4, depth_min=2, branch=None,
+                      width=8, kv_len=[0, 17, 100, 63], hidden=256, vocab=512)
+    sc = oracle.scale_of(wl.head_dim)
+    ref, lref, st = oracle.attention(wl.cu_nodes, wl.parent, wl.kv_len, wl.slot_base, wl.q,
+                                     wl.k_tree, wl.v_tree, wl.k_cache, wl.v_cache, wl.hq, wl.hkv,
+                                     sc)
+    assert st == 0
+    for P in (16, 64):
+        pc = wlm.paged(wl, P, seed=P)
+        out, lse, st = oracle.attention_paged(wl.cu_nodes, wl.parent, wl.kv_len, pc.block_table,
+                                              P, wl.q, wl.k_tree, wl.v_tree, pc.k_pool,
+                                              pc.v_pool, wl.hq, wl.hkv, sc)
+        assert st == 0 and np.array_equal(out, ref) and np.array_equal(lse, lref)
+
+
+def test_page_slots_by_hand():
+    bt = np.array([[5, 2, 7], [0, 3, -1]], dtype=np.int32)
+    assert list(oracle.page_slots(bt, 4, 0, [0, 3, 4, 9])) == [20, 23, 8, 29]
+    assert list(oracle.page_slots(bt, 4, 1, [0, 5])) == [0, 13]
+
+
+def test_paged_compaction_equals_contiguous_compaction_of_the_logical_cache():
+    """Compacting into pages, then gathering each request's logical cache back through its block
+    table, equals compacting the contiguous logical cache."""
+    wl = wlm.generate("tiny", B=3, n_nodes=[5, 16, 2], depth=4, depth_min=2, branch=None,
+                      width=8, kv_len=[14, 33, 0], hidden=256, vocab=512)
+    P = 16
+    pc = wlm.paged(wl, P, seed=1)
+    a = np.array([2, 3, 1], dtype=np.int32)
+    path = np.full((3, 64), -1, dtype=np.int32)
+    path[0, :3] = [0, 1, 3]
+    path[1, :4] = [0, 2, 5, 9]
+    path[2, :2] = [0, 1]
+    kt = oracle._u16(wl.k_tree)[None]
+    vt = oracle._u16(wl.v_tree)[None]
+    kpool = oracle._u16(pc.k_pool)[None].copy()
+    vpool = oracle._u16(pc.v_pool)[None].copy()
+    st, newlen = oracle.kv_compact_paged(wl.cu_nodes, wl.kv_len, pc.block_table, P, pc.slot_cap,
+                                         a, path, kt, vt, kpool, vpool, 1)
+    assert st == 0 and list(newlen) == list(wl.kv_len + a + 1)
+    ck, cv = oracle._u16(wl.k_cache).copy(), oracle._u16(wl.v_cache).copy()
+    d = wl.hkv * wl.head_dim
+    st2, newlen2 = oracle.kv_compact(wl.cu_nodes, wl.kv_len, wl.slot_base, wl.slot_cap, a, path,
+                                     wl.k_tree, wl.v_tree, ck, cv, 1, wl.n_total * d,
+                                     ck.shape[0] * d, wl.hkv, wl.head_dim)
+    assert st2 == 0 and list(newlen2) == list(newlen)
+    for r in range(3):
+        t = np.arange(int(newlen[r]))
+        sl = oracle.page_slots(pc.block_table, P, r, t)
+        b = int(wl.slot_base[r])
+        assert np.array_equal(kpool[0, sl], ck[b + t]) and np.array_equal(vpool[0, sl], cv[b + t])
+
+
 def test_kv_compact_capacity_overflow_leaves_request_untouched():
     cu = np.array([0, 4], dtype=np.int32)
     kv_len = np.array([10], dtype=np.int32)
