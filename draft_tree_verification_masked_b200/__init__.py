@@ -29,6 +29,7 @@ __all__ = [
     "EtreeError", "Batch", "make_batch", "lib", "library_path", "etree_workspace_size",
     "etree_workspace_init", "etree_verify_attn", "etree_verify_attn_noalloc",
     "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact",
+    "etree_verify_attn_paged", "etree_kv_compact_paged",
     "etree_device_status", "etree_strerror", "etree_version", "etree_attn_plan", "STATUS",
 ]
 
@@ -41,6 +42,7 @@ DETAIL = {0: "none", 1: "bad parent", 2: "bad node count", 3: "bad kv_len", 4: "
           5: "not a chain", 6: "bad path", 7: "attention wait", 8: "gemm wait", 9: "bad token"}
 
 EXPORTS = ["etree_workspace_size", "etree_workspace_init", "etree_verify_attn",
+           "etree_verify_attn_paged", "etree_kv_compact_paged",
            "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact", "etree_device_status", "etree_strerror",
            "etree_version", "etree_last_error", "etree_attn_plan", "etree_verify_attn_noalloc"]
 
@@ -92,6 +94,14 @@ def lib():
     L.etree_kv_compact.argtypes = [bp, vp, vp, vp, vp, vp, vp, C.c_int, i64, i64, C.c_int,
                                    C.c_int, vp, vp, C.c_size_t, vp]
     L.etree_kv_compact.restype = C.c_int
+    L.etree_verify_attn_paged.argtypes = [bp, vp, C.c_int32, C.c_int32, vp, vp, vp, vp, vp, i64,
+                                          C.c_int, C.c_int, C.c_int, f32, vp, vp, vp, C.c_size_t,
+                                          vp]
+    L.etree_verify_attn_paged.restype = C.c_int
+    L.etree_kv_compact_paged.argtypes = [bp, vp, C.c_int32, C.c_int32, vp, vp, vp, vp, vp, vp,
+                                         i64, C.c_int, i64, i64, C.c_int, C.c_int, vp, vp,
+                                         C.c_size_t, vp]
+    L.etree_kv_compact_paged.restype = C.c_int
     L.etree_device_status.argtypes = [vp, vp, C.POINTER(i32)]
     L.etree_device_status.restype = C.c_int
     L.etree_strerror.argtypes = [C.c_int]
@@ -230,6 +240,40 @@ def etree_lmhead_accept_tree(batch: Batch, hidden, w_lm, temperature: float, q_d
         _ptr(accept_len, torch.int32, "accept_len"), _ptr(path, torch.int32, "path"),
         _ptr(out_tokens, torch.int32, "out_tokens"), _ptr(zbuf, torch.float32, "zbuf"), rows,
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
+    return _check(st) if check else st
+
+
+def etree_verify_attn_paged(batch: Batch, block_table, page_size: int, q, k_tree, v_tree,
+                            k_pool, v_pool, scale: float, out, lse, workspace, stream=None,
+                            check: bool = True) -> int:
+    """block_table: int32 [B, max_pages] device tensor; pools [num_pages * page_size, hkv, d]."""
+    bf = torch.bfloat16
+    hq, d = q.shape[1], q.shape[2]
+    hkv = k_tree.shape[1]
+    num_pages = k_pool.shape[0] // int(page_size)
+    st = lib().etree_verify_attn_paged(
+        C.byref(batch), _ptr(block_table, torch.int32, "block_table"), block_table.shape[1],
+        int(page_size), _ptr(q, bf, "q"), _ptr(k_tree, bf, "k_tree"), _ptr(v_tree, bf, "v_tree"),
+        _ptr(k_pool, bf, "k_pool"), _ptr(v_pool, bf, "v_pool"), num_pages, hq, hkv, d,
+        float(scale), _ptr(out, bf, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
+    return _check(st) if check else st
+
+
+def etree_kv_compact_paged(batch: Batch, block_table, page_size: int, accept_len, path, k_tree,
+                           v_tree, k_pool, v_pool, num_pages: int, n_layers: int,
+                           tree_layer_stride: int, cache_layer_stride: int, kv_len_out,
+                           workspace, stream=None, check: bool = True) -> int:
+    bf = torch.bfloat16
+    hkv, d = k_tree.shape[-2], k_tree.shape[-1]
+    st = lib().etree_kv_compact_paged(
+        C.byref(batch), _ptr(block_table, torch.int32, "block_table"), block_table.shape[1],
+        int(page_size), _ptr(accept_len, torch.int32, "accept_len"),
+        _ptr(path, torch.int32, "path"), _ptr(k_tree, bf, "k_tree"), _ptr(v_tree, bf, "v_tree"),
+        _ptr(k_pool, bf, "k_pool"), _ptr(v_pool, bf, "v_pool"), int(num_pages), int(n_layers),
+        int(tree_layer_stride), int(cache_layer_stride), hkv, d,
+        _ptr(kv_len_out, torch.int32, "kv_len_out"), _ptr(workspace, torch.uint8, "workspace"),
+        workspace.numel(), _stream(stream))
     return _check(st) if check else st
 
 

@@ -360,11 +360,40 @@ etree_status etree_device_status(void* workspace, void* stream, int32_t* detail)
   return static_cast<etree_status>(h[0]);
 }
 
-etree_status etree_verify_attn(const etree_batch* b, const uint16_t* q, const uint16_t* k_tree,
-                               const uint16_t* v_tree, const uint16_t* k_cache,
-                               const uint16_t* v_cache, int64_t cache_slots, int hq, int hkv,
-                               int head_dim, float scale, uint16_t* out, float* lse,
-                               void* workspace, size_t workspace_bytes, void* stream) {
+// A paged cache: the block table [B][max_pages] and the page size (a power of two >= 16).
+struct PagedArgs {
+  const int32_t* block_table;
+  int32_t max_pages;
+  int32_t page_size;
+};
+
+static etree_status check_paged(const PagedArgs* pg, int64_t num_pages) {
+  if (!pg) return ETREE_OK;
+  if (!pg->block_table || ((uintptr_t)pg->block_table & 3))
+    return fail(ETREE_EINVAL, "block_table is NULL or misaligned");
+  if (pg->max_pages < 1) return fail(ETREE_EINVAL, "max_pages=%d", pg->max_pages);
+  const int P = pg->page_size;
+  if (P < 16 || P > (1 << 20) || (P & (P - 1)))
+    return fail(ETREE_EINVAL, "page_size=%d: need a power of two in [16, 2^20]", P);
+  if (num_pages < 1 || num_pages * P > INT32_MAX)
+    return fail(ETREE_EINVAL, "num_pages=%lld: need 1 <= num_pages * page_size < 2^31",
+                (long long)num_pages);
+  return ETREE_OK;
+}
+
+static int log2i(int x) {
+  int k = 0;
+  while ((1 << k) < x) ++k;
+  return k;
+}
+
+static etree_status verify_attn_impl(const etree_batch* b, const uint16_t* q,
+                                     const uint16_t* k_tree, const uint16_t* v_tree,
+                                     const uint16_t* k_cache, const uint16_t* v_cache,
+                                     int64_t cache_slots, int hq, int hkv, int head_dim,
+                                     float scale, uint16_t* out, float* lse,
+                                     const PagedArgs* pg, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
   etree_status st = check_batch(b);
   if (st) return st;
   if (head_dim != ETREE_HEAD_DIM)
@@ -382,10 +411,12 @@ etree_status etree_verify_attn(const etree_batch* b, const uint16_t* q, const ui
   if ((st = check_ws(b, hq, hkv, 0, 0, workspace, workspace_bytes))) return st;
 
   const AttnPlan pl = plan_attn(b, hq, hkv);
+  if (pg && !pl.tc) return fail(ETREE_EUNSUPPORTED, "paged caches need the tcgen05 kernel");
   CUtensorMap kc, vc, kt, vt;
   const uint32_t kb = (uint32_t)pl.keys;
-  if ((st = get_map(k_cache, 3, 128, hkv, cache_slots, 64, 1, kb, &kc))) return st;
-  if ((st = get_map(v_cache, 3, 128, hkv, cache_slots, 64, 1, kb, &vc))) return st;
+  const uint32_t cbox = pg ? (uint32_t)std::min(pl.keys, pg->page_size) : kb;
+  if ((st = get_map(k_cache, 3, 128, hkv, cache_slots, 64, 1, cbox, &kc))) return st;
+  if ((st = get_map(v_cache, 3, 128, hkv, cache_slots, 64, 1, cbox, &vc))) return st;
   if ((st = get_map(k_tree, 3, 128, hkv, b->n_total, 64, 1, kb, &kt))) return st;
   if ((st = get_map(v_tree, 3, 128, hkv, b->n_total, 64, 1, kb, &vt))) return st;
 
@@ -414,6 +445,10 @@ etree_status etree_verify_attn(const etree_batch* b, const uint16_t* q, const ui
   p.tps = pl.tps;
   p.keys = pl.keys;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.block_table = pg ? pg->block_table : nullptr;
+  p.max_pages = pg ? pg->max_pages : 0;
+  p.page_shift = pg ? log2i(pg->page_size) : 0;
+  p.cache_box = (int)cbox;
   cudaError_t e;
   // with many requests of mixed lengths, dispatch the longest first
   p.order = nullptr;
@@ -433,6 +468,29 @@ etree_status etree_verify_attn(const etree_batch* b, const uint16_t* q, const ui
                     static_cast<cudaStream_t>(stream));
   }
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_verify_attn launch");
+}
+
+etree_status etree_verify_attn(const etree_batch* b, const uint16_t* q, const uint16_t* k_tree,
+                               const uint16_t* v_tree, const uint16_t* k_cache,
+                               const uint16_t* v_cache, int64_t cache_slots, int hq, int hkv,
+                               int head_dim, float scale, uint16_t* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  return verify_attn_impl(b, q, k_tree, v_tree, k_cache, v_cache, cache_slots, hq, hkv, head_dim,
+                          scale, out, lse, nullptr, workspace, workspace_bytes, stream);
+}
+
+etree_status etree_verify_attn_paged(const etree_batch* b, const int32_t* block_table,
+                                     int32_t max_pages, int32_t page_size, const uint16_t* q,
+                                     const uint16_t* k_tree, const uint16_t* v_tree,
+                                     const uint16_t* k_pool, const uint16_t* v_pool,
+                                     int64_t num_pages, int hq, int hkv, int head_dim,
+                                     float scale, uint16_t* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  const PagedArgs pg{block_table, max_pages, page_size};
+  etree_status st = check_paged(&pg, num_pages);
+  if (st) return st;
+  return verify_attn_impl(b, q, k_tree, v_tree, k_pool, v_pool, num_pages * page_size, hq, hkv,
+                          head_dim, scale, out, lse, &pg, workspace, workspace_bytes, stream);
 }
 
 // The caller's logit buffer of the branching-tree sampler (etree_lmhead_accept_tree).
@@ -602,13 +660,13 @@ etree_status etree_lmhead_accept_tree(const etree_batch* b, const uint16_t* hidd
                             stream);
 }
 
-etree_status etree_kv_compact(const etree_batch* b, const int32_t* accept_len,
-                              const int32_t* path, const uint16_t* k_tree,
-                              const uint16_t* v_tree, uint16_t* k_cache, uint16_t* v_cache,
-                              int n_layers, int64_t tree_layer_stride,
-                              int64_t cache_layer_stride, int hkv, int head_dim,
-                              int32_t* kv_len_out, void* workspace, size_t workspace_bytes,
-                              void* stream) {
+static etree_status kv_compact_impl(const etree_batch* b, const int32_t* accept_len,
+                                    const int32_t* path, const uint16_t* k_tree,
+                                    const uint16_t* v_tree, uint16_t* k_cache,
+                                    uint16_t* v_cache, int n_layers, int64_t tree_layer_stride,
+                                    int64_t cache_layer_stride, int hkv, int head_dim,
+                                    int32_t* kv_len_out, const PagedArgs* pg, int64_t pool_slots,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
   etree_status st = check_batch(b);
   if (st) return st;
   if (head_dim != ETREE_HEAD_DIM)
@@ -624,6 +682,8 @@ etree_status etree_kv_compact(const etree_batch* b, const int32_t* accept_len,
   if (n_layers > 1 && (tree_layer_stride < row * b->n_total || cache_layer_stride < row ||
                        tree_layer_stride % 8 || cache_layer_stride % 8))
     return fail(ETREE_EINVAL, "layer strides must cover a layer and be multiples of 8");
+  if (pg && n_layers > 1 && cache_layer_stride < row * pool_slots)
+    return fail(ETREE_EINVAL, "cache_layer_stride must cover a layer's page pool");
   if ((st = check_ws(b, 0, 0, 0, 0, workspace, workspace_bytes))) return st;
   CompactParams p{};
   p.cu_nodes = b->cu_nodes;
@@ -644,8 +704,41 @@ etree_status etree_kv_compact(const etree_batch* b, const int32_t* accept_len,
   p.tree_layer_stride16 = tree_layer_stride / 8;
   p.cache_layer_stride16 = cache_layer_stride / 8;
   p.row16 = (int)(row / 8);
+  p.block_table = pg ? pg->block_table : nullptr;
+  p.max_pages = pg ? pg->max_pages : 0;
+  p.page_shift = pg ? log2i(pg->page_size) : 0;
+  p.cache_slots = pool_slots;
   cudaError_t e = launch_compact(p, sm_count(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_kv_compact launch");
+}
+
+etree_status etree_kv_compact(const etree_batch* b, const int32_t* accept_len,
+                              const int32_t* path, const uint16_t* k_tree,
+                              const uint16_t* v_tree, uint16_t* k_cache, uint16_t* v_cache,
+                              int n_layers, int64_t tree_layer_stride,
+                              int64_t cache_layer_stride, int hkv, int head_dim,
+                              int32_t* kv_len_out, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  return kv_compact_impl(b, accept_len, path, k_tree, v_tree, k_cache, v_cache, n_layers,
+                         tree_layer_stride, cache_layer_stride, hkv, head_dim, kv_len_out,
+                         nullptr, 0, workspace, workspace_bytes, stream);
+}
+
+etree_status etree_kv_compact_paged(const etree_batch* b, const int32_t* block_table,
+                                    int32_t max_pages, int32_t page_size,
+                                    const int32_t* accept_len, const int32_t* path,
+                                    const uint16_t* k_tree, const uint16_t* v_tree,
+                                    uint16_t* k_pool, uint16_t* v_pool, int64_t num_pages,
+                                    int n_layers, int64_t tree_layer_stride,
+                                    int64_t cache_layer_stride, int hkv, int head_dim,
+                                    int32_t* kv_len_out, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  const PagedArgs pg{block_table, max_pages, page_size};
+  etree_status st = check_paged(&pg, num_pages);
+  if (st) return st;
+  return kv_compact_impl(b, accept_len, path, k_tree, v_tree, k_pool, v_pool, n_layers,
+                         tree_layer_stride, cache_layer_stride, hkv, head_dim, kv_len_out, &pg,
+                         num_pages * page_size, workspace, workspace_bytes, stream);
 }
 
 // Tree attention without a caller workspace: the split partials and the status words live in

@@ -81,8 +81,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int n = p.cu_nodes[r + 1] - base;
   const int L = p.kv_len[r];
   const int64_t sbase = p.slot_base[r];
-  if (n < 1 || n > p.n_max || L < 0 || L > p.kv_len_max || sbase < 0 ||
-      sbase + L > p.cache_slots) {
+  const bool paged = p.block_table != nullptr;
+  if (n < 1 || n > p.n_max || L < 0 || L > p.kv_len_max ||
+      (!paged && (sbase < 0 || sbase + L > p.cache_slots)) ||
+      (paged && L > ((int64_t)p.max_pages << p.page_shift))) {
     if (threadIdx.x == 0 && s == 0 && mb == 0 && kvh == 0)
       report(p.ws, ETREE_EDEVICE, (n < 1 || n > p.n_max) ? DET_BAD_NODES : DET_KV_LEN);
     return;
@@ -181,12 +183,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         uint8_t* dst = sKV + st * Sh::kKV;
         mbar_arrive_expect_tx(&sh->kv_full[st], Sh::kKV);
-        if (t < nt_cache) {
+        if (t < nt_cache && !paged) {
           const int32_t slot = static_cast<int32_t>(sbase + (int64_t)t * KEYS);
           tma_load_3d(dst, &tm_kc, &sh->kv_full[st], 0, kvh, slot);
           tma_load_3d(dst + Sh::kBox, &tm_kc, &sh->kv_full[st], 64, kvh, slot);
           tma_load_3d(dst + 2 * Sh::kBox, &tm_vc, &sh->kv_full[st], 0, kvh, slot);
           tma_load_3d(dst + 3 * Sh::kBox, &tm_vc, &sh->kv_full[st], 64, kvh, slot);
+        } else if (t < nt_cache) {
+          // paged: KEYS / cache_box boxes per half, each inside one page.  An entry outside
+          // the pool is reported; its box then lies past the tensor and TMA fills zeros.
+          const int cb = p.cache_box, P = 1 << p.page_shift;
+          const int32_t* bt = p.block_table + (size_t)r * p.max_pages;
+          for (int i = 0; i < KEYS / cb; ++i) {
+            const int pos = t * KEYS + i * cb;
+            const int pi = pos >> p.page_shift;
+            int32_t page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+            if (page < 0 || (int64_t)page * P >= p.cache_slots) {
+              if (pos < L) report(p.ws, ETREE_EDEVICE, DET_BAD_PAGE);
+              page = (int32_t)(p.cache_slots >> p.page_shift);
+            }
+            const int32_t slot = page * P + (pos & (P - 1));
+            const uint32_t off = (uint32_t)(i * cb * 128);
+            tma_load_3d(dst + off, &tm_kc, &sh->kv_full[st], 0, kvh, slot);
+            tma_load_3d(dst + Sh::kBox + off, &tm_kc, &sh->kv_full[st], 64, kvh, slot);
+            tma_load_3d(dst + 2 * Sh::kBox + off, &tm_vc, &sh->kv_full[st], 0, kvh, slot);
+            tma_load_3d(dst + 3 * Sh::kBox + off, &tm_vc, &sh->kv_full[st], 64, kvh, slot);
+          }
         } else {
           const int node = base + (t - nt_cache) * KEYS;
           tma_load_3d(dst, &tm_kt, &sh->kv_full[st], 0, kvh, node);

@@ -32,6 +32,7 @@ enum Detail : int32_t {
   DET_WAIT_GEMM = 8,        // a bounded wait gave up in the LM-head GEMM
   DET_BAD_TOKEN = 9,        // a token id outside [0, vocab)
   DET_ZBUF = 10,            // more branching tree nodes than rows in the caller's logit buffer
+  DET_BAD_PAGE = 11,        // a block-table entry outside [0, num_pages) for a used position
 };
 
 __device__ __forceinline__ void report(WsHeader* ws, int32_t code, int32_t detail) {

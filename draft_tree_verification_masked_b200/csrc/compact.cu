@@ -7,6 +7,7 @@
 // step's tree K/V, in path order) are copied to the request's next cache slots, layer by layer.
 //
 // The copy is a bit copy and is HBM-bound: every byte moved is read once and written once.
+// With a paged cache the destination of each row goes through the request's block table.
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -20,8 +21,8 @@ namespace etree {
 // tensor (K, V), four rows in flight per thread.
 __global__ void __launch_bounds__(256) kv_compact_kernel(CompactParams p, int layers_per_cta) {
   __shared__ int src_s[64];
-  __shared__ int rows_s, code_s, detail_s, bad_s;
-  __shared__ long long dst_s;
+  __shared__ long long dst_s[64];
+  __shared__ int rows_s, code_s, detail_s, bad_s, badpage_s;
   const int r = blockIdx.x;
   const int l0 = blockIdx.y * layers_per_cta;
   const int l1 = min(p.n_layers, l0 + layers_per_cta);
@@ -43,16 +44,26 @@ __global__ void __launch_bounds__(256) kv_compact_kernel(CompactParams p, int la
     detail_s = detail;
     rows_s = code == ETREE_OK ? a + 1 : 0;
     bad_s = 0;
-    dst_s = p.slot_base[r] + L;
+    badpage_s = 0;
   }
   __syncthreads();
   const int rows0 = rows_s;
-  if (tid < rows0) {                                   // path entries, read in parallel
+  if (tid < rows0) {                                   // path entries and destinations
     const int base = p.cu_nodes[r];
     const int n = p.cu_nodes[r + 1] - base;
     const int j = p.path[(size_t)r * ETREE_PATH_STRIDE + tid];
     if (j < 0 || j >= n) atomicOr(&bad_s, 1);
     src_s[tid] = base + j;
+    const long long pos = (long long)p.kv_len[r] + tid;
+    if (!p.block_table) {
+      dst_s[tid] = p.slot_base[r] + pos;
+    } else {
+      const long long pi = pos >> p.page_shift;
+      const int page = pi < p.max_pages ? p.block_table[(size_t)r * p.max_pages + pi] : -1;
+      const long long slot = ((long long)page << p.page_shift) + (pos & ((1 << p.page_shift) - 1));
+      if (page < 0 || slot >= p.cache_slots) atomicOr(&badpage_s, 1);
+      dst_s[tid] = slot;
+    }
   }
   __syncthreads();
   if (tid == 0 && blockIdx.y == 0) {
@@ -60,13 +71,15 @@ __global__ void __launch_bounds__(256) kv_compact_kernel(CompactParams p, int la
     if (code == ETREE_OK && bad_s) {
       code = ETREE_EDEVICE;
       detail = DET_BAD_PATH;
+    } else if (code == ETREE_OK && badpage_s) {
+      code = ETREE_EDEVICE;
+      detail = DET_BAD_PAGE;
     }
     if (code != ETREE_OK) report(p.ws, code, detail);
     p.kv_len_out[r] = code == ETREE_OK ? p.kv_len[r] + rows0 : p.kv_len[r];
   }
-  const int rows = bad_s ? 0 : rows0;
+  const int rows = (bad_s || badpage_s) ? 0 : rows0;
   if (rows == 0) return;
-  const long long dst0 = dst_s;
   const int w16 = p.row16;                            // 16-byte words per row
   for (int layer = l0; layer < l1; ++layer) {
     const uint4* kt = p.k_tree + (size_t)layer * p.tree_layer_stride16;
@@ -84,12 +97,12 @@ __global__ void __launch_bounds__(256) kv_compact_kernel(CompactParams p, int la
         uint4 v1 = __ldg(src + (size_t)src_s[k + 1] * w16 + cc);
         uint4 v2 = __ldg(src + (size_t)src_s[k + 2] * w16 + cc);
         uint4 v3 = __ldg(src + (size_t)src_s[k + 3] * w16 + cc);
-        dst[(size_t)(dst0 + k) * w16 + cc] = v0;
-        dst[(size_t)(dst0 + k + 1) * w16 + cc] = v1;
-        dst[(size_t)(dst0 + k + 2) * w16 + cc] = v2;
-        dst[(size_t)(dst0 + k + 3) * w16 + cc] = v3;
+        dst[(size_t)dst_s[k] * w16 + cc] = v0;
+        dst[(size_t)dst_s[k + 1] * w16 + cc] = v1;
+        dst[(size_t)dst_s[k + 2] * w16 + cc] = v2;
+        dst[(size_t)dst_s[k + 3] * w16 + cc] = v3;
       }
-      for (; k < rows; ++k) dst[(size_t)(dst0 + k) * w16 + cc] = __ldg(src + (size_t)src_s[k] * w16 + cc);
+      for (; k < rows; ++k) dst[(size_t)dst_s[k] * w16 + cc] = __ldg(src + (size_t)src_s[k] * w16 + cc);
     }
   }
 }

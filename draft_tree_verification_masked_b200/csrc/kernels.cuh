@@ -22,6 +22,11 @@ struct AttnParams {
   int keys;                 // keys per KV tile (the tree takes ceil(n / keys) tiles at the end)
   const int32_t* order;     // [B] requests by decreasing KV length (dispatch order), or null
   float scale_log2;
+  // Paged cache (block_table != null): position t of request r is pool slot
+  // block_table[r * max_pages + t / 2^page_shift] * 2^page_shift + t % 2^page_shift; cache
+  // tiles are loaded in boxes of cache_box rows (KEYS, or the page size when pages are smaller).
+  const int32_t* block_table;
+  int max_pages, page_shift, cache_box;
 };
 cudaError_t launch_attn(const CUtensorMap& kc, const CUtensorMap& vc, const CUtensorMap& kt,
                         const CUtensorMap& vt, const AttnParams& p, int nw, int stages,
@@ -111,6 +116,12 @@ struct CompactParams {
   int B, n_max, n_layers;
   int64_t tree_layer_stride16, cache_layer_stride16;
   int row16;
+  // Paged cache (block_table != null): destination position t of request r is pool slot
+  // block_table[r * max_pages + t / 2^page_shift] * 2^page_shift + t % 2^page_shift, and
+  // slot_base is unused; pool slots per layer: cache_slots.
+  const int32_t* block_table;
+  int max_pages, page_shift;
+  int64_t cache_slots;
 };
 cudaError_t launch_compact(const CompactParams& p, int sms, cudaStream_t s);
 

@@ -10,9 +10,9 @@ import torch
 
 import numpy as np
 
-from . import (etree_device_status, etree_kv_compact, etree_lmhead_accept,
-               etree_lmhead_accept_tree, etree_verify_attn, etree_workspace_init,
-               etree_workspace_size, make_batch)
+from . import (etree_device_status, etree_kv_compact, etree_kv_compact_paged,
+               etree_lmhead_accept, etree_lmhead_accept_tree, etree_verify_attn,
+               etree_verify_attn_paged, etree_workspace_init, etree_workspace_size, make_batch)
 
 
 def branching_nodes(wl) -> int:
@@ -27,10 +27,12 @@ def branching_nodes(wl) -> int:
 
 class DeviceStep:
     """tree: None picks the branching-tree sampler (etree_lmhead_accept_tree) when T > 0 and a
-    node has two or more children; zbuf_rows overrides the size of its logit buffer."""
+    node has two or more children; zbuf_rows overrides the size of its logit buffer.
+    page_size: lay the caches out in pages of that many tokens at shuffled pool pages and use
+    the paged attention and compaction calls (the pools replace k_cache / v_cache)."""
 
     def __init__(self, wl, device: str = "cuda", n_layers: int = 1, pin: bool = False,
-                 tree=None, zbuf_rows=None):
+                 tree=None, zbuf_rows=None, page_size=None):
         self.wl = wl
         self.device = device
         dev = torch.device(device)
@@ -47,14 +49,19 @@ class DeviceStep:
         self.tokens = up(wl.tokens, i32)
         self.kv_len = up(wl.kv_len, i32)
         self.slot_base = up(wl.slot_base, torch.int64)
-        self.slot_cap = up(wl.slot_cap, i32)
+        self.paged = None
+        if page_size:
+            from .workload import paged
+            self.paged = paged(wl, int(page_size))
+            self.block_table = up(self.paged.block_table, i32)
+        self.slot_cap = up(self.paged.slot_cap if self.paged else wl.slot_cap, i32)
         self.batch = make_batch(self.cu_nodes, self.parent, self.tokens, self.kv_len,
                                 self.slot_base, self.slot_cap, wl.n_max, wl.kv_len_max)
         self.q = up(wl.q)
         self.k_tree = up(wl.k_tree)
         self.v_tree = up(wl.v_tree)
-        self.k_cache = up(wl.k_cache)
-        self.v_cache = up(wl.v_cache)
+        self.k_cache = up(self.paged.k_pool if self.paged else wl.k_cache)
+        self.v_cache = up(self.paged.v_pool if self.paged else wl.v_cache)
         self.hidden = up(wl.hidden)
         self.w_lm = up(wl.w_lm)
         self.q_draft = up(wl.q_draft) if wl.q_draft is not None else None
@@ -93,6 +100,11 @@ class DeviceStep:
 
     # --- the three calls
     def attn(self, stream=None):
+        if self.paged:
+            etree_verify_attn_paged(self.batch, self.block_table, self.paged.page_size, self.q,
+                                    self.k_tree, self.v_tree, self.k_cache, self.v_cache,
+                                    self.scale, self.out, self.lse, self.ws, stream)
+            return
         etree_verify_attn(self.batch, self.q, self.k_tree, self.v_tree, self.k_cache,
                           self.v_cache, self.scale, self.out, self.lse, self.ws, stream)
 
@@ -107,6 +119,13 @@ class DeviceStep:
                             self.out_tokens, self.node_argmax, self.node_gap, self.ws, stream)
 
     def compact(self, stream=None):
+        if self.paged:
+            etree_kv_compact_paged(self.batch, self.block_table, self.paged.page_size,
+                                   self.accept_len, self.path, self.kt_layers, self.vt_layers,
+                                   self.kc_layers, self.vc_layers, self.paged.num_pages,
+                                   self.n_layers, self.tree_layer_stride,
+                                   self.cache_layer_stride, self.kv_len_out, self.ws, stream)
+            return
         etree_kv_compact(self.batch, self.accept_len, self.path, self.kt_layers, self.vt_layers,
                          self.kc_layers, self.vc_layers, self.n_layers, self.tree_layer_stride,
                          self.cache_layer_stride, self.kv_len_out, self.ws, stream)

@@ -136,6 +136,28 @@ etree_status etree_verify_attn_noalloc(const etree_batch *batch, const uint16_t 
                                        int32_t *status_out, void *stream);
 
 /*
+ * Tree attention over a paged KV cache (block tables, as serving engines hold KV).  Same result
+ * as etree_verify_attn on the logical caches: position t (0 <= t < kv_len[r]) of request r lives
+ * at pool slot  block_table[r * max_pages + t / page_size] * page_size + t % page_size  of
+ * k_pool / v_pool, each [num_pages * page_size][hkv][head_dim] bf16 (16-byte aligned).
+ * batch->slot_base is not used.  page_size is a power of two in [16, 2^20]; pages smaller than
+ * the kernel's key tile are loaded page by page.  block_table is a device int32 array
+ * [B][max_pages]; only entries covering positions below kv_len[r] are read for keys.  An entry
+ * outside [0, num_pages) records ETREE_EDEVICE (detail 11) and its keys read as zeros;
+ * kv_len[r] > max_pages * page_size records ETREE_EDEVICE (detail 3).  Needs the tcgen05
+ * kernel (ETREE_ATTN=mma returns ETREE_EUNSUPPORTED).  Other arguments, workspace and errors as
+ * etree_verify_attn, with num_pages * page_size in place of cache_slots.
+ */
+etree_status etree_verify_attn_paged(const etree_batch *batch, const int32_t *block_table,
+                                     int32_t max_pages, int32_t page_size, const uint16_t *q,
+                                     const uint16_t *k_tree, const uint16_t *v_tree,
+                                     const uint16_t *k_pool, const uint16_t *v_pool,
+                                     int64_t num_pages, int hq, int hkv, int head_dim,
+                                     float scale, uint16_t *out, float *lse, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
+/*
+ * LM head + acceptance.  z = hidden W^T/*
  * LM head + acceptance.  z = hidden W^T (fp32 accumulate over bf16 inputs) for every node row.
  *  T == 0 (greedy): t*(u) = argmax z_u (lowest id on ties).  From the root, repeatedly move to
  *    the lowest-index child whose token equals t*(current); the node where no child matches
@@ -212,6 +234,26 @@ etree_status etree_kv_compact(const etree_batch *batch, const int32_t *accept_le
                               void *stream);
 
 /*
+ * KV compaction into a paged cache: as etree_kv_compact, with destination position
+ * t = kv_len[r] + k going to pool slot block_table[r * max_pages + t / page_size] * page_size +
+ * t % page_size (layout and page rules of etree_verify_attn_paged).  slot_cap[r] is the
+ * request's mapped capacity in tokens; a request whose new rows would pass it is left untouched
+ * with ETREE_ENOSPACE, and one whose destination page entry lies outside [0, num_pages) is left
+ * untouched with ETREE_EDEVICE (detail 11).  For n_layers > 1, cache_layer_stride must cover
+ * num_pages * page_size rows.
+ */
+etree_status etree_kv_compact_paged(const etree_batch *batch, const int32_t *block_table,
+                                    int32_t max_pages, int32_t page_size,
+                                    const int32_t *accept_len, const int32_t *path,
+                                    const uint16_t *k_tree, const uint16_t *v_tree,
+                                    uint16_t *k_pool, uint16_t *v_pool, int64_t num_pages,
+                                    int n_layers, int64_t tree_layer_stride,
+                                    int64_t cache_layer_stride, int hkv, int head_dim,
+                                    int32_t *kv_len_out, void *workspace,
+                                    size_t workspace_bytes, void *stream);
+
+/*
+ * Synchronizes `stream`, reads the workspace status word/*
  * Synchronizes `stream`, reads the workspace status word (the first device-detected error since
  * the last read, ETREE_OK if none), stores its detail code in *detail (if not NULL) and clears
  * both words.

@@ -45,6 +45,60 @@ def attn_compare(wl, dev, rows=None, nthreads=0):
     return res
 
 
+def attn_compare_paged(wl, dev, rows=None, nthreads=0):
+    """attn_compare for a DeviceStep on a paged cache: the oracle gathers each request's logical
+    cache through the same block table."""
+    pc = dev.paged
+    out_o, lse_o, st = oracle.attention_paged(wl.cu_nodes, wl.parent, wl.kv_len, pc.block_table,
+                                              pc.page_size, wl.q, wl.k_tree, wl.v_tree,
+                                              pc.k_pool, pc.v_pool, wl.hq, wl.hkv,
+                                              oracle.scale_of(wl.head_dim), rows=rows,
+                                              nthreads=nthreads)
+    assert st == 0
+    g_out = dev.out.float().cpu().numpy().reshape(-1, wl.head_dim)
+    g_lse = dev.lse.cpu().numpy().reshape(-1)
+    if rows is not None:
+        rr = np.asarray(rows, dtype=np.int64).reshape(-1, 2)
+        idx = rr[:, 0] * wl.hq + rr[:, 1]
+        g_out, g_lse = g_out[idx], g_lse[idx]
+    err = g_out - out_o
+    res = dict(max_abs=float(np.abs(err).max()),
+               rel_rms=float(np.sqrt((err ** 2).mean() / (out_o ** 2).mean())),
+               lse_err=float(np.abs(g_lse - lse_o).max()))
+    assert res["max_abs"] <= ATTN_MAX_ABS, res
+    assert res["rel_rms"] <= ATTN_REL_RMS, res
+    assert res["lse_err"] <= LSE_ABS, res
+    return res
+
+
+def compact_compare_paged(wl, dev, ores, requests, excused):
+    """Bit-exact check of a paged compaction: the oracle scatters the same accepted rows through
+    the block table into a copy of the initial pool; the slots of the checked requests (and
+    their kv_len_out) must match."""
+    pc = dev.paged
+    kpool = oracle._u16(pc.k_pool)[None].copy()
+    vpool = oracle._u16(pc.v_pool)[None].copy()
+    a = np.zeros(wl.B, dtype=np.int32)
+    path = np.full((wl.B, 64), -1, dtype=np.int32)
+    path[:, 0] = 0
+    for r in requests:
+        a[r] = ores[r]["accept_len"]
+        path[r] = ores[r]["path"]
+    st, newlen = oracle.kv_compact_paged(wl.cu_nodes, wl.kv_len, pc.block_table, pc.page_size,
+                                         pc.slot_cap, a, path, oracle._u16(wl.k_tree)[None],
+                                         oracle._u16(wl.v_tree)[None], kpool, vpool, 1)
+    assert st == 0
+    gk = oracle._u16(dev.k_cache.cpu())
+    gv = oracle._u16(dev.v_cache.cpu())
+    kv_out = dev.kv_len_out.cpu().numpy()
+    for r in requests:
+        if r in excused:
+            continue
+        sl = oracle.page_slots(pc.block_table, pc.page_size, r, np.arange(int(newlen[r])))
+        assert np.array_equal(gk[sl], kpool[0, sl]) and np.array_equal(gv[sl], vpool[0, sl]), r
+        assert kv_out[r] == newlen[r], (r, kv_out[r], newlen[r])
+
+
 def sample_rows(wl, per_request: int, seed: int = 0):
     """(node, head) pairs: the last node of every request (deepest, all heads of one KV group)
     plus random (node, head) pairs."""

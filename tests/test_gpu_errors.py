@@ -54,6 +54,23 @@ def test_malformed_node_counts_answer_every_request(T):
     _still_works()
 
 
+def test_bad_page_entry_reports_and_leaves_compaction_untouched():
+    wl = W.generate("tiny", B=2, kv_len=[100, 300], hidden=256, vocab=512)
+    dev = DeviceStep(wl, page_size=32)
+    nump = dev.paged.num_pages
+    dev.block_table[1, 2] = nump + 5                  # a used page of request 1, past the pool
+    dev.attn()
+    assert dev.status() == (EDEVICE, 11)
+    dev.block_table[1, 2] = int(dev.paged.block_table[1, 2])
+    L1 = int(wl.kv_len[1])
+    dev.block_table[1, L1 // 32] = -1                 # request 1's next compaction page
+    dev.lmhead()
+    dev.compact()
+    assert dev.status() == (EDEVICE, 11)
+    assert int(dev.kv_len_out[1]) == L1
+    _still_works()
+
+
 def test_kv_len_above_declared_bound():
     wl, dev = _dev()
     dev.kv_len[0] = wl.kv_len_max + 1

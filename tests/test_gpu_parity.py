@@ -276,3 +276,42 @@ def test_logit_buffer_overflow_reports_and_answers_the_rest():
             assert res["accept_len"][r] == 0 and res["out_tokens"][r][0] >= 0   # root draw only
     excused, near, ores = P.tree_compare(wl, res, got)
     assert near <= 1
+
+
+# ------------------------------------------------------------------------- paged KV caches
+def _paged_check(wl, page_size, attn_rows=None, requests=None):
+    dev, res = _run(wl, page_size=page_size)
+    P.attn_compare_paged(wl, dev, rows=attn_rows)
+    reqs = list(range(wl.B)) if requests is None else requests
+    if wl.temperature == 0.0:
+        excused, near, ores = P.greedy_compare(wl, res, reqs)
+    else:
+        excused, near, ores = P.chain_compare(wl, res, reqs)
+    P.compact_compare_paged(wl, dev, ores, reqs, excused)
+    assert near <= max(1, len(reqs) // 10), near
+    return dev, res
+
+
+@pytest.mark.parametrize("page_size", [16, 32, 64, 256])
+@pytest.mark.parametrize("keys", ["32", "64"])
+def test_paged_cache(page_size, keys, monkeypatch):
+    """Pages smaller than, equal to and larger than the key tile, both tile shapes, ragged
+    lengths including an empty cache and lengths that end mid-page."""
+    monkeypatch.setenv("ETREE_ATTN_KEYS", keys)
+    wl = W.generate("tiny", B=6, n_nodes=[1, 4, 16, 33, 64, 2],
+                    kv_len=[0, 1, 31, 64, 65, 700], depth=8, depth_min=1, branch=None,
+                    width=16, vocab=1000, hidden=256)
+    _paged_check(wl, page_size)
+
+
+def test_paged_cache_splits_and_stochastic_chains(monkeypatch):
+    monkeypatch.setenv("ETREE_NSPLIT", "3")
+    wl = W.generate("conc512", B=9, kv_len=(30, 900), hidden=256, vocab=512)
+    _paged_check(wl, 16)
+
+
+def test_batch64_paged16_full_size():
+    wl = W.generate("batch64")
+    g = np.random.default_rng(4)
+    reqs = sorted(g.choice(wl.B, 6, replace=False).tolist())
+    _paged_check(wl, 16, attn_rows=P.sample_rows(wl, 4), requests=reqs)
