@@ -345,8 +345,9 @@ def run_config(name, steps, warmup, peaks, rank, flush, with_e2e=True):
     from draft_tree_verification_masked_b200 import workload as W
     from draft_tree_verification_masked_b200.runner import DeviceStep
 
-    wl = W.generate(name, seed=W.config_seed(name) + 7919 * rank)
-    dev = DeviceStep(wl)
+    base, _, pg = name.partition("@p")                 # "<workload>@p<page size>": paged cache
+    wl = W.generate(base, seed=W.config_seed(base) + 7919 * rank)
+    dev = DeviceStep(wl, page_size=int(pg) if pg else None)
     dev.step()
     st, det = dev.status()
     if st != 0:
@@ -415,8 +416,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="etree", choices=["etree", "reference"])
     ap.add_argument("--config", default="dense27b_b1")
-    ap.add_argument("--by-batch", default="batch64,conc512,tree64_t1",
-                    help="extra workloads measured in the same run (comma list, '' for none)")
+    ap.add_argument("--by-batch", default="batch64,conc512,tree64_t1,batch64@p16",
+                    help="extra workloads measured in the same run (comma list, '' for none; "
+                         "<workload>@p<N> runs it on a paged cache of N-token pages)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

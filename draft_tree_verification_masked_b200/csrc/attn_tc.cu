@@ -173,10 +173,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tma_load_3d(sQ + rot * 128, &tm_q, &sh->q_full, 0, kvh * G, base + node0);
       tma_load_3d(sQ + 16384 + rot * 128, &tm_q, &sh->q_full, 64, kvh * G, base + node0);
       int issued = 0;
+      // paged: the page entries of tile j + 1 are fetched while tile j's slot is awaited
+      const int nbox = paged ? KEYS / p.cache_box : 0;
+      const int32_t* bt = paged ? p.block_table + (size_t)r * p.max_pages : nullptr;
+      int32_t pg_cur[4], pg_nxt[4];
+      auto fetch_pages = [&](int t, int32_t (&dst)[4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int pi = (t * KEYS + i * p.cache_box) >> p.page_shift;
+          dst[i] = (i < nbox && t < nt_cache && pi < p.max_pages) ? __ldg(bt + pi) : -1;
+        }
+      };
+      if (paged) fetch_pages(t0, pg_cur);
       for (int j = 0; j < T; ++j) {
         const int t = t0 + j;
         const int st = j % STAGES;
         const uint32_t ph = (j / STAGES) & 1;
+        if (paged) fetch_pages(t + 1, pg_nxt);
         if (j >= STAGES && !mbar_wait(&sh->kv_empty[st], ph ^ 1)) {
           report(p.ws, ETREE_ETIMEOUT, DET_WAIT_ATTN);
           break;
@@ -193,11 +206,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           // paged: KEYS / cache_box boxes per half, each inside one page.  An entry outside
           // the pool is reported; its box then lies past the tensor and TMA fills zeros.
           const int cb = p.cache_box, P = 1 << p.page_shift;
-          const int32_t* bt = p.block_table + (size_t)r * p.max_pages;
-          for (int i = 0; i < KEYS / cb; ++i) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (i >= nbox) break;
             const int pos = t * KEYS + i * cb;
-            const int pi = pos >> p.page_shift;
-            int32_t page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+            int32_t page = pg_cur[i];
             if (page < 0 || (int64_t)page * P >= p.cache_slots) {
               if (pos < L) report(p.ws, ETREE_EDEVICE, DET_BAD_PAGE);
               page = (int32_t)(p.cache_slots >> p.page_shift);
@@ -215,6 +228,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tma_load_3d(dst + Sh::kBox, &tm_kt, &sh->kv_full[st], 64, kvh, node);
           tma_load_3d(dst + 2 * Sh::kBox, &tm_vt, &sh->kv_full[st], 0, kvh, node);
           tma_load_3d(dst + 3 * Sh::kBox, &tm_vt, &sh->kv_full[st], 64, kvh, node);
+        }
+        if (paged) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) pg_cur[i] = pg_nxt[i];
         }
         issued = j + 1;
       }
