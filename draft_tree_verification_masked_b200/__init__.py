@@ -29,8 +29,8 @@ __all__ = [
     "EtreeError", "Batch", "make_batch", "lib", "library_path", "etree_workspace_size",
     "etree_workspace_init", "etree_verify_attn", "etree_verify_attn_noalloc",
     "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact",
-    "etree_verify_attn_paged", "etree_kv_compact_paged",
-    "etree_device_status", "etree_strerror", "etree_version", "etree_attn_plan", "STATUS",
+    "etree_verify_attn_paged", "etree_kv_compact_paged", "etree_verify_cost", "etree_plan_tree",
+    "cost_table", "load_cost_table", "etree_device_status", "etree_strerror", "etree_version", "etree_attn_plan", "STATUS",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +42,8 @@ DETAIL = {0: "none", 1: "bad parent", 2: "bad node count", 3: "bad kv_len", 4: "
           5: "not a chain", 6: "bad path", 7: "attention wait", 8: "gemm wait", 9: "bad token"}
 
 EXPORTS = ["etree_workspace_size", "etree_workspace_init", "etree_verify_attn",
-           "etree_verify_attn_paged", "etree_kv_compact_paged",
+           "etree_verify_attn_paged", "etree_kv_compact_paged", "etree_verify_cost",
+           "etree_plan_tree",
            "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact", "etree_device_status", "etree_strerror",
            "etree_version", "etree_last_error", "etree_attn_plan", "etree_verify_attn_noalloc"]
 
@@ -98,6 +99,13 @@ def lib():
                                           C.c_int, C.c_int, C.c_int, f32, vp, vp, vp, C.c_size_t,
                                           vp]
     L.etree_verify_attn_paged.restype = C.c_int
+    L.etree_verify_cost.argtypes = [C.POINTER(CostTable), C.c_double, C.c_double, C.c_double,
+                                    C.POINTER(C.c_double)]
+    L.etree_verify_cost.restype = C.c_int
+    L.etree_plan_tree.argtypes = [C.POINTER(CostTable), C.c_int32, C.c_int32,
+                                  C.POINTER(C.c_float), C.c_int32, C.c_float, C.c_float,
+                                  C.c_int32, C.c_int32, C.c_int32, C.POINTER(TreePlan)]
+    L.etree_plan_tree.restype = C.c_int
     L.etree_kv_compact_paged.argtypes = [bp, vp, C.c_int32, C.c_int32, vp, vp, vp, vp, vp, vp,
                                          i64, C.c_int, i64, i64, C.c_int, C.c_int, vp, vp,
                                          C.c_size_t, vp]
@@ -146,6 +154,61 @@ def _stream(stream) -> int | None:
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)
+
+
+class CostTable(C.Structure):
+    _fields_ = [("nB", C.c_int32), ("nN", C.c_int32), ("nL", C.c_int32),
+                ("B", C.POINTER(C.c_int32)), ("N", C.POINTER(C.c_int32)),
+                ("L", C.POINTER(C.c_int32)), ("us", C.POINTER(C.c_float))]
+
+
+class TreePlan(C.Structure):
+    _fields_ = [("depth", C.c_int32), ("width", C.c_int32), ("nodes", C.c_int32),
+                ("expected_accept", C.c_double), ("step_us", C.c_double),
+                ("tokens_per_s", C.c_double)]
+
+
+def cost_table(d: dict) -> CostTable:
+    """An etree_cost_table over the dict {"B", "N", "L", "us"} (as calibrate.py writes it)."""
+    import numpy as np
+    arrs = [np.ascontiguousarray(d[k], dtype=np.int32) for k in ("B", "N", "L")]
+    us = np.ascontiguousarray(d["us"], dtype=np.float32)
+    if us.shape != (len(arrs[0]), len(arrs[1]), len(arrs[2])):
+        raise ValueError(f"us has shape {us.shape}, want (|B|, |N|, |L|)")
+    i32p, f32p = C.POINTER(C.c_int32), C.POINTER(C.c_float)
+    t = CostTable(len(arrs[0]), len(arrs[1]), len(arrs[2]), arrs[0].ctypes.data_as(i32p),
+                  arrs[1].ctypes.data_as(i32p), arrs[2].ctypes.data_as(i32p),
+                  us.ctypes.data_as(f32p))
+    t._keep = (arrs, us)
+    return t
+
+
+def load_cost_table(name: str = "b200_dense27b") -> dict:
+    """A packaged calibration (cost_tables/<name>.json) or a path to one."""
+    import json
+    path = name if os.path.exists(name) else os.path.join(HERE, "cost_tables", name + ".json")
+    with open(path) as f:
+        return json.load(f)
+
+
+def etree_verify_cost(table, B: float, N: float, L: float) -> float:
+    t = table if isinstance(table, CostTable) else cost_table(table)
+    out = C.c_double()
+    _check(lib().etree_verify_cost(C.byref(t), float(B), float(N), float(L), C.byref(out)))
+    return out.value
+
+
+def etree_plan_tree(table, B: int, L: int, acc_rank, draft_us_per_level: float,
+                    draft_us_fixed: float = 0.0, max_depth: int = 16, max_width: int = 16,
+                    max_nodes: int = 64) -> dict:
+    """The static (depth, width) draft tree with the most expected tokens/s (host only)."""
+    t = table if isinstance(table, CostTable) else cost_table(table)
+    acc = (C.c_float * len(acc_rank))(*[float(a) for a in acc_rank])
+    out = TreePlan()
+    _check(lib().etree_plan_tree(C.byref(t), int(B), int(L), acc, len(acc_rank),
+                                 float(draft_us_per_level), float(draft_us_fixed),
+                                 int(max_depth), int(max_width), int(max_nodes), C.byref(out)))
+    return {k: getattr(out, k) for k, _ in TreePlan._fields_}
 
 
 def make_batch(cu_nodes, parent, tokens, kv_len, slot_base, slot_cap, n_max: int,

@@ -157,7 +157,6 @@ etree_status etree_verify_attn_paged(const etree_batch *batch, const int32_t *bl
                                      size_t workspace_bytes, void *stream);
 
 /*
- * LM head + acceptance.  z = hidden W^T/*
  * LM head + acceptance.  z = hidden W^T (fp32 accumulate over bf16 inputs) for every node row.
  *  T == 0 (greedy): t*(u) = argmax z_u (lowest id on ties).  From the root, repeatedly move to
  *    the lowest-index child whose token equals t*(current); the node where no child matches
@@ -253,7 +252,55 @@ etree_status etree_kv_compact_paged(const etree_batch *batch, const int32_t *blo
                                     size_t workspace_bytes, void *stream);
 
 /*
- * Synchronizes `stream`, reads the workspace status word/*
+ * Hardware-aware tree sizing (host-only; no device work).  The pages size the draft tree from the
+ * measured cost of drafting and verifying at the running batch size and hardware
+ * ("EAGLE-4 官方推理代码发布 ...", arex-research.com, section "投机树多大，由实测成本决定").
+ *
+ * etree_cost_table: measured µs of one verification step (attention, LM head with acceptance,
+ * compaction; draft_tree_verification_masked_b200/calibrate.py writes one) on the grid
+ * B[0..nB) x N[0..nN) x L[0..nL) (each strictly ascending; N = tree nodes per request, root
+ * included; L = cached tokens per request), us[(i * nN + j) * nL + k] for (B[i], N[j], L[k]).
+ * All pointers are host pointers owned by the caller.
+ */
+typedef struct {
+  int32_t nB, nN, nL;
+  const int32_t *B, *N, *L;
+  const float *us;
+} etree_cost_table;
+
+/*
+ * Step time at (B, N, L): trilinear interpolation on the grid, each axis extended linearly past
+ * its first and last points; negative results clamp to 0.  ETREE_EINVAL for a malformed table.
+ */
+etree_status etree_verify_cost(const etree_cost_table *table, double B, double N, double L,
+                               double *us_out);
+
+typedef struct {
+  int32_t depth, width, nodes;      /* chosen static tree; depth 0 = no speculation (1 node) */
+  double expected_accept;           /* expected accepted draft tokens per request and step */
+  double step_us;                   /* draft time + interpolated verification time */
+  double tokens_per_s;              /* B (expected_accept + 1) / step_us, whole batch */
+} etree_tree_plan;
+
+/*
+ * The static draft tree that maximises expected tokens per second for B requests of L cached
+ * tokens.  Shape: `depth` levels; at each level the top draft candidate continues the spine and
+ * width - 1 lower-ranked candidates sit beside it as leaves, so nodes = 1 + depth * width
+ * (<= max_nodes <= 64, depth <= max_depth <= 63, width <= max_width).  Acceptance model: at
+ * every level the target's token is the rank-k draft candidate with probability acc_rank[k]
+ * (k = 0 .. n_rank-1, sum <= 1, independent across levels); the walk continues only through the
+ * spine, so E[accepted] = sum_{j=1..depth} acc_rank[0]^(j-1) (acc_rank[0] + ... + acc_rank[width-1]).
+ * Step time = draft_us_fixed + depth * draft_us_per_level (both 0 when depth = 0) plus
+ * etree_verify_cost(B, nodes, L); a step time of 0 (a table extrapolated below zero) counts as
+ * 0 tokens/s.  Ties (within 1e-12 relative) go to the fewer nodes, then the shallower tree.
+ * ETREE_EINVAL for out-of-range arguments or a malformed table.
+ */
+etree_status etree_plan_tree(const etree_cost_table *table, int32_t B, int32_t L,
+                             const float *acc_rank, int32_t n_rank, float draft_us_per_level,
+                             float draft_us_fixed, int32_t max_depth, int32_t max_width,
+                             int32_t max_nodes, etree_tree_plan *out);
+
+/*
  * Synchronizes `stream`, reads the workspace status word (the first device-detected error since
  * the last read, ETREE_OK if none), stores its detail code in *detail (if not NULL) and clears
  * both words.
