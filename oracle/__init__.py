@@ -73,6 +73,12 @@ def lib():
                                                C.c_double, C.c_uint64, C.c_uint64, I32P, I32P,
                                                I32P, I32P, F64P, C.c_int]
         L.oracle_accept_tree_batch.restype = None
+        L.oracle_bf16_round.argtypes = [C.c_double]
+        L.oracle_bf16_round.restype = C.c_uint16
+        L.oracle_lowrank_candidates.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                                U16P, U16P, U16P, U16P, I32P, F64P, C.c_void_p,
+                                                C.c_void_p, C.c_int]
+        L.oracle_lowrank_candidates.restype = None
         L.oracle_race_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
                                        C.c_int, I32P, C.c_int]
         L.oracle_race_many.restype = None
@@ -282,6 +288,28 @@ def kv_compact(cu_nodes, kv_len, slot_base, slot_cap, accept_len, path, k_tree, 
                                  _u16(v_tree).reshape(-1), kc.reshape(-1), vc.reshape(-1),
                                  n_layers, tree_layer_stride, cache_layer_stride, hkv, d, out)
     return st, out
+
+
+def bf16_round(x) -> int:
+    return int(lib().oracle_bf16_round(float(x)))
+
+
+def lowrank_candidates(hidden, D, U, W, k, keep_approx=False, nthreads=0):
+    """The low-rank candidate head over the rows of `hidden`: returns (ids [M,k], exact logits
+    [M,k], k-th approximate logit [M], approximate logits [M,V] or None)."""
+    h, d, u, w = _u16(hidden), _u16(D), _u16(U), _u16(W)
+    M, H = h.shape
+    r, V = d.shape[0], u.shape[0]
+    ids = np.empty((M, k), dtype=np.int32)
+    lg = np.empty((M, k), dtype=np.float64)
+    kth = np.empty(M, dtype=np.float64)
+    za = np.empty((M, V), dtype=np.float64) if keep_approx else None
+    lib().oracle_lowrank_candidates(M, H, V, r, k, h.reshape(-1), d.reshape(-1), u.reshape(-1),
+                                    w.reshape(-1), ids.reshape(-1), lg.reshape(-1),
+                                    kth.ctypes.data_as(C.c_void_p),
+                                    za.ctypes.data_as(C.c_void_p) if keep_approx else None,
+                                    int(nthreads))
+    return ids, lg, kth, za
 
 
 # ------------------------------------------------------------------------------- paged caches

@@ -439,6 +439,108 @@ int oracle_accept_chain(int n, const int32_t *parent, const int32_t *tokens, con
 }
 
 /* ---------------------------------------------------------------------------------------------
+ * Round-to-nearest-even of x to bf16 (8 significant bits, fp32's exponent range), returned as
+ * bits.  Written from the definition: among the two bf16 values around x, the nearer; on a tie,
+ * the one whose last significand bit is 0.  Finite inputs within bf16 range only.
+ * ------------------------------------------------------------------------------------------- */
+uint16_t oracle_bf16_round(double x) {
+    if (x == 0.0) return signbit(x) ? 0x8000u : 0u;
+    const double ax = fabs(x);
+    int e;
+    frexp(ax, &e);                                /* ax = m 2^e, m in [0.5, 1) */
+    if (e < -125) e = -125;                        /* subnormal range: fixed spacing 2^-133 */
+    const double ulp = ldexp(1.0, e - 8);          /* spacing of bf16 values in [2^(e-1), 2^e) */
+    double lo = floor(ax / ulp) * ulp;
+    double hi = lo + ulp;
+    double r;
+    const double dl = ax - lo, dh = hi - ax;
+    if (dl < dh) r = lo;
+    else if (dh < dl) r = hi;
+    else r = fmod(lo / ulp, 2.0) == 0.0 ? lo : hi;
+    float f = (float)(x < 0 ? -r : r);             /* exact: r has <= 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Low-rank candidate head (the draft's output layer in the pages: "EAGLE-4 是什麼？...",
+ * aiposthub.com, section "EAGLE-4 是什麼？先看推測解碼為什麼能變快": a small matrix screens
+ * candidate tokens, then only the few candidates are scored exactly).  For each of M rows h
+ * (bf16, [M][H]):
+ *   g = h D^T                  D [r][H] bf16; g rounded to bf16 (the precision of the second
+ *                              product's operand);
+ *   z~ = g U^T                 U [V][r] bf16: approximate logits;
+ *   C = the k ids of largest z~ (ties to the lowest id);
+ *   z_c = h . W_c for c in C   W [V][H] bf16: exact logits of the candidates;
+ * out_ids [M][k]: C ordered by z_c descending (ties to the lowest id), out_logit [M][k] the z_c;
+ * kth [M] (nullable): the k-th largest z~; z_approx [M][V] (nullable): z~.  fp64 throughout.
+ * ------------------------------------------------------------------------------------------- */
+void oracle_lowrank_candidates(int M, int H, int V, int r, int k, const uint16_t *hid,
+                               const uint16_t *D, const uint16_t *U, const uint16_t *W,
+                               int32_t *out_ids, double *out_logit, double *kth,
+                               double *z_approx, int nthreads) {
+    set_threads(nthreads);
+    double *g = (double *)malloc(sizeof(double) * (size_t)M * r);
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < M * r; ++t) {
+        const int m = t / r, j = t % r;
+        double acc = 0.0;
+        for (int h = 0; h < H; ++h)
+            acc += bf16_value(hid[(size_t)m * H + h]) * bf16_value(D[(size_t)j * H + h]);
+        g[t] = bf16_value(oracle_bf16_round(acc));
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int m = 0; m < M; ++m) {
+        double *z = (double *)malloc(sizeof(double) * (size_t)V);
+        for (int v = 0; v < V; ++v) {
+            double acc = 0.0;
+            for (int j = 0; j < r; ++j) acc += g[(size_t)m * r + j] * bf16_value(U[(size_t)v * r + j]);
+            z[v] = acc;
+        }
+        if (z_approx) memcpy(z_approx + (size_t)m * V, z, sizeof(double) * (size_t)V);
+        /* top-k by z~: repeated selection of the largest remaining (lowest id on ties) */
+        int32_t cand[64];
+        char *taken = (char *)calloc((size_t)V, 1);
+        for (int i = 0; i < k; ++i) {
+            int best = -1;
+            for (int v = 0; v < V; ++v)
+                if (!taken[v] && (best < 0 || z[v] > z[best])) best = v;
+            taken[best] = 1;
+            cand[i] = best;
+        }
+        if (kth) kth[m] = z[cand[k - 1]];
+        free(taken);
+        double ex[64];
+        for (int i = 0; i < k; ++i) {
+            double acc = 0.0;
+            for (int h = 0; h < H; ++h)
+                acc += bf16_value(hid[(size_t)m * H + h]) * bf16_value(W[(size_t)cand[i] * H + h]);
+            ex[i] = acc;
+        }
+        /* order by exact logit, descending, lowest id on ties (insertion sort of <= 64) */
+        for (int i = 1; i < k; ++i) {
+            const int ci = cand[i];
+            const double xi = ex[i];
+            int j = i - 1;
+            while (j >= 0 && (ex[j] < xi || (ex[j] == xi && cand[j] > ci))) {
+                ex[j + 1] = ex[j];
+                cand[j + 1] = cand[j];
+                --j;
+            }
+            ex[j + 1] = xi;
+            cand[j + 1] = ci;
+        }
+        for (int i = 0; i < k; ++i) {
+            out_ids[(size_t)m * k + i] = cand[i];
+            out_logit[(size_t)m * k + i] = ex[i];
+        }
+        free(z);
+    }
+    free(g);
+}
+
+/* ---------------------------------------------------------------------------------------------
  * Stochastic (T>0) acceptance over a general tree: multi-candidate speculative sampling (the
  * multi-step rule of SpecInfer, Miao et al., "SpecInfer: Accelerating Large Language Model Serving
  * with Tree-based Speculative Inference and Verification", 2023, restated here).

@@ -687,3 +687,70 @@ def test_kv_compact_capacity_overflow_leaves_request_untouched():
     st, newlen = oracle.kv_compact(cu, kv_len, np.zeros(1, np.int64), cap, np.array([3], np.int32),
                                    path, tk, tk, ck, ck.copy(), 1, 32, 96, 1, 8)
     assert st == oracle.ENOSPACE and newlen[0] == 10 and not ck.any()
+
+
+# -------------------------------------------------------------------- low-rank candidate head
+def _bf16_bits(x):
+    return oracle._u16(torch.as_tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16))
+
+
+def _bits_value(b):
+    return np.asarray(b, dtype=np.uint32).astype(np.uint32) << 16
+
+
+def test_bf16_rounding_is_nearest_even():
+    g = np.random.default_rng(61)
+    xs = np.concatenate([g.normal(0, 3, 2000), g.normal(0, 1e-3, 500), [1.0 + 2 ** -8,
+                         1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 2 ** -130, 3.5 * 2 ** -133]])
+    for x in xs:
+        b = oracle.bf16_round(float(x))
+        v = np.frombuffer(np.uint32(b << 16).tobytes(), np.float32)[0]
+        for nb in (b - 1, b + 1):                     # the bf16 neighbours (same sign)
+            nv = np.frombuffer(np.uint32((nb & 0xFFFF) << 16).tobytes(), np.float32)[0]
+            if np.isfinite(nv) and np.sign(nv) == np.sign(v):
+                d, dn = abs(float(x) - float(v)), abs(float(x) - float(nv))
+                assert d < dn or (d == dn and (b & 1) == 0), (x, v, nv)
+    # fp32-exact inputs: the library's fp32 -> bf16 rounding agrees
+    f = g.normal(0, 5, 5000).astype(np.float32)
+    want = _bf16_bits(f)
+    got = np.array([oracle.bf16_round(float(x)) for x in f], dtype=np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_lowrank_head_with_identity_factors_is_the_exact_top_k():
+    """r = H, D = I and U = W: the screen is the exact logits, so the candidates are numpy's
+    top-k of h W^T, in exact order."""
+    g = np.random.default_rng(62)
+    M, H, V, k = 5, 64, 300, 12
+    hid = _bf16_bits(g.normal(size=(M, H)))
+    W = _bf16_bits(g.normal(0, 0.3, size=(V, H)))
+    D = _bf16_bits(np.eye(H))
+    ids, lg, kth, _ = oracle.lowrank_candidates(hid, D, W, W, k)
+    hf = hid.astype(np.uint32) << 16
+    z = np.frombuffer(hf.tobytes(), np.float32).reshape(M, H).astype(np.float64) @ \
+        np.frombuffer((W.astype(np.uint32) << 16).tobytes(), np.float32).reshape(V, H).astype(
+            np.float64).T
+    for m in range(M):
+        order = np.lexsort((np.arange(V), -z[m]))[:k]
+        assert list(ids[m]) == list(order)
+        assert np.allclose(lg[m], z[m, order], rtol=0, atol=1e-9)
+
+
+def test_lowrank_head_with_all_ids_is_the_exact_sort_and_permutes_with_the_vocab():
+    g = np.random.default_rng(63)
+    M, H, V, r = 3, 32, 48, 8
+    hid = _bf16_bits(g.normal(size=(M, H)))
+    D = _bf16_bits(g.normal(0, 0.2, size=(r, H)))
+    U = _bf16_bits(g.normal(0, 0.2, size=(V, r)))
+    W = _bf16_bits(g.normal(0, 0.2, size=(V, H)))
+    ids, lg, _, _ = oracle.lowrank_candidates(hid, D, U, W, V)
+    Wf = np.frombuffer((W.astype(np.uint32) << 16).tobytes(), np.float32).reshape(V, H)
+    hf = np.frombuffer((hid.astype(np.uint32) << 16).tobytes(), np.float32).reshape(M, H)
+    z = hf.astype(np.float64) @ Wf.astype(np.float64).T
+    for m in range(M):
+        assert list(ids[m]) == list(np.lexsort((np.arange(V), -z[m])))
+    perm = g.permutation(V)
+    ids2, lg2, _, _ = oracle.lowrank_candidates(hid, D, U[perm], W[perm], 10)
+    ids1, lg1, _, _ = oracle.lowrank_candidates(hid, D, U, W, 10)
+    assert np.array_equal(perm[ids2], ids1)          # the same tokens, renamed
+    assert np.allclose(lg1, lg2, rtol=0, atol=1e-12)
