@@ -365,6 +365,46 @@ def run_config(name, steps, warmup, peaks, rank, flush, with_e2e=True):
     return res
 
 
+def lowrank_report(name, flush, peaks, reps=20, warmup=3):
+    """Device time of one etree_lowrank_candidates call (screen + exact rescoring of the k
+    candidates) against its algorithmic bytes: |U| + |D| + |hidden| + the M k rows of W read."""
+    from draft_tree_verification_masked_b200 import (etree_lowrank_candidates,
+                                                     etree_lowrank_workspace_size,
+                                                     etree_workspace_init)
+    from draft_tree_verification_masked_b200 import workload as W
+    lw = W.lowrank(name)
+    dev = torch.device("cuda")
+    h, D, U, Wt = (x.to(dev) for x in (lw.hidden, lw.D, lw.U, lw.W))
+    ws = torch.zeros(etree_lowrank_workspace_size(lw.M, lw.H, lw.r, lw.V), dtype=torch.uint8,
+                     device=dev)
+    etree_workspace_init(ws)
+    ids = torch.empty(lw.M, lw.k, dtype=torch.int32, device=dev)
+    lg = torch.empty(lw.M, lw.k, dtype=torch.float32, device=dev)
+
+    def one():
+        etree_lowrank_candidates(h, D, U, Wt, lw.k, ids, lg, ws)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        one()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b) * 1e-3)
+    t = statistics.mean(ts)
+    nbytes = 2 * (lw.V * lw.r + lw.r * lw.H + lw.M * lw.H + lw.M * lw.k * lw.H)
+    hbm = float(peaks["hbm_gbs"])
+    return {"M": lw.M, "rank": lw.r, "k": lw.k, "vocab": lw.V, "hidden": lw.H,
+            "us": t * 1e6, "bytes": nbytes, "GB/s": nbytes / t / 1e9,
+            "hbm_frac": nbytes / t / 1e9 / hbm,
+            "full_head_bytes": 2 * lw.V * lw.H}
+
+
 def compact_layers_report(dev, wl, flush, peaks, layers=64):
     us, nbytes = time_compact_layers(dev, wl, flush, layers)
     hbm = float(peaks["hbm_gbs"])
@@ -420,6 +460,8 @@ def main():
                     help="extra workloads measured in the same run (comma list, '' for none; "
                          "<workload>@p<N> runs it on a paged cache of N-token pages)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lowrank", default="lowrank_r512,lowrank_r128",
+                    help="low-rank candidate-head workloads timed after the step ('' for none)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -482,6 +524,13 @@ def main():
         }
         main_res = r
 
+    lowrank = {}
+    if args.lowrank:
+        del main_res["dev"]
+        torch.cuda.empty_cache()
+        for name in [x for x in args.lowrank.split(",") if x]:
+            lowrank[name] = lowrank_report(name, flush, peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
@@ -523,6 +572,7 @@ def main():
                     for k, v in rep.items()},
         "cpu_baseline": cpu,
         "by_batch": by_batch,
+        "lowrank_head": lowrank,
     }
     print(json.dumps(line))
 

@@ -30,7 +30,8 @@ __all__ = [
     "etree_workspace_init", "etree_verify_attn", "etree_verify_attn_noalloc",
     "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact",
     "etree_verify_attn_paged", "etree_kv_compact_paged", "etree_verify_cost", "etree_plan_tree",
-    "cost_table", "load_cost_table", "etree_device_status", "etree_strerror", "etree_version", "etree_attn_plan", "STATUS",
+    "cost_table", "load_cost_table", "etree_lowrank_workspace_size",
+    "etree_lowrank_candidates", "etree_device_status", "etree_strerror", "etree_version", "etree_attn_plan", "STATUS",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -43,7 +44,7 @@ DETAIL = {0: "none", 1: "bad parent", 2: "bad node count", 3: "bad kv_len", 4: "
 
 EXPORTS = ["etree_workspace_size", "etree_workspace_init", "etree_verify_attn",
            "etree_verify_attn_paged", "etree_kv_compact_paged", "etree_verify_cost",
-           "etree_plan_tree",
+           "etree_plan_tree", "etree_lowrank_workspace_size", "etree_lowrank_candidates",
            "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact", "etree_device_status", "etree_strerror",
            "etree_version", "etree_last_error", "etree_attn_plan", "etree_verify_attn_noalloc"]
 
@@ -99,6 +100,11 @@ def lib():
                                           C.c_int, C.c_int, C.c_int, f32, vp, vp, vp, C.c_size_t,
                                           vp]
     L.etree_verify_attn_paged.restype = C.c_int
+    L.etree_lowrank_workspace_size.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int]
+    L.etree_lowrank_workspace_size.restype = C.c_size_t
+    L.etree_lowrank_candidates.argtypes = [vp, C.c_int, C.c_int, vp, vp, C.c_int, vp, C.c_int,
+                                           C.c_int, vp, vp, vp, C.c_size_t, vp]
+    L.etree_lowrank_candidates.restype = C.c_int
     L.etree_verify_cost.argtypes = [C.POINTER(CostTable), C.c_double, C.c_double, C.c_double,
                                     C.POINTER(C.c_double)]
     L.etree_verify_cost.restype = C.c_int
@@ -154,6 +160,25 @@ def _stream(stream) -> int | None:
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)
+
+
+def etree_lowrank_workspace_size(M: int, hidden_dim: int, rank: int, vocab: int) -> int:
+    return int(lib().etree_lowrank_workspace_size(int(M), int(hidden_dim), int(rank),
+                                                  int(vocab)))
+
+
+def etree_lowrank_candidates(hidden, D, U, W, k: int, out_ids, out_logit, workspace,
+                             stream=None, check: bool = True) -> int:
+    """hidden [M, H], D [r, H], U [V, r], W [V, H] bf16; out_ids int32 / out_logit fp32 [M, k]."""
+    bf = torch.bfloat16
+    M, H = hidden.shape
+    r, V = D.shape[0], U.shape[0]
+    st = lib().etree_lowrank_candidates(
+        _ptr(hidden, bf, "hidden"), M, H, _ptr(D, bf, "D"), _ptr(U, bf, "U"), r,
+        _ptr(W, bf, "W"), V, int(k), _ptr(out_ids, torch.int32, "out_ids"),
+        _ptr(out_logit, torch.float32, "out_logit"), _ptr(workspace, torch.uint8, "workspace"),
+        workspace.numel(), _stream(stream))
+    return _check(st) if check else st
 
 
 class CostTable(C.Structure):

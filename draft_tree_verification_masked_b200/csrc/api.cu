@@ -345,6 +345,98 @@ etree_status etree_workspace_init(void* workspace, size_t workspace_bytes, void*
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_workspace_init");
 }
 
+// ------------------------------------------------------------------ low-rank candidate head
+struct LowrankLayout {
+  size_t part, g, lists, cand, tkth, total;
+  int nk, nlists;
+};
+
+static LowrankLayout lowrank_layout(int M, int H, int r, int V) {
+  LowrankLayout w{};
+  size_t off = sizeof(WsHeader);
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = up256(off + bytes);
+    return at;
+  };
+  w.nk = lowrank_down_chunks(H);
+  w.nlists = 2 * ((V + 127) / 128);                 // per vocab tile at the narrowest width
+  // the sample's chunk partials, then its summed logits
+  const size_t sample = (size_t)((r + 127) / 128 + 1) * M * lowrank_sample_cols(V);
+  w.part = take(std::max((size_t)w.nk * M * r, sample) * sizeof(float));
+  w.g = take((size_t)M * r * 2);
+  w.lists = take((size_t)M * w.nlists * 16 * sizeof(float2));
+  w.cand = take((size_t)M * 16 * sizeof(int32_t));
+  w.tkth = take((size_t)M * sizeof(uint32_t));
+  w.total = off;
+  return w;
+}
+
+size_t etree_lowrank_workspace_size(int M, int hidden_dim, int rank, int vocab) {
+  if (M < 1 || hidden_dim < 1 || rank < 1 || vocab < 1) return 0;
+  return lowrank_layout(M, hidden_dim, rank, vocab).total;
+}
+
+etree_status etree_lowrank_candidates(const uint16_t* hidden, int M, int hidden_dim,
+                                      const uint16_t* D, const uint16_t* U, int rank,
+                                      const uint16_t* W, int vocab, int k, int32_t* out_ids,
+                                      float* out_logit, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  if (!hidden || !D || !U || !W || !out_ids || !out_logit || !workspace)
+    return fail(ETREE_EINVAL, "a pointer is NULL");
+  if (M < 1 || M > (1 << 20)) return fail(ETREE_EINVAL, "M=%d", M);
+  if (hidden_dim < 64 || hidden_dim % 64 || hidden_dim > 8192)
+    return fail(ETREE_EUNSUPPORTED, "hidden_dim=%d must be a multiple of 64 in [64, 8192]",
+                hidden_dim);
+  if (rank < 64 || rank % 64 || rank > 8192)
+    return fail(ETREE_EUNSUPPORTED, "rank=%d must be a multiple of 64 in [64, 8192]", rank);
+  if (k < 1 || k > 16 || vocab < k) return fail(ETREE_EINVAL, "k=%d (1..16, <= vocab)", k);
+  if (!aligned16(hidden) || !aligned16(D) || !aligned16(U) || !aligned16(W) || !aligned16(workspace))
+    return fail(ETREE_EINVAL, "hidden, D, U, W and the workspace must be 16-byte aligned");
+  const LowrankLayout w = lowrank_layout(M, hidden_dim, rank, vocab);
+  if (workspace_bytes < w.total)
+    return fail(ETREE_EINVAL, "workspace has %zu bytes, needs %zu", workspace_bytes, w.total);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(hidden);
+  __nv_bfloat16* g = at<__nv_bfloat16>(workspace, w.g);
+  uint32_t* tkth = at<uint32_t>(workspace, w.tkth);
+  cudaError_t e = launch_lowrank_down(hb, reinterpret_cast<const __nv_bfloat16*>(D), M,
+                                      hidden_dim, rank, at<float>(workspace, w.part), g, tkth, s);
+  if (e == cudaSuccess)
+    e = launch_lowrank_sample(g, reinterpret_cast<const __nv_bfloat16*>(U), M, rank, vocab,
+                              at<float>(workspace, w.part), tkth, s);
+  if (e != cudaSuccess) return cuda_fail(e, "etree_lowrank_candidates (down, sample)");
+
+  const int sms = sm_count();
+  const int bn = lmhead_pick_bn(M, vocab, sms);
+  const int bm = M <= 64 ? 64 : 128;
+  CUtensorMap ta, tb;
+  etree_status st;
+  if ((st = get_map(g, 2, rank, M, 1, 64, bm, 1, &ta))) return st;
+  if ((st = get_map(U, 2, rank, vocab, 1, 64, bn, 1, &tb))) return st;
+  GemmParams gp{};
+  gp.M = M;
+  gp.V = vocab;
+  gp.K = rank;
+  gp.m_tiles = (M + bm - 1) / bm;
+  gp.n_tiles = (vocab + bn - 1) / bn;
+  gp.num_tiles = gp.m_tiles * gp.n_tiles;
+  gp.k_blocks = rank / 64;
+  gp.ws = at<WsHeader>(workspace, 0);
+  const int grid = std::min(gp.num_tiles, sms);
+  gp.per_cta = gp.m_tiles == 1;
+  gp.n_parts = gp.per_cta ? grid : gp.n_tiles;
+  gp.topk = at<float2>(workspace, w.lists);
+  gp.tkth = tkth;
+  e = launch_lmhead(3, bn, bm, ta, tb, gp, grid, s);
+  if (e != cudaSuccess) return cuda_fail(e, "etree_lowrank_candidates (screen)");
+  e = launch_lowrank_finish(gp.topk, 2 * gp.n_parts, tkth, M, k, at<int32_t>(workspace, w.cand),
+                            hb,
+                            reinterpret_cast<const __nv_bfloat16*>(W), hidden_dim, vocab,
+                            out_ids, out_logit, s);
+  return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lowrank_candidates (rescore)");
+}
+
 etree_status etree_device_status(void* workspace, void* stream, int32_t* detail) {
   if (!workspace) return fail(ETREE_EINVAL, "workspace is NULL");
   cudaStream_t s = static_cast<cudaStream_t>(stream);

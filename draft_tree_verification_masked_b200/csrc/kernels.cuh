@@ -5,6 +5,20 @@
 
 namespace etree {
 
+// Order-preserving map of fp32 to uint32 (monotone: a < b iff enc(a) < enc(b)), so that atomicMax
+// on the code keeps a running maximum of floats of either sign.
+__host__ __device__ __forceinline__ uint32_t enc_order(float x) {
+  uint32_t u;
+  memcpy(&u, &x, 4);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__host__ __device__ __forceinline__ float dec_order(uint32_t c) {
+  const uint32_t u = (c & 0x80000000u) ? (c & 0x7fffffffu) : ~c;
+  float x;
+  memcpy(&x, &u, 4);
+  return x;
+}
+
 struct AttnParams {
   const int32_t* cu_nodes;
   const int32_t* parent;
@@ -47,6 +61,8 @@ struct GemmParams {
   int cnt_n;
   const int32_t* zrow;              // EPI_LSE, if set: row g's logits go to zbuf[zrow[g]][V]
   float* zbuf;                      // when zrow[g] >= 0 (rows of branching tree nodes)
+  float2* topk;                     // EPI_TOPK: per (row, slot, half) 16 (value, id bits)
+  uint32_t* tkth;                   // EPI_TOPK: per row, order-encoded lower bound of the k-th
   WsHeader* ws;
   float4* part;
   const int32_t* child_tok;
@@ -99,6 +115,19 @@ cudaError_t launch_tree_prep(const AcceptParams& p, const __nv_bfloat16* w_lm, i
                              int32_t* zrow, int zbuf_rows, float* zc, cudaStream_t s);
 cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32_t* zrow,
                              const float* zbuf, cudaStream_t s);
+
+int lowrank_down_chunks(int H);
+cudaError_t launch_lowrank_down(const __nv_bfloat16* hid, const __nv_bfloat16* D, int M, int H,
+                                int r, float* part, __nv_bfloat16* g, uint32_t* tkth,
+                                cudaStream_t s);
+int lowrank_sample_cols(int V);
+cudaError_t launch_lowrank_sample(const __nv_bfloat16* g, const __nv_bfloat16* U, int M, int r,
+                                  int V, float* part, uint32_t* tkth, cudaStream_t s);
+cudaError_t launch_lowrank_finish(const float2* lists, int nlists, const uint32_t* tkth, int M,
+                                  int k,
+                                  int32_t* cand, const __nv_bfloat16* hid,
+                                  const __nv_bfloat16* W, int H, int V, int32_t* out_ids,
+                                  float* out_logit, cudaStream_t s);
 
 struct CompactParams {
   const int32_t* cu_nodes;

@@ -19,6 +19,8 @@
 //   EPI_LSE     per row and tile: m = max z*log2(e)/T and sum 2^(z*log2(e)/T - m), plus the
 //               logit of the row's child token when it falls in the tile; rows of branching tree
 //               nodes also write their logits out (the sibling residuals need whole rows);
+//   EPI_TOPK    per row and tile half: the 16 largest values and their ids (the low-rank
+//               candidate head's screen, lowrank.cu);
 //   EPI_RACE    per row and 128-id block: the block total of the draw's weights
 //               max(0, p - c q) (c = 0: p; c = 1: the residual after one rejection; larger c
 //               after sibling rejections), the id where the block's running sum passes u_b times
@@ -35,7 +37,55 @@ constexpr int kBK = 64;
 __host__ __device__ constexpr int gemm_stages(int bm, int bn) {
   return (210 * 1024) / ((bm + bn) * kBK * 2) < 6 ? (210 * 1024) / ((bm + bn) * kBK * 2) : 6;
 }
-enum Epi { EPI_ARGMAX = 0, EPI_LSE = 1, EPI_RACE = 2 };
+enum Epi { EPI_ARGMAX = 0, EPI_LSE = 1, EPI_RACE = 2, EPI_TOPK = 3 };
+
+// EPI_TOPK: the 16 largest values seen by one thread, sorted descending (equal values: lower id
+// first); empty entries are (-inf, -1).
+struct TopK16 {
+  float v[16];
+  int id[16];
+  __device__ __forceinline__ void clear() {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      v[i] = -INFINITY;
+      id[i] = -1;
+    }
+  }
+  // Columns arrive in increasing id, so a value equal to the 16th never displaces it.
+  __device__ __forceinline__ void insert(float x, int c) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {                  // one compare-exchange pass down the list
+      const bool in = x > v[i];
+      const float tv = v[i];
+      const int tc = id[i];
+      v[i] = in ? x : tv;
+      id[i] = in ? c : tc;
+      x = in ? tv : x;
+      c = in ? tc : c;
+    }
+  }
+  // W consecutive columns: the values above the current 16th are staged (in column order) and
+  // inserted by one rolled loop, so the insertion code appears once instead of W times.
+  // Values below `floor` (a lower bound of the row's k-th largest over the whole vocabulary)
+  // cannot be selected and are skipped.
+  template <int W>
+  __device__ __forceinline__ void push_chunk(const float (&x)[W], int col0, int V, float floor) {
+    const float t = v[15];
+    bool any = false;
+#pragma unroll
+    for (int j = 0; j < W; ++j) any |= x[j] > t && x[j] >= floor && col0 + j < V;
+    if (!any) return;
+    float2 buf[W];
+    int n = 0;
+#pragma unroll
+    for (int j = 0; j < W; ++j)
+      if (x[j] > t && x[j] >= floor && col0 + j < V)
+        buf[n++] = make_float2(x[j], __int_as_float(col0 + j));
+#pragma unroll 1
+    for (int i = 0; i < n; ++i)
+      if (buf[i].x > v[15]) insert(buf[i].x, __float_as_int(buf[i].y));
+  }
+};
 
 // Per-row running state of the epilogue over one vocab tile.
 struct EpiRow {
@@ -248,6 +298,8 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
                                                         // with fewer full chunks
     int ai = 0;
     EpiRow st;
+    TopK16 tk;
+    tk.clear();
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++ai) {
       const int buf = ai & 1;
       const uint32_t aph = (ai >> 1) & 1;
@@ -264,7 +316,13 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       const bool active = (BM == 128 || lane < 16) && grow < p.M;
       const uint32_t tbase = tmem + ((uint32_t)(wq * 32) << 16) + buf * BN;
 
-      if (!p.per_cta) st = EpiRow();
+      if (!p.per_cta) {
+        st = EpiRow();
+        if (EPI == EPI_TOPK) tk.clear();
+      }
+      // EPI_TOPK: the largest 16th-best published so far by any thread bounds the row's k-th
+      float tfloor = -INFINITY;
+      if (EPI == EPI_TOPK && active) tfloor = dec_order(__ldcg(p.tkth + grow));
       if (EPI == EPI_LSE && active && p.child_tok) st.ct = p.child_tok[grow];
       const int zr = (EPI == EPI_LSE && active && p.zrow) ? p.zrow[grow] : -1;
       float* zdst = zr >= 0 ? p.zbuf + (size_t)zr * p.V : nullptr;
@@ -349,14 +407,22 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         for (int c = half; c < kChunks; c += 2) {
           float v[32];
           tmem_ld32(tbase + c * 32, v);
-          if (active) epi_chunk<EPI, 32>(p, st, v, nt * BN + c * 32);
+          if constexpr (EPI == EPI_TOPK) {
+            if (active) tk.push_chunk<32>(v, nt * BN + c * 32, p.V, tfloor);
+          } else {
+            if (active) epi_chunk<EPI, 32>(p, st, v, nt * BN + c * 32);
+          }
           if (EPI == EPI_LSE && zdst) store_logits<32>(p, zdst, v, nt * BN + c * 32);
         }
         if constexpr (BN % 32 == 16) {
           if (half == kTailHalf) {
             float v[16];
             tmem_ld16(tbase + kChunks * 32, v);
-            if (active) epi_chunk<EPI, 16>(p, st, v, nt * BN + kChunks * 32);
+            if constexpr (EPI == EPI_TOPK) {
+              if (active) tk.push_chunk<16>(v, nt * BN + kChunks * 32, p.V, tfloor);
+            } else {
+              if (active) epi_chunk<EPI, 16>(p, st, v, nt * BN + kChunks * 32);
+            }
             if (EPI == EPI_LSE && zdst) store_logits<16>(p, zdst, v, nt * BN + kChunks * 32);
           }
         }
@@ -366,7 +432,15 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       if (lane == 0) mbar_arrive(&acce[buf]);
       // per_cta: the row state runs on over this CTA's tiles (increasing ids, so first-seen
       // still means lowest id) and is written once, after the CTA's last tile.
-      if (active && (!p.per_cta || tile + (int)gridDim.x >= p.num_tiles)) {
+      if (EPI == EPI_TOPK && active && tk.v[15] > tfloor)   // 16 values >= it: a valid bound
+        atomicMax(p.tkth + grow, enc_order(tk.v[15]));
+      if (EPI == EPI_TOPK && active && (!p.per_cta || tile + (int)gridDim.x >= p.num_tiles)) {
+        float2* dst = p.topk + ((size_t)grow * p.n_parts * 2 +
+                                (p.per_cta ? (int)blockIdx.x : nt) * 2 + half) * 16;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dst[i] = make_float2(tk.v[i], __int_as_float(tk.id[i]));
+      }
+      if (EPI != EPI_TOPK && active && (!p.per_cta || tile + (int)gridDim.x >= p.num_tiles)) {
         float4 out;
         if (EPI == EPI_ARGMAX)
           out = make_float4(st.r0, __int_as_float(st.r1), st.r2, 0.f);
@@ -448,6 +522,9 @@ static cudaError_t launch_epi(int bn, const CUtensorMap& ta, const CUtensorMap& 
 
 cudaError_t launch_lmhead(int epi, int bn, int bm, const CUtensorMap& ta, const CUtensorMap& tb,
                           const GemmParams& p, int grid, cudaStream_t stream) {
+  if (epi == EPI_TOPK)
+    return bm == 64 ? launch_epi<EPI_TOPK, 64>(bn, ta, tb, p, grid, stream)
+                    : launch_epi<EPI_TOPK, 128>(bn, ta, tb, p, grid, stream);
   if (bm == 64) {
     if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX, 64>(bn, ta, tb, p, grid, stream);
     if (epi == EPI_LSE) return launch_epi<EPI_LSE, 64>(bn, ta, tb, p, grid, stream);

@@ -38,7 +38,7 @@ GAMMA = 10.0
 _TAGS = {
     "tree": 1, "tokens": 2, "plant": 3, "q": 4, "k_tree": 5, "v_tree": 6, "k_cache": 7,
     "v_cache": 8, "hidden": 9, "w_lm": 10, "kv_len": 11, "draft_logits": 12, "draft_pick": 13,
-    "pages": 14,
+    "pages": 14, "lr_u": 15, "lr_d": 16, "lr_noise": 17, "lr_hidden": 18,
 }
 
 CONFIGS: dict[str, dict] = {
@@ -380,3 +380,47 @@ def paged(wl: "Workload", page_size: int, spare_pages: int = 3, seed: int = 0) -
             vp[page * P:page * P + hi - lo] = wl.v_cache[base + lo:base + hi]
     return PagedCache(page_size=P, max_pages=maxp, num_pages=total, block_table=bt, k_pool=kp,
                       v_pool=vp, slot_cap=np.array([n * P for n in npg], dtype=np.int32))
+
+
+# ----------------------------------------------------------------- low-rank candidate head
+LOWRANK = {
+    # the draft head's shape at the 27B-class vocabulary: 64 tree nodes per call
+    "lowrank_r512": dict(M=64, H=5120, V=151936, r=512, k=16),
+    "lowrank_r128": dict(M=64, H=5120, V=151936, r=128, k=16),
+    "lowrank_tiny": dict(M=9, H=256, V=4096 + 77, r=64, k=8),
+}
+
+
+@dataclass
+class LowRankWorkload:
+    name: str
+    M: int
+    H: int
+    V: int
+    r: int
+    k: int
+    hidden: torch.Tensor     # bf16 [M, H]
+    D: torch.Tensor          # bf16 [r, H]
+    U: torch.Tensor          # bf16 [V, r]
+    W: torch.Tensor          # bf16 [V, H]
+
+
+def lowrank(name: str, **over) -> LowRankWorkload:
+    """Factors and head of a low-rank candidate screen.  U, D ~ N(0, s) with s^4 r = 0.02^2, so
+    U D has the full head's N(0, 0.02) scale; the exact head is W = U D + N(0, 0.005) (a head
+    that the factors approximate but do not equal); hidden rows N(0, 1)."""
+    cfg = dict(LOWRANK[name])
+    cfg.update(over)
+    M, H, V, r, k = cfg["M"], cfg["H"], cfg["V"], cfg["r"], cfg["k"]
+    seed = 0xE7EE0100 + sum(map(ord, name))
+    s = (0.02 ** 2 / r) ** 0.25
+    Uf = normal_f32(V * r, s, seed, "lr_u").reshape(V, r)
+    Df = normal_f32(r * H, s, seed, "lr_d").reshape(r, H)
+    Ub = torch.from_numpy(Uf).to(torch.bfloat16)
+    Db = torch.from_numpy(Df).to(torch.bfloat16)
+    Wf = torch.from_numpy(normal_f32(V * H, 0.005, seed, "lr_noise").reshape(V, H))
+    Wf += Ub.float() @ Db.float()
+    hidden = torch.from_numpy(normal_f32(M * H, 1.0, seed, "lr_hidden").reshape(M, H))
+    return LowRankWorkload(name=name, M=M, H=H, V=V, r=r, k=k,
+                           hidden=hidden.to(torch.bfloat16), D=Db, U=Ub,
+                           W=Wf.to(torch.bfloat16))

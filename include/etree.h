@@ -252,6 +252,29 @@ etree_status etree_kv_compact_paged(const etree_batch *batch, const int32_t *blo
                                     size_t workspace_bytes, void *stream);
 
 /*
+ * Low-rank candidate head: screen the vocabulary with a factorised projection, then score only
+ * the survivors exactly.  EAGLE-4's draft uses such a head in place of its full vocabulary
+ * projection ("EAGLE-4 是什麼？...", aiposthub.com, section "EAGLE-4 是什麼？先看推測解碼為什麼能變快",
+ * Fig. 2: the vocab head is 65.4% of a 574 us draft forward; rank 512 brings the forward to
+ * 326 us, rank 128 to 255 us).  For each of M rows h (hidden [M][hidden_dim] bf16):
+ *   g  = h D^T   (D [rank][hidden_dim] bf16), fp32 accumulation, rounded to bf16;
+ *   z~ = g U^T   (U [vocab][rank] bf16), fp32 accumulation: the approximate logits;
+ *   C  = the k ids of largest z~ (lower id first on equal values), 1 <= k <= 16;
+ *   z_c = h . W_c (W [vocab][hidden_dim] bf16, the exact head), fp32 accumulation;
+ * out_ids [M][k] holds C ordered by z_c descending (lower id first on equal values) and
+ * out_logit [M][k] the z_c.  hidden_dim and rank are multiples of 64, at most 8192.  The
+ * workspace (etree_lowrank_workspace_size bytes, 16-byte aligned, status words cleared by
+ * etree_workspace_init) is independent of the verification workspace; etree_device_status reads
+ * its status.  All pointers are device pointers, 16-byte aligned.  Asynchronous on `stream`.
+ */
+size_t etree_lowrank_workspace_size(int M, int hidden_dim, int rank, int vocab);
+etree_status etree_lowrank_candidates(const uint16_t *hidden, int M, int hidden_dim,
+                                      const uint16_t *D, const uint16_t *U, int rank,
+                                      const uint16_t *W, int vocab, int k, int32_t *out_ids,
+                                      float *out_logit, void *workspace, size_t workspace_bytes,
+                                      void *stream);
+
+/*
  * Hardware-aware tree sizing (host-only; no device work).  The pages size the draft tree from the
  * measured cost of drafting and verifying at the running batch size and hardware
  * ("EAGLE-4 官方推理代码发布 ...", arex-research.com, section "投机树多大，由实测成本决定").

@@ -302,3 +302,35 @@ def compact_compare(wl, dev, ores, requests, excused):
         assert np.array_equal(gk, sub_k), r
         assert np.array_equal(gv, sub_v), r
         assert kv_out[r] == newlen[0], (r, kv_out[r], newlen[0])
+
+
+LR_SCREEN_TOL = 1e-3    # |z~ - k-th z~| allowed for a candidate-set difference (g's bf16 rounding)
+
+
+def lowrank_compare(lw, ids, logit, nthreads=0):
+    """The GPU's candidates against the oracle's.  Candidate sets must agree except for ids whose
+    approximate logit lies within LR_SCREEN_TOL (1 + |k-th|) of the k-th (the screen's operand g is
+    bf16, so fp32-vs-fp64 rounding of g can move such ids across the cut); exact logits of common
+    ids within 1e-3 (1 + |z|); the order by exact logit must agree except between candidates whose
+    fp64 logits differ by less than 1e-3.  Returns the number of rows with a set difference."""
+    oid, olg, kth, za = oracle.lowrank_candidates(lw.hidden, lw.D, lw.U, lw.W, lw.k,
+                                                  keep_approx=True, nthreads=nthreads)
+    differ = 0
+    for m in range(lw.M):
+        sg, so = set(ids[m].tolist()), set(oid[m].tolist())
+        tol = LR_SCREEN_TOL * (1.0 + abs(kth[m]))
+        for c in sg ^ so:
+            assert 0 <= c < lw.V and abs(za[m, c] - kth[m]) <= tol, (m, c, za[m, c], kth[m])
+        differ += int(sg != so)
+        o_of = dict(zip(oid[m].tolist(), olg[m].tolist()))
+        for i, c in enumerate(ids[m].tolist()):
+            if c in o_of:
+                z = o_of[c]
+                assert abs(logit[m, i] - z) <= 1e-3 * (1.0 + abs(z)), (m, c, logit[m, i], z)
+        # ordering: consecutive GPU entries that are both oracle candidates keep the oracle order
+        # unless their fp64 logits are within 1e-3
+        common = [c for c in ids[m].tolist() if c in o_of]
+        for a, b in zip(common, common[1:]):
+            za_, zb_ = o_of[a], o_of[b]
+            assert za_ > zb_ or abs(za_ - zb_) < 1e-3 or (za_ == zb_ and a < b), (m, a, b, za_, zb_)
+    return differ

@@ -315,3 +315,37 @@ def test_batch64_paged16_full_size():
     g = np.random.default_rng(4)
     reqs = sorted(g.choice(wl.B, 6, replace=False).tolist())
     _paged_check(wl, 16, attn_rows=P.sample_rows(wl, 4), requests=reqs)
+
+
+# -------------------------------------------------------------------- low-rank candidate head
+def _lowrank_run(lw):
+    from draft_tree_verification_masked_b200 import (etree_lowrank_candidates,
+                                                     etree_lowrank_workspace_size,
+                                                     etree_workspace_init, etree_device_status)
+    dev = torch.device("cuda")
+    h, D, U, Wt = (x.to(dev) for x in (lw.hidden, lw.D, lw.U, lw.W))
+    ws = torch.zeros(etree_lowrank_workspace_size(lw.M, lw.H, lw.r, lw.V), dtype=torch.uint8,
+                     device=dev)
+    etree_workspace_init(ws)
+    ids = torch.full((lw.M, lw.k), -7, dtype=torch.int32, device=dev)
+    lg = torch.empty(lw.M, lw.k, dtype=torch.float32, device=dev)
+    etree_lowrank_candidates(h, D, U, Wt, lw.k, ids, lg, ws)
+    assert etree_device_status(ws) == (0, 0)
+    return ids.cpu().numpy(), lg.cpu().numpy()
+
+
+@pytest.mark.parametrize("over", [dict(), dict(k=16), dict(k=1), dict(r=128, k=5),
+                                  dict(M=130, V=3000, k=12), dict(M=64, V=20000, r=192, k=16)])
+def test_lowrank_candidates_small(over):
+    lw = W.lowrank("lowrank_tiny", **over)
+    ids, lg = _lowrank_run(lw)
+    differ = P.lowrank_compare(lw, ids, lg)
+    assert differ <= max(1, lw.M // 10), differ
+
+
+@pytest.mark.parametrize("name", ["lowrank_r512", "lowrank_r128"])
+def test_lowrank_candidates_full_size(name):
+    lw = W.lowrank(name)
+    ids, lg = _lowrank_run(lw)
+    differ = P.lowrank_compare(lw, ids, lg)
+    assert differ <= max(1, lw.M // 10), differ
