@@ -314,21 +314,38 @@ __global__ void attn_combine_kernel(AttnParams p, int n_total) {
   if (n < 1 || n > p.n_max || L < 0 || L > p.kv_len_max) return;   // reported by the main kernel
   const int total = (L + p.keys - 1) / p.keys + (n + p.keys - 1) / p.keys;
   const int used = min(p.nsplit, (total + p.tps - 1) / p.tps);
+  // splits in groups of 4 so that each group's loads are in flight together
+  const float2* mlp = p.ml_part + (size_t)gw * p.nsplit;
+  const float4* op = reinterpret_cast<const float4*>(p.o_part + (size_t)gw * p.nsplit * 128);
   float M = -INFINITY;
-  for (int s = 0; s < used; ++s) M = fmaxf(M, p.ml_part[(size_t)gw * p.nsplit + s].x);
+  for (int s0 = 0; s0 < used; s0 += 4) {
+    float mx[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mx[i] = s0 + i < used ? mlp[s0 + i].x : -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) M = fmaxf(M, mx[i]);
+  }
   const float Mb = (M == -INFINITY) ? 0.f : M;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float lsum = 0.f;
-  for (int s = 0; s < used; ++s) {
-    const float2 ml = p.ml_part[(size_t)gw * p.nsplit + s];
-    const float w = exp2f(ml.x - Mb);
-    lsum += ml.y * w;
-    const float4 v =
-        reinterpret_cast<const float4*>(p.o_part + ((size_t)gw * p.nsplit + s) * 128)[lane];
-    acc.x += v.x * w;
-    acc.y += v.y * w;
-    acc.z += v.z * w;
-    acc.w += v.w * w;
+  for (int s0 = 0; s0 < used; s0 += 4) {
+    float2 ml[4];
+    float4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool in = s0 + i < used;
+      ml[i] = in ? mlp[s0 + i] : make_float2(-INFINITY, 0.f);
+      v[i] = in ? op[(size_t)(s0 + i) * 32 + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float w = s0 + i < used ? exp2f(ml[i].x - Mb) : 0.f;
+      lsum += ml[i].y * w;
+      acc.x += v[i].x * w;
+      acc.y += v[i].y * w;
+      acc.z += v[i].z * w;
+      acc.w += v[i].w * w;
+    }
   }
   const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
   uint2 packed;
