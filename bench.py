@@ -456,7 +456,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="etree", choices=["etree", "reference"])
     ap.add_argument("--config", default="dense27b_b1")
-    ap.add_argument("--by-batch", default="batch64,conc512,tree64_t1,batch64@p16",
+    ap.add_argument("--by-batch", default="batch64,conc512,tree64_t1,long32k,long128k,batch64@p16",
                     help="extra workloads measured in the same run (comma list, '' for none; "
                          "<workload>@p<N> runs it on a paged cache of N-token pages)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

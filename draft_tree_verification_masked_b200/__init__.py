@@ -348,11 +348,18 @@ def etree_verify_attn_paged(batch: Batch, block_table, page_size: int, q, k_tree
     return _check(st) if check else st
 
 
+def _check_path(batch: Batch, path):
+    # the library reads a full row of ETREE_PATH_STRIDE entries per request
+    if isinstance(path, torch.Tensor) and path.numel() < batch.B * 64:
+        raise ValueError(f"path must hold [B][64] entries, got {tuple(path.shape)}")
+
+
 def etree_kv_compact_paged(batch: Batch, block_table, page_size: int, accept_len, path, k_tree,
                            v_tree, k_pool, v_pool, num_pages: int, n_layers: int,
                            tree_layer_stride: int, cache_layer_stride: int, kv_len_out,
                            workspace, stream=None, check: bool = True) -> int:
     bf = torch.bfloat16
+    _check_path(batch, path)
     hkv, d = k_tree.shape[-2], k_tree.shape[-1]
     st = lib().etree_kv_compact_paged(
         C.byref(batch), _ptr(block_table, torch.int32, "block_table"), block_table.shape[1],
@@ -369,6 +376,7 @@ def etree_kv_compact(batch: Batch, accept_len, path, k_tree, v_tree, k_cache, v_
                      n_layers: int, tree_layer_stride: int, cache_layer_stride: int, kv_len_out,
                      workspace, stream=None, check: bool = True) -> int:
     bf = torch.bfloat16
+    _check_path(batch, path)
     hkv, d = k_tree.shape[-2], k_tree.shape[-1]
     st = lib().etree_kv_compact(
         C.byref(batch), _ptr(accept_len, torch.int32, "accept_len"),

@@ -58,7 +58,8 @@ struct AttnPlan {
 
 // Launch plan of the attention call.  The tcgen05 kernel (default) takes 128-row blocks of
 // nb = min(floor(128 / G), n_max) whole nodes; with at least one (request, KV head, row block) per
-// SM it uses 32-key tiles and two CTAs per SM, otherwise 64-key tiles and one CTA per SM.  The KV range
+// SM, or 64K or more cached keys, it uses 32-key tiles and two CTAs per SM, otherwise 64-key tiles
+// and one CTA per SM.  The KV range
 // is split only to fill one wave of CTAs (a second, partial wave costs more than longer splits),
 // keeping >= 4 key tiles per split.  The warp-MMA kernel (ETREE_ATTN=mma) takes 16-row warps,
 // 64-key tiles, and aims at about four CTAs per SM.
@@ -73,9 +74,10 @@ static AttnPlan plan_attn(const etree_batch* b, int hq, int hkv) {
     pl.mchunks = (b->n_max + pl.nb - 1) / pl.nb;
     pl.nw = 4;
     const int pairs0 = b->B * hkv * pl.mchunks;
-    // 32-key tiles (two CTAs per SM) pay off once there is at least one row block per SM;
-    // few, long work items (one request, long context) prefer 64-key tiles split over the SMs
-    pl.keys = pairs0 >= sms ? 32 : 64;
+    // 32-key tiles (two CTAs per SM) pay off once there is at least one row block per SM, and
+    // on very long contexts (>= 64K keys: measured 5-8% faster at 128K, 5% slower at 32K);
+    // otherwise few, long work items prefer 64-key tiles split over the SMs
+    pl.keys = (pairs0 >= sms || b->kv_len_max >= 65536) ? 32 : 64;
     const int forced = env_int("ETREE_ATTN_KEYS", 0);
     if (forced == 32 || forced == 64) pl.keys = forced;
   } else {
@@ -800,7 +802,9 @@ static etree_status kv_compact_impl(const etree_batch* b, const int32_t* accept_
   p.max_pages = pg ? pg->max_pages : 0;
   p.page_shift = pg ? log2i(pg->page_size) : 0;
   p.cache_slots = pool_slots;
-  cudaError_t e = launch_compact(p, sm_count(), static_cast<cudaStream_t>(stream));
+  // the layers are spread over about 16 CTAs per SM (ETREE_COMPACT_PER_SM overrides)
+  const int per_sm = std::max(1, env_int("ETREE_COMPACT_PER_SM", 16));
+  cudaError_t e = launch_compact(p, per_sm * sm_count(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_kv_compact launch");
 }
 

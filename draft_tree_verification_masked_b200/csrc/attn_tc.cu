@@ -16,8 +16,9 @@
 // warps share a row, 32 keys each, and exchange row maxima): they read S from TMEM, apply
 // the key mask (cache length, or the row's ancestor bitmask on the tree tiles), run the online
 // softmax in log2 units, and write P (bf16) back into their own TMEM lane, where the PV product
-// takes it as its A operand; shared memory holds only Q and the K/V ring.  S and P are
-// double-buffered so QK^T of tile j+1 and PV of tile j overlap the softmax.  O is rescaled
+// takes it as its A operand; shared memory holds only Q and the K/V ring.  S and P have three
+// buffers each in the 64-key shape (QK^T issued two tiles ahead of PV) and two in the 32-key
+// shape (one tile ahead), so the tensor core works on later tiles while the softmax runs.  O is rescaled
 // lazily: only when a row's running maximum grows by more than 2^8 does the softmax
 // read-modify-write O in TMEM, so P stays below 256 and the usual case has no O traffic.
 //
@@ -35,13 +36,13 @@ constexpr float kLazy = 8.0f;               // rescale O only when the max grows
 
 struct TcSmem {
   // barriers and small arrays, placed after the 1024-aligned tile area
-  uint64_t kv_full[6], kv_empty[6], q_full, s_full[2], s_free[2], p_full[2], p_free[2];
+  uint64_t kv_full[6], kv_empty[6], q_full, s_full[3], s_free[3], p_full[3], p_free[3];
   uint64_t drain;                           // the MMA issuer's last commit, waited on at exit
   uint64_t anc[64];
   int32_t par[64];
-  float xmax[2][2][128];                    // row-max exchange: [tile parity][key half][row]
-  float xl[2][128];                         // final row sums of the two key halves
-  uint64_t xbar[4][2], xlbar[4];            // exchange barriers of the warp pairs (bounded waits)
+  float xmax[2][4][128];                    // row-max exchange: [tile parity][key part][row]
+  float xl[4][128];                         // final row sums of the key parts
+  uint64_t xbar[4][2], xlbar[4];            // exchange barriers per lane quarter (bounded waits)
   uint32_t tmem;
 };
 
@@ -49,10 +50,20 @@ template <int KEYS>
 struct TcShape {
   static constexpr int kBox = KEYS * 128;   // one [KEYS keys][64 dims] bf16 box
   static constexpr int kKV = 4 * kBox;      // K lo/hi + V lo/hi
-  // TMEM columns: S double buffer at [0, 2 KEYS), O at [128, 256), then the P double buffer
-  // (bf16, KEYS / 2 columns each) at kPCol; the 64-key shape allocates 512 columns.
-  static constexpr int kPCol = KEYS == 64 ? 256 : 64;
+  // kNS S buffers (fp32, KEYS columns each) at [0, kNS KEYS), O (128 columns) at kOCol, kNP P
+  // buffers (bf16 pairs, KEYS / 2 columns each) at kPCol.  QK^T runs kLag tiles ahead of PV.
+  // 64 keys: S [0, 192), O [256, 384), P [384, 480) of 512 columns; 32 keys (two CTAs per SM):
+  // S [0, 64), P [64, 96), O [128, 256) of 256 columns.  (Measured on the 32-key shape, a third
+  // S buffer with a two-tile lead was slower.)
+  static constexpr int kNS = KEYS == 64 ? 3 : 2;
+  static constexpr int kNP = KEYS == 64 ? 3 : 2;
+  static constexpr int kLag = kNS - 1;
+  static constexpr int kOCol = KEYS == 64 ? 256 : 128;
+  static constexpr int kPCol = KEYS == 64 ? 384 : 64;
   static constexpr int kTmemCols = KEYS == 64 ? 512 : 256;
+  static_assert(kNS * KEYS <= kPCol && kNS * KEYS <= kOCol, "S overlaps P or O");
+  static_assert(kPCol + kNP * KEYS / 2 <= kOCol || kOCol + 128 <= kPCol, "P overlaps O");
+  static_assert(kPCol + kNP * KEYS / 2 <= kTmemCols && kOCol + 128 <= kTmemCols, "TMEM");
 };
 }  // namespace
 
@@ -113,16 +124,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     mbar_init(&sh->q_full, 1);
     mbar_init(&sh->drain, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&sh->s_full[b], 1);
       mbar_init(&sh->s_free[b], SW);
       mbar_init(&sh->p_full[b], SW);
       mbar_init(&sh->p_free[b], 1);
     }
     for (int q = 0; q < 4; ++q) {
-      mbar_init(&sh->xbar[q][0], 2);
-      mbar_init(&sh->xbar[q][1], 2);
-      mbar_init(&sh->xlbar[q], 2);
+      mbar_init(&sh->xbar[q][0], SW / 4);
+      mbar_init(&sh->xbar[q][1], SW / 4);
+      mbar_init(&sh->xlbar[q], SW / 4);
     }
     fence_barrier_init();
   }
@@ -251,25 +262,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc_fence_after();
       const uint64_t dq0 = smem_desc_sw128(sQ), dq1 = smem_desc_sw128(sQ + 16384);
       auto pv = [&](int jj) -> bool {
-        const int pb = jj & 1;
-        if (!mbar_wait(&sh->p_full[pb], (jj >> 1) & 1)) return false;
+        const int pb = jj % Sh::kNP;
+        if (!mbar_wait(&sh->p_full[pb], (jj / Sh::kNP) & 1)) return false;
         tc_fence_after();
         // A = P from TMEM (16 keys = 8 columns per MMA), B = V from shared memory
         const uint32_t pa = tmem + Sh::kPCol + pb * (KEYS / 2);
         const uint8_t* v0 = sKV + (jj % STAGES) * Sh::kKV + 2 * Sh::kBox;
 #pragma unroll
         for (int k = 0; k < KEYS / 16; ++k)
-          tc_mma_bf16_ts(tmem + 128, pa + 8 * k, smem_desc_sw128_mn(v0 + k * 2048, Sh::kBox), idO,
+          tc_mma_bf16_ts(tmem + Sh::kOCol, pa + 8 * k, smem_desc_sw128_mn(v0 + k * 2048, Sh::kBox), idO,
                          (jj > 0 || k > 0) ? 1u : 0u);
         tc_commit(&sh->p_free[pb]);
         tc_commit(&sh->kv_empty[jj % STAGES]);
         return true;
       };
+      // QK^T of tile j is issued before PV of tile j - kLag, so the softmax finds the next
+      // kLag score tiles computed while it works on one
       for (int j = 0; ok && j < T; ++j) {
         const int st = j % STAGES;
-        const int sb = j & 1;
+        const int sb = j % Sh::kNS;
         if (!mbar_wait(&sh->kv_full[st], (j / STAGES) & 1)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(&sh->s_free[sb], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+        if (j >= Sh::kNS && !mbar_wait(&sh->s_free[sb], ((j / Sh::kNS) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint8_t* k0 = sKV + st * Sh::kKV;
         const uint64_t dk0 = smem_desc_sw128(k0), dk1 = smem_desc_sw128(k0 + Sh::kBox);
@@ -278,9 +294,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tc_mma_bf16(tmem + sb * KEYS, (k < 4 ? dq0 : dq1) + 2 * (k & 3),
                       (k < 4 ? dk0 : dk1) + 2 * (k & 3), idS, k > 0 ? 1u : 0u);
         tc_commit(&sh->s_full[sb]);
-        if (j >= 1 && !pv(j - 1)) { ok = false; break; }
+        if (j >= Sh::kLag && !pv(j - Sh::kLag)) { ok = false; break; }
       }
-      if (ok && !pv(T - 1)) ok = false;
+      for (int jj = T > Sh::kLag ? T - Sh::kLag : 0; ok && jj < T; ++jj)
+        if (!pv(jj)) ok = false;
       // every MMA issued above completes before TMEM is released
       tc_commit(&sh->drain);
       if (!mbar_wait(&sh->drain, 0)) ok = false;
@@ -288,7 +305,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------------- softmax warps
-    // SW/4 warps per TMEM lane quarter; warp half `kh` of a quarter owns keys
+    // SW/4 warps per TMEM lane quarter; key part `kh` of a quarter owns keys
     // [kh*CW, kh*CW + CW) of every tile (CW = KEYS / (SW/4)) and O columns [kh*OW, kh*OW + OW).
     constexpr int NH = SW / 4;
     constexpr int CW = KEYS / NH;
@@ -307,20 +324,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int t = t0 + j;
-      const int sb = j & 1;
-      if (!mbar_wait(&sh->s_full[sb], (j >> 1) & 1)) { ok = false; break; }
+      const int sb = j % Sh::kNS;
+      if (!mbar_wait(&sh->s_full[sb], (j / Sh::kNS) & 1)) { ok = false; break; }
       tc_fence_after();
       float sc[CW];
-      {
-        float a[32];
-        tmem_ld32(lane_base + sb * KEYS + kh * CW, a);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) sc[c] = a[c];
-        if constexpr (CW == 64) {
-          tmem_ld32(lane_base + sb * KEYS + 32, a);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) sc[32 + c] = a[c];
-        }
+      if constexpr (CW == 32) {
+        tmem_ld32(lane_base + sb * KEYS + kh * CW, sc);
+      } else {
+        tmem_ld16(lane_base + sb * KEYS + kh * CW, sc);
       }
       tc_fence_before();
       __syncwarp();
@@ -332,25 +343,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int k0 = kh * CW;                           // first key of this thread in the tile
       const bool full_tile = t < nt_cache && L - t * KEYS >= KEYS;
       if (!full_tile) {
-        uint32_t kw[CW / 32];
+        uint32_t kw;                                    // bit c: key k0 + c is visible
         if (!valid) {
-#pragma unroll
-          for (int w = 0; w < CW / 32; ++w) kw[w] = 0u;
+          kw = 0u;
         } else if (t >= nt_cache) {
-          const int sh0 = (t - nt_cache) * KEYS + k0;
-#pragma unroll
-          for (int w = 0; w < CW / 32; ++w) kw[w] = static_cast<uint32_t>(anc >> (sh0 + 32 * w));
+          const int sh0 = (t - nt_cache) * KEYS + k0;   // < 64: tree tiles start at node 0
+          kw = static_cast<uint32_t>(anc >> sh0);
         } else {
           const int lim = L - t * KEYS - k0;
-#pragma unroll
-          for (int w = 0; w < CW / 32; ++w) {
-            const int lw = lim - 32 * w;
-            kw[w] = lw >= 32 ? 0xffffffffu : (lw > 0 ? ((1u << lw) - 1u) : 0u);
-          }
+          kw = lim >= 32 ? 0xffffffffu : (lim > 0 ? ((1u << lim) - 1u) : 0u);
         }
 #pragma unroll
         for (int c = 0; c < CW; ++c)
-          if (!((kw[c >> 5] >> (c & 31)) & 1u)) sc[c] = -INFINITY;
+          if (!((kw >> c) & 1u)) sc[c] = -INFINITY;
       }
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -380,19 +385,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ls0 = a0;
         ls1 = a1;
       };
-      // With two warps per row the row maximum needs the partner's half.  A row that already
-      // has a reference computes P against it while the partner's maximum is in flight, and
+      // With NH warps per row the row maximum needs the other warps' key parts.  A row that
+      // already has a reference computes P against it while those maxima are in flight, and
       // recomputes only when the combined maximum moves the reference (rare: see kLazy).
-      if constexpr (NH == 2) {
+      if constexpr (NH > 1) {
         sh->xmax[j & 1][kh][row] = tmax;
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->xbar[wq][j & 1]);
       }
-      const bool early = NH == 2 && __all_sync(0xffffffffu, m_ref != -INFINITY);
+      const bool early = NH > 1 && __all_sync(0xffffffffu, m_ref != -INFINITY);
       if (early) exps(m_ref);
-      if constexpr (NH == 2) {
+      if constexpr (NH > 1) {
         if (!mbar_wait(&sh->xbar[wq][j & 1], (j >> 1) & 1)) { ok = false; break; }
-        tmax = fmaxf(tmax, sh->xmax[j & 1][kh ^ 1][row]);
+#pragma unroll
+        for (int h = 1; h < NH; ++h) tmax = fmaxf(tmax, sh->xmax[j & 1][kh ^ h][row]);
       }
       const float tms = tmax * sl;                      // row maximum in log2 units
       const bool need = tms > m_ref + kLazy;            // also true for the first finite max
@@ -404,39 +410,48 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       m_ref = m_new;
       // A rescale of O needs every earlier PV product finished (the last one wrote O).
       if (any && j >= 1) {
-        if (!mbar_wait(&sh->p_free[(j - 1) & 1], ((j - 1) >> 1) & 1)) { ok = false; break; }
+        if (!mbar_wait(&sh->p_free[(j - 1) % Sh::kNP], ((j - 1) / Sh::kNP) & 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < OW / 32; ++c) {
           float o[32];
-          const uint32_t ta = lane_base + 128 + kh * OW + c * 32;
+          const uint32_t ta = lane_base + Sh::kOCol + kh * OW + c * 32;
           tmem_ld32(ta, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= corr;
           tmem_st32(ta, o);
         }
       }
-      // P buffer j % 2 is free once PV(j - 2) has completed
-      const int pb = j & 1;
-      if (j >= 2) {
-        if (!mbar_wait(&sh->p_free[pb], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+      // P buffer j % kNP is free once PV(j - kNP) has completed
+      const int pb = j % Sh::kNP;
+      if (j >= Sh::kNP) {
+        if (!mbar_wait(&sh->p_free[pb], ((j / Sh::kNP) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
       }
       // this thread's CW keys of P into its own TMEM lane (the PV product's A operand)
-      static_assert(CW == 32, "one 16-column P store per thread");
-      tmem_st16(lane_base + Sh::kPCol + pb * (KEYS / 2) + kh * (CW / 2), pk);
+      static_assert(CW == 32 || CW == 16, "a 16- or 8-column P store per thread");
+      if constexpr (CW == 32) {
+        tmem_st16(lane_base + Sh::kPCol + pb * (KEYS / 2) + kh * (CW / 2), pk);
+      } else {
+        tmem_st8(lane_base + Sh::kPCol + pb * (KEYS / 2) + kh * (CW / 2), pk);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->p_full[pb]);
     }
-    if (ok && !mbar_wait(&sh->p_free[(T - 1) & 1], ((T - 1) >> 1) & 1)) ok = false;
+    if (ok && !mbar_wait(&sh->p_free[(T - 1) % Sh::kNP], ((T - 1) / Sh::kNP) & 1)) ok = false;
     if (!ok) report(p.ws, ETREE_ETIMEOUT, DET_WAIT_ATTN);
-    if constexpr (NH == 2) {                            // the row sum covers both key halves
+    if constexpr (NH > 1) {                             // the row sum covers every key part
       sh->xl[kh][row] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->xlbar[wq]);
       if (!mbar_wait(&sh->xlbar[wq], 0)) report(p.ws, ETREE_ETIMEOUT, DET_WAIT_ATTN);
-      l += sh->xl[kh ^ 1][row];
+      l = 0.f;
+#pragma unroll
+      for (int h = 0; h < NH; ++h) l += sh->xl[h][row];
     }
     tc_fence_after();
     const size_t gidx = (size_t)(base + (valid ? node : 0)) * p.hq + kvh * G + g;
@@ -446,7 +461,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       for (int c = 0; c < OW / 32; ++c) {
         const int col = kh * OW + c * 32;
         float o[32];
-        tmem_ld32(lane_base + 128 + col, o);
+        tmem_ld32(lane_base + Sh::kOCol + col, o);
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(p.out + gidx * 128 + col);
 #pragma unroll
@@ -464,7 +479,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       for (int c = 0; c < OW / 32; ++c) {
         const int col = kh * OW + c * 32;
         float o[32];
-        tmem_ld32(lane_base + 128 + col, o);
+        tmem_ld32(lane_base + Sh::kOCol + col, o);
         if (valid) {
           float4* dst = reinterpret_cast<float4*>(op + col);
 #pragma unroll

@@ -15,28 +15,39 @@
 namespace etree {
 
 
-// One CTA per (request, chunk of layers).  Its first two warps read the request's accept length
-// and path entries in parallel and validate them once; then all 256 threads stream the
-// 2 x (a + 1) rows of every layer in the chunk, one 16-byte word per thread per row and
-// tensor (K, V), four rows in flight per thread.
-__global__ void __launch_bounds__(256) kv_compact_kernel(CompactParams p, int layers_per_cta) {
-  __shared__ int src_s[64];
-  __shared__ long long dst_s[64];
-  __shared__ int rows_s, code_s, detail_s, bad_s, badpage_s;
+// One CTA per (request, chunk of layers).  Thread 0 reads and validates the request's header
+// while the first 64 threads read its path row; the first a + 1 threads then form the source
+// rows and the destination slots.  The copy treats the chunk as a flat list of items, one item being one moved row
+// (layer, k) for both tensors.  A row is w16 16-byte words for K followed by w16 for V; each
+// thread owns one word column and walks the items with kUnroll independent loads in flight
+// before their stores, so a copy of a few rows per layer is not serialised layer by layer.
+constexpr int kCompactThreads = 256;
+constexpr int kUnroll = 8;
+
+__global__ void __launch_bounds__(kCompactThreads)
+    kv_compact_kernel(CompactParams p, int layers_per_cta) {
+  __shared__ int path_s[ETREE_PATH_STRIDE], src_s[64];
+  __shared__ long long dst_s[64], slot0_s;
+  __shared__ int rows_s, code_s, detail_s, bad_s, badpage_s, nbase_s, n_s, L_s;
   const int r = blockIdx.x;
   const int l0 = blockIdx.y * layers_per_cta;
   const int l1 = min(p.n_layers, l0 + layers_per_cta);
   const int tid = threadIdx.x;
+  // One DRAM round trip: the whole path row (it always has ETREE_PATH_STRIDE entries) is read
+  // beside the request's header, before the accept length says how much of it is used.
+  if (tid < ETREE_PATH_STRIDE) path_s[tid] = p.path[(size_t)r * ETREE_PATH_STRIDE + tid];
   if (tid == 0) {
     const int base = p.cu_nodes[r];
     const int n = p.cu_nodes[r + 1] - base;
     const int a = p.accept_len[r];
     const int L = p.kv_len[r];
+    const int cap = p.slot_cap[r];
+    const long long sb = p.slot_base[r];
     int code = ETREE_OK, detail = DET_NONE;
     if (n < 1 || n > p.n_max || a < 0 || a >= n || L < 0) {
       code = ETREE_EDEVICE;
       detail = DET_BAD_PATH;
-    } else if ((int64_t)L + a + 1 > (int64_t)p.slot_cap[r]) {
+    } else if ((int64_t)L + a + 1 > (int64_t)cap) {
       code = ETREE_ENOSPACE;
       detail = DET_CAPACITY;
     }
@@ -45,19 +56,21 @@ __global__ void __launch_bounds__(256) kv_compact_kernel(CompactParams p, int la
     rows_s = code == ETREE_OK ? a + 1 : 0;
     bad_s = 0;
     badpage_s = 0;
+    nbase_s = base;
+    n_s = n;
+    L_s = L;
+    slot0_s = sb + L;
   }
   __syncthreads();
   const int rows0 = rows_s;
-  if (tid < rows0) {                                   // path entries and destinations
-    const int base = p.cu_nodes[r];
-    const int n = p.cu_nodes[r + 1] - base;
-    const int j = p.path[(size_t)r * ETREE_PATH_STRIDE + tid];
-    if (j < 0 || j >= n) atomicOr(&bad_s, 1);
-    src_s[tid] = base + j;
-    const long long pos = (long long)p.kv_len[r] + tid;
+  if (tid < rows0) {                                   // sources and destinations
+    const int j = path_s[tid];
+    if (j < 0 || j >= n_s) atomicOr(&bad_s, 1);
+    src_s[tid] = nbase_s + j;
     if (!p.block_table) {
-      dst_s[tid] = p.slot_base[r] + pos;
+      dst_s[tid] = slot0_s + tid;
     } else {
+      const long long pos = (long long)L_s + tid;
       const long long pi = pos >> p.page_shift;
       const int page = pi < p.max_pages ? p.block_table[(size_t)r * p.max_pages + pi] : -1;
       const long long slot = ((long long)page << p.page_shift) + (pos & ((1 << p.page_shift) - 1));
@@ -76,44 +89,52 @@ __global__ void __launch_bounds__(256) kv_compact_kernel(CompactParams p, int la
       detail = DET_BAD_PAGE;
     }
     if (code != ETREE_OK) report(p.ws, code, detail);
-    p.kv_len_out[r] = code == ETREE_OK ? p.kv_len[r] + rows0 : p.kv_len[r];
+    p.kv_len_out[r] = L_s + (code == ETREE_OK ? rows0 : 0);
   }
   const int rows = (bad_s || badpage_s) ? 0 : rows0;
   if (rows == 0) return;
-  const int w16 = p.row16;                            // 16-byte words per row
-  for (int layer = l0; layer < l1; ++layer) {
-    const uint4* kt = p.k_tree + (size_t)layer * p.tree_layer_stride16;
-    const uint4* vt = p.v_tree + (size_t)layer * p.tree_layer_stride16;
-    uint4* kc = p.k_cache + (size_t)layer * p.cache_layer_stride16;
-    uint4* vc = p.v_cache + (size_t)layer * p.cache_layer_stride16;
-    for (int c = tid; c < 2 * w16; c += blockDim.x) {
-      const bool isv = c >= w16;
-      const int cc = isv ? c - w16 : c;
-      const uint4* src = isv ? vt : kt;
-      uint4* dst = isv ? vc : kc;
-      int k = 0;
-      for (; k + 4 <= rows; k += 4) {
-        uint4 v0 = __ldg(src + (size_t)src_s[k] * w16 + cc);
-        uint4 v1 = __ldg(src + (size_t)src_s[k + 1] * w16 + cc);
-        uint4 v2 = __ldg(src + (size_t)src_s[k + 2] * w16 + cc);
-        uint4 v3 = __ldg(src + (size_t)src_s[k + 3] * w16 + cc);
-        dst[(size_t)dst_s[k] * w16 + cc] = v0;
-        dst[(size_t)dst_s[k + 1] * w16 + cc] = v1;
-        dst[(size_t)dst_s[k + 2] * w16 + cc] = v2;
-        dst[(size_t)dst_s[k + 3] * w16 + cc] = v3;
+  const int w16 = p.row16;                            // 16-byte words per row and tensor
+  const int cw = 2 * w16;                              // words per item (K row, then V row)
+  const int span = min(cw, kCompactThreads);           // threads on one item
+  const int groups = kCompactThreads / span;           // items side by side in the CTA
+  const int g = tid / span;
+  if (g >= groups) return;
+  const int items = rows * (l1 - l0);
+  for (int c = tid - g * span; c < cw; c += span) {
+    const bool isv = c >= w16;
+    const int cc = isv ? c - w16 : c;
+    const uint4* src = (isv ? p.v_tree : p.k_tree) + cc;
+    uint4* dst = (isv ? p.v_cache : p.k_cache) + cc;
+    int layer = l0 + g / rows, k = g % rows;           // item g
+    for (int i = g; i < items; i += groups * kUnroll) {
+      uint4 v[kUnroll];
+      size_t to[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (i + u * groups < items) {
+          v[u] = __ldg(src + (size_t)layer * p.tree_layer_stride16 + (size_t)src_s[k] * w16);
+          to[u] = (size_t)layer * p.cache_layer_stride16 + (size_t)dst_s[k] * w16;
+        }
+        k += groups;                                   // next item of this thread
+        while (k >= rows) {
+          k -= rows;
+          ++layer;
+        }
       }
-      for (; k < rows; ++k) dst[(size_t)dst_s[k] * w16 + cc] = __ldg(src + (size_t)src_s[k] * w16 + cc);
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (i + u * groups < items) dst[to[u]] = v[u];
     }
   }
 }
 
-cudaError_t launch_compact(const CompactParams& p, int sms, cudaStream_t s) {
-  // spread the layers over enough CTAs to give every SM a few, at least one layer per CTA
-  const int want = std::max(1, (4 * sms + p.B - 1) / p.B);
+cudaError_t launch_compact(const CompactParams& p, int ctas, cudaStream_t s) {
+  // about `ctas` CTAs over all requests, at least one layer per CTA
+  const int want = std::max(1, (ctas + p.B - 1) / p.B);
   const int chunks = std::min(p.n_layers, want);
   const int per = (p.n_layers + chunks - 1) / chunks;
   dim3 grid(p.B, (p.n_layers + per - 1) / per);
-  kv_compact_kernel<<<grid, 256, 0, s>>>(p, per);
+  kv_compact_kernel<<<grid, kCompactThreads, 0, s>>>(p, per);
   return cudaGetLastError();
 }
 

@@ -152,6 +152,6 @@ struct CompactParams {
   int max_pages, page_shift;
   int64_t cache_slots;
 };
-cudaError_t launch_compact(const CompactParams& p, int sms, cudaStream_t s);
+cudaError_t launch_compact(const CompactParams& p, int ctas, cudaStream_t s);
 
 }  // namespace etree

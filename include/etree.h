@@ -220,6 +220,7 @@ etree_status etree_lmhead_accept_tree(const etree_batch *batch, const uint16_t *
  * KV compaction.  For each of n_layers layers and each request r with a = accept_len[r]:
  *   cache[slot_base[r] + kv_len[r] + k] <- tree[cu_nodes[r] + path[r][k]],  k = 0 .. a,
  * for K and V, then kv_len_out[r] = kv_len[r] + a + 1 (the bonus token's K/V come next step).
+ * path is the [B][64] array etree_lmhead_accept writes; all 64 entries of a row are read.
  * Rows are [hkv][head_dim] bf16.  Layer l of the tree K/V starts tree_layer_stride ELEMENTS after
  * layer l-1, likewise for the caches.  kv_len_out must not alias batch->kv_len.  A request whose
  * new rows would pass slot_cap[r] is left untouched (kv_len_out = kv_len) with ETREE_ENOSPACE.
