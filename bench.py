@@ -177,8 +177,20 @@ class L2Flush:
 
 
 def time_steps(dev, steps, warmup, flush):
+    """Whole steps timed with events around the step only (the calls run back to back, as a
+    serving loop issues them), then a second pass with events between the three calls for the
+    per-call breakdown."""
     for _ in range(warmup):
         dev.step()
+    torch.cuda.synchronize()
+    whole = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for i in range(steps):
+        flush()
+        whole[i][0].record()
+        dev.attn()
+        dev.lmhead()
+        dev.compact()
+        whole[i][1].record()
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     for i in range(steps):
@@ -195,7 +207,7 @@ def time_steps(dev, steps, warmup, flush):
     attn = [e[0].elapsed_time(e[1]) for e in ev]
     lm = [e[1].elapsed_time(e[2]) for e in ev]
     cp = [e[2].elapsed_time(e[3]) for e in ev]
-    step = [e[0].elapsed_time(e[3]) for e in ev]
+    step = [e[0].elapsed_time(e[1]) for e in whole]
     return dict(attn_ms=attn, lmhead_ms=lm, compact_ms=cp, step_ms=step)
 
 

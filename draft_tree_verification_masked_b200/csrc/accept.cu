@@ -158,6 +158,8 @@ __device__ void answer_malformed(const AcceptParams& p, int r, int lane) {
 __global__ void __launch_bounds__(256) greedy_accept_kernel(AcceptParams p, int32_t* arg_ws,
                                                             int32_t* cnt) {
   __shared__ int am_s[8][64], par_s[8][64], tok_s[8][64], pth_s[8][64];
+  pdl_wait();                                      // the LM-head summaries (launch_pdl)
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int item = blockIdx.x * 8 + warp;
   if (item >= p.n_total + p.B) return;
@@ -655,8 +657,8 @@ __global__ void bonus_kernel(AcceptParams p) {
 
 cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, int32_t* cnt,
                                  cudaStream_t s) {
-  greedy_accept_kernel<<<(p.n_total + p.B + 7) / 8, 256, 0, s>>>(p, arg_ws, cnt);
-  return cudaGetLastError();
+  return launch_pdl(greedy_accept_kernel, dim3((p.n_total + p.B + 7) / 8), dim3(256), 0, s, p,
+                    arg_ws, cnt);
 }
 
 cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStream_t s) {

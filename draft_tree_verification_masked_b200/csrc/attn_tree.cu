@@ -300,6 +300,8 @@ attn_tree_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
 // Merge the split partials of each (node, head) row by log-sum-exp: one warp per row, each lane
 // owning 4 of the 128 output dims.
 __global__ void attn_combine_kernel(AttnParams p, int n_total) {
+  pdl_wait();                                      // the split partials of the attention kernel
+  pdl_trigger();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= n_total * p.hq) return;
@@ -424,8 +426,7 @@ cudaError_t launch_attn_combine(const AttnParams& p, int n_total, cudaStream_t s
   const int rows = n_total * p.hq;
   const int threads = 256;
   const int blocks = (rows * 32 + threads - 1) / threads;
-  attn_combine_kernel<<<blocks, threads, 0, stream>>>(p, n_total);
-  return cudaGetLastError();
+  return launch_pdl(attn_combine_kernel, dim3(blocks), dim3(threads), 0, stream, p, n_total);
 }
 
 }  // namespace etree

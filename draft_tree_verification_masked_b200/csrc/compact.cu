@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(kCompactThreads)
   __shared__ int path_s[ETREE_PATH_STRIDE], src_s[64];
   __shared__ long long dst_s[64], slot0_s;
   __shared__ int rows_s, code_s, detail_s, bad_s, badpage_s, nbase_s, n_s, L_s;
+  pdl_wait();                                      // the accept results (launch_pdl)
+  pdl_trigger();
   const int r = blockIdx.x;
   const int l0 = blockIdx.y * layers_per_cta;
   const int l1 = min(p.n_layers, l0 + layers_per_cta);
@@ -134,8 +136,7 @@ cudaError_t launch_compact(const CompactParams& p, int ctas, cudaStream_t s) {
   const int chunks = std::min(p.n_layers, want);
   const int per = (p.n_layers + chunks - 1) / chunks;
   dim3 grid(p.B, (p.n_layers + per - 1) / per);
-  kv_compact_kernel<<<grid, kCompactThreads, 0, s>>>(p, per);
-  return cudaGetLastError();
+  return launch_pdl(kv_compact_kernel, grid, dim3(kCompactThreads), 0, s, p, per);
 }
 
 }  // namespace etree

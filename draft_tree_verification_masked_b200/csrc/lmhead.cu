@@ -198,8 +198,6 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (p.cnt && blockIdx.x == 0)
-    for (int i = threadIdx.x; i < p.cnt_n; i += blockDim.x) p.cnt[i] = 0;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kGStages; ++i) {
       mbar_init(&full[i], 1);
@@ -220,12 +218,30 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Everything above overlaps the previous kernel of the stream (launch_pdl); the weight tiles
+  // of the first stages are requested before waiting too, since no kernel of the step writes W.
+  if (warp != 0) {
+    pdl_wait();
+    pdl_trigger();
+    if (p.cnt && blockIdx.x == 0)
+      for (int i = threadIdx.x - 32; i < p.cnt_n; i += blockDim.x - 32) p.cnt[i] = 0;
+  }
 
   if (warp == 0) {
     // ----------------------------------------------------------------------- TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_a);
       prefetch_tmap(&tm_b);
+      // W tiles of this CTA's first kGStages k-blocks, each stage armed for its full bytes
+      const int pre = blockIdx.x < p.num_tiles ? min(kGStages, p.k_blocks) : 0;
+      {
+        const int nt0 = blockIdx.x / p.m_tiles;
+        for (int kb = 0; kb < pre; ++kb) {
+          mbar_arrive_expect_tx(&full[kb], kABytes + kBBytes);
+          tma_load_2d(sB + kb * kBBytes, &tm_b, &full[kb], kb * kBK, nt0 * BN);
+        }
+      }
+      pdl_wait();
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
@@ -233,6 +249,10 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int st = it % kGStages;
           const uint32_t ph = (it / kGStages) & 1;
+          if (it < pre) {                             // W already requested, stage armed
+            tma_load_2d(sA + st * kABytes, &tm_a, &full[st], kb * kBK, mt * kBM);
+            continue;
+          }
           if (!mbar_wait(&empty[st], ph ^ 1)) {
             report(p.ws, ETREE_ETIMEOUT, DET_WAIT_GEMM);
             ok = false;
@@ -500,8 +520,7 @@ static cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const
   auto k = lmhead_gemm_kernel<EPI, BN, BM>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<grid, kGemmThreads, smem, stream>>>(ta, tb, p);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(grid), dim3(kGemmThreads), smem, stream, ta, tb, p);
 }
 
 template <int EPI, int BM>
