@@ -212,29 +212,20 @@ def time_steps(dev, steps, warmup, flush):
 
 
 def time_e2e(dev, wl, steps, warmup, flush):
-    """Same step through the C ABI with inputs in pinned host memory: H2D of the step's inputs
-    and D2H of the accept results inside the timed region."""
-    ins = [(dev.cu_nodes, wl.cu_nodes), (dev.parent, wl.parent), (dev.tokens, wl.tokens),
-           (dev.kv_len, wl.kv_len), (dev.slot_base, wl.slot_base), (dev.slot_cap, wl.slot_cap),
-           (dev.q, wl.q), (dev.k_tree, wl.k_tree), (dev.v_tree, wl.v_tree),
-           (dev.hidden, wl.hidden)]
-    if dev.q_draft is not None:
-        ins.append((dev.q_draft, wl.q_draft))
-    host_in = []
-    for d, h in ins:
-        t = torch.as_tensor(h) if not isinstance(h, torch.Tensor) else h
-        host_in.append((d, t.to(d.dtype).contiguous().pin_memory()))
-    outs = [dev.accept_len, dev.path, dev.out_tokens]
-    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
-    d2h = sum(h.numel() * h.element_size() for h in host_out)
+    """Same step through the C ABI with inputs in pinned host memory: the H2D copy of the step's
+    inputs and the D2H copy of the accept results inside the timed region.  The step's inputs
+    (tree, tokens, lengths, Q, tree K/V, hiddens, draft probabilities) sit back to back in one
+    device buffer and the accept results in another, so each direction is one copy."""
+    host_in = torch.empty(dev.inputs.buf.shape, dtype=torch.uint8).pin_memory()
+    host_in.copy_(dev.inputs.buf)
+    host_out = torch.empty(dev.outputs.buf.shape, dtype=torch.uint8).pin_memory()
+    h2d = host_in.numel()
+    d2h = host_out.numel()
 
     def one():
-        for d, h in host_in:
-            d.copy_(h, non_blocking=True)
+        dev.inputs.buf.copy_(host_in, non_blocking=True)
         dev.step()
-        for o, h in zip(outs, host_out):
-            h.copy_(o, non_blocking=True)
+        host_out.copy_(dev.outputs.buf, non_blocking=True)
 
     for _ in range(warmup):
         one()

@@ -25,6 +25,23 @@ def branching_nodes(wl) -> int:
     return int((cnt >= 2).sum())
 
 
+class Packed:
+    """Tensors laid out back to back, each at a 256-byte boundary, in one device byte buffer."""
+
+    def __init__(self, specs, device):
+        self.slots = {}
+        off = 0
+        for name, shape, dtype in specs:
+            nbytes = int(np.prod(shape, dtype=np.int64)) * torch.empty((), dtype=dtype).element_size()
+            self.slots[name] = (off, tuple(shape), dtype, nbytes)
+            off = (off + nbytes + 255) // 256 * 256
+        self.buf = torch.zeros(max(off, 256), dtype=torch.uint8, device=device)
+
+    def view(self, name):
+        off, shape, dtype, nbytes = self.slots[name]
+        return self.buf[off:off + nbytes].view(dtype).view(shape)
+
+
 class DeviceStep:
     """tree: None picks the branching-tree sampler (etree_lmhead_accept_tree) when T > 0 and a
     node has two or more children; zbuf_rows overrides the size of its logit buffer.
@@ -44,33 +61,46 @@ class DeviceStep:
                 t = t.to(dtype)
             return t.contiguous().to(dev)
 
-        self.cu_nodes = up(wl.cu_nodes, i32)
-        self.parent = up(wl.parent, i32)
-        self.tokens = up(wl.tokens, i32)
-        self.kv_len = up(wl.kv_len, i32)
-        self.slot_base = up(wl.slot_base, torch.int64)
         self.paged = None
         if page_size:
             from .workload import paged
             self.paged = paged(wl, int(page_size))
-            self.block_table = up(self.paged.block_table, i32)
-        self.slot_cap = up(self.paged.slot_cap if self.paged else wl.slot_cap, i32)
+        # The per-step inputs live back to back in one device buffer (`inputs.buf`), and the
+        # accept results in another (`outputs.buf`), so that a serving loop moves each direction
+        # in a single copy.  The caches and the LM-head weight stay resident on their own.
+        srcs = [("cu_nodes", wl.cu_nodes, i32), ("parent", wl.parent, i32),
+                ("tokens", wl.tokens, i32), ("kv_len", wl.kv_len, i32),
+                ("slot_base", wl.slot_base, torch.int64),
+                ("slot_cap", self.paged.slot_cap if self.paged else wl.slot_cap, i32)]
+        if self.paged:
+            srcs.append(("block_table", self.paged.block_table, i32))
+        srcs += [("q", wl.q, None), ("k_tree", wl.k_tree, None), ("v_tree", wl.v_tree, None),
+                 ("hidden", wl.hidden, None)]
+        if wl.q_draft is not None:
+            srcs.append(("q_draft", wl.q_draft, None))
+        host = {}
+        for name, x, dtype in srcs:
+            t = torch.as_tensor(x) if not isinstance(x, torch.Tensor) else x
+            host[name] = (t.to(dtype) if dtype is not None else t).contiguous()
+        self.inputs = Packed([(k, tuple(t.shape), t.dtype) for k, t in host.items()], dev)
+        for name, t in host.items():
+            v = self.inputs.view(name)
+            v.copy_(t)
+            setattr(self, name, v)
         self.batch = make_batch(self.cu_nodes, self.parent, self.tokens, self.kv_len,
                                 self.slot_base, self.slot_cap, wl.n_max, wl.kv_len_max)
-        self.q = up(wl.q)
-        self.k_tree = up(wl.k_tree)
-        self.v_tree = up(wl.v_tree)
         self.k_cache = up(self.paged.k_pool if self.paged else wl.k_cache)
         self.v_cache = up(self.paged.v_pool if self.paged else wl.v_cache)
-        self.hidden = up(wl.hidden)
         self.w_lm = up(wl.w_lm)
         self.q_draft = up(wl.q_draft) if wl.q_draft is not None else None
         ntot, B = wl.n_total, wl.B
         self.out = torch.empty(ntot, wl.hq, wl.head_dim, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(ntot, wl.hq, dtype=torch.float32, device=dev)
-        self.accept_len = torch.empty(B, dtype=i32, device=dev)
-        self.path = torch.empty(B, 64, dtype=i32, device=dev)
-        self.out_tokens = torch.empty(B, 65, dtype=i32, device=dev)
+        self.outputs = Packed([("accept_len", (B,), i32), ("path", (B, 64), i32),
+                               ("out_tokens", (B, 65), i32)], dev)
+        self.accept_len = self.outputs.view("accept_len")
+        self.path = self.outputs.view("path")
+        self.out_tokens = self.outputs.view("out_tokens")
         self.node_argmax = torch.empty(ntot, dtype=i32, device=dev)
         self.node_gap = torch.empty(ntot, dtype=torch.float32, device=dev)
         self.kv_len_out = torch.empty(B, dtype=i32, device=dev)
