@@ -159,7 +159,6 @@ __global__ void __launch_bounds__(256) greedy_accept_kernel(AcceptParams p, int3
                                                             int32_t* cnt) {
   __shared__ int am_s[8][64], par_s[8][64], tok_s[8][64], pth_s[8][64];
   pdl_wait();                                      // the LM-head summaries (launch_pdl)
-  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int item = blockIdx.x * 8 + warp;
   if (item >= p.n_total + p.B) return;

@@ -349,7 +349,7 @@ etree_status etree_workspace_init(void* workspace, size_t workspace_bytes, void*
 
 // ------------------------------------------------------------------ low-rank candidate head
 struct LowrankLayout {
-  size_t part, g, lists, cand, tkth, total;
+  size_t part, g, lists, cand, tkth, fmax, fcnt, total;
   int nk, nlists;
 };
 
@@ -363,13 +363,15 @@ static LowrankLayout lowrank_layout(int M, int H, int r, int V) {
   };
   w.nk = lowrank_down_chunks(H);
   w.nlists = 2 * ((V + 127) / 128);                 // per vocab tile at the narrowest width
-  // the sample's chunk partials, then its summed logits
-  const size_t sample = (size_t)((r + 127) / 128 + 1) * M * lowrank_sample_cols(V);
+  // the down projection's chunk partials, or the sample's
+  const size_t sample = (size_t)((r + 127) / 128) * M * lowrank_sample_cols(V);
   w.part = take(std::max((size_t)w.nk * M * r, sample) * sizeof(float));
   w.g = take((size_t)M * r * 2);
   w.lists = take((size_t)M * w.nlists * 16 * sizeof(float2));
   w.cand = take((size_t)M * 16 * sizeof(int32_t));
   w.tkth = take((size_t)M * sizeof(uint32_t));
+  w.fmax = take((size_t)lowrank_floor_maxima(M) * sizeof(float));
+  w.fcnt = take((size_t)M * sizeof(int32_t));
   w.total = off;
   return w;
 }
@@ -402,11 +404,14 @@ etree_status etree_lowrank_candidates(const uint16_t* hidden, int M, int hidden_
   const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(hidden);
   __nv_bfloat16* g = at<__nv_bfloat16>(workspace, w.g);
   uint32_t* tkth = at<uint32_t>(workspace, w.tkth);
+  int32_t* fcnt = at<int32_t>(workspace, w.fcnt);
   cudaError_t e = launch_lowrank_down(hb, reinterpret_cast<const __nv_bfloat16*>(D), M,
-                                      hidden_dim, rank, at<float>(workspace, w.part), g, tkth, s);
+                                      hidden_dim, rank, at<float>(workspace, w.part), g, tkth,
+                                      fcnt, s);
   if (e == cudaSuccess)
     e = launch_lowrank_sample(g, reinterpret_cast<const __nv_bfloat16*>(U), M, rank, vocab,
-                              at<float>(workspace, w.part), tkth, s);
+                              at<float>(workspace, w.part), at<float>(workspace, w.fmax), fcnt,
+                              tkth, s);
   if (e != cudaSuccess) return cuda_fail(e, "etree_lowrank_candidates (down, sample)");
 
   const int sms = sm_count();

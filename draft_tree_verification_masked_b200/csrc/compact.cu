@@ -30,7 +30,6 @@ __global__ void __launch_bounds__(kCompactThreads)
   __shared__ long long dst_s[64], slot0_s;
   __shared__ int rows_s, code_s, detail_s, bad_s, badpage_s, nbase_s, n_s, L_s;
   pdl_wait();                                      // the accept results (launch_pdl)
-  pdl_trigger();
   const int r = blockIdx.x;
   const int l0 = blockIdx.y * layers_per_cta;
   const int l1 = min(p.n_layers, l0 + layers_per_cta);

@@ -119,10 +119,12 @@ cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32
 int lowrank_down_chunks(int H);
 cudaError_t launch_lowrank_down(const __nv_bfloat16* hid, const __nv_bfloat16* D, int M, int H,
                                 int r, float* part, __nv_bfloat16* g, uint32_t* tkth,
-                                cudaStream_t s);
+                                int32_t* fcnt, cudaStream_t s);
 int lowrank_sample_cols(int V);
+int lowrank_floor_maxima(int M);
 cudaError_t launch_lowrank_sample(const __nv_bfloat16* g, const __nv_bfloat16* U, int M, int r,
-                                  int V, float* part, uint32_t* tkth, cudaStream_t s);
+                                  int V, float* part, float* fmax, int32_t* fcnt, uint32_t* tkth,
+                                  cudaStream_t s);
 cudaError_t launch_lowrank_finish(const float2* lists, int nlists, const uint32_t* tkth, int M,
                                   int k,
                                   int32_t* cand, const __nv_bfloat16* hid,

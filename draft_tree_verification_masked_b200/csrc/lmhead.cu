@@ -220,9 +220,10 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   const uint32_t tmem = *tmem_slot;
   // Everything above overlaps the previous kernel of the stream (launch_pdl); the weight tiles
   // of the first stages are requested before waiting too, since no kernel of the step writes W.
+  // No early signal to dependents: the kernels after the GEMM have no set-up to overlap, and an
+  // early signal measured slower.
   if (warp != 0) {
     pdl_wait();
-    pdl_trigger();
     if (p.cnt && blockIdx.x == 0)
       for (int i = threadIdx.x - 32; i < p.cnt_n; i += blockDim.x - 32) p.cnt[i] = 0;
   }

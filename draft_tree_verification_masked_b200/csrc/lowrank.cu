@@ -38,6 +38,10 @@ __global__ void __launch_bounds__(256) lr_down_kernel(const __nv_bfloat16* __res
   const int j0 = blockIdx.x * kDT, kc = blockIdx.y, m0 = blockIdx.z * kDT;
   const int h0 = kc * kDK;
   const int tid = threadIdx.x;
+  // Every kernel here is launched with launch_pdl.  Only the floor kernel signals its dependent
+  // early: the screen GEMM after it has set-up and U tiles to load before it waits.  An early
+  // signal to a dependent with nothing to overlap measured slower than none.
+  pdl_wait();
   // stage the two tiles, 16 bytes per thread per step (zeros past M, r or H)
   for (int e = tid; e < kDT * (kDK / 8); e += 256) {
     const int row = e / (kDK / 8), c8 = (e % (kDK / 8)) * 8;
@@ -84,25 +88,21 @@ __global__ void __launch_bounds__(256) lr_down_kernel(const __nv_bfloat16* __res
   }
 }
 
-// g[m][j] = bf16(sum over chunks, in chunk order); also resets the screen's per-row bounds.
+// g[m][j] = bf16(sum over chunks, in chunk order); also resets the screen's per-row bounds and
+// the floor kernel's per-row counters.
 __global__ void lr_reduce_kernel(const float* __restrict__ part, int nk, int M, int r,
-                                 __nv_bfloat16* __restrict__ g, uint32_t* __restrict__ tkth) {
+                                 __nv_bfloat16* __restrict__ g, uint32_t* __restrict__ tkth,
+                                 int32_t* __restrict__ fcnt) {
+  pdl_wait();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t < M) tkth[t] = enc_order(-INFINITY);
+  if (t < M) {
+    tkth[t] = enc_order(-INFINITY);
+    fcnt[t] = 0;
+  }
   if (t >= M * r) return;
   float s = 0.f;
   for (int k = 0; k < nk; ++k) s += part[(size_t)k * M * r + t];
   g[t] = __float2bfloat16_rn(s);
-}
-
-// zs[m][j] = sum over the chunk partials (in chunk order) of the sampled approximate logits.
-__global__ void sample_sum_kernel(const float* __restrict__ part, int nk, int MS,
-                                  float* __restrict__ zs) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= MS) return;
-  float x = 0.f;
-  for (int k = 0; k < nk; ++k) x += part[(size_t)k * MS + t];
-  zs[t] = x;
 }
 
 // (va, ia) ranks before (vb, ib): larger value first, then the lower id; empty entries (id < 0)
@@ -111,24 +111,54 @@ __device__ __forceinline__ bool before(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia >= 0 && (ib < 0 || ia < ib));
 }
 
-// One CTA per row: a floor for the screen.  Each thread takes the maximum of its sampled
-// approximate logits; the 16th largest of these 256 maxima is a value that 16 distinct logits
-// reach (each maximum is one), so no logit below it can be among the k <= 16 selected.  For a
-// sample of 8192 it sits near the row's 99.8th percentile.  It is lowered by a rounding margin
-// that covers the sample's fp32 sums differing from the tensor-core sums of the same values.
-__global__ void __launch_bounds__(256) sample_floor_kernel(const float* __restrict__ zs, int S,
+// A floor for the screen, kFloorParts CTAs per row.  Each sampled approximate logit is the sum
+// of the split-K partials part[kc][m][j] in chunk order.  Thread t of every CTA of a row covers
+// a fixed set of sampled columns; the maximum over its columns in all parts is one logit of the
+// row, so the 16th largest of the 256 thread maxima is a value that 16 distinct logits reach, and
+// no logit below it can be among the k <= 16 selected.  For a sample of 8192 it sits near the
+// row's 99.8th percentile.  The CTA that completes a row (per-row counter, fence, atomic, fence)
+// ranks the maxima.  The floor is lowered by a rounding margin that covers the sample's fp32 sums
+// differing from the tensor-core sums of the same values.
+constexpr int kFloorParts = 8;
+
+__global__ void __launch_bounds__(256) sample_floor_kernel(const float* __restrict__ part,
+                                                           int nk, int M, int S,
+                                                           float* __restrict__ fmax,
+                                                           int32_t* __restrict__ fcnt,
                                                            uint32_t* __restrict__ tkth) {
   __shared__ float mx[256];
-  const int m = blockIdx.x, tid = threadIdx.x;
-  const float* row = zs + (size_t)m * S;
+  __shared__ int last_s;
+  pdl_wait();
+  pdl_trigger();
+  const int m = blockIdx.x / kFloorParts, q = blockIdx.x % kFloorParts, tid = threadIdx.x;
+  const int span = (S + kFloorParts - 1) / kFloorParts;
+  const int c0 = q * span, c1 = min(S, c0 + span);
+  const size_t cs = (size_t)M * S;                    // stride between chunk partials
+  const float* row = part + (size_t)m * S;
   float best = -INFINITY;
-  for (int j0 = tid; j0 < S; j0 += 256 * 8) {
-    float x[8];
+  for (int j0 = c0 + tid; j0 < c1; j0 += 256 * 4) {
+    float x[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = j0 + u * 256 < S ? row[j0 + u * 256] : -INFINITY;
+    for (int u = 0; u < 4; ++u) x[u] = 0.f;
+    for (int kc = 0; kc < nk; ++kc) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) best = fmaxf(best, x[u]);
+      for (int u = 0; u < 4; ++u)
+        if (j0 + u * 256 < c1) x[u] += row[kc * cs + j0 + u * 256];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (j0 + u * 256 < c1) best = fmaxf(best, x[u]);
   }
+  fmax[((size_t)m * kFloorParts + q) * 256 + tid] = best;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last_s = atomicAdd(fcnt + m, 1) == kFloorParts - 1;
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+  best = -INFINITY;
+  for (int q2 = 0; q2 < kFloorParts; ++q2)
+    best = fmaxf(best, __ldcg(fmax + ((size_t)m * kFloorParts + q2) * 256 + tid));
   mx[tid] = best;
   __syncthreads();
   int rank = 0;                                       // maxima ranked before this thread's
@@ -141,34 +171,46 @@ __global__ void __launch_bounds__(256) sample_floor_kernel(const float* __restri
 
 // One CTA per row.  The screen published a lower bound T of the row's 16th largest value, so
 // only list entries >= T can be selected: each thread scans its share of the 16 x nlists
-// entries (8 loads in flight) and appends the survivors (usually a few hundred) to shared
-// memory, where a bitonic sort orders them and the first k go to cand[m][0..k).  More than
-// kGather survivors (not seen in practice) fall back to ranking them in passes over the lists.
+// entries (8 loads in flight) and each warp appends its survivors (150-500 per row measured on
+// the rank-128 and rank-512 workloads) to shared memory together.  A bitonic sort orders them
+// and the first k go to cand[m][0..k).  (Counting each survivor's rank against the others was
+// measured 27 us slower.)  More than kGather survivors fall back to ranking them in passes over
+// the lists.
 constexpr int kGather = 2048;
+constexpr int kMergeThreads = 1024;
 
-__global__ void __launch_bounds__(256) topk_merge_kernel(const float2* __restrict__ lists,
-                                                         int nlists, const uint32_t* tkth, int k,
-                                                         int32_t* __restrict__ cand) {
+__global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(const float2* __restrict__ lists,
+                                                                   int nlists, const uint32_t* tkth,
+                                                                   int k,
+                                                                   int32_t* __restrict__ cand) {
   __shared__ float gv[kGather];
   __shared__ int gi[kGather];
   __shared__ int gn;
-  const int m = blockIdx.x, tid = threadIdx.x;
+  pdl_wait();
+  const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
   const float T = dec_order(tkth[m]);
   const float2* rowl = lists + (size_t)m * nlists * 16;
   const int total = nlists * 16;
   if (tid == 0) gn = 0;
   __syncthreads();
-  for (int e0 = tid; e0 < total; e0 += 256 * 8) {
+  // every lane of a warp runs the same iterations, so survivors are appended a warp at a time
+  for (int eb = tid - lane; eb < total; eb += kMergeThreads * 8) {
     float2 x[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      x[u] = e0 + u * 256 < total ? rowl[e0 + u * 256] : make_float2(-INFINITY, __int_as_float(-1));
+    for (int u = 0; u < 8; ++u) {
+      const int e = eb + lane + u * kMergeThreads;
+      x[u] = e < total ? rowl[e] : make_float2(-INFINITY, __int_as_float(-1));
+    }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int xi = __float_as_int(x[u].y);
-      if (xi >= 0 && x[u].x >= T) {
-        const int at = atomicAdd(&gn, 1);
-        if (at < kGather) {
+      const bool sv = xi >= 0 && x[u].x >= T;
+      const unsigned b = __ballot_sync(0xffffffffu, sv);
+      if (b) {
+        int at = 0;
+        if (lane == 0) at = atomicAdd(&gn, __popc(b));
+        at = __shfl_sync(0xffffffffu, at, 0) + __popc(b & ((1u << lane) - 1u));
+        if (sv && at < kGather) {
           gv[at] = x[u].x;
           gi[at] = xi;
         }
@@ -178,17 +220,16 @@ __global__ void __launch_bounds__(256) topk_merge_kernel(const float2* __restric
   __syncthreads();
   const int n = gn;
   if (n <= kGather) {
-    // bitonic sort of the survivors (padded with empty entries to a power of two), best first
     int P = 16;
     while (P < n) P <<= 1;
-    for (int e = n + tid; e < P; e += 256) {
+    for (int e = n + tid; e < P; e += kMergeThreads) {
       gv[e] = -INFINITY;
       gi[e] = -1;
     }
     __syncthreads();
     for (int size = 2; size <= P; size <<= 1) {
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < P / 2; i += 256) {
+        for (int i = tid; i < P / 2; i += kMergeThreads) {
           const int lo = 2 * stride * (i / stride) + (i % stride), hi = lo + stride;
           const bool best_first = (lo & size) == 0;
           const bool swap = best_first ? before(gv[hi], gi[hi], gv[lo], gi[lo])
@@ -209,7 +250,7 @@ __global__ void __launch_bounds__(256) topk_merge_kernel(const float2* __restric
     return;
   }
   // fallback: every entry >= T is ranked against every other by a pass over the lists
-  for (int e = tid; e < total; e += 256) {
+  for (int e = tid; e < total; e += kMergeThreads) {
     const float2 x = rowl[e];
     const int xi = __float_as_int(x.y);
     if (xi < 0 || x.x < T) continue;
@@ -222,8 +263,10 @@ __global__ void __launch_bounds__(256) topk_merge_kernel(const float2* __restric
   }
 }
 
+constexpr int kRescoreLoads = 20;        // 16-byte words of W per lane requested up front
+
 // One CTA per row, one warp per candidate: z_c = h . W_c in fp32 (the row staged in shared
-// memory, ten W loads in flight per lane); then the k candidates are ordered by z_c descending
+// memory, the lane's W words requested first); then the k candidates are ordered by z_c descending
 // (lower id first on equal values).
 __global__ void __launch_bounds__(512) lr_rescore_kernel(const __nv_bfloat16* __restrict__ hid,
                                                          const __nv_bfloat16* __restrict__ W,
@@ -234,17 +277,43 @@ __global__ void __launch_bounds__(512) lr_rescore_kernel(const __nv_bfloat16* __
   __shared__ uint4 hsm[1024];                     // H <= 8192
   __shared__ float zs[16];
   __shared__ int cs[16];
+  pdl_wait();
   const int m = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint4* hrow = reinterpret_cast<const uint4*>(hid + (size_t)m * H);
+  // this lane's first kRescoreLoads words of the candidate's W row (all of it at H <= 5120) are
+  // requested before the hidden row is staged, so both loads are in flight together
+  const int c = warp < k ? cand[(size_t)m * 16 + warp] : -1;
+  const bool live = warp < k && c >= 0 && c < V;
+  uint4 wv[kRescoreLoads];
+  {
+    const uint4* w = reinterpret_cast<const uint4*>(W + (size_t)(live ? c : 0) * H);
+#pragma unroll
+    for (int u = 0; u < kRescoreLoads; ++u) {
+      const int i = lane + 32 * u;
+      wv[u] = (live && i < H / 8) ? __ldg(w + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
   for (int i = threadIdx.x; i < H / 8; i += blockDim.x) hsm[i] = hrow[i];
   __syncthreads();
   if (warp < k) {
-    const int c = cand[(size_t)m * 16 + warp];
     float acc = 0.f;
-    if (c >= 0 && c < V) {
+    if (live) {
+#pragma unroll
+      for (int u = 0; u < kRescoreLoads; ++u) {
+        const int i = lane + 32 * u;
+        if (i >= H / 8) break;
+        const uint4 a = hsm[i], b = wv[u];
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 fa = __bfloat1622float2(a2[q]), fb = __bfloat1622float2(b2[q]);
+          acc = fmaf(fa.x, fb.x, acc);
+          acc = fmaf(fa.y, fb.y, acc);
+        }
+      }
       const uint4* w = reinterpret_cast<const uint4*>(W + (size_t)c * H);
-#pragma unroll 10
-      for (int i = lane; i < H / 8; i += 32) {
+      for (int i = lane + 32 * kRescoreLoads; i < H / 8; i += 32) {   // H > 5120
         const uint4 a = hsm[i], b = __ldg(w + i);
         const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
@@ -290,35 +359,40 @@ int lowrank_down_chunks(int H) { return (H + kDK - 1) / kDK; }
 
 cudaError_t launch_lowrank_down(const __nv_bfloat16* hid, const __nv_bfloat16* D, int M, int H,
                                 int r, float* part, __nv_bfloat16* g, uint32_t* tkth,
-                                cudaStream_t s) {
+                                int32_t* fcnt, cudaStream_t s) {
   const int nk = lowrank_down_chunks(H);
   dim3 grid((r + kDT - 1) / kDT, nk, (M + kDT - 1) / kDT);
-  lr_down_kernel<<<grid, 256, 0, s>>>(hid, D, M, H, r, 1, part);
-  lr_reduce_kernel<<<(M * r + 255) / 256, 256, 0, s>>>(part, nk, M, r, g, tkth);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(lr_down_kernel, grid, dim3(256), 0, s, hid, D, M, H, r, 1, part);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(lr_reduce_kernel, dim3((M * r + 255) / 256), dim3(256), 0, s, part, nk, M, r,
+                    g, tkth, fcnt);
 }
 
 int lowrank_sample_cols(int V) { return V < 8192 ? V : 8192; }
 
+int lowrank_floor_maxima(int M) { return M * kFloorParts * 256; }
+
 cudaError_t launch_lowrank_sample(const __nv_bfloat16* g, const __nv_bfloat16* U, int M, int r,
-                                  int V, float* part, uint32_t* tkth, cudaStream_t s) {
+                                  int V, float* part, float* fmax, int32_t* fcnt, uint32_t* tkth,
+                                  cudaStream_t s) {
   const int S = lowrank_sample_cols(V), stride = V / S;
   const int nk = (r + kDK - 1) / kDK;
   dim3 grid((S + kDT - 1) / kDT, nk, (M + kDT - 1) / kDT);
-  lr_down_kernel<<<grid, 256, 0, s>>>(g, U, M, r, S, stride, part);
-  float* zs = part + (size_t)nk * M * S;
-  sample_sum_kernel<<<(M * S + 255) / 256, 256, 0, s>>>(part, nk, M * S, zs);
-  sample_floor_kernel<<<M, 256, 0, s>>>(zs, S, tkth);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(lr_down_kernel, grid, dim3(256), 0, s, g, U, M, r, S, stride, part);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(sample_floor_kernel, dim3(M * kFloorParts), dim3(256), 0, s, part, nk, M, S,
+                    fmax, fcnt, tkth);
 }
 
 cudaError_t launch_lowrank_finish(const float2* lists, int nlists, const uint32_t* tkth, int M,
                                   int k, int32_t* cand, const __nv_bfloat16* hid,
                                   const __nv_bfloat16* W, int H, int V, int32_t* out_ids,
                                   float* out_logit, cudaStream_t s) {
-  topk_merge_kernel<<<M, 256, 0, s>>>(lists, nlists, tkth, k, cand);
-  lr_rescore_kernel<<<M, 32 * k, 0, s>>>(hid, W, H, V, k, cand, out_ids, out_logit);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(topk_merge_kernel, dim3(M), dim3(kMergeThreads), 0, s, lists,
+                             nlists, tkth, k, cand);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(lr_rescore_kernel, dim3(M), dim3(32 * k), 0, s, hid, W, H, V, k, cand,
+                    out_ids, out_logit);
 }
 
 }  // namespace etree
