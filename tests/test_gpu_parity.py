@@ -349,3 +349,31 @@ def test_lowrank_candidates_full_size(name):
     ids, lg = _lowrank_run(lw)
     differ = P.lowrank_compare(lw, ids, lg)
     assert differ <= max(1, lw.M // 10), differ
+
+
+def test_inputs_written_by_the_kernel_before_each_call():
+    """Every input a call reads is produced by the kernel launched just before it on the same
+    stream (device-to-device copies from a scrambled start), as a model's layers would produce
+    them.  The calls start their set-up early (programmatic dependent launch) and must still see
+    the finished inputs: the results match the oracle."""
+    wl = W.generate("tiny")
+    dev = DeviceStep(wl)
+    good = dev.inputs.buf.clone()
+    hid, q = dev.hidden.clone(), dev.q.clone()
+    for _ in range(3):
+        dev.inputs.buf.copy_(good)
+        dev.q.zero_()
+        dev.hidden.zero_()
+        torch.cuda.synchronize()
+        dev.q.copy_(q)                                   # written right before the attention
+        dev.attn()
+        dev.hidden.copy_(hid)                            # written right before the LM head
+        dev.lmhead()
+        dev.compact()
+        st, det = dev.status()
+        assert st == 0, (st, det)
+    res = dev.results()
+    P.attn_compare(wl, dev)
+    excused, near, ores = P.greedy_compare(wl, res, list(range(wl.B)))
+    P.compact_compare(wl, dev, ores, list(range(wl.B)), excused)
+    assert near <= 1, near
