@@ -172,12 +172,19 @@ __global__ void __launch_bounds__(256) sample_floor_kernel(const float* __restri
 // One CTA per row.  The screen published a lower bound T of the row's 16th largest value, so
 // only list entries >= T can be selected: each thread scans its share of the 16 x nlists
 // entries (8 loads in flight) and each warp appends its survivors (150-500 per row measured on
-// the rank-128 and rank-512 workloads) to shared memory together.  A bitonic sort orders them
-// and the first k go to cand[m][0..k).  (Counting each survivor's rank against the others was
-// measured 27 us slower.)  More than kGather survivors fall back to ranking them in passes over
-// the lists.
+// the rank-128 and rank-512 workloads) to shared memory together.  A bitonic sort on the first
+// 256 threads orders them and the first k go to cand[m][0..k).  (Counting ranks, a bisection for
+// the k-th key over the CTA or one warp, and a register tournament in one warp all measured
+// within -1 .. +5 us of it.)  More than kGather survivors fall back to ranking them in passes
+// over the lists.
 constexpr int kGather = 2048;
 constexpr int kMergeThreads = 1024;
+constexpr int kSortThreads = 256;
+
+// Barrier 1 among the first kSortThreads threads of the CTA (barrier 0 is __syncthreads).
+__device__ __forceinline__ void sort_barrier() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kSortThreads) : "memory");
+}
 
 __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(const float2* __restrict__ lists,
                                                                    int nlists, const uint32_t* tkth,
@@ -220,17 +227,21 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(const float2*
   __syncthreads();
   const int n = gn;
   if (n <= kGather) {
+    // The sort runs on the first kSortThreads threads only, synchronised by a named barrier of
+    // that many threads (the rest of the CTA leaves); strides are powers of two, so the pair
+    // indices are bit operations.
+    if (tid >= kSortThreads) return;
     int P = 16;
     while (P < n) P <<= 1;
-    for (int e = n + tid; e < P; e += kMergeThreads) {
+    for (int e = n + tid; e < P; e += kSortThreads) {
       gv[e] = -INFINITY;
       gi[e] = -1;
     }
-    __syncthreads();
+    sort_barrier();
     for (int size = 2; size <= P; size <<= 1) {
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < P / 2; i += kMergeThreads) {
-          const int lo = 2 * stride * (i / stride) + (i % stride), hi = lo + stride;
+        for (int i = tid; i < P / 2; i += kSortThreads) {
+          const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1)), hi = lo + stride;
           const bool best_first = (lo & size) == 0;
           const bool swap = best_first ? before(gv[hi], gi[hi], gv[lo], gi[lo])
                                        : before(gv[lo], gi[lo], gv[hi], gi[hi]);
@@ -243,7 +254,7 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(const float2*
             gi[hi] = ti;
           }
         }
-        __syncthreads();
+        sort_barrier();
       }
     }
     if (tid < k) cand[(size_t)m * 16 + tid] = gi[tid];
