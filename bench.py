@@ -127,11 +127,36 @@ def compact_work(wl, accept_len, n_layers=1):
     return 2 * 2 * int((accept_len + 1).sum()) * wl.hkv * wl.head_dim * 2 * n_layers
 
 
+def strip_comments(src: str) -> str:
+    """C++ source without comments and with runs of whitespace collapsed (string and character
+    literals kept), so that a comment edit does not count as a change of the kernel."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":                                  # literal: copy through its closing quote
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_hash(*names):
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "draft_tree_verification_masked_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "draft_tree_verification_masked_b200", "csrc", n)) as f:
+            h.update(strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

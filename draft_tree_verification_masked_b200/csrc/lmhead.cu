@@ -10,11 +10,12 @@
 // in the epilogue, straight out of tensor memory, to a few numbers per row.
 //
 // Kernel shape.  Persistent: one CTA per SM walks the (row tile, vocab tile) list, vocab-major
-// so that concurrently running CTAs share W tiles through L2.  Warp 0 streams 128x64 hidden
-// tiles and 256x64 W tiles with TMA (128-byte swizzle) into a 4-deep shared-memory ring; warp 1
-// issues tcgen05.mma (M=128, N=256, K=16, bf16 in, fp32 out) into one of two 256-column TMEM
-// accumulators; warps 2-5 drain the other accumulator with tcgen05.ld, one TMEM lane (= one
-// output row) per thread, and apply the epilogue:
+// so that concurrently running CTAs share W tiles through L2.  Warp 0 streams BMx64 hidden tiles
+// (BM = 128, or 64 when all rows fit) and BNx64 W tiles with TMA (128-byte swizzle) into a
+// shared-memory ring of as many stages as fit (4 at 128x256, 6 at 64x208); warp 1 issues
+// tcgen05.mma (M=BM, N=BN, K=16, bf16 in, fp32 out) into one of two BN-column TMEM accumulators;
+// eight epilogue warps drain the other accumulator with tcgen05.ld, one TMEM lane (= one output
+// row) per thread, two warps per lane quarter, and apply the epilogue:
 //   EPI_ARGMAX  per row and tile: top-1 value, its vocab id (lowest on ties) and top-2 value;
 //   EPI_LSE     per row and tile: m = max z*log2(e)/T and sum 2^(z*log2(e)/T - m), plus the
 //               logit of the row's child token when it falls in the tile; rows of branching tree

@@ -48,8 +48,8 @@ class DeviceStep:
     page_size: lay the caches out in pages of that many tokens at shuffled pool pages and use
     the paged attention and compaction calls (the pools replace k_cache / v_cache)."""
 
-    def __init__(self, wl, device: str = "cuda", n_layers: int = 1, pin: bool = False,
-                 tree=None, zbuf_rows=None, page_size=None):
+    def __init__(self, wl, device: str = "cuda", n_layers: int = 1, tree=None, zbuf_rows=None,
+                 page_size=None):
         self.wl = wl
         self.device = device
         dev = torch.device(device)
