@@ -41,6 +41,10 @@ class Packed:
         off, shape, dtype, nbytes = self.slots[name]
         return self.buf[off:off + nbytes].view(dtype).view(shape)
 
+    def offset(self, name) -> int:
+        """Byte offset of a tensor in the buffer (tensors after it follow contiguously)."""
+        return self.slots[name][0]
+
 
 class DeviceStep:
     """tree: None picks the branching-tree sampler (etree_lmhead_accept_tree) when T > 0 and a
@@ -67,7 +71,10 @@ class DeviceStep:
             self.paged = paged(wl, int(page_size))
         # The per-step inputs live back to back in one device buffer (`inputs.buf`), and the
         # accept results in another (`outputs.buf`), so that a serving loop moves each direction
-        # in a single copy.  The caches and the LM-head weight stay resident on their own.
+        # in a single copy.  The attention's inputs come first and the LM head's (hidden states,
+        # draft probabilities) last, from byte `inputs.offset("hidden")` on, so the second part
+        # can be copied while the attention runs.  The caches and the LM-head weight stay
+        # resident on their own.
         srcs = [("cu_nodes", wl.cu_nodes, i32), ("parent", wl.parent, i32),
                 ("tokens", wl.tokens, i32), ("kv_len", wl.kv_len, i32),
                 ("slot_base", wl.slot_base, torch.int64),
