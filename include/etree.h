@@ -27,6 +27,12 @@
  *  - Pointers are DEVICE pointers unless stated; the caller owns all memory.  bf16 tensors are
  *    passed as uint16_t bit patterns.  `stream` is a cudaStream_t (NULL = legacy default stream).
  *  - Calls are asynchronous: they validate host-visible arguments, enqueue kernels and return.
+ *    Stream order holds as usual: every input a call reads may be produced by the work enqueued
+ *    just before it on the same stream.  Some kernels are launched with programmatic dependent
+ *    launch and start their set-up (barriers, tensor memory, descriptor and weight prefetch)
+ *    while the previous kernel finishes, but read their inputs and write their outputs only
+ *    after it has completed.  W (and U, D for the low-rank head) must not be written by work
+ *    still running on the stream when a call that reads them is enqueued.
  *  - Problems visible on the host return at once (ETREE_EINVAL / ETREE_EUNSUPPORTED) and enqueue
  *    nothing.  Problems visible only on the device (a malformed parent array, a KV length past
  *    its bound, a full cache) are recorded in the workspace status word; the affected request is
