@@ -31,8 +31,10 @@
  *    just before it on the same stream.  Some kernels are launched with programmatic dependent
  *    launch and start their set-up (barriers, tensor memory, descriptor and weight prefetch)
  *    while the previous kernel finishes, but read their inputs and write their outputs only
- *    after it has completed.  W (and U, D for the low-rank head) must not be written by work
- *    still running on the stream when a call that reads them is enqueued.
+ *    after it has completed.  The LM-head GEMM requests its first weight tiles (W, or U for the
+ *    low-rank screen) before that wait, so the one case to avoid is a kernel that signals its
+ *    dependents early (griddepcontrol.launch_dependents) and writes those weights, enqueued right
+ *    before the call; no kernel of this library writes them.
  *  - Problems visible on the host return at once (ETREE_EINVAL / ETREE_EUNSUPPORTED) and enqueue
  *    nothing.  Problems visible only on the device (a malformed parent array, a KV length past
  *    its bound, a full cache) are recorded in the workspace status word; the affected request is
