@@ -499,10 +499,13 @@ __device__ double residual_mass(const AcceptParams& p, const float* zr, const fl
 // evaluates N(c) when a rejected child has a younger sibling still to test.  Writes accept_len,
 // path, the accepted tokens, the stop row / node, the draw offset cval (negative: fall back to
 // argmax p) and the stop row's hidden state for the draw pass.
-__global__ void __launch_bounds__(512) tree_walk_kernel(AcceptParams p, const float* zc,
-                                                        const int32_t* zrow, const float* zbuf) {
+constexpr int kWalkThreads = 1024;
+
+__global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p, const float* zc,
+                                                                 const int32_t* zrow,
+                                                                 const float* zbuf) {
   __shared__ int par_s[64], tok_s[64];
-  __shared__ double red_s[16];
+  __shared__ double red_s[kWalkThreads / 32];
   __shared__ int act_s, u_s, ok_s, fell_s;
   __shared__ double c_s;
   const int r = blockIdx.x, tid = threadIdx.x;
@@ -616,14 +619,20 @@ __global__ void __launch_bounds__(512) tree_walk_kernel(AcceptParams p, const fl
 // bonus is the inverse-CDF pick the GEMM epilogue made inside the winning block.  A residual
 // with no positive weight anywhere (p <= q everywhere: p = q up to rounding) gives the argmax
 // of p instead, taken from the per-block logit maxima.
-__global__ void bonus_kernel(AcceptParams p) {
+constexpr int kBonusThreads = 256;
+
+__global__ void __launch_bounds__(kBonusThreads) bonus_kernel(AcceptParams p) {
+  __shared__ float kb_s[kBonusThreads / 32], zm_s[kBonusThreads / 32];
+  __shared__ int ib_s[kBonusThreads / 32], iz_s[kBonusThreads / 32];
   const int r = blockIdx.x;
-  const int lane = threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int node = p.stop_node[r];
   const float4* row = p.part2 + (size_t)r * p.n_tiles2;
   float kb = -INFINITY, zm = -INFINITY;
   int ib = -1, iz = -1;
-  for (int g = lane; g * 8 < p.n_tiles2; g += 32) {
+  // blocks in groups of 8 (one Philox draw) over the CTA; the merges are a total order (larger
+  // key, then lower id), so the split does not change the result
+  for (int g = threadIdx.x; g * 8 < p.n_tiles2; g += kBonusThreads) {
     float u[8];
     uniforms8(p.seed, p.step, (uint32_t)g, (uint32_t)node, (uint32_t)r, 2u, u);
 #pragma unroll
@@ -646,6 +655,17 @@ __global__ void bonus_kernel(AcceptParams p) {
     merge_key(zm, iz, ozm, oiz);
   }
   if (lane == 0) {
+    kb_s[warp] = kb;
+    ib_s[warp] = ib;
+    zm_s[warp] = zm;
+    iz_s[warp] = iz;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kBonusThreads / 32; ++w) {
+      merge_key(kb, ib, kb_s[w], ib_s[w]);
+      merge_key(zm, iz, zm_s[w], iz_s[w]);
+    }
     const int base = p.cu_nodes[r];
     const int n = p.cu_nodes[r + 1] - base;
     if (n < 1 || n > p.n_max) return;
@@ -680,12 +700,12 @@ cudaError_t launch_tree_prep(const AcceptParams& p, const __nv_bfloat16* w_lm, i
 cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32_t* zrow,
                              const float* zbuf, cudaStream_t s) {
   row_lse_kernel<<<(p.n_total + 7) / 8, 256, 0, s>>>(p);
-  tree_walk_kernel<<<p.B, 512, 0, s>>>(p, zc, zrow, zbuf);
+  tree_walk_kernel<<<p.B, kWalkThreads, 0, s>>>(p, zc, zrow, zbuf);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bonus(const AcceptParams& p, cudaStream_t s) {
-  bonus_kernel<<<p.B, 32, 0, s>>>(p);
+  bonus_kernel<<<p.B, kBonusThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
