@@ -316,31 +316,28 @@ __global__ void attn_combine_kernel(AttnParams p, int n_total) {
   if (n < 1 || n > p.n_max || L < 0 || L > p.kv_len_max) return;   // reported by the main kernel
   const int total = (L + p.keys - 1) / p.keys + (n + p.keys - 1) / p.keys;
   const int used = min(p.nsplit, (total + p.tps - 1) / p.tps);
-  // splits in groups of 4 so that each group's loads are in flight together
   const float2* mlp = p.ml_part + (size_t)gw * p.nsplit;
   const float4* op = reinterpret_cast<const float4*>(p.o_part + (size_t)gw * p.nsplit * 128);
+  // the maximum: one split per lane, then across the warp
   float M = -INFINITY;
-  for (int s0 = 0; s0 < used; s0 += 4) {
-    float mx[4];
+  for (int s = lane; s < used; s += 32) M = fmaxf(M, mlp[s].x);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) mx[i] = s0 + i < used ? mlp[s0 + i].x : -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) M = fmaxf(M, mx[i]);
-  }
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   const float Mb = (M == -INFINITY) ? 0.f : M;
+  // the weighted sums in split order, eight splits' loads in flight at a time
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float lsum = 0.f;
-  for (int s0 = 0; s0 < used; s0 += 4) {
-    float2 ml[4];
-    float4 v[4];
+  for (int s0 = 0; s0 < used; s0 += 8) {
+    float2 ml[8];
+    float4 v[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       const bool in = s0 + i < used;
       ml[i] = in ? mlp[s0 + i] : make_float2(-INFINITY, 0.f);
       v[i] = in ? op[(size_t)(s0 + i) * 32 + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       const float w = s0 + i < used ? exp2f(ml[i].x - Mb) : 0.f;
       lsum += ml[i].y * w;
       acc.x += v[i].x * w;
