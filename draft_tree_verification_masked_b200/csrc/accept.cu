@@ -173,12 +173,12 @@ __global__ void __launch_bounds__(256) greedy_accept_kernel(AcceptParams p, int3
   float t1 = -INFINITY, t2 = -INFINITY;
   int id = -1;
   int t = lane;
-  for (; t + 96 < p.n_tiles; t += 128) {             // four loads in flight per lane
-    const float4 a = part[t], b = part[t + 32], c = part[t + 64], d = part[t + 96];
-    merge_top2(t1, id, t2, a.x, __float_as_int(a.y), a.z);
-    merge_top2(t1, id, t2, b.x, __float_as_int(b.y), b.z);
-    merge_top2(t1, id, t2, c.x, __float_as_int(c.y), c.z);
-    merge_top2(t1, id, t2, d.x, __float_as_int(d.y), d.z);
+  for (; t + 224 < p.n_tiles; t += 256) {            // eight loads in flight per lane
+    float4 x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = part[t + 32 * u];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) merge_top2(t1, id, t2, x[u].x, __float_as_int(x[u].y), x[u].z);
   }
   for (; t < p.n_tiles; t += 32) {
     const float4 a = part[t];
@@ -304,12 +304,12 @@ __global__ void __launch_bounds__(256) chain_accept_kernel(AcceptParams p, int32
   const float4* part = p.part + (size_t)row * p.n_tiles;
   float m = -INFINITY, s = 0.f;
   int t = lane;
-  for (; t + 96 < p.n_tiles; t += 128) {
-    const float4 a = part[t], b = part[t + 32], c = part[t + 64], d = part[t + 96];
-    merge_lse(m, s, a.x, a.y);
-    merge_lse(m, s, b.x, b.y);
-    merge_lse(m, s, c.x, c.y);
-    merge_lse(m, s, d.x, d.y);
+  for (; t + 224 < p.n_tiles; t += 256) {            // eight loads in flight, merged in order
+    float4 x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = part[t + 32 * u];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) merge_lse(m, s, x[u].x, x[u].y);
   }
   for (; t < p.n_tiles; t += 32) {
     const float4 a = part[t];
@@ -423,12 +423,12 @@ __global__ void __launch_bounds__(256) row_lse_kernel(AcceptParams p) {
   const float4* part = p.part + (size_t)row * p.n_tiles;
   float m = -INFINITY, s = 0.f;
   int t = lane;
-  for (; t + 96 < p.n_tiles; t += 128) {
-    const float4 a = part[t], b = part[t + 32], c = part[t + 64], d = part[t + 96];
-    merge_lse(m, s, a.x, a.y);
-    merge_lse(m, s, b.x, b.y);
-    merge_lse(m, s, c.x, c.y);
-    merge_lse(m, s, d.x, d.y);
+  for (; t + 224 < p.n_tiles; t += 256) {            // eight loads in flight, merged in order
+    float4 x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = part[t + 32 * u];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) merge_lse(m, s, x[u].x, x[u].y);
   }
   for (; t < p.n_tiles; t += 32) {
     const float4 a = part[t];
