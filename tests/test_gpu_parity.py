@@ -377,3 +377,29 @@ def test_inputs_written_by_the_kernel_before_each_call():
     excused, near, ores = P.greedy_compare(wl, res, list(range(wl.B)))
     P.compact_compare(wl, dev, ores, list(range(wl.B)), excused)
     assert near <= 1, near
+
+
+def test_lowrank_hidden_written_by_the_kernel_before_the_call():
+    """The hidden rows are produced by the kernel launched just before the low-rank call on the
+    same stream (its kernels start their set-up early under programmatic dependent launch), and
+    the call repeats on the same workspace: the candidates still match the oracle."""
+    from draft_tree_verification_masked_b200 import (etree_lowrank_candidates,
+                                                     etree_lowrank_workspace_size,
+                                                     etree_workspace_init, etree_device_status)
+    lw = W.lowrank("lowrank_tiny")
+    dev = torch.device("cuda")
+    h, D, U, Wt = (x.to(dev) for x in (lw.hidden, lw.D, lw.U, lw.W))
+    ws = torch.zeros(etree_lowrank_workspace_size(lw.M, lw.H, lw.r, lw.V), dtype=torch.uint8,
+                     device=dev)
+    etree_workspace_init(ws)
+    ids = torch.full((lw.M, lw.k), -7, dtype=torch.int32, device=dev)
+    lg = torch.empty(lw.M, lw.k, dtype=torch.float32, device=dev)
+    h_in = torch.zeros_like(h)
+    for _ in range(3):
+        h_in.zero_()
+        torch.cuda.synchronize()
+        h_in.copy_(h)                                    # written right before the call
+        etree_lowrank_candidates(h_in, D, U, Wt, lw.k, ids, lg, ws)
+    assert etree_device_status(ws) == (0, 0)
+    differ = P.lowrank_compare(lw, ids.cpu().numpy(), lg.cpu().numpy())
+    assert differ <= max(1, lw.M // 10), differ
