@@ -1,0 +1,35 @@
+"""Host-side helpers of bench.py (no GPU): the source fingerprint that ties a committed ncu
+traffic figure to the kernel sources it was measured on."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_strip_comments_keeps_code_and_literals():
+    src = ('int a = 1; // trailing\n'
+           '/* block\n comment */ float b = 2.f;\n'
+           'const char* s = "not // a comment";\n'
+           "char c = '/';  char d = '\\'';\n"
+           '  int   e  =  3 ;')
+    out = bench.strip_comments(src)
+    assert "trailing" not in out and "block" not in out
+    assert '"not // a comment"' in out
+    assert "'/'" in out and "'\\''" in out
+    assert "int a = 1;" in out and "float b = 2.f;" in out and "int e = 3 ;" in out
+
+
+def test_comment_edits_do_not_change_the_fingerprint(tmp_path, monkeypatch):
+    csrc = tmp_path / "draft_tree_verification_masked_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (csrc / "k.cu").write_text("// v1\n__global__ void k(int* p) { p[0] = 1; }\n")
+    h1 = bench.source_hash("k.cu")
+    (csrc / "k.cu").write_text("/* a new comment */\n__global__  void k(int* p) {\n  p[0] = 1; }\n")
+    assert bench.source_hash("k.cu") == h1
+    (csrc / "k.cu").write_text("__global__ void k(int* p) { p[0] = 2; }\n")
+    assert bench.source_hash("k.cu") != h1
+
