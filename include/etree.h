@@ -64,7 +64,7 @@ typedef enum {
   ETREE_ENOSPACE = -6       /* a request's cache slots cannot hold the accepted tokens        */
 } etree_status;
 
-/* Limits of this build. */
+/* Compile-time limits of the library. */
 #define ETREE_MAX_NODES 64      /* nodes per tree, root included (ancestor masks are uint64)  */
 #define ETREE_MAX_REQUESTS 4096
 #define ETREE_HEAD_DIM 128
