@@ -33,3 +33,27 @@ def test_comment_edits_do_not_change_the_fingerprint(tmp_path, monkeypatch):
     (csrc / "k.cu").write_text("__global__ void k(int* p) { p[0] = 2; }\n")
     assert bench.source_hash("k.cu") != h1
 
+
+
+def test_packed_buffer_layout():
+    """The step's inputs share one buffer: every tensor starts on a 256-byte boundary, none
+    overlaps the next, and the views alias the buffer (a copy into the buffer reaches them)."""
+    import torch
+    from draft_tree_verification_masked_b200.runner import Packed
+    specs = [("a", (5,), torch.int32), ("b", (3, 7), torch.int64), ("c", (2, 3, 4), torch.bfloat16),
+             ("d", (1,), torch.float32)]
+    pk = Packed(specs, "cpu")
+    prev_end = 0
+    for name, shape, dtype in specs:
+        off = pk.offset(name)
+        v = pk.view(name)
+        assert off % 256 == 0 and off >= prev_end, name
+        assert tuple(v.shape) == shape and v.dtype == dtype, name
+        prev_end = off + v.numel() * v.element_size()
+    assert pk.buf.numel() >= prev_end
+    pk.buf.copy_(torch.arange(pk.buf.numel(), dtype=torch.int64).to(torch.uint8))
+    a = pk.view("a")
+    assert bytes(a.numpy().tobytes()) == bytes(pk.buf[:20].numpy().tobytes())
+    # the tail from a tensor's offset holds it and everything after it
+    tail = pk.buf[pk.offset("c"):]
+    assert tail.numel() >= pk.view("c").numel() * 2 + pk.view("d").numel() * 4
