@@ -31,7 +31,8 @@ __all__ = [
     "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact",
     "etree_verify_attn_paged", "etree_kv_compact_paged", "etree_verify_cost", "etree_plan_tree",
     "cost_table", "load_cost_table", "etree_lowrank_workspace_size",
-    "etree_lowrank_candidates", "etree_device_status", "etree_strerror", "etree_version", "etree_attn_plan", "STATUS",
+    "etree_lowrank_candidates", "etree_device_status", "etree_selftest_timeout", "etree_strerror",
+    "etree_version", "etree_attn_plan", "STATUS",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -40,13 +41,15 @@ _LIB_PATH = os.path.join(HERE, "libetree.so")
 STATUS = {0: "ETREE_OK", -1: "ETREE_EINVAL", -2: "ETREE_EUNSUPPORTED", -3: "ETREE_ECUDA",
           -4: "ETREE_EDEVICE", -5: "ETREE_ETIMEOUT", -6: "ETREE_ENOSPACE"}
 DETAIL = {0: "none", 1: "bad parent", 2: "bad node count", 3: "bad kv_len", 4: "capacity",
-          5: "not a chain", 6: "bad path", 7: "attention wait", 8: "gemm wait", 9: "bad token"}
+          5: "not a chain", 6: "bad path", 7: "attention wait", 8: "gemm wait", 9: "bad token",
+          10: "logit rows", 11: "bad page", 12: "self-test wait"}
 
 EXPORTS = ["etree_workspace_size", "etree_workspace_init", "etree_verify_attn",
            "etree_verify_attn_paged", "etree_kv_compact_paged", "etree_verify_cost",
            "etree_plan_tree", "etree_lowrank_workspace_size", "etree_lowrank_candidates",
            "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact", "etree_device_status", "etree_strerror",
-           "etree_version", "etree_last_error", "etree_attn_plan", "etree_verify_attn_noalloc"]
+           "etree_version", "etree_last_error", "etree_attn_plan", "etree_verify_attn_noalloc",
+           "etree_selftest_timeout"]
 
 
 class EtreeError(RuntimeError):
@@ -118,6 +121,8 @@ def lib():
     L.etree_kv_compact_paged.restype = C.c_int
     L.etree_device_status.argtypes = [vp, vp, C.POINTER(i32)]
     L.etree_device_status.restype = C.c_int
+    L.etree_selftest_timeout.argtypes = [vp, C.c_size_t, vp]
+    L.etree_selftest_timeout.restype = C.c_int
     L.etree_strerror.argtypes = [C.c_int]
     L.etree_strerror.restype = C.c_char_p
     L.etree_last_error.argtypes = []
@@ -393,6 +398,13 @@ def etree_attn_plan(batch: Batch, hq: int, hkv: int) -> dict:
     _check(lib().etree_attn_plan(C.byref(batch), hq, hkv, *[C.byref(x) for x in v]))
     return dict(zip(["kernel", "rows_per_cta", "row_blocks", "splits", "tiles_per_split",
                      "launches"], [int(x.value) for x in v]))
+
+
+def etree_selftest_timeout(workspace: torch.Tensor, stream=None, check: bool = True) -> int:
+    """Enqueue the bounded-wait self-test; etree_device_status then reports ETREE_ETIMEOUT."""
+    st = lib().etree_selftest_timeout(_ptr(workspace, torch.uint8, "workspace"),
+                                      workspace.numel(), _stream(stream))
+    return _check(st) if check else st
 
 
 def etree_device_status(workspace: torch.Tensor, stream=None) -> tuple[int, int]:

@@ -459,6 +459,28 @@ etree_status etree_device_status(void* workspace, void* stream, int32_t* detail)
   return static_cast<etree_status>(h[0]);
 }
 
+// The bounded-wait path every pipeline relies on, exercised on purpose: one thread waits on an
+// mbarrier that no thread ever arrives at; the wait gives up after its iteration cap and the
+// kernel records ETREE_ETIMEOUT (detail DET_SELFTEST) in the workspace status word.  Nothing
+// traps, and the context stays usable.
+__global__ void selftest_wait_kernel(WsHeader* ws) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    if (!mbar_wait(&bar, 0)) report(ws, ETREE_ETIMEOUT, DET_SELFTEST);
+  }
+}
+
+etree_status etree_selftest_timeout(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || workspace_bytes < sizeof(WsHeader) || ((uintptr_t)workspace & 255))
+    return fail(ETREE_EINVAL, "workspace is NULL, smaller than its header or misaligned");
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      at<WsHeader>(workspace, 0));
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_selftest_timeout launch");
+}
+
 // A paged cache: the block table [B][max_pages] and the page size (a power of two >= 16).
 struct PagedArgs {
   const int32_t* block_table;

@@ -35,6 +35,7 @@ enum Detail : int32_t {
   DET_BAD_TOKEN = 9,        // a token id outside [0, vocab)
   DET_ZBUF = 10,            // more branching tree nodes than rows in the caller's logit buffer
   DET_BAD_PAGE = 11,        // a block-table entry outside [0, num_pages) for a used position
+  DET_SELFTEST = 12,        // etree_selftest_timeout: the deliberately unfinished wait gave up
 };
 
 __device__ __forceinline__ void report(WsHeader* ws, int32_t code, int32_t detail) {
@@ -81,7 +82,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Iteration cap of every mbarrier wait.  try_wait suspends for a hardware-chosen interval per
-// call, so the cap bounds a wait to well under a few seconds; a wait that runs out returns false.
+// call (about 4 us when nothing arrives), so the cap bounds a wait to about 8 s on a B200; a wait
+// that runs out returns false.
 constexpr uint32_t kWaitCap = 1u << 21;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {

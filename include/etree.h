@@ -339,6 +339,15 @@ etree_status etree_plan_tree(const etree_cost_table *table, int32_t B, int32_t L
  */
 etree_status etree_device_status(void *workspace, void *stream, int32_t *detail);
 
+/*
+ * Diagnostic: launches one thread that waits on a barrier nothing ever completes, through the same
+ * bounded wait every kernel of the library uses.  The wait gives up after its iteration cap
+ * (about 8 s on a B200) and records ETREE_ETIMEOUT with detail 12 in the workspace status word,
+ * which etree_device_status then returns; nothing traps and the context stays usable.  The
+ * workspace needs only its 256-byte status header (256-byte aligned).
+ */
+etree_status etree_selftest_timeout(void *workspace, size_t workspace_bytes, void *stream);
+
 /* Static description of a status code. */
 const char *etree_strerror(etree_status status);
 

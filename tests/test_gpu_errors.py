@@ -136,3 +136,20 @@ def test_host_argument_errors():
                                dev.v_cache, 1, 0, 0, dev.kv_len, dev.ws, **call) == EINVAL
     assert dev.status() == (0, 0)
     _still_works()
+
+
+def test_bounded_wait_runs_out_reports_and_leaves_the_context_usable():
+    """A wait that nothing completes, through the library's own bounded wait: it gives up after
+    its iteration cap, the status word says ETREE_ETIMEOUT (detail 12), nothing traps, and a normal
+    step runs correctly afterwards."""
+    import time
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    et.etree_workspace_init(ws)
+    t0 = time.perf_counter()
+    et.etree_selftest_timeout(ws)
+    st, det = et.etree_device_status(ws)
+    elapsed = time.perf_counter() - t0
+    assert (st, det) == (-5, 12), (st, det)
+    assert elapsed < 120.0, elapsed
+    assert et.etree_device_status(ws) == (0, 0)           # read clears the word
+    _still_works()
