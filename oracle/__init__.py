@@ -28,66 +28,70 @@ F32P = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
 OK, EINVAL, EUNSUPPORTED, ENOSPACE = 0, -1, -2, -6
 
 
+def _bind(path: str):
+    """Load the oracle library at `path` and declare its signatures."""
+    L = C.CDLL(path)
+    L.oracle_max_threads.restype = C.c_int
+    L.oracle_ancestry.argtypes = [C.c_int, I32P, U64P, I32P]
+    L.oracle_ancestry.restype = C.c_int
+    L.oracle_attention.argtypes = [C.c_int, I32P, I32P, I32P, I64P, U16P, U16P, U16P, U16P,
+                                   U16P, C.c_int, C.c_int, C.c_int, C.c_double, C.c_int,
+                                   C.c_void_p, F64P, F64P, C.c_int]
+    L.oracle_attention.restype = C.c_int
+    L.oracle_logits.argtypes = [C.c_int, I32P, C.c_int, C.c_int, U16P, U16P, F64P, C.c_int]
+    L.oracle_logits.restype = None
+    L.oracle_row_top2.argtypes = [C.c_int, C.c_int, F64P, I32P, F64P, F64P]
+    L.oracle_row_top2.restype = None
+    L.oracle_walk_greedy.argtypes = [C.c_int, I32P, I32P, I32P, I32P, I32P]
+    L.oracle_walk_greedy.restype = C.c_int
+    L.oracle_philox4x64.argtypes = [U64P, U64P, U64P]
+    L.oracle_philox4x64.restype = None
+    L.oracle_uniform.argtypes = [C.c_uint64, C.c_uint64, C.c_uint32, C.c_uint32, C.c_uint32,
+                                 C.c_uint32]
+    L.oracle_uniform.restype = C.c_double
+    L.oracle_race.argtypes = [C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int, C.c_int,
+                              C.POINTER(C.c_double)]
+    L.oracle_race.restype = C.c_int
+    L.oracle_accept_chain.argtypes = [C.c_int, I32P, I32P, F64P, F32P, C.c_int, C.c_double,
+                                      C.c_uint64, C.c_uint64, C.c_int, I32P, I32P, I32P]
+    L.oracle_accept_chain.restype = C.c_int
+    L.oracle_kv_compact.argtypes = [C.c_int, I32P, I32P, I64P, I32P, I32P, I32P, U16P, U16P,
+                                    U16P, U16P, C.c_int, C.c_int64, C.c_int64, C.c_int,
+                                    C.c_int, I32P]
+    L.oracle_kv_compact.restype = C.c_int
+    L.oracle_accept_chain_batch.argtypes = [C.c_int, I32P, I32P, I32P, F64P, F32P, C.c_int,
+                                            C.c_double, C.c_uint64, C.c_uint64, I32P, I32P,
+                                            I32P, I32P, C.c_int]
+    L.oracle_accept_chain_batch.restype = None
+    L.oracle_accept_tree.argtypes = [C.c_int, I32P, I32P, F64P, F32P, C.c_int, C.c_double,
+                                     C.c_uint64, C.c_uint64, C.c_int, I32P, I32P, I32P,
+                                     C.POINTER(C.c_double)]
+    L.oracle_accept_tree.restype = C.c_int
+    L.oracle_accept_tree_batch.argtypes = [C.c_int, I32P, I32P, I32P, F64P, F32P, C.c_int,
+                                           C.c_double, C.c_uint64, C.c_uint64, I32P, I32P,
+                                           I32P, I32P, F64P, C.c_int]
+    L.oracle_accept_tree_batch.restype = None
+    L.oracle_bf16_round.argtypes = [C.c_double]
+    L.oracle_bf16_round.restype = C.c_uint16
+    L.oracle_lowrank_candidates.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                            U16P, U16P, U16P, U16P, I32P, F64P, C.c_void_p,
+                                            C.c_void_p, C.c_int]
+    L.oracle_lowrank_candidates.restype = None
+    L.oracle_race_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
+                                   C.c_int, I32P, C.c_int]
+    L.oracle_race_many.restype = None
+    L.oracle_draw.argtypes = [C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int, C.c_int, I32P]
+    L.oracle_draw.restype = C.c_int
+    L.oracle_draw_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
+                                   C.c_int, I32P, C.c_int]
+    L.oracle_draw_many.restype = None
+    return L
+
+
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
-        L = C.CDLL(path)
-        L.oracle_max_threads.restype = C.c_int
-        L.oracle_ancestry.argtypes = [C.c_int, I32P, U64P, I32P]
-        L.oracle_ancestry.restype = C.c_int
-        L.oracle_attention.argtypes = [C.c_int, I32P, I32P, I32P, I64P, U16P, U16P, U16P, U16P,
-                                       U16P, C.c_int, C.c_int, C.c_int, C.c_double, C.c_int,
-                                       C.c_void_p, F64P, F64P, C.c_int]
-        L.oracle_attention.restype = C.c_int
-        L.oracle_logits.argtypes = [C.c_int, I32P, C.c_int, C.c_int, U16P, U16P, F64P, C.c_int]
-        L.oracle_logits.restype = None
-        L.oracle_row_top2.argtypes = [C.c_int, C.c_int, F64P, I32P, F64P, F64P]
-        L.oracle_row_top2.restype = None
-        L.oracle_walk_greedy.argtypes = [C.c_int, I32P, I32P, I32P, I32P, I32P]
-        L.oracle_walk_greedy.restype = C.c_int
-        L.oracle_philox4x64.argtypes = [U64P, U64P, U64P]
-        L.oracle_philox4x64.restype = None
-        L.oracle_uniform.argtypes = [C.c_uint64, C.c_uint64, C.c_uint32, C.c_uint32, C.c_uint32,
-                                     C.c_uint32]
-        L.oracle_uniform.restype = C.c_double
-        L.oracle_race.argtypes = [C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int, C.c_int,
-                                  C.POINTER(C.c_double)]
-        L.oracle_race.restype = C.c_int
-        L.oracle_accept_chain.argtypes = [C.c_int, I32P, I32P, F64P, F32P, C.c_int, C.c_double,
-                                          C.c_uint64, C.c_uint64, C.c_int, I32P, I32P, I32P]
-        L.oracle_accept_chain.restype = C.c_int
-        L.oracle_kv_compact.argtypes = [C.c_int, I32P, I32P, I64P, I32P, I32P, I32P, U16P, U16P,
-                                        U16P, U16P, C.c_int, C.c_int64, C.c_int64, C.c_int,
-                                        C.c_int, I32P]
-        L.oracle_kv_compact.restype = C.c_int
-        L.oracle_accept_chain_batch.argtypes = [C.c_int, I32P, I32P, I32P, F64P, F32P, C.c_int,
-                                                C.c_double, C.c_uint64, C.c_uint64, I32P, I32P,
-                                                I32P, I32P, C.c_int]
-        L.oracle_accept_chain_batch.restype = None
-        L.oracle_accept_tree.argtypes = [C.c_int, I32P, I32P, F64P, F32P, C.c_int, C.c_double,
-                                         C.c_uint64, C.c_uint64, C.c_int, I32P, I32P, I32P,
-                                         C.POINTER(C.c_double)]
-        L.oracle_accept_tree.restype = C.c_int
-        L.oracle_accept_tree_batch.argtypes = [C.c_int, I32P, I32P, I32P, F64P, F32P, C.c_int,
-                                               C.c_double, C.c_uint64, C.c_uint64, I32P, I32P,
-                                               I32P, I32P, F64P, C.c_int]
-        L.oracle_accept_tree_batch.restype = None
-        L.oracle_bf16_round.argtypes = [C.c_double]
-        L.oracle_bf16_round.restype = C.c_uint16
-        L.oracle_lowrank_candidates.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
-                                                U16P, U16P, U16P, U16P, I32P, F64P, C.c_void_p,
-                                                C.c_void_p, C.c_int]
-        L.oracle_lowrank_candidates.restype = None
-        L.oracle_race_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
-                                       C.c_int, I32P, C.c_int]
-        L.oracle_race_many.restype = None
-        L.oracle_draw.argtypes = [C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int, C.c_int, I32P]
-        L.oracle_draw.restype = C.c_int
-        L.oracle_draw_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
-                                       C.c_int, I32P, C.c_int]
-        L.oracle_draw_many.restype = None
-        _lib = L
+        _lib = _bind(_build.build())
     return _lib
 
 

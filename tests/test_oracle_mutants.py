@@ -1,0 +1,195 @@
+"""Planted mistakes: each case edits one spot of the oracle's C source (a dropped term, a wrong sign
+or index, a swapped operand, an off-by-one), compiles the edited copy into a scratch library and
+runs the pins that should notice.  Every case must make at least one of its pins fail, which shows
+the pins constrain that spot; the unedited oracle passes the same pins in test_oracle_pins.py.
+
+Only the oracle is edited, on the CPU, in a temporary directory; the committed source stays as it
+is.  Edits are chosen so that the edited program stays inside its buffers.
+"""
+import os
+
+import pytest
+
+import oracle
+from oracle import _build
+
+from . import test_oracle_pins as P
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+# (name, exact text in oracle.c, replacement, [(pin, args), ...])
+MUTANTS = [
+    # tree ancestry
+    ("ancestry_parent_bit_only",
+     "anc[i] = anc[p] | (1ull << i);", "anc[i] = (1ull << p) | (1ull << i);",
+     [(P.test_ancestry_equals_transitive_closure, ())]),
+    ("ancestry_root_not_its_own_ancestor",
+     "anc[0] = 1ull;", "anc[0] = 0ull;",
+     [(P.test_ancestry_equals_transitive_closure, ())]),
+    ("ancestry_depth_not_advanced",
+     "depth[i] = depth[p] + 1;", "depth[i] = depth[p];",
+     [(P.test_ancestry_equals_transitive_closure, ())]),
+    # attention
+    ("attention_mask_by_index_order",
+     "if (!((anc[i] >> j) & 1ull)) { s[L + j] = -INFINITY; continue; }",
+     "if (j > i) { s[L + j] = -INFINITY; continue; }",
+     [(P.test_tree_attention_equals_dense_closure_mask, (16, 6, 4, None))]),
+    ("attention_cache_scores_unscaled",
+     "                s[t] = scale * acc;\n", "                s[t] = acc;\n",
+     [(P.test_chain_tree_equals_causal_attention, ())]),
+    ("attention_gqa_heads_round_robin",
+     "int kvh = h / group;", "int kvh = h % hkv;",
+     [(P.test_tree_attention_equals_dense_closure_mask, (16, 6, 4, None))]),
+    ("attention_cache_rows_ignore_slot_base",
+     "const uint16_t *kr = k_cache + ((size_t)(slot_base[r] + t) * hkv + kvh) * d;",
+     "const uint16_t *kr = k_cache + ((size_t)(t) * hkv + kvh) * d;",
+     [(P.test_single_node_tree_equals_one_token_decode, ())]),
+    ("attention_tree_values_read_from_keys",
+     ": v_tree + ((size_t)(base + (t - L)) * hkv + kvh) * d;",
+     ": k_tree + ((size_t)(base + (t - L)) * hkv + kvh) * d;",
+     [(P.test_chain_tree_equals_causal_attention, ())]),
+    ("attention_lse_without_max",
+     "if (lse) lse[k] = mx + log(den);", "if (lse) lse[k] = log(den);",
+     [(P.test_chain_tree_equals_causal_attention, ())]),
+    # LM head
+    ("logits_weight_transposed",
+     "wrow[h] = bf16_value(w[(size_t)v * H + h]);", "wrow[h] = bf16_value(w[(size_t)h * V + v]);",
+     [(P.test_logits_equal_numpy_matmul, ())]),
+    ("argmax_ties_to_highest_id",
+     "if (row[v] > row[best]) best = v;", "if (row[v] >= row[best]) best = v;",
+     [(P.test_row_top2_ties_and_order, ())]),
+    ("top2_skips_a_repeated_maximum",
+     "if (v != best && row[v] > second) second = row[v];",
+     "if (row[v] != row[best] && row[v] > second) second = row[v];",
+     [(P.test_row_top2_ties_and_order, ())]),
+    # greedy walk
+    ("greedy_highest_index_duplicate_child",
+     "if (parent[c] == u && tokens[c] == want) { next = c; break; }",
+     "if (parent[c] == u && tokens[c] == want) { next = c; }",
+     [(P.test_greedy_walk_duplicate_siblings_take_the_lowest_index, ())]),
+    ("greedy_bonus_from_the_root",
+     "    out_tokens[a] = arg[u];\n    return a;", "    out_tokens[a] = arg[0];\n    return a;",
+     [(P.test_greedy_walk_equals_sequential_greedy_decoding, (s,)) for s in range(12)]),
+    # Philox and the uniforms
+    ("philox_key_words_swapped",
+     "uint64_t n0 = hi1 ^ c1 ^ k0, n1 = lo1, n2 = hi0 ^ c3 ^ k1, n3 = lo0;",
+     "uint64_t n0 = hi1 ^ c1 ^ k1, n1 = lo1, n2 = hi0 ^ c3 ^ k0, n3 = lo0;",
+     [(P.test_philox_random_counters_match_numpy, ())]),
+    ("philox_weyl_constant",
+     "W1 = 0xBB67AE8584CAA73Bull", "W1 = 0xBB67AE8584CAA73Aull",
+     [(P.test_philox_random_counters_match_numpy, ())]),
+    ("philox_nine_rounds",
+     "for (int round = 0; round < 10; ++round)", "for (int round = 0; round < 9; ++round)",
+     [(P.test_philox_random_counters_match_numpy, ())]),
+    ("uniform_field_too_wide",
+     ": (x >> 41);", ": (x >> 40);",
+     [(P.test_uniform_is_23bit_centred_exact_in_float32_and_uniform, ())]),
+    ("uniform_not_centred",
+     "return ((double)field + 0.5) * (1.0 / 8388608.0);",
+     "return ((double)field) * (1.0 / 8388608.0);",
+     [(P.test_uniform_is_23bit_centred_exact_in_float32_and_uniform, ())]),
+    # samplers
+    ("race_gumbel_sign",
+     "double key = log(w[v]) - log(-log(U));", "double key = log(w[v]) + log(-log(U));",
+     [(P.test_exponential_race_is_an_exact_sampler, ())]),
+    ("draw_block_total_not_summed",
+     "for (int v = b * 128; v < V && v < b * 128 + 128; ++v) W += w[v];",
+     "for (int v = b * 128; v < V && v < b * 128 + 128; ++v) W = w[v];",
+     [(P.test_two_level_draw_is_an_exact_sampler, (300,))]),
+    ("draw_inverse_cdf_reuses_the_race_stream",
+     "oracle_uniform(seed, step, (uint32_t)r, (uint32_t)node, (uint32_t)bstar, 3);",
+     "oracle_uniform(seed, step, (uint32_t)r, (uint32_t)node, (uint32_t)bstar, 2);",
+     [(P.test_two_level_draw_blocks_and_inverse_cdf_by_hand, ())]),
+    # stochastic acceptance on chains
+    ("chain_test_p_and_q_swapped",
+     "if (U * qx < p[x]) {", "if (U * p[x] < qx) {",
+     [(P.test_first_emitted_token_follows_target, (1.0,))]),
+    ("chain_residual_without_q",
+     "double d = p[v] - (double)q[(size_t)u * V + v];", "double d = p[v];",
+     [(P.test_rejected_draft_residual_excludes_the_rejected_token_mass, ())]),
+    ("chain_bonus_at_the_root",
+     "int u = a;  /* stop node", "int u = 0;  /* stop node",
+     [(P.test_second_emitted_token_follows_target_given_accepted_prefix, ())]),
+    ("softmax_drops_the_temperature",
+     "for (int v = 0; v < V; ++v) p[v] = exp(z[v] / T - lse);",
+     "for (int v = 0; v < V; ++v) p[v] = exp(z[v] - lse);",
+     [(P.test_first_emitted_token_follows_target, (0.7,))]),
+    # stochastic acceptance on branching trees
+    ("tree_residual_not_renormalised",
+     "rx = rx > 0.0 ? rx / Nc : 0.0;", "rx = rx > 0.0 ? rx : 0.0;",
+     [(P.test_multi_candidate_first_token_follows_target, (2, 1.0))]),
+    ("tree_scale_advanced_by_one",
+     "            c += Nc;\n", "            c += 1.0;\n",
+     [(P.test_multi_candidate_first_token_follows_target, (2, 1.0))]),
+    ("tree_siblings_share_one_uniform",
+     "oracle_uniform(seed, step, (uint32_t)r, (uint32_t)j, 0, 1);",
+     "oracle_uniform(seed, step, (uint32_t)r, (uint32_t)u + 1u, 0, 1);",
+     [(P.test_multi_candidate_sibling_acceptance_rates_match_the_closed_form, ())]),
+    ("tree_bonus_ignores_rejections",
+     "            const double d = p[v] - c * (double)qu[v];\n"
+     "            w[v] = d > 0.0 ? d : 0.0;",
+     "            const double d = p[v] + 0.0 * c * (double)qu[v];\n"
+     "            w[v] = d > 0.0 ? d : 0.0;",
+     [(P.test_multi_candidate_residual_excludes_rejected_mass, ())]),
+    # compaction
+    ("compact_destination_ignores_kv_len",
+     "+ (size_t)(slot_base[r] + kv_len[r] + k) * row;", "+ (size_t)(slot_base[r] + k) * row;",
+     [(P.test_kv_compact_equals_numpy_gather, ())]),
+    ("compact_new_length_misses_the_root",
+     "kv_len_out[r] = kv_len[r] + a + 1;\n    }", "kv_len_out[r] = kv_len[r] + a;\n    }",
+     [(P.test_kv_compact_equals_numpy_gather, ())]),
+    ("compact_capacity_off_by_one",
+     "if ((int64_t)kv_len[r] + a + 1 > (int64_t)slot_cap[r])",
+     "if ((int64_t)kv_len[r] + a > (int64_t)slot_cap[r])",
+     [(P.test_kv_compact_fills_capacity_exactly_and_no_further, ())]),
+    ("compact_source_row_from_path_index",
+     "size_t src = (size_t)l * tree_layer_stride + (size_t)(cu_nodes[r] + j) * row;",
+     "size_t src = (size_t)l * tree_layer_stride + (size_t)(cu_nodes[r] + k) * row;",
+     [(P.test_kv_compact_equals_numpy_gather, ())]),
+    # bf16 rounding and the low-rank head
+    ("bf16_ties_away_from_zero",
+     "else r = fmod(lo / ulp, 2.0) == 0.0 ? lo : hi;", "else r = hi;",
+     [(P.test_bf16_rounding_is_nearest_even, ())]),
+    ("lowrank_down_projection_not_rounded",
+     "g[t] = bf16_value(oracle_bf16_round(acc));", "g[t] = acc;",
+     [(P.test_lowrank_screen_rounds_the_down_projection_to_bf16, ())]),
+    ("lowrank_screen_ties_to_highest_id",
+     "if (!taken[v] && (best < 0 || z[v] > z[best])) best = v;",
+     "if (!taken[v] && (best < 0 || z[v] >= z[best])) best = v;",
+     [(P.test_lowrank_screen_rounds_the_down_projection_to_bf16, ())]),
+    ("lowrank_exact_order_ascending",
+     "while (j >= 0 && (ex[j] < xi || (ex[j] == xi && cand[j] > ci))) {",
+     "while (j >= 0 && (ex[j] > xi || (ex[j] == xi && cand[j] > ci))) {",
+     [(P.test_lowrank_head_with_identity_factors_is_the_exact_top_k, ())]),
+]
+
+
+def _source():
+    with open(_build.SRC) as f:
+        return f.read()
+
+
+def test_every_planted_spot_exists_once():
+    src = _source()
+    for name, old, new, _ in MUTANTS:
+        assert src.count(old) == 1, name
+        assert old != new, name
+    assert len({m[0] for m in MUTANTS}) == len(MUTANTS)
+
+
+@pytest.mark.parametrize("name,old,new,pins", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_the_planted_mistake(name, old, new, pins, tmp_path, monkeypatch):
+    src = _source()
+    assert src.count(old) == 1
+    c_path = os.path.join(tmp_path, "mutant.c")
+    with open(c_path, "w") as f:
+        f.write(src.replace(old, new))
+    lib_path = _build.compile_to(c_path, os.path.join(tmp_path, "libmutant.so"))
+    monkeypatch.setattr(oracle, "_lib", oracle._bind(lib_path))
+    caught = []
+    for pin, args in pins:
+        try:
+            pin(*args)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"{name}: no pin failed"

@@ -293,6 +293,20 @@ def test_greedy_walk_equals_sequential_greedy_decoding(seed):
     assert (out[a + 1:] == -1).all() and (path[a + 1:] == -1).all()
 
 
+def test_greedy_walk_duplicate_siblings_take_the_lowest_index():
+    """Reading: when several children of the current node carry the argmax token, the walk takes
+    the lowest node index.  Hand-worked tree: root 0 has children 1 (token 7), 2 (token 3) and
+    3 (token 3); node 2 has child 4 (token 5), node 3 has child 5 (token 5).  The argmax rows are
+    root -> 3, node 2 -> 5, node 3 -> 5, node 4 -> 9, node 5 -> 1, so the walk is 0 -> 2 -> 4
+    and emits 3, 5 and the bonus 9 (through node 3 the bonus would be 1)."""
+    par = np.array([-1, 0, 0, 0, 2, 3], dtype=np.int32)
+    tok = np.array([0, 7, 3, 3, 5, 5], dtype=np.int32)
+    arg = np.array([3, 0, 5, 5, 9, 1], dtype=np.int32)
+    a, path, out = oracle.walk_greedy(par, tok, arg)
+    assert a == 2 and list(path[:3]) == [0, 2, 4] and list(out[:3]) == [3, 5, 9]
+    assert (path[3:] == -1).all() and (out[3:] == -1).all()
+
+
 # ------------------------------------------------------------------------ stochastic acceptance
 def _softmax(x):
     e = np.exp(x - x.max())
@@ -515,9 +529,11 @@ def _tree_trials(k, pz, qz, T, ntrial, seed, chunk=100_000):
         for j in range(2 * k):
             parent_tok = tok[:, 1 + j // 2]
             u = g.random(m)
-            tok[:, 1 + k + j] = np.minimum(
-                V - 1, np.array([np.searchsorted(cq[1 + x], uu * cq[1 + x, -1])
-                                 for x, uu in zip(parent_tok, u)]))
+            t = np.empty(m, dtype=np.int64)
+            for x in range(V):                          # inverse CDF of q_x, grouped by x
+                sel = parent_tok == x
+                t[sel] = np.searchsorted(cq[1 + x], u[sel] * cq[1 + x, -1])
+            tok[:, 1 + k + j] = np.minimum(V - 1, t)
             rowsel[:, 1 + k + j] = 0                    # grandchildren are leaves: rows unused
         z = pz[rowsel.reshape(-1)]
         q = q_of[rowsel.reshape(-1)]
@@ -550,6 +566,37 @@ def test_multi_candidate_first_token_follows_target(k, T):
     x = np.bincount(first[acc], minlength=V).argmax()
     sel = acc & (first == x)
     assert _chisq_p(second[sel], _softmax(pz[1 + x] / T)) > 1e-4
+
+
+@pytest.mark.slow
+def test_multi_candidate_sibling_acceptance_rates_match_the_closed_form():
+    """10^6 trials of a root with two leaf children drafted independently from q, V=16.  The first
+    child is accepted with probability A1 = sum min(p, q).  After its rejection the target is
+    r1 = max(0, p - q) / (1 - A1) whatever token was rejected, and the second child, a fresh draw
+    from q tested with a fresh uniform, is accepted with probability A2 = sum min(q, r1)."""
+    V, T, m = 16, 1.0, 1_000_000
+    g = np.random.default_rng(45)
+    z = g.normal(0, 1.5, size=V)
+    qv = _softmax(g.normal(0, 1.5, size=V)).astype(np.float32)
+    p = _softmax(z / T)
+    q64 = qv.astype(np.float64)
+    A1 = np.minimum(p, q64).sum()
+    r1 = np.maximum(0.0, p - q64) / (1.0 - A1)
+    A2 = np.minimum(q64, r1).sum()
+    cq = np.cumsum(q64)
+    tok = np.zeros((m, 3), dtype=np.int32)
+    tok[:, 1:] = np.minimum(V - 1, np.searchsorted(cq, g.random((m, 2)) * cq[-1]))
+    cu = (np.arange(m + 1) * 3).astype(np.int32)
+    par = np.tile(np.array([-1, 0, 0], dtype=np.int32), m)
+    zz = np.broadcast_to(z, (3 * m, V))
+    qq = np.broadcast_to(qv, (3 * m, V))
+    a, path, out, info, c = oracle.accept_tree_batch(cu, par, tok.reshape(-1), zz, qq, T,
+                                                      0xE7EE0700, 0)
+    first = (path[:, 1] == 1).mean()
+    second = (path[:, 1] == 2).mean()
+    for got, want in ((first, A1), (second, (1 - A1) * A2)):
+        assert abs(got - want) < 5 * np.sqrt(want * (1 - want) / m), (got, want)
+    assert _chisq_p(out[:, 0], p) > 1e-4
 
 
 def test_multi_candidate_identical_draft_accepts_the_first_child():
@@ -689,6 +736,30 @@ def test_kv_compact_capacity_overflow_leaves_request_untouched():
     assert st == oracle.ENOSPACE and newlen[0] == 10 and not ck.any()
 
 
+def test_kv_compact_fills_capacity_exactly_and_no_further():
+    """kv_len + a + 1 == slot_cap is accepted; one slot short is refused and the request left
+    untouched; no slot outside a request's written rows changes (the pool has spare slots past
+    each capacity)."""
+    cu = np.array([0, 4, 8], dtype=np.int32)
+    kv_len = np.array([8, 8], dtype=np.int32)
+    cap = np.array([12, 11], dtype=np.int32)
+    base = np.array([0, 16], dtype=np.int64)
+    a = np.array([3, 3], dtype=np.int32)
+    path = np.full((2, 64), -1, dtype=np.int32)
+    path[:, :4] = [0, 1, 2, 3]
+    tk = (np.arange(8, dtype=np.uint16)[:, None, None] + 1) * np.ones((8, 1, 8), np.uint16)
+    tv = tk + 100
+    ck = np.zeros((32, 1, 8), dtype=np.uint16)
+    cv = np.zeros((32, 1, 8), dtype=np.uint16)
+    st, newlen = oracle.kv_compact(cu, kv_len, base, cap, a, path, tk, tv, ck, cv, 1, 64, 256,
+                                   1, 8)
+    assert st == oracle.ENOSPACE and list(newlen) == [12, 8]
+    assert np.array_equal(ck[8:12], tk[0:4]) and np.array_equal(cv[8:12], tv[0:4])
+    touched = np.zeros(32, dtype=bool)
+    touched[8:12] = True
+    assert not ck[~touched].any() and not cv[~touched].any()
+
+
 # -------------------------------------------------------------------- low-rank candidate head
 def _bf16_bits(x):
     return oracle._u16(torch.as_tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16))
@@ -754,3 +825,37 @@ def test_lowrank_head_with_all_ids_is_the_exact_sort_and_permutes_with_the_vocab
     ids1, lg1, _, _ = oracle.lowrank_candidates(hid, D, U, W, 10)
     assert np.array_equal(perm[ids2], ids1)          # the same tokens, renamed
     assert np.allclose(lg1, lg2, rtol=0, atol=1e-12)
+
+
+def test_lowrank_screen_rounds_the_down_projection_to_bf16():
+    """U = I (r = V): the screen's logits are g = h D^T itself, which shows g's rounding to bf16.
+    Inputs are multiples of 1/8 in [-2, 2], so every product and sum (a multiple of 1/64, at most
+    256 in size) is exact in fp32 and torch's fp32 -> bf16 conversion rounds the exact g once.
+    D's rows repeat five distinct vectors, so each row's screen has groups of equal values and the
+    top-k cut falls inside one: the screen keeps the lowest ids of that group.  The k survivors
+    are then ordered by their exact logits h . W_c."""
+    g = np.random.default_rng(64)
+    M, H, V, k = 4, 64, 40, 6
+    hv = g.integers(-16, 17, size=(M, H)) / 8.0
+    dv = (g.integers(-16, 17, size=(5, H)) / 8.0)[g.integers(0, 5, size=V)]
+    hid, D = _bf16_bits(hv), _bf16_bits(dv)
+    U = _bf16_bits(np.eye(V))
+    Wv = g.normal(0, 0.3, size=(V, H)).astype(np.float32)
+    W = _bf16_bits(Wv)
+    ids, lg, kth, za = oracle.lowrank_candidates(hid, D, U, W, k, keep_approx=True)
+    exact = hv @ dv.T
+    want = torch.as_tensor(exact.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert not np.array_equal(want, exact)               # some screen logits do round
+    assert np.array_equal(za, want)
+    Wb = np.frombuffer((W.astype(np.uint32) << 16).tobytes(), np.float32).reshape(V, H)
+    zx = hv @ Wb.astype(np.float64).T
+    ties = 0
+    for m in range(M):
+        top = np.lexsort((np.arange(V), -want[m]))[:k]
+        ties += int(want[m, top[-1]] == want[m, np.lexsort((np.arange(V), -want[m]))[k]])
+        assert kth[m] == want[m, top[-1]]
+        assert sorted(ids[m]) == sorted(top)
+        order = sorted(top, key=lambda c: (-zx[m, c], c))
+        assert list(ids[m]) == order
+        assert np.allclose(lg[m], zx[m, order], rtol=0, atol=1e-12)
+    assert ties > 0                                      # the tie rule was exercised
