@@ -379,7 +379,8 @@ def cpu_baseline(wl, min_seconds=10.0, max_reps=5):
         toks += oracle_step(wl, reqs)
         reps += 1
     dt = time.perf_counter() - t0
-    return {"value": toks / dt, "unit": "tok/s", "cores": oracle.max_threads(), "kind": "oracle",
+    return {"value": toks / dt, "unit": "accepted tok/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
             "sample": f"{len(reqs)} of {wl.B} requests ({sum(wl.nodes(r) for r in reqs)} tree "
                       f"nodes) of workload {wl.name}, {reps} full oracle steps (attention all "
                       f"rows, LM head + acceptance, compaction), {dt:.1f} s"}
