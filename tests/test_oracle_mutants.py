@@ -193,3 +193,46 @@ def test_pins_catch_the_planted_mistake(name, old, new, pins, tmp_path, monkeypa
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"{name}: no pin failed"
+
+
+# The paged forms are numpy compositions in oracle/__init__.py: each case edits one function's
+# source text, rebinds the edited function in the oracle module and runs the paged pins.
+PY_MUTANTS = [
+    ("page_slots_offset_in_page_dropped", "page_slots",
+     "[r, t // page_size].astype(np.int64) * page_size + t % page_size",
+     "[r, t // page_size].astype(np.int64) * page_size",
+     [(P.test_page_slots_by_hand, ())]),
+    ("paged_attention_every_request_at_offset_zero", "attention_paged",
+     "        base[r] = off\n", "        base[r] = 0\n",
+     [(P.test_paged_attention_is_independent_of_page_placement, ())]),
+    ("paged_compaction_writes_from_position_zero", "kv_compact_paged",
+     "np.arange(L, L + a + 1))", "np.arange(0, a + 1))",
+     [(P.test_paged_compaction_equals_contiguous_compaction_of_the_logical_cache, ())]),
+    ("paged_compaction_source_ignores_request_offset", "kv_compact_paged",
+     "src = int(cu[r]) + pr", "src = pr",
+     [(P.test_paged_compaction_equals_contiguous_compaction_of_the_logical_cache, ())]),
+]
+
+
+def test_every_planted_python_spot_exists_once():
+    import inspect
+    for name, fn, old, new, _ in PY_MUTANTS:
+        assert inspect.getsource(getattr(oracle, fn)).count(old) == 1, name
+        assert old != new, name
+
+
+@pytest.mark.parametrize("name,fn,old,new,pins", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_pins_catch_the_planted_python_mistake(name, fn, old, new, pins, monkeypatch):
+    import inspect
+    src = inspect.getsource(getattr(oracle, fn))
+    assert src.count(old) == 1
+    scope = dict(vars(oracle))
+    exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), scope)
+    monkeypatch.setattr(oracle, fn, scope[fn])
+    caught = []
+    for pin, args in pins:
+        try:
+            pin(*args)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"{name}: no pin failed"
