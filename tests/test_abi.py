@@ -95,3 +95,116 @@ def test_product_path_does_not_import_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "liboracle" not in text, f
+
+
+ALIGNED_WS = C.c_void_p(0x100000)          # 256-byte aligned; never dereferenced: every call
+                                           # below fails a host check before any device work
+OTHER = C.c_void_p(0x200000)               # a second fake address (outputs that must not alias)
+
+
+def _rejects(status, code, words):
+    """The call failed with `code` and the host message names the failing check."""
+    msg = et.lib().etree_last_error()
+    assert status == code, (status, msg)
+    assert words.encode() in msg, msg
+
+
+def test_host_validation_of_the_paged_calls(L):
+    b = _batch()
+
+    def attn_paged(bt=FAKE, max_pages=4, page=16, num_pages=8, hq=8, hkv=2, head_dim=128):
+        return L.etree_verify_attn_paged(C.byref(b), bt, max_pages, page, FAKE, FAKE, FAKE, FAKE,
+                                         FAKE, num_pages, hq, hkv, head_dim, 0.1, FAKE, None,
+                                         ALIGNED_WS, 1 << 30, None)
+
+    _rejects(attn_paged(bt=None), -1, "block_table")
+    _rejects(attn_paged(bt=C.c_void_p(0x100002)), -1, "block_table")    # not 4-byte aligned
+    _rejects(attn_paged(max_pages=0), -1, "max_pages")
+    for page in (0, 8, 24, 1 << 21):                                     # power of 2, [16, 2^20]
+        _rejects(attn_paged(page=page), -1, "page_size")
+    _rejects(attn_paged(num_pages=0), -1, "num_pages")
+    _rejects(attn_paged(num_pages=1 << 27, page=16), -1, "num_pages")   # 2^31 pool slots
+    _rejects(attn_paged(head_dim=64), -2, "head_dim")
+
+    def compact_paged(page=16, num_pages=8, n_layers=1, cache_stride=0, head_dim=128,
+                      kv_len_out=OTHER):
+        return L.etree_kv_compact_paged(C.byref(b), FAKE, 4, page, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                        FAKE, num_pages, n_layers, 4 * 2 * 128, cache_stride, 2,
+                                        head_dim, kv_len_out, ALIGNED_WS, 1 << 30, None)
+
+    _rejects(compact_paged(page=12), -1, "page_size")
+    _rejects(compact_paged(num_pages=0), -1, "num_pages")
+    _rejects(compact_paged(head_dim=96), -2, "head_dim")
+    _rejects(compact_paged(n_layers=0), -1, "n_layers")
+    _rejects(compact_paged(kv_len_out=FAKE), -1, "aliases")
+    # two layers: the cache stride must cover a whole page pool (8 pages x 16 slots x 256)
+    _rejects(compact_paged(n_layers=2, cache_stride=8 * 16 * 256 - 8), -1, "page pool")
+
+
+def test_host_validation_of_the_tree_sampler_and_lm_head(L):
+    b = _batch()
+
+    def tree(zbuf=FAKE, rows=4, T=1.0, q=FAKE, hidden_dim=128):
+        return L.etree_lmhead_accept_tree(C.byref(b), FAKE, FAKE, hidden_dim, 1000, T, q, 0, 0,
+                                          FAKE, FAKE, FAKE, zbuf, rows, ALIGNED_WS, 1 << 30, None)
+
+    _rejects(tree(rows=-1), -1, "zbuf_rows")
+    _rejects(tree(zbuf=None, rows=2), -1, "zbuf_rows")
+    _rejects(tree(zbuf=C.c_void_p(0x100004)), -1, "zbuf must be 16-byte aligned")
+    _rejects(tree(q=None), -1, "q_draft")                                # T > 0 needs draft rows
+    for T in (float("nan"), -0.5, float("inf")):
+        _rejects(tree(T=T), -1, "temperature")
+    _rejects(tree(hidden_dim=96), -2, "hidden_dim")
+
+    def head(hidden=FAKE, vocab=1000, ws=ALIGNED_WS, ws_bytes=1 << 30):
+        return L.etree_lmhead_accept(C.byref(b), hidden, FAKE, 128, vocab, 0.0, None, 0, 0, FAKE,
+                                     FAKE, FAKE, None, None, ws, ws_bytes, None)
+
+    _rejects(head(vocab=0), -1, "vocab")
+    _rejects(head(hidden=None), -1, "NULL")
+    _rejects(head(hidden=C.c_void_p(0x100008)), -1, "aligned")          # not 16-byte aligned
+    _rejects(head(ws=None), -1, "workspace is NULL")
+    _rejects(head(ws_bytes=64), -1, "needs")
+
+
+def test_host_validation_of_the_attention_scalars(L):
+    _rejects(_attn(L, _batch(), hq=130, hkv=2), -1, "hq=130")           # > 64 heads per group
+    b = _batch()
+    for slots in (0, 1 << 31):
+        _rejects(L.etree_verify_attn(C.byref(b), FAKE, FAKE, FAKE, FAKE, FAKE, slots, 8, 2, 128,
+                                     0.1, FAKE, None, ALIGNED_WS, 1 << 30, None), -1,
+                 "cache_slots")
+    _rejects(L.etree_verify_attn(C.byref(b), FAKE, FAKE, FAKE, FAKE, FAKE, 100, 8, 2, 128,
+                                 float("nan"), FAKE, None, ALIGNED_WS, 1 << 30, None), -1,
+             "scale")
+    _rejects(L.etree_verify_attn_noalloc(C.byref(b), FAKE, FAKE, FAKE, FAKE, FAKE, 100, 6, 4, 128,
+                                         0.1, FAKE, None, None, None), -1, "hq=6")
+    _rejects(_attn(L, _batch(B=2, n_total=1)), -1, "n_total")           # fewer nodes than B
+
+
+def test_host_validation_of_the_low_rank_head(L):
+    def lowrank(hidden=FAKE, M=4, H=128, r=64, V=1000, k=8, ws=ALIGNED_WS, ws_bytes=1 << 30):
+        return L.etree_lowrank_candidates(hidden, M, H, FAKE, FAKE, r, FAKE, V, k, FAKE, FAKE,
+                                          ws, ws_bytes, None)
+
+    _rejects(lowrank(hidden=None), -1, "NULL")
+    _rejects(lowrank(M=0), -1, "M=0")
+    for H in (100, 8256):
+        _rejects(lowrank(H=H), -2, "hidden_dim")
+    for r in (32, 96):
+        _rejects(lowrank(r=r), -2, "rank")
+    for k, V in ((0, 1000), (17, 1000), (8, 4)):
+        _rejects(lowrank(k=k, V=V), -1, "k=")
+    _rejects(lowrank(hidden=C.c_void_p(0x100008)), -1, "aligned")
+    _rejects(lowrank(ws_bytes=16), -1, "needs")
+    assert L.etree_lowrank_workspace_size(0, 128, 64, 1000) == 0
+    assert 0 < L.etree_lowrank_workspace_size(4, 128, 64, 1000) < \
+        L.etree_lowrank_workspace_size(64, 128, 64, 1000)
+
+
+def test_host_validation_of_the_status_calls(L):
+    _rejects(L.etree_workspace_init(None, 1 << 20, None), -1, "workspace")
+    _rejects(L.etree_workspace_init(ALIGNED_WS, 16, None), -1, "workspace")
+    _rejects(L.etree_device_status(None, None, None), -1, "workspace")
+    for ws, n in ((None, 1 << 20), (C.c_void_p(0x100010), 1 << 20), (ALIGNED_WS, 16)):
+        _rejects(L.etree_selftest_timeout(ws, n, None), -1, "workspace")
