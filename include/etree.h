@@ -212,7 +212,8 @@ etree_status etree_lmhead_accept(const etree_batch *batch, const uint16_t *hidde
  *              because each sibling rejection needs a pass over the whole row.  At most
  *              floor((n_total - B) / 2) rows are ever needed.  A batch with more branching nodes
  *              than zbuf_rows records ETREE_ENOSPACE (detail 10) and the requests left without a
- *              row accept nothing: their bonus is drawn from the root's p (a one-token decode).  zbuf may be NULL when zbuf_rows == 0 (chains need no rows).
+ *              row accept nothing: their bonus is drawn from the root's p (a one-token
+ *              decode).  zbuf may be NULL when zbuf_rows == 0 (chains need no rows).
  *   Other arguments as in etree_lmhead_accept (no node_argmax / node_gap outputs).
  * Errors: host-side as etree_lmhead_accept, plus ETREE_EINVAL for zbuf_rows < 0, a NULL zbuf
  * with zbuf_rows > 0, or a misaligned zbuf.
