@@ -387,6 +387,15 @@ def cpu_baseline(wl, min_seconds=10.0, max_reps=5):
 
 
 # -------------------------------------------------------------------------------------- main
+def workload_config(name, wl, world):
+    """The workload keys both arms' JSON lines carry in `config`."""
+    return {"workload": name, "B": wl.B, "tree_nodes": int(wl.n_max),
+            "kv_len": int(wl.kv_len_max), "hidden": wl.hidden_dim, "vocab": wl.vocab,
+            "heads": f"{wl.hq}/{wl.hkv}", "head_dim": wl.head_dim,
+            "temperature": wl.temperature, "layers": 1,
+            "parallelism": f"dp{world} (independent requests per rank)"}
+
+
 def run_config(name, steps, warmup, peaks, rank, flush, with_e2e=True):
     from draft_tree_verification_masked_b200 import etree_attn_plan
     from draft_tree_verification_masked_b200 import workload as W
@@ -605,14 +614,10 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; random-init LM head, N(0,1) activations and KV)",
-        "config": {"workload": args.config, "B": wl.B, "tree_nodes": int(wl.n_max),
-                   "kv_len": int(wl.kv_len_max), "hidden": wl.hidden_dim, "vocab": wl.vocab,
-                   "heads": f"{wl.hq}/{wl.hkv}", "head_dim": wl.head_dim,
-                   "temperature": wl.temperature, "layers": 1,
+        "config": {**workload_config(args.config, wl, world),
                    "l2": "flushed before every timed step: 512 MiB write, then 256 MiB read "
                          "(dirty lines written back before the timed region)",
-                   "attn_plan": head_plan,
-                   "parallelism": f"dp{world} (independent requests per rank)"},
+                   "attn_plan": head_plan},
         "clocks": clk,
         "e2e": {"value": tokens_all / e2e_s, "unit": "accepted tok/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -650,7 +655,7 @@ def main_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.config, "B": wl.B, "sampled_requests": len(reqs)},
+        "config": {**workload_config(args.config, wl, world), "sampled_requests": len(reqs)},
         "cpu_baseline": {"value": value, "unit": "accepted tok/s", "cores": oracle.max_threads(),
                          "kind": "oracle",
                          "sample": f"{len(reqs)} of {wl.B} requests per step, full oracle "

@@ -1,5 +1,6 @@
-"""Host-side helpers of bench.py (no GPU): the source fingerprint that ties a committed ncu
-traffic figure to the kernel sources it was measured on."""
+"""Host-side parts of bench.py (no GPU): the source fingerprint that ties a committed ncu traffic
+figure to the kernel sources it was measured on, the packed step-input buffer, and the oracle
+(reference) arm's JSON line."""
 import os
 import sys
 
@@ -57,3 +58,35 @@ def test_packed_buffer_layout():
     # the tail from a tensor's offset holds it and everything after it
     tail = pk.buf[pk.offset("c"):]
     assert tail.numel() >= pk.view("c").numel() * 2 + pk.view("d").numel() * 4
+
+
+def _reference_arm(env_extra):
+    import json
+    import subprocess
+    env = dict(os.environ, **env_extra)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--config", "tiny", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, env=env, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_prints_one_contract_line():
+    """The oracle arm runs on host cores only: one JSON line with the main arm's metric, unit and
+    workload keys, an oracle cpu_baseline and an e2e block that moves no bytes."""
+    from draft_tree_verification_masked_b200 import workload as W
+    (line,) = _reference_arm({"RANK": "0", "WORLD_SIZE": "1"})
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "accepted tok/s" and line["higher_is_better"] is True
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["n_gpus"] == 1
+    assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    want = bench.workload_config("tiny", W.generate("tiny"), 1)
+    assert {k: line["config"][k] for k in want} == want
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    assert _reference_arm({"RANK": "1", "WORLD_SIZE": "2"}) == []
