@@ -208,3 +208,21 @@ def test_host_validation_of_the_status_calls(L):
     _rejects(L.etree_device_status(None, None, None), -1, "workspace")
     for ws, n in ((None, 1 << 20), (C.c_void_p(0x100010), 1 << 20), (ALIGNED_WS, 16)):
         _rejects(L.etree_selftest_timeout(ws, n, None), -1, "workspace")
+
+
+def test_binding_fails_loudly_without_the_library_or_on_host_memory(tmp_path, monkeypatch):
+    """No fallback: a missing library raises on first use, and host tensors are refused before
+    any call reaches the library."""
+    import torch
+    monkeypatch.setattr(et, "_LIB_PATH", str(tmp_path / "libetree.so"))
+    monkeypatch.setattr(et, "_lib", None)
+    with pytest.raises(et.EtreeError, match="missing"):
+        et.lib()
+    with pytest.raises(et.EtreeError):
+        et.etree_version()
+    monkeypatch.undo()
+    host = torch.zeros(4, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA device"):
+        et.make_batch(host, host, host, host, host.long(), host, 4, 0)
+    with pytest.raises(ValueError, match="CUDA device"):
+        et.etree_workspace_init(torch.zeros(1024, dtype=torch.uint8))
