@@ -476,6 +476,12 @@ def compact_layers_report(dev, wl, flush, peaks, layers=64):
             "bytes": nbytes}
 
 
+# Nominal B200 figures (HBM3e 7.7 TB/s, dense bf16 2.25 PFLOP/s), reported beside the measured
+# ones for context; the roofline object uses the measured peaks.
+NOMINAL_HBM_GBS = 7700.0
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
 def kernel_report(wl, t, acc, peaks):
     hbm = float(peaks["hbm_gbs"])
     tc = float(peaks["bf16_tflops"])
@@ -495,6 +501,10 @@ def kernel_report(wl, t, acc, peaks):
         "compact": {"us": cm * 1e6, "GB/s": cb / cm / 1e9, "hbm_frac": cb / cm / 1e9 / hbm,
                     "bytes": cb},
     }
+    for k in rep.values():
+        k["hbm_frac_nominal"] = k["GB/s"] / NOMINAL_HBM_GBS
+        if "TFLOP/s" in k:
+            k["tc_frac_nominal"] = k["TFLOP/s"] / NOMINAL_BF16_TFLOPS
     return rep
 
 

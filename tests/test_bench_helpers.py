@@ -90,3 +90,31 @@ def test_reference_arm_prints_one_contract_line():
 
 def test_reference_arm_runs_on_rank_zero_only():
     assert _reference_arm({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_algorithmic_work_matches_the_per_unit_figures():
+    """The roofline numerators: attention reads the KV cache once (2 L Hkv D 2 bytes) plus the
+    tree K/V, Q and O, and does 4 Hq D FLOPs per (query node, visible key); the LM head reads W
+    once and does 2 N V H FLOPs; compaction reads and writes (a + 1) K and V rows per layer."""
+    from types import SimpleNamespace
+
+    import numpy as np
+    from draft_tree_verification_masked_b200 import workload as W
+
+    wl = W.generate("dense27b_b1", hidden=64, vocab=256)
+    L, Hkv, Hq, D, N = 4096, 8, 40, 128, 64
+    b, f = bench.attn_work(wl)
+    assert b == 2 * L * Hkv * D * 2 + 2 * N * Hkv * D * 2 + 2 * N * Hq * D * 2
+    # visible tree keys = sum over nodes of their subtree sizes (pairs ancestor-or-self, node)
+    size = np.ones(N, dtype=np.int64)
+    for i in range(N - 1, 0, -1):
+        size[wl.parent[i]] += size[i]
+    assert f == 4 * Hq * D * (N * L + int(size.sum()))
+    assert abs(f / 5.37e9 - 1) < 0.01                         # 5.37 GFLOP at this shape
+    head = SimpleNamespace(vocab=151936, hidden_dim=5120, n_total=64)
+    hb, hf = bench.lmhead_work(head)
+    assert hb == 151936 * 5120 * 2 + 64 * 5120 * 2 and abs(hb / 1.556e9 - 1) < 0.001
+    assert hf == 2 * 64 * 151936 * 5120
+    kv = SimpleNamespace(hkv=8, head_dim=128)
+    assert bench.compact_work(kv, np.array([3, 0])) == 2 * 2 * (4 + 1) * 8 * 128 * 2
+    assert bench.compact_work(kv, np.array([3, 0]), n_layers=64) == 64 * 2 * 2 * 5 * 8 * 128 * 2
