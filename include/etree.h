@@ -336,7 +336,20 @@ etree_status etree_plan_tree(const etree_cost_table *table, int32_t B, int32_t L
 /*
  * Synchronizes `stream`, reads the workspace status word (the first device-detected error since
  * the last read, ETREE_OK if none), stores its detail code in *detail (if not NULL) and clears
- * both words.
+ * both words.  Detail codes:
+ *    0  none
+ *    1  bad parent: parent[0] != -1 or parent[i] outside [0, i)
+ *    2  bad node count: a request with 0 or more than n_max nodes
+ *    3  bad kv_len: negative, above kv_len_max, or past the cache pool
+ *    4  capacity: kv_len + accepted + 1 > slot_cap
+ *    5  not a chain: T > 0 on a node with more than one child (etree_lmhead_accept)
+ *    6  bad path: path or accept_len out of range in compaction
+ *    7  attention wait: a bounded wait gave up in attention
+ *    8  gemm wait: a bounded wait gave up in the LM-head GEMM
+ *    9  bad token: a token id outside [0, vocab)
+ *   10  logit rows: more branching nodes than zbuf rows (etree_lmhead_accept_tree)
+ *   11  bad page: a block-table entry outside [0, num_pages) for a used position
+ *   12  self-test wait: etree_selftest_timeout's deliberately unfinished wait gave up
  */
 etree_status etree_device_status(void *workspace, void *stream, int32_t *detail);
 

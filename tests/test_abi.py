@@ -226,3 +226,19 @@ def test_binding_fails_loudly_without_the_library_or_on_host_memory(tmp_path, mo
         et.make_batch(host, host, host, host, host.long(), host, 4, 0)
     with pytest.raises(ValueError, match="CUDA device"):
         et.etree_workspace_init(torch.zeros(1024, dtype=torch.uint8))
+
+
+def test_status_and_detail_codes_agree_across_header_kernels_and_binding():
+    """The detail codes the header documents, the kernels' enum and the binding's names list the
+    same numbers in the same order; likewise the status codes."""
+    hdr = open(os.path.join(ROOT, "include", "etree.h")).read()
+    cuh = open(os.path.join(ROOT, "draft_tree_verification_masked_b200", "csrc",
+                            "common.cuh")).read()
+    det_enum = {int(v): k for k, v in re.findall(r"\b(DET_[A-Z_]+)\s*=\s*(\d+)", cuh)}
+    block = hdr[hdr.index("Detail codes:"):hdr.index("etree_device_status(void")]
+    det_hdr = {int(n): w.strip() for n, w in re.findall(r"\*\s+(\d+)\s+([a-z_ -]+?)(?::|\n)",
+                                                         block)}
+    assert sorted(det_enum) == sorted(det_hdr) == sorted(et.DETAIL) == list(range(len(et.DETAIL)))
+    assert det_hdr == et.DETAIL
+    st_hdr = {int(v): k for k, v in re.findall(r"\b(ETREE_[A-Z]+)\s*=\s*(-?\d+)", hdr)}
+    assert st_hdr == {k: v for k, v in et.STATUS.items()}
