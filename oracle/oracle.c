@@ -292,8 +292,9 @@ void oracle_philox4x64(const uint64_t ctr[4], const uint64_t key[2], uint64_t ou
  * under key (seed, step)) gives 4 words of 64 bits; each word holds two 23-bit fields, bits
  * 63..41 and bits 31..9.  Vocab id v takes word (v/2) % 4, the high field for even v and the
  * low field for odd v, centred: U = (field + 0.5) * 2^-23, a value that single precision holds
- * exactly and that lies in [2^-24, 1 - 2^-24].  stream 0 feeds the bonus/residual race
- * (v = vocab id), stream 1 the accept tests (v = 0, node = the child). */
+ * exactly and that lies in [2^-24, 1 - 2^-24].  Streams: 1 the accept tests (v = 0, node = the
+ * child); 2 the draw's block race and 3 its inverse CDF (v = block); 0 the flat race over vocab
+ * ids that oracle_race keeps as a reference sampler. */
 double oracle_uniform(uint64_t seed, uint64_t step, uint32_t r, uint32_t node, uint32_t v,
                       uint32_t stream) {
     uint64_t ctr[4] = {v >> 3, node, r, stream};
