@@ -146,6 +146,19 @@ MUTANTS = [
      "size_t src = (size_t)l * tree_layer_stride + (size_t)(cu_nodes[r] + j) * row;",
      "size_t src = (size_t)l * tree_layer_stride + (size_t)(cu_nodes[r] + k) * row;",
      [(P.test_kv_compact_equals_numpy_gather, ())]),
+    ("compact_first_layer_only",
+     "        for (int l = 0; l < n_layers; ++l)\n", "        for (int l = 0; l < 1; ++l)\n",
+     [(P.test_kv_compact_equals_numpy_gather, ())]),
+    ("greedy_accepts_any_child",
+     "if (parent[c] == u && tokens[c] == want) { next = c; break; }",
+     "if (parent[c] == u) { next = c; break; }",
+     [(P.test_greedy_walk_equals_sequential_greedy_decoding, (s,)) for s in range(12)]),
+    ("tree_keeps_testing_siblings_after_an_accept",
+     "                next = j;\n                break;", "                next = j;",
+     [(P.test_multi_candidate_sibling_acceptance_rates_match_the_closed_form, ())]),
+    ("attention_last_tree_key_left_out_of_the_sum",
+     "for (long t = 0; t < nkeys; ++t) {", "for (long t = 0; t < nkeys - 1; ++t) {",
+     [(P.test_chain_tree_equals_causal_attention, ())]),
     # bf16 rounding and the low-rank head
     ("bf16_ties_away_from_zero",
      "else r = fmod(lo / ulp, 2.0) == 0.0 ? lo : hi;", "else r = hi;",
@@ -156,6 +169,9 @@ MUTANTS = [
     ("lowrank_screen_ties_to_highest_id",
      "if (!taken[v] && (best < 0 || z[v] > z[best])) best = v;",
      "if (!taken[v] && (best < 0 || z[v] >= z[best])) best = v;",
+     [(P.test_lowrank_screen_rounds_the_down_projection_to_bf16, ())]),
+    ("lowrank_kth_is_the_best_screen_value",
+     "if (kth) kth[m] = z[cand[k - 1]];", "if (kth) kth[m] = z[cand[0]];",
      [(P.test_lowrank_screen_rounds_the_down_projection_to_bf16, ())]),
     ("lowrank_exact_order_ascending",
      "while (j >= 0 && (ex[j] < xi || (ex[j] == xi && cand[j] > ci))) {",
