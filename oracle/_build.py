@@ -1,7 +1,7 @@
 """Compile the fp64 CPU oracle (plain C, gcc, OpenMP) into oracle/liboracle.so.
 
-The oracle is test infrastructure: building it is part of the build, using it is reserved to the
-tests, the smoke check and the benchmark's CPU-baseline leg.
+The oracle is test infrastructure: it is compiled with the package, and only the tests, the smoke
+check and the benchmark's CPU-baseline leg use it.
 """
 import os
 import subprocess
