@@ -80,11 +80,6 @@ def _bind(path: str):
     L.oracle_race_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
                                    C.c_int, I32P, C.c_int]
     L.oracle_race_many.restype = None
-    L.oracle_draw.argtypes = [C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int, C.c_int, I32P]
-    L.oracle_draw.restype = C.c_int
-    L.oracle_draw_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
-                                   C.c_int, I32P, C.c_int]
-    L.oracle_draw_many.restype = None
     return L
 
 
@@ -256,21 +251,6 @@ def accept_tree_batch(cu_nodes, parent, tokens, z, q, T, seed, step, nthreads=0)
     return a, path, out, info, c
 
 
-def draw(w, seed, step, r, node):
-    """The acceptance rule's two-level draw; returns (token, block, fell_to_last)."""
-    w = np.ascontiguousarray(w, dtype=np.float64)
-    info = np.zeros(2, dtype=np.int32)
-    tok = lib().oracle_draw(len(w), w, seed, step, r, node, info)
-    return tok, int(info[0]), int(info[1])
-
-
-def draw_many(w, n, seed, step, r0, node, nthreads=0):
-    w = np.ascontiguousarray(w, dtype=np.float64)
-    out = np.empty(n, dtype=np.int32)
-    lib().oracle_draw_many(n, len(w), w, seed, step, r0, node, out, int(nthreads))
-    return out
-
-
 def race_many(w, n, seed, step, r0, node, nthreads=0):
     w = np.ascontiguousarray(w, dtype=np.float64)
     out = np.empty(n, dtype=np.int32)
@@ -409,6 +389,58 @@ def lmhead_accept(wl, requests=None, nthreads=0, keep_logits=False):
             res[r] = dict(accept_len=a, path=path, out_tokens=out, info=info, c=c,
                           z=z if keep_logits else None)
     return res
+
+
+def lmhead_accept_many(wl, requests=None, nthreads=0, keep_logits=False, chunk_rows=512):
+    """lmhead_accept for many requests at once: the logits of up to chunk_rows node rows come
+    from one oracle_logits call (one pass over the head per chunk instead of one per request);
+    the per-request definitions that follow are the same calls as in lmhead_accept."""
+    reqs = list(range(wl.B) if requests is None else requests)
+    res = {}
+    i = 0
+    while i < len(reqs):
+        group, nrow = [], 0
+        while i < len(reqs) and (not group or nrow + wl.nodes(reqs[i]) <= chunk_rows):
+            group.append(reqs[i])
+            nrow += wl.nodes(reqs[i])
+            i += 1
+        rows = np.concatenate([np.arange(int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1]),
+                                         dtype=np.int32) for r in group])
+        zall = logits(wl.hidden, wl.w_lm, rows, nthreads)
+        off = 0
+        for r in group:
+            a0, a1 = int(wl.cu_nodes[r]), int(wl.cu_nodes[r + 1])
+            z = zall[off:off + a1 - a0]
+            off += a1 - a0
+            par = wl.parent[a0:a1]
+            tok = wl.tokens[a0:a1]
+            if wl.temperature == 0.0:
+                arg, t1, t2 = row_top2(z)
+                a, path, out = walk_greedy(par, tok, arg)
+                res[r] = dict(accept_len=a, path=path, out_tokens=out, argmax=arg, top1=t1,
+                              top2=t2)
+            else:
+                qd = wl.q_draft[a0:a1].numpy()
+                if np.array_equal(par, np.arange(-1, a1 - a0 - 1)):
+                    a, path, out, info = accept_chain(par, tok, z, qd, wl.temperature, wl.seed,
+                                                      wl.step, r)
+                    c = 1.0 if info[1] else 0.0
+                else:
+                    a, path, out, info, c = accept_tree(par, tok, z, qd, wl.temperature,
+                                                        wl.seed, wl.step, r)
+                res[r] = dict(accept_len=a, path=path, out_tokens=out, info=info, c=c,
+                              z=z.copy() if keep_logits else None)
+    return res
+
+
+def row_argmax(hidden, w, nthreads=0, chunk_rows=512):
+    """Each hidden row's argmax of hidden . w^T (fp64, lowest id on ties)."""
+    n = int(hidden.shape[0])
+    out = np.empty(n, dtype=np.int32)
+    for i in range(0, n, chunk_rows):
+        rows = np.arange(i, min(n, i + chunk_rows), dtype=np.int32)
+        out[i:i + len(rows)] = row_top2(logits(hidden, w, rows, nthreads))[0]
+    return out
 
 
 def scale_of(head_dim: int) -> float:

@@ -13,15 +13,18 @@
  * tree lets one verification cover several candidate paths).  All floating point is fp64 on the
  * exact bf16/fp32 input values; the only library routines are exp and log from libm.
  *
- * Readings taken where the pages are silent (each is listed in the design notes):
+ * Readings taken where the pages are silent:
  *  - node 0 of a request is the root (the last committed token); its K/V are produced by this pass
  *    and are not yet in the cache;
  *  - attention has no positional term, soft-cap or window: q and k arrive ready to dot;
  *  - greedy: argmax ties go to the lowest vocab id; among children carrying the argmax token the
  *    lowest node index is taken;
  *  - T>0 on chains: node k's token was drafted from q of node k-1; accept iff U*q < p (strict);
- *    the bonus/residual token is drawn in two levels with Philox4x64-10 uniforms: an exponential
- *    race among 128-id block totals, then an inverse CDF inside the winning block (oracle_draw);
+ *    the bonus/residual token is drawn by an exponential race over all vocab ids with
+ *    Philox4x64-10 uniforms (oracle_race), an exact sampler of the normalised weights;
+ *  - a residual with no positive weight (p <= q everywhere, which in exact arithmetic means
+ *    p = q, where the rejected draft would have been accepted with probability 1) draws the
+ *    bonus from p itself, so the emitted token still follows the target's distribution;
  *  - T>0 on branching trees (the pages give no rule): siblings are candidates drafted
  *    independently from their parent's q and are tested in index order by multi-candidate
  *    speculative sampling, each rejection replacing the target by its normalised residual
@@ -292,9 +295,8 @@ void oracle_philox4x64(const uint64_t ctr[4], const uint64_t key[2], uint64_t ou
  * under key (seed, step)) gives 4 words of 64 bits; each word holds two 23-bit fields, bits
  * 63..41 and bits 31..9.  Vocab id v takes word (v/2) % 4, the high field for even v and the
  * low field for odd v, centred: U = (field + 0.5) * 2^-23, a value that single precision holds
- * exactly and that lies in [2^-24, 1 - 2^-24].  Streams: 1 the accept tests (v = 0, node = the
- * child); 2 the draw's block race and 3 its inverse CDF (v = block); 0 the flat race over vocab
- * ids that oracle_race keeps as a reference sampler. */
+ * exactly and that lies in [2^-24, 1 - 2^-24].  Streams: 0 the bonus draw's race over vocab ids
+ * (node = the stop node), 1 the accept tests (v = 0, node = the child). */
 double oracle_uniform(uint64_t seed, uint64_t step, uint32_t r, uint32_t node, uint32_t v,
                       uint32_t stream) {
     uint64_t ctr[4] = {v >> 3, node, r, stream};
@@ -306,10 +308,13 @@ double oracle_uniform(uint64_t seed, uint64_t step, uint32_t r, uint32_t node, u
     return ((double)field + 0.5) * (1.0 / 8388608.0);
 }
 
-/* Exponential race over weights w (>= 0): the winner is argmax over w_v > 0 of
- * log w_v - log(-log U_v), ties to the lowest v.  P(winner = v) = w_v / sum w exactly.
- * Returns the token, or -1 when no weight is positive.  *best_key receives the winning key.
- * (Kept as a reference sampler for the tests; the acceptance rule uses oracle_draw below.) */
+/* The bonus draw: an exponential race over weights w (>= 0).  Every id with w_v > 0 gets the
+ * key log w_v - log(-log U_v), U_v = oracle_uniform(seed, step, r, node, v, 0); the winner is the
+ * largest key, ties to the lowest v.  -log U_v is a standard exponential E_v, and the id with
+ * the smallest E_v / w_v is id v with probability w_v / sum w exactly (the minimum of
+ * independent exponentials of rates w_v), so the race samples the normalised weights without
+ * forming them.  Returns the token, or -1 when no weight is positive; *best_key (nullable)
+ * receives the winning key. */
 int oracle_race(int V, const double *w, uint64_t seed, uint64_t step, int r, int node,
                 double *best_key) {
     int best = -1;
@@ -322,44 +327,6 @@ int oracle_race(int V, const double *w, uint64_t seed, uint64_t step, int r, int
     }
     if (best_key) *best_key = bk;
     return best;
-}
-
-/* The method's draw from weights w (>= 0) in two levels, an exact sampler of w / sum w:
- *  1. vocab ids form blocks of 128 consecutive ids (b = v / 128); block totals
- *     W_b = sum_{v in b} w_v (summed in increasing v) race: b* = argmax_{W_b > 0} of
- *     log W_b - log(-log U_b) with U_b = oracle_uniform(seed, step, r, node, b, 2), ties to the
- *     lowest b;
- *  2. inside b*, an inverse CDF with u = oracle_uniform(seed, step, r, node, b*, 3): the first
- *     v (in increasing order) whose running sum exceeds u * W_b*; if rounding leaves none, the
- *     last v of b* with w_v > 0.
- * Returns the token, or -1 when no weight is positive; info (nullable) gets {b*, 0}. */
-int oracle_draw(int V, const double *w, uint64_t seed, uint64_t step, int r, int node,
-                int32_t *info) {
-    const int nb = (V + 127) / 128;
-    int bstar = -1;
-    double bk = -INFINITY, Wstar = 0.0;
-    for (int b = 0; b < nb; ++b) {
-        double W = 0.0;
-        for (int v = b * 128; v < V && v < b * 128 + 128; ++v) W += w[v];
-        if (!(W > 0.0)) continue;
-        double U = oracle_uniform(seed, step, (uint32_t)r, (uint32_t)node, (uint32_t)b, 2);
-        double key = log(W) - log(-log(U));
-        if (bstar < 0 || key > bk) { bk = key; bstar = b; Wstar = W; }
-    }
-    if (bstar < 0) return -1;
-    double u = oracle_uniform(seed, step, (uint32_t)r, (uint32_t)node, (uint32_t)bstar, 3);
-    double thr = u * Wstar, run = 0.0;
-    int last = -1;
-    for (int v = bstar * 128; v < V && v < bstar * 128 + 128; ++v) {
-        run += w[v];
-        if (w[v] > 0.0) last = v;
-        if (run > thr) {
-            if (info) { info[0] = bstar; info[1] = 0; }
-            return v;
-        }
-    }
-    if (info) { info[0] = bstar; info[1] = 1; }
-    return last;
 }
 
 /* p = softmax(z / T) of one row, in fp64. */
@@ -378,8 +345,9 @@ static void softmax_t(int V, const double *z, double T, double *p) {
  * p_u = softmax(z_u / T).  Walk k = 1, 2, ...: accept x_k iff U_k * q_{k-1}(x_k) < p_{k-1}(x_k)
  * (U_k = oracle_uniform(seed, step, r, k, 0, 1)).  At the first rejection (stop node u = k-1) the
  * bonus is drawn from norm(max(0, p_u - q_u)); when every node is accepted (u = n-1) it is drawn
- * from p_u.  Both draws use oracle_draw at node u.  If the residual has no positive weight
- * (p <= q everywhere, which only rounding can produce) the bonus is the argmax of p_u.
+ * from p_u.  Both draws are oracle_race at node u.  If the residual has no positive weight
+ * (p <= q everywhere, i.e. p = q up to rounding, where exact arithmetic would have accepted the
+ * draft) the bonus is drawn from p_u by the same race.
  * z and q are the request's rows [n][V] (q fp32 as given).  info (nullable) receives
  * {stop node, 1 if a rejection happened else 0, 1 if the residual fell back to p}.
  * Returns a, OR_EINVAL for a malformed tree or OR_EUNSUPPORTED for a tree that is not a chain.
@@ -420,17 +388,15 @@ int oracle_accept_chain(int n, const int32_t *parent, const int32_t *tokens, con
             double d = p[v] - (double)q[(size_t)u * V + v];
             w[v] = d > 0.0 ? d : 0.0;
         }
-        bonus = oracle_draw(V, w, seed, step, r, u, NULL);
+        bonus = oracle_race(V, w, seed, step, r, u, NULL);
         if (bonus < 0) {
             /* no positive residual weight: p <= q everywhere, i.e. p = q up to rounding; the
-             * bonus is then the mode of p (lowest id on ties) */
+             * bonus is drawn from p, the distribution exact arithmetic would have emitted */
             fell_back = 1;
-            bonus = 0;
-            for (int v = 1; v < V; ++v)
-                if (p[v] > p[bonus]) bonus = v;
+            bonus = oracle_race(V, p, seed, step, r, u, NULL);
         }
     } else {
-        bonus = oracle_draw(V, p, seed, step, r, u, NULL);
+        bonus = oracle_race(V, p, seed, step, r, u, NULL);
     }
     out_tokens[a] = bonus;
     if (info) { info[0] = u; info[1] = rejected; info[2] = fell_back; }
@@ -558,10 +524,10 @@ void oracle_lowrank_candidates(int M, int H, int V, int r, int k, const uint16_t
  * from the current residual, so the emitted token follows p_u.
  *
  * The walk stops at a node with no children or whose children are all rejected; the bonus is
- * then drawn with oracle_draw at that node from the weights max(0, p_u - c q_u) (c = 0 when no
- * child was rejected: the weights are p_u).  If a rejection leaves N(c) = 0 (r = q up to
- * rounding; probability zero in exact arithmetic) the walk stops there and the bonus is the
- * argmax of p_u, lowest id on ties -- the chain rule's fallback.  On a chain this is exactly
+ * then drawn with oracle_race at that node from the weights max(0, p_u - c q_u) (c = 0 when no
+ * child was rejected: the weights are p_u).  If a rejection leaves N(c) = 0 (the running target
+ * equalled q up to rounding; probability zero in exact arithmetic) the walk stops there and the
+ * bonus is drawn from p_u by the same race, as in the chain rule.  On a chain this is exactly
  * oracle_accept_chain (c = 1 after the single rejection).
  *
  * z and q are the request's rows [n][V].  info (nullable): {stop node, rejections at the stop
@@ -623,14 +589,10 @@ int oracle_accept_tree(int n, const int32_t *parent, const int32_t *tokens, cons
             const double d = p[v] - c * (double)qu[v];
             w[v] = d > 0.0 ? d : 0.0;
         }
-        bonus = oracle_draw(V, w, seed, step, r, u, NULL);
+        bonus = oracle_race(V, w, seed, step, r, u, NULL);
         if (bonus < 0) fell_back = 1;
     }
-    if (fell_back) {
-        bonus = 0;
-        for (int v = 1; v < V; ++v)
-            if (p[v] > p[bonus]) bonus = v;
-    }
+    if (fell_back) bonus = oracle_race(V, p, seed, step, r, u, NULL);
     out_tokens[a] = bonus;
     if (info) { info[0] = u; info[1] = nrej; info[2] = fell_back; }
     if (c_out) *c_out = c;
@@ -725,12 +687,4 @@ void oracle_race_many(int n, int V, const double *w, uint64_t seed, uint64_t ste
     set_threads(nthreads);
 #pragma omp parallel for schedule(static)
     for (int k = 0; k < n; ++k) out[k] = oracle_race(V, w, seed, step, r0 + k, node, NULL);
-}
-
-/* n two-level draws over the same weights, draw k using request index r0 + k. */
-void oracle_draw_many(int n, int V, const double *w, uint64_t seed, uint64_t step, int r0,
-                      int node, int32_t *out, int nthreads) {
-    set_threads(nthreads);
-#pragma omp parallel for schedule(static)
-    for (int k = 0; k < n; ++k) out[k] = oracle_draw(V, w, seed, step, r0 + k, node, NULL);
 }

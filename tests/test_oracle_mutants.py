@@ -92,14 +92,18 @@ MUTANTS = [
     ("race_gumbel_sign",
      "double key = log(w[v]) - log(-log(U));", "double key = log(w[v]) + log(-log(U));",
      [(P.test_exponential_race_is_an_exact_sampler, ())]),
-    ("draw_block_total_not_summed",
-     "for (int v = b * 128; v < V && v < b * 128 + 128; ++v) W += w[v];",
-     "for (int v = b * 128; v < V && v < b * 128 + 128; ++v) W = w[v];",
-     [(P.test_two_level_draw_is_an_exact_sampler, (300,))]),
-    ("draw_inverse_cdf_reuses_the_race_stream",
-     "oracle_uniform(seed, step, (uint32_t)r, (uint32_t)node, (uint32_t)bstar, 3);",
-     "oracle_uniform(seed, step, (uint32_t)r, (uint32_t)node, (uint32_t)bstar, 2);",
-     [(P.test_two_level_draw_blocks_and_inverse_cdf_by_hand, ())]),
+    ("race_ignores_the_weights",
+     "double key = log(w[v]) - log(-log(U));", "double key = -log(-log(U));",
+     [(P.test_exponential_race_is_an_exact_sampler, ())]),
+    ("chain_fallback_takes_the_mode_of_p",
+     "            fell_back = 1;\n            bonus = oracle_race(V, p, seed, step, r, u, NULL);",
+     "            fell_back = 1;\n            bonus = 0;\n"
+     "            for (int v = 1; v < V; ++v) if (p[v] > p[bonus]) bonus = v;",
+     [(P.test_empty_residual_draws_the_bonus_from_the_target, ())]),
+    ("tree_fallback_returns_a_fixed_token",
+     "    if (fell_back) bonus = oracle_race(V, p, seed, step, r, u, NULL);",
+     "    if (fell_back) bonus = 0;",
+     [(P.test_empty_residual_draws_the_bonus_from_the_target, ())]),
     # stochastic acceptance on chains
     ("chain_test_p_and_q_swapped",
      "if (U * qx < p[x]) {", "if (U * p[x] < qx) {",
