@@ -75,7 +75,7 @@ def _bind(path: str):
     L.oracle_bf16_round.restype = C.c_uint16
     L.oracle_lowrank_candidates.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                             U16P, U16P, U16P, U16P, I32P, F64P, C.c_void_p,
-                                            C.c_void_p, C.c_int]
+                                            C.c_void_p, C.c_void_p, C.c_int]
     L.oracle_lowrank_candidates.restype = None
     L.oracle_race_many.argtypes = [C.c_int, C.c_int, F64P, C.c_uint64, C.c_uint64, C.c_int,
                                    C.c_int, I32P, C.c_int]
@@ -278,9 +278,10 @@ def bf16_round(x) -> int:
     return int(lib().oracle_bf16_round(float(x)))
 
 
-def lowrank_candidates(hidden, D, U, W, k, keep_approx=False, nthreads=0):
+def lowrank_candidates(hidden, D, U, W, k, keep_approx=False, nthreads=0, keep_g=False):
     """The low-rank candidate head over the rows of `hidden`: returns (ids [M,k], exact logits
-    [M,k], k-th approximate logit [M], approximate logits [M,V] or None)."""
+    [M,k], k-th approximate logit [M], approximate logits [M,V] or None), plus the down
+    projection g [M,r] when keep_g."""
     h, d, u, w = _u16(hidden), _u16(D), _u16(U), _u16(W)
     M, H = h.shape
     r, V = d.shape[0], u.shape[0]
@@ -288,11 +289,15 @@ def lowrank_candidates(hidden, D, U, W, k, keep_approx=False, nthreads=0):
     lg = np.empty((M, k), dtype=np.float64)
     kth = np.empty(M, dtype=np.float64)
     za = np.empty((M, V), dtype=np.float64) if keep_approx else None
+    g = np.empty((M, r), dtype=np.float64) if keep_g else None
     lib().oracle_lowrank_candidates(M, H, V, r, k, h.reshape(-1), d.reshape(-1), u.reshape(-1),
                                     w.reshape(-1), ids.reshape(-1), lg.reshape(-1),
                                     kth.ctypes.data_as(C.c_void_p),
                                     za.ctypes.data_as(C.c_void_p) if keep_approx else None,
+                                    g.ctypes.data_as(C.c_void_p) if keep_g else None,
                                     int(nthreads))
+    if keep_g:
+        return ids, lg, kth, za, g
     return ids, lg, kth, za
 
 

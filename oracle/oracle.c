@@ -435,18 +435,18 @@ uint16_t oracle_bf16_round(double x) {
  * aiposthub.com, section "EAGLE-4 是什麼？先看推測解碼為什麼能變快": a small matrix screens
  * candidate tokens, then only the few candidates are scored exactly).  For each of M rows h
  * (bf16, [M][H]):
- *   g = h D^T                  D [r][H] bf16; g rounded to bf16 (the precision of the second
- *                              product's operand);
+ *   g = h D^T                  D [r][H] bf16: the down projection;
  *   z~ = g U^T                 U [V][r] bf16: approximate logits;
  *   C = the k ids of largest z~ (ties to the lowest id);
  *   z_c = h . W_c for c in C   W [V][H] bf16: exact logits of the candidates;
  * out_ids [M][k]: C ordered by z_c descending (ties to the lowest id), out_logit [M][k] the z_c;
- * kth [M] (nullable): the k-th largest z~; z_approx [M][V] (nullable): z~.  fp64 throughout.
+ * kth [M] (nullable): the k-th largest z~; z_approx [M][V] (nullable): z~; g_out [M][r]
+ * (nullable): g.  fp64 throughout, on the exact bf16 input values.
  * ------------------------------------------------------------------------------------------- */
 void oracle_lowrank_candidates(int M, int H, int V, int r, int k, const uint16_t *hid,
                                const uint16_t *D, const uint16_t *U, const uint16_t *W,
                                int32_t *out_ids, double *out_logit, double *kth,
-                               double *z_approx, int nthreads) {
+                               double *z_approx, double *g_out, int nthreads) {
     set_threads(nthreads);
     double *g = (double *)malloc(sizeof(double) * (size_t)M * r);
 #pragma omp parallel for schedule(static)
@@ -455,8 +455,9 @@ void oracle_lowrank_candidates(int M, int H, int V, int r, int k, const uint16_t
         double acc = 0.0;
         for (int h = 0; h < H; ++h)
             acc += bf16_value(hid[(size_t)m * H + h]) * bf16_value(D[(size_t)j * H + h]);
-        g[t] = bf16_value(oracle_bf16_round(acc));
+        g[t] = acc;
     }
+    if (g_out) memcpy(g_out, g, sizeof(double) * (size_t)M * r);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int m = 0; m < M; ++m) {
         double *z = (double *)malloc(sizeof(double) * (size_t)V);

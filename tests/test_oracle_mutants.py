@@ -167,16 +167,16 @@ MUTANTS = [
     ("bf16_ties_away_from_zero",
      "else r = fmod(lo / ulp, 2.0) == 0.0 ? lo : hi;", "else r = hi;",
      [(P.test_bf16_rounding_is_nearest_even, ())]),
-    ("lowrank_down_projection_not_rounded",
-     "g[t] = bf16_value(oracle_bf16_round(acc));", "g[t] = acc;",
-     [(P.test_lowrank_screen_rounds_the_down_projection_to_bf16, ())]),
+    ("lowrank_down_projection_rounded_to_bf16",
+     "        g[t] = acc;\n", "        g[t] = bf16_value(oracle_bf16_round(acc));\n",
+     [(P.test_lowrank_screen_is_the_factorised_product, ())]),
     ("lowrank_screen_ties_to_highest_id",
      "if (!taken[v] && (best < 0 || z[v] > z[best])) best = v;",
      "if (!taken[v] && (best < 0 || z[v] >= z[best])) best = v;",
-     [(P.test_lowrank_screen_rounds_the_down_projection_to_bf16, ())]),
+     [(P.test_lowrank_screen_is_the_factorised_product, ())]),
     ("lowrank_kth_is_the_best_screen_value",
      "if (kth) kth[m] = z[cand[k - 1]];", "if (kth) kth[m] = z[cand[0]];",
-     [(P.test_lowrank_screen_rounds_the_down_projection_to_bf16, ())]),
+     [(P.test_lowrank_screen_is_the_factorised_product, ())]),
     ("lowrank_exact_order_ascending",
      "while (j >= 0 && (ex[j] < xi || (ex[j] == xi && cand[j] > ci))) {",
      "while (j >= 0 && (ex[j] > xi || (ex[j] == xi && cand[j] > ci))) {",

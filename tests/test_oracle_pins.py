@@ -873,13 +873,13 @@ def test_lowrank_head_with_all_ids_is_the_exact_sort_and_permutes_with_the_vocab
     assert np.allclose(lg1, lg2, rtol=0, atol=1e-12)
 
 
-def test_lowrank_screen_rounds_the_down_projection_to_bf16():
-    """U = I (r = V): the screen's logits are g = h D^T itself, which shows g's rounding to bf16.
-    Inputs are multiples of 1/8 in [-2, 2], so every product and sum (a multiple of 1/64, at most
-    256 in size) is exact in fp32 and torch's fp32 -> bf16 conversion rounds the exact g once.
-    D's rows repeat five distinct vectors, so each row's screen has groups of equal values and the
-    top-k cut falls inside one: the screen keeps the lowest ids of that group.  The k survivors
-    are then ordered by their exact logits h . W_c."""
+def test_lowrank_screen_is_the_factorised_product():
+    """U = I (r = V): the screen's logits are g = h D^T itself, unrounded.  Inputs are multiples
+    of 1/8 in [-2, 2], so every product and sum is exact in fp64 and numpy's product is the
+    definition; some of those values need more than bf16's 8 significant bits, so a screen that
+    rounded g would differ.  D's rows repeat five distinct vectors, so each row's screen has
+    groups of equal values and the top-k cut falls inside one: the screen keeps the lowest ids of
+    that group.  The k survivors are then ordered by their exact logits h . W_c."""
     g = np.random.default_rng(64)
     M, H, V, k = 4, 64, 40, 6
     hv = g.integers(-16, 17, size=(M, H)) / 8.0
@@ -888,18 +888,20 @@ def test_lowrank_screen_rounds_the_down_projection_to_bf16():
     U = _bf16_bits(np.eye(V))
     Wv = g.normal(0, 0.3, size=(V, H)).astype(np.float32)
     W = _bf16_bits(Wv)
-    ids, lg, kth, za = oracle.lowrank_candidates(hid, D, U, W, k, keep_approx=True)
+    ids, lg, kth, za, gg = oracle.lowrank_candidates(hid, D, U, W, k, keep_approx=True,
+                                                     keep_g=True)
     exact = hv @ dv.T
-    want = torch.as_tensor(exact.astype(np.float32)).to(torch.bfloat16).double().numpy()
-    assert not np.array_equal(want, exact)               # some screen logits do round
-    assert np.array_equal(za, want)
+    rounded = torch.as_tensor(exact.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert not np.array_equal(rounded, exact)            # bf16 would change some values
+    assert np.array_equal(za, exact) and np.array_equal(gg, exact)
     Wb = np.frombuffer((W.astype(np.uint32) << 16).tobytes(), np.float32).reshape(V, H)
     zx = hv @ Wb.astype(np.float64).T
     ties = 0
     for m in range(M):
-        top = np.lexsort((np.arange(V), -want[m]))[:k]
-        ties += int(want[m, top[-1]] == want[m, np.lexsort((np.arange(V), -want[m]))[k]])
-        assert kth[m] == want[m, top[-1]]
+        srt = np.lexsort((np.arange(V), -exact[m]))
+        top = srt[:k]
+        ties += int(exact[m, top[-1]] == exact[m, srt[k]])
+        assert kth[m] == exact[m, top[-1]]
         assert sorted(ids[m]) == sorted(top)
         order = sorted(top, key=lambda c: (-zx[m, c], c))
         assert list(ids[m]) == order
