@@ -233,7 +233,24 @@ def time_steps(dev, steps, warmup, flush):
     lm = [e[1].elapsed_time(e[2]) for e in ev]
     cp = [e[2].elapsed_time(e[3]) for e in ev]
     step = [e[0].elapsed_time(e[1]) for e in whole]
-    return dict(attn_ms=attn, lmhead_ms=lm, compact_ms=cp, step_ms=step)
+    # a third pass splits the LM-head call at its phase marks: set-up kernels, the first GEMM
+    # (the algorithmic pass), the acceptance kernels, the draw GEMM (T > 0), the last kernel
+    ph = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    for e in ph:                      # torch creates the CUDA event on its first record
+        for x in e:
+            x.record()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush()
+        e = ph[i]
+        dev.attn()
+        e[0].record()
+        dev.lmhead_marked(e[1:5])
+        e[5].record()
+    torch.cuda.synchronize()
+    names = ["setup", "gemm", "accept", "draw_gemm", "draw_pick"]
+    phases = {n: [e[k].elapsed_time(e[k + 1]) for e in ph] for k, n in enumerate(names)}
+    return dict(attn_ms=attn, lmhead_ms=lm, compact_ms=cp, step_ms=step, lmhead_phases=phases)
 
 
 def time_e2e(dev, wl, steps, warmup, flush):
@@ -395,13 +412,27 @@ def cpu_baseline(wl, min_seconds=10.0, max_reps=5):
 
 
 # -------------------------------------------------------------------------------------- main
+L2_POLICY = ("flushed before every timed step: 512 MiB write, then 256 MiB read (dirty lines "
+             "written back before the timed region)")
+
+
 def workload_config(name, wl, world):
-    """The workload keys both arms' JSON lines carry in `config`."""
+    """The workload keys both arms' JSON lines carry in `config` (identical for both arms)."""
     return {"workload": name, "B": wl.B, "tree_nodes": int(wl.n_max),
             "kv_len": int(wl.kv_len_max), "hidden": wl.hidden_dim, "vocab": wl.vocab,
             "heads": f"{wl.hq}/{wl.hkv}", "head_dim": wl.head_dim,
             "temperature": wl.temperature, "layers": 1,
-            "parallelism": f"dp{world} (independent requests per rank)"}
+            "parallelism": f"dp{world} (independent requests per rank)", "l2": L2_POLICY}
+
+
+def near_tie_rows(dev, wl):
+    """T = 0: node rows whose top-1 / top-2 logit gap (the library's own node_gap) is below the
+    near-tie bound 1e-3, where fp32 and fp64 may legitimately pick different argmaxes."""
+    if wl.temperature != 0.0:
+        return None
+    gap = dev.node_gap.cpu().numpy()
+    return {"rows": int(gap.size), "gap_lt_1e-3": int((gap < 1e-3).sum()),
+            "min_gap": float(gap.min()) if gap.size else None}
 
 
 def run_config(name, steps, warmup, peaks, rank, flush, with_e2e=True):
@@ -501,8 +532,23 @@ def kernel_report(wl, t, acc, peaks):
         "compact": {"us": cm * 1e6, "GB/s": cb / cm / 1e9, "hbm_frac": cb / cm / 1e9 / hbm,
                     "bytes": cb},
     }
+    # the LM-head call by phase (events between its kernels): the first GEMM against the
+    # algorithmic work; the draw GEMM (T > 0) is implementation overhead, reported on its own
+    # with the FLOPs it performs (2 B V H)
+    ph = {n: statistics.mean(v) * 1e-3 for n, v in t["lmhead_phases"].items()}
+    g1 = ph["gemm"]
+    rep["lmhead_phases_us"] = {n: v * 1e6 for n, v in ph.items()}
+    rep["lmhead_gemm"] = {"us": g1 * 1e6, "GB/s": lb / g1 / 1e9, "TFLOP/s": lf / g1 / 1e12,
+                          "hbm_frac": lb / g1 / 1e9 / hbm, "tc_frac": lf / g1 / 1e12 / tc}
+    if wl.temperature > 0.0:
+        g2 = ph["draw_gemm"]
+        df = 2.0 * wl.B * wl.vocab * wl.hidden_dim
+        rep["lmhead_draw_gemm"] = {"us": g2 * 1e6, "TFLOP/s": df / g2 / 1e12,
+                                   "tc_frac": df / g2 / 1e12 / tc, "flops": df,
+                                   "note": "second W pass over the B stop rows; not algorithmic"}
     for k in rep.values():
-        k["hbm_frac_nominal"] = k["GB/s"] / NOMINAL_HBM_GBS
+        if "GB/s" in k:
+            k["hbm_frac_nominal"] = k["GB/s"] / NOMINAL_HBM_GBS
         if "TFLOP/s" in k:
             k["tc_frac_nominal"] = k["TFLOP/s"] / NOMINAL_BF16_TFLOPS
     return rep
@@ -573,6 +619,7 @@ def main():
     e2e_s = sum(e2e_ms) * 1e-3
     step_s, e2e_s, tokens_all = reduce_over_ranks(step_s, e2e_s, tokens, world, "cuda")
     acc = main_res["dev"].accept_len.cpu().numpy()
+    near = near_tie_rows(main_res["dev"], wl)
     rep = kernel_report(wl, t, acc, peaks)
     rep["compact_64layers"] = compact_layers_report(main_res["dev"], wl, flush, peaks)
     rl = roofline(wl, rep, peaks, peak_kind, args.config)
@@ -598,6 +645,7 @@ def main():
                             for kk, vv in v.items()} for k, v in rrep.items()},
             "roofline": roofline(r["wl"], rrep, peaks, peak_kind, name),
             "attn_plan": r["plan"], "gpu_launches_per_step": r["launches"],
+            "near_ties": near_tie_rows(r["dev"], r["wl"]),
         }
         main_res = r
 
@@ -632,10 +680,9 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; random-init LM head, N(0,1) activations and KV)",
-        "config": {**workload_config(args.config, wl, world),
-                   "l2": "flushed before every timed step: 512 MiB write, then 256 MiB read "
-                         "(dirty lines written back before the timed region)",
-                   "attn_plan": head_plan},
+        "config": workload_config(args.config, wl, world),
+        "attn_plan": head_plan,
+        "near_ties": near,
         "clocks": clk,
         "e2e": {"value": tokens_all / e2e_s, "unit": "accepted tok/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -673,7 +720,7 @@ def main_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {**workload_config(args.config, wl, world), "sampled_requests": len(reqs)},
+        "config": workload_config(args.config, wl, world),
         "cpu_baseline": {"value": value, "unit": "accepted tok/s", "cores": oracle.max_threads(),
                          "kind": "oracle",
                          "sample": f"{len(reqs)} of {wl.B} requests per step, full oracle "

@@ -28,7 +28,8 @@ import torch
 __all__ = [
     "EtreeError", "Batch", "make_batch", "lib", "library_path", "etree_workspace_size",
     "etree_workspace_init", "etree_verify_attn", "etree_verify_attn_noalloc",
-    "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact",
+    "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_lmhead_accept_timed",
+    "etree_kv_compact",
     "etree_verify_attn_paged", "etree_kv_compact_paged", "etree_verify_cost", "etree_plan_tree",
     "cost_table", "load_cost_table", "etree_lowrank_workspace_size",
     "etree_lowrank_candidates", "etree_device_status", "etree_selftest_timeout", "etree_strerror",
@@ -47,7 +48,8 @@ DETAIL = {0: "none", 1: "bad parent", 2: "bad node count", 3: "bad kv_len", 4: "
 EXPORTS = ["etree_workspace_size", "etree_workspace_init", "etree_verify_attn",
            "etree_verify_attn_paged", "etree_kv_compact_paged", "etree_verify_cost",
            "etree_plan_tree", "etree_lowrank_workspace_size", "etree_lowrank_candidates",
-           "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_kv_compact", "etree_device_status", "etree_strerror",
+           "etree_lmhead_accept", "etree_lmhead_accept_tree", "etree_lmhead_accept_timed",
+           "etree_kv_compact", "etree_device_status", "etree_strerror",
            "etree_version", "etree_last_error", "etree_attn_plan", "etree_verify_attn_noalloc",
            "etree_selftest_timeout"]
 
@@ -96,6 +98,10 @@ def lib():
     L.etree_lmhead_accept_tree.argtypes = [bp, vp, vp, C.c_int, C.c_int, f32, vp, u64, u64, vp,
                                            vp, vp, vp, C.c_int32, vp, C.c_size_t, vp]
     L.etree_lmhead_accept_tree.restype = C.c_int
+    L.etree_lmhead_accept_timed.argtypes = [bp, vp, vp, C.c_int, C.c_int, f32, vp, u64, u64, vp,
+                                            vp, vp, vp, vp, vp, C.c_int32, C.c_int32,
+                                            C.POINTER(C.c_void_p), vp, C.c_size_t, vp]
+    L.etree_lmhead_accept_timed.restype = C.c_int
     L.etree_kv_compact.argtypes = [bp, vp, vp, vp, vp, vp, vp, C.c_int, i64, i64, C.c_int,
                                    C.c_int, vp, vp, C.c_size_t, vp]
     L.etree_kv_compact.restype = C.c_int
@@ -332,6 +338,29 @@ def etree_lmhead_accept_tree(batch: Batch, hidden, w_lm, temperature: float, q_d
         int(seed) & (2**64 - 1), int(step) & (2**64 - 1),
         _ptr(accept_len, torch.int32, "accept_len"), _ptr(path, torch.int32, "path"),
         _ptr(out_tokens, torch.int32, "out_tokens"), _ptr(zbuf, torch.float32, "zbuf"), rows,
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
+    return _check(st) if check else st
+
+
+def etree_lmhead_accept_timed(batch: Batch, hidden, w_lm, temperature: float, q_draft, seed: int,
+                              step: int, accept_len, path, out_tokens, node_argmax, node_gap,
+                              zbuf, branching: bool, marks, workspace, stream=None,
+                              check: bool = True) -> int:
+    """etree_lmhead_accept(_tree) with phase marks: `marks` is a list of 4 torch.cuda.Event
+    (or None entries) recorded after the set-up kernels, the first GEMM, the acceptance kernels
+    and the draw GEMM.  torch creates an Event's CUDA event on its first record(): record each
+    once before passing it, or its handle is NULL and the mark is skipped."""
+    bf = torch.bfloat16
+    rows = 0 if zbuf is None else int(zbuf.shape[0])
+    arr = (C.c_void_p * 4)(*[None if m is None else m.cuda_event for m in marks])
+    st = lib().etree_lmhead_accept_timed(
+        C.byref(batch), _ptr(hidden, bf, "hidden"), _ptr(w_lm, bf, "w_lm"), hidden.shape[1],
+        w_lm.shape[0], float(temperature), _ptr(q_draft, torch.float32, "q_draft"),
+        int(seed) & (2**64 - 1), int(step) & (2**64 - 1),
+        _ptr(accept_len, torch.int32, "accept_len"), _ptr(path, torch.int32, "path"),
+        _ptr(out_tokens, torch.int32, "out_tokens"),
+        _ptr(node_argmax, torch.int32, "node_argmax"), _ptr(node_gap, torch.float32, "node_gap"),
+        _ptr(zbuf, torch.float32, "zbuf"), rows, int(bool(branching)), arr,
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
     return _check(st) if check else st
 

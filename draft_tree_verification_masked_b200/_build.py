@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libetree.so")
-SOURCES = ["api.cu", "attn_tree.cu", "attn_tc.cu", "lmhead.cu", "accept.cu", "compact.cu",
+SOURCES = ["api.cu", "attn_combine.cu", "attn_tc.cu", "lmhead.cu", "accept.cu", "compact.cu",
            "plan.cu", "lowrank.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC = os.environ.get("NVCC", "nvcc")

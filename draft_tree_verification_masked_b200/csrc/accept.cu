@@ -113,10 +113,18 @@ __device__ void walk_greedy(const AcceptParams& p, const int32_t* arg_ws, int r,
   }
   ok = __all_sync(0xffffffffu, ok);
   __syncwarp();
-  if (!ok && lane == 0) report(p.ws, ETREE_EDEVICE, DET_BAD_PARENT);
+  if (!ok) {                                       // no valid tree: nothing accepted, no bonus
+    if (lane == 0) {
+      report(p.ws, ETREE_EDEVICE, DET_BAD_PARENT);
+      p.accept_len[r] = 0;
+    }
+    for (int k = lane; k < 64; k += 32) path[k] = -1;
+    for (int k = lane; k < 65; k += 32) outt[k] = -1;
+    return;
+  }
   int u = 0, a = 0;
   if (lane == 0) pth[0] = 0;
-  if (ok) {
+  {
     for (int step = 0; step < 64; ++step) {
       const int want = am[u];
       const bool m0 = lane >= 1 && par[lane] == u && tok[lane] == want;
@@ -272,6 +280,8 @@ __device__ void accept_chain(const AcceptParams& p, int r, int base, int n, int 
     p.stop_row[r] = src;
     p.stop_node[r] = chain ? a : 0;
     p.cval[r] = (chain && rejected) ? 1.f : 0.f;
+    p.rfloor[2 * r] = 0u;
+    p.rfloor[2 * r + 1] = 0u;
   }
   const uint4* hs = reinterpret_cast<const uint4*>(p.hidden + (size_t)src * p.H);
   uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
@@ -294,6 +304,8 @@ __global__ void __launch_bounds__(256) chain_accept_kernel(AcceptParams p, int32
       p.stop_row[r] = 0;
       p.stop_node[r] = 0;
       p.cval[r] = 0.f;
+      p.rfloor[2 * r] = 0u;
+      p.rfloor[2 * r + 1] = 0u;
     }
     const uint4* hs = reinterpret_cast<const uint4*>(p.hidden);
     uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
@@ -497,8 +509,9 @@ __device__ double residual_mass(const AcceptParams& p, const float* zr, const fl
 
 // One CTA per request: the multi-candidate walk.  Thread 0 takes the decisions; the whole CTA
 // evaluates N(c) when a rejected child has a younger sibling still to test.  Writes accept_len,
-// path, the accepted tokens, the stop row / node, the draw offset cval (negative: fall back to
-// argmax p) and the stop row's hidden state for the draw pass.
+// path, the accepted tokens, the stop row / node, the draw offset cval (negative: the residual
+// has no positive weight and the bonus is drawn from p) and the stop row's hidden state for the
+// draw pass.
 constexpr int kWalkThreads = 1024;
 
 __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p, const float* zc,
@@ -541,6 +554,8 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
       p.stop_row[r] = n_ok ? base : 0;
       p.stop_node[r] = 0;
       p.cval[r] = 0.f;
+      p.rfloor[2 * r] = 0u;
+      p.rfloor[2 * r + 1] = 0u;
       u_s = n_ok ? base : 0;
     }
   } else {
@@ -592,7 +607,7 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
                                         p.q_draft + (size_t)ur * p.V, p.lse2[ur], c_s, red_s);
         if (tid == 0) {
           N = Nn;
-          if (!(N > 0.0)) fell_s = 1;                   // no positive residual: argmax p
+          if (!(N > 0.0)) fell_s = 1;                   // no positive residual: draw from p
         }
         __syncthreads();
         if (fell_s) break;
@@ -605,6 +620,8 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
       p.stop_row[r] = base + u;
       p.stop_node[r] = u;
       p.cval[r] = fell_s ? -1.f : (float)c;
+      p.rfloor[2 * r] = 0u;
+      p.rfloor[2 * r + 1] = 0u;
       u_s = base + u;
     }
   }
@@ -614,63 +631,48 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
   for (int i = tid; i < p.H / 8; i += blockDim.x) hd[i] = hs[i];
 }
 
-// The first level of the two-level draw, per request: the exponential race among the 128-id
-// block totals (key W_b / E_b with E_b = -log U_b, stream 2), ties to the lowest block; the
-// bonus is the inverse-CDF pick the GEMM epilogue made inside the winning block.  A residual
-// with no positive weight anywhere (p <= q everywhere: p = q up to rounding) gives the argmax
-// of p instead, taken from the per-block logit maxima.
-constexpr int kBonusThreads = 256;
-
-__global__ void __launch_bounds__(kBonusThreads) bonus_kernel(AcceptParams p) {
-  __shared__ float kb_s[kBonusThreads / 32], zm_s[kBonusThreads / 32];
-  __shared__ int ib_s[kBonusThreads / 32], iz_s[kBonusThreads / 32];
-  const int r = blockIdx.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int node = p.stop_node[r];
+// The bonus draw's last step, one warp per request: the largest race key over the draw pass's
+// summaries (ties to the lower id), for the residual weights and for p.  The bonus is the
+// residual's winner, or p's when the residual has no positive weight (or no rejection happened,
+// in which case the draw weights are p and only p's race ran).
+__global__ void __launch_bounds__(256) bonus_kernel(AcceptParams p) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= p.B) return;
   const float4* row = p.part2 + (size_t)r * p.n_tiles2;
-  float kb = -INFINITY, zm = -INFINITY;
-  int ib = -1, iz = -1;
-  // blocks in groups of 8 (one Philox draw) over the CTA; the merges are a total order (larger
-  // key, then lower id), so the split does not change the result
-  for (int g = threadIdx.x; g * 8 < p.n_tiles2; g += kBonusThreads) {
-    float u[8];
-    uniforms8(p.seed, p.step, (uint32_t)g, (uint32_t)node, (uint32_t)r, 2u, u);
+  float kr = -INFINITY, kp = -INFINITY;
+  int ir = -1, ip = -1;
+  int t = lane;
+  for (; t + 96 < p.n_tiles2; t += 128) {             // four loads in flight per lane
+    float4 x[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int b = g * 8 + e;
-      if (b < p.n_tiles2) {
-        const float4 v = row[b];
-        if (v.x > 0.f) merge_key(kb, ib, __fdividef(v.x, -logf(u[e])), __float_as_int(v.y));
-        merge_key(zm, iz, v.z, __float_as_int(v.w));
-      }
+    for (int u = 0; u < 4; ++u) x[u] = row[t + 32 * u];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      merge_key(kr, ir, x[u].x, __float_as_int(x[u].y));
+      merge_key(kp, ip, x[u].z, __float_as_int(x[u].w));
     }
+  }
+  for (; t < p.n_tiles2; t += 32) {
+    const float4 x = row[t];
+    merge_key(kr, ir, x.x, __float_as_int(x.y));
+    merge_key(kp, ip, x.z, __float_as_int(x.w));
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-    const float okb = __shfl_xor_sync(0xffffffffu, kb, off);
-    const int oib = __shfl_xor_sync(0xffffffffu, ib, off);
-    const float ozm = __shfl_xor_sync(0xffffffffu, zm, off);
-    const int oiz = __shfl_xor_sync(0xffffffffu, iz, off);
-    merge_key(kb, ib, okb, oib);
-    merge_key(zm, iz, ozm, oiz);
+    const float okr = __shfl_xor_sync(0xffffffffu, kr, off);
+    const int oir = __shfl_xor_sync(0xffffffffu, ir, off);
+    const float okp = __shfl_xor_sync(0xffffffffu, kp, off);
+    const int oip = __shfl_xor_sync(0xffffffffu, ip, off);
+    merge_key(kr, ir, okr, oir);
+    merge_key(kp, ip, okp, oip);
   }
   if (lane == 0) {
-    kb_s[warp] = kb;
-    ib_s[warp] = ib;
-    zm_s[warp] = zm;
-    iz_s[warp] = iz;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < kBonusThreads / 32; ++w) {
-      merge_key(kb, ib, kb_s[w], ib_s[w]);
-      merge_key(zm, iz, zm_s[w], iz_s[w]);
-    }
     const int base = p.cu_nodes[r];
     const int n = p.cu_nodes[r + 1] - base;
     if (n < 1 || n > p.n_max) return;
     const int a = p.accept_len[r];
-    p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = ib >= 0 ? ib : iz;
+    p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = ir >= 0 ? ir : ip;
   }
 }
 
@@ -705,7 +707,7 @@ cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32
 }
 
 cudaError_t launch_bonus(const AcceptParams& p, cudaStream_t s) {
-  bonus_kernel<<<p.B, kBonusThreads, 0, s>>>(p);
+  bonus_kernel<<<(p.B + 7) / 8, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -1,6 +1,6 @@
 // api.cu -- the C ABI of libetree: argument validation, workspace layout, TMA descriptors and
 // launch planning for the three verification calls.  Every step of the computation runs in the
-// kernels of attn_tree.cu, lmhead.cu, accept.cu and compact.cu; this file only plans and
+// kernels of attn_tc.cu, attn_combine.cu, lmhead.cu, accept.cu and compact.cu; this file only plans and
 // enqueues them.
 #include <algorithm>
 #include <cmath>
@@ -45,71 +45,42 @@ static int sm_count() {
   return cached[dev];
 }
 
-static int env_int(const char* name, int dflt) {
-  const char* v = getenv(name);
-  if (!v || !*v) return dflt;
-  return atoi(v);
-}
-
 // ------------------------------------------------------------------------------ attention plan
 struct AttnPlan {
-  int G, tc, keys, nw, nb, mchunks, nsplit, tps, stages;
+  int G, keys, nb, mchunks, nsplit, tps;
 };
 
-// Launch plan of the attention call.  The tcgen05 kernel (default) takes 128-row blocks of
-// nb = min(floor(128 / G), n_max) whole nodes; with at least one (request, KV head, row block) per
-// SM, or 64K or more cached keys, it uses 32-key tiles and two CTAs per SM, otherwise 64-key tiles
-// and one CTA per SM.  The KV range
-// is split only to fill one wave of CTAs (a second, partial wave costs more than longer splits),
-// keeping >= 4 key tiles per split.  The warp-MMA kernel (ETREE_ATTN=mma) takes 16-row warps,
-// 64-key tiles, and aims at about four CTAs per SM.
+// Launch plan of the attention call.  The tcgen05 kernel takes 128-row blocks of
+// nb = min(floor(128 / G), n_max) whole nodes; with at least one (request, KV head, row block)
+// per SM, or 64K or more cached keys, it uses 32-key tiles and two CTAs per SM, otherwise 64-key
+// tiles and one CTA per SM.  The KV range is split only to fill one wave of CTAs (a second,
+// partial wave costs more than longer splits), keeping >= 4 key tiles per split.
 static AttnPlan plan_attn(const etree_batch* b, int hq, int hkv) {
   AttnPlan pl{};
   pl.G = hq / hkv;
-  const char* kind = getenv("ETREE_ATTN");
-  pl.tc = !(kind && strcmp(kind, "mma") == 0) && pl.G <= 128;
   const int sms = sm_count();
-  if (pl.tc) {
-    pl.nb = std::min(128 / pl.G, b->n_max);           // nodes per Q box (row block)
-    pl.mchunks = (b->n_max + pl.nb - 1) / pl.nb;
-    pl.nw = 4;
-    const int pairs0 = b->B * hkv * pl.mchunks;
-    // 32-key tiles (two CTAs per SM) pay off once there is at least one row block per SM, and
-    // on very long contexts (>= 64K keys: measured 5-8% faster at 128K, 5% slower at 32K);
-    // otherwise few, long work items prefer 64-key tiles split over the SMs
-    pl.keys = (pairs0 >= sms || b->kv_len_max >= 65536) ? 32 : 64;
-    const int forced = env_int("ETREE_ATTN_KEYS", 0);
-    if (forced == 32 || forced == 64) pl.keys = forced;
-  } else {
-    pl.keys = 64;
-    const int m16 = (b->n_max * pl.G + 15) / 16;
-    if (m16 <= 8) {
-      pl.nw = std::max(1, m16);
-      pl.mchunks = 1;
-    } else {
-      pl.mchunks = (m16 + 7) / 8;
-      pl.nw = (m16 + pl.mchunks - 1) / pl.mchunks;
-    }
-  }
+  pl.nb = std::min(128 / pl.G, b->n_max);             // nodes per Q box (row block)
+  pl.mchunks = (b->n_max + pl.nb - 1) / pl.nb;
   const int pairs = b->B * hkv * pl.mchunks;
+  // 32-key tiles (two CTAs per SM) pay off once there is at least one row block per SM, and on
+  // very long contexts (>= 64K keys: measured 5-8% faster at 128K, 5% slower at 32K); otherwise
+  // few, long work items prefer 64-key tiles split over the SMs
+  pl.keys = (pairs >= sms || b->kv_len_max >= 65536) ? 32 : 64;
   const int tiles_max =
       (b->kv_len_max + pl.keys - 1) / pl.keys + (b->n_max + pl.keys - 1) / pl.keys;
-  const int per_sm = pl.tc ? (pl.keys == 32 ? 2 : 1) : 4;
-  int nsplit = pl.tc ? std::max(1, per_sm * sms / pairs) : (per_sm * sms + pairs - 1) / pairs;
+  const int per_sm = pl.keys == 32 ? 2 : 1;
+  int nsplit = std::max(1, per_sm * sms / pairs);
   nsplit = std::min(nsplit, std::max(1, tiles_max / 4));
   nsplit = std::max(1, std::min(nsplit, tiles_max));
-  const int forced = env_int("ETREE_NSPLIT", 0);
-  if (forced > 0) nsplit = std::min(forced, tiles_max);
   pl.tps = (tiles_max + nsplit - 1) / nsplit;
   pl.nsplit = (tiles_max + pl.tps - 1) / pl.tps;
-  pl.stages = env_int("ETREE_STAGES", 3) == 4 ? 4 : 3;
   return pl;
 }
 
 // ------------------------------------------------------------------------------ workspace map
 struct WsLayout {
   size_t order, o_part, ml_part, part, child_tok, zchild, lse2, stop_row, stop_node, cval, hid2,
-      part2, cnt, ccount, zrow, zc;
+      part2, rfloor, cnt, ccount, zrow, zc;
   size_t total;
   int n_tiles;
 };
@@ -143,6 +114,7 @@ static WsLayout layout(const etree_batch* b, int hq, int hkv, int hidden_dim, in
   w.cval = take(B * sizeof(float));
   w.hid2 = take(B * (size_t)std::max(0, hidden_dim) * 2);
   w.part2 = take(B * (size_t)w.n_tiles * sizeof(float4));
+  w.rfloor = take(B * 2 * sizeof(uint32_t));
   w.cnt = take(B * sizeof(int32_t));
   w.ccount = take(nt * sizeof(int32_t));
   w.zrow = take(nt * sizeof(int32_t));
@@ -265,29 +237,64 @@ static T* at(void* ws, size_t off) {
 
 // ------------------------------------------------------------------ statically backed scratch
 // Scratch for etree_verify_attn_noalloc: a fixed array in device global memory, created when the
-// library's module is loaded on a device and held until the process exits.  Host code must not
-// use the symbol as a pointer; it asks the runtime for the device address once per device.
-constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+// library's module is loaded in a context and held until that context ends.  Host code must not
+// use the symbol as a pointer; it asks the runtime for the device address in the current
+// context.  The address is cached per context, keyed by the driver's context id, which is unique
+// for the life of the process: a device reset or a caller-made context gets a fresh lookup.
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) uint8_t g_attn_scratch[kStaticScratchBytes];
 
-static std::mutex g_scratch_mu;
-static void* g_scratch_ptr[64] = {nullptr};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// Device address of g_attn_scratch on the current device, resolved on the first call per device.
+static std::mutex g_scratch_mu;
+static std::unordered_map<unsigned long long, void*> g_scratch_ptr;
+
+// Device address of g_attn_scratch in the calling thread's current context.
 static etree_status static_scratch(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "etree_verify_attn_noalloc: cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(ETREE_EUNSUPPORTED, "device ordinal %d >= 64", dev);
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_attn_scratch);
-    if (e != cudaSuccess || !p)
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id)
+    return fail(ETREE_ECUDA, "etree_verify_attn_noalloc: cuCtxGetCurrent / cuCtxGetId unavailable");
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS)
+    return fail(ETREE_ECUDA, "etree_verify_attn_noalloc: cuCtxGetCurrent failed");
+  void* fresh = nullptr;
+  if (!ctx) {
+    // no context yet on this thread: the lookup itself makes the device's primary context
+    // current (the runtime's usual lazy initialisation)
+    const cudaError_t e = cudaGetSymbolAddress(&fresh, g_attn_scratch);
+    if (e != cudaSuccess || !fresh)
       return cuda_fail(e, "etree_verify_attn_noalloc: cudaGetSymbolAddress");
-    g_scratch_ptr[dev] = p;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx)
+      return fail(ETREE_ECUDA, "etree_verify_attn_noalloc: no current context");
   }
-  *out = g_scratch_ptr[dev];
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS)
+    return fail(ETREE_ECUDA, "etree_verify_attn_noalloc: cuCtxGetId failed");
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  auto it = g_scratch_ptr.find(id);
+  if (it == g_scratch_ptr.end()) {
+    if (!fresh) {
+      const cudaError_t e = cudaGetSymbolAddress(&fresh, g_attn_scratch);
+      if (e != cudaSuccess || !fresh)
+        return cuda_fail(e, "etree_verify_attn_noalloc: cudaGetSymbolAddress");
+    }
+    if (g_scratch_ptr.size() > 1024) g_scratch_ptr.clear();
+    it = g_scratch_ptr.emplace(id, fresh).first;
+  }
+  *out = it->second;
   return ETREE_OK;
 }
 
@@ -323,8 +330,8 @@ etree_status etree_attn_plan(const etree_batch* batch, int hq, int hkv, int32_t*
   if (hq < 1 || hkv < 1 || hq % hkv != 0 || hq / hkv > 64)
     return fail(ETREE_EINVAL, "hq=%d, hkv=%d", hq, hkv);
   const AttnPlan pl = plan_attn(batch, hq, hkv);
-  if (kernel) *kernel = pl.tc;
-  if (rows_per_cta) *rows_per_cta = pl.tc ? pl.nb * pl.G : pl.nw * 16;
+  if (kernel) *kernel = 1;
+  if (rows_per_cta) *rows_per_cta = pl.nb * pl.G;
   if (row_blocks) *row_blocks = pl.mchunks;
   if (splits) *splits = pl.nsplit;
   if (tiles_per_split) *tiles_per_split = pl.tps;
@@ -462,13 +469,16 @@ etree_status etree_device_status(void* workspace, void* stream, int32_t* detail)
 // The bounded-wait path every pipeline relies on, exercised on purpose: one thread waits on an
 // mbarrier that no thread ever arrives at; the wait gives up after its iteration cap and the
 // kernel records ETREE_ETIMEOUT (detail DET_SELFTEST) in the workspace status word.  Nothing
-// traps, and the context stays usable.
+// traps, and the context stays usable.  The self-test runs the same wait loop with a cap of 256
+// tries (about a millisecond) instead of the pipelines' (about 8 s), so the test is brief.
+constexpr uint32_t kSelftestWaitCap = 256;
+
 __global__ void selftest_wait_kernel(WsHeader* ws) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     fence_barrier_init();
-    if (!mbar_wait(&bar, 0)) report(ws, ETREE_ETIMEOUT, DET_SELFTEST);
+    if (!mbar_wait(&bar, 0, kSelftestWaitCap)) report(ws, ETREE_ETIMEOUT, DET_SELFTEST);
   }
 }
 
@@ -508,13 +518,12 @@ static int log2i(int x) {
   return k;
 }
 
-static etree_status verify_attn_impl(const etree_batch* b, const uint16_t* q,
-                                     const uint16_t* k_tree, const uint16_t* v_tree,
-                                     const uint16_t* k_cache, const uint16_t* v_cache,
-                                     int64_t cache_slots, int hq, int hkv, int head_dim,
-                                     float scale, uint16_t* out, float* lse,
-                                     const PagedArgs* pg, void* workspace,
-                                     size_t workspace_bytes, void* stream) {
+// Host-visible checks of the attention arguments other than the workspace.
+static etree_status check_attn_args(const etree_batch* b, const uint16_t* q,
+                                    const uint16_t* k_tree, const uint16_t* v_tree,
+                                    const uint16_t* k_cache, const uint16_t* v_cache,
+                                    int64_t cache_slots, int hq, int hkv, int head_dim,
+                                    float scale, const uint16_t* out, const float* lse) {
   etree_status st = check_batch(b);
   if (st) return st;
   if (head_dim != ETREE_HEAD_DIM)
@@ -529,10 +538,22 @@ static etree_status verify_attn_impl(const etree_batch* b, const uint16_t* q,
   if (cache_slots < 1 || cache_slots > INT32_MAX)
     return fail(ETREE_EINVAL, "cache_slots=%lld outside [1, 2^31)", (long long)cache_slots);
   if (!std::isfinite(scale)) return fail(ETREE_EINVAL, "scale is not finite");
+  return ETREE_OK;
+}
+
+static etree_status verify_attn_impl(const etree_batch* b, const uint16_t* q,
+                                     const uint16_t* k_tree, const uint16_t* v_tree,
+                                     const uint16_t* k_cache, const uint16_t* v_cache,
+                                     int64_t cache_slots, int hq, int hkv, int head_dim,
+                                     float scale, uint16_t* out, float* lse,
+                                     const PagedArgs* pg, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  etree_status st = check_attn_args(b, q, k_tree, v_tree, k_cache, v_cache, cache_slots, hq, hkv,
+                                    head_dim, scale, out, lse);
+  if (st) return st;
   if ((st = check_ws(b, hq, hkv, 0, 0, workspace, workspace_bytes))) return st;
 
   const AttnPlan pl = plan_attn(b, hq, hkv);
-  if (pg && !pl.tc) return fail(ETREE_EUNSUPPORTED, "paged caches need the tcgen05 kernel");
   CUtensorMap kc, vc, kt, vt;
   const uint32_t kb = (uint32_t)pl.keys;
   const uint32_t cbox = pg ? (uint32_t)std::min(pl.keys, pg->page_size) : kb;
@@ -573,21 +594,15 @@ static etree_status verify_attn_impl(const etree_batch* b, const uint16_t* q,
   cudaError_t e;
   // with many requests of mixed lengths, dispatch the longest first
   p.order = nullptr;
-  if (b->B >= 8 && env_int("ETREE_ATTN_LPT", 1)) {
+  if (b->B >= 8) {
     p.order = at<int32_t>(workspace, w.order);
     e = launch_attn_order(b->kv_len, b->B, at<int32_t>(workspace, w.order),
                           static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "etree_verify_attn order");
   }
-  if (pl.tc) {
-    CUtensorMap tq;
-    if ((st = get_map(q, 3, 128, hq, b->n_total, 64, pl.G, pl.nb, &tq))) return st;
-    e = launch_attn_tc(tq, kc, vc, kt, vt, p, pl.nb, b->n_total,
-                       static_cast<cudaStream_t>(stream));
-  } else {
-    e = launch_attn(kc, vc, kt, vt, p, pl.nw, pl.stages, b->n_total,
-                    static_cast<cudaStream_t>(stream));
-  }
+  CUtensorMap tq;
+  if ((st = get_map(q, 3, 128, hq, b->n_total, 64, pl.G, pl.nb, &tq))) return st;
+  e = launch_attn_tc(tq, kc, vc, kt, vt, p, pl.nb, b->n_total, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_verify_attn launch");
 }
 
@@ -626,7 +641,8 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
                                        uint64_t step, int32_t* accept_len, int32_t* path,
                                        int32_t* out_tokens, int32_t* node_argmax,
                                        float* node_gap, const TreeRows* tree, void* workspace,
-                                       size_t workspace_bytes, void* stream) {
+                                       size_t workspace_bytes, void* stream,
+                                       void* const* marks = nullptr) {
   etree_status st = check_batch(b);
   if (st) return st;
   if (hidden_dim < 64 || hidden_dim % 64 != 0)
@@ -648,7 +664,7 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
   const int sms = sm_count();
   const int bn = lmhead_pick_bn(b->n_total, vocab, sms);
   // up to 64 rows: M=64 MMAs with half-height hidden tiles (the W stream is the cost)
-  const int bm = (b->n_total <= 64 && env_int("ETREE_BM", 0) != 128) ? 64 : 128;
+  const int bm = b->n_total <= 64 ? 64 : 128;
   CUtensorMap ta, tb;
   if ((st = get_map(hidden, 2, hidden_dim, b->n_total, 1, 64, bm, 1, &ta))) return st;
   if ((st = get_map(w_lm, 2, hidden_dim, vocab, 1, 64, bn, 1, &tb))) return st;
@@ -674,7 +690,7 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
   g.seed = seed;
   g.step = step;
   const int grid = std::min(g.num_tiles, sms);
-  g.per_cta = g.m_tiles == 1 && env_int("ETREE_PER_TILE", 0) == 0;
+  g.per_cta = g.m_tiles == 1;
   g.n_parts = g.per_cta ? grid : g.n_tiles;
   int32_t* cnt = at<int32_t>(workspace, w.cnt);
   g.cnt = cnt;
@@ -709,33 +725,49 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
   a.hid2 = at<__nv_bfloat16>(workspace, w.hid2);
   a.H = hidden_dim;
   a.part2 = at<float4>(workspace, w.part2);
+  a.rfloor = at<uint32_t>(workspace, w.rfloor);
 
+  // phase marks (measurement only): events recorded after the set-up kernels, the first GEMM,
+  // the acceptance kernels and the draw GEMM
+  auto mark = [&](int k) {
+    if (marks && marks[k]) cudaEventRecord(static_cast<cudaEvent_t>(marks[k]), s);
+  };
   cudaError_t e;
   if (temperature == 0.f) {
+    mark(0);
     e = launch_lmhead(0, bn, bm, ta, tb, g, grid, s);
+    mark(1);
     if (e == cudaSuccess) e = launch_accept_greedy(a, at<int32_t>(workspace, w.child_tok), cnt, s);
+    mark(2);
+    mark(3);
     return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T=0)");
   }
   if (!tree) {                               // chains: accept tests fused with the row merge
     e = launch_chain_prep(a, at<int32_t>(workspace, w.child_tok), s);
+    mark(0);
     if (e == cudaSuccess) e = launch_lmhead(1, bn, bm, ta, tb, g, grid, s);
+    mark(1);
     if (e == cudaSuccess) e = launch_accept_chain(a, cnt, s);
   } else {                                   // trees: materialised rows of branching nodes
     int32_t* zrow = at<int32_t>(workspace, w.zrow);
     float* zc = at<float>(workspace, w.zc);
     e = launch_tree_prep(a, reinterpret_cast<const __nv_bfloat16*>(w_lm),
                          at<int32_t>(workspace, w.ccount), zrow, tree->rows, zc, s);
+    mark(0);
     g.child_tok = nullptr;
     g.zrow = zrow;
     g.zbuf = tree->zbuf;
     if (e == cudaSuccess) e = launch_lmhead(1, bn, bm, ta, tb, g, grid, s);
+    mark(1);
     g.zrow = nullptr;
     g.zbuf = nullptr;
     if (e == cudaSuccess) e = launch_tree_walk(a, zc, zrow, tree->zbuf, s);
   }
+  mark(2);
   if (e != cudaSuccess) return cuda_fail(e, "etree_lmhead_accept (T>0, pass 1)");
-  const int bn2 = 256;                       // the draw's 128-id blocks pair up in a tile
-  const int bm2 = (b->B <= 64 && env_int("ETREE_BM", 0) != 128) ? 64 : 128;
+  // the draw pass: the stop row of every request, M = B rows
+  const int bn2 = lmhead_pick_bn(b->B, vocab, sms);
+  const int bm2 = b->B <= 64 ? 64 : 128;
   CUtensorMap th, tb2;
   if ((st = get_map(a.hid2, 2, hidden_dim, b->B, 1, 64, bm2, 1, &th))) return st;
   if ((st = get_map(w_lm, 2, hidden_dim, vocab, 1, 64, bn2, 1, &tb2))) return st;
@@ -745,11 +777,14 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
   g2.n_tiles = (vocab + bn2 - 1) / bn2;
   g2.num_tiles = g2.m_tiles * g2.n_tiles;
   g2.part = at<float4>(workspace, w.part2);
-  g2.per_cta = 0;                            // the draw needs every 128-id block's summary
-  g2.n_parts = g2.n_tiles;
+  const int grid2 = std::min(g2.num_tiles, sms);
+  g2.per_cta = g2.m_tiles == 1;
+  g2.n_parts = g2.per_cta ? grid2 : g2.n_tiles;
   g2.cnt = nullptr;
-  a.n_tiles2 = 2 * g2.n_tiles;
-  e = launch_lmhead(2, bn2, bm2, th, tb2, g2, std::min(g2.num_tiles, sms), s);
+  g2.rfloor = a.rfloor;
+  a.n_tiles2 = 2 * g2.n_parts;
+  e = launch_lmhead(2, bn2, bm2, th, tb2, g2, grid2, s);
+  mark(3);
   if (e == cudaSuccess) e = launch_bonus(a, s);
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T>0, pass 2)");
 }
@@ -779,6 +814,26 @@ etree_status etree_lmhead_accept_tree(const etree_batch* b, const uint16_t* hidd
                             accept_len, path, out_tokens, nullptr, nullptr,
                             temperature > 0.f ? &tr : nullptr, workspace, workspace_bytes,
                             stream);
+}
+
+etree_status etree_lmhead_accept_timed(const etree_batch* b, const uint16_t* hidden,
+                                       const uint16_t* w_lm, int hidden_dim, int vocab,
+                                       float temperature, const float* q_draft, uint64_t seed,
+                                       uint64_t step, int32_t* accept_len, int32_t* path,
+                                       int32_t* out_tokens, int32_t* node_argmax,
+                                       float* node_gap, float* zbuf, int32_t zbuf_rows,
+                                       int32_t branching, void* const* marks, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  if (branching && (zbuf_rows < 0 || (zbuf_rows > 0 && !zbuf)))
+    return fail(ETREE_EINVAL, "zbuf_rows=%d with zbuf=%p", zbuf_rows, (void*)zbuf);
+  if (branching && zbuf && !aligned16(zbuf))
+    return fail(ETREE_EINVAL, "zbuf must be 16-byte aligned");
+  const TreeRows tr{zbuf, zbuf_rows};
+  return lmhead_accept_impl(b, hidden, w_lm, hidden_dim, vocab, temperature, q_draft, seed, step,
+                            accept_len, path, out_tokens, branching ? nullptr : node_argmax,
+                            branching ? nullptr : node_gap,
+                            (branching && temperature > 0.f) ? &tr : nullptr, workspace,
+                            workspace_bytes, stream, marks);
 }
 
 static etree_status kv_compact_impl(const etree_batch* b, const int32_t* accept_len,
@@ -829,9 +884,8 @@ static etree_status kv_compact_impl(const etree_batch* b, const int32_t* accept_
   p.max_pages = pg ? pg->max_pages : 0;
   p.page_shift = pg ? log2i(pg->page_size) : 0;
   p.cache_slots = pool_slots;
-  // the layers are spread over about 16 CTAs per SM (ETREE_COMPACT_PER_SM overrides)
-  const int per_sm = std::max(1, env_int("ETREE_COMPACT_PER_SM", 16));
-  cudaError_t e = launch_compact(p, per_sm * sm_count(), static_cast<cudaStream_t>(stream));
+  // the layers are spread over about 16 CTAs per SM
+  cudaError_t e = launch_compact(p, 16 * sm_count(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_kv_compact launch");
 }
 
@@ -872,10 +926,12 @@ etree_status etree_verify_attn_noalloc(const etree_batch* b, const uint16_t* q,
                                        int64_t cache_slots, int hq, int hkv, int head_dim,
                                        float scale, uint16_t* out, float* lse,
                                        int32_t* status_out, void* stream) {
-  etree_status st = check_batch(b);
+  // every host check runs before the shared array is touched: a rejected call changes nothing
+  etree_status st = check_attn_args(b, q, k_tree, v_tree, k_cache, v_cache, cache_slots, hq, hkv,
+                                    head_dim, scale, out, lse);
   if (st) return st;
-  if (hq < 1 || hkv < 1 || hq % hkv != 0 || hq / hkv > 64)
-    return fail(ETREE_EINVAL, "hq=%d, hkv=%d: need hq %% hkv == 0 and hq/hkv <= 64", hq, hkv);
+  if (status_out && ((uintptr_t)status_out & 3))
+    return fail(ETREE_EINVAL, "status_out must be 4-byte aligned");
   const size_t need = layout(b, hq, hkv, 0, 0).total;
   if (need > kStaticScratchBytes)
     return fail(ETREE_EINVAL,

@@ -86,8 +86,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // that runs out returns false.
 constexpr uint32_t kWaitCap = 1u << 21;
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitCap; ++i)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint32_t cap = kWaitCap) {
+  for (uint32_t i = 0; i < cap; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }

@@ -42,9 +42,6 @@ struct AttnParams {
   const int32_t* block_table;
   int max_pages, page_shift, cache_box;
 };
-cudaError_t launch_attn(const CUtensorMap& kc, const CUtensorMap& vc, const CUtensorMap& kt,
-                        const CUtensorMap& vt, const AttnParams& p, int nw, int stages,
-                        int n_total, cudaStream_t stream);
 cudaError_t launch_attn_combine(const AttnParams& p, int n_total, cudaStream_t stream);
 cudaError_t launch_attn_order(const int32_t* kv_len, int B, int32_t* order, cudaStream_t stream);
 cudaError_t launch_attn_tc(const CUtensorMap& q, const CUtensorMap& kc, const CUtensorMap& vc,
@@ -71,8 +68,10 @@ struct GemmParams {
   const int32_t* stop_row;
   const int32_t* stop_node;
   // Draw weights of the race pass per request: w = max(0, p - cval q); cval = 0 draws from p,
-  // cval < 0 marks a residual without positive weight (the bonus falls back to argmax p).
+  // cval < 0 marks a residual without positive weight (the bonus is drawn from p).
   const float* cval;
+  uint32_t* rfloor;                 // RACE: per request, the best (residual, p) keys published
+                                    // so far (fp32 bits; zeroed by the acceptance kernels)
   const float* lse2;
   const float* q_draft;
   uint64_t seed, step;
@@ -105,6 +104,7 @@ struct AcceptParams {
   __nv_bfloat16* hid2;
   int H;
   const float4* part2;
+  uint32_t* rfloor;                 // [B][2] race floors of the draw pass, zeroed per request
 };
 cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, int32_t* cnt,
                                  cudaStream_t s);

@@ -22,11 +22,11 @@
 //               nodes also write their logits out (the sibling residuals need whole rows);
 //   EPI_TOPK    per row and tile half: the 16 largest values and their ids (the low-rank
 //               candidate head's screen, lowrank.cu);
-//   EPI_RACE    per row and 128-id block: the block total of the draw's weights
-//               max(0, p - c q) (c = 0: p; c = 1: the residual after one rejection; larger c
-//               after sibling rejections), the id where the block's running sum passes u_b times
-//               that total, and the block's largest logit; the block race happens in
-//               bonus_kernel.
+//   EPI_RACE    per row and tile half: the leading entries of two exponential races over the
+//               vocabulary (key w_v / E_v, E_v = -log U_v), one over the draw's weights
+//               max(0, p - c q) (c = 1 after one rejection, larger c after sibling rejections)
+//               and one over p itself (used when c = 0, or when the residual has no positive
+//               weight); bonus_kernel takes the largest key over the tiles.
 #include "kernels.cuh"
 #include "philox.cuh"
 
@@ -91,6 +91,7 @@ struct TopK16 {
 // Per-row running state of the epilogue over one vocab tile.
 struct EpiRow {
   float r0 = -INFINITY, r2 = -INFINITY, r1f = 0.f;   // ARGMAX: top1, top2 | LSE: max, sum
+                                                     // RACE: best keys (residual, p)
   int r1 = -1, r3 = -1;                              // ARGMAX: id | RACE: ids (residual, p)
   int ct = -1;                                       // LSE: child token of the row
   float zc = 0.f;                                    // LSE: its logit
@@ -98,8 +99,63 @@ struct EpiRow {
   int unode = 0, req = 0;                            // RACE: stop node, request
   float c = 0.f;                                     // RACE: residual offset (cval)
   float L2 = 0.f;                                    // RACE: log2 sum 2^(z k)
+  float fr = 0.f, fp = 0.f;                          // RACE: the row's published floors
   const float* qrow = nullptr;                       // RACE: q_draft row
 };
+
+// Screening margin of the race: an id is skipped only when its key is certainly below the
+// threshold, allowing for the rounding of -log U (a few ulp) and of the quotient.
+constexpr float kRaceShrink = 1.0f - 1.0f / 1048576.0f;
+
+// The exponential race over W consecutive ids (col0 a multiple of 8).  Each id's key is
+// w_v / E_v with E_v = -log U_v > 0 (U_v the stream-0 uniform of (id, stop node, request)), and
+// the race keeps the largest key, the lower id on equal keys.  Since E_v >= 1 - U_v, an id whose
+// weight is below threshold * (1 - U_v) cannot beat the threshold and skips the logarithm; the
+// threshold is the larger of this thread's best key and the floor other threads published for
+// the row (keys of real ids, so never above the row's final maximum).
+template <int W>
+__device__ __forceinline__ void race_chunk(const GemmParams& p, EpiRow& st, const float (&z)[W],
+                                           const float (&q)[W], int col0) {
+  const bool resid = st.c > 0.f;
+  float thr_p = fmaxf(st.fp, st.r2 > 0.f ? st.r2 : 0.f) * kRaceShrink;
+  float thr_r = fmaxf(st.fr, st.r0 > 0.f ? st.r0 : 0.f) * kRaceShrink;
+#pragma unroll
+  for (int g = 0; g < W / 8; ++g) {
+    const int c0 = col0 + 8 * g;
+    if (c0 >= p.V) break;
+    float u[8];
+    uniforms8(p.seed, p.step, (uint32_t)(c0 >> 3), (uint32_t)st.unode, (uint32_t)st.req, 0u, u);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int v = c0 + e;
+      if (v >= p.V) break;
+      const float pv = exp2f(z[8 * g + e] * p.k_log2 - st.L2);
+      const float wr = resid ? fmaxf(pv - st.c * q[8 * g + e], 0.f) : 0.f;
+      const float d = 1.f - u[e];                      // exact: U has 24 significant bits
+      const bool cp = pv > 0.f && pv >= thr_p * d;
+      const bool cr = wr > 0.f && wr >= thr_r * d;
+      if (cp || cr) {
+        const float E = -logf(u[e]);
+        if (cp) {
+          const float key = __fdiv_rn(pv, E);
+          if (key > st.r2) {
+            st.r2 = key;
+            st.r3 = v;
+            thr_p = fmaxf(thr_p, key * kRaceShrink);
+          }
+        }
+        if (cr) {
+          const float key = __fdiv_rn(wr, E);
+          if (key > st.r0) {
+            st.r0 = key;
+            st.r1 = v;
+            thr_r = fmaxf(thr_r, key * kRaceShrink);
+          }
+        }
+      }
+    }
+  }
+}
 
 // Folds W consecutive logits v (columns col0 .. col0+W-1) into the row state.
 template <int EPI, int W>
@@ -156,12 +212,13 @@ __device__ __forceinline__ void store_logits(const GemmParams& p, float* zdst, c
   }
 }
 
-// Draft probabilities of 32 consecutive ids (zero past the vocabulary).
-__device__ __forceinline__ void load_q32(const GemmParams& p, const float* qrow, int col0,
-                                         float (&q)[32]) {
+// Draft probabilities of W consecutive ids (zero past the vocabulary).
+template <int W>
+__device__ __forceinline__ void load_q(const GemmParams& p, const float* qrow, int col0,
+                                       float (&q)[W]) {
   if ((p.V & 3) == 0) {
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
+    for (int j = 0; j < W; j += 4) {
       float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
       if (col0 + j < p.V) t = __ldg(reinterpret_cast<const float4*>(qrow + col0 + j));
       q[j] = t.x;
@@ -171,7 +228,7 @@ __device__ __forceinline__ void load_q32(const GemmParams& p, const float* qrow,
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) q[j] = col0 + j < p.V ? __ldg(qrow + col0 + j) : 0.f;
+    for (int j = 0; j < W; ++j) q[j] = col0 + j < p.V ? __ldg(qrow + col0 + j) : 0.f;
   }
 }
 
@@ -355,82 +412,27 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         st.req = grow;
         st.L2 = p.lse2[g];
         st.qrow = p.q_draft + (size_t)g * p.V;
+        st.fr = __uint_as_float(__ldcg(p.rfloor + 2 * grow));
+        st.fp = __uint_as_float(__ldcg(p.rfloor + 2 * grow + 1));
       }
-      if constexpr (EPI == EPI_RACE) {
-        // This half owns one whole 128-id block (columns half*128 .. +127 of the tile).
-        // Pass 1 turns the logits into the draw's weights -- max(0, p - q) after a rejection,
-        // p otherwise -- sums them in increasing id order, tracks the block's largest logit,
-        // and writes the weights back over the logits in TMEM.  Pass 2 rescans those weights
-        // for the first id whose running sum passes u_b times the block total.
-        static_assert(BN == 256, "the two-level draw works on 128-id blocks");
-        const int blk = nt * 2 + half;
-        const int colb = blk * 128;
-        const uint32_t tcol = tbase + half * 128;
-        float W = 0.f, zmax = -INFINITY;
-        int zarg = -1;
-        float qa[32], qb[32];
-        const bool md = st.c > 0.f;                     // q enters the weights
-        if (active && md) load_q32(p, st.qrow, colb, qa);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float (&q)[32] = (c & 1) ? qb : qa;
-          float (&qn)[32] = (c & 1) ? qa : qb;
-          if (active && md && c < 3) load_q32(p, st.qrow, colb + (c + 1) * 32, qn);
-          float v[32];
-          tmem_ld32(tcol + c * 32, v);
-          if (active) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int col = colb + c * 32 + j;
-              float w = 0.f;
-              if (col < p.V) {
-                if (v[j] > zmax) {
-                  zmax = v[j];
-                  zarg = col;
-                }
-                const float pv = exp2f(v[j] * p.k_log2 - st.L2);
-                w = md ? fmaxf(pv - st.c * q[j], 0.f) : (st.c < 0.f ? 0.f : pv);
-                W += w;
-              }
-              v[j] = w;
-            }
-          }
-          tmem_st32(tcol + c * 32, v);
-        }
-        float u[8];
-        uniforms8(p.seed, p.step, (uint32_t)(blk >> 3), (uint32_t)st.unode, (uint32_t)st.req, 3u,
-                  u);
-        float ub = u[0];
-#pragma unroll
-        for (int e = 1; e < 8; ++e)
-          if ((blk & 7) == e) ub = u[e];
-        const float thr = ub * W;
-        float run = 0.f;
-        int pick = -1, last = -1;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(tcol + c * 32, v);
-          if (active) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              run += v[j];
-              if (v[j] > 0.f) last = colb + c * 32 + j;
-              if (pick < 0 && run > thr) pick = colb + c * 32 + j;
-            }
-          }
-        }
-        st.r0 = W;
-        st.r1 = pick >= 0 ? pick : last;
-        st.r2 = zmax;
-        st.r3 = zarg;
-      } else {
+      {
 #pragma unroll 1
         for (int c = half; c < kChunks; c += 2) {
           float v[32];
           tmem_ld32(tbase + c * 32, v);
           if constexpr (EPI == EPI_TOPK) {
             if (active) tk.push_chunk<32>(v, nt * BN + c * 32, p.V, tfloor);
+          } else if constexpr (EPI == EPI_RACE) {
+            if (active) {
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {          // two 16-id halves keep registers low
+                const int col0 = nt * BN + c * 32 + 16 * hh;
+                float q[16];
+                if (st.c > 0.f) load_q<16>(p, st.qrow, col0, q);
+                race_chunk<16>(p, st, *reinterpret_cast<const float(*)[16]>(v + 16 * hh), q,
+                               col0);
+              }
+            }
           } else {
             if (active) epi_chunk<EPI, 32>(p, st, v, nt * BN + c * 32);
           }
@@ -442,6 +444,12 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
             tmem_ld16(tbase + kChunks * 32, v);
             if constexpr (EPI == EPI_TOPK) {
               if (active) tk.push_chunk<16>(v, nt * BN + kChunks * 32, p.V, tfloor);
+            } else if constexpr (EPI == EPI_RACE) {
+              if (active) {
+                float q[16];
+                if (st.c > 0.f) load_q<16>(p, st.qrow, nt * BN + kChunks * 32, q);
+                race_chunk<16>(p, st, v, q, nt * BN + kChunks * 32);
+              }
             } else {
               if (active) epi_chunk<EPI, 16>(p, st, v, nt * BN + kChunks * 32);
             }
@@ -456,6 +464,10 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       // still means lowest id) and is written once, after the CTA's last tile.
       if (EPI == EPI_TOPK && active && tk.v[15] > tfloor)   // 16 values >= it: a valid bound
         atomicMax(p.tkth + grow, enc_order(tk.v[15]));
+      if (EPI == EPI_RACE && active) {                  // positive keys order as their bits
+        if (st.r1 >= 0 && st.r0 > st.fr) atomicMax(p.rfloor + 2 * grow, __float_as_uint(st.r0));
+        if (st.r3 >= 0 && st.r2 > st.fp) atomicMax(p.rfloor + 2 * grow + 1, __float_as_uint(st.r2));
+      }
       if (EPI == EPI_TOPK && active && (!p.per_cta || tile + (int)gridDim.x >= p.num_tiles)) {
         float2* dst = p.topk + ((size_t)grow * p.n_parts * 2 +
                                 (p.per_cta ? (int)blockIdx.x : nt) * 2 + half) * 16;
@@ -468,7 +480,7 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           out = make_float4(st.r0, __int_as_float(st.r1), st.r2, 0.f);
         else if (EPI == EPI_LSE)
           out = make_float4(st.r0, st.r1f, 0.f, 0.f);
-        else
+        else                                            // RACE: (key, id) residual, p
           out = make_float4(st.r0, __int_as_float(st.r1), st.r2, __int_as_float(st.r3));
         p.part[(size_t)grow * p.n_parts * 2 + (p.per_cta ? (int)blockIdx.x : nt) * 2 + half] = out;
         if (EPI == EPI_LSE && st.found) p.zchild[grow] = st.zc;
@@ -488,9 +500,6 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
 static const int kWidths[] = {256, 224, 208, 192, 176, 160, 144, 128};
 
 int lmhead_pick_bn(int M, int V, int grid) {
-  const int forced = getenv("ETREE_BN") ? atoi(getenv("ETREE_BN")) : 0;
-  for (int bn : kWidths)
-    if (bn == forced) return bn;
   // With several row tiles the GEMM is tensor-bound and the widest tile is the most efficient.
   // With one row tile it streams W once: time ~ (rounds of tiles per CTA) x (tile width + a
   // fixed per-tile cost of ~48 columns), so pick the width that balances the last round.
@@ -549,13 +558,11 @@ cudaError_t launch_lmhead(int epi, int bn, int bm, const CUtensorMap& ta, const 
   if (bm == 64) {
     if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX, 64>(bn, ta, tb, p, grid, stream);
     if (epi == EPI_LSE) return launch_epi<EPI_LSE, 64>(bn, ta, tb, p, grid, stream);
-    if (bn != 256) return cudaErrorInvalidValue;
-    return launch_bn<EPI_RACE, 256, 64>(ta, tb, p, grid, stream);
+    return launch_epi<EPI_RACE, 64>(bn, ta, tb, p, grid, stream);
   }
   if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX, 128>(bn, ta, tb, p, grid, stream);
   if (epi == EPI_LSE) return launch_epi<EPI_LSE, 128>(bn, ta, tb, p, grid, stream);
-  if (bn != 256) return cudaErrorInvalidValue;
-  return launch_bn<EPI_RACE, 256, 128>(ta, tb, p, grid, stream);
+  return launch_epi<EPI_RACE, 128>(bn, ta, tb, p, grid, stream);
 }
 
 }  // namespace etree

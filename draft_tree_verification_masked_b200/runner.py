@@ -11,7 +11,8 @@ import torch
 import numpy as np
 
 from . import (etree_device_status, etree_kv_compact, etree_kv_compact_paged,
-               etree_lmhead_accept, etree_lmhead_accept_tree, etree_verify_attn,
+               etree_lmhead_accept, etree_lmhead_accept_timed, etree_lmhead_accept_tree,
+               etree_verify_attn,
                etree_verify_attn_paged, etree_workspace_init, etree_workspace_size, make_batch)
 
 
@@ -50,10 +51,12 @@ class DeviceStep:
     """tree: None picks the branching-tree sampler (etree_lmhead_accept_tree) when T > 0 and a
     node has two or more children; zbuf_rows overrides the size of its logit buffer.
     page_size: lay the caches out in pages of that many tokens at shuffled pool pages and use
-    the paged attention and compaction calls (the pools replace k_cache / v_cache)."""
+    the paged attention and compaction calls (the pools replace k_cache / v_cache).
+    kv_len_max: the batch's host-side bound on kv_len (default: the largest kv_len); a looser
+    bound is valid and sizes the attention grid for it."""
 
     def __init__(self, wl, device: str = "cuda", n_layers: int = 1, tree=None, zbuf_rows=None,
-                 page_size=None):
+                 page_size=None, kv_len_max=None):
         self.wl = wl
         self.device = device
         dev = torch.device(device)
@@ -95,7 +98,8 @@ class DeviceStep:
             v.copy_(t)
             setattr(self, name, v)
         self.batch = make_batch(self.cu_nodes, self.parent, self.tokens, self.kv_len,
-                                self.slot_base, self.slot_cap, wl.n_max, wl.kv_len_max)
+                                self.slot_base, self.slot_cap, wl.n_max,
+                                wl.kv_len_max if kv_len_max is None else int(kv_len_max))
         self.k_cache = up(self.paged.k_pool if self.paged else wl.k_cache)
         self.v_cache = up(self.paged.v_pool if self.paged else wl.v_cache)
         self.w_lm = up(wl.w_lm)
@@ -154,6 +158,13 @@ class DeviceStep:
         etree_lmhead_accept(self.batch, self.hidden, self.w_lm, self.wl.temperature,
                             self.q_draft, self.wl.seed, self.wl.step, self.accept_len, self.path,
                             self.out_tokens, self.node_argmax, self.node_gap, self.ws, stream)
+
+    def lmhead_marked(self, marks, stream=None):
+        """The LM-head call with its phase marks (see etree_lmhead_accept_timed)."""
+        etree_lmhead_accept_timed(self.batch, self.hidden, self.w_lm, self.wl.temperature,
+                                  self.q_draft, self.wl.seed, self.wl.step, self.accept_len,
+                                  self.path, self.out_tokens, self.node_argmax, self.node_gap,
+                                  self.zbuf, self.tree, marks, self.ws, stream)
 
     def compact(self, stream=None):
         if self.paged:

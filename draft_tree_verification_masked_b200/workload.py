@@ -17,7 +17,10 @@ vocab 151936).  The synthetic recipe and every reading it takes are listed in th
   N(0,1) plus GAMMA times the unit vector of LM-head row t*_u, which makes t*_u the target's
   argmax with overwhelming probability.  A child carries its parent's planted token with the
   configured match probability (at most one sibling does), else a uniform random token distinct
-  from its siblings and from t*_u.
+  from its siblings and from t*_u.  With `target_argmax` given (a function of the hidden rows
+  and the head that returns each row's argmax, supplied by the caller), the hidden states are
+  plain N(0,1) and t*_u is that function's answer instead: the natural recipe, whose top-1 /
+  top-2 margins are those of N(0, 1.43) logits over the whole vocabulary.
 * T>0: target logits come out N(0,2) by drawing W ~ N(0, 2/sqrt(hidden)); draft distributions
   are softmax of N(0,2) logits and each draft token is sampled from its parent's draft
   distribution, independently for siblings (chains and branching trees alike).
@@ -246,8 +249,13 @@ def _draft_tokens_greedy(parent: np.ndarray, planted: np.ndarray, vocab: int, ma
     return tok
 
 
-def generate(name: str, *, seed: int | None = None, step: int = 0, **overrides) -> Workload:
-    """Build the named workload (overrides replace config fields, e.g. vocab=4224)."""
+def generate(name: str, *, seed: int | None = None, step: int = 0, target_argmax=None,
+             **overrides) -> Workload:
+    """Build the named workload (overrides replace config fields, e.g. vocab=4224).
+
+    target_argmax (T = 0 only): callable(hidden bf16 [n, H], w_lm bf16 [V, H]) -> int array [n]
+    of each row's argmax; when given, hidden states are unplanted N(0, 1) and the drafts follow
+    the returned argmaxes (see the module notes)."""
     cfg = dict(CONFIGS[name])
     cfg.update(overrides)
     seed = config_seed(name) if seed is None else int(seed)
@@ -297,15 +305,20 @@ def generate(name: str, *, seed: int | None = None, step: int = 0, **overrides) 
         w_lm = normal_bf16((V, H), cfg["w_sigma"], seed, "w_lm")
         h = normal_f32(ntot * H, 1.0, seed, "hidden").reshape(ntot, H)
         tokens = np.empty(ntot, dtype=np.int32)
+        if target_argmax is not None:
+            hidden = torch.from_numpy(h).to(torch.bfloat16)
+            planted[:] = np.asarray(target_argmax(hidden, w_lm), dtype=np.int32)
         for r in range(B):
             a, b = int(cu[r]), int(cu[r + 1])
-            planted[a:b] = _rng(seed, "plant", r).integers(V, size=b - a)
+            if target_argmax is None:
+                planted[a:b] = _rng(seed, "plant", r).integers(V, size=b - a)
             tokens[a:b] = _draft_tokens_greedy(parent[a:b], planted[a:b], V, cfg["match"],
                                                _rng(seed, "tokens", r))
-        rows = w_lm[torch.from_numpy(planted.astype(np.int64))].float().numpy()
-        rows /= np.linalg.norm(rows, axis=1, keepdims=True)
-        h += np.float32(GAMMA) * rows
-        hidden = torch.from_numpy(h).to(torch.bfloat16)
+        if target_argmax is None:
+            rows = w_lm[torch.from_numpy(planted.astype(np.int64))].float().numpy()
+            rows /= np.linalg.norm(rows, axis=1, keepdims=True)
+            h += np.float32(GAMMA) * rows
+            hidden = torch.from_numpy(h).to(torch.bfloat16)
     else:
         w_lm = normal_bf16((V, H), 2.0 / np.sqrt(H), seed, "w_lm")
         hidden = normal_bf16((ntot, H), 1.0, seed, "hidden")

@@ -98,7 +98,12 @@ size_t etree_workspace_size(const etree_batch *batch, int hq, int hkv, int head_
 etree_status etree_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * Tree-masked GQA attention.  For node i of request r and query head h (KV head h / (hq/hkv)):
+ * Tree-masked GQA attention.  The target scores every drafted token in one parallel forward, and
+ * a draft tree lets that pass cover several candidate paths ("Eagle-4 Released: Outpaces DFlash2
+ * and DSpark ...", section "Technical Background"); each node therefore sees its request's cache
+ * and exactly its own ancestors.  The KV cache stays unquantized bf16 ("EAGLE-4 官方推理代码发布
+ * ...", paragraph on hardware coverage and limits).
+ * For node i of request r and query head h (KV head h / (hq/hkv)):
  * keys = the kv_len[r] cached positions (pooled rows slot_base[r] + t) followed by the tree nodes
  * j with j == i or j an ancestor of i;  out = softmax(scale * q k^T) v;  lse = log sum exp.
  *   q        [n_total][hq][head_dim]  bf16
@@ -123,13 +128,18 @@ etree_status etree_verify_attn(const etree_batch *batch, const uint16_t *q,
  * some plugin hosts hand their plugins no allocator at all.  Such callers cannot size and pass a
  * workspace.  The paper has no counterpart: this is a deployment convenience.
  * Same arguments, computation and output as etree_verify_attn, without a workspace: the split
- * partials and the status words live in one static 32 MiB device array inside the library, which
- * every device that loads the library holds until the process exits.  The call allocates nothing
- * (no cudaMalloc / cudaFree, no allocating library routine).
- *  - A batch that needs more than 32 MiB of scratch (etree_workspace_size with hidden_dim = 0 and
+ * partials and the status words live in one static 16 MiB device array inside the library, which
+ * every context that loads the library holds until the context ends.  16 MiB covers the largest
+ * KV split the planner makes at the shapes this library is measured on (about 12 MiB at a
+ * 128K-token cache, 40/8 heads, 16 nodes).  The call allocates nothing (no cudaMalloc / cudaFree,
+ * no allocating library routine).
+ *  - Every host-side check of etree_verify_attn runs first; a rejected call touches nothing.
+ *  - A batch that needs more than 16 MiB of scratch (etree_workspace_size with hidden_dim = 0 and
  *    vocab = 0) is rejected with ETREE_EINVAL before any device work; use etree_verify_attn.
- *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress) and
- *    caches it; make that first call before any stream capture.
+ *  - The first call in a CUDA context looks up the array's device address there
+ *    (cudaGetSymbolAddress) and caches it under the context's unique id, so a device reset or a
+ *    context of the caller's own gets its own lookup; make that first call before any stream
+ *    capture.
  *  - Every call clears the status words, then reuses the array, which keeps the last call's
  *    contents.  Calls whose kernels overlap on the GPU (other streams, other threads) race on
  *    the array: serialise them.
@@ -152,9 +162,10 @@ etree_status etree_verify_attn_noalloc(const etree_batch *batch, const uint16_t 
  * the kernel's key tile are loaded page by page.  block_table is a device int32 array
  * [B][max_pages]; only entries covering positions below kv_len[r] are read for keys.  An entry
  * outside [0, num_pages) records ETREE_EDEVICE (detail 11) and its keys read as zeros;
- * kv_len[r] > max_pages * page_size records ETREE_EDEVICE (detail 3).  Needs the tcgen05
- * kernel (ETREE_ATTN=mma returns ETREE_EUNSUPPORTED).  Other arguments, workspace and errors as
- * etree_verify_attn, with num_pages * page_size in place of cache_slots.
+ * kv_len[r] > max_pages * page_size records ETREE_EDEVICE (detail 3).  Other arguments,
+ * workspace and errors as etree_verify_attn, with num_pages * page_size in place of cache_slots.
+ * (Paged caches are how the engines the pages plug into hold KV: "EAGLE-4 官方推理代码发布 ...",
+ * section on the harness being a plug-in for SGLang and vLLM.)
  */
 etree_status etree_verify_attn_paged(const etree_batch *batch, const int32_t *block_table,
                                      int32_t max_pages, int32_t page_size, const uint16_t *q,
@@ -165,14 +176,22 @@ etree_status etree_verify_attn_paged(const etree_batch *batch, const int32_t *bl
                                      size_t workspace_bytes, void *stream);
 
 /*
- * LM head + acceptance.  z = hidden W^T (fp32 accumulate over bf16 inputs) for every node row.
+ * LM head + acceptance.  The target keeps the longest drafted prefix consistent with its own
+ * distribution and adds one token of its own after the first rejection ("Eagle-4 Released ...",
+ * section "Technical Background"); at T > 0 the rule must keep the target's output distribution
+ * ("EAGLE-4 官方推理代码发布 ...", section on sizing the tree by measured cost).  The vocab head
+ * is the costly part of an LM head (65.4% of a draft forward: "EAGLE-4 是什麼？...",
+ * aiposthub.com, Fig. 2), so its logits are reduced where they are computed and never stored.
+ * z = hidden W^T (fp32 accumulate over bf16 inputs) for every node row.
  *  T == 0 (greedy): t*(u) = argmax z_u (lowest id on ties).  From the root, repeatedly move to
  *    the lowest-index child whose token equals t*(current); the node where no child matches
  *    stops the walk and t* there is the bonus token.
  *  T > 0 (chains only, every node has <= 1 child): p_u = softmax(z_u / T); node k's token x was
  *    drafted from q_draft row k-1; it is accepted iff U * q(x) < p(x), U a seeded uniform.  At
  *    the first rejection (node u) the bonus is drawn from norm(max(0, p_u - q_u)); when all are
- *    accepted it is drawn from p of the last node.  Draws use an exponential race with
+ *    accepted it is drawn from p of the last node; a residual with no positive weight (p <= q
+ *    everywhere: p = q up to rounding) is answered by a draw from p_u.  Draws are exponential
+ *    races over every vocab id (the id with the largest w_v / E_v, E_v = -log U_v) with
  *    Philox4x64-10 uniforms keyed by (seed, step) and countered by (vocab id / 8, node, request,
  *    stream), so results are reproducible bit for bit.  A branching tree records
  *    ETREE_EUNSUPPORTED (detail 5, "not a chain") and that request accepts nothing; sample
@@ -205,8 +224,8 @@ etree_status etree_lmhead_accept(const etree_batch *batch, const uint16_t *hidde
  * N(c) = sum_v max(0, p_u(v) - c q_u(v)) per rejection.  An accepted child becomes the node
  * whose children are tested next.  The walk stops at a leaf or when all children of a node are
  * rejected; the bonus is drawn there from max(0, p_u - c q_u) (from p_u when nothing was
- * rejected there) with the two-level draw of etree_lmhead_accept; a residual without positive
- * weight falls back to argmax p_u.  On chains the results equal etree_lmhead_accept's.
+ * rejected there) with the exponential race of etree_lmhead_accept; a residual without positive
+ * weight is answered by a draw from p_u.  On chains the results equal etree_lmhead_accept's.
  *   zbuf       caller-owned device buffer [zbuf_rows][vocab] fp32, 16-byte aligned: the logits
  *              of every node with two or more children are written there (in node order),
  *              because each sibling rejection needs a pass over the whole row.  At most
@@ -226,7 +245,31 @@ etree_status etree_lmhead_accept_tree(const etree_batch *batch, const uint16_t *
                                       void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * KV compaction.  For each of n_layers layers and each request r with a = accept_len[r]:
+ * etree_lmhead_accept (branching = 0) or etree_lmhead_accept_tree (branching = 1, with zbuf and
+ * zbuf_rows; node_argmax / node_gap are then unused), with phase marks for measuring where the
+ * call's device time goes.  marks (host array of 4 cudaEvent_t, each may be NULL; the whole
+ * array may be NULL) are recorded on `stream` after: [0] the set-up kernels before the first
+ * GEMM, [1] the first GEMM (every node row), [2] the acceptance kernels, [3] the draw GEMM over
+ * the stop rows (T > 0; at T = 0 marks 2 and 3 coincide).  Results are identical to the
+ * unmarked calls; the event records keep kernels from overlapping their neighbours' set-up, so
+ * time whole steps with the unmarked calls.  The pages report end-to-end figures only; this
+ * call exists to report the second (draw) pass separately from the algorithmic first pass.
+ */
+etree_status etree_lmhead_accept_timed(const etree_batch *batch, const uint16_t *hidden,
+                                       const uint16_t *w_lm, int hidden_dim, int vocab,
+                                       float temperature, const float *q_draft, uint64_t seed,
+                                       uint64_t step, int32_t *accept_len, int32_t *path,
+                                       int32_t *out_tokens, int32_t *node_argmax,
+                                       float *node_gap, float *zbuf, int32_t zbuf_rows,
+                                       int32_t branching, void *const *marks, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
+/*
+ * KV compaction.  Requests accept different numbers of drafted tokens each step, and keeping
+ * their caches aligned under continuous batching is the engineering difficulty the pages name
+ * ("Eagle-4 Released ...", section "Community Reaction and Future Outlook"): the accepted nodes'
+ * K/V move into the request's next contiguous slots.
+ * For each of n_layers layers and each request r with a = accept_len[r]:
  *   cache[slot_base[r] + kv_len[r] + k] <- tree[cu_nodes[r] + path[r][k]],  k = 0 .. a,
  * for K and V, then kv_len_out[r] = kv_len[r] + a + 1 (the bonus token's K/V come next step).
  * path is the [B][64] array etree_lmhead_accept writes; all 64 entries of a row are read.
@@ -370,10 +413,9 @@ const char *etree_last_error(void);
 
 /*
  * The launch plan etree_verify_attn uses for this batch and head shape (host-only, no device
- * work): which kernel (1 = tcgen05/TMEM kernel, the default; 0 = warp-level mma.sync kernel,
- * selected by the environment variable ETREE_ATTN=mma), query rows per CTA, row blocks per
- * (request, KV head), KV splits, 64-key tiles per split, and the number of kernels the call
- * launches (1, or 2 with the split combine).  Any output pointer may be NULL.
+ * work): the kernel (always 1, the tcgen05/TMEM kernel), query rows per CTA, row blocks per
+ * (request, KV head), KV splits, key tiles per split, and the number of kernels the call
+ * launches.  Any output pointer may be NULL.
  */
 etree_status etree_attn_plan(const etree_batch *batch, int hq, int hkv, int32_t *kernel,
                              int32_t *rows_per_cta, int32_t *row_blocks, int32_t *splits,

@@ -248,15 +248,15 @@ def test_lm_head_workspace_is_the_documented_regions():
     """Without attention (hq = 0) the workspace is the 256-byte status header plus, each rounded
     up to 256 bytes: LM-head summaries float4 [n_total][2 ceil(V/128)], child token, child logit
     and log2-sum-exp per node, stop row, stop node and offset per request, stop-row hiddens
-    bf16 [B][H], draw summaries float4 [B][2 ceil(V/128)], arrival counters [B], and per node
-    the child count, logit-row index and parent-row logit."""
+    bf16 [B][H], draw summaries float4 [B][2 ceil(V/128)], the draw's race floors [B][2],
+    arrival counters [B], and per node the child count, logit-row index and parent-row logit."""
     def up(x):
         return (x + 255) // 256 * 256
 
     for B, nt, H, V in [(1, 16, 1024, 4096), (64, 1024, 5120, 151936), (3, 5, 64, 300)]:
         tiles = 2 * ((V + 127) // 128)
         regions = [nt * tiles * 16, nt * 4, nt * 4, nt * 4, B * 4, B * 4, B * 4, B * H * 2,
-                   B * tiles * 16, B * 4, nt * 4, nt * 4, nt * 4]
+                   B * tiles * 16, B * 8, B * 4, nt * 4, nt * 4, nt * 4]
         off = 256
         for r in regions:
             off = up(off + r)

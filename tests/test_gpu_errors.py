@@ -25,10 +25,18 @@ def _still_works():
 
 
 def test_malformed_parent_sets_device_status():
+    """A malformed parent array reports ETREE_EDEVICE (detail 1) and that request is answered
+    like any request without a valid tree: nothing accepted, path and tokens all -1 (no bonus
+    token that a caller might emit before reading the status); the other request runs."""
     wl, dev = _dev()
     dev.parent[int(wl.cu_nodes[1]) + 3] = 7          # parent not below its child
+    dev.accept_len.fill_(7)
     dev.step()
     assert dev.status() == (EDEVICE, 1)
+    res = dev.results()
+    assert res["accept_len"][1] == 0
+    assert (res["path"][1] == -1).all() and (res["out_tokens"][1] == -1).all()
+    assert res["out_tokens"][0][int(res["accept_len"][0])] >= 0
     assert dev.status() == (0, 0)                     # read clears
     _still_works()
 

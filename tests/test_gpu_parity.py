@@ -1,20 +1,30 @@
 """GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same seeded inputs.
 
-Small cases compare every output; full-size workloads (the launch configuration the benchmark
-times) compare every output the oracle can afford and sampled attention rows otherwise.
-"""
-import os
+Every workload is compared at full size, in the launch configuration the benchmark times: every
+request's acceptance outputs, compacted rows and every attention row.  Other launch plans (KV
+split counts, 32- and 64-key tiles, LM-head row tiles) are reached through the shapes that make
+the library's planner choose them, which etree_attn_plan reports.
 
+Near-ties (a decision that the fp32 and fp64 arithmetic can legitimately take differently:
+a top-1 / top-2 logit gap under 1e-3 at T = 0, a sampling comparison within rounding at T > 0)
+are replayed, counted and logged in the session summary.  Each test allows at most one excused
+request: the chance of even one is about 1e-5 per decision (an argmax flips only when the gap is
+within the fp32 error of the logits, a few 1e-6; a sampling decision only when the fp64
+quantities it compares agree to 1e-5), far below one per test.
+"""
 import numpy as np
 import pytest
 import torch
 
+import draft_tree_verification_masked_b200 as et
 from draft_tree_verification_masked_b200 import workload as W
 from draft_tree_verification_masked_b200.runner import DeviceStep
 
 from . import _parity as P
 
 pytestmark = pytest.mark.gpu
+
+MAX_EXCUSED = 1
 
 
 def _run(wl, n_layers=1, **kw):
@@ -25,19 +35,30 @@ def _run(wl, n_layers=1, **kw):
     return dev, dev.results()
 
 
-def _full_check(wl, attn_rows=None, requests=None, **kw):
-    dev, res = _run(wl, **kw)
-    P.attn_compare(wl, dev, rows=attn_rows)
-    reqs = list(range(wl.B)) if requests is None else requests
+def _accept_check(wl, dev, res, reqs, label):
     if wl.temperature == 0.0:
         excused, near, ores = P.greedy_compare(wl, res, reqs)
     elif dev.tree:
         excused, near, ores = P.tree_compare(wl, res, reqs)
     else:
         excused, near, ores = P.chain_compare(wl, res, reqs)
+    P.log_near(label, wl, res, ores, reqs, near)
+    assert near <= MAX_EXCUSED, near
+    return excused, ores
+
+
+def _full_check(wl, attn_rows=None, requests=None, label=None, **kw):
+    dev, res = _run(wl, **kw)
+    P.attn_compare(wl, dev, rows=attn_rows)
+    reqs = list(range(wl.B)) if requests is None else requests
+    excused, ores = _accept_check(wl, dev, res, reqs, label or wl.name)
     P.compact_compare(wl, dev, ores, reqs, excused)
-    assert near <= max(1, len(reqs) // 10), near
     return dev, res
+
+
+def _plan(wl, kv_len_max=None):
+    dev_batch = DeviceStep(wl, kv_len_max=kv_len_max).batch
+    return et.etree_attn_plan(dev_batch, wl.hq, wl.hkv)
 
 
 def test_tiny_config():
@@ -50,22 +71,15 @@ def test_dense27b_single_request_full_size():
 
 @pytest.mark.parametrize("name", ["long32k", "long128k"])
 def test_long_context(name):
-    wl = W.generate(name)
-    _full_check(wl, attn_rows=P.sample_rows(wl, 40))
+    _full_check(W.generate(name))
 
 
 def test_batch64():
-    wl = W.generate("batch64")
-    g = np.random.default_rng(1)
-    reqs = sorted(g.choice(wl.B, 8, replace=False).tolist())
-    _full_check(wl, attn_rows=P.sample_rows(wl, 4), requests=reqs)
+    _full_check(W.generate("batch64"))
 
 
 def test_conc512_stochastic_chains():
-    wl = W.generate("conc512")
-    g = np.random.default_rng(2)
-    reqs = sorted(g.choice(wl.B, 24, replace=False).tolist())
-    _full_check(wl, attn_rows=P.sample_rows(wl, 1), requests=reqs)
+    _full_check(W.generate("conc512"))
 
 
 def test_ragged_trees_and_lengths():
@@ -87,10 +101,13 @@ def test_chain_of_64_and_single_node():
     _full_check(wl)
 
 
-@pytest.mark.parametrize("nsplit", ["1", "2", "3", "7"])
-def test_split_count_does_not_change_results(nsplit, monkeypatch):
-    monkeypatch.setenv("ETREE_NSPLIT", nsplit)
-    wl = W.generate("tiny", B=2, kv_len=[1000, 333], hidden=256, vocab=512)
+# KV lengths of a two-request tiny batch (16-node trees, 2 KV heads) whose plan splits the keys
+# 1, 2, 3 and 7 ways (64-key tiles: tiles = ceil(L / 64) + 1, splits = min(37, tiles / 4)).
+@pytest.mark.parametrize("nsplit,kv", [(1, [300, 100]), (2, [500, 64]), (3, [800, 333]),
+                                       (7, [1700, 1000])])
+def test_split_count_does_not_change_results(nsplit, kv):
+    wl = W.generate("tiny", B=2, kv_len=kv, hidden=256, vocab=512)
+    assert _plan(wl)["splits"] == nsplit
     _full_check(wl)
 
 
@@ -104,12 +121,6 @@ def test_many_row_tiles_and_ragged_vocab():
 def test_stochastic_chains_small(T):
     wl = W.generate("conc512", B=37, n_nodes=[4, 5, 6, 1, 2] * 7 + [4, 4], depth=5,
                     depth_min=5, kv_len=(20, 400), hidden=512, vocab=4096 + 3, temperature=T)
-    _full_check(wl)
-
-
-def test_four_stage_kv_ring(monkeypatch):
-    monkeypatch.setenv("ETREE_STAGES", "4")
-    wl = W.generate("tiny", B=2, kv_len=[700, 64], hidden=256, vocab=512)
     _full_check(wl)
 
 
@@ -164,28 +175,11 @@ def test_multi_layer_compaction_against_oracle():
     assert np.array_equal(dev.kv_len_out.cpu().numpy(), newlen)
 
 
-def test_env_is_clean():
-    assert "ETREE_NSPLIT" not in os.environ
-
-
-@pytest.mark.parametrize("case", ["tiny", "ragged"])
-def test_warp_mma_attention_kernel(case, monkeypatch):
-    """The warp-level mma.sync attention kernel, kept for comparison, against the oracle."""
-    monkeypatch.setenv("ETREE_ATTN", "mma")
-    if case == "tiny":
-        wl = W.generate("tiny")
-    else:
-        wl = W.generate("tiny", B=6, n_nodes=[1, 4, 16, 33, 64, 2],
-                        kv_len=[0, 1, 63, 64, 65, 200], depth=8, depth_min=1, branch=None,
-                        width=16, vocab=1000, hidden=256)
-    _full_check(wl)
-
-
 @pytest.mark.parametrize("case", ["ragged", "g1", "g8_chain", "conc_like", "two_blocks"])
-def test_attention_32key_tiles(case, monkeypatch):
-    """The 32-key, two-CTAs-per-SM attention shape: two tree tiles for trees over 32 nodes,
-    lane-quarter rotation of small row blocks, ragged lengths."""
-    monkeypatch.setenv("ETREE_ATTN_KEYS", "32")
+def test_attention_32key_tiles(case):
+    """The 32-key, two-CTAs-per-SM attention shape (chosen for 64K or more cached keys: here a
+    loose kv_len_max bound asks for it): two tree tiles for trees over 32 nodes, lane-quarter
+    rotation of small row blocks, ragged lengths, splits with nothing to do."""
     if case == "ragged":
         wl = W.generate("tiny", B=6, n_nodes=[1, 4, 16, 33, 64, 2],
                         kv_len=[0, 1, 31, 32, 33, 200], depth=8, depth_min=1, branch=None,
@@ -200,24 +194,30 @@ def test_attention_32key_tiles(case, monkeypatch):
     else:
         wl = W.generate("tiny", B=2, hq=40, hkv=8, n_nodes=[64, 30], depth=8, depth_min=8,
                         branch=None, width=16, kv_len=[500, 77], hidden=256, vocab=512)
+    assert _plan(wl, kv_len_max=65536)["rows_per_cta"] > 0
+    _full_check(wl, kv_len_max=65536)
+
+
+def test_attention_32key_tiles_from_many_work_items():
+    """The other route to 32-key tiles: at least one (request, KV head, row block) per SM."""
+    wl = W.generate("tiny", B=80, n_nodes=[1, 3, 5, 8] * 20, depth=4, depth_min=2, branch=None,
+                    width=16, kv_len=(0, 200), hidden=256, vocab=512)
+    assert _plan(wl)["splits"] >= 1 and wl.B * wl.hkv >= 148
     _full_check(wl)
 
 
-@pytest.mark.parametrize("bm", ["auto", "128", "per_tile"])
+@pytest.mark.parametrize("rows", [64, 100, 200])
 @pytest.mark.parametrize("T", [0.0, 1.0])
-def test_lmhead_row_tile_heights(bm, T, monkeypatch):
+def test_lmhead_row_tile_heights(rows, T):
     """Up to 64 rows the LM head runs M=64 MMAs (rows 16q..16q+15 in the first half of TMEM
-    lane quarter q) and folds each CTA's vocab tiles into one summary per row; the 128-row tile
-    and per-tile summaries must give the same results."""
-    if bm == "128":
-        monkeypatch.setenv("ETREE_BM", bm)
-    elif bm == "per_tile":
-        monkeypatch.setenv("ETREE_PER_TILE", "1")
+    lane quarter q); up to 128 rows one M=128 row tile; with more row tiles the summaries are
+    per vocab tile instead of per CTA.  All must give the oracle's results."""
+    sizes = {64: [20, 1, 31, 12], 100: [20, 1, 31, 12, 36], 200: [20, 1, 31, 12, 36, 50, 50]}[rows]
     shape = dict(depth=6, depth_min=4, branch=None, width=16) if T == 0.0 else \
         dict(depth=63, depth_min=63, branch=1)            # sampling verifies chains
-    wl = W.generate("tiny", B=4, n_nodes=[20, 1, 31, 12], kv_len=(50, 400), hidden=512,
+    wl = W.generate("tiny", B=len(sizes), n_nodes=sizes, kv_len=(50, 400), hidden=512,
                     vocab=8192 + 77, temperature=T, **shape)
-    assert wl.n_total == 64
+    assert wl.n_total == rows
     _full_check(wl)
 
 
@@ -243,14 +243,12 @@ def test_tree_sampler_on_chains_matches_chain_rule():
     dev, res = _run(wl, tree=True)
     assert dev.zbuf is None
     excused, near, ores = P.chain_compare(wl, res, list(range(wl.B)))
-    assert near <= 3
+    P.log_near("tree_entry_on_chains", wl, res, ores, list(range(wl.B)), near)
+    assert near <= MAX_EXCUSED
 
 
 def test_tree64_t1_full_size():
-    wl = W.generate("tree64_t1")
-    g = np.random.default_rng(3)
-    reqs = sorted(g.choice(wl.B, 8, replace=False).tolist())
-    _full_check(wl, attn_rows=P.sample_rows(wl, 2), requests=reqs)
+    _full_check(W.generate("tree64_t1"))
 
 
 def test_logit_buffer_overflow_reports_and_answers_the_rest():
@@ -275,46 +273,39 @@ def test_logit_buffer_overflow_reports_and_answers_the_rest():
         else:
             assert res["accept_len"][r] == 0 and res["out_tokens"][r][0] >= 0   # root draw only
     excused, near, ores = P.tree_compare(wl, res, got)
-    assert near <= 1
+    assert near <= MAX_EXCUSED
 
 
 # ------------------------------------------------------------------------- paged KV caches
-def _paged_check(wl, page_size, attn_rows=None, requests=None):
-    dev, res = _run(wl, page_size=page_size)
+def _paged_check(wl, page_size, attn_rows=None, requests=None, **kw):
+    dev, res = _run(wl, page_size=page_size, **kw)
     P.attn_compare_paged(wl, dev, rows=attn_rows)
     reqs = list(range(wl.B)) if requests is None else requests
-    if wl.temperature == 0.0:
-        excused, near, ores = P.greedy_compare(wl, res, reqs)
-    else:
-        excused, near, ores = P.chain_compare(wl, res, reqs)
+    excused, ores = _accept_check(wl, dev, res, reqs, f"{wl.name}@p{page_size}")
     P.compact_compare_paged(wl, dev, ores, reqs, excused)
-    assert near <= max(1, len(reqs) // 10), near
     return dev, res
 
 
 @pytest.mark.parametrize("page_size", [16, 32, 64, 256])
-@pytest.mark.parametrize("keys", ["32", "64"])
-def test_paged_cache(page_size, keys, monkeypatch):
-    """Pages smaller than, equal to and larger than the key tile, both tile shapes, ragged
-    lengths including an empty cache and lengths that end mid-page."""
-    monkeypatch.setenv("ETREE_ATTN_KEYS", keys)
+@pytest.mark.parametrize("keys", [32, 64])
+def test_paged_cache(page_size, keys):
+    """Pages smaller than, equal to and larger than the key tile, both tile shapes (32-key tiles
+    through a loose kv_len_max bound), ragged lengths including an empty cache and lengths that
+    end mid-page."""
     wl = W.generate("tiny", B=6, n_nodes=[1, 4, 16, 33, 64, 2],
                     kv_len=[0, 1, 31, 64, 65, 700], depth=8, depth_min=1, branch=None,
                     width=16, vocab=1000, hidden=256)
-    _paged_check(wl, page_size)
+    _paged_check(wl, page_size, kv_len_max=65536 if keys == 32 else None)
 
 
-def test_paged_cache_splits_and_stochastic_chains(monkeypatch):
-    monkeypatch.setenv("ETREE_NSPLIT", "3")
+def test_paged_cache_splits_and_stochastic_chains():
     wl = W.generate("conc512", B=9, kv_len=(30, 900), hidden=256, vocab=512)
+    assert _plan(wl)["splits"] > 1
     _paged_check(wl, 16)
 
 
 def test_batch64_paged16_full_size():
-    wl = W.generate("batch64")
-    g = np.random.default_rng(4)
-    reqs = sorted(g.choice(wl.B, 6, replace=False).tolist())
-    _paged_check(wl, 16, attn_rows=P.sample_rows(wl, 4), requests=reqs)
+    _paged_check(W.generate("batch64"), 16)
 
 
 # -------------------------------------------------------------------- low-rank candidate head
@@ -339,16 +330,14 @@ def _lowrank_run(lw):
 def test_lowrank_candidates_small(over):
     lw = W.lowrank("lowrank_tiny", **over)
     ids, lg = _lowrank_run(lw)
-    differ = P.lowrank_compare(lw, ids, lg)
-    assert differ <= max(1, lw.M // 10), differ
+    P.lowrank_compare(lw, ids, lg)
 
 
 @pytest.mark.parametrize("name", ["lowrank_r512", "lowrank_r128"])
 def test_lowrank_candidates_full_size(name):
     lw = W.lowrank(name)
     ids, lg = _lowrank_run(lw)
-    differ = P.lowrank_compare(lw, ids, lg)
-    assert differ <= max(1, lw.M // 10), differ
+    P.lowrank_compare(lw, ids, lg)
 
 
 def test_inputs_written_by_the_kernel_before_each_call():
@@ -401,5 +390,4 @@ def test_lowrank_hidden_written_by_the_kernel_before_the_call():
         h_in.copy_(h)                                    # written right before the call
         etree_lowrank_candidates(h_in, D, U, Wt, lw.k, ids, lg, ws)
     assert etree_device_status(ws) == (0, 0)
-    differ = P.lowrank_compare(lw, ids.cpu().numpy(), lg.cpu().numpy())
-    assert differ <= max(1, lw.M // 10), differ
+    P.lowrank_compare(lw, ids.cpu().numpy(), lg.cpu().numpy())
