@@ -302,9 +302,9 @@ def time_e2e(dev, wl, steps, warmup, flush):
     return ms, h2d, d2h
 
 
-def time_compact_layers(dev, wl, flush, layers=64, reps=10):
+def compact_layers_call(dev, wl, layers=64):
     """KV compaction over `layers` stacked layers with the step's real accept lengths and paths,
-    into a compaction-only pool (every request given 64 free slots), timed alone."""
+    into a compaction-only pool (every request given 64 free slots): returns the call."""
     from draft_tree_verification_masked_b200 import etree_kv_compact, make_batch
     B, hkv, D = wl.B, wl.hkv, wl.head_dim
     i32 = dict(dtype=torch.int32, device="cuda")
@@ -324,6 +324,12 @@ def time_compact_layers(dev, wl, flush, layers=64, reps=10):
         etree_kv_compact(batch, dev.accept_len, dev.path, kt, vt, kc, vc, layers,
                          kt[0].numel(), kc[0].numel(), out, dev.ws)
 
+    return one
+
+
+def time_compact_layers(dev, wl, flush, layers=64, reps=10):
+    """KV compaction over `layers` stacked layers (compact_layers_call), timed alone."""
+    one = compact_layers_call(dev, wl, layers)
     for _ in range(3):
         one()
     torch.cuda.synchronize()
@@ -339,7 +345,7 @@ def time_compact_layers(dev, wl, flush, layers=64, reps=10):
     us = tot / reps * 1e3
     acc = dev.accept_len.cpu().numpy()
     nbytes = compact_work(wl, acc, layers)
-    del kt, vt, kc, vc
+    del one
     torch.cuda.empty_cache()
     return us, nbytes
 
@@ -582,8 +588,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lowrank", default="lowrank_r512,lowrank_r128",
                     help="low-rank candidate-head workloads timed after the step ('' for none)")
+    ap.add_argument("--ncu-case", default="", choices=["", "attn", "lmhead", "compact64"],
+                    help="profiling driver: run one step of --config, then only this call "
+                         "--steps times (no flush, no timing, no JSON), for ncu captures")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.ncu_case:
+        return ncu_case(args)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -696,6 +707,29 @@ def main():
         "lowrank_head": lowrank,
     }
     print(json.dumps(line))
+
+
+def ncu_case(args):
+    """Runs one verification step of the workload, then the selected call alone `steps` times:
+    the launches an ncu capture filters with -k / -s / -c.  compact64 moves the accepted rows of
+    64 stacked layers."""
+    from draft_tree_verification_masked_b200 import workload as W
+    from draft_tree_verification_masked_b200.runner import DeviceStep
+    base, _, pg = args.config.partition("@p")
+    wl = W.generate(base)
+    dev = DeviceStep(wl, page_size=int(pg) if pg else None)
+    dev.step()
+    st = dev.status()
+    if st[0] != 0:
+        raise RuntimeError(f"device status {st}")
+    if args.ncu_case == "compact64":
+        call = compact_layers_call(dev, wl, 64)
+    else:
+        call = {"attn": dev.attn, "lmhead": dev.lmhead}[args.ncu_case]
+    for _ in range(args.steps):
+        call()
+    torch.cuda.synchronize()
+    print(f"ncu case {args.config} {args.ncu_case}: {args.steps} calls")
 
 
 def main_reference(args, rank, world):

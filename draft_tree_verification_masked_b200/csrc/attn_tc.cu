@@ -46,15 +46,8 @@ struct TcSmem {
   float xmax[2][4][128];                    // row-max exchange: [tile parity][key part][row]
   float xl[4][128];                         // final row sums of the key parts
   uint64_t xbar[4][2], xlbar[4];            // exchange barriers per lane quarter (bounded waits)
-  float inv[128];                           // 1 / row sum, for the staged bf16 output
   uint32_t tmem;
 };
-
-// The epilogue stages O through shared memory (over the Q box and the K/V ring, both free once
-// the last PV product has completed) as [128 rows][kStageLd] fp32, so that every warp then writes
-// whole rows with coalesced stores.  The 4-float pad puts consecutive rows 4 banks apart.
-constexpr int kStageLd = 132;
-constexpr int kStageBytes = 128 * kStageLd * 4;
 
 template <int KEYS>
 struct TcShape {
@@ -127,66 +120,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     else if (qrows <= 64) rot = 64 * (blockIdx.x & 1);
   }
 
-  // ---------------------------------------------------------------- producer state and loads
-  // Thread 0 is the TMA producer (warp 0, lane 0).  It initialises the barriers and issues Q and
-  // the first ring of K/V tiles before the rest of the CTA's set-up (tensor memory, tree masks),
-  // so that the first loads are in flight while that set-up runs.
-  const int nbox = paged ? KEYS / p.cache_box : 0;
-  const int32_t* bt = paged ? p.block_table + (size_t)r * p.max_pages : nullptr;
-  int32_t pg_cur[4], pg_nxt[4];
-  // paged: the page entries of tile t (positions outside the cache read as -1)
-  auto fetch_pages = [&](int t, int32_t (&dst)[4]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int pi = (t * KEYS + i * p.cache_box) >> p.page_shift;
-      dst[i] = (i < nbox && t < nt_cache && pi < p.max_pages) ? __ldg(bt + pi) : -1;
-    }
-  };
-  // tile j of this split into ring stage j % STAGES, armed for its bytes
-  auto issue = [&](int j) {
-    const int t = t0 + j;
-    const int st = j % STAGES;
-    uint8_t* dst = sKV + st * Sh::kKV;
-    mbar_arrive_expect_tx(&sh->kv_full[st], Sh::kKV);
-    if (t < nt_cache && !paged) {
-      const int32_t slot = static_cast<int32_t>(sbase + (int64_t)t * KEYS);
-      tma_load_3d(dst, &tm_kc, &sh->kv_full[st], 0, kvh, slot);
-      tma_load_3d(dst + Sh::kBox, &tm_kc, &sh->kv_full[st], 64, kvh, slot);
-      tma_load_3d(dst + 2 * Sh::kBox, &tm_vc, &sh->kv_full[st], 0, kvh, slot);
-      tma_load_3d(dst + 3 * Sh::kBox, &tm_vc, &sh->kv_full[st], 64, kvh, slot);
-    } else if (t < nt_cache) {
-      // paged: KEYS / cache_box boxes per half, each inside one page.  An entry outside the pool
-      // is reported; its box then lies past the tensor and TMA fills zeros.
-      const int cb = p.cache_box, P = 1 << p.page_shift;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (i >= nbox) break;
-        const int pos = t * KEYS + i * cb;
-        int32_t page = pg_cur[i];
-        if (page < 0 || (int64_t)page * P >= p.cache_slots) {
-          if (pos < L) report(p.ws, ETREE_EDEVICE, DET_BAD_PAGE);
-          page = (int32_t)(p.cache_slots >> p.page_shift);
-        }
-        const int32_t slot = page * P + (pos & (P - 1));
-        const uint32_t off = (uint32_t)(i * cb * 128);
-        tma_load_3d(dst + off, &tm_kc, &sh->kv_full[st], 0, kvh, slot);
-        tma_load_3d(dst + Sh::kBox + off, &tm_kc, &sh->kv_full[st], 64, kvh, slot);
-        tma_load_3d(dst + 2 * Sh::kBox + off, &tm_vc, &sh->kv_full[st], 0, kvh, slot);
-        tma_load_3d(dst + 3 * Sh::kBox + off, &tm_vc, &sh->kv_full[st], 64, kvh, slot);
-      }
-    } else {
-      const int node = base + (t - nt_cache) * KEYS;
-      tma_load_3d(dst, &tm_kt, &sh->kv_full[st], 0, kvh, node);
-      tma_load_3d(dst + Sh::kBox, &tm_kt, &sh->kv_full[st], 64, kvh, node);
-      tma_load_3d(dst + 2 * Sh::kBox, &tm_vt, &sh->kv_full[st], 0, kvh, node);
-      tma_load_3d(dst + 3 * Sh::kBox, &tm_vt, &sh->kv_full[st], 64, kvh, node);
-    }
-  };
-  const int pre = T < STAGES ? T : STAGES;
   if (threadIdx.x == 0) {
-    prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_kc);
-    prefetch_tmap(&tm_vc);
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&sh->kv_full[i], 1);
       mbar_init(&sh->kv_empty[i], 1);
@@ -205,18 +139,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(&sh->xlbar[q], SW / 4);
     }
     fence_barrier_init();
-    mbar_arrive_expect_tx(&sh->q_full, 2 * qrows * 128);
-    tma_load_3d(sQ + rot * 128, &tm_q, &sh->q_full, 0, kvh * G, base + node0);
-    tma_load_3d(sQ + 16384 + rot * 128, &tm_q, &sh->q_full, 64, kvh * G, base + node0);
-    if (paged) fetch_pages(t0, pg_cur);
-    for (int j = 0; j < pre; ++j) {
-      if (paged) fetch_pages(t0 + j + 1, pg_nxt);
-      issue(j);
-      if (paged) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) pg_cur[i] = pg_nxt[i];
-      }
-    }
   }
   if (warp == 1) {
     tmem_alloc(&sh->tmem, Sh::kTmemCols);
@@ -259,14 +181,68 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (warp == 0) {
     // ------------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int issued = pre;
-      for (int j = pre; j < T; ++j) {
-        if (paged) fetch_pages(t0 + j + 1, pg_nxt);
-        if (!mbar_wait(&sh->kv_empty[j % STAGES], ((j / STAGES) & 1) ^ 1)) {
+      prefetch_tmap(&tm_kc);
+      prefetch_tmap(&tm_vc);
+      mbar_arrive_expect_tx(&sh->q_full, 2 * qrows * 128);
+      tma_load_3d(sQ + rot * 128, &tm_q, &sh->q_full, 0, kvh * G, base + node0);
+      tma_load_3d(sQ + 16384 + rot * 128, &tm_q, &sh->q_full, 64, kvh * G, base + node0);
+      int issued = 0;
+      // paged: the page entries of tile j + 1 are fetched while tile j's slot is awaited
+      const int nbox = paged ? KEYS / p.cache_box : 0;
+      const int32_t* bt = paged ? p.block_table + (size_t)r * p.max_pages : nullptr;
+      int32_t pg_cur[4], pg_nxt[4];
+      auto fetch_pages = [&](int t, int32_t (&dst)[4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int pi = (t * KEYS + i * p.cache_box) >> p.page_shift;
+          dst[i] = (i < nbox && t < nt_cache && pi < p.max_pages) ? __ldg(bt + pi) : -1;
+        }
+      };
+      if (paged) fetch_pages(t0, pg_cur);
+      for (int j = 0; j < T; ++j) {
+        const int t = t0 + j;
+        const int st = j % STAGES;
+        const uint32_t ph = (j / STAGES) & 1;
+        if (paged) fetch_pages(t + 1, pg_nxt);
+        if (j >= STAGES && !mbar_wait(&sh->kv_empty[st], ph ^ 1)) {
           report(p.ws, ETREE_ETIMEOUT, DET_WAIT_ATTN);
           break;
         }
-        issue(j);
+        uint8_t* dst = sKV + st * Sh::kKV;
+        mbar_arrive_expect_tx(&sh->kv_full[st], Sh::kKV);
+        if (t < nt_cache && !paged) {
+          const int32_t slot = static_cast<int32_t>(sbase + (int64_t)t * KEYS);
+          tma_load_3d(dst, &tm_kc, &sh->kv_full[st], 0, kvh, slot);
+          tma_load_3d(dst + Sh::kBox, &tm_kc, &sh->kv_full[st], 64, kvh, slot);
+          tma_load_3d(dst + 2 * Sh::kBox, &tm_vc, &sh->kv_full[st], 0, kvh, slot);
+          tma_load_3d(dst + 3 * Sh::kBox, &tm_vc, &sh->kv_full[st], 64, kvh, slot);
+        } else if (t < nt_cache) {
+          // paged: KEYS / cache_box boxes per half, each inside one page.  An entry outside
+          // the pool is reported; its box then lies past the tensor and TMA fills zeros.
+          const int cb = p.cache_box, P = 1 << p.page_shift;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (i >= nbox) break;
+            const int pos = t * KEYS + i * cb;
+            int32_t page = pg_cur[i];
+            if (page < 0 || (int64_t)page * P >= p.cache_slots) {
+              if (pos < L) report(p.ws, ETREE_EDEVICE, DET_BAD_PAGE);
+              page = (int32_t)(p.cache_slots >> p.page_shift);
+            }
+            const int32_t slot = page * P + (pos & (P - 1));
+            const uint32_t off = (uint32_t)(i * cb * 128);
+            tma_load_3d(dst + off, &tm_kc, &sh->kv_full[st], 0, kvh, slot);
+            tma_load_3d(dst + Sh::kBox + off, &tm_kc, &sh->kv_full[st], 64, kvh, slot);
+            tma_load_3d(dst + 2 * Sh::kBox + off, &tm_vc, &sh->kv_full[st], 0, kvh, slot);
+            tma_load_3d(dst + 3 * Sh::kBox + off, &tm_vc, &sh->kv_full[st], 64, kvh, slot);
+          }
+        } else {
+          const int node = base + (t - nt_cache) * KEYS;
+          tma_load_3d(dst, &tm_kt, &sh->kv_full[st], 0, kvh, node);
+          tma_load_3d(dst + Sh::kBox, &tm_kt, &sh->kv_full[st], 64, kvh, node);
+          tma_load_3d(dst + 2 * Sh::kBox, &tm_vt, &sh->kv_full[st], 0, kvh, node);
+          tma_load_3d(dst + 3 * Sh::kBox, &tm_vt, &sh->kv_full[st], 64, kvh, node);
+        }
         if (paged) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) pg_cur[i] = pg_nxt[i];
@@ -481,46 +457,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       for (int h = 0; h < NH; ++h) l += sh->xl[h][row];
     }
     tc_fence_after();
-    // Stage this thread's O columns in shared memory (row = TMEM lane), then write whole rows.
-    float* stage = reinterpret_cast<float*>(sQ);
-    static_assert(kQBytes + STAGES * Sh::kKV >= kStageBytes, "O staging needs Q + the ring");
-#pragma unroll 1
-    for (int c = 0; c < OW / 32; ++c) {
-      const int col = kh * OW + c * 32;
-      float o[32];
-      tmem_ld32(lane_base + Sh::kOCol + col, o);
-      float4* dst = reinterpret_cast<float4*>(stage + row * kStageLd + col);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-    }
     const size_t gidx = (size_t)(base + (valid ? node : 0)) * p.hq + kvh * G + g;
-    if (kh == 0) {
-      if (p.nsplit == 1) {
-        sh->inv[row] = l > 0.f ? 1.f / l : 0.f;
-        if (valid && p.lse) p.lse[gidx] = (m_ref + log2f(l)) * 0.69314718055994531f;
-      } else if (valid) {
-        p.ml_part[gidx * p.nsplit + s] = make_float2(m_ref, l);
-      }
-    }
-    asm volatile("bar.sync 1, %0;" ::"r"(SW * 32) : "memory");   // the softmax warps only
-    // Warp wsm writes rows wsm, wsm + SW, ...: 32 lanes cover one row's 128 values.
-    const int wsm = warp - 2;
+    if (p.nsplit == 1) {
+      const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-    for (int i = wsm; i < 128; i += SW) {
-      const int li = i - rot;
-      if (li < 0 || li >= qrows) continue;
-      const int nl = li / G, gi = li - nl * G;
-      if (node0 + nl >= n) continue;
-      const size_t gi_row = (size_t)(base + node0 + nl) * p.hq + kvh * G + gi;
-      const float4 v = reinterpret_cast<const float4*>(stage + i * kStageLd)[lane];
-      if (p.nsplit == 1) {
-        const float inv = sh->inv[i];
-        reinterpret_cast<uint2*>(p.out + gi_row * 128)[lane] =
-            make_uint2(pack_bf16x2(v.x * inv, v.y * inv), pack_bf16x2(v.z * inv, v.w * inv));
-      } else {
-        reinterpret_cast<float4*>(p.o_part + (gi_row * p.nsplit + s) * 128)[lane] = v;
+      for (int c = 0; c < OW / 32; ++c) {
+        const int col = kh * OW + c * 32;
+        float o[32];
+        tmem_ld32(lane_base + Sh::kOCol + col, o);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + gidx * 128 + col);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+        }
       }
+      if (valid && kh == 0 && p.lse) p.lse[gidx] = (m_ref + log2f(l)) * 0.69314718055994531f;
+    } else {
+      float* op = p.o_part + (gidx * p.nsplit + s) * 128;
+#pragma unroll 1
+      for (int c = 0; c < OW / 32; ++c) {
+        const int col = kh * OW + c * 32;
+        float o[32];
+        tmem_ld32(lane_base + Sh::kOCol + col, o);
+        if (valid) {
+          float4* dst = reinterpret_cast<float4*>(op + col);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        }
+      }
+      if (valid && kh == 0) p.ml_part[gidx * p.nsplit + s] = make_float2(m_ref, l);
     }
   }
   tc_fence_before();
