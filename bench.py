@@ -160,6 +160,16 @@ def source_hash(*names):
     return h.hexdigest()[:16]
 
 
+# The sources a kernel's DRAM traffic depends on (the traffic entries record their hash).
+KERNEL_SOURCES = {"attn": ("attn_tc.cu", "common.cuh", "kernels.cuh"),
+                  "lmhead": ("lmhead.cu", "race.cuh", "philox.cuh", "common.cuh", "kernels.cuh"),
+                  "compact": ("compact.cu", "common.cuh", "kernels.cuh")}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    return source_hash(*KERNEL_SOURCES[kernel])
+
+
 def ncu_traffic(kernel: str, workload: str, src_hash: str):
     """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -448,7 +458,9 @@ def run_config(name, steps, warmup, peaks, rank, flush, with_e2e=True):
 
     base, _, pg = name.partition("@p")                 # "<workload>@p<page size>": paged cache
     wl = W.generate(base, seed=W.config_seed(base) + 7919 * rank)
-    dev = DeviceStep(wl, page_size=int(pg) if pg else None)
+    # T > 0: every row's logits are kept (n_total x vocab fp32), so the bonus draw reads the stop
+    # rows instead of a second pass over the head
+    dev = DeviceStep(wl, page_size=int(pg) if pg else None, materialize=True)
     dev.step()
     st, det = dev.status()
     if st != 0:
@@ -457,9 +469,9 @@ def run_config(name, steps, warmup, peaks, rank, flush, with_e2e=True):
     toks = int((acc + 1).sum())
     t = time_steps(dev, steps, warmup, flush)
     plan = etree_attn_plan(dev.batch, wl.hq, wl.hkv)
-    # attention + LM head (T=0: GEMM, fused accept; chains: prep, GEMM, accept, draw GEMM, race;
-    # branching trees: prep, child logits, GEMM, row merge, walk, draw GEMM, race) + compaction
-    launches = plan["launches"] + (2 if wl.temperature == 0.0 else (7 if dev.tree else 5)) + 1
+    # attention + LM head (T=0: GEMM, fused accept; T>0 with every row materialised: prep, child
+    # logits, GEMM, row merge, walk, draw over the stored rows) + compaction
+    launches = plan["launches"] + (2 if wl.temperature == 0.0 else 6) + 1
     res = dict(wl=wl, dev=dev, toks=toks, t=t, plan=plan, launches=launches)
     if with_e2e:
         res["e2e"] = time_e2e(dev, wl, steps, max(3, warmup), flush)
@@ -547,11 +559,13 @@ def kernel_report(wl, t, acc, peaks):
     rep["lmhead_gemm"] = {"us": g1 * 1e6, "GB/s": lb / g1 / 1e9, "TFLOP/s": lf / g1 / 1e12,
                           "hbm_frac": lb / g1 / 1e9 / hbm, "tc_frac": lf / g1 / 1e12 / tc}
     if wl.temperature > 0.0:
-        g2 = ph["draw_gemm"]
-        df = 2.0 * wl.B * wl.vocab * wl.hidden_dim
-        rep["lmhead_draw_gemm"] = {"us": g2 * 1e6, "TFLOP/s": df / g2 / 1e12,
-                                   "tc_frac": df / g2 / 1e12 / tc, "flops": df,
-                                   "note": "second W pass over the B stop rows; not algorithmic"}
+        # the bonus draw reads each stop row's stored logits and its draft row (fp32)
+        d = ph["draw_gemm"] + ph["draw_pick"]
+        db = 8.0 * wl.B * wl.vocab
+        rep["lmhead_draw"] = {"us": d * 1e6, "bytes": db, "GB/s": db / d / 1e9,
+                              "hbm_frac": db / d / 1e9 / hbm,
+                              "note": "bonus draw over the B stop rows' stored logits and draft "
+                                      "rows; implementation overhead, not algorithmic"}
     for k in rep.values():
         if "GB/s" in k:
             k["hbm_frac_nominal"] = k["GB/s"] / NOMINAL_HBM_GBS
@@ -564,8 +578,7 @@ def roofline(wl, rep, peaks, peak_kind, workload):
     dom = max(("attn", "lmhead", "compact"), key=lambda k: rep[k]["us"])
     k = rep[dom]
     hbm, tc = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
-    src = {"attn": "attn_tc.cu", "lmhead": "lmhead.cu", "compact": "compact.cu"}[dom]
-    traffic = ncu_traffic(dom, workload, source_hash(src, "common.cuh", "kernels.cuh"))
+    traffic = ncu_traffic(dom, workload, kernel_source_hash(dom))
     if dom == "compact" or k["bytes"] / (hbm * 1e9) >= k.get("flops", 0) / (tc * 1e12):
         return {"kernel": dom, "bound": "hbm", "achieved": k["GB/s"], "peak": hbm,
                 "unit": "GB/s", "frac": k["GB/s"] / hbm, "traffic": traffic,
@@ -591,6 +604,9 @@ def main():
     ap.add_argument("--ncu-case", default="", choices=["", "attn", "lmhead", "compact64"],
                     help="profiling driver: run one step of --config, then only this call "
                          "--steps times (no flush, no timing, no JSON), for ncu captures")
+    ap.add_argument("--ncu-kv", default="",
+                    help="with --ncu-case: LO:HI replaces the workload's KV-length range (a "
+                         "smaller capture of the same kernels)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.ncu_case:
@@ -716,7 +732,11 @@ def ncu_case(args):
     from draft_tree_verification_masked_b200 import workload as W
     from draft_tree_verification_masked_b200.runner import DeviceStep
     base, _, pg = args.config.partition("@p")
-    wl = W.generate(base)
+    over = {}
+    if args.ncu_kv:
+        lo, hi = (int(x) for x in args.ncu_kv.split(":"))
+        over["kv_len"] = (lo, hi)
+    wl = W.generate(base, **over)
     dev = DeviceStep(wl, page_size=int(pg) if pg else None)
     dev.step()
     st = dev.status()
@@ -729,7 +749,8 @@ def ncu_case(args):
     for _ in range(args.steps):
         call()
     torch.cuda.synchronize()
-    print(f"ncu case {args.config} {args.ncu_case}: {args.steps} calls")
+    print(f"ncu case {args.config} {args.ncu_case} kv {args.ncu_kv or 'as configured'}: "
+          f"{args.steps} calls")
 
 
 def main_reference(args, rank, world):

@@ -14,6 +14,7 @@
 // the <= 64 nodes at T = 0, the sequential accept test along the chain at T > 0).
 #include "kernels.cuh"
 #include "philox.cuh"
+#include "race.cuh"
 
 namespace etree {
 
@@ -350,7 +351,9 @@ __global__ void __launch_bounds__(256) chain_accept_kernel(AcceptParams p, int32
 
 // One CTA: per-node child counts, then a row of the caller's logit buffer for every node with
 // two or more children (in node order).  Nodes past zbuf_rows get none: their requests are
-// answered as malformed by the walk and the status reports ETREE_ENOSPACE.
+// answered as malformed by the walk and the status reports ETREE_ENOSPACE.  With a buffer of at
+// least n_total rows every node gets its own row (row g for node g), and the bonus draw reads the
+// stop row's logits there instead of recomputing them.
 __global__ void __launch_bounds__(1024) tree_prep_kernel(AcceptParams p, int32_t* ccount,
                                                          int32_t* zrow, int zbuf_rows) {
   __shared__ int32_t part_s[1024];
@@ -379,6 +382,10 @@ __global__ void __launch_bounds__(1024) tree_prep_kernel(AcceptParams p, int32_t
   }
   int next = part_s[tid] - cnt;
   bool over = false;
+  if (zbuf_rows >= p.n_total) {                       // every row materialised
+    for (int g = g0; g < g1; ++g) zrow[g] = g;
+    return;
+  }
   for (int g = g0; g < g1; ++g) {
     int zr = -1;
     if (ccount[g] >= 2) {
@@ -674,6 +681,97 @@ __global__ void __launch_bounds__(256) bonus_kernel(AcceptParams p) {
     const int a = p.accept_len[r];
     p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = ir >= 0 ? ir : ip;
   }
+}
+
+// The bonus draw from materialised logits, one CTA per request: the races of race.cuh over the
+// stop row's stored logits and its draft row (the same fp32 logits the first GEMM pass produced,
+// so the tokens equal those of a second pass over W).  Thread t takes the 8-id groups t,
+// t + blockDim, ...; a CTA-wide floor in shared memory (keys of real ids) sharpens each thread's
+// screen; the leaders are merged by a total order (larger key, then lower id), so the result does
+// not depend on the thread mapping.
+constexpr int kDrawThreads = 512;
+
+__global__ void __launch_bounds__(kDrawThreads) draw_rows_kernel(AcceptParams p,
+                                                                 const int32_t* zrow,
+                                                                 const float* zbuf) {
+  __shared__ unsigned fl_s[2];                        // floors (fp32 bits of positive keys)
+  __shared__ float kr_s[kDrawThreads / 32], kp_s[kDrawThreads / 32];
+  __shared__ int ir_s[kDrawThreads / 32], ip_s[kDrawThreads / 32];
+  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int base, n;
+  if (!request_ok(p, r, base, n)) return;            // answered by the walk
+  if (tid == 0) fl_s[0] = fl_s[1] = 0u;
+  __syncthreads();
+  const int srow = p.stop_row[r];
+  const int zr = zrow[srow];
+  const float c = p.cval[r];
+  const float L2 = p.lse2[srow];
+  const float* z = zbuf + (size_t)(zr < 0 ? 0 : zr) * p.V;
+  const float* q = p.q_draft + (size_t)srow * p.V;
+  const uint32_t node = (uint32_t)p.stop_node[r];
+  float kr = -INFINITY, kp = -INFINITY;
+  int ir = -1, ip = -1;
+  float thr_r = 0.f, thr_p = 0.f;
+  const int groups = (p.V + 7) / 8;
+  for (int g = tid; zr >= 0 && g < groups; g += kDrawThreads) {
+    const int c0 = g * 8;
+    float zz[8], qq[8];
+    if ((p.V & 7) == 0) {
+      const float4 a = *reinterpret_cast<const float4*>(z + c0);
+      const float4 b = *reinterpret_cast<const float4*>(z + c0 + 4);
+      zz[0] = a.x; zz[1] = a.y; zz[2] = a.z; zz[3] = a.w;
+      zz[4] = b.x; zz[5] = b.y; zz[6] = b.z; zz[7] = b.w;
+      if (c > 0.f) {
+        const float4 x = __ldg(reinterpret_cast<const float4*>(q + c0));
+        const float4 y = __ldg(reinterpret_cast<const float4*>(q + c0 + 4));
+        qq[0] = x.x; qq[1] = x.y; qq[2] = x.z; qq[3] = x.w;
+        qq[4] = y.x; qq[5] = y.y; qq[6] = y.z; qq[7] = y.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        zz[e] = c0 + e < p.V ? z[c0 + e] : 0.f;
+        qq[e] = (c > 0.f && c0 + e < p.V) ? __ldg(q + c0 + e) : 0.f;
+      }
+    }
+    thr_r = fmaxf(thr_r, __uint_as_float(fl_s[0]) * kRaceShrink);
+    thr_p = fmaxf(thr_p, __uint_as_float(fl_s[1]) * kRaceShrink);
+    const float kr0 = kr, kp0 = kp;
+    race8(zz, qq, c0, p.V, p.k_log2, L2, c, p.seed, p.step, node, (uint32_t)r, thr_r, thr_p, kr,
+          ir, kp, ip);
+    if (kr > kr0 && kr > 0.f) atomicMax(&fl_s[0], __float_as_uint(kr));
+    if (kp > kp0 && kp > 0.f) atomicMax(&fl_s[1], __float_as_uint(kp));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float okr = __shfl_xor_sync(0xffffffffu, kr, off);
+    const int oir = __shfl_xor_sync(0xffffffffu, ir, off);
+    const float okp = __shfl_xor_sync(0xffffffffu, kp, off);
+    const int oip = __shfl_xor_sync(0xffffffffu, ip, off);
+    merge_key(kr, ir, okr, oir);
+    merge_key(kp, ip, okp, oip);
+  }
+  if (lane == 0) {
+    kr_s[warp] = kr;
+    ir_s[warp] = ir;
+    kp_s[warp] = kp;
+    ip_s[warp] = ip;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int w = 1; w < kDrawThreads / 32; ++w) {
+      merge_key(kr, ir, kr_s[w], ir_s[w]);
+      merge_key(kp, ip, kp_s[w], ip_s[w]);
+    }
+    const int a = p.accept_len[r];
+    p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = ir >= 0 ? ir : ip;
+  }
+}
+
+cudaError_t launch_draw_rows(const AcceptParams& p, const int32_t* zrow, const float* zbuf,
+                             cudaStream_t s) {
+  draw_rows_kernel<<<p.B, kDrawThreads, 0, s>>>(p, zrow, zbuf);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, int32_t* cnt,

@@ -762,6 +762,13 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
     g.zrow = nullptr;
     g.zbuf = nullptr;
     if (e == cudaSuccess) e = launch_tree_walk(a, zc, zrow, tree->zbuf, s);
+    if (e == cudaSuccess && tree->rows >= b->n_total) {
+      // every row's logits are in zbuf: the draw reads the stop rows there (no second W pass)
+      mark(2);
+      mark(3);
+      e = launch_draw_rows(a, zrow, tree->zbuf, s);
+      return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T>0, draw)");
+    }
   }
   mark(2);
   if (e != cudaSuccess) return cuda_fail(e, "etree_lmhead_accept (T>0, pass 1)");

@@ -15,8 +15,8 @@
 // head) pairs of one KV head, row = node * G + g; one TMA box {64 dims, G heads, NB nodes} of the
 // [n_total][hq][128] query tensor lands them in exactly that order (NB = floor(128 / G)).
 // Warp 0 streams Q once and the KEYS-key K/V tiles through a STAGES-deep ring; warp 1 issues the
-// MMAs; the softmax warps own one query row per thread (= one TMEM lane; with 64-key tiles two
-// warps share a row, 32 keys each, and exchange row maxima): they read S from TMEM, apply
+// MMAs; four softmax warps own one query row per thread (= one TMEM lane, all of the tile's keys;
+// the kernel also supports SW = 8, two warps per row exchanging row maxima): they read S from TMEM, apply
 // the key mask (cache length, or the row's ancestor bitmask on the tree tiles), run the online
 // softmax in log2 units, and write P (bf16) back into their own TMEM lane, where the PV product
 // takes it as its A operand; shared memory holds only Q and the K/V ring.  S and P have three
@@ -331,7 +331,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (!mbar_wait(&sh->s_full[sb], (j / Sh::kNS) & 1)) { ok = false; break; }
       tc_fence_after();
       float sc[CW];
-      if constexpr (CW == 32) {
+      if constexpr (CW == 64) {
+        tmem_ld32(lane_base + sb * KEYS, *reinterpret_cast<float(*)[32]>(sc));
+        tmem_ld32(lane_base + sb * KEYS + 32, *reinterpret_cast<float(*)[32]>(sc + 32));
+      } else if constexpr (CW == 32) {
         tmem_ld32(lane_base + sb * KEYS + kh * CW, sc);
       } else {
         tmem_ld16(lane_base + sb * KEYS + kh * CW, sc);
@@ -346,19 +349,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int k0 = kh * CW;                           // first key of this thread in the tile
       const bool full_tile = t < nt_cache && L - t * KEYS >= KEYS;
       if (!full_tile) {
-        uint32_t kw;                                    // bit c: key k0 + c is visible
+        uint64_t kw;                                    // bit c: key k0 + c is visible
         if (!valid) {
-          kw = 0u;
+          kw = 0ull;
         } else if (t >= nt_cache) {
           const int sh0 = (t - nt_cache) * KEYS + k0;   // < 64: tree tiles start at node 0
-          kw = static_cast<uint32_t>(anc >> sh0);
+          kw = anc >> sh0;
         } else {
           const int lim = L - t * KEYS - k0;
-          kw = lim >= 32 ? 0xffffffffu : (lim > 0 ? ((1u << lim) - 1u) : 0u);
+          kw = lim >= 64 ? ~0ull : (lim > 0 ? ((1ull << lim) - 1ull) : 0ull);
         }
 #pragma unroll
         for (int c = 0; c < CW; ++c)
-          if (!((kw >> c) & 1u)) sc[c] = -INFINITY;
+          if (!((kw >> c) & 1ull)) sc[c] = -INFINITY;
       }
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -435,8 +438,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc_fence_after();
       }
       // this thread's CW keys of P into its own TMEM lane (the PV product's A operand)
-      static_assert(CW == 32 || CW == 16, "a 16- or 8-column P store per thread");
-      if constexpr (CW == 32) {
+      static_assert(CW == 64 || CW == 32 || CW == 16, "a 32-, 16- or 8-column P store");
+      if constexpr (CW == 64) {
+        float pf[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pf[c] = __uint_as_float(pk[c]);
+        tmem_st32(lane_base + Sh::kPCol + pb * (KEYS / 2), pf);
+      } else if constexpr (CW == 32) {
         tmem_st16(lane_base + Sh::kPCol + pb * (KEYS / 2) + kh * (CW / 2), pk);
       } else {
         tmem_st8(lane_base + Sh::kPCol + pb * (KEYS / 2) + kh * (CW / 2), pk);
@@ -519,7 +527,7 @@ cudaError_t launch_attn_tc(const CUtensorMap& q, const CUtensorMap& kc, const CU
                            const CUtensorMap& kt, const CUtensorMap& vt, const AttnParams& p,
                            int nb, int n_total, cudaStream_t stream) {
   cudaError_t e = p.keys == 32 ? launch_shape<32, 4, 4>(q, kc, vc, kt, vt, p, nb, stream)
-                               : launch_shape<64, 5, 8>(q, kc, vc, kt, vt, p, nb, stream);
+                               : launch_shape<64, 5, 4>(q, kc, vc, kt, vt, p, nb, stream);
   if (e != cudaSuccess || p.nsplit == 1) return e;
   return launch_attn_combine(p, n_total, stream);
 }

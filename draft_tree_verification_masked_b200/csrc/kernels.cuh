@@ -111,6 +111,8 @@ cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, int32_t
 cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStream_t s);
 cudaError_t launch_accept_chain(const AcceptParams& p, int32_t* cnt, cudaStream_t s);
 cudaError_t launch_bonus(const AcceptParams& p, cudaStream_t s);
+cudaError_t launch_draw_rows(const AcceptParams& p, const int32_t* zrow, const float* zbuf,
+                             cudaStream_t s);
 cudaError_t launch_tree_prep(const AcceptParams& p, const __nv_bfloat16* w_lm, int32_t* ccount,
                              int32_t* zrow, int zbuf_rows, float* zc, cudaStream_t s);
 cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32_t* zrow,

@@ -29,6 +29,7 @@
 //               weight); bonus_kernel takes the largest key over the tiles.
 #include "kernels.cuh"
 #include "philox.cuh"
+#include "race.cuh"
 
 namespace etree {
 
@@ -103,57 +104,20 @@ struct EpiRow {
   const float* qrow = nullptr;                       // RACE: q_draft row
 };
 
-// Screening margin of the race: an id is skipped only when its key is certainly below the
-// threshold, allowing for the rounding of -log U (a few ulp) and of the quotient.
-constexpr float kRaceShrink = 1.0f - 1.0f / 1048576.0f;
-
-// The exponential race over W consecutive ids (col0 a multiple of 8).  Each id's key is
-// w_v / E_v with E_v = -log U_v > 0 (U_v the stream-0 uniform of (id, stop node, request)), and
-// the race keeps the largest key, the lower id on equal keys.  Since E_v >= 1 - U_v, an id whose
-// weight is below threshold * (1 - U_v) cannot beat the threshold and skips the logarithm; the
+// The exponential race (race.cuh) over W consecutive ids (col0 a multiple of 8).  The screening
 // threshold is the larger of this thread's best key and the floor other threads published for
 // the row (keys of real ids, so never above the row's final maximum).
 template <int W>
 __device__ __forceinline__ void race_chunk(const GemmParams& p, EpiRow& st, const float (&z)[W],
                                            const float (&q)[W], int col0) {
-  const bool resid = st.c > 0.f;
   float thr_p = fmaxf(st.fp, st.r2 > 0.f ? st.r2 : 0.f) * kRaceShrink;
   float thr_r = fmaxf(st.fr, st.r0 > 0.f ? st.r0 : 0.f) * kRaceShrink;
 #pragma unroll
   for (int g = 0; g < W / 8; ++g) {
     const int c0 = col0 + 8 * g;
     if (c0 >= p.V) break;
-    float u[8];
-    uniforms8(p.seed, p.step, (uint32_t)(c0 >> 3), (uint32_t)st.unode, (uint32_t)st.req, 0u, u);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int v = c0 + e;
-      if (v >= p.V) break;
-      const float pv = exp2f(z[8 * g + e] * p.k_log2 - st.L2);
-      const float wr = resid ? fmaxf(pv - st.c * q[8 * g + e], 0.f) : 0.f;
-      const float d = 1.f - u[e];                      // exact: U has 24 significant bits
-      const bool cp = pv > 0.f && pv >= thr_p * d;
-      const bool cr = wr > 0.f && wr >= thr_r * d;
-      if (cp || cr) {
-        const float E = -logf(u[e]);
-        if (cp) {
-          const float key = __fdiv_rn(pv, E);
-          if (key > st.r2) {
-            st.r2 = key;
-            st.r3 = v;
-            thr_p = fmaxf(thr_p, key * kRaceShrink);
-          }
-        }
-        if (cr) {
-          const float key = __fdiv_rn(wr, E);
-          if (key > st.r0) {
-            st.r0 = key;
-            st.r1 = v;
-            thr_r = fmaxf(thr_r, key * kRaceShrink);
-          }
-        }
-      }
-    }
+    race8(z + 8 * g, q + 8 * g, c0, p.V, p.k_log2, st.L2, st.c, p.seed, p.step,
+          (uint32_t)st.unode, (uint32_t)st.req, thr_r, thr_p, st.r0, st.r1, st.r2, st.r3);
   }
 }
 

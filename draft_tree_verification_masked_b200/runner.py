@@ -53,10 +53,12 @@ class DeviceStep:
     page_size: lay the caches out in pages of that many tokens at shuffled pool pages and use
     the paged attention and compaction calls (the pools replace k_cache / v_cache).
     kv_len_max: the batch's host-side bound on kv_len (default: the largest kv_len); a looser
-    bound is valid and sizes the attention grid for it."""
+    bound is valid and sizes the attention grid for it.
+    materialize (T > 0): use the tree entry point with a logit buffer of n_total rows, so that the
+    bonus draw reads the stop rows' stored logits instead of making a second pass over the head."""
 
     def __init__(self, wl, device: str = "cuda", n_layers: int = 1, tree=None, zbuf_rows=None,
-                 page_size=None, kv_len_max=None):
+                 page_size=None, kv_len_max=None, materialize: bool = False):
         self.wl = wl
         self.device = device
         dev = torch.device(device)
@@ -134,6 +136,9 @@ class DeviceStep:
         etree_workspace_init(self.ws)
         self.scale = 1.0 / float(wl.head_dim) ** 0.5
         nbr = branching_nodes(wl)
+        self.materialize = bool(materialize) and wl.temperature > 0
+        if self.materialize:
+            tree, zbuf_rows = True, wl.n_total
         self.tree = (wl.temperature > 0 and nbr > 0) if tree is None else bool(tree)
         rows = nbr if zbuf_rows is None else int(zbuf_rows)
         self.zbuf = (torch.empty(rows, wl.vocab, dtype=torch.float32, device=dev)

@@ -233,6 +233,11 @@ etree_status etree_lmhead_accept(const etree_batch *batch, const uint16_t *hidde
  *              than zbuf_rows records ETREE_ENOSPACE (detail 10) and the requests left without a
  *              row accept nothing: their bonus is drawn from the root's p (a one-token
  *              decode).  zbuf may be NULL when zbuf_rows == 0 (chains need no rows).
+ *              With zbuf_rows >= n_total, every node's logits are stored (row g for node g) and
+ *              the bonus draw reads the stop row there instead of making a second pass over
+ *              w_lm for the B stop rows: the tokens are the same, the second W pass (a GEMM of B
+ *              rows) is replaced by reading B logit rows, at the cost of n_total x vocab x 4
+ *              bytes of buffer.  This works for chains as well as trees.
  *   Other arguments as in etree_lmhead_accept (no node_argmax / node_gap outputs).
  * Errors: host-side as etree_lmhead_accept, plus ETREE_EINVAL for zbuf_rows < 0, a NULL zbuf
  * with zbuf_rows > 0, or a misaligned zbuf.

@@ -251,6 +251,22 @@ def test_tree64_t1_full_size():
     _full_check(W.generate("tree64_t1"))
 
 
+@pytest.mark.parametrize("name", ["conc512", "tree64_t1"])
+def test_materialised_draw_full_size(name):
+    """Every row's logits kept (zbuf of n_total rows): the bonus draw reads the stop rows there
+    instead of a second pass over W, chains and branching trees alike."""
+    dev, res = _full_check(W.generate(name), materialize=True, label=f"{name}_materialised")
+    assert dev.tree and dev.zbuf.shape[0] == dev.wl.n_total
+
+
+@pytest.mark.parametrize("T", [1.0, 0.6])
+def test_materialised_draw_small(T):
+    wl = W.generate("conc512", B=37, n_nodes=[4, 5, 6, 1, 2] * 7 + [4, 4], depth=5,
+                    depth_min=5, kv_len=(20, 400), hidden=512, vocab=4096 + 3, temperature=T)
+    _full_check(wl, materialize=True)
+    _full_check(_branching(T, 8192 + 5), materialize=True)
+
+
 def test_logit_buffer_overflow_reports_and_answers_the_rest():
     """Fewer logit rows than branching nodes: ETREE_ENOSPACE (detail 10); the requests whose
     branching nodes all got a row still match the oracle, the others accept nothing."""

@@ -48,7 +48,7 @@ class _Setup:
     """Head, hidden rows and draft rows of a V-token toy target, and a batch of R requests of
     n nodes each with parent array `par` (the same shape for every request)."""
 
-    def __init__(self, par, seed, q_scale=None):
+    def __init__(self, par, seed, q_scale=None, full=False):
         g = np.random.default_rng(seed)
         self.n = len(par)
         hid = torch.from_numpy(g.normal(0, 1, size=(self.n, H)).astype(np.float32)).bfloat16()
@@ -83,7 +83,9 @@ class _Setup:
         self.out = torch.empty(R, 65, **i32)
         self.node_argmax = torch.empty(R * self.n, **i32)
         self.node_gap = torch.empty(R * self.n, dtype=torch.float32, device=dev)
-        self.zbuf = torch.empty(R, V, dtype=torch.float32, device=dev)
+        # a row per branching node (the root), or with `full` a row per node: the draw then
+        # reads the stored stop rows instead of a second pass over the head
+        self.zbuf = torch.empty(R * (self.n if full else 1), V, dtype=torch.float32, device=dev)
 
     def draft(self, parent_rows):
         """Draft tokens for the given parent rows of every request, each drawn from that row's q
@@ -109,16 +111,19 @@ class _Setup:
         return (self.accept_len.cpu().numpy(), self.path.cpu().numpy(), self.out.cpu().numpy())
 
 
-def test_chain_sampler_emits_the_target_distribution():
+@pytest.mark.parametrize("mode", ["chain", "materialised"])
+def test_chain_sampler_emits_the_target_distribution(mode):
     """2-node chains: the first emitted token (the accepted draft, or the residual draw after a
     rejection) follows p_root; the draft is accepted with probability sum min(p, q); after an
-    acceptance the bonus follows p of the child."""
-    s = _Setup([-1, 0], seed=91)
+    acceptance the bonus follows p of the child.  `materialised`: the same through the tree entry
+    with every row's logits kept, whose draw reads the stored rows."""
+    full = mode == "materialised"
+    s = _Setup([-1, 0], seed=91, full=full)
     first, second, acc = [], [], []
     for step in range(CALLS):
         tok = np.zeros((R, 2), dtype=np.int32)
         tok[:, 1] = s.draft([0])[:, 0]
-        a, path, out = s.run(tok, step)
+        a, path, out = s.run(tok, step, tree=full)
         assert set(np.unique(a)) <= {0, 1}
         first.append(out[:, 0])
         second.append(out[a == 1, 1])
@@ -130,12 +135,14 @@ def test_chain_sampler_emits_the_target_distribution():
     assert _chisq_p(second, s.p[1]) > 1e-4
 
 
-def test_tree_sampler_emits_the_target_distribution_and_sibling_rates():
+@pytest.mark.parametrize("full", [False, True])
+def test_tree_sampler_emits_the_target_distribution_and_sibling_rates(full):
     """A root with three children drafted independently from q_root: the first emitted token
     follows p_root; child 1 is accepted with A1 = sum min(p, q); after its rejection the target
     is r1 = max(0, p - q) / (1 - A1) and child 2 is accepted with sum min(q, r1); after both
-    rejections r2 = max(0, p - c2 q) / N(c2) with c2 = 2 - A1, and child 3 with sum min(q, r2)."""
-    s = _Setup([-1, 0, 0, 0], seed=92)
+    rejections r2 = max(0, p - c2 q) / N(c2) with c2 = 2 - A1, and child 3 with sum min(q, r2).
+    With `full`, every row's logits are kept and the draw reads them."""
+    s = _Setup([-1, 0, 0, 0], seed=92, full=full)
     first, which = [], []
     for step in range(CALLS):
         tok = np.zeros((R, 4), dtype=np.int32)
@@ -159,13 +166,13 @@ def test_tree_sampler_emits_the_target_distribution_and_sibling_rates():
         assert abs(got - want) < 5 * np.sqrt(want * (1 - want) / n), (k, got, want)
 
 
-@pytest.mark.parametrize("tree", [False, True])
-def test_empty_residual_bonus_is_drawn_from_the_target(tree):
+@pytest.mark.parametrize("tree,full", [(False, False), (True, False), (True, True)])
+def test_empty_residual_bonus_is_drawn_from_the_target(tree, full):
     """q = 2p (an over-confident draft): every residual max(0, p - q) is empty, so each rejection
     (probability 1/2) is answered by a draw from p itself; together with the accepted drafts
     (x ~ q / 2 = p) the first emitted token follows p, and so does the bonus alone."""
     par = [-1, 0, 0] if tree else [-1, 0]
-    s = _Setup(par, seed=93, q_scale=2.0)
+    s = _Setup(par, seed=93, q_scale=2.0, full=full)
     first, rej = [], []
     calls = CALLS // 5
     for step in range(calls):
