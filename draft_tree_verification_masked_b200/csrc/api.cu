@@ -202,6 +202,23 @@ static etree_status get_map(const void* ptr, int rank, uint64_t d0, uint64_t d1,
   return ETREE_OK;
 }
 
+// fp32 2-D tensor map {d0 (contiguous), d1} with row stride d0 * 4 bytes and 64-byte swizzle, for
+// the TMA stores of materialised logit rows (box {b0, b1}).  Not cached: encoded per call.
+static etree_status get_map_f32_sw64(const void* ptr, uint64_t d0, uint64_t d1, uint32_t b0,
+                                     uint32_t b1, CUtensorMap* out) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(ETREE_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {d0, d1};
+  cuuint64_t strides[1] = {d0 * 4};
+  cuuint32_t box[2] = {b0, b1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ETREE_ECUDA, "cuTensorMapEncodeTiled (fp32) failed (%d)", (int)r);
+  return ETREE_OK;
+}
+
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 static etree_status check_batch(const etree_batch* b) {
@@ -442,7 +459,7 @@ etree_status etree_lowrank_candidates(const uint16_t* hidden, int M, int hidden_
   gp.n_parts = gp.per_cta ? grid : gp.n_tiles;
   gp.topk = at<float2>(workspace, w.lists);
   gp.tkth = tkth;
-  e = launch_lmhead(3, bn, bm, ta, tb, gp, grid, s);
+  e = launch_lmhead(3, bn, bm, ta, tb, tb, gp, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "etree_lowrank_candidates (screen)");
   e = launch_lowrank_finish(gp.topk, 2 * gp.n_parts, tkth, M, k, at<int32_t>(workspace, w.cand),
                             hb,
@@ -735,7 +752,7 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
   cudaError_t e;
   if (temperature == 0.f) {
     mark(0);
-    e = launch_lmhead(0, bn, bm, ta, tb, g, grid, s);
+    e = launch_lmhead(0, bn, bm, ta, tb, tb, g, grid, s);
     mark(1);
     if (e == cudaSuccess) e = launch_accept_greedy(a, at<int32_t>(workspace, w.child_tok), cnt, s);
     mark(2);
@@ -745,7 +762,7 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
   if (!tree) {                               // chains: accept tests fused with the row merge
     e = launch_chain_prep(a, at<int32_t>(workspace, w.child_tok), s);
     mark(0);
-    if (e == cudaSuccess) e = launch_lmhead(1, bn, bm, ta, tb, g, grid, s);
+    if (e == cudaSuccess) e = launch_lmhead(1, bn, bm, ta, tb, tb, g, grid, s);
     mark(1);
     if (e == cudaSuccess) e = launch_accept_chain(a, cnt, s);
   } else {                                   // trees: materialised rows of branching nodes
@@ -757,7 +774,15 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
     g.child_tok = nullptr;
     g.zrow = zrow;
     g.zbuf = tree->zbuf;
-    if (e == cudaSuccess) e = launch_lmhead(1, bn, bm, ta, tb, g, grid, s);
+    // every row kept at M >= 128 rows: the rows leave through TMA stores of 32 x 16 boxes
+    CUtensorMap tz = tb;
+    if (tree->rows >= b->n_total && bm == 128 && (vocab & 3) == 0 && aligned16(tree->zbuf)) {
+      if ((st = get_map_f32_sw64(tree->zbuf, (uint64_t)vocab, (uint64_t)b->n_total, 16, 32, &tz)))
+        return st;
+      g.z_tma = 1;
+    }
+    if (e == cudaSuccess) e = launch_lmhead(1, bn, bm, ta, tb, tz, g, grid, s);
+    g.z_tma = 0;
     mark(1);
     g.zrow = nullptr;
     g.zbuf = nullptr;
@@ -790,7 +815,7 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
   g2.cnt = nullptr;
   g2.rfloor = a.rfloor;
   a.n_tiles2 = 2 * g2.n_parts;
-  e = launch_lmhead(2, bn2, bm2, th, tb2, g2, grid2, s);
+  e = launch_lmhead(2, bn2, bm2, th, tb2, tb2, g2, grid2, s);
   mark(3);
   if (e == cudaSuccess) e = launch_bonus(a, s);
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T>0, pass 2)");

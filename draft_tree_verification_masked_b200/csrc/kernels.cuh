@@ -58,6 +58,8 @@ struct GemmParams {
   int cnt_n;
   const int32_t* zrow;              // EPI_LSE, if set: row g's logits go to zbuf[zrow[g]][V]
   float* zbuf;                      // when zrow[g] >= 0 (rows of branching tree nodes)
+  int z_tma;                        // EPI_LSE, BM = 128: every row is stored (zrow[g] = g) through
+                                    // the tm_z tensor map (32-row x 16-column boxes)
   float2* topk;                     // EPI_TOPK: per (row, slot, half) 16 (value, id bits)
   uint32_t* tkth;                   // EPI_TOPK: per row, order-encoded lower bound of the k-th
   WsHeader* ws;
@@ -78,7 +80,8 @@ struct GemmParams {
 };
 int lmhead_pick_bn(int M, int V, int grid);
 cudaError_t launch_lmhead(int epi, int bn, int bm, const CUtensorMap& ta, const CUtensorMap& tb,
-                          const GemmParams& p, int grid, cudaStream_t stream);
+                          const CUtensorMap& tz, const GemmParams& p, int grid,
+                          cudaStream_t stream);
 
 struct AcceptParams {
   int B, n_total, n_max, V, n_tiles, n_tiles2;

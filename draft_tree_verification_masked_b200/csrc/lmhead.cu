@@ -196,17 +196,46 @@ __device__ __forceinline__ void load_q(const GemmParams& p, const float* qrow, i
   }
 }
 
+// One 16-column slice of a warp's 32 rows to the materialised logit rows by a TMA store: each
+// lane writes its row's 16 values (from v[off ..]) into the warp's staging box in the tensor
+// map's 64-byte swizzle (16-byte chunk k of row r sits at chunk k ^ ((r >> 1) & 3)), then lane 0
+// stores the box at (col0, row0).  Rows past n_total and columns past the vocabulary lie outside
+// the tensor and are not written.  zpend: lane 0 has a store in flight that may still read zbox.
+template <int W, int N>
+__device__ __forceinline__ void stage_z(const CUtensorMap* tm, float* zbox, const float (&v)[N],
+                                        int off, int col0, int row0, int lane, bool& zpend,
+                                        int V, int M) {
+  static_assert(W == 16, "16-column boxes");
+  if (col0 >= V || row0 >= M) return;                 // wholly outside the tensor: nothing to store
+  if (lane == 0 && zpend) tma_store_wait_read();
+  __syncwarp();
+  float4* rowp = reinterpret_cast<float4*>(zbox + lane * 16);
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    rowp[k ^ sw] = make_float4(v[off + 4 * k], v[off + 4 * k + 1], v[off + 4 * k + 2],
+                               v[off + 4 * k + 3]);
+  fence_proxy_async();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm, zbox, col0, row0);
+    tma_store_commit();
+    zpend = true;
+  }
+}
+
 constexpr int kEpiWarps = 8;                 // two warps per TMEM lane quarter
 constexpr int kGemmThreads = 32 * (2 + kEpiWarps);
 
 template <int EPI, int BN, int BM>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                   GemmParams p) {
+                   const __grid_constant__ CUtensorMap tm_z, GemmParams p) {
   constexpr int kABytes = BM * kBK * 2;
   constexpr int kBBytes = BN * kBK * 2;
   constexpr int kGStages = gemm_stages(BM, BN);
   constexpr int kBM = BM;
+  constexpr bool kZTma = EPI == EPI_LSE && BM == 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -218,6 +247,10 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   uint64_t* acce = accf + 2;
   uint64_t* drain = acce + 2;                // the MMA issuer's last commit, waited on at exit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  // EPI_LSE at BM = 128: one 32-row x 16-column fp32 staging box per epilogue warp (64-byte
+  // swizzle) for the TMA stores of materialised logit rows, 1024-aligned after the barriers
+  float* zstage = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(tmem_slot + 4) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -343,6 +376,8 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     EpiRow st;
     TopK16 tk;
     tk.clear();
+    float* zbox = zstage + (warp - 2) * (32 * 16);    // this warp's staging box
+    bool zpend = false;                               // a TMA store from zbox may be reading it
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++ai) {
       const int buf = ai & 1;
       const uint32_t aph = (ai >> 1) & 1;
@@ -367,8 +402,9 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       float tfloor = -INFINITY;
       if (EPI == EPI_TOPK && active) tfloor = dec_order(__ldcg(p.tkth + grow));
       if (EPI == EPI_LSE && active && p.child_tok) st.ct = p.child_tok[grow];
-      const int zr = (EPI == EPI_LSE && active && p.zrow) ? p.zrow[grow] : -1;
+      const int zr = (EPI == EPI_LSE && active && p.zrow && !p.z_tma) ? p.zrow[grow] : -1;
       float* zdst = zr >= 0 ? p.zbuf + (size_t)zr * p.V : nullptr;
+      const int row0 = mt * kBM + wq * 32;            // first row of this warp's TMA boxes
       if (EPI == EPI_RACE && active) {
         const int g = p.stop_row[grow];
         st.unode = p.stop_node[grow];
@@ -400,7 +436,16 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           } else {
             if (active) epi_chunk<EPI, 32>(p, st, v, nt * BN + c * 32);
           }
-          if (EPI == EPI_LSE && zdst) store_logits<32>(p, zdst, v, nt * BN + c * 32);
+          if constexpr (kZTma) {
+            if (p.z_tma) {
+              stage_z<16>(&tm_z, zbox, v, 0, nt * BN + c * 32, row0, lane, zpend, p.V, p.M);
+              stage_z<16>(&tm_z, zbox, v, 16, nt * BN + c * 32 + 16, row0, lane, zpend, p.V, p.M);
+            } else if (zdst) {
+              store_logits<32>(p, zdst, v, nt * BN + c * 32);
+            }
+          } else {
+            if (EPI == EPI_LSE && zdst) store_logits<32>(p, zdst, v, nt * BN + c * 32);
+          }
         }
         if constexpr (BN % 32 == 16) {
           if (half == kTailHalf) {
@@ -417,7 +462,14 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
             } else {
               if (active) epi_chunk<EPI, 16>(p, st, v, nt * BN + kChunks * 32);
             }
-            if (EPI == EPI_LSE && zdst) store_logits<16>(p, zdst, v, nt * BN + kChunks * 32);
+            if constexpr (kZTma) {
+              if (p.z_tma)
+                stage_z<16>(&tm_z, zbox, v, 0, nt * BN + kChunks * 32, row0, lane, zpend, p.V, p.M);
+              else if (zdst)
+                store_logits<16>(p, zdst, v, nt * BN + kChunks * 32);
+            } else {
+              if (EPI == EPI_LSE && zdst) store_logits<16>(p, zdst, v, nt * BN + kChunks * 32);
+            }
           }
         }
       }
@@ -450,6 +502,8 @@ lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         if (EPI == EPI_LSE && st.found) p.zchild[grow] = st.zc;
       }
     }
+    // the materialised rows' TMA stores complete before the CTA exits
+    if (kZTma && lane == 0 && zpend) tma_store_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -483,50 +537,54 @@ int lmhead_pick_bn(int M, int V, int grid) {
   return best;
 }
 
-template <int BM>
+template <int EPI, int BM>
 static size_t lmhead_smem_bytes(int bn) {
-  return (size_t)gemm_stages(BM, bn) * (BM + bn) * kBK * 2 + 1024 + (2 * 6 + 5) * 8 + 16;
+  const size_t base = (size_t)gemm_stages(BM, bn) * (BM + bn) * kBK * 2 + 1024 + (2 * 6 + 5) * 8 + 16;
+  // EPI_LSE at BM = 128: 1 KB of alignment and eight 2 KB staging boxes for the TMA stores
+  return (EPI == EPI_LSE && BM == 128) ? base + 1024 + kEpiWarps * 32 * 16 * 4 : base;
 }
 
 template <int EPI, int BN, int BM>
-static cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
-                             int grid, cudaStream_t stream) {
-  const size_t smem = lmhead_smem_bytes<BM>(BN);
+static cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tz,
+                             const GemmParams& p, int grid, cudaStream_t stream) {
+  const size_t smem = lmhead_smem_bytes<EPI, BM>(BN);
   auto k = lmhead_gemm_kernel<EPI, BN, BM>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k, dim3(grid), dim3(kGemmThreads), smem, stream, ta, tb, p);
+  return launch_pdl(k, dim3(grid), dim3(kGemmThreads), smem, stream, ta, tb, tz, p);
 }
 
 template <int EPI, int BM>
 static cudaError_t launch_epi(int bn, const CUtensorMap& ta, const CUtensorMap& tb,
-                              const GemmParams& p, int grid, cudaStream_t s) {
+                              const CUtensorMap& tz, const GemmParams& p, int grid,
+                              cudaStream_t s) {
   switch (bn) {
-    case 256: return launch_bn<EPI, 256, BM>(ta, tb, p, grid, s);
-    case 224: return launch_bn<EPI, 224, BM>(ta, tb, p, grid, s);
-    case 208: return launch_bn<EPI, 208, BM>(ta, tb, p, grid, s);
-    case 192: return launch_bn<EPI, 192, BM>(ta, tb, p, grid, s);
-    case 176: return launch_bn<EPI, 176, BM>(ta, tb, p, grid, s);
-    case 160: return launch_bn<EPI, 160, BM>(ta, tb, p, grid, s);
-    case 144: return launch_bn<EPI, 144, BM>(ta, tb, p, grid, s);
-    case 128: return launch_bn<EPI, 128, BM>(ta, tb, p, grid, s);
+    case 256: return launch_bn<EPI, 256, BM>(ta, tb, tz, p, grid, s);
+    case 224: return launch_bn<EPI, 224, BM>(ta, tb, tz, p, grid, s);
+    case 208: return launch_bn<EPI, 208, BM>(ta, tb, tz, p, grid, s);
+    case 192: return launch_bn<EPI, 192, BM>(ta, tb, tz, p, grid, s);
+    case 176: return launch_bn<EPI, 176, BM>(ta, tb, tz, p, grid, s);
+    case 160: return launch_bn<EPI, 160, BM>(ta, tb, tz, p, grid, s);
+    case 144: return launch_bn<EPI, 144, BM>(ta, tb, tz, p, grid, s);
+    case 128: return launch_bn<EPI, 128, BM>(ta, tb, tz, p, grid, s);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_lmhead(int epi, int bn, int bm, const CUtensorMap& ta, const CUtensorMap& tb,
-                          const GemmParams& p, int grid, cudaStream_t stream) {
+                          const CUtensorMap& tz, const GemmParams& p, int grid,
+                          cudaStream_t stream) {
   if (epi == EPI_TOPK)
-    return bm == 64 ? launch_epi<EPI_TOPK, 64>(bn, ta, tb, p, grid, stream)
-                    : launch_epi<EPI_TOPK, 128>(bn, ta, tb, p, grid, stream);
+    return bm == 64 ? launch_epi<EPI_TOPK, 64>(bn, ta, tb, tz, p, grid, stream)
+                    : launch_epi<EPI_TOPK, 128>(bn, ta, tb, tz, p, grid, stream);
   if (bm == 64) {
-    if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX, 64>(bn, ta, tb, p, grid, stream);
-    if (epi == EPI_LSE) return launch_epi<EPI_LSE, 64>(bn, ta, tb, p, grid, stream);
-    return launch_epi<EPI_RACE, 64>(bn, ta, tb, p, grid, stream);
+    if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX, 64>(bn, ta, tb, tz, p, grid, stream);
+    if (epi == EPI_LSE) return launch_epi<EPI_LSE, 64>(bn, ta, tb, tz, p, grid, stream);
+    return launch_epi<EPI_RACE, 64>(bn, ta, tb, tz, p, grid, stream);
   }
-  if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX, 128>(bn, ta, tb, p, grid, stream);
-  if (epi == EPI_LSE) return launch_epi<EPI_LSE, 128>(bn, ta, tb, p, grid, stream);
-  return launch_epi<EPI_RACE, 128>(bn, ta, tb, p, grid, stream);
+  if (epi == EPI_ARGMAX) return launch_epi<EPI_ARGMAX, 128>(bn, ta, tb, tz, p, grid, stream);
+  if (epi == EPI_LSE) return launch_epi<EPI_LSE, 128>(bn, ta, tb, tz, p, grid, stream);
+  return launch_epi<EPI_RACE, 128>(bn, ta, tb, tz, p, grid, stream);
 }
 
 }  // namespace etree

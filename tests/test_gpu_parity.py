@@ -255,16 +255,37 @@ def test_tree64_t1_full_size():
 def test_materialised_draw_full_size(name):
     """Every row's logits kept (zbuf of n_total rows): the bonus draw reads the stop rows there
     instead of a second pass over W, chains and branching trees alike."""
-    dev, res = _full_check(W.generate(name), materialize=True, label=f"{name}_materialised")
-    assert dev.tree and dev.zbuf.shape[0] == dev.wl.n_total
+    wl = W.generate(name)
+    dev, res = _full_check(wl, materialize=True, label=f"{name}_materialised")
+    assert dev.tree and dev.zbuf.shape[0] == wl.n_total
+    _stored_logits_check(wl, dev)
+
+
+def _stored_logits_check(wl, dev, nrows=40):
+    """The stored rows are the logits themselves (fp32 accumulation of bf16 products over the
+    hidden size: within 1e-3 (1 + |z|) of fp64), each in its own row, on sampled rows including
+    the first and last (row tiles and vocab tails)."""
+    import oracle
+    g = np.random.default_rng(7)
+    rows = np.unique(np.concatenate([[0, wl.n_total - 1],
+                                     g.integers(0, wl.n_total, nrows)])).astype(np.int32)
+    z = oracle.logits(wl.hidden, wl.w_lm, rows)
+    got = dev.zbuf[torch.as_tensor(rows, dtype=torch.long, device=dev.zbuf.device)].cpu().numpy()
+    assert np.all(np.abs(got - z) <= 1e-3 * (1.0 + np.abs(z))), float(np.abs(got - z).max())
 
 
 @pytest.mark.parametrize("T", [1.0, 0.6])
 def test_materialised_draw_small(T):
     wl = W.generate("conc512", B=37, n_nodes=[4, 5, 6, 1, 2] * 7 + [4, 4], depth=5,
                     depth_min=5, kv_len=(20, 400), hidden=512, vocab=4096 + 3, temperature=T)
-    _full_check(wl, materialize=True)
-    _full_check(_branching(T, 8192 + 5), materialize=True)
+    dev, _ = _full_check(wl, materialize=True)
+    _stored_logits_check(wl, dev)
+    wl = _branching(T, 8192 + 4)
+    dev, _ = _full_check(wl, materialize=True)
+    _stored_logits_check(wl, dev)
+    wl = _branching(T, 8192 + 5)                          # vocab not a multiple of 4: direct stores
+    dev, _ = _full_check(wl, materialize=True)
+    _stored_logits_check(wl, dev)
 
 
 def test_logit_buffer_overflow_reports_and_answers_the_rest():
