@@ -917,7 +917,7 @@ static etree_status kv_compact_impl(const etree_batch* b, const int32_t* accept_
   p.page_shift = pg ? log2i(pg->page_size) : 0;
   p.cache_slots = pool_slots;
   // the layers are spread over about 16 CTAs per SM
-  cudaError_t e = launch_compact(p, 16 * sm_count(), static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_compact(p, 32 * sm_count(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_kv_compact launch");
 }
 

@@ -17,12 +17,14 @@ namespace etree {
 
 // One CTA per (request, chunk of layers).  Thread 0 reads and validates the request's header
 // while the first 64 threads read its path row; the first a + 1 threads then form the source
-// rows and the destination slots.  The copy treats the chunk as a flat list of items, one item being one moved row
-// (layer, k) for both tensors.  A row is w16 16-byte words for K followed by w16 for V; each
-// thread owns one word column and walks the items with kUnroll independent loads in flight
-// before their stores, so a copy of a few rows per layer is not serialised layer by layer.
-constexpr int kCompactThreads = 256;
-constexpr int kUnroll = 8;
+// rows and the destination slots.  The copy treats the chunk as a flat list of items, one item
+// being one moved row (layer, k) for both tensors.  A row is w16 16-byte words for K followed by
+// w16 for V; each thread owns every kCompactThreads-th word column and walks the items with
+// kUnroll independent loads in flight before their stores, so a copy of a few rows per layer is
+// not serialised layer by layer.  The shape (128 threads, 4 loads in flight, about 32 CTAs per
+// SM) was the fastest of the swept ones at 64 layers for batches of 64 and 512 requests.
+constexpr int kCompactThreads = 128;
+constexpr int kUnroll = 4;
 
 __global__ void __launch_bounds__(kCompactThreads)
     kv_compact_kernel(CompactParams p, int layers_per_cta) {
