@@ -12,6 +12,8 @@
 // One warp per node row reduces the row across the LM head's partial summaries; the warp that
 // completes a request's last row then takes the request's acceptance step (a ballot walk over
 // the <= 64 nodes at T = 0, the sequential accept test along the chain at T > 0).
+#include <algorithm>
+
 #include "kernels.cuh"
 #include "philox.cuh"
 #include "race.cuh"
@@ -683,21 +685,26 @@ __global__ void __launch_bounds__(256) bonus_kernel(AcceptParams p) {
   }
 }
 
-// The bonus draw from materialised logits, one CTA per request: the races of race.cuh over the
-// stop row's stored logits and its draft row (the same fp32 logits the first GEMM pass produced,
-// so the tokens equal those of a second pass over W).  Thread t takes the 8-id groups t,
-// t + blockDim, ...; a CTA-wide floor in shared memory (keys of real ids) sharpens each thread's
-// screen; the leaders are merged by a total order (larger key, then lower id), so the result does
-// not depend on the thread mapping.
-constexpr int kDrawThreads = 512;
+// The bonus draw from materialised logits: the races of race.cuh over the stop row's stored
+// logits and its draft row (the same fp32 logits the first GEMM pass produced, so the tokens
+// equal those of a second pass over W).  A request's vocabulary is split into `parts` ranges of
+// whole 8-id groups, one CTA each, so that small batches still fill the SMs.  Thread t of a CTA
+// takes the groups t, t + blockDim, ... of its range; a CTA-wide floor in shared memory (keys of
+// real ids) sharpens each thread's screen.  Leaders are merged by a total order (larger key, then
+// lower id), so the result does not depend on the mapping: within the CTA by shuffles, across
+// the parts by the CTA that arrives last (a per-request counter that the first GEMM pass zeroed)
+// over the parts' summaries.
+constexpr int kDrawThreads = 256;
 
 __global__ void __launch_bounds__(kDrawThreads) draw_rows_kernel(AcceptParams p,
                                                                  const int32_t* zrow,
-                                                                 const float* zbuf) {
+                                                                 const float* zbuf, int parts,
+                                                                 float4* dpart, int32_t* dcnt) {
   __shared__ unsigned fl_s[2];                        // floors (fp32 bits of positive keys)
   __shared__ float kr_s[kDrawThreads / 32], kp_s[kDrawThreads / 32];
   __shared__ int ir_s[kDrawThreads / 32], ip_s[kDrawThreads / 32];
-  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r = blockIdx.x / parts, part = blockIdx.x % parts;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int base, n;
   if (!request_ok(p, r, base, n)) return;            // answered by the walk
   if (tid == 0) fl_s[0] = fl_s[1] = 0u;
@@ -713,7 +720,9 @@ __global__ void __launch_bounds__(kDrawThreads) draw_rows_kernel(AcceptParams p,
   int ir = -1, ip = -1;
   float thr_r = 0.f, thr_p = 0.f;
   const int groups = (p.V + 7) / 8;
-  for (int g = tid; zr >= 0 && g < groups; g += kDrawThreads) {
+  const int per = (groups + parts - 1) / parts;
+  const int g1 = min(groups, (part + 1) * per);
+  for (int g = part * per + tid; zr >= 0 && g < g1; g += kDrawThreads) {
     const int c0 = g * 8;
     float zz[8], qq[8];
     if ((p.V & 7) == 0) {
@@ -758,19 +767,41 @@ __global__ void __launch_bounds__(kDrawThreads) draw_rows_kernel(AcceptParams p,
     ip_s[warp] = ip;
   }
   __syncthreads();
-  if (tid == 0) {
-    for (int w = 1; w < kDrawThreads / 32; ++w) {
-      merge_key(kr, ir, kr_s[w], ir_s[w]);
-      merge_key(kp, ip, kp_s[w], ip_s[w]);
-    }
-    const int a = p.accept_len[r];
-    p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = ir >= 0 ? ir : ip;
+  if (tid != 0) return;
+  for (int w = 1; w < kDrawThreads / 32; ++w) {
+    merge_key(kr, ir, kr_s[w], ir_s[w]);
+    merge_key(kp, ip, kp_s[w], ip_s[w]);
   }
+  if (parts > 1) {
+    dpart[(size_t)r * parts + part] =
+        make_float4(kr, __int_as_float(ir), kp, __int_as_float(ip));
+    __threadfence();
+    if (atomicAdd(dcnt + r, 1) != parts - 1) return;   // not the last part to finish
+    __threadfence();
+    for (int q2 = 0; q2 < parts; ++q2) {
+      const float4 x = __ldcg(dpart + (size_t)r * parts + q2);
+      merge_key(kr, ir, x.x, __float_as_int(x.y));
+      merge_key(kp, ip, x.z, __float_as_int(x.w));
+    }
+  }
+  const int a = p.accept_len[r];
+  p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = ir >= 0 ? ir : ip;
+}
+
+// Parts per request: about 8 CTAs per SM in all, at most 32 per request, no more than the
+// request's 8-id groups or the summary slots (max_parts).
+int draw_parts(int B, int V, int sms, int max_parts) {
+  const int groups = (V + 7) / 8;
+  int parts = (8 * sms + B - 1) / std::max(1, B);
+  parts = std::min(parts, 32);
+  parts = std::min(parts, std::max(1, groups / kDrawThreads));
+  parts = std::min(parts, max_parts);
+  return std::max(1, parts);
 }
 
 cudaError_t launch_draw_rows(const AcceptParams& p, const int32_t* zrow, const float* zbuf,
-                             cudaStream_t s) {
-  draw_rows_kernel<<<p.B, kDrawThreads, 0, s>>>(p, zrow, zbuf);
+                             int parts, float4* dpart, int32_t* dcnt, cudaStream_t s) {
+  draw_rows_kernel<<<p.B * parts, kDrawThreads, 0, s>>>(p, zrow, zbuf, parts, dpart, dcnt);
   return cudaGetLastError();
 }
 

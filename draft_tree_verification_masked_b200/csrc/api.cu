@@ -145,19 +145,19 @@ static EncodeTiledFn encode_fn() {
 
 struct MapKey {
   uintptr_t ptr;
-  uint64_t d0, d1, d2;
+  uint64_t d0, d1, d2, rs;
   uint32_t b0, b1, b2, rank;
   int dev;
   bool operator==(const MapKey& o) const {
-    return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && b0 == o.b0 && b1 == o.b1 &&
-           b2 == o.b2 && rank == o.rank && dev == o.dev;
+    return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && rs == o.rs && b0 == o.b0 &&
+           b1 == o.b1 && b2 == o.b2 && rank == o.rank && dev == o.dev;
   }
 };
 struct MapKeyHash {
   size_t operator()(const MapKey& k) const {
     size_t h = std::hash<uintptr_t>()(k.ptr);
-    h ^= std::hash<uint64_t>()(k.d0 * 1315423911u + k.d1 * 2654435761u + k.d2) + 0x9e3779b9 +
-         (h << 6) + (h >> 2);
+    h ^= std::hash<uint64_t>()(k.d0 * 1315423911u + k.d1 * 2654435761u + k.d2 + k.rs * 40503u) +
+         0x9e3779b9 + (h << 6) + (h >> 2);
     h ^= (size_t)k.b0 * 31 + k.b1 * 17 + k.b2 * 7 + k.rank + (size_t)k.dev * 101;
     return h;
   }
@@ -168,11 +168,15 @@ static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
 
 // bf16 tensor map with 128-byte swizzle.  rank 2: dims {d0, d1}, row stride d0*2 bytes;
 // rank 3: dims {d0, d1, d2}, strides {d0*2, d0*d1*2}.  Cached per (pointer, shape, box, device).
-static etree_status get_map(const void* ptr, int rank, uint64_t d0, uint64_t d1, uint64_t d2,
-                            uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMap* out) {
+// A bf16 tensor map with 128-byte swizzle, dims {d0 (contiguous), d1, d2}, box {b0, b1, b2}.  Rows
+// (dimension 1) are row_bytes apart, or d0 * 2 bytes when row_bytes is 0.  Cached per key.
+static etree_status get_map_rows(const void* ptr, int rank, uint64_t d0, uint64_t d1, uint64_t d2,
+                                 uint64_t row_bytes, uint32_t b0, uint32_t b1, uint32_t b2,
+                                 CUtensorMap* out) {
   int dev = 0;
   cudaGetDevice(&dev);
-  MapKey key{reinterpret_cast<uintptr_t>(ptr), d0, d1, d2, b0, b1, b2, (uint32_t)rank, dev};
+  MapKey key{reinterpret_cast<uintptr_t>(ptr), d0, d1, d2, row_bytes, b0, b1, b2,
+             (uint32_t)rank, dev};
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto it = g_maps.find(key);
@@ -184,7 +188,8 @@ static etree_status get_map(const void* ptr, int rank, uint64_t d0, uint64_t d1,
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(ETREE_ECUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const uint64_t rb = row_bytes ? row_bytes : d0 * 2;
+  cuuint64_t strides[2] = {rb, rb * d1};
   cuuint32_t box[3] = {b0, b1, b2};
   cuuint32_t estr[3] = {1, 1, 1};
   CUtensorMap m;
@@ -200,6 +205,11 @@ static etree_status get_map(const void* ptr, int rank, uint64_t d0, uint64_t d1,
   }
   *out = m;
   return ETREE_OK;
+}
+
+static etree_status get_map(const void* ptr, int rank, uint64_t d0, uint64_t d1, uint64_t d2,
+                            uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMap* out) {
+  return get_map_rows(ptr, rank, d0, d1, d2, 0, b0, b1, b2, out);
 }
 
 // fp32 2-D tensor map {d0 (contiguous), d1} with row stride d0 * 4 bytes and 64-byte swizzle, for
@@ -387,7 +397,7 @@ static LowrankLayout lowrank_layout(int M, int H, int r, int V) {
   };
   w.nk = lowrank_down_chunks(H);
   w.nlists = 2 * ((V + 127) / 128);                 // per vocab tile at the narrowest width
-  // the down projection's chunk partials, or the sample's
+  // the sample's split-K partials (or the down projection's, in its split-K form)
   const size_t sample = (size_t)((r + 127) / 128) * M * lowrank_sample_cols(V);
   w.part = take(std::max((size_t)w.nk * M * r, sample) * sizeof(float));
   w.g = take((size_t)M * r * 2);
@@ -428,21 +438,28 @@ etree_status etree_lowrank_candidates(const uint16_t* hidden, int M, int hidden_
   const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(hidden);
   __nv_bfloat16* g = at<__nv_bfloat16>(workspace, w.g);
   uint32_t* tkth = at<uint32_t>(workspace, w.tkth);
+  CUtensorMap th, td, tg, tus;
+  etree_status st;
+  if ((st = get_map(hidden, 2, hidden_dim, M, 1, 64, 64, 1, &th))) return st;
+  if ((st = get_map(D, 2, hidden_dim, rank, 1, 64, 64, 1, &td))) return st;
+  if ((st = get_map(g, 2, rank, M, 1, 64, 64, 1, &tg))) return st;
+  // the sample: every stride-th row of U
+  const int S = lowrank_sample_cols(vocab), stride = vocab / S;
+  if ((st = get_map_rows(U, 2, rank, S, 1, (uint64_t)stride * rank * 2, 64, 64, 1, &tus)))
+    return st;
   int32_t* fcnt = at<int32_t>(workspace, w.fcnt);
-  cudaError_t e = launch_lowrank_down(hb, reinterpret_cast<const __nv_bfloat16*>(D), M,
-                                      hidden_dim, rank, at<float>(workspace, w.part), g, tkth,
-                                      fcnt, s);
+  float* part = at<float>(workspace, w.part);
+  WsHeader* ws = at<WsHeader>(workspace, 0);
+  cudaError_t e = launch_lowrank_down(th, td, M, hidden_dim, rank, part, g, tkth, fcnt, ws, s);
   if (e == cudaSuccess)
-    e = launch_lowrank_sample(g, reinterpret_cast<const __nv_bfloat16*>(U), M, rank, vocab,
-                              at<float>(workspace, w.part), at<float>(workspace, w.fmax), fcnt,
-                              tkth, s);
+    e = launch_lowrank_sample(tg, tus, M, rank, vocab, part, at<float>(workspace, w.fmax), fcnt,
+                              tkth, ws, s);
   if (e != cudaSuccess) return cuda_fail(e, "etree_lowrank_candidates (down, sample)");
 
   const int sms = sm_count();
   const int bn = lmhead_pick_bn(M, vocab, sms);
   const int bm = M <= 64 ? 64 : 128;
   CUtensorMap ta, tb;
-  etree_status st;
   if ((st = get_map(g, 2, rank, M, 1, 64, bm, 1, &ta))) return st;
   if ((st = get_map(U, 2, rank, vocab, 1, 64, bn, 1, &tb))) return st;
   GemmParams gp{};
@@ -461,8 +478,7 @@ etree_status etree_lowrank_candidates(const uint16_t* hidden, int M, int hidden_
   gp.tkth = tkth;
   e = launch_lmhead(3, bn, bm, ta, tb, tb, gp, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "etree_lowrank_candidates (screen)");
-  e = launch_lowrank_finish(gp.topk, 2 * gp.n_parts, tkth, M, k, at<int32_t>(workspace, w.cand),
-                            hb,
+  e = launch_lowrank_finish(gp.topk, 2 * gp.n_parts, M, k, at<int32_t>(workspace, w.cand), hb,
                             reinterpret_cast<const __nv_bfloat16*>(W), hidden_dim, vocab,
                             out_ids, out_logit, s);
   return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lowrank_candidates (rescore)");
@@ -791,7 +807,8 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
       // every row's logits are in zbuf: the draw reads the stop rows there (no second W pass)
       mark(2);
       mark(3);
-      e = launch_draw_rows(a, zrow, tree->zbuf, s);
+      const int parts = draw_parts(b->B, vocab, sms, w.n_tiles);
+      e = launch_draw_rows(a, zrow, tree->zbuf, parts, at<float4>(workspace, w.part2), cnt, s);
       return e == cudaSuccess ? ETREE_OK : cuda_fail(e, "etree_lmhead_accept (T>0, draw)");
     }
   }

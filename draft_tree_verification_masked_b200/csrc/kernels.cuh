@@ -114,27 +114,26 @@ cudaError_t launch_accept_greedy(const AcceptParams& p, int32_t* arg_ws, int32_t
 cudaError_t launch_chain_prep(const AcceptParams& p, int32_t* child_tok, cudaStream_t s);
 cudaError_t launch_accept_chain(const AcceptParams& p, int32_t* cnt, cudaStream_t s);
 cudaError_t launch_bonus(const AcceptParams& p, cudaStream_t s);
+int draw_parts(int B, int V, int sms, int max_parts);
 cudaError_t launch_draw_rows(const AcceptParams& p, const int32_t* zrow, const float* zbuf,
-                             cudaStream_t s);
+                             int parts, float4* dpart, int32_t* dcnt, cudaStream_t s);
 cudaError_t launch_tree_prep(const AcceptParams& p, const __nv_bfloat16* w_lm, int32_t* ccount,
                              int32_t* zrow, int zbuf_rows, float* zc, cudaStream_t s);
 cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32_t* zrow,
                              const float* zbuf, cudaStream_t s);
 
 int lowrank_down_chunks(int H);
-cudaError_t launch_lowrank_down(const __nv_bfloat16* hid, const __nv_bfloat16* D, int M, int H,
-                                int r, float* part, __nv_bfloat16* g, uint32_t* tkth,
-                                int32_t* fcnt, cudaStream_t s);
 int lowrank_sample_cols(int V);
 int lowrank_floor_maxima(int M);
-cudaError_t launch_lowrank_sample(const __nv_bfloat16* g, const __nv_bfloat16* U, int M, int r,
+cudaError_t launch_lowrank_down(const CUtensorMap& tm_h, const CUtensorMap& tm_d, int M, int H,
+                                int r, float* part, __nv_bfloat16* g, uint32_t* tkth,
+                                int32_t* fcnt, WsHeader* ws, cudaStream_t s);
+cudaError_t launch_lowrank_sample(const CUtensorMap& tm_g, const CUtensorMap& tm_us, int M, int r,
                                   int V, float* part, float* fmax, int32_t* fcnt, uint32_t* tkth,
-                                  cudaStream_t s);
-cudaError_t launch_lowrank_finish(const float2* lists, int nlists, const uint32_t* tkth, int M,
-                                  int k,
-                                  int32_t* cand, const __nv_bfloat16* hid,
-                                  const __nv_bfloat16* W, int H, int V, int32_t* out_ids,
-                                  float* out_logit, cudaStream_t s);
+                                  WsHeader* ws, cudaStream_t s);
+cudaError_t launch_lowrank_finish(const float2* lists, int nlists, int M, int k, int32_t* cand,
+                                  const __nv_bfloat16* hid, const __nv_bfloat16* W, int H, int V,
+                                  int32_t* out_ids, float* out_logit, cudaStream_t s);
 
 struct CompactParams {
   const int32_t* cu_nodes;

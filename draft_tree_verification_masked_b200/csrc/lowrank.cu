@@ -6,11 +6,16 @@
 // head) to 326 us at rank 512 and 255 us at rank 128 ("EAGLE-4 是什麼？...", aiposthub.com,
 // section "EAGLE-4 是什麼？先看推測解碼為什麼能變快", Fig. 2).  For M hidden rows h:
 //
-//   g  = h D^T        D [r][H]: split-K over H on the CUDA cores (lr_down_kernel), the
-//                     partials summed in a fixed order and rounded to bf16 (lr_reduce_kernel);
+//   g  = h D^T        D [r][H]: lr_splitk_kernel, tcgen05 tiles of 64 x 64 with K split in
+//                     chunks of 128 over many CTAs; lr_reduce_kernel sums the chunk partials in
+//                     chunk order (the same order every call) and rounds g to bf16;
+//   floor             the same split-K kernel on every stride-th row of U (8192 samples per
+//                     row), and sample_floor_kernel: a lower bound of each row's 16th largest z~;
 //   z~ = g U^T        U [V][r]: the LM-head GEMM on tcgen05 with the EPI_TOPK epilogue, which
-//                     keeps each thread's 16 largest (value, id) per row -- z~ never reaches HBM;
-//   C  = top-k of z~  topk_merge_kernel: one CTA per row merges the sorted 16-lists;
+//                     keeps each thread's 16 largest (value, id) per row above the floor -- z~
+//                     never reaches HBM;
+//   C  = top-k of z~  topk_select_kernel: one CTA per row finds the k-th largest list entry by
+//                     a radix select over all the lists and keeps the entries ranked above it;
 //   z_c = h . W_c     lr_rescore_kernel: one warp per candidate, then the k are ordered by z_c.
 //
 // The screen streams |U| = V r 2 bytes (155 MB at r = 512, 39 MB at r = 128) instead of the full
@@ -19,72 +24,104 @@
 
 namespace etree {
 
-namespace {
-constexpr int kDT = 64;        // rows (m) and columns (j) per CTA tile
-constexpr int kDK = 128;       // H per CTA (the split-K chunk)
-constexpr int kDPad = 8;       // bf16 padding per smem row (breaks the 512-byte bank stride)
-}  // namespace
 
-// part[kc][m][j] = sum_{h in chunk kc} A[m][h] B[j * bstride][h], fp32 (A [M][K], B rows of K;
-// j < N).  The down projection has A = hidden, B = D; the screen's sample has A = g and B = every
-// bstride-th row of U.  CTA tile 64 m x 64 j x 128 h staged in padded shared memory (row
-// stride 272 bytes: the 8 rows an ldmatrix reads fall in distinct banks).
-__global__ void __launch_bounds__(256) lr_down_kernel(const __nv_bfloat16* __restrict__ hid,
-                                                      const __nv_bfloat16* __restrict__ D, int M,
-                                                      int H, int r, int bstride,
-                                                      float* __restrict__ part) {
-  __shared__ __align__(16) __nv_bfloat16 hs[kDT][kDK + kDPad];
-  __shared__ __align__(16) __nv_bfloat16 ds[kDT][kDK + kDPad];
-  const int j0 = blockIdx.x * kDT, kc = blockIdx.y, m0 = blockIdx.z * kDT;
-  const int h0 = kc * kDK;
-  const int tid = threadIdx.x;
-  // Every kernel here is launched with launch_pdl.  Only the floor kernel signals its dependent
-  // early: the screen GEMM after it has set-up and U tiles to load before it waits.  An early
-  // signal to a dependent with nothing to overlap measured slower than none.
-  pdl_wait();
-  // stage the two tiles, 16 bytes per thread per step (zeros past M, r or H)
-  for (int e = tid; e < kDT * (kDK / 8); e += 256) {
-    const int row = e / (kDK / 8), c8 = (e % (kDK / 8)) * 8;
-    uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
-    if (m0 + row < M && h0 + c8 < H)
-      a = *reinterpret_cast<const uint4*>(hid + (size_t)(m0 + row) * H + h0 + c8);
-    if (j0 + row < r && h0 + c8 < H)
-      b = __ldg(reinterpret_cast<const uint4*>(D + (size_t)(j0 + row) * bstride * H + h0 + c8));
-    *reinterpret_cast<uint4*>(&hs[row][c8]) = a;
-    *reinterpret_cast<uint4*>(&ds[row][c8]) = b;
+// part[kc][m][j] = sum over k in chunk kc of A[m][k] B[j][k], fp32, for m < M and j < N; chunk
+// kc covers k in [128 kc, 128 kc + 128) of K (a multiple of 64).  The down projection has A =
+// hidden, B = D; the screen's sample has A = g and B = every stride-th row of U (a tensor map
+// whose rows step over the others).  One CTA = 64 m x 64 j x 128 k, many CTAs in flight: thread 0
+// issues the chunk's (at most) two K steps of 128-byte-swizzled boxes {64 k, 64 rows} of A and B
+// on one barrier, thread 32 issues tcgen05.mma M=64 N=64 K=16 into 64 TMEM columns, and the four
+// warps store their accumulator rows (lanes 0..15 of each TMEM lane quarter) as fp32.
+constexpr int kSkTile = 64;     // m and j per CTA
+constexpr int kSkChunk = 128;   // k per CTA
+
+__global__ void __launch_bounds__(128) lr_splitk_kernel(const __grid_constant__ CUtensorMap tm_a,
+                                                        const __grid_constant__ CUtensorMap tm_b,
+                                                        int M, int K, int N,
+                                                        float* __restrict__ part, WsHeader* ws) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));   // [step][A 8 KB, B 8 KB]
+  __shared__ uint64_t full, done;
+  __shared__ uint32_t tmem_s;
+  const int j0 = blockIdx.x * kSkTile, kc = blockIdx.y, m0 = blockIdx.z * kSkTile;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int steps = min(kSkChunk / 64, K / 64 - kc * (kSkChunk / 64));
+  if (threadIdx.x == 0) {
+    mbar_init(&full, 1);
+    mbar_init(&done, 1);
+    fence_barrier_init();
   }
+  if (warp == 1) {
+    tmem_alloc(&tmem_s, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
-  // 8 warps: warp (wm, wn) computes rows wm*16 .. +15 and columns wn*32 .. +31 with
-  // mma.m16n8k16 (bf16 in, fp32 accumulate), fragments loaded by ldmatrix
-  const int warp = tid >> 5, lane = tid & 31;
-  const int wm = warp & 3, wn = warp >> 2;
-  float acc[4][4] = {};
-#pragma unroll
-  for (int kk = 0; kk < kDK / 16; ++kk) {
-    uint32_t a[4];
-    ldmatrix_x4(smem_u32(&hs[wm * 16 + (lane & 15)][kk * 16 + (lane >> 4) * 8]), a[0], a[1],
-                a[2], a[3]);
-#pragma unroll
-    for (int np = 0; np < 2; ++np) {
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4(smem_u32(&ds[wn * 32 + np * 16 + (lane & 7) + ((lane >> 4) << 3)]
-                              [kk * 16 + ((lane >> 3) & 1) * 8]),
-                  b0, b1, b2, b3);
-      mma_bf16_16816(acc[2 * np], a, b0, b1);
-      mma_bf16_16816(acc[2 * np + 1], a, b2, b3);
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  pdl_wait();                                           // A (hidden or g) of an earlier kernel
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+    mbar_arrive_expect_tx(&full, steps * 16384);
+    for (int s = 0; s < steps; ++s) {
+      const int k = (kc * (kSkChunk / 64) + s) * 64;
+      tma_load_2d(tiles + s * 16384, &tm_a, &full, k, m0);
+      tma_load_2d(tiles + s * 16384 + 8192, &tm_b, &full, k, j0);
     }
-  }
+  } else if (threadIdx.x == 32) {
+    ok = mbar_wait(&full, 0);
+    tc_fence_after();
+    if (ok) {
+      const uint32_t idesc = idesc_bf16_f32(kSkTile, kSkTile);
+      for (int s = 0; s < steps; ++s) {
+        const uint64_t da = smem_desc_sw128(tiles + s * 16384);
+        const uint64_t db = smem_desc_sw128(tiles + s * 16384 + 8192);
 #pragma unroll
-  for (int t = 0; t < 4; ++t) {
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const int m = m0 + wm * 16 + (lane >> 2) + 8 * hf;
-      const int j = j0 + wn * 32 + t * 8 + (lane & 3) * 2;
-      if (m < M) {
-        if (j < r) part[((size_t)kc * M + m) * r + j] = acc[t][2 * hf];
-        if (j + 1 < r) part[((size_t)kc * M + m) * r + j + 1] = acc[t][2 * hf + 1];
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (s > 0 || kk > 0) ? 1u : 0u);
       }
     }
+    tc_commit(&done);
+  }
+  __syncwarp();
+  const bool got = mbar_wait(&done, 0);
+  __syncwarp();
+  tc_fence_after();
+  float v0[32], v1[32];
+  tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), v0);
+  tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32, v1);
+  const int m = m0 + 16 * warp + lane;
+  if (ok && got && lane < 16 && m < M) {
+    float* dst = part + ((size_t)kc * M + m) * N + j0;
+    if (j0 + kSkTile <= N && (N & 3) == 0) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        reinterpret_cast<float4*>(dst)[q] = make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2],
+                                                        v0[4 * q + 3]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        reinterpret_cast<float4*>(dst + 32)[q] = make_float4(v1[4 * q], v1[4 * q + 1],
+                                                             v1[4 * q + 2], v1[4 * q + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j0 + j < N) dst[j] = v0[j];
+        if (j0 + 32 + j < N) dst[32 + j] = v1[j];
+      }
+    }
+  }
+  if (threadIdx.x == 0) {                               // the boxes have landed before exit
+    if (!mbar_wait(&full, 0)) ok = false;
+  }
+  if (!ok || !got) report(ws, ETREE_ETIMEOUT, DET_WAIT_GEMM);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
   }
 }
 
@@ -103,12 +140,6 @@ __global__ void lr_reduce_kernel(const float* __restrict__ part, int nk, int M, 
   float s = 0.f;
   for (int k = 0; k < nk; ++k) s += part[(size_t)k * M * r + t];
   g[t] = __float2bfloat16_rn(s);
-}
-
-// (va, ia) ranks before (vb, ib): larger value first, then the lower id; empty entries (id < 0)
-// rank last.
-__device__ __forceinline__ bool before(float va, int ia, float vb, int ib) {
-  return va > vb || (va == vb && ia >= 0 && (ib < 0 || ia < ib));
 }
 
 // A floor for the screen, kFloorParts CTAs per row.  Each sampled approximate logit is the sum
@@ -169,111 +200,179 @@ __global__ void __launch_bounds__(256) sample_floor_kernel(const float* __restri
   }
 }
 
-// One CTA per row.  The screen published a lower bound T of the row's 16th largest value, so
-// only list entries >= T can be selected: each thread scans its share of the 16 x nlists
-// entries (8 loads in flight) and each warp appends its survivors (150-500 per row measured on
-// the rank-128 and rank-512 workloads) to shared memory together.  A bitonic sort on the first
-// 256 threads orders them and the first k go to cand[m][0..k).  (Counting ranks, a bisection for
-// the k-th key over the CTA or one warp, and a register tournament in one warp all measured
-// within -1 .. +5 us of it.)  More than kGather survivors fall back to ranking them in passes
-// over the lists.
-constexpr int kGather = 2048;
-constexpr int kMergeThreads = 1024;
-constexpr int kSortThreads = 256;
-
-// Barrier 1 among the first kSortThreads threads of the CTA (barrier 0 is __syncthreads).
-__device__ __forceinline__ void sort_barrier() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kSortThreads) : "memory");
+// (va, ia) ranks before (vb, ib): larger value first, then the lower id.
+__device__ __forceinline__ bool before(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
 }
 
-__global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(const float2* __restrict__ lists,
-                                                                   int nlists, const uint32_t* tkth,
-                                                                   int k,
-                                                                   int32_t* __restrict__ cand) {
-  __shared__ float gv[kGather];
-  __shared__ int gi[kGather];
-  __shared__ int gn;
+// The top k of a row from its screen lists.  Each vocab id appears in at most one list, and
+// every list holds its thread's 16 largest values, so the row's k <= 16 largest values are
+// among the list entries: the k-th largest entry, with equal values ranked by the lower id,
+// splits them exactly.  One CTA per row finds it by a radix select on order-preserving 32-bit
+// codes of the values (-0 counted as +0, empty entries excluded): each pass histograms the next
+// 8 bits of the entries that match the digits fixed so far, and one warp finds the digit that
+// holds the k-th largest.  The select stops early when every entry of that digit is needed.
+// Entries above the final prefix are taken, then those on it (all of them, or the lowest ids
+// when the k-th value is shared), and one warp orders the k by (value desc, id asc).
+constexpr int kSelThreads = 1024;
+constexpr int kSelRegs = 8;              // entries per thread kept in registers (8192 per row)
+
+__device__ __forceinline__ uint32_t sel_code(float2 x) {
+  if (__float_as_int(x.y) < 0) return 0u;            // empty entry
+  return enc_order(x.x == 0.f ? 0.f : x.x);          // >= 0x007fffff for every non-NaN value
+}
+
+__global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float2* __restrict__ lists,
+                                                                  int nlists, int k,
+                                                                  int32_t* __restrict__ cand) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_digit, s_above, s_count, s_n;
+  __shared__ int s_min[kSelThreads / 32];
+  __shared__ float sv[16];
+  __shared__ int si[16];
   pdl_wait();
-  const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
-  const float T = dec_order(tkth[m]);
+  const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float2* rowl = lists + (size_t)m * nlists * 16;
   const int total = nlists * 16;
-  if (tid == 0) gn = 0;
-  __syncthreads();
-  // every lane of a warp runs the same iterations, so survivors are appended a warp at a time
-  for (int eb = tid - lane; eb < total; eb += kMergeThreads * 8) {
-    float2 x[8];
+  const int in_regs = kSelRegs * kSelThreads;
+  uint32_t code[kSelRegs];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = eb + lane + u * kMergeThreads;
-      x[u] = e < total ? rowl[e] : make_float2(-INFINITY, __int_as_float(-1));
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int xi = __float_as_int(x[u].y);
-      const bool sv = xi >= 0 && x[u].x >= T;
-      const unsigned b = __ballot_sync(0xffffffffu, sv);
-      if (b) {
-        int at = 0;
-        if (lane == 0) at = atomicAdd(&gn, __popc(b));
-        at = __shfl_sync(0xffffffffu, at, 0) + __popc(b & ((1u << lane) - 1u));
-        if (sv && at < kGather) {
-          gv[at] = x[u].x;
-          gi[at] = xi;
-        }
-      }
-    }
+  for (int u = 0; u < kSelRegs; ++u) {
+    const int e = tid + u * kSelThreads;
+    code[u] = e < total ? sel_code(__ldg(rowl + e)) : 0u;
   }
-  __syncthreads();
-  const int n = gn;
-  if (n <= kGather) {
-    // The sort runs on the first kSortThreads threads only, synchronised by a named barrier of
-    // that many threads (the rest of the CTA leaves); strides are powers of two, so the pair
-    // indices are bit operations.
-    if (tid >= kSortThreads) return;
-    int P = 16;
-    while (P < n) P <<= 1;
-    for (int e = n + tid; e < P; e += kSortThreads) {
-      gv[e] = -INFINITY;
-      gi[e] = -1;
+  uint32_t prefix = 0u, pmask = 0u;
+  uint32_t krem = (uint32_t)k;            // entries still to take among those on the prefix
+  bool whole = false;                     // every entry on the prefix is taken
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    if (tid < 256) hist[tid] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kSelRegs; ++u)
+      if (code[u] && (code[u] & pmask) == prefix) atomicAdd(&hist[(code[u] >> shift) & 255u], 1u);
+    for (int e = in_regs + tid; e < total; e += kSelThreads) {
+      const uint32_t cc = sel_code(__ldg(rowl + e));
+      if (cc && (cc & pmask) == prefix) atomicAdd(&hist[(cc >> shift) & 255u], 1u);
     }
-    sort_barrier();
-    for (int size = 2; size <= P; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < P / 2; i += kSortThreads) {
-          const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1)), hi = lo + stride;
-          const bool best_first = (lo & size) == 0;
-          const bool swap = best_first ? before(gv[hi], gi[hi], gv[lo], gi[lo])
-                                       : before(gv[lo], gi[lo], gv[hi], gi[hi]);
-          if (swap) {
-            const float tv = gv[lo];
-            const int ti = gi[lo];
-            gv[lo] = gv[hi];
-            gi[lo] = gi[hi];
-            gv[hi] = tv;
-            gi[hi] = ti;
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds digits 255 - 8l down to 248 - 8l; counts are scanned from the top digit
+      uint32_t cnt[8], sum = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cnt[i] = hist[255 - 8 * lane - i];
+        sum += cnt[i];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      const uint32_t excl = incl - sum;
+      if (excl < krem && krem <= incl) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (run + cnt[i] >= krem) {
+            s_digit = 255u - 8u * lane - i;
+            s_above = run;
+            s_count = cnt[i];
+            break;
           }
+          run += cnt[i];
         }
-        sort_barrier();
+      }
+      if (lane == 31 && incl < krem) {                  // fewer than k entries in the lists
+        s_digit = 256u;
+        s_above = incl;
+        s_count = 0u;
       }
     }
-    if (tid < k) cand[(size_t)m * 16 + tid] = gi[tid];
-    return;
-  }
-  // fallback: every entry >= T is ranked against every other by a pass over the lists
-  for (int e = tid; e < total; e += kMergeThreads) {
-    const float2 x = rowl[e];
-    const int xi = __float_as_int(x.y);
-    if (xi < 0 || x.x < T) continue;
-    int rank = 0;
-    for (int f = 0; f < total && rank < k; ++f) {
-      const float2 y = rowl[f];
-      rank += before(y.x, __float_as_int(y.y), x.x, xi);
+    __syncthreads();
+    const uint32_t d = s_digit;
+    if (d > 255u) {                                     // take every entry (first pass only)
+      whole = true;
+      break;
     }
-    if (rank < k) cand[(size_t)m * 16 + rank] = xi;
+    prefix |= d << shift;
+    pmask |= 255u << shift;
+    krem -= s_above;
+    if (s_count == krem) {
+      whole = true;
+      break;
+    }
+  }
+  if (tid == 0) s_n = 0u;
+  __syncthreads();
+  // entries above the prefix (fewer than k), and all entries on it when `whole`
+  auto take = [&](uint32_t cc, int e) {
+    const uint32_t cm = cc & pmask;
+    if (cc && (cm > prefix || (whole && cm == prefix))) {
+      const uint32_t at = atomicAdd(&s_n, 1u);
+      const float2 x = __ldg(rowl + e);
+      if (at < 16u) {
+        sv[at] = x.x;
+        si[at] = __float_as_int(x.y);
+      }
+    }
+  };
+#pragma unroll
+  for (int u = 0; u < kSelRegs; ++u) take(code[u], tid + u * kSelThreads);
+  for (int e = in_regs + tid; e < total; e += kSelThreads) take(sel_code(__ldg(rowl + e)), e);
+  __syncthreads();
+  if (!whole) {
+    // the k-th value is shared by more entries than are still needed: the krem lowest ids
+    // among the entries whose code is exactly the prefix, one block-wide minimum at a time
+    int last = -1;
+    for (uint32_t t = 0; t < krem; ++t) {
+      int best = 0x7fffffff;
+#pragma unroll
+      for (int u = 0; u < kSelRegs; ++u) {
+        if (code[u] == prefix) {
+          const int id = __float_as_int(__ldg(rowl + tid + u * kSelThreads).y);
+          if (id > last && id < best) best = id;
+        }
+      }
+      for (int e = in_regs + tid; e < total; e += kSelThreads) {
+        const float2 x = __ldg(rowl + e);
+        const int id = __float_as_int(x.y);
+        if (sel_code(x) == prefix && id > last && id < best) best = id;
+      }
+      best = __reduce_min_sync(0xffffffffu, best);
+      if (lane == 0) s_min[warp] = best;
+      __syncthreads();
+      if (warp == 0) {
+        int b = lane < kSelThreads / 32 ? s_min[lane] : 0x7fffffff;
+        b = __reduce_min_sync(0xffffffffu, b);
+        if (lane == 0) {
+          const uint32_t at = s_n++;
+          if (at < 16u) {
+            sv[at] = dec_order(prefix);
+            si[at] = b;
+          }
+          s_min[0] = b;
+        }
+      }
+      __syncthreads();
+      last = s_min[0];
+      __syncthreads();
+    }
+  }
+  if (warp == 0) {
+    const int n = min((int)s_n, k);
+    float v = -INFINITY;
+    int id = 0x7fffffff;
+    if (lane < n) {
+      v = sv[lane];
+      id = si[lane];
+    }
+    int rank = 0;
+    for (int j = 0; j < n; ++j) rank += before(sv[j], si[j], v, id);
+    if (lane < n) cand[(size_t)m * 16 + rank] = id;
+    else if (lane < k) cand[(size_t)m * 16 + lane] = -1;
   }
 }
-
 constexpr int kRescoreLoads = 20;        // 16-byte words of W per lane requested up front
 
 // One CTA per row, one warp per candidate: z_c = h . W_c in fp32 (the row staged in shared
@@ -366,41 +465,46 @@ __global__ void __launch_bounds__(512) lr_rescore_kernel(const __nv_bfloat16* __
   }
 }
 
-int lowrank_down_chunks(int H) { return (H + kDK - 1) / kDK; }
 
-cudaError_t launch_lowrank_down(const __nv_bfloat16* hid, const __nv_bfloat16* D, int M, int H,
+int lowrank_down_chunks(int H) { return (H + kSkChunk - 1) / kSkChunk; }
+
+static const int kSkSmem = 1024 + 2 * 16384;     // two K steps of A and B boxes, 1 KB aligned
+
+static cudaError_t launch_splitk(const CUtensorMap& ta, const CUtensorMap& tb, int M, int K, int N,
+                                 float* part, WsHeader* ws, cudaStream_t s) {
+  dim3 grid((N + kSkTile - 1) / kSkTile, (K + kSkChunk - 1) / kSkChunk, (M + kSkTile - 1) / kSkTile);
+  return launch_pdl(lr_splitk_kernel, grid, dim3(128), (size_t)kSkSmem, s, ta, tb, M, K, N, part,
+                    ws);
+}
+
+cudaError_t launch_lowrank_down(const CUtensorMap& tm_h, const CUtensorMap& tm_d, int M, int H,
                                 int r, float* part, __nv_bfloat16* g, uint32_t* tkth,
-                                int32_t* fcnt, cudaStream_t s) {
-  const int nk = lowrank_down_chunks(H);
-  dim3 grid((r + kDT - 1) / kDT, nk, (M + kDT - 1) / kDT);
-  cudaError_t e = launch_pdl(lr_down_kernel, grid, dim3(256), 0, s, hid, D, M, H, r, 1, part);
+                                int32_t* fcnt, WsHeader* ws, cudaStream_t s) {
+  cudaError_t e = launch_splitk(tm_h, tm_d, M, H, r, part, ws, s);
   if (e != cudaSuccess) return e;
-  return launch_pdl(lr_reduce_kernel, dim3((M * r + 255) / 256), dim3(256), 0, s, part, nk, M, r,
-                    g, tkth, fcnt);
+  return launch_pdl(lr_reduce_kernel, dim3((M * r + 255) / 256), dim3(256), 0, s, part,
+                    lowrank_down_chunks(H), M, r, g, tkth, fcnt);
 }
 
 int lowrank_sample_cols(int V) { return V < 8192 ? V : 8192; }
 
 int lowrank_floor_maxima(int M) { return M * kFloorParts * 256; }
 
-cudaError_t launch_lowrank_sample(const __nv_bfloat16* g, const __nv_bfloat16* U, int M, int r,
+cudaError_t launch_lowrank_sample(const CUtensorMap& tm_g, const CUtensorMap& tm_us, int M, int r,
                                   int V, float* part, float* fmax, int32_t* fcnt, uint32_t* tkth,
-                                  cudaStream_t s) {
-  const int S = lowrank_sample_cols(V), stride = V / S;
-  const int nk = (r + kDK - 1) / kDK;
-  dim3 grid((S + kDT - 1) / kDT, nk, (M + kDT - 1) / kDT);
-  cudaError_t e = launch_pdl(lr_down_kernel, grid, dim3(256), 0, s, g, U, M, r, S, stride, part);
+                                  WsHeader* ws, cudaStream_t s) {
+  const int S = lowrank_sample_cols(V);
+  cudaError_t e = launch_splitk(tm_g, tm_us, M, r, S, part, ws, s);
   if (e != cudaSuccess) return e;
-  return launch_pdl(sample_floor_kernel, dim3(M * kFloorParts), dim3(256), 0, s, part, nk, M, S,
-                    fmax, fcnt, tkth);
+  return launch_pdl(sample_floor_kernel, dim3(M * kFloorParts), dim3(256), 0, s, part,
+                    lowrank_down_chunks(r), M, S, fmax, fcnt, tkth);
 }
 
-cudaError_t launch_lowrank_finish(const float2* lists, int nlists, const uint32_t* tkth, int M,
-                                  int k, int32_t* cand, const __nv_bfloat16* hid,
-                                  const __nv_bfloat16* W, int H, int V, int32_t* out_ids,
-                                  float* out_logit, cudaStream_t s) {
-  cudaError_t e = launch_pdl(topk_merge_kernel, dim3(M), dim3(kMergeThreads), 0, s, lists,
-                             nlists, tkth, k, cand);
+cudaError_t launch_lowrank_finish(const float2* lists, int nlists, int M, int k, int32_t* cand,
+                                  const __nv_bfloat16* hid, const __nv_bfloat16* W, int H, int V,
+                                  int32_t* out_ids, float* out_logit, cudaStream_t s) {
+  cudaError_t e = launch_pdl(topk_select_kernel, dim3(M), dim3(kSelThreads), 0, s, lists, nlists,
+                             k, cand);
   if (e != cudaSuccess) return e;
   return launch_pdl(lr_rescore_kernel, dim3(M), dim3(32 * k), 0, s, hid, W, H, V, k, cand,
                     out_ids, out_logit);

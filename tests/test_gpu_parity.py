@@ -12,6 +12,8 @@ request: the chance of even one is about 1e-5 per decision (an argmax flips only
 within the fp32 error of the logits, a few 1e-6; a sampling decision only when the fp64
 quantities it compares agree to 1e-5), far below one per test.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -367,6 +369,35 @@ def _lowrank_run(lw):
 def test_lowrank_candidates_small(over):
     lw = W.lowrank("lowrank_tiny", **over)
     ids, lg = _lowrank_run(lw)
+    P.lowrank_compare(lw, ids, lg)
+
+
+def test_lowrank_select_beyond_the_register_entries():
+    """Two row tiles make the screen keep lists per vocab tile: at V = 60,000 a row has more than
+    8,192 list entries, so the select reads the rest of them again in every pass."""
+    lw = W.lowrank("lowrank_tiny", M=130, V=60000, k=16)
+    ids, lg = _lowrank_run(lw)
+    P.lowrank_compare(lw, ids, lg)
+
+
+def test_lowrank_select_takes_the_lowest_ids_of_a_shared_value():
+    """Forty vocab ids spread over the vocabulary (so over different CTAs' lists) share one U
+    row, scaled by 8 so that it dominates the rows where it scores positive: there more than k
+    ids tie for the largest screen values, bit for bit, and the select must take the lowest of
+    them.  Checked directly on the GPU's sets and against the oracle."""
+    lw = W.lowrank("lowrank_tiny", M=32, V=20000, k=16)
+    U = lw.U.clone()
+    group = [37 + 487 * i for i in range(40)]
+    U[group] = (U[5].float() * 8).to(torch.bfloat16)
+    lw = dataclasses.replace(lw, U=U)
+    ids, lg = _lowrank_run(lw)
+    gset = set(group)
+    full = 0
+    for m in range(lw.M):
+        sel = sorted(c for c in ids[m].tolist() if c in gset)
+        assert sel == group[:len(sel)], (m, sel)
+        full += len(sel) == lw.k
+    assert full >= 1                                   # some rows cut through the tie
     P.lowrank_compare(lw, ids, lg)
 
 
