@@ -737,7 +737,7 @@ def ncu_case(args):
         lo, hi = (int(x) for x in args.ncu_kv.split(":"))
         over["kv_len"] = (lo, hi)
     wl = W.generate(base, **over)
-    dev = DeviceStep(wl, page_size=int(pg) if pg else None)
+    dev = DeviceStep(wl, page_size=int(pg) if pg else None, materialize=True)   # as timed
     dev.step()
     st = dev.status()
     if st[0] != 0:
