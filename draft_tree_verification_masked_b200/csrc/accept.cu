@@ -360,6 +360,10 @@ __global__ void __launch_bounds__(1024) tree_prep_kernel(AcceptParams p, int32_t
                                                          int32_t* zrow, int zbuf_rows) {
   __shared__ int32_t part_s[1024];
   const int tid = threadIdx.x, nt = blockDim.x;
+  if (zbuf_rows >= p.n_total) {                       // every row materialised: row g is node g
+    for (int g = tid; g < p.n_total; g += nt) zrow[g] = g;
+    return;
+  }
   for (int g = tid; g < p.n_total; g += nt) ccount[g] = 0;
   __syncthreads();
   for (int g = tid; g < p.n_total; g += nt) {
@@ -384,10 +388,6 @@ __global__ void __launch_bounds__(1024) tree_prep_kernel(AcceptParams p, int32_t
   }
   int next = part_s[tid] - cnt;
   bool over = false;
-  if (zbuf_rows >= p.n_total) {                       // every row materialised
-    for (int g = g0; g < g1; ++g) zrow[g] = g;
-    return;
-  }
   for (int g = g0; g < g1; ++g) {
     int zr = -1;
     if (ccount[g] >= 2) {
@@ -520,7 +520,8 @@ __device__ double residual_mass(const AcceptParams& p, const float* zr, const fl
 // evaluates N(c) when a rejected child has a younger sibling still to test.  Writes accept_len,
 // path, the accepted tokens, the stop row / node, the draw offset cval (negative: the residual
 // has no positive weight and the bonus is drawn from p) and the stop row's hidden state for the
-// draw pass.
+// draw pass.  A child's logit under its parent's row comes from child_logit_kernel (zc), or, with
+// zc null (every row materialised), from the parent's stored row.
 constexpr int kWalkThreads = 1024;
 
 __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p, const float* zc,
@@ -528,14 +529,17 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
                                                                  const float* zbuf) {
   __shared__ int par_s[64], tok_s[64];
   __shared__ double red_s[kWalkThreads / 32];
-  __shared__ int act_s, u_s, ok_s, fell_s;
+  __shared__ int act_s, u_s, ok_s, fell_s, bad_s;
   __shared__ double c_s;
   const int r = blockIdx.x, tid = threadIdx.x;
   int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
   int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
   int base, n;
   const bool n_ok = request_ok(p, r, base, n);
-  if (tid == 0) ok_s = n_ok ? 1 : 0;
+  if (tid == 0) {
+    ok_s = n_ok ? 1 : 0;
+    bad_s = 0;                                          // malformed input (not a full buffer)
+  }
   if (n_ok && tid < n) {
     par_s[tid] = p.parent[base + tid];
     tok_s[tid] = p.tokens[base + tid];
@@ -548,20 +552,30 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
     int kids = 0;
     for (int j = tid + 1; j < n; ++j) kids += par_s[j] == tid;
     if (kids >= 2 && zrow[base + tid] < 0) fits = false;
-    if (!good) { report(p.ws, ETREE_EDEVICE, DET_BAD_PARENT); atomicAnd(&ok_s, 0); }
-    if (tid >= 1 && (tok_s[tid] < 0 || tok_s[tid] >= p.V)) atomicAnd(&ok_s, 0);  // reported by
-                                                                               // child_logit
+    if (!good) {
+      report(p.ws, ETREE_EDEVICE, DET_BAD_PARENT);
+      atomicAnd(&ok_s, 0);
+      atomicOr(&bad_s, 1);
+    }
+    if (tid >= 1 && (tok_s[tid] < 0 || tok_s[tid] >= p.V)) {
+      if (!zc) report(p.ws, ETREE_EDEVICE, DET_BAD_TOKEN);   // else child_logit reported it
+      atomicAnd(&ok_s, 0);
+      atomicOr(&bad_s, 1);
+    }
     if (!fits) atomicAnd(&ok_s, 0);                      // reported by tree_prep_kernel
   }
   __syncthreads();
-  if (!ok_s) {                                          // accept nothing, draw from the root's p
+  if (!ok_s) {
+    // accept nothing.  A request without a logit row for a branching node (a full buffer) draws
+    // its bonus from the root's p; a malformed one gets no bonus (stop node -1, which the draws
+    // skip), so a caller that emits tokens before reading the status emits none.
     if (!n_ok && tid == 0) report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
     for (int k = tid; k < 64; k += blockDim.x) path[k] = (n_ok && k == 0) ? 0 : -1;
     for (int k = tid; k < 65; k += blockDim.x) outt[k] = -1;
     if (tid == 0) {
       p.accept_len[r] = 0;
       p.stop_row[r] = n_ok ? base : 0;
-      p.stop_node[r] = 0;
+      p.stop_node[r] = (n_ok && !bad_s) ? 0 : -1;
       p.cval[r] = 0.f;
       p.rfloor[2 * r] = 0u;
       p.rfloor[2 * r + 1] = 0u;
@@ -584,7 +598,10 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
           const int x = tok_s[j];
           const float L2 = p.lse2[base + u];
           const double qx = (double)__ldg(p.q_draft + (size_t)(base + u) * p.V + x);
-          const double pz = (double)exp2f(zc[base + j] * p.k_log2 - L2);
+          // the parent row's logit of x: from the materialised row itself when every row is
+          // kept (the same fp32 accumulator the row's log-sum-exp came from), else child_logit's
+          const float zx = zc ? zc[base + j] : zbuf[(size_t)zrow[base + u] * p.V + x];
+          const double pz = (double)exp2f(zx * p.k_log2 - L2);
           const double rx = pz - c * qx > 0.0 ? (pz - c * qx) / N : 0.0;
           float U[8];
           uniforms8(p.seed, p.step, 0u, (uint32_t)j, (uint32_t)r, 1u, U);
@@ -679,7 +696,7 @@ __global__ void __launch_bounds__(256) bonus_kernel(AcceptParams p) {
   if (lane == 0) {
     const int base = p.cu_nodes[r];
     const int n = p.cu_nodes[r + 1] - base;
-    if (n < 1 || n > p.n_max) return;
+    if (n < 1 || n > p.n_max || p.stop_node[r] < 0) return;   // malformed: no bonus
     const int a = p.accept_len[r];
     p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = ir >= 0 ? ir : ip;
   }
@@ -706,7 +723,7 @@ __global__ void __launch_bounds__(kDrawThreads) draw_rows_kernel(AcceptParams p,
   const int r = blockIdx.x / parts, part = blockIdx.x % parts;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int base, n;
-  if (!request_ok(p, r, base, n)) return;            // answered by the walk
+  if (!request_ok(p, r, base, n) || p.stop_node[r] < 0) return;   // answered by the walk
   if (tid == 0) fl_s[0] = fl_s[1] = 0u;
   __syncthreads();
   const int srow = p.stop_row[r];
@@ -824,6 +841,7 @@ cudaError_t launch_accept_chain(const AcceptParams& p, int32_t* cnt, cudaStream_
 cudaError_t launch_tree_prep(const AcceptParams& p, const __nv_bfloat16* w_lm, int32_t* ccount,
                              int32_t* zrow, int zbuf_rows, float* zc, cudaStream_t s) {
   tree_prep_kernel<<<1, 1024, 0, s>>>(p, ccount, zrow, zbuf_rows);
+  if (zbuf_rows >= p.n_total) return cudaGetLastError();   // the walk reads the kept rows
   child_logit_kernel<<<(p.n_total + 7) / 8, 256, 0, s>>>(p, w_lm, zc);
   return cudaGetLastError();
 }

@@ -233,6 +233,9 @@ etree_status etree_lmhead_accept(const etree_batch *batch, const uint16_t *hidde
  *              than zbuf_rows records ETREE_ENOSPACE (detail 10) and the requests left without a
  *              row accept nothing: their bonus is drawn from the root's p (a one-token
  *              decode).  zbuf may be NULL when zbuf_rows == 0 (chains need no rows).
+ *              A malformed request (a parent not below its child: ETREE_EDEVICE detail 1; a
+ *              token outside [0, vocab): detail 9) accepts nothing and gets no bonus token:
+ *              path[r][0] = 0, out_tokens[r] all -1.
  *              With zbuf_rows >= n_total, every node's logits are stored (row g for node g) and
  *              the bonus draw reads the stop row there instead of making a second pass over
  *              w_lm for the B stop rows: the tokens are the same, the second W pass (a GEMM of B

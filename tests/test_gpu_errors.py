@@ -62,6 +62,28 @@ def test_malformed_node_counts_answer_every_request(T):
     _still_works()
 
 
+@pytest.mark.parametrize("materialize", [False, True])
+def test_bad_token_on_a_tree_reports_and_answers_the_request(materialize):
+    """A draft token outside [0, vocab) at T > 0 on a branching tree reports ETREE_EDEVICE
+    (detail 9) whether the child logits are dot products or read from the materialised rows; that
+    request accepts nothing and gets no bonus token (as for a malformed parent), and the other
+    one runs."""
+    wl = W.generate("tiny", B=2, n_nodes=[7, 9], depth=3, branch=3, kv_len=[100, 300],
+                    hidden=256, vocab=512)
+    wl.temperature = 1.0
+    wl.q_draft = torch.full((wl.n_total, wl.vocab), 1.0 / wl.vocab)
+    dev = DeviceStep(wl, tree=True, materialize=materialize)
+    dev.accept_len.fill_(7)
+    dev.tokens[int(wl.cu_nodes[1]) + 2] = wl.vocab + 3
+    dev.lmhead()
+    assert dev.status() == (EDEVICE, 9)
+    res = dev.results()
+    assert res["accept_len"][1] == 0
+    assert (res["out_tokens"][1] == -1).all()
+    assert res["out_tokens"][0][int(res["accept_len"][0])] >= 0
+    _still_works()
+
+
 def test_bad_page_entry_reports_and_leaves_compaction_untouched():
     wl = W.generate("tiny", B=2, kv_len=[100, 300], hidden=256, vocab=512)
     dev = DeviceStep(wl, page_size=32)
