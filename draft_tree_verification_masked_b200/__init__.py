@@ -43,7 +43,7 @@ STATUS = {0: "ETREE_OK", -1: "ETREE_EINVAL", -2: "ETREE_EUNSUPPORTED", -3: "ETRE
           -4: "ETREE_EDEVICE", -5: "ETREE_ETIMEOUT", -6: "ETREE_ENOSPACE"}
 DETAIL = {0: "none", 1: "bad parent", 2: "bad node count", 3: "bad kv_len", 4: "capacity",
           5: "not a chain", 6: "bad path", 7: "attention wait", 8: "gemm wait", 9: "bad token",
-          10: "logit rows", 11: "bad page", 12: "self-test wait"}
+          10: "logit rows", 11: "bad page", 12: "self-test wait", 13: "walk wait"}
 
 EXPORTS = ["etree_workspace_size", "etree_workspace_init", "etree_verify_attn",
            "etree_verify_attn_paged", "etree_kv_compact_paged", "etree_verify_cost",

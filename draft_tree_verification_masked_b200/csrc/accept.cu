@@ -464,18 +464,21 @@ __global__ void __launch_bounds__(256) row_lse_kernel(AcceptParams p) {
   if (lane == 0) p.lse2[row] = m + log2f(s);
 }
 
-// N(c) = sum_v max(0, p_u(v) - c q_u(v)) over one materialised logit row, by the whole CTA:
-// p_u(v) = 2^(z_v log2(e) / T - lse2_u) and the difference in fp32, summed in fp32 over 16
+// The part of N(c) = sum_v max(0, p_u(v) - c q_u(v)) over one materialised logit row that falls
+// in slice `part` of `parts` (whole float4 groups when vocab is a multiple of 4), by the whole
+// CTA: p_u(v) = 2^(z_v log2(e) / T - lse2_u) and the difference in fp32, summed in fp32 over 16
 // terms, then in fp64 (each thread's partials, then the CTA's).
 __device__ double residual_mass(const AcceptParams& p, const float* zr, const float* qr, float L2,
-                                double c, double* red) {
+                                double c, double* red, int part, int parts) {
   const int tid = threadIdx.x, nt = blockDim.x;
   const float cf = (float)c, kl = p.k_log2;
   double acc = 0.0;
   if ((p.V & 3) == 0) {
-    const float4* z4 = reinterpret_cast<const float4*>(zr);
-    const float4* q4 = reinterpret_cast<const float4*>(qr);
-    const int n4 = p.V / 4;
+    const int all4 = p.V / 4, per = (all4 + parts - 1) / parts;
+    const int o4 = min(all4, part * per);
+    const float4* z4 = reinterpret_cast<const float4*>(zr) + o4;
+    const float4* q4 = reinterpret_cast<const float4*>(qr) + o4;
+    const int n4 = min(all4, o4 + per) - o4;
     int i = tid;
     for (; i + 3 * nt < n4; i += 4 * nt) {            // four float4 pairs in flight per thread
       float4 z[4], q[4];
@@ -503,7 +506,9 @@ __device__ double residual_mass(const AcceptParams& p, const float* zr, const fl
       acc += (double)part;
     }
   } else {
-    for (int v = tid; v < p.V; v += nt)
+    const int per = (p.V + parts - 1) / parts;
+    const int v1 = min(p.V, (part + 1) * per);
+    for (int v = part * per + tid; v < v1; v += nt)
       acc += (double)fmaxf(exp2f(zr[v] * kl - L2) - cf * __ldg(qr + v), 0.f);
   }
 #pragma unroll
@@ -516,22 +521,49 @@ __device__ double residual_mass(const AcceptParams& p, const float* zr, const fl
   return tot;
 }
 
-// One CTA per request: the multi-candidate walk.  Thread 0 takes the decisions; the whole CTA
-// evaluates N(c) when a rejected child has a younger sibling still to test.  Writes accept_len,
-// path, the accepted tokens, the stop row / node, the draw offset cval (negative: the residual
-// has no positive weight and the bonus is drawn from p) and the stop row's hidden state for the
-// draw pass.  A child's logit under its parent's row comes from child_logit_kernel (zc), or, with
-// zc null (every row materialised), from the parent's stored row.
-constexpr int kWalkThreads = 1024;
+// The multi-candidate walk, CS CTAs (a thread-block cluster) per request.  Thread 0 of every CTA
+// takes the same decisions from the same data, so the CTAs move in step; each CTA evaluates its
+// slice of N(c) when a rejected child has a younger sibling still to test.  It publishes the slice
+// in its shared memory (a release store of the pass number), and every CTA adds the CS slices in
+// rank order, so N(c) is the same in all of them.  Reading the other CTAs' slices polls a bounded
+// number of times.  Rank 0 writes accept_len, path, the accepted tokens, the stop row / node, the
+// draw offset cval (negative: the residual has no positive weight and the bonus is drawn from p)
+// and the stop row's hidden state for the draw pass.  A child's logit under its parent's row comes
+// from child_logit_kernel (zc), or, with zc null (every row materialised), from the parent's
+// stored row.
+__device__ __forceinline__ uint32_t walk_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
 
-__global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p, const float* zc,
-                                                                 const int32_t* zrow,
-                                                                 const float* zbuf) {
+__device__ __forceinline__ void walk_cluster_sync() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t walk_mapa(const void* p, uint32_t rank) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(p)), "r"(rank));
+  return ra;
+}
+
+constexpr uint32_t kWalkPollCap = 1u << 22;     // polls of a peer's pass number (a few seconds)
+
+template <int CS, int NT>
+__global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NT)
+    tree_walk_kernel(AcceptParams p, const float* zc, const int32_t* zrow, const float* zbuf) {
   __shared__ int par_s[64], tok_s[64];
-  __shared__ double red_s[kWalkThreads / 32];
+  __shared__ double red_s[NT / 32];
   __shared__ int act_s, u_s, ok_s, fell_s, bad_s;
   __shared__ double c_s;
-  const int r = blockIdx.x, tid = threadIdx.x;
+  __shared__ double slice_s[2], got_s[CS];     // this CTA's N(c) slice by pass parity; gathered
+  __shared__ uint32_t pass_s;                  // passes published so far
+  __shared__ int late_s;
+  const int r = blockIdx.x / CS, tid = threadIdx.x;
+  const int rank = CS > 1 ? (int)walk_cluster_rank() : 0;
+  const bool lead = rank == 0;
   int32_t* path = p.path + (size_t)r * ETREE_PATH_STRIDE;
   int32_t* outt = p.out_tokens + (size_t)r * ETREE_OUT_STRIDE;
   int base, n;
@@ -539,12 +571,15 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
   if (tid == 0) {
     ok_s = n_ok ? 1 : 0;
     bad_s = 0;                                          // malformed input (not a full buffer)
+    pass_s = 0u;
+    late_s = 0;
   }
   if (n_ok && tid < n) {
     par_s[tid] = p.parent[base + tid];
     tok_s[tid] = p.tokens[base + tid];
   }
   __syncthreads();
+  if constexpr (CS > 1) walk_cluster_sync();           // every pass counter starts at 0
   if (n_ok && tid < n) {
     const int pj = par_s[tid];
     const bool good = tid == 0 ? pj == -1 : (pj >= 0 && pj < tid);
@@ -553,12 +588,12 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
     for (int j = tid + 1; j < n; ++j) kids += par_s[j] == tid;
     if (kids >= 2 && zrow[base + tid] < 0) fits = false;
     if (!good) {
-      report(p.ws, ETREE_EDEVICE, DET_BAD_PARENT);
+      if (lead) report(p.ws, ETREE_EDEVICE, DET_BAD_PARENT);
       atomicAnd(&ok_s, 0);
       atomicOr(&bad_s, 1);
     }
     if (tid >= 1 && (tok_s[tid] < 0 || tok_s[tid] >= p.V)) {
-      if (!zc) report(p.ws, ETREE_EDEVICE, DET_BAD_TOKEN);   // else child_logit reported it
+      if (!zc && lead) report(p.ws, ETREE_EDEVICE, DET_BAD_TOKEN);   // else child_logit did
       atomicAnd(&ok_s, 0);
       atomicOr(&bad_s, 1);
     }
@@ -569,24 +604,27 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
     // accept nothing.  A request without a logit row for a branching node (a full buffer) draws
     // its bonus from the root's p; a malformed one gets no bonus (stop node -1, which the draws
     // skip), so a caller that emits tokens before reading the status emits none.
-    if (!n_ok && tid == 0) report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
-    for (int k = tid; k < 64; k += blockDim.x) path[k] = (n_ok && k == 0) ? 0 : -1;
-    for (int k = tid; k < 65; k += blockDim.x) outt[k] = -1;
-    if (tid == 0) {
-      p.accept_len[r] = 0;
-      p.stop_row[r] = n_ok ? base : 0;
-      p.stop_node[r] = (n_ok && !bad_s) ? 0 : -1;
-      p.cval[r] = 0.f;
-      p.rfloor[2 * r] = 0u;
-      p.rfloor[2 * r + 1] = 0u;
-      u_s = n_ok ? base : 0;
+    if (lead) {
+      if (!n_ok && tid == 0) report(p.ws, ETREE_EDEVICE, DET_BAD_NODES);
+      for (int k = tid; k < 64; k += NT) path[k] = (n_ok && k == 0) ? 0 : -1;
+      for (int k = tid; k < 65; k += NT) outt[k] = -1;
+      if (tid == 0) {
+        p.accept_len[r] = 0;
+        p.stop_row[r] = n_ok ? base : 0;
+        p.stop_node[r] = (n_ok && !bad_s) ? 0 : -1;
+        p.cval[r] = 0.f;
+        p.rfloor[2 * r] = 0u;
+        p.rfloor[2 * r + 1] = 0u;
+      }
     }
+    if (tid == 0) u_s = n_ok ? base : 0;
   } else {
     // thread 0's walk state: node u, last child tested, c and N(c) of the current residual
     int u = 0, j = 0, a = 0;
     double c = 0.0, N = 1.0;
+    uint32_t npass = 0u;                                // residual passes so far (every thread)
     if (tid == 0) {
-      path[0] = 0;
+      if (lead) path[0] = 0;
       fell_s = 0;
     }
     for (int it = 0; it < 2 * 64 + 2; ++it) {          // each node is tested once: bounded
@@ -607,8 +645,10 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
           uniforms8(p.seed, p.step, 0u, (uint32_t)j, (uint32_t)r, 1u, U);
           if ((double)U[0] * qx < rx) {                 // accepted: the walk moves to child j
             ++a;
-            path[a] = j;
-            outt[a - 1] = x;
+            if (lead) {
+              path[a] = j;
+              outt[a - 1] = x;
+            }
             u = j;
             c = 0.0;
             N = 1.0;
@@ -629,8 +669,44 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
       if (act == 2) break;
       if (act == 1) {
         const int ur = base + u_s;
-        const double Nn = residual_mass(p, zbuf + (size_t)zrow[ur] * p.V,
-                                        p.q_draft + (size_t)ur * p.V, p.lse2[ur], c_s, red_s);
+        const double mine = residual_mass(p, zbuf + (size_t)zrow[ur] * p.V,
+                                          p.q_draft + (size_t)ur * p.V, p.lse2[ur], c_s, red_s,
+                                          rank, CS);
+        double Nn = mine;
+        if constexpr (CS > 1) {
+          const uint32_t k = npass++;                   // this pass, the same in every CTA
+          if (tid == 0) {
+            slice_s[k & 1] = mine;
+            asm volatile("st.release.cluster.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(&pass_s)),
+                         "r"(k + 1u)
+                         : "memory");
+          }
+          if (tid < CS) {                               // thread q reads CTA q's slice
+            const uint32_t ra = walk_mapa(&pass_s, (uint32_t)tid);
+            uint32_t seen = 0u, tries = 0u;
+            do {
+              asm volatile("ld.acquire.cluster.shared::cluster.u32 %0, [%1];"
+                           : "=r"(seen)
+                           : "r"(ra)
+                           : "memory");
+              if (seen > k) break;
+              __nanosleep(32);
+            } while (++tries < kWalkPollCap);
+            double v = __longlong_as_double(0x7ff8000000000000ll);   // NaN: gave up
+            if (seen > k) {
+              asm volatile("ld.shared::cluster.f64 %0, [%1];"
+                           : "=d"(v)
+                           : "r"(walk_mapa(&slice_s[k & 1], (uint32_t)tid))
+                           : "memory");
+            } else {
+              atomicOr(&late_s, 1);
+            }
+            got_s[tid] = v;
+          }
+          __syncthreads();
+          Nn = 0.0;
+          for (int q = 0; q < CS; ++q) Nn += got_s[q];  // rank order: the same sum everywhere
+        }
         if (tid == 0) {
           N = Nn;
           if (!(N > 0.0)) fell_s = 1;                   // no positive residual: draw from p
@@ -639,7 +715,8 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
         if (fell_s) break;
       }
     }
-    if (tid == 0) {
+    if (tid == 0 && late_s) report(p.ws, ETREE_ETIMEOUT, DET_WAIT_WALK);
+    if (tid == 0 && lead) {
       for (int k = a + 1; k < 64; ++k) path[k] = -1;
       for (int k = a; k < 65; ++k) outt[k] = -1;
       p.accept_len[r] = a;
@@ -648,13 +725,16 @@ __global__ void __launch_bounds__(kWalkThreads) tree_walk_kernel(AcceptParams p,
       p.cval[r] = fell_s ? -1.f : (float)c;
       p.rfloor[2 * r] = 0u;
       p.rfloor[2 * r + 1] = 0u;
-      u_s = base + u;
     }
+    if (tid == 0) u_s = base + u;
   }
   __syncthreads();
-  const uint4* hs = reinterpret_cast<const uint4*>(p.hidden + (size_t)u_s * p.H);
-  uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
-  for (int i = tid; i < p.H / 8; i += blockDim.x) hd[i] = hs[i];
+  if (lead) {
+    const uint4* hs = reinterpret_cast<const uint4*>(p.hidden + (size_t)u_s * p.H);
+    uint4* hd = reinterpret_cast<uint4*>(p.hid2 + (size_t)r * p.H);
+    for (int i = tid; i < p.H / 8; i += NT) hd[i] = hs[i];
+  }
+  if constexpr (CS > 1) walk_cluster_sync();           // no CTA leaves while its slice is read
 }
 
 // The bonus draw's last step, one warp per request: the largest race key over the draw pass's
@@ -847,9 +927,14 @@ cudaError_t launch_tree_prep(const AcceptParams& p, const __nv_bfloat16* w_lm, i
 }
 
 cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32_t* zrow,
-                             const float* zbuf, cudaStream_t s) {
+                             const float* zbuf, int sms, cudaStream_t s) {
   row_lse_kernel<<<(p.n_total + 7) / 8, 256, 0, s>>>(p);
-  tree_walk_kernel<<<p.B, kWalkThreads, 0, s>>>(p, zc, zrow, zbuf);
+  // small batches: a cluster of 8 CTAs per request splits each residual pass; large batches
+  // already fill the SMs with one CTA per request
+  if (p.B * 8 <= 4 * sms)
+    tree_walk_kernel<8, 256><<<p.B * 8, 256, 0, s>>>(p, zc, zrow, zbuf);
+  else
+    tree_walk_kernel<1, 1024><<<p.B, 1024, 0, s>>>(p, zc, zrow, zbuf);
   return cudaGetLastError();
 }
 

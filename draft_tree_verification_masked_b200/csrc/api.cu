@@ -803,7 +803,7 @@ static etree_status lmhead_accept_impl(const etree_batch* b, const uint16_t* hid
     g.zrow = nullptr;
     g.zbuf = nullptr;
     if (e == cudaSuccess)
-      e = launch_tree_walk(a, tree->rows >= b->n_total ? nullptr : zc, zrow, tree->zbuf, s);
+      e = launch_tree_walk(a, tree->rows >= b->n_total ? nullptr : zc, zrow, tree->zbuf, sms, s);
     if (e == cudaSuccess && tree->rows >= b->n_total) {
       // every row's logits are in zbuf: the draw reads the stop rows there (no second W pass)
       mark(2);

@@ -36,6 +36,7 @@ enum Detail : int32_t {
   DET_ZBUF = 10,            // more branching tree nodes than rows in the caller's logit buffer
   DET_BAD_PAGE = 11,        // a block-table entry outside [0, num_pages) for a used position
   DET_SELFTEST = 12,        // etree_selftest_timeout: the deliberately unfinished wait gave up
+  DET_WAIT_WALK = 13,       // the tree walk gave up waiting for another CTA's residual slice
 };
 
 __device__ __forceinline__ void report(WsHeader* ws, int32_t code, int32_t detail) {

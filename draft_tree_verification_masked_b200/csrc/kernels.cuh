@@ -120,7 +120,7 @@ cudaError_t launch_draw_rows(const AcceptParams& p, const int32_t* zrow, const f
 cudaError_t launch_tree_prep(const AcceptParams& p, const __nv_bfloat16* w_lm, int32_t* ccount,
                              int32_t* zrow, int zbuf_rows, float* zc, cudaStream_t s);
 cudaError_t launch_tree_walk(const AcceptParams& p, const float* zc, const int32_t* zrow,
-                             const float* zbuf, cudaStream_t s);
+                             const float* zbuf, int sms, cudaStream_t s);
 
 int lowrank_down_chunks(int H);
 int lowrank_sample_cols(int V);

@@ -401,6 +401,7 @@ etree_status etree_plan_tree(const etree_cost_table *table, int32_t B, int32_t L
  *   10  logit rows: more branching nodes than zbuf rows (etree_lmhead_accept_tree)
  *   11  bad page: a block-table entry outside [0, num_pages) for a used position
  *   12  self-test wait: etree_selftest_timeout's deliberately unfinished wait gave up
+ *   13  walk wait: the tree walk gave up waiting for another CTA's part of a residual sum
  */
 etree_status etree_device_status(void *workspace, void *stream, int32_t *detail);
 
