@@ -561,6 +561,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NT)
   __shared__ double slice_s[2], got_s[CS];     // this CTA's N(c) slice by pass parity; gathered
   __shared__ uint32_t pass_s;                  // passes published so far
   __shared__ int late_s;
+  __shared__ float qx_s[64], zx_s[64], l2_s[64], uni_s[64];   // per child: its test's inputs
   const int r = blockIdx.x / CS, tid = threadIdx.x;
   const int rank = CS > 1 ? (int)walk_cluster_rank() : 0;
   const bool lead = rank == 0;
@@ -619,6 +620,18 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NT)
     }
     if (tid == 0) u_s = n_ok ? base : 0;
   } else {
+    // Each child's test inputs do not depend on the walk's state: its parent row's log-sum-exp,
+    // q and logit of its token, and its uniform.  They are read (and the uniform drawn) by one
+    // thread per child up front, so thread 0's serial walk reads shared memory only.
+    if (tid >= 1 && tid < n) {
+      const int pu = par_s[tid], x = tok_s[tid];
+      qx_s[tid] = __ldg(p.q_draft + (size_t)(base + pu) * p.V + x);
+      zx_s[tid] = zc ? zc[base + tid] : zbuf[(size_t)zrow[base + pu] * p.V + x];
+      l2_s[tid] = p.lse2[base + pu];
+      float U[8];
+      uniforms8(p.seed, p.step, 0u, (uint32_t)tid, (uint32_t)r, 1u, U);
+      uni_s[tid] = U[0];
+    }
     // thread 0's walk state: node u, last child tested, c and N(c) of the current residual
     int u = 0, j = 0, a = 0;
     double c = 0.0, N = 1.0;
@@ -634,16 +647,12 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NT)
         for (j = j + 1; j < n && par_s[j] != u; ++j) {}
         if (j < n) {
           const int x = tok_s[j];
-          const float L2 = p.lse2[base + u];
-          const double qx = (double)__ldg(p.q_draft + (size_t)(base + u) * p.V + x);
+          const double qx = (double)qx_s[j];
           // the parent row's logit of x: from the materialised row itself when every row is
           // kept (the same fp32 accumulator the row's log-sum-exp came from), else child_logit's
-          const float zx = zc ? zc[base + j] : zbuf[(size_t)zrow[base + u] * p.V + x];
-          const double pz = (double)exp2f(zx * p.k_log2 - L2);
+          const double pz = (double)exp2f(zx_s[j] * p.k_log2 - l2_s[j]);
           const double rx = pz - c * qx > 0.0 ? (pz - c * qx) / N : 0.0;
-          float U[8];
-          uniforms8(p.seed, p.step, 0u, (uint32_t)j, (uint32_t)r, 1u, U);
-          if ((double)U[0] * qx < rx) {                 // accepted: the walk moves to child j
+          if ((double)uni_s[j] * qx < rx) {             // accepted: the walk moves to child j
             ++a;
             if (lead) {
               path[a] = j;
