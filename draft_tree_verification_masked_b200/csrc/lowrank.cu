@@ -16,7 +16,7 @@
 //                     never reaches HBM;
 //   C  = top-k of z~  topk_select_kernel: one CTA per row finds the k-th largest list entry by
 //                     a radix select over all the lists and keeps the entries ranked above it;
-//   z_c = h . W_c     lr_rescore_kernel: one warp per candidate, then the k are ordered by z_c.
+//   z_c = h . W_c     in the same CTA: one warp per candidate, then the k are ordered by z_c.
 //
 // The screen streams |U| = V r 2 bytes (155 MB at r = 512, 39 MB at r = 128) instead of the full
 // head's |W| = V H 2 (1.56 GB at H = 5120), plus k rows of W per hidden row.
@@ -222,16 +222,23 @@ __device__ __forceinline__ uint32_t sel_code(float2 x) {
   return enc_order(x.x == 0.f ? 0.f : x.x);          // >= 0x007fffff for every non-NaN value
 }
 
-__global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float2* __restrict__ lists,
-                                                                  int nlists, int k,
-                                                                  int32_t* __restrict__ cand) {
+__global__ void __launch_bounds__(kSelThreads) topk_select_kernel(
+    const float2* __restrict__ lists, int nlists, int k, int32_t* __restrict__ cand,
+    const __nv_bfloat16* __restrict__ hid,
+    const __nv_bfloat16* __restrict__ W, int H, int V, int32_t* __restrict__ out_ids,
+    float* __restrict__ out_logit) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_digit, s_above, s_count, s_n;
   __shared__ int s_min[kSelThreads / 32];
-  __shared__ float sv[16];
-  __shared__ int si[16];
+  __shared__ float sv[16], zs[16];
+  __shared__ int si[16], cs[16];
+  __shared__ uint4 hsm[1024];                          // the hidden row (H <= 8192)
   pdl_wait();
   const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  {                                                    // staged for the rescoring at the end
+    const uint4* hrow = reinterpret_cast<const uint4*>(hid + (size_t)m * H);
+    for (int i = tid; i < H / 8; i += kSelThreads) hsm[i] = hrow[i];
+  }
   const float2* rowl = lists + (size_t)m * nlists * 16;
   const int total = nlists * 16;
   const int in_regs = kSelRegs * kSelThreads;
@@ -359,85 +366,53 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float2* 
       __syncthreads();
     }
   }
-  if (warp == 0) {
-    const int n = min((int)s_n, k);
+  if (warp == 0) {                                     // the candidates in screen order
     float v = -INFINITY;
     int id = 0x7fffffff;
-    if (lane < n) {
+    const int nn = min((int)s_n, k);
+    if (lane < nn) {
       v = sv[lane];
       id = si[lane];
     }
     int rank = 0;
-    for (int j = 0; j < n; ++j) rank += before(sv[j], si[j], v, id);
-    if (lane < n) cand[(size_t)m * 16 + rank] = id;
+    for (int j = 0; j < nn; ++j) rank += before(sv[j], si[j], v, id);
+    if (lane < nn) cand[(size_t)m * 16 + rank] = id;
     else if (lane < k) cand[(size_t)m * 16 + lane] = -1;
   }
-}
-constexpr int kRescoreLoads = 20;        // 16-byte words of W per lane requested up front
-
-// One CTA per row, one warp per candidate: z_c = h . W_c in fp32 (the row staged in shared
-// memory, the lane's W words requested first); then the k candidates are ordered by z_c descending
-// (lower id first on equal values).
-__global__ void __launch_bounds__(512) lr_rescore_kernel(const __nv_bfloat16* __restrict__ hid,
-                                                         const __nv_bfloat16* __restrict__ W,
-                                                         int H, int V, int k,
-                                                         const int32_t* __restrict__ cand,
-                                                         int32_t* __restrict__ out_ids,
-                                                         float* __restrict__ out_logit) {
-  __shared__ uint4 hsm[1024];                     // H <= 8192
-  __shared__ float zs[16];
-  __shared__ int cs[16];
-  pdl_wait();
-  const int m = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint4* hrow = reinterpret_cast<const uint4*>(hid + (size_t)m * H);
-  // this lane's first kRescoreLoads words of the candidate's W row (all of it at H <= 5120) are
-  // requested before the hidden row is staged, so both loads are in flight together
-  const int c = warp < k ? cand[(size_t)m * 16 + warp] : -1;
-  const bool live = warp < k && c >= 0 && c < V;
-  uint4 wv[kRescoreLoads];
-  {
-    const uint4* w = reinterpret_cast<const uint4*>(W + (size_t)(live ? c : 0) * H);
-#pragma unroll
-    for (int u = 0; u < kRescoreLoads; ++u) {
-      const int i = lane + 32 * u;
-      wv[u] = (live && i < H / 8) ? __ldg(w + i) : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-  for (int i = threadIdx.x; i < H / 8; i += blockDim.x) hsm[i] = hrow[i];
-  __syncthreads();
+  // The exact logits z_c = h . W_c of the k candidates, one warp each (fp32, the hidden row from
+  // shared memory, four W words per lane in flight), then the k ordered by z_c descending, the
+  // lower id first on equal values.  Missing candidates (fewer than k entries) are (-1, -inf).
+  const int n = min((int)s_n, k);
   if (warp < k) {
-    float acc = 0.f;
-    if (live) {
-#pragma unroll
-      for (int u = 0; u < kRescoreLoads; ++u) {
-        const int i = lane + 32 * u;
-        if (i >= H / 8) break;
-        const uint4 a = hsm[i], b = wv[u];
-        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 fa = __bfloat1622float2(a2[q]), fb = __bfloat1622float2(b2[q]);
-          acc = fmaf(fa.x, fb.x, acc);
-          acc = fmaf(fa.y, fb.y, acc);
-        }
-      }
+    const int c = warp < n ? si[warp] : -1;
+    float acc = -INFINITY;
+    if (c >= 0 && c < V) {
       const uint4* w = reinterpret_cast<const uint4*>(W + (size_t)c * H);
-      for (int i = lane + 32 * kRescoreLoads; i < H / 8; i += 32) {   // H > 5120
-        const uint4 a = hsm[i], b = __ldg(w + i);
-        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+      acc = 0.f;
+      for (int i0 = lane; i0 < H / 8; i0 += 32 * 4) {
+        uint4 wv[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 fa = __bfloat1622float2(a2[q]), fb = __bfloat1622float2(b2[q]);
-          acc = fmaf(fa.x, fb.x, acc);
-          acc = fmaf(fa.y, fb.y, acc);
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + 32 * u;
+          wv[u] = i < H / 8 ? __ldg(w + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + 32 * u;
+          if (i >= H / 8) break;
+          const uint4 a = hsm[i];
+          const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&wv[u]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 fa = __bfloat1622float2(a2[q]), fb = __bfloat1622float2(b2[q]);
+            acc = fmaf(fa.x, fb.x, acc);
+            acc = fmaf(fa.y, fb.y, acc);
+          }
         }
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    } else {
-      acc = -INFINITY;
     }
     if (lane == 0) {
       zs[warp] = acc;
@@ -445,12 +420,12 @@ __global__ void __launch_bounds__(512) lr_rescore_kernel(const __nv_bfloat16* __
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     for (int i = 1; i < k; ++i) {                    // insertion sort of <= 16
       const float x = zs[i];
       const int ci = cs[i];
       int j = i - 1;
-      while (j >= 0 && (zs[j] < x || (zs[j] == x && cs[j] > ci))) {
+      while (j >= 0 && (zs[j] < x || (zs[j] == x && (unsigned)cs[j] > (unsigned)ci))) {
         zs[j + 1] = zs[j];
         cs[j + 1] = cs[j];
         --j;
@@ -464,8 +439,6 @@ __global__ void __launch_bounds__(512) lr_rescore_kernel(const __nv_bfloat16* __
     }
   }
 }
-
-
 int lowrank_down_chunks(int H) { return (H + kSkChunk - 1) / kSkChunk; }
 
 static const int kSkSmem = 1024 + 2 * 16384;     // two K steps of A and B boxes, 1 KB aligned
@@ -503,11 +476,8 @@ cudaError_t launch_lowrank_sample(const CUtensorMap& tm_g, const CUtensorMap& tm
 cudaError_t launch_lowrank_finish(const float2* lists, int nlists, int M, int k, int32_t* cand,
                                   const __nv_bfloat16* hid, const __nv_bfloat16* W, int H, int V,
                                   int32_t* out_ids, float* out_logit, cudaStream_t s) {
-  cudaError_t e = launch_pdl(topk_select_kernel, dim3(M), dim3(kSelThreads), 0, s, lists, nlists,
-                             k, cand);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(lr_rescore_kernel, dim3(M), dim3(32 * k), 0, s, hid, W, H, V, k, cand,
-                    out_ids, out_logit);
+  return launch_pdl(topk_select_kernel, dim3(M), dim3(kSelThreads), 0, s, lists, nlists, k, cand,
+                    hid, W, H, V, out_ids, out_logit);
 }
 
 }  // namespace etree
