@@ -894,8 +894,8 @@ __global__ void __launch_bounds__(kDrawThreads) draw_rows_kernel(AcceptParams p,
   p.out_tokens[(size_t)r * ETREE_OUT_STRIDE + a] = ir >= 0 ? ir : ip;
 }
 
-// Parts per request: about 8 CTAs per SM in all, at most 32 per request, no more than the
-// request's 8-id groups or the summary slots (max_parts).
+// Parts per request: about 8 CTAs per SM in all, at most 32 per request, at least one 8-id group
+// per thread of each part, and no more parts than summary slots (max_parts).
 int draw_parts(int B, int V, int sms, int max_parts) {
   const int groups = (V + 7) / 8;
   int parts = (8 * sms + B - 1) / std::max(1, B);
